@@ -1,0 +1,49 @@
+// Shared device helpers of the gated delta-rule kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+constexpr int kChunk = 64;  // chunk length of the chunkwise form (64, as the pages' kernels use)
+
+// ---- element conversion ------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <class T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+// ---- problem description passed to every kernel by value ---------------------------------
+struct Problem {
+    int B, T, Hk, Hv, dk, dv;
+    int NT;         // number of chunks, ceil(T / 64)
+    float scale;
+    const int32_t* head_map;  // may be null: hv / (Hv / Hk)
+
+    __device__ __forceinline__ int key_head(int hv) const {
+        return head_map ? head_map[hv] : hv / (Hv / Hk);
+    }
+    // Element offsets of one token row in the token-major layouts.
+    __device__ __forceinline__ long qk_row(int b, int t, int hk) const {
+        return ((long)(b * T + t) * Hk + hk) * dk;
+    }
+    __device__ __forceinline__ long v_row(int b, int t, int hv) const {
+        return ((long)(b * T + t) * Hv + hv) * dv;
+    }
+    __device__ __forceinline__ long gate_row(int b, int t, int hv, int width) const {
+        return ((long)(b * T + t) * Hv + hv) * width;
+    }
+    __device__ __forceinline__ long state_off(int b, int hv) const {
+        return ((long)b * Hv + hv) * dk * dv;
+    }
+};
+
+}  // namespace gdn

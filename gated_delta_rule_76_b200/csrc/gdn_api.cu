@@ -1,0 +1,428 @@
+// C ABI of libgdn (see include/gdn.h): argument validation on the host, workspace carving and
+// dispatch to the kernels.  No device memory is allocated here and nothing synchronises.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "gdn.h"
+#include "launch.h"
+
+namespace gdn {
+
+namespace {
+
+thread_local std::string g_last_error;
+
+gdn_status fail(gdn_status code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+gdn_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(GDN_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t elem_size(int dtype) { return dtype == GDN_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Buf {
+    const void* p;
+    size_t bytes;
+    const char* name;
+};
+
+bool overlaps(const Buf& a, const Buf& b) {
+    if (!a.p || !b.p || !a.bytes || !b.bytes) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+// Every output against every input and every other output.
+gdn_status check_buffers(const Buf* in, int nin, const Buf* out, int nout) {
+    for (int i = 0; i < nin; ++i)
+        if (in[i].p && !aligned16(in[i].p))
+            return fail(GDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", in[i].name);
+    for (int i = 0; i < nout; ++i) {
+        if (out[i].p && !aligned16(out[i].p))
+            return fail(GDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", out[i].name);
+        for (int j = 0; j < nin; ++j)
+            if (overlaps(out[i], in[j]))
+                return fail(GDN_ERR_INVALID_ARG, "output %s overlaps input %s", out[i].name, in[j].name);
+        for (int j = 0; j < i; ++j)
+            if (overlaps(out[i], out[j]))
+                return fail(GDN_ERR_INVALID_ARG, "outputs %s and %s overlap", out[i].name, out[j].name);
+    }
+    return GDN_OK;
+}
+
+// Shared checks of sizes, modes and dtypes.
+gdn_status check_common(int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                        const int32_t* head_map, int32_t apc, int32_t gpc, int32_t dtype,
+                        int32_t gate_dtype) {
+    if (B < 1 || T < 0 || Hk < 1 || Hv < 1)
+        return fail(GDN_ERR_INVALID_ARG, "bad sizes B=%lld T=%lld Hk=%lld Hv=%lld", (long long)B,
+                    (long long)T, (long long)Hk, (long long)Hv);
+    if (dk != dv || (dk != 64 && dk != 128))
+        return fail(GDN_ERR_UNSUPPORTED, "dk=%lld dv=%lld: supported are dk = dv in {64, 128}",
+                    (long long)dk, (long long)dv);
+    if (!head_map && Hv % Hk != 0)
+        return fail(GDN_ERR_INVALID_ARG, "Hv=%lld is not a multiple of Hk=%lld and no head_map given",
+                    (long long)Hv, (long long)Hk);
+    if ((apc != 0 && apc != 1) || (gpc != 0 && gpc != 1))
+        return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel and gates_per_channel must be 0 or 1");
+    if ((dtype != GDN_BF16 && dtype != GDN_F32) || (gate_dtype != GDN_BF16 && gate_dtype != GDN_F32))
+        return fail(GDN_ERR_INVALID_ARG, "unknown dtype %d / gate_dtype %d", dtype, gate_dtype);
+    if (dtype == GDN_F32 && gate_dtype != GDN_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "fp32 tensors need fp32 gates");
+    if (B * T * (Hk > Hv ? Hk : Hv) * dk >= (int64_t(1) << 40) || B * T >= (int64_t(1) << 30))
+        return fail(GDN_ERR_UNSUPPORTED, "problem too large for 32-bit token indices");
+    return GDN_OK;
+}
+
+Problem make_problem(int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
+                     float scale, const int32_t* head_map) {
+    Problem pb;
+    pb.B = (int)B; pb.T = (int)T; pb.Hk = (int)Hk; pb.Hv = (int)Hv; pb.dk = (int)dk; pb.dv = (int)dv;
+    pb.NT = (int)((T + kChunk - 1) / kChunk);
+    pb.scale = scale;
+    pb.head_map = head_map;
+    return pb;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int variant(int32_t dtype, int32_t gate_dtype) {
+    if (dtype == GDN_F32) return 2;
+    return gate_dtype == GDN_F32 ? 1 : 0;
+}
+
+bool identity_heads(const Problem& pb) { return pb.Hk == pb.Hv && pb.head_map == nullptr; }
+
+}  // namespace
+
+WsPlan plan_chunk_ws(const Problem& pb, bool bwd, bool gqa_partials) {
+    WsPlan w{};
+    const size_t nch = (size_t)pb.B * pb.Hv * pb.NT, C = kChunk, dk = pb.dk, dv = pb.dv;
+    size_t off = 0;
+    auto take = [&](size_t floats) {
+        size_t o = off;
+        off = align256(off + floats * sizeof(float));
+        return o;
+    };
+    const size_t none = ~size_t(0);
+    w.T = take(nch * C * C);
+    w.P = take(nch * C * C);
+    w.Eh = take(nch * C * dk);
+    w.Qh = take(nch * C * dk);
+    w.Kb = take(nch * C * dk);
+    w.gam = take(nch * dk);
+    w.Kt = bwd ? take(nch * C * dk) : none;
+    w.Gm = bwd ? take(nch * C * dk) : none;
+    w.S0 = bwd ? take(nch * dk * dv) : none;
+    w.dSC = bwd ? take(nch * dk * dv) : none;
+    w.V = bwd ? take(nch * C * dv) : none;
+    w.Y = bwd ? take(nch * C * dv) : none;
+    w.dV = bwd ? take(nch * C * dv) : none;
+    w.dY = bwd ? take(nch * C * dv) : none;
+    w.dbw = bwd ? take(nch * (dv / kDvTile) * C) : none;
+    const size_t part = (size_t)pb.B * pb.T * pb.Hv * dk;
+    w.dq_v = (bwd && gqa_partials) ? take(part) : none;
+    w.dk_v = (bwd && gqa_partials) ? take(part) : none;
+    w.bytes = off;
+    return w;
+}
+
+ChunkWs carve_chunk_ws(const WsPlan& w, void* base) {
+    const size_t none = ~size_t(0);
+    char* b = static_cast<char*>(base);
+    auto at = [&](size_t o) { return o == none ? nullptr : reinterpret_cast<float*>(b + o); };
+    ChunkWs ws;
+    ws.T = at(w.T); ws.P = at(w.P); ws.Eh = at(w.Eh); ws.Qh = at(w.Qh); ws.Kb = at(w.Kb);
+    ws.Kt = at(w.Kt); ws.Gm = at(w.Gm); ws.gam = at(w.gam); ws.S0 = at(w.S0); ws.dSC = at(w.dSC);
+    ws.V = at(w.V); ws.Y = at(w.Y); ws.dV = at(w.dV); ws.dY = at(w.dY); ws.dbw = at(w.dbw);
+    ws.dq_v = at(w.dq_v); ws.dk_v = at(w.dk_v);
+    return ws;
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+namespace {
+
+gdn_status check_fwd(const gdn_fwd_args* a) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    gdn_status s = check_common(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->head_map,
+                                a->alpha_per_channel, a->gates_per_channel, a->dtype, a->gate_dtype);
+    if (s) return s;
+    if (a->T > 0 && (!a->q || !a->k || !a->v || !a->alpha || !a->b || !a->o))
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, alpha, b and o are required");
+    if (a->gates_per_channel && a->T > 0 && !a->w)
+        return fail(GDN_ERR_INVALID_ARG, "w is required when gates_per_channel = 1");
+    if (!a->gates_per_channel && a->w)
+        return fail(GDN_ERR_INVALID_ARG, "w must be NULL for scalar gates (b holds beta)");
+    const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
+    const size_t BT = (size_t)(a->B * a->T);
+    const Buf in[] = {
+        {a->q, BT * a->Hk * a->dk * es, "q"},
+        {a->k, BT * a->Hk * a->dk * es, "k"},
+        {a->v, BT * a->Hv * a->dv * es, "v"},
+        {a->alpha, BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
+        {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
+        {a->w, BT * a->Hv * a->dv * gs, "w"},
+        {a->h0, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "h0"},
+        {a->z, BT * a->Hv * a->dv * es, "z"},
+        {a->head_map, (size_t)a->Hv * 4, "head_map"},
+    };
+    const Buf out[] = {
+        {a->o, BT * a->Hv * a->dv * es, "o"},
+        {a->ht, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "ht"},
+    };
+    return check_buffers(in, 9, out, 2);
+}
+
+gdn_status check_bwd(const gdn_bwd_args* a) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    gdn_status s = check_common(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->head_map,
+                                a->alpha_per_channel, a->gates_per_channel, a->dtype, a->gate_dtype);
+    if (s) return s;
+    if (a->T > 0 && (!a->q || !a->k || !a->v || !a->alpha || !a->b || !a->grad_o || !a->grad_q ||
+                     !a->grad_k || !a->grad_v || !a->grad_alpha || !a->grad_b))
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, alpha, b, grad_o and grad_q/k/v/alpha/b are required");
+    if (a->gates_per_channel && a->T > 0 && (!a->w || !a->grad_w))
+        return fail(GDN_ERR_INVALID_ARG, "w and grad_w are required when gates_per_channel = 1");
+    if (!a->gates_per_channel && (a->w || a->grad_w))
+        return fail(GDN_ERR_INVALID_ARG, "w and grad_w must be NULL for scalar gates");
+    const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
+    const size_t BT = (size_t)(a->B * a->T);
+    const size_t st = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
+    const size_t na = BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs;
+    const size_t nb = BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs;
+    const Buf in[] = {
+        {a->q, BT * a->Hk * a->dk * es, "q"}, {a->k, BT * a->Hk * a->dk * es, "k"},
+        {a->v, BT * a->Hv * a->dv * es, "v"}, {a->alpha, na, "alpha"}, {a->b, nb, "b"},
+        {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        {a->grad_o, BT * a->Hv * a->dv * es, "grad_o"}, {a->grad_ht, st, "grad_ht"},
+    };
+    const Buf out[] = {
+        {a->grad_q, BT * a->Hk * a->dk * es, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * es, "grad_k"},
+        {a->grad_v, BT * a->Hv * a->dv * es, "grad_v"}, {a->grad_alpha, na, "grad_alpha"},
+        {a->grad_b, nb, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * gs, "grad_w"}, {a->grad_h0, st, "grad_h0"},
+    };
+    return check_buffers(in, 10, out, 7);
+}
+
+gdn_status check_workspace(void* ws, size_t have, size_t need) {
+    if (need == 0) return GDN_OK;
+    if (!ws) return fail(GDN_ERR_WORKSPACE, "workspace is NULL, %zu bytes needed", need);
+    if (have < need) return fail(GDN_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", have, need);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(GDN_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    return GDN_OK;
+}
+
+ChunkIO io_from(const gdn_fwd_args* a) {
+    ChunkIO io{};
+    io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
+    io.z = a->z; io.h0 = a->h0; io.o = a->o; io.ht = a->ht;
+    return io;
+}
+
+cudaError_t run_fwd(int var, const Problem& pb, const ChunkIO& io, const ChunkWs& ws, Flags f,
+                    cudaStream_t st) {
+    switch (var) {
+        case 0: return bf16_chunk_fwd(pb, io, ws, f, st);
+        case 1: return bf16_f32g_chunk_fwd(pb, io, ws, f, st);
+        default: return f32_chunk_fwd(pb, io, ws, f, st);
+    }
+}
+
+// ht = h0 (or zeros) when there is no token to process.
+gdn_status copy_state(float* dst, const float* src, size_t bytes, cudaStream_t st, const char* what) {
+    if (!dst) return GDN_OK;
+    cudaError_t e = src ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st)
+                        : cudaMemsetAsync(dst, 0, bytes, st);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, what);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    return plan_chunk_ws(pb, false, false).bytes;
+}
+
+gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspace_bytes,
+                         gdn_stream stream) {
+    gdn_status s = check_fwd(a);
+    if (s) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t sbytes = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
+    if (a->T == 0) return copy_state(a->ht, a->h0, sbytes, st, "gdn_chunk_fwd");
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    WsPlan plan = plan_chunk_ws(pb, false, false);
+    if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
+    cudaError_t e = run_fwd(variant(a->dtype, a->gate_dtype), pb, io_from(a),
+                            carve_chunk_ws(plan, workspace), f, st);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_fwd");
+}
+
+size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    return plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
+}
+
+gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspace_bytes,
+                         gdn_stream stream) {
+    gdn_status s = check_bwd(a);
+    if (s) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t sbytes = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
+    if (a->T == 0) return copy_state(a->grad_h0, a->grad_ht, sbytes, st, "gdn_chunk_bwd");
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    const bool direct = identity_heads(pb);
+    WsPlan plan = plan_chunk_ws(pb, true, !direct);
+    if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
+    ChunkIO io{};
+    io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
+    io.h0 = a->h0; io.dout = a->grad_o; io.dht = a->grad_ht; io.dq = a->grad_q; io.dk = a->grad_k;
+    io.dv = a->grad_v; io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = a->grad_w;
+    io.dh0 = a->grad_h0;
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
+    ChunkWs ws = carve_chunk_ws(plan, workspace);
+    cudaError_t e;
+    switch (variant(a->dtype, a->gate_dtype)) {
+        case 0: e = bf16_chunk_bwd(pb, io, ws, f, direct, st); break;
+        case 1: e = bf16_f32g_chunk_bwd(pb, io, ws, f, direct, st); break;
+        default: e = f32_chunk_bwd(pb, io, ws, f, direct, st); break;
+    }
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_bwd");
+}
+
+gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    gdn_status s = check_common(a->N, 1, a->Hk, a->Hv, a->dk, a->dv, a->head_map,
+                                a->alpha_per_channel, a->gates_per_channel, a->dtype, a->gate_dtype);
+    if (s) return s;
+    if (!a->q || !a->k || !a->v || !a->alpha || !a->b || !a->state || !a->o)
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v, alpha, b, state and o are required");
+    if (a->gates_per_channel ? !a->w : a->w != nullptr)
+        return fail(GDN_ERR_INVALID_ARG, "w is required with channel gates and must be NULL otherwise");
+    if (a->conv_state && !a->conv_w)
+        return fail(GDN_ERR_INVALID_ARG, "conv_w is required with conv_state");
+    const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype), N = (size_t)a->N;
+    const size_t cch = (size_t)(2 * a->Hk * a->dk + a->Hv * a->dv);
+    const size_t st = N * a->Hv * a->dk * a->dv * 4;
+    const Buf in[] = {
+        {a->q, N * a->Hk * a->dk * es, "q"}, {a->k, N * a->Hk * a->dk * es, "k"},
+        {a->v, N * a->Hv * a->dv * es, "v"},
+        {a->alpha, N * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
+        {a->b, N * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
+        {a->w, N * a->Hv * a->dv * gs, "w"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        {a->conv_w, cch * 4 * es, "conv_w"}, {a->z, N * a->Hv * a->dv * es, "z"},
+    };
+    const Buf out[] = {
+        {a->o, N * a->Hv * a->dv * es, "o"}, {a->state, st, "state"},
+        {a->conv_state, a->conv_state ? N * cch * 3 * es : 0, "conv_state"},
+    };
+    if ((s = check_buffers(in, 9, out, 3))) return s;
+    DecodeParams p{};
+    p.q = a->q; p.k = a->k; p.v = a->v; p.alpha = a->alpha; p.b = a->b; p.w = a->w;
+    p.state = a->state; p.o = a->o; p.head_map = a->head_map; p.conv_state = a->conv_state;
+    p.conv_w = a->conv_w; p.z = a->z;
+    p.N = (int)a->N; p.Hk = (int)a->Hk; p.Hv = (int)a->Hv; p.dk = (int)a->dk; p.dv = (int)a->dv;
+    p.scale = a->scale;
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
+    cudaStream_t sm = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch (variant(a->dtype, a->gate_dtype)) {
+        case 0: e = bf16_decode(p, f, sm); break;
+        case 1: e = bf16_f32g_decode(p, f, sm); break;
+        default: e = f32_decode(p, f, sm); break;
+    }
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_step");
+}
+
+size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    const size_t es = elem_size(a->dtype);
+    const size_t conv = align256((size_t)(a->B * a->T) * (2 * a->Hk * a->dk + a->Hv * a->dv) * es);
+    return conv + plan_chunk_ws(pb, false, false).bytes;
+}
+
+gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t workspace_bytes,
+                              gdn_stream stream) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    gdn_status s = check_common(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->head_map,
+                                a->alpha_per_channel, a->gates_per_channel, a->dtype, a->gate_dtype);
+    if (s) return s;
+    if (a->T > 0 && (!a->xq || !a->xk || !a->xv || !a->conv_w || !a->alpha || !a->b || !a->z || !a->y))
+        return fail(GDN_ERR_INVALID_ARG, "xq, xk, xv, conv_w, alpha, b, z and y are required");
+    if (a->gates_per_channel ? (a->T > 0 && !a->w) : a->w != nullptr)
+        return fail(GDN_ERR_INVALID_ARG, "w is required with channel gates and must be NULL otherwise");
+    const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
+    const size_t BT = (size_t)(a->B * a->T);
+    const size_t cch = (size_t)(2 * a->Hk * a->dk + a->Hv * a->dv);
+    const size_t st = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
+    const Buf in[] = {
+        {a->xq, BT * a->Hk * a->dk * es, "xq"}, {a->xk, BT * a->Hk * a->dk * es, "xk"},
+        {a->xv, BT * a->Hv * a->dv * es, "xv"}, {a->conv_w, cch * 4 * es, "conv_w"},
+        {a->alpha, BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
+        {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
+        {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->z, BT * a->Hv * a->dv * es, "z"},
+        {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+    };
+    const Buf out[] = {
+        {a->y, BT * a->Hv * a->dv * es, "y"}, {a->ht, st, "ht"},
+        {a->conv_state_out, (size_t)a->B * cch * 3 * es, "conv_state_out"},
+    };
+    if ((s = check_buffers(in, 10, out, 3))) return s;
+    cudaStream_t sm = static_cast<cudaStream_t>(stream);
+    if (a->T == 0) {
+        if (a->conv_state_out) {
+            cudaError_t e = cudaMemsetAsync(a->conv_state_out, 0, (size_t)a->B * cch * 3 * es, sm);
+            if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_fwd");
+        }
+        return copy_state(a->ht, a->h0, st, sm, "gdn_layer_core_fwd");
+    }
+    const size_t need = gdn_layer_core_fwd_workspace_size(a);
+    if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
+    char* base = static_cast<char*>(workspace);
+    void* qc = base;
+    void* kc = base + BT * a->Hk * a->dk * es;
+    void* vc = base + 2 * BT * a->Hk * a->dk * es;
+    const size_t conv_bytes = align256(BT * cch * es);
+    ConvParams cp{};
+    cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
+    cp.q = qc; cp.k = kc; cp.v = vc; cp.conv_state_out = a->conv_state_out;
+    cp.B = (int)a->B; cp.T = (int)a->T; cp.Hk = (int)a->Hk; cp.Hv = (int)a->Hv; cp.d = (int)a->dk;
+    const int var = variant(a->dtype, a->gate_dtype);
+    cudaError_t e = var == 2 ? f32_conv(cp, sm) : bf16_conv(cp, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_fwd (conv)");
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    WsPlan plan = plan_chunk_ws(pb, false, false);
+    ChunkIO io{};
+    io.q = qc; io.k = kc; io.v = vc; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.z = a->z;
+    io.h0 = a->h0; io.o = a->y; io.ht = a->ht;
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
+    e = run_fwd(var, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
+}
+
+const char* gdn_last_error(void) { return g_last_error.c_str(); }
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

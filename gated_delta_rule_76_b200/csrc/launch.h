@@ -1,0 +1,42 @@
+// Host-side launch interface between the C ABI (gdn_api.cu) and the per-dtype kernel
+// instantiation units (inst_*.cu).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "simt_chunk.cuh"
+#include "decode.cuh"
+#include "conv.cuh"
+
+namespace gdn {
+
+struct Flags {
+    bool apc;   // alpha per channel
+    bool gpc;   // b, w per channel (else scalar beta)
+    bool gate;  // swish(z) output gate in the forward
+};
+
+// Workspace carving.  Every array is 256-byte aligned.
+struct WsPlan {
+    size_t bytes = 0;
+    size_t T, P, Eh, Qh, Kb, Kt, Gm, gam, S0, dSC, V, Y, dV, dY, dbw, dq_v, dk_v;
+};
+WsPlan plan_chunk_ws(const Problem& pb, bool bwd, bool gqa_partials);
+ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
+
+// Per (TIn, TG) instantiation units define these (TIn: q/k/v dtype, TG: gate dtype).
+#define GDN_DECLARE_LAUNCHERS(NAME)                                                           \
+    cudaError_t NAME##_chunk_fwd(const Problem&, const ChunkIO&, const ChunkWs&, Flags,       \
+                                 cudaStream_t);                                              \
+    cudaError_t NAME##_chunk_bwd(const Problem&, const ChunkIO&, const ChunkWs&, Flags, bool, \
+                                 cudaStream_t);                                              \
+    cudaError_t NAME##_decode(const DecodeParams&, Flags, cudaStream_t);                       \
+    cudaError_t NAME##_conv(const ConvParams&, cudaStream_t);
+
+GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
+GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates
+GDN_DECLARE_LAUNCHERS(f32)        // fp32 tensors, fp32 gates
+
+}  // namespace gdn

@@ -1,0 +1,284 @@
+"""Thin Python binding of libgdn (include/gdn.h), same names as the C ABI.
+
+Only argument marshalling lives here: torch allocates device memory (outputs and the
+workspace) and provides the stream; every step of the recurrence runs in the CUDA kernels of
+libgdn.so.  There is no CPU fallback: if the library is missing or a tensor is not on a CUDA
+device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_BF16, GDN_F32 = 0, 1
+_STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
+           4: "GDN_ERR_WORKSPACE"}
+
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+I32 = ctypes.c_int32
+F32 = ctypes.c_float
+
+
+class FwdArgs(ctypes.Structure):
+    _fields_ = [("q", P), ("k", P), ("v", P), ("alpha", P), ("b", P), ("w", P), ("h0", P),
+                ("z", P), ("o", P), ("ht", P), ("head_map", P),
+                ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
+                ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
+                ("dtype", I32), ("gate_dtype", I32)]
+
+
+class BwdArgs(ctypes.Structure):
+    _fields_ = [("q", P), ("k", P), ("v", P), ("alpha", P), ("b", P), ("w", P), ("h0", P),
+                ("head_map", P), ("grad_o", P), ("grad_ht", P), ("grad_q", P), ("grad_k", P),
+                ("grad_v", P), ("grad_alpha", P), ("grad_b", P), ("grad_w", P), ("grad_h0", P),
+                ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
+                ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
+                ("dtype", I32), ("gate_dtype", I32)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("q", P), ("k", P), ("v", P), ("alpha", P), ("b", P), ("w", P), ("state", P),
+                ("o", P), ("head_map", P), ("conv_state", P), ("conv_w", P), ("z", P),
+                ("N", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
+                ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
+                ("dtype", I32), ("gate_dtype", I32)]
+
+
+class LayerArgs(ctypes.Structure):
+    _fields_ = [("xq", P), ("xk", P), ("xv", P), ("conv_w", P), ("alpha", P), ("b", P), ("w", P),
+                ("z", P), ("h0", P), ("y", P), ("ht", P), ("conv_state_out", P), ("head_map", P),
+                ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
+                ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
+                ("dtype", I32), ("gate_dtype", I32)]
+
+
+EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
+            "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
+            "gdn_layer_core_fwd", "gdn_last_error", "gdn_version"]
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH):
+    """Load libgdn.so and declare its C signatures.  Raises if the library is missing."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise GdnError(f"{path} is missing: build it with `python -m gated_delta_rule_76_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.gdn_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
+    lib.gdn_chunk_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(FwdArgs), P, ctypes.c_size_t, P]
+    lib.gdn_chunk_fwd.restype = ctypes.c_int
+    lib.gdn_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
+    lib.gdn_chunk_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_chunk_bwd.argtypes = [ctypes.POINTER(BwdArgs), P, ctypes.c_size_t, P]
+    lib.gdn_chunk_bwd.restype = ctypes.c_int
+    lib.gdn_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), P]
+    lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_layer_core_fwd_workspace_size.argtypes = [ctypes.POINTER(LayerArgs)]
+    lib.gdn_layer_core_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_layer_core_fwd.argtypes = [ctypes.POINTER(LayerArgs), P, ctypes.c_size_t, P]
+    lib.gdn_layer_core_fwd.restype = ctypes.c_int
+    lib.gdn_last_error.argtypes = []
+    lib.gdn_last_error.restype = ctypes.c_char_p
+    lib.gdn_version.argtypes = []
+    lib.gdn_version.restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def check(status: int, what: str):
+    if status != 0:
+        msg = load().gdn_last_error().decode(errors="replace")
+        raise GdnError(f"{what}: {_STATUS.get(status, status)}: {msg}")
+
+
+# ---------------------------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------------------------
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise GdnError("libgdn takes CUDA tensors only (there is no CPU path)")
+    if not t.is_contiguous():
+        raise GdnError("libgdn takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise GdnError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    if workspace is not None and workspace.numel() * workspace.element_size() >= nbytes:
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _gates(alpha, b, w, beta):
+    if beta is not None:
+        if b is not None or w is not None:
+            raise GdnError("give either beta or (b, w)")
+        return beta, None, 0
+    if b is None or w is None:
+        raise GdnError("channel gates need both b and w")
+    return b, w, 1
+
+
+def _head_map(head_map, device):
+    if head_map is None:
+        return None
+    if not torch.is_tensor(head_map):
+        head_map = torch.tensor(head_map, dtype=torch.int32)
+    return head_map.to(device=device, dtype=torch.int32).contiguous()
+
+
+# ---------------------------------------------------------------------------------------------
+# public calls
+# ---------------------------------------------------------------------------------------------
+def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
+             scale: float = 1.0, o=None, ht=None) -> Tuple[FwdArgs, list]:
+    """Build the gdn_fwd_args struct (the returned list keeps referenced tensors alive)."""
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    hm = _head_map(head_map, q.device)
+    a = FwdArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
+                h0=_ptr(h0), z=_ptr(z), o=_ptr(o), ht=_ptr(ht), head_map=_ptr(hm),
+                B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
+                alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
+                dtype=_dt(q), gate_dtype=_dt(alpha))
+    return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm]
+
+
+def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
+                  scale: float = 1.0, *, o=None, ht=None, want_ht: bool = True,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """Chunkwise forward.  Returns (o [B,T,Hv,dv], ht [B,Hv,dk,dv] or None)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=q.dtype, device=q.device)
+    if ht is None and want_ht:
+        ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    lib = load()
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht)
+    need = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a))
+    ws = _workspace(need, q.device, workspace)
+    check(lib.gdn_chunk_fwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_fwd")
+    return o, ht
+
+
+def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, scale=1.0,
+             grad_o=None, grad_ht=None, grads=None) -> Tuple[BwdArgs, list]:
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    hm = _head_map(head_map, q.device)
+    g = grads
+    a = BwdArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
+                h0=_ptr(h0), head_map=_ptr(hm), grad_o=_ptr(grad_o), grad_ht=_ptr(grad_ht),
+                grad_q=_ptr(g["dq"]), grad_k=_ptr(g["dk"]), grad_v=_ptr(g["dv"]),
+                grad_alpha=_ptr(g["dalpha"]), grad_b=_ptr(g["db"] if gpc else g["dbeta"]),
+                grad_w=_ptr(g.get("dw")), grad_h0=_ptr(g.get("dh0")),
+                B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
+                alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
+                dtype=_dt(q), gate_dtype=_dt(alpha))
+    return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g]
+
+
+def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
+                  scale: float = 1.0, *, grad_o, grad_ht=None, want_dh0: bool = True,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """Chunkwise backward.  Returns dq, dk, dv, dalpha and db/dw (or dbeta), dh0."""
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    grads = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+             "dalpha": torch.empty_like(alpha)}
+    if gpc:
+        grads["db"] = torch.empty_like(b)
+        grads["dw"] = torch.empty_like(w)
+    else:
+        grads["dbeta"] = torch.empty_like(beta)
+    if want_dh0:
+        B, T, Hk, dk = q.shape
+        Hv, dv = v.shape[2], v.shape[3]
+        grads["dh0"] = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    lib = load()
+    a, keep = bwd_args(q, k, v, alpha, b, w, beta, h0, head_map, scale, grad_o, grad_ht, grads)
+    need = lib.gdn_chunk_bwd_workspace_size(ctypes.byref(a))
+    ws = _workspace(need, q.device, workspace)
+    check(lib.gdn_chunk_bwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_bwd")
+    return grads
+
+
+def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=None,
+                    scale: float = 1.0, *, conv_state=None, conv_w=None, z=None, o=None,
+                    stream=None):
+    """One token for N sequences; ``state`` [N,Hv,dk,dv] fp32 is updated in place.  Returns o."""
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    N, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if o is None:
+        o = torch.empty((N, Hv, dv), dtype=q.dtype, device=q.device)
+    hm = _head_map(head_map, q.device)
+    a = DecodeArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
+                   state=_ptr(state), o=_ptr(o), head_map=_ptr(hm), conv_state=_ptr(conv_state),
+                   conv_w=_ptr(conv_w), z=_ptr(z), N=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
+                   alpha_per_channel=int(alpha.dim() == 3), gates_per_channel=gpc,
+                   dtype=_dt(q), gate_dtype=_dt(alpha))
+    check(load().gdn_decode_step(ctypes.byref(a), _stream(stream)), "gdn_decode_step")
+    return o
+
+
+def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, h0=None,
+                       head_map=None, scale: float = 1.0, *, want_ht: bool = True,
+                       want_conv_state: bool = False, y=None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """GQA layer core forward.  Returns (y, ht or None, conv_state or None)."""
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    B, T, Hk, dk = xq.shape
+    Hv, dv = xv.shape[2], xv.shape[3]
+    if y is None:
+        y = torch.empty((B, T, Hv, dv), dtype=xq.dtype, device=xq.device)
+    ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=xq.device) if want_ht else None
+    cs = (torch.empty((B, 2 * Hk * dk + Hv * dv, 3), dtype=xq.dtype, device=xq.device)
+          if want_conv_state else None)
+    hm = _head_map(head_map, xq.device)
+    a = LayerArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
+                  b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
+                  conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
+                  dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
+                  gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha))
+    lib = load()
+    need = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(a))
+    ws = _workspace(need, xq.device, workspace)
+    check(lib.gdn_layer_core_fwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)),
+          "gdn_layer_core_fwd")
+    return y, ht, cs

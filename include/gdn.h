@@ -1,0 +1,221 @@
+/*
+ * gdn.h — C ABI of the gated delta-rule recurrence library (libgdn.so, CUDA for sm_100a).
+ *
+ * The operation (Gated DeltaNet-2 summary, gist.science, «Méthodologie» §1 «Règle Delta
+ * Portée-2»; restated in the zubnet.ai news item on Gated DeltaNet-2):
+ *
+ *     S_t = (I - k_t e_t^T) Diag(alpha_t) S_{t-1} + k_t z_t^T,   e_t = b_t .* k_t,  z_t = w_t .* v_t
+ *     o_t = scale * S_t^T q_t
+ *
+ * with S_t in R^{dk x dv} (dk rows, dv contiguous columns), the erase gate b_t in [0,1]^dk on the
+ * key axis, the write gate w_t in [0,1]^dv on the value axis and the channel decay alpha_t in
+ * (0,1)^dk.  With b = w = beta (one scalar per token and head) and a scalar alpha this is Gated
+ * DeltaNet (Gated DeltaNet explainer, docsaid.org, «Réunir les deux»); with alpha = 1 as well it
+ * is DeltaNet («DeltaNet : ne corriger que l'entrée visée»).  Channel alpha with scalar beta is
+ * the KDA case named on the same GDN-2 page.
+ *
+ * Conventions shared by every call
+ *  - Ownership: the caller owns every buffer.  The library allocates no device memory; scratch
+ *    memory is a caller workspace whose size the *_workspace_size() calls return (the workspace
+ *    may be reused across calls on the same stream; its contents on entry do not matter).
+ *  - Pointers: every tensor pointer is a device pointer (cudaMalloc'd or equivalent) to a dense,
+ *    contiguous array in the layout stated; all must be 16-byte aligned.  Outputs must not
+ *    overlap inputs or each other (in-place arguments say so explicitly).
+ *  - Execution: every call is asynchronous on the given stream and never synchronises.
+ *    Outputs are valid once the stream reaches the end of the call.
+ *  - Layouts: token-major.  q, k: [B,T,Hk,dk]; v, o, z: [B,T,Hv,dv]; channel gates alpha, b:
+ *    [B,T,Hv,dk], w: [B,T,Hv,dv]; scalar gates alpha, beta: [B,T,Hv]; states: [B,Hv,dk,dv] fp32.
+ *  - GQA: value head hv reads key head head_map[hv] (int32 device array of Hv entries).  NULL
+ *    means contiguous groups hv / (Hv / Hk) (Hv must then be a multiple of Hk).  Several value
+ *    heads share each key head in the 16-key / 128-value layer of the mkdocs chapter «Gated
+ *    DeltaNet», «Les projections d'entrée».
+ *  - Sizes: dk, dv in {64, 128}; B, T, Hk, Hv >= 1 (T = 0 is accepted and does nothing but copy
+ *    h0 to ht).  T need not be a multiple of the chunk length 64.
+ *  - Dtypes: q, k, v, o, z, gradients of q/k/v in `dtype`; alpha, b, w, beta and their gradients
+ *    in `gate_dtype`; states and their gradients are always fp32.
+ *  - Range: the chunked kernels factor the decay as exp(g_r) * exp(-g_s) inside a chunk of 64
+ *    tokens (g = cumulative log alpha).  The product of alpha over one chunk must stay above
+ *    1e-30 per channel, otherwise the factors overflow and the result is NaN/Inf (never a
+ *    silently clamped number).  The single-token decode step has no such limit.
+ *  - Errors: every call returns a gdn_status.  Invalid arguments are detected on the host before
+ *    any launch and nothing is written.  gdn_last_error() returns a thread-local message about
+ *    the last failure of the calling thread.  No C++ exception crosses this interface.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int gdn_status;
+#define GDN_OK 0
+#define GDN_ERR_INVALID_ARG 1 /* null required pointer, bad size, misaligned or overlapping buffer */
+#define GDN_ERR_UNSUPPORTED 2 /* valid but not implemented here: dk/dv outside {64,128}, dtype */
+#define GDN_ERR_CUDA 3        /* a CUDA call or kernel launch failed (message has the CUDA error) */
+#define GDN_ERR_WORKSPACE 4   /* workspace NULL or smaller than *_workspace_size() */
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+/* Opaque stream handle: a cudaStream_t (NULL = the legacy default stream). */
+typedef void* gdn_stream;
+
+/* ------------------------------------------------------------------------------------------
+ * Chunkwise forward.  Chunkwise-parallel form with chunk length 64: inside a chunk the decay is
+ * absorbed into the erase and write factors and the lower-triangular system (I + A)^-1 is solved
+ * for the erase-side and write-side auxiliaries (GDN-2 summary, «Entraînement Parallèle
+ * Efficace par Blocs»; explainer «Rendre l'entraînement parallèle»); the state is carried from
+ * chunk to chunk in fp32.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct gdn_fwd_args {
+    const void* q;        /* [B,T,Hk,dk]  dtype */
+    const void* k;        /* [B,T,Hk,dk]  dtype */
+    const void* v;        /* [B,T,Hv,dv]  dtype */
+    const void* alpha;    /* [B,T,Hv,dk] if alpha_per_channel else [B,T,Hv]; gate_dtype, in (0,1] */
+    const void* b;        /* erase gate [B,T,Hv,dk] if gates_per_channel, else beta [B,T,Hv] */
+    const void* w;        /* write gate [B,T,Hv,dv] if gates_per_channel, else must be NULL */
+    const float* h0;      /* [B,Hv,dk,dv] initial state, NULL = zeros */
+    const void* z;        /* optional swish output gate [B,T,Hv,dv] dtype: o <- o * z * sigmoid(z) */
+    void* o;              /* out [B,T,Hv,dv] dtype */
+    float* ht;            /* out [B,Hv,dk,dv] final state, may be NULL */
+    const int32_t* head_map; /* [Hv] value head -> key head, NULL = contiguous groups */
+    int64_t B, T, Hk, Hv, dk, dv;
+    float scale;          /* readout scale (the pages use 1) */
+    int32_t alpha_per_channel; /* 1: alpha in (0,1)^dk; 0: one scalar per token and value head */
+    int32_t gates_per_channel; /* 1: separate b (dk) and w (dv); 0: scalar beta, b = w = beta */
+    int32_t dtype;        /* gdn_dtype of q, k, v, z, o */
+    int32_t gate_dtype;   /* gdn_dtype of alpha, b, w */
+} gdn_fwd_args;
+
+GDN_API size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args);
+GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size_t workspace_bytes,
+                         gdn_stream stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Chunkwise backward.  Reverse mode of gdn_chunk_fwd (without z): the chunk-boundary states are
+ * recomputed, the state gradient is scanned from the last chunk to the first, and per chunk the
+ * gradients of the auxiliary matrices carry the channel gates b and w inside their accumulation
+ * (GDN-2 summary, «Passage Arrière Conscient des Portes»).
+ * grad_alpha is the gradient with respect to alpha itself (not log alpha).  grad_q and grad_k are summed
+ * over the value heads that share a key head, in a fixed order (deterministic).
+ * ------------------------------------------------------------------------------------------ */
+typedef struct gdn_bwd_args {
+    const void* q;        /* forward inputs, same layouts and dtypes as gdn_fwd_args */
+    const void* k;
+    const void* v;
+    const void* alpha;
+    const void* b;
+    const void* w;
+    const float* h0;      /* NULL = zeros */
+    const int32_t* head_map;
+    const void* grad_o;   /* [B,T,Hv,dv] dtype, gradient of o */
+    const float* grad_ht; /* [B,Hv,dk,dv] gradient of the final state, NULL = zeros */
+    void* grad_q;         /* out [B,T,Hk,dk] dtype */
+    void* grad_k;         /* out [B,T,Hk,dk] dtype */
+    void* grad_v;         /* out [B,T,Hv,dv] dtype */
+    void* grad_alpha;     /* out, shape of alpha, gate_dtype */
+    void* grad_b;         /* out, shape of b (grad of beta [B,T,Hv] when gates are scalar) */
+    void* grad_w;         /* out, shape of w; must be NULL when gates are scalar */
+    float* grad_h0;       /* out [B,Hv,dk,dv], may be NULL */
+    int64_t B, T, Hk, Hv, dk, dv;
+    float scale;
+    int32_t alpha_per_channel;
+    int32_t gates_per_channel;
+    int32_t dtype;
+    int32_t gate_dtype;
+} gdn_bwd_args;
+
+GDN_API size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args);
+GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args* args, void* workspace, size_t workspace_bytes,
+                         gdn_stream stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Single-token decode step for N sequences: the recurrence applied once, with the fp32 state
+ * read, updated and written back in place (constant memory per sequence; mkdocs chapter «Gated
+ * DeltaNet», «L'état, en mémoire»).
+ * Optional fusions (mkdocs chapter «La convolution causale», «La porte de sortie»; explainer
+ * Figure 1 caption):
+ *  - conv_state != NULL: q, k, v are the raw projections of the new token; each of the
+ *    Cch = 2*Hk*dk + Hv*dv channels (ordered q, k, v) is convolved with its 4 taps over the
+ *    3 stored previous inputs and the new one (conv_w[ch][3] weights the new token), passed
+ *    through SiLU, and q, k are L2-normalised (x / sqrt(sum x^2 + 1e-6)); conv_state
+ *    [N, Cch, 3] (dtype, oldest first) is then shifted to hold the last 3 inputs.
+ *  - z != NULL: o <- o * z * sigmoid(z).
+ * ------------------------------------------------------------------------------------------ */
+typedef struct gdn_decode_args {
+    const void* q;        /* [N,Hk,dk] dtype */
+    const void* k;        /* [N,Hk,dk] dtype */
+    const void* v;        /* [N,Hv,dv] dtype */
+    const void* alpha;    /* [N,Hv,dk] or [N,Hv], gate_dtype */
+    const void* b;        /* [N,Hv,dk] or beta [N,Hv] */
+    const void* w;        /* [N,Hv,dv] or NULL */
+    float* state;         /* in/out [N,Hv,dk,dv] fp32, updated in place */
+    void* o;              /* out [N,Hv,dv] dtype */
+    const int32_t* head_map;
+    void* conv_state;     /* optional in/out [N, 2*Hk*dk + Hv*dv, 3] dtype */
+    const void* conv_w;   /* [2*Hk*dk + Hv*dv, 4] dtype, required with conv_state */
+    const void* z;        /* optional [N,Hv,dv] dtype */
+    int64_t N, Hk, Hv, dk, dv;
+    float scale;
+    int32_t alpha_per_channel;
+    int32_t gates_per_channel;
+    int32_t dtype;
+    int32_t gate_dtype;
+} gdn_decode_args;
+
+GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, gdn_stream stream);
+
+/* ------------------------------------------------------------------------------------------
+ * GQA layer core (forward): causal depthwise convolution (kernel 4, no bias, zero history)
+ * + SiLU on the q, k, v projections, L2 normalisation of q and k, the chunkwise recurrence, and
+ * the swish(z) output gate.  Explainer «Architecture et versions hybrides» (Figure 1 caption);
+ * mkdocs chapter «Gated DeltaNet» (16 key heads, 128 value heads, kernel 4, swish gate).
+ * Convolution channels are ordered q (Hk*dk), k (Hk*dk), v (Hv*dv); conv_w is [Cch, 4] with
+ * conv_w[ch][3] weighting the current token.  conv_state_out, if not NULL, receives the last
+ * three raw inputs of every channel ([B, Cch, 3], dtype) so that decoding can continue.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct gdn_layer_args {
+    const void* xq;       /* [B,T,Hk,dk] dtype (pre-convolution projections) */
+    const void* xk;       /* [B,T,Hk,dk] */
+    const void* xv;       /* [B,T,Hv,dv] */
+    const void* conv_w;   /* [Cch, 4] dtype */
+    const void* alpha;    /* as gdn_fwd_args */
+    const void* b;
+    const void* w;
+    const void* z;        /* [B,T,Hv,dv] swish gate, required */
+    const float* h0;      /* NULL = zeros */
+    void* y;              /* out [B,T,Hv,dv] dtype */
+    float* ht;            /* out, may be NULL */
+    void* conv_state_out; /* out, may be NULL */
+    const int32_t* head_map;
+    int64_t B, T, Hk, Hv, dk, dv;
+    float scale;
+    int32_t alpha_per_channel;
+    int32_t gates_per_channel;
+    int32_t dtype;
+    int32_t gate_dtype;
+} gdn_layer_args;
+
+GDN_API size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* args);
+GDN_API gdn_status gdn_layer_core_fwd(const gdn_layer_args* args, void* workspace, size_t workspace_bytes,
+                              gdn_stream stream);
+
+/* Thread-local description of the calling thread's last failure ("" if none). */
+GDN_API const char* gdn_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GDN_API int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_H */

@@ -1,0 +1,117 @@
+"""The C ABI library loads, exports every symbol include/gdn.h declares, its ctypes structs match
+the C layouts, and host-side argument validation rejects bad calls before any launch.
+Runs without a GPU: no call here reaches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from gated_delta_rule_76_b200 import build as gbuild
+from gated_delta_rule_76_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gbuild.build()
+    return gdn.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(gdn.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gdn_\w+)", out))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert hasattr(lib, f)
+    assert lib.gdn_version() >= 100
+
+
+STRUCTS = {"gdn_fwd_args": gdn.FwdArgs, "gdn_bwd_args": gdn.BwdArgs,
+           "gdn_decode_args": gdn.DecodeArgs, "gdn_layer_args": gdn.LayerArgs}
+
+
+def test_ctypes_structs_match_c_layout():
+    """Compile a host program that prints sizeof/offsetof of every field of every struct."""
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "gdn.h"', "int main(void) {"]
+    for cname, py in STRUCTS.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines.append("return 0; }")
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        open(src, "w").write("\n".join(lines))
+        subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), src, "-o", exe])
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {}
+    for line in out:
+        if line.strip():
+            parts = line.split()
+            got[(parts[0], parts[1])] = int(parts[2])
+    for cname, py in STRUCTS.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def _fwd(**kw):
+    base = dict(q=16, k=32, v=48, alpha=64, b=80, w=96, h0=None, z=None, o=1 << 20, ht=None,
+                head_map=None, B=1, T=64, Hk=1, Hv=1, dk=64, dv=64, scale=1.0,
+                alpha_per_channel=1, gates_per_channel=1, dtype=0, gate_dtype=0)
+    base.update(kw)
+    return gdn.FwdArgs(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=96, dv=96), 2),                  # unsupported head size
+    (dict(dk=64, dv=128), 2),                 # dk != dv
+    (dict(Hk=3, Hv=4), 1),                    # Hv not a multiple of Hk without a map
+    (dict(B=0), 1),
+    (dict(q=None), 1),                        # missing input
+    (dict(w=None), 1),                        # channel gates without w
+    (dict(gates_per_channel=0), 1),           # scalar gates but w given
+    (dict(dtype=1, gate_dtype=0), 2),         # fp32 tensors with bf16 gates
+    (dict(q=18), 1),                          # misaligned
+    (dict(o=32), 1),                          # output overlaps an input
+    (dict(dtype=7), 1),
+])
+def test_host_validation_rejects_before_launch(lib, kw, code):
+    a = _fwd(**kw)
+    ws = ctypes.c_void_p(1 << 30)
+    rc = lib.gdn_chunk_fwd(ctypes.byref(a), ws, 1 << 30, None)
+    assert rc == code, lib.gdn_last_error()
+    assert lib.gdn_last_error().decode()
+
+
+def test_workspace_checks(lib):
+    a = _fwd()
+    need = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a))
+    assert need > 0
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), None, 0, None) == 4
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), need - 1, None) == 4
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p((1 << 30) + 16), need, None) == 4
+    assert lib.gdn_chunk_fwd(None, None, 0, None) == 1
+
+
+def test_workspace_size_scales_with_chunks(lib):
+    small = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(_fwd(T=64)))
+    big = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(_fwd(T=65)))
+    assert big > small  # a ragged tail adds a chunk
+    assert lib.gdn_chunk_fwd_workspace_size(None) == 0
