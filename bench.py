@@ -1,0 +1,591 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule library on B200.
+
+`python bench.py --gpus N --steps K --warmup W` prints ONE JSON line.
+
+Headline (`value`): GDN-2 chunkwise forward + backward tokens/s on the workload
+B=8, T=4096, H=16, dk=dv=128, bf16 inputs, fp32 state, chunk 64 (whole job over all ranks; one
+step = one gdn_chunk_fwd + one gdn_chunk_bwd over the batch).  The same run also measures the
+decode step (256 sequences x 1024 tokens, H=16, d=128; "decode"), the forward alone, the
+scalar-gate Gated DeltaNet forward and the GQA layer core ("parts"), each with its roofline.
+
+Timing: CUDA events on the launching stream, W untimed warm-up steps, K timed steps bracketed
+by a barrier and a device synchronisation, max over ranks.  Every workload's inputs are larger
+than the 126 MB L2, so no flush is needed between steps.  Multi-GPU runs (torchrun) shard
+nothing: every rank runs the full per-GPU workload (weak scaling, no collective on the data
+path).
+
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN-2 chunkwise fwd+bwd tokens/s and decode tokens/s on 1 B200; % roofline"
+HEADLINE = "gdn2_fwd_bwd_bf16"
+DECODE = "gdn2_decode_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------------------------
+# algorithmic work per token (all heads of one token), from the recurrence's definition
+# --------------------------------------------------------------------------------------------
+def _es(dt):
+    return 4 if dt == "f32" else 2
+
+
+def fwd_bytes_per_token(wl, T=None, with_h0=None, gate=False):
+    """API-level bytes of one forward token: inputs read + output written (+ states amortised)."""
+    T = T or wl.T
+    es, gs = _es(wl.dtype), _es(wl.gate_dtype)
+    b = wl.Hk * 2 * wl.dk * es                                     # q, k
+    b += wl.Hv * wl.dv * es * 2                                    # v, o
+    b += wl.Hv * (wl.dk if wl.alpha_per_channel else 1) * gs       # alpha
+    b += wl.Hv * ((wl.dk + wl.dv) if wl.gates_per_channel else 1) * gs  # b, w or beta
+    if gate:
+        b += wl.Hv * wl.dv * es                                    # z
+    nstates = 1 + (1 if (wl.has_h0 if with_h0 is None else with_h0) else 0)
+    b += nstates * wl.Hv * wl.dk * wl.dv * 4 / T
+    return b
+
+
+def bwd_bytes_per_token(wl, T=None):
+    """Reads q, k, v, alpha, b, w, dO (+ h0); writes fp32 dq, dk, dv, dalpha, db, dw (+ dh0)."""
+    T = T or wl.T
+    es, gs = _es(wl.dtype), _es(wl.gate_dtype)
+    n_qk = wl.Hk * 2 * wl.dk
+    n_v = wl.Hv * wl.dv
+    n_a = wl.Hv * (wl.dk if wl.alpha_per_channel else 1)
+    n_g = wl.Hv * ((wl.dk + wl.dv) if wl.gates_per_channel else 1)
+    b = (n_qk + n_v) * es + (n_a + n_g) * gs + n_v * es           # inputs and dO read
+    b += (n_qk + n_v + n_a + n_g) * 4                              # fp32 gradients written
+    b += (2 if wl.has_h0 else 1) * wl.Hv * wl.dk * wl.dv * 4 / T   # h0 read, dh0 written
+    return b
+
+
+def fwd_flops_per_token(wl, C=64):
+    d = wl.dk
+    return wl.Hv * (5 * 2 * C * d + 3 * 2 * d * d)
+
+
+def bwd_flops_per_token(wl, C=64):
+    return 2 * fwd_flops_per_token(wl, C) + wl.Hv * 4 * C * C
+
+
+def decode_bytes_per_token(wl):
+    es, gs = _es(wl.dtype), _es(wl.gate_dtype)
+    b = wl.Hv * 2 * wl.dk * wl.dv * 4                              # state read + write
+    b += wl.Hk * 2 * wl.dk * es + wl.Hv * 2 * wl.dv * es           # q, k, v, o
+    b += wl.Hv * ((wl.dk if wl.alpha_per_channel else 1) + ((wl.dk + wl.dv) if wl.gates_per_channel else 1)) * gs
+    return b
+
+
+def decode_flops_per_token(wl):
+    return wl.Hv * 7 * wl.dk * wl.dv
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False):
+    t_mem = bytes_per_launch / (peaks["hbm_gbs"] * 1e9)
+    fpk = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    t_flop = flops_per_launch / (fpk * 1e12)
+    if t_mem >= t_flop:
+        achieved = bytes_per_launch / seconds / 1e9
+        out = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+               "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    else:
+        achieved = flops_per_launch / seconds / 1e12
+        out = {"bound": "tensor", "achieved": round(achieved, 2), "peak": fpk, "unit": "TFLOP/s",
+               "frac": round(achieved / fpk, 4)}
+    out.update({"traffic": None, "peak_source": peak_kind, "scope": scope,
+                "algorithmic_bytes": int(bytes_per_launch), "algorithmic_flops": int(flops_per_launch)})
+    return out
+
+
+# --------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["index", "pci.bus_id", "clocks.sm", "clocks.max.sm", "power.draw",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, bus_id=None, index=None):
+        self.bus_id, self.index = bus_id, index
+        self.proc = None
+        self.out = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.out.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        rows = []
+        for line in self.out:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            if self.bus_id and parts[1].lower()[-12:] != self.bus_id.lower()[-12:]:
+                continue
+            if self.bus_id is None and self.index is not None and parts[0] != str(self.index):
+                continue
+            rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[2]) for r in rows]
+        smax = max(float(r[3]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[4]) for r in rows if r[4] not in ("[N/A]", ""))}
+
+
+# --------------------------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------------------------
+class Dist:
+    def __init__(self, ngpus):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        elif torch.cuda.is_available():
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def timed(fn, steps, warmup, dist, stream):
+    """Device time per step (ms) of fn(), CUDA events on `stream`, max over ranks."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = a.elapsed_time(b) / steps
+    return dist.max(ms)
+
+
+# --------------------------------------------------------------------------------------------
+# workloads
+# --------------------------------------------------------------------------------------------
+def chunk_inputs(name, device, with_dout):
+    import torch
+    from gated_delta_rule_76_b200.inputs import workload_inputs
+    x = workload_inputs(name, with_dout=with_dout)
+    return x, {k: v.to(device) for k, v in x.items() if torch.is_tensor(v)}
+
+
+def gates(g):
+    return dict(beta=g["beta"]) if "beta" in g else dict(b=g["b"], w=g["w"])
+
+
+def bench_headline(args, dist, peaks, peak_kind, stream, device):
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import WORKLOADS
+    wl = WORKLOADS[HEADLINE]
+    x, g = chunk_inputs(HEADLINE, device, with_dout=True)
+    B, T = wl.B, wl.T
+    o = torch.empty_like(g["v"])
+    ht = torch.empty((B, wl.Hv, wl.dk, wl.dv), dtype=torch.float32, device=device)
+    fa, _ = gdn.fwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], o=o, ht=ht, **gates(g))
+    import ctypes
+    lib = gdn.load()
+    ws_f = torch.empty(lib.gdn_chunk_fwd_workspace_size(ctypes.byref(fa)), dtype=torch.uint8, device=device)
+    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=device)
+    grads = {"dq": f32(g["q"]), "dk": f32(g["k"]), "dv": f32(g["v"]), "dalpha": f32(g["alpha"]),
+             "db": f32(g["b"]), "dw": f32(g["w"]), "dh0": f32(g["h0"])}
+    ba, _ = gdn.bwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], grads=grads, **gates(g))
+    ws_b = torch.empty(lib.gdn_chunk_bwd_workspace_size(ctypes.byref(ba)), dtype=torch.uint8, device=device)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+
+    def fwd():
+        gdn.check(lib.gdn_chunk_fwd(ctypes.byref(fa), ctypes.c_void_p(ws_f.data_ptr()), ws_f.numel(), sptr), "fwd")
+
+    def bwd():
+        gdn.check(lib.gdn_chunk_bwd(ctypes.byref(ba), ctypes.c_void_p(ws_b.data_ptr()), ws_b.numel(), sptr), "bwd")
+
+    # per-call device times inside the timed step (for the dominant call's roofline)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    per_call = {"fwd": [], "bwd": []}
+
+    def step_timed():
+        ev[0].record(stream)
+        fwd()
+        ev[1].record(stream)
+        bwd()
+        ev[2].record(stream)
+
+    launches0 = gdn.kernel_launches()
+    with torch.cuda.stream(stream):
+        ms = timed(lambda: (fwd(), bwd()), args.steps, args.warmup, dist, stream)
+    launches = gdn.kernel_launches() - launches0
+    launches_per_step = launches // (args.steps + args.warmup)
+    # separate pass for the per-call split (not part of the headline number)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.steps // 2)):
+            step_timed()
+            torch.cuda.synchronize()
+            per_call["fwd"].append(ev[0].elapsed_time(ev[1]))
+            per_call["bwd"].append(ev[1].elapsed_time(ev[2]))
+    fwd_ms = float(np.mean(per_call["fwd"]))
+    bwd_ms = float(np.mean(per_call["bwd"]))
+    tokens = B * T
+    bytes_f = fwd_bytes_per_token(wl) * tokens
+    bytes_b = bwd_bytes_per_token(wl) * tokens
+    flops_f = fwd_flops_per_token(wl) * tokens
+    flops_b = bwd_flops_per_token(wl) * tokens
+    dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
+    dom = {"fwd": (bytes_f, flops_f, fwd_ms), "bwd": (bytes_b, flops_b, bwd_ms)}[dominant]
+    roof = roofline(dom[0], dom[1], dom[2] * 1e-3, peaks, peak_kind,
+                    f"gdn_chunk_{dominant} call (dominant call of the step; its kernels back to back)")
+    step_roof = roofline(bytes_f + bytes_b, flops_f + flops_b, ms * 1e-3, peaks, peak_kind,
+                         "whole fwd+bwd step")
+    return {"ms": ms, "tokens": tokens, "launches_per_step": launches_per_step, "fwd_ms": fwd_ms,
+            "bwd_ms": bwd_ms, "roofline": roof, "step_roofline": step_roof,
+            "fwd_roofline": roofline(bytes_f, flops_f, fwd_ms * 1e-3, peaks, peak_kind, "gdn_chunk_fwd call")}, (x, g, o, ht, grads)
+
+
+def bench_headline_e2e(args, dist, x, stream, device):
+    """Same metric through the public API with host buffers: H2D of the step's inputs from pinned
+    memory, forward + backward, D2H of every result, all inside the timed region."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    names_in = ["q", "k", "v", "alpha", "b", "w", "h0", "dout"]
+    host = {n: x[n].pin_memory() for n in names_in}
+    dev = {n: torch.empty_like(host[n], device=device) for n in names_in}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    out_host = {}
+
+    def step():
+        for n in names_in:
+            dev[n].copy_(host[n], non_blocking=True)
+        o, ht = gdn.gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
+                                  h0=dev["h0"], stream=stream)
+        gr = gdn.gdn_chunk_bwd(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
+                               h0=dev["h0"], grad_o=dev["dout"], stream=stream)
+        res = {"o": o, "ht": ht, **gr}
+        for n, t in res.items():
+            if n not in out_host:
+                out_host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            out_host[n].copy_(t, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        ms = timed(step, max(2, args.steps // 4), 1, dist, stream)
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    return ms, h2d, d2h
+
+
+def bench_decode(args, dist, peaks, peak_kind, stream, device):
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import WORKLOADS, decode_initial_state, decode_inputs
+    wl = WORKLOADS[DECODE]
+    steps = wl.decode_steps
+    xs = decode_inputs(DECODE, steps, threads=min(16, os.cpu_count() or 4))
+    g = {k: v.to(device) for k, v in xs.items()}
+    state = decode_initial_state(DECODE).to(device)
+    o = torch.empty((steps, wl.B, wl.Hv, wl.dv), dtype=torch.bfloat16, device=device)
+
+    def run_all():
+        for s in range(steps):
+            gdn.gdn_decode_step(state, g["q"][s], g["k"][s], g["v"][s], g["alpha"][s], b=g["b"][s],
+                                w=g["w"][s], o=o[s], stream=stream)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        run_all()  # warm up (sets kernel attributes) before capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            run_all()
+        launches0 = gdn.kernel_launches()
+        ms = timed(graph.replay, max(2, args.steps // 4), max(1, args.warmup // 2), dist, stream)
+    tokens = wl.B * steps
+    per_step_s = ms * 1e-3 / steps
+    roof = roofline(decode_bytes_per_token(wl) * wl.B, decode_flops_per_token(wl) * wl.B, per_step_s, peaks,
+                    peak_kind, "decode_step_kernel (one launch = one token for 256 sequences x 16 heads)")
+
+    # e2e: per step, H2D of that step's inputs (pinned) and D2H of its output.
+    host = {k: v.pin_memory() for k, v in xs.items()}
+    dev = {k: torch.empty_like(v[0], device=device) for k, v in xs.items()}
+    oh = torch.empty((steps,) + tuple(o.shape[1:]), dtype=o.dtype, pin_memory=True)
+    e2e_steps = 256
+
+    def e2e():
+        for s in range(e2e_steps):
+            for k in dev:
+                dev[k].copy_(host[k][s], non_blocking=True)
+            gdn.gdn_decode_step(state, dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
+                                o=o[s], stream=stream)
+            oh[s].copy_(o[s], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_ms = timed(e2e, 2, 1, dist, stream)
+    h2d = sum(v[0].numel() * v.element_size() for v in host.values())
+    d2h = o[0].numel() * o.element_size()
+    return {"workload": DECODE, "value": tokens / (ms * 1e-3) * dist.world, "unit": "tokens/s",
+            "ms_per_1024_tokens": round(ms, 4), "us_per_token_step": round(per_step_s * 1e6, 2),
+            "graph": True, "roofline": roof,
+            "e2e": {"value": e2e_steps * wl.B / (e2e_ms * 1e-3) * dist.world, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+            "config": {"N": wl.B, "H": wl.Hv, "dk": wl.dk, "dv": wl.dv, "steps": steps,
+                       "state_bytes": wl.B * wl.Hv * wl.dk * wl.dv * 4, "l2": "state (268 MB) larger than L2"}}
+
+
+def bench_part_fwd(name, args, dist, peaks, peak_kind, stream, device):
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import WORKLOADS
+    wl = WORKLOADS[name]
+    x, g = chunk_inputs(name, device, with_dout=False)
+    o = torch.empty_like(g["v"])
+    ws = None
+    with torch.cuda.stream(stream):
+        if wl.conv:
+            def fn():
+                gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], y=o,
+                                       want_ht=True, stream=stream, **gates(g))
+        else:
+            def fn():
+                gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g.get("h0"), o=o, stream=stream,
+                                  **gates(g))
+        ms = timed(fn, max(2, args.steps // 2), args.warmup, dist, stream)
+    tokens = wl.B * wl.T
+    by = fwd_bytes_per_token(wl, gate=wl.swish_gate) * tokens
+    if wl.conv:
+        by += (2 * wl.Hk * wl.dk + wl.Hv * wl.dv) * 4 * _es(wl.dtype) / wl.T * wl.B * 0  # weights: negligible
+    fl = fwd_flops_per_token(wl) * tokens
+    del x, g
+    return {"workload": name, "value": tokens / (ms * 1e-3) * dist.world, "unit": "tokens/s",
+            "ms_per_step": round(ms, 4),
+            "roofline": roofline(by, fl, ms * 1e-3, peaks, peak_kind,
+                                 "gdn_layer_core_fwd call" if wl.conv else "gdn_chunk_fwd call"),
+            "config": {"B": wl.B, "T": wl.T, "Hk": wl.Hk, "Hv": wl.Hv, "dk": wl.dk, "dv": wl.dv,
+                       "alpha": "channel" if wl.alpha_per_channel else "scalar",
+                       "gates": "channel" if wl.gates_per_channel else "scalar beta"}}
+
+
+# --------------------------------------------------------------------------------------------
+# CPU oracle timings (baseline and reference arm)
+# --------------------------------------------------------------------------------------------
+def oracle_sample_run(x, nb, threads):
+    """Oracle forward + backward over the first nb sequences of the headline batch."""
+    from oracle import oracle
+    sl = {k: v[:nb] for k, v in x.items()}
+    t0 = time.perf_counter()
+    oracle.fwd(sl["q"], sl["k"], sl["v"], sl["alpha"], b=sl["b"], w=sl["w"], h0=sl["h0"], nthreads=threads)
+    oracle.bwd(sl["q"], sl["k"], sl["v"], sl["alpha"], b=sl["b"], w=sl["w"], h0=sl["h0"],
+               dout=sl["dout"], nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_threads():
+    from oracle import oracle
+    return oracle.threads()
+
+
+def cpu_baseline(x, wl):
+    threads = cpu_threads()
+    nb = 1
+    secs = oracle_sample_run(x, nb, threads)
+    tokens = nb * wl.T
+    return {"value": round(tokens / secs, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle forward+backward of {nb} of {wl.B} sequences ({nb * wl.Hv} (batch, head) "
+                      f"pairs x {wl.T} tokens, all heads of a token counted once), {secs:.1f} s wall"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle, as it stands, on the headline workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gated_delta_rule_76_b200.inputs import WORKLOADS, workload_inputs
+    wl = WORKLOADS[HEADLINE]
+    x = workload_inputs(HEADLINE, with_dout=True, B=1)
+    threads = cpu_threads()
+    for _ in range(args.warmup):
+        oracle_sample_run(x, 1, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_run(x, 1, threads)
+    secs = (time.perf_counter() - t0) / args.steps
+    value = wl.T / secs
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": HEADLINE, "B": wl.B, "T": wl.T, "H": wl.Hv,
+                                            "dk": wl.dk, "dv": wl.dv, "chunk": 64},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"one of {wl.B} sequences per step (16 (batch, head) pairs x {wl.T} "
+                                       f"tokens), forward + backward, fp64 sequential recurrence"},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--parts", default="all", help="all | headline | comma list of: decode,fwd,gdn,layer")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import WORKLOADS
+    gdn.load()  # fail loudly if the CUDA library is missing
+    dist = Dist(args.gpus)
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream(device=device)
+    peaks, peak_kind = load_peaks()
+    props = torch.cuda.get_device_properties(device)
+    bus = getattr(props, "pci_bus_id", None)
+    if isinstance(bus, int):
+        bus = None
+    parts = {"decode", "fwd", "gdn", "layer"} if args.parts == "all" else (
+        set() if args.parts == "headline" else set(args.parts.split(",")))
+    if dist.world > 1 and args.parts == "all":
+        parts = {"decode"}
+
+    clocks = ClockSampler(bus_id=bus, index=dist.local)
+    clocks.start()
+    head, keep = bench_headline(args, dist, peaks, peak_kind, stream, device)
+    x = keep[0]
+    del keep
+    torch.cuda.empty_cache()
+    e2e_ms, h2d, d2h = bench_headline_e2e(args, dist, x, stream, device)
+    torch.cuda.empty_cache()
+    extra = {}
+    if "decode" in parts:
+        extra["decode"] = bench_decode(args, dist, peaks, peak_kind, stream, device)
+        torch.cuda.empty_cache()
+    sub = {}
+    if "fwd" in parts:
+        sub["gdn2_fwd"] = {"workload": HEADLINE, "value": head["tokens"] / (head["fwd_ms"] * 1e-3) * dist.world,
+                           "unit": "tokens/s", "ms_per_step": round(head["fwd_ms"], 4),
+                           "roofline": head["fwd_roofline"]}
+    if "gdn" in parts:
+        sub["gdn_fwd_scalar"] = bench_part_fwd("gdn_fwd_scalar_bf16", args, dist, peaks, peak_kind, stream, device)
+        torch.cuda.empty_cache()
+    if "layer" in parts:
+        sub["gqa_layer_core"] = bench_part_fwd("gqa_layer_core_bf16", args, dist, peaks, peak_kind, stream, device)
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+
+    wl = WORKLOADS[HEADLINE]
+    value = head["tokens"] * dist.world / (head["ms"] * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(head["ms"], 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy draws, recipe in gated_delta_rule_76_b200/inputs.py)",
+        "config": {"workload": HEADLINE, "B": wl.B, "T": wl.T, "H": wl.Hv, "dk": wl.dk, "dv": wl.dv,
+                   "chunk": 64, "state": "fp32", "gates": "channel alpha, b, w (bf16)",
+                   "parallelism": f"dp{dist.world} (independent replicas of the workload)",
+                   "l2": "inputs larger than L2 (~0.9 GB read per step); no flush needed",
+                   "step": "gdn_chunk_fwd + gdn_chunk_bwd"},
+        "roofline": head["roofline"],
+        "step_roofline": head["step_roofline"],
+        "fwd_ms": round(head["fwd_ms"], 4), "bwd_ms": round(head["bwd_ms"], 4),
+        "e2e": {"value": round(head["tokens"] * dist.world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(head["launches_per_step"] * args.steps),
+        "clocks": clk,
+    }
+    line.update(extra)
+    if sub:
+        line["parts"] = sub
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, wl)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,5 +1,6 @@
 // C ABI of libgdn (see include/gdn.h): argument validation on the host, workspace carving and
 // dispatch to the kernels.  No device memory is allocated here and nothing synchronises.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -9,6 +10,12 @@
 #include "launch.h"
 
 namespace gdn {
+
+namespace {
+std::atomic<long long> g_launches{0};
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
@@ -211,10 +218,11 @@ gdn_status check_bwd(const gdn_bwd_args* a) {
         {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_o, BT * a->Hv * a->dv * es, "grad_o"}, {a->grad_ht, st, "grad_ht"},
     };
+    const size_t na4 = na / gs * 4, nb4 = nb / gs * 4;
     const Buf out[] = {
-        {a->grad_q, BT * a->Hk * a->dk * es, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * es, "grad_k"},
-        {a->grad_v, BT * a->Hv * a->dv * es, "grad_v"}, {a->grad_alpha, na, "grad_alpha"},
-        {a->grad_b, nb, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * gs, "grad_w"}, {a->grad_h0, st, "grad_h0"},
+        {a->grad_q, BT * a->Hk * a->dk * 4, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * 4, "grad_k"},
+        {a->grad_v, BT * a->Hv * a->dv * 4, "grad_v"}, {a->grad_alpha, na4, "grad_alpha"},
+        {a->grad_b, nb4, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * 4, "grad_w"}, {a->grad_h0, st, "grad_h0"},
     };
     return check_buffers(in, 10, out, 7);
 }
@@ -424,5 +432,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
 const char* gdn_last_error(void) { return g_last_error.c_str(); }
 
 int gdn_version(void) { return 100; }
+
+long long gdn_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -14,6 +14,7 @@ cudaError_t launch_kernel(K kernel, dim3 grid, dim3 block, size_t smem, cudaStre
         if (e != cudaSuccess) return e;
     }
     kernel<<<grid, block, smem, st>>>(args...);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -51,10 +52,10 @@ cudaError_t chunk_bwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
     if (!direct_qk) {
         const long total = (long)pb.B * pb.T * pb.Hk * pb.dk;
         const int blocks = static_cast<int>((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
-        GDN_TRY(launch_kernel(gqa_reduce_kernel<TIn>, dim3(blocks), dim3(256), 0, st, pb,
-                              (const float*)ws.dq_v, io.dq));
-        GDN_TRY(launch_kernel(gqa_reduce_kernel<TIn>, dim3(blocks), dim3(256), 0, st, pb,
-                              (const float*)ws.dk_v, io.dk));
+        GDN_TRY(launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb,
+                              (const float*)ws.dq_v, static_cast<float*>(io.dq)));
+        GDN_TRY(launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb,
+                              (const float*)ws.dk_v, static_cast<float*>(io.dk)));
     }
     return cudaSuccess;
 }

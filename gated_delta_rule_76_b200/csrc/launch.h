@@ -12,6 +12,9 @@
 
 namespace gdn {
 
+// Process-wide count of kernel launches issued by the library (gdn_kernel_launches()).
+void count_launch();
+
 struct Flags {
     bool apc;   // alpha per channel
     bool gpc;   // b, w per channel (else scalar beta)

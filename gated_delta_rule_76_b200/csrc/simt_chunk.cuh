@@ -400,8 +400,8 @@ chunk_scan_bwd_kernel(Problem pb, ChunkIO io, ChunkWs ws) {
                 const int t = t0 + r;
                 const long io_off = pb.v_row(b, t, hv) + j0 + j;
                 const float ww = to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
-                static_cast<TIn*>(io.dv)[io_off] = from_f32<TIn>(dY[idx] * ww);
-                if (GPC) static_cast<TG*>(io.dw)[io_off] = from_f32<TG>(dY[idx] * to_f32(vin[io_off]));
+                static_cast<float*>(io.dv)[io_off] = dY[idx] * ww;
+                if (GPC) static_cast<float*>(io.dw)[io_off] = dY[idx] * to_f32(vin[io_off]);
             }
         }
         if (!GPC && tid < C) {
@@ -544,8 +544,8 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
         for (int j = 0; j < GCK::TN; ++j) dk_acc[i][j] = dg_acc[i][j] = 0.f;
     }
     float* dq_out = nullptr;
-    TIn* dq_direct = nullptr;
-    if (direct_qk) dq_direct = static_cast<TIn*>(io.dq);
+    float* dq_direct = nullptr;
+    if (direct_qk) dq_direct = static_cast<float*>(io.dq);
     else dq_out = ws.dq_v;
     {   // dQhat = (scale dO) S0^T + dP Ktil
         GCK g;
@@ -561,7 +561,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
                 dg_acc[i][j] += v * Qh[r * DK + c];
                 if (r < L) {
                     const float gq = v * Gm[r * DK + c];
-                    if (direct_qk) dq_direct[pb.qk_row(b, t0 + r, hk) + c] = from_f32<TIn>(gq);
+                    if (direct_qk) dq_direct[pb.qk_row(b, t0 + r, hk) + c] = gq;
                     else dq_out[pb.v_row(b, t0 + r, hv) / pb.dv * DK + c] = gq;
                 }
             }
@@ -584,7 +584,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
                     const float kv = to_f32(kin[pb.qk_row(b, t, hk) + c]);
                     const float bv = to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]);
                     dk_acc[i][j] += de * bv;
-                    if (GPC) static_cast<TG*>(io.db)[pb.gate_row(b, t, hv, DK) + c] = from_f32<TG>(de * kv);
+                    if (GPC) static_cast<float*>(io.db)[pb.gate_row(b, t, hv, DK) + c] = de * kv;
                     else rsum[i] += de * kv;
                 }
             }
@@ -626,7 +626,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
     // Write dk; stage dg; deterministic column sums of dKbar .* Kbar.
     {
         GCK g;  // mapping only
-        TIn* dk_direct = static_cast<TIn*>(io.dk);
+        float* dk_direct = static_cast<float*>(io.dk);
 #pragma unroll
         for (int i = 0; i < GCK::TM; ++i) {
             const int r = g.row(i);
@@ -635,7 +635,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
                 const int c = g.col(j);
                 dg[r * DK + c] = dg_acc[i][j];
                 if (r < L) {
-                    if (direct_qk) dk_direct[pb.qk_row(b, t0 + r, hk) + c] = from_f32<TIn>(dk_acc[i][j]);
+                    if (direct_qk) dk_direct[pb.qk_row(b, t0 + r, hk) + c] = dk_acc[i][j];
                     else ws.dk_v[pb.v_row(b, t0 + r, hv) / pb.dv * DK + c] = dk_acc[i][j];
                 }
             }
@@ -678,7 +678,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
             const int r = idx / DK, c = idx % DK;
             if (r < L) {
                 const long off = pb.gate_row(b, t0 + r, hv, DK) + c;
-                static_cast<TG*>(io.dalpha)[off] = from_f32<TG>(dg[idx] / to_f32(al[off]));
+                static_cast<float*>(io.dalpha)[off] = dg[idx] / to_f32(al[off]);
             }
         }
     } else if (tid < C) {
@@ -687,7 +687,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
             float s = 0.f;
             for (int c = 0; c < DK; ++c) s += dg[r * DK + c];
             const long off = pb.gate_row(b, t0 + r, hv, 1);
-            static_cast<TG*>(io.dalpha)[off] = from_f32<TG>(s / to_f32(al[off]));
+            static_cast<float*>(io.dalpha)[off] = s / to_f32(al[off]);
         }
     }
     if (!GPC && tid < C) {
@@ -695,7 +695,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
         if (r < L) {
             float s = rowsum[r];
             for (int tl = 0; tl < ntile; ++tl) s += ws.dbw[(ci * ntile + tl) * C + r];
-            static_cast<TG*>(io.db)[pb.gate_row(b, t0 + r, hv, 1)] = from_f32<TG>(s);
+            static_cast<float*>(io.db)[pb.gate_row(b, t0 + r, hv, 1)] = s;
         }
     }
 }
@@ -706,9 +706,9 @@ constexpr size_t chunk_grad_smem() {
                             kChunk + BlockGemm<kChunk, DK, kSimtThreads, 32>::kScratch);
 }
 
-// Sum per-value-head dq/dk [B,T,Hv,dk] over the value heads of each key head, ascending hv.
-template <class TIn>
-__global__ void gqa_reduce_kernel(Problem pb, const float* part, void* out) {
+// Sum per-value-head dq/dk [B,T,Hv,dk] over the value heads of each key head, ascending hv
+// (fixed order: deterministic).
+static __global__ void gqa_reduce_kernel(Problem pb, const float* part, float* out) {
     const long total = (long)pb.B * pb.T * pb.Hk * pb.dk;
     for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total;
          idx += (long)gridDim.x * blockDim.x) {
@@ -719,7 +719,7 @@ __global__ void gqa_reduce_kernel(Problem pb, const float* part, void* out) {
         float s = 0.f;
         for (int hv = 0; hv < pb.Hv; ++hv)
             if (pb.key_head(hv) == hk) s += part[(bt * pb.Hv + hv) * pb.dk + c];
-        static_cast<TIn*>(out)[idx] = from_f32<TIn>(s);
+        out[idx] = s;
     }
 }
 

@@ -61,7 +61,7 @@ class LayerArgs(ctypes.Structure):
 
 EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
-            "gdn_layer_core_fwd", "gdn_last_error", "gdn_version"]
+            "gdn_layer_core_fwd", "gdn_last_error", "gdn_kernel_launches", "gdn_version"]
 
 _lib = None
 
@@ -94,11 +94,18 @@ def load(path: str = LIB_PATH):
     lib.gdn_layer_core_fwd.restype = ctypes.c_int
     lib.gdn_last_error.argtypes = []
     lib.gdn_last_error.restype = ctypes.c_char_p
+    lib.gdn_kernel_launches.argtypes = []
+    lib.gdn_kernel_launches.restype = ctypes.c_longlong
     lib.gdn_version.argtypes = []
     lib.gdn_version.restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
     return lib
+
+
+def kernel_launches() -> int:
+    """Kernels launched by libgdn in this process so far."""
+    return int(load().gdn_kernel_launches())
 
 
 def check(status: int, what: str):
@@ -217,15 +224,15 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
 def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
                   scale: float = 1.0, *, grad_o, grad_ht=None, want_dh0: bool = True,
                   workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """Chunkwise backward.  Returns dq, dk, dv, dalpha and db/dw (or dbeta), dh0."""
+    """Chunkwise backward.  Returns fp32 dq, dk, dv, dalpha and db/dw (or dbeta), dh0."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
-    grads = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
-             "dalpha": torch.empty_like(alpha)}
+    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=t.device)
+    grads = {"dq": f32(q), "dk": f32(k), "dv": f32(v), "dalpha": f32(alpha)}
     if gpc:
-        grads["db"] = torch.empty_like(b)
-        grads["dw"] = torch.empty_like(w)
+        grads["db"] = f32(b)
+        grads["dw"] = f32(w)
     else:
-        grads["dbeta"] = torch.empty_like(beta)
+        grads["dbeta"] = f32(beta)
     if want_dh0:
         B, T, Hk, dk = q.shape
         Hv, dv = v.shape[2], v.shape[3]

@@ -31,8 +31,9 @@
  *    DeltaNet», «Les projections d'entrée».
  *  - Sizes: dk, dv in {64, 128}; B, T, Hk, Hv >= 1 (T = 0 is accepted and does nothing but copy
  *    h0 to ht).  T need not be a multiple of the chunk length 64.
- *  - Dtypes: q, k, v, o, z, gradients of q/k/v in `dtype`; alpha, b, w, beta and their gradients
- *    in `gate_dtype`; states and their gradients are always fp32.
+ *  - Dtypes: q, k, v, o, z in `dtype`; alpha, b, w, beta in `gate_dtype`; states and every
+ *    gradient are fp32 (gradients leave the fp32 accumulators unrounded: several of them are
+ *    heavy-tailed, and a bf16 store alone would cost up to half an ulp of their largest entry).
  *  - Range: the chunked kernels factor the decay as exp(g_r) * exp(-g_s) inside a chunk of 64
  *    tokens (g = cumulative log alpha).  The product of alpha over one chunk must stay above
  *    1e-30 per channel, otherwise the factors overflow and the result is NaN/Inf (never a
@@ -119,12 +120,12 @@ typedef struct gdn_bwd_args {
     const int32_t* head_map;
     const void* grad_o;   /* [B,T,Hv,dv] dtype, gradient of o */
     const float* grad_ht; /* [B,Hv,dk,dv] gradient of the final state, NULL = zeros */
-    void* grad_q;         /* out [B,T,Hk,dk] dtype */
-    void* grad_k;         /* out [B,T,Hk,dk] dtype */
-    void* grad_v;         /* out [B,T,Hv,dv] dtype */
-    void* grad_alpha;     /* out, shape of alpha, gate_dtype */
-    void* grad_b;         /* out, shape of b (grad of beta [B,T,Hv] when gates are scalar) */
-    void* grad_w;         /* out, shape of w; must be NULL when gates are scalar */
+    float* grad_q;        /* out [B,T,Hk,dk] fp32 */
+    float* grad_k;        /* out [B,T,Hk,dk] fp32 */
+    float* grad_v;        /* out [B,T,Hv,dv] fp32 */
+    float* grad_alpha;    /* out, shape of alpha, fp32 */
+    float* grad_b;        /* out, shape of b (grad of beta [B,T,Hv] when gates are scalar), fp32 */
+    float* grad_w;        /* out, shape of w, fp32; must be NULL when gates are scalar */
     float* grad_h0;       /* out [B,Hv,dk,dv], may be NULL */
     int64_t B, T, Hk, Hv, dk, dv;
     float scale;
@@ -211,6 +212,10 @@ GDN_API gdn_status gdn_layer_core_fwd(const gdn_layer_args* args, void* workspac
 
 /* Thread-local description of the calling thread's last failure ("" if none). */
 GDN_API const char* gdn_last_error(void);
+
+/* Number of CUDA kernels this library has launched in the calling process so far (all
+ * devices and threads).  For benchmarking and diagnostics; it never resets. */
+GDN_API long long gdn_kernel_launches(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 GDN_API int gdn_version(void);
