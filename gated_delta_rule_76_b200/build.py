@@ -18,6 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdn.so")
+SELFTEST_LIB = os.path.join(PKG, "libgdn_selftest.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
@@ -35,27 +36,36 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _deps():
-    return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
-        + [os.path.join(INCLUDE, "gdn.h"), os.path.abspath(__file__)]
+def selftest_sources():
+    return sorted(glob.glob(os.path.join(CSRC, "selftest", "*.cu")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def _deps(srcs):
+    return srcs + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
+        + glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
+
+
+def up_to_date(lib, srcs) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in _deps())
+    t = os.path.getmtime(lib)
+    return all(os.path.getmtime(d) <= t for d in _deps(srcs))
 
 
 def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
-    if not force and up_to_date():
-        return LIB
+    """Build libgdn.so and the test-only libgdn_selftest.so; returns the libgdn.so path."""
+    _build_lib(SELFTEST_LIB, selftest_sources(), "selftest_", force, verbose, jobs)
+    return _build_lib(LIB, sources(), "", force, verbose, jobs)
+
+
+def _build_lib(lib, srcs, prefix, force, verbose, jobs):
+    if not force and up_to_date(lib, srcs):
+        return lib
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
-    srcs = sources()
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(BUILD, prefix + os.path.basename(src)[:-3] + ".o")
         cmd = [cc] + ARCH + NVCC_FLAGS + ["-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -64,15 +74,15 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
             raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}\n{r.stderr}")
         return obj
 
-    with ThreadPoolExecutor(max_workers=jobs or min(len(srcs), os.cpu_count() or 4)) as ex:
+    with ThreadPoolExecutor(max_workers=jobs or max(1, min(len(srcs), os.cpu_count() or 4))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + ".tmp"
-    cmd = [cc] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs + ["-lcuda"]
+    tmp = lib + ".tmp"
+    cmd = [cc] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

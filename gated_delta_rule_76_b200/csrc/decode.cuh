@@ -16,6 +16,7 @@ struct DecodeParams {
     const void* q; const void* k; const void* v;
     const void* alpha; const void* b; const void* w;
     float* state; void* o;
+    int o_f32;  // o written in fp32 instead of TIn
     const int32_t* head_map;
     const void* conv_state; const void* conv_w; const void* z;
     int N, Hk, Hv, dk, dv;
@@ -141,8 +142,13 @@ decode_step_kernel(DecodeParams p) {
                 ov[c] *= zz * sigmoidf_(zz);
             }
         }
+        if (p.o_f32) {
+            *reinterpret_cast<float4*>(static_cast<float*>(p.o) + ((long)n * p.Hv + hv) * DV + 4 * cq) =
+                make_float4(ov[0], ov[1], ov[2], ov[3]);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[c] = from_f32<TIn>(ov[c]);
+            for (int c = 0; c < 4; ++c) o[c] = from_f32<TIn>(ov[c]);
+        }
     }
 }
 

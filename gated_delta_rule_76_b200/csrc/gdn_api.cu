@@ -188,8 +188,9 @@ gdn_status check_fwd(const gdn_fwd_args* a) {
         {a->z, BT * a->Hv * a->dv * es, "z"},
         {a->head_map, (size_t)a->Hv * 4, "head_map"},
     };
+    if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
     const Buf out[] = {
-        {a->o, BT * a->Hv * a->dv * es, "o"},
+        {a->o, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "o"},
         {a->ht, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "ht"},
     };
     return check_buffers(in, 9, out, 2);
@@ -238,7 +239,7 @@ gdn_status check_workspace(void* ws, size_t have, size_t need) {
 ChunkIO io_from(const gdn_fwd_args* a) {
     ChunkIO io{};
     io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
-    io.z = a->z; io.h0 = a->h0; io.o = a->o; io.ht = a->ht;
+    io.z = a->z; io.h0 = a->h0; io.o = a->o; io.ht = a->ht; io.o_f32 = a->out_f32;
     return io;
 }
 
@@ -340,14 +341,15 @@ gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
         {a->w, N * a->Hv * a->dv * gs, "w"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->conv_w, cch * 4 * es, "conv_w"}, {a->z, N * a->Hv * a->dv * es, "z"},
     };
+    if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
     const Buf out[] = {
-        {a->o, N * a->Hv * a->dv * es, "o"}, {a->state, st, "state"},
+        {a->o, N * a->Hv * a->dv * (a->out_f32 ? 4 : es), "o"}, {a->state, st, "state"},
         {a->conv_state, a->conv_state ? N * cch * 3 * es : 0, "conv_state"},
     };
     if ((s = check_buffers(in, 9, out, 3))) return s;
     DecodeParams p{};
     p.q = a->q; p.k = a->k; p.v = a->v; p.alpha = a->alpha; p.b = a->b; p.w = a->w;
-    p.state = a->state; p.o = a->o; p.head_map = a->head_map; p.conv_state = a->conv_state;
+    p.state = a->state; p.o = a->o; p.o_f32 = a->out_f32; p.head_map = a->head_map; p.conv_state = a->conv_state;
     p.conv_w = a->conv_w; p.z = a->z;
     p.N = (int)a->N; p.Hk = (int)a->Hk; p.Hv = (int)a->Hv; p.dk = (int)a->dk; p.dv = (int)a->dv;
     p.scale = a->scale;
@@ -392,8 +394,9 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
         {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->z, BT * a->Hv * a->dv * es, "z"},
         {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
     };
+    if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
     const Buf out[] = {
-        {a->y, BT * a->Hv * a->dv * es, "y"}, {a->ht, st, "ht"},
+        {a->y, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "y"}, {a->ht, st, "ht"},
         {a->conv_state_out, (size_t)a->B * cch * 3 * es, "conv_state_out"},
     };
     if ((s = check_buffers(in, 10, out, 3))) return s;
@@ -423,7 +426,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     WsPlan plan = plan_chunk_ws(pb, false, false);
     ChunkIO io{};
     io.q = qc; io.k = kc; io.v = vc; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.z = a->z;
-    io.h0 = a->h0; io.o = a->y; io.ht = a->ht;
+    io.h0 = a->h0; io.o = a->y; io.ht = a->ht; io.o_f32 = a->out_f32;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
     e = run_fwd(var, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");

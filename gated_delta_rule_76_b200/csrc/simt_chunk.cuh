@@ -37,6 +37,7 @@ struct ChunkIO {
     const void *q, *k, *v, *alpha, *b, *w, *z;
     const float* h0;
     void* o;
+    int o_f32;  // o written in fp32 instead of TIn
     float* ht;
     const void* dout;
     const float* dht;
@@ -249,7 +250,8 @@ chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int sav
                             const float zz = to_f32(static_cast<const TIn*>(io.z)[off]);
                             ov *= zz * sigmoidf_(zz);
                         }
-                        o[off] = from_f32<TIn>(ov);
+                        if (io.o_f32) static_cast<float*>(io.o)[off] = ov;
+                        else o[off] = from_f32<TIn>(ov);
                     }
                 }
         }

@@ -31,7 +31,7 @@ class FwdArgs(ctypes.Structure):
                 ("z", P), ("o", P), ("ht", P), ("head_map", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -48,7 +48,7 @@ class DecodeArgs(ctypes.Structure):
                 ("o", P), ("head_map", P), ("conv_state", P), ("conv_w", P), ("z", P),
                 ("N", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
 
 
 class LayerArgs(ctypes.Structure):
@@ -56,7 +56,7 @@ class LayerArgs(ctypes.Structure):
                 ("z", P), ("h0", P), ("y", P), ("ht", P), ("conv_state_out", P), ("head_map", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
 
 
 EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
@@ -181,18 +181,20 @@ def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_ma
                 h0=_ptr(h0), z=_ptr(z), o=_ptr(o), ht=_ptr(ht), head_map=_ptr(hm),
                 B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                 alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
-                dtype=_dt(q), gate_dtype=_dt(alpha))
+                dtype=_dt(q), gate_dtype=_dt(alpha),
+                out_f32=int(o is not None and o.dtype == torch.float32 and q.dtype != torch.float32))
     return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm]
 
 
 def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
-                  scale: float = 1.0, *, o=None, ht=None, want_ht: bool = True,
+                  scale: float = 1.0, *, o=None, ht=None, want_ht: bool = True, out_f32: bool = False,
                   workspace: Optional[torch.Tensor] = None, stream=None):
-    """Chunkwise forward.  Returns (o [B,T,Hv,dv], ht [B,Hv,dk,dv] or None)."""
+    """Chunkwise forward.  Returns (o [B,T,Hv,dv], ht [B,Hv,dk,dv] or None).
+    ``out_f32`` writes o in fp32 (the unrounded accumulator) instead of the input dtype."""
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     if o is None:
-        o = torch.empty((B, T, Hv, dv), dtype=q.dtype, device=q.device)
+        o = torch.empty((B, T, Hv, dv), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
     if ht is None and want_ht:
         ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
     lib = load()
@@ -247,33 +249,34 @@ def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=N
 
 def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=None,
                     scale: float = 1.0, *, conv_state=None, conv_w=None, z=None, o=None,
-                    stream=None):
+                    out_f32: bool = False, stream=None):
     """One token for N sequences; ``state`` [N,Hv,dk,dv] fp32 is updated in place.  Returns o."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     N, Hk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if o is None:
-        o = torch.empty((N, Hv, dv), dtype=q.dtype, device=q.device)
+        o = torch.empty((N, Hv, dv), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
     hm = _head_map(head_map, q.device)
     a = DecodeArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
                    state=_ptr(state), o=_ptr(o), head_map=_ptr(hm), conv_state=_ptr(conv_state),
                    conv_w=_ptr(conv_w), z=_ptr(z), N=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                    alpha_per_channel=int(alpha.dim() == 3), gates_per_channel=gpc,
-                   dtype=_dt(q), gate_dtype=_dt(alpha))
+                   dtype=_dt(q), gate_dtype=_dt(alpha),
+                   out_f32=int(o.dtype == torch.float32 and q.dtype != torch.float32))
     check(load().gdn_decode_step(ctypes.byref(a), _stream(stream)), "gdn_decode_step")
     return o
 
 
 def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, h0=None,
                        head_map=None, scale: float = 1.0, *, want_ht: bool = True,
-                       want_conv_state: bool = False, y=None,
+                       want_conv_state: bool = False, y=None, out_f32: bool = False,
                        workspace: Optional[torch.Tensor] = None, stream=None):
     """GQA layer core forward.  Returns (y, ht or None, conv_state or None)."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
     if y is None:
-        y = torch.empty((B, T, Hv, dv), dtype=xq.dtype, device=xq.device)
+        y = torch.empty((B, T, Hv, dv), dtype=torch.float32 if out_f32 else xq.dtype, device=xq.device)
     ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=xq.device) if want_ht else None
     cs = (torch.empty((B, 2 * Hk * dk + Hv * dv, 3), dtype=xq.dtype, device=xq.device)
           if want_conv_state else None)
@@ -282,7 +285,8 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
                   b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
                   conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
                   dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
-                  gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha))
+                  gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha),
+                  out_f32=int(y.dtype == torch.float32 and xq.dtype != torch.float32))
     lib = load()
     need = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, xq.device, workspace)

@@ -86,7 +86,7 @@ typedef struct gdn_fwd_args {
     const void* w;        /* write gate [B,T,Hv,dv] if gates_per_channel, else must be NULL */
     const float* h0;      /* [B,Hv,dk,dv] initial state, NULL = zeros */
     const void* z;        /* optional swish output gate [B,T,Hv,dv] dtype: o <- o * z * sigmoid(z) */
-    void* o;              /* out [B,T,Hv,dv] dtype */
+    void* o;              /* out [B,T,Hv,dv] dtype (fp32 if out_f32) */
     float* ht;            /* out [B,Hv,dk,dv] final state, may be NULL */
     const int32_t* head_map; /* [Hv] value head -> key head, NULL = contiguous groups */
     int64_t B, T, Hk, Hv, dk, dv;
@@ -95,6 +95,7 @@ typedef struct gdn_fwd_args {
     int32_t gates_per_channel; /* 1: separate b (dk) and w (dv); 0: scalar beta, b = w = beta */
     int32_t dtype;        /* gdn_dtype of q, k, v, z, o */
     int32_t gate_dtype;   /* gdn_dtype of alpha, b, w */
+    int32_t out_f32;      /* 1: o is written in fp32 (unrounded accumulator) instead of dtype */
 } gdn_fwd_args;
 
 GDN_API size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args);
@@ -171,6 +172,7 @@ typedef struct gdn_decode_args {
     int32_t gates_per_channel;
     int32_t dtype;
     int32_t gate_dtype;
+    int32_t out_f32;      /* 1: o is written in fp32 instead of dtype */
 } gdn_decode_args;
 
 GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, gdn_stream stream);
@@ -204,6 +206,7 @@ typedef struct gdn_layer_args {
     int32_t gates_per_channel;
     int32_t dtype;
     int32_t gate_dtype;
+    int32_t out_f32;      /* 1: y is written in fp32 instead of dtype */
 } gdn_layer_args;
 
 GDN_API size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* args);

@@ -41,3 +41,11 @@ def assert_parity(gpu, ref, kind: str, name: str = ""):
 
 def kind_of(t: torch.Tensor) -> str:
     return "f32" if t.dtype == torch.float32 else "bf16"
+
+
+def assert_bf16_is_rounding(out_bf16: torch.Tensor, out_f32: torch.Tensor, name: str = ""):
+    """A bf16 output must be exactly the round-to-nearest-even of the same call's fp32 output.
+    (The parity bound is checked on the fp32 output: a bf16 store alone costs up to 2^-8 of
+    the largest entry, which on heavy-tailed outputs exceeds 2e-2 of the RMS by itself.)"""
+    assert out_bf16.dtype == torch.bfloat16 and out_f32.dtype == torch.float32
+    assert torch.equal(out_bf16, out_f32.to(torch.bfloat16)), f"{name}: bf16 output is not the rounded fp32 output"

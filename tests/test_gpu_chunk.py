@@ -7,7 +7,7 @@ import torch
 from gated_delta_rule_76_b200 import gdn
 from gated_delta_rule_76_b200.inputs import draw, workload_inputs
 from oracle import oracle
-from parity import assert_parity, kind_of, to_cuda
+from parity import assert_bf16_is_rounding, assert_parity, kind_of, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -39,14 +39,19 @@ def gate_kw(x):
 def test_chunk_fwd_matches_oracle(name):
     x, scale = make(name)
     g = to_cuda(x)
+    kind = kind_of(x["q"])
     o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g.get("h0"), scale=scale,
-                              **gate_kw(g))
+                              out_f32=True, **gate_kw(g))
     torch.cuda.synchronize()
     o_ref, ht_ref = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=x.get("h0"), scale=scale,
                                **gate_kw(x))
-    kind = kind_of(x["q"])
     assert_parity(o, o_ref, kind, "o")
     assert_parity(ht, ht_ref, kind, "ht")
+    if kind == "bf16":
+        o16, ht16 = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g.get("h0"),
+                                      scale=scale, **gate_kw(g))
+        assert_bf16_is_rounding(o16, o, "o")
+        assert torch.equal(ht16, ht)
 
 
 def test_tiny_fp32_workload_fwd():
@@ -78,9 +83,12 @@ def test_swish_gated_forward():
     z = torch.randn(x["v"].shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
     g = to_cuda(x)
     y, _ = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], b=g["b"], w=g["w"], h0=g["h0"],
-                             z=z.cuda())
+                             z=z.cuda(), out_f32=True)
     o_ref, _ = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], b=x["b"], w=x["w"], h0=x["h0"])
     assert_parity(y, oracle.swish_gate(o_ref, z), "bf16", "y")
+    y16, _ = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], b=g["b"], w=g["w"], h0=g["h0"],
+                               z=z.cuda())
+    assert_bf16_is_rounding(y16, y, "y")
 
 
 def test_explicit_head_map():
@@ -106,15 +114,16 @@ def test_split_sequence_carry_on_gpu():
     """Two calls with the first call's final state as the second's h0 equal one call."""
     x, _ = make("gdn2_bf16_ragged")
     g = to_cuda(x)
-    o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], b=g["b"], w=g["w"], h0=g["h0"])
+    o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], b=g["b"], w=g["w"], h0=g["h0"],
+                              out_f32=True)
     cut = 77
     sl = lambda t, a, b_: t[:, a:b_].contiguous()
     o1, h1 = gdn.gdn_chunk_fwd(sl(g["q"], 0, cut), sl(g["k"], 0, cut), sl(g["v"], 0, cut),
                                sl(g["alpha"], 0, cut), b=sl(g["b"], 0, cut), w=sl(g["w"], 0, cut),
-                               h0=g["h0"])
+                               h0=g["h0"], out_f32=True)
     o2, h2 = gdn.gdn_chunk_fwd(sl(g["q"], cut, None), sl(g["k"], cut, None), sl(g["v"], cut, None),
                                sl(g["alpha"], cut, None), b=sl(g["b"], cut, None),
-                               w=sl(g["w"], cut, None), h0=h1)
+                               w=sl(g["w"], cut, None), h0=h1, out_f32=True)
     assert_parity(torch.cat([o1, o2], 1), o, "bf16", "o split")
     assert_parity(h2, ht, "bf16", "ht split")
 

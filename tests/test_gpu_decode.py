@@ -7,7 +7,7 @@ import torch
 from gated_delta_rule_76_b200 import gdn
 from gated_delta_rule_76_b200.inputs import draw
 from oracle import oracle
-from parity import assert_parity, npf, to_cuda
+from parity import assert_bf16_is_rounding, assert_parity, npf, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -35,10 +35,17 @@ def test_decode_steps_match_oracle(N, Hk, Hv, d, apc, gpc, dtype, gdt):
         tk = lambda src, key: src[key][:, t].contiguous()
         gk = dict(beta=tk(g, "beta")) if not gpc else dict(b=tk(g, "b"), w=tk(g, "w"))
         xk = dict(beta=tk(x, "beta")) if not gpc else dict(b=tk(x, "b"), w=tk(x, "w"))
-        o = gdn.gdn_decode_step(state, tk(g, "q"), tk(g, "k"), tk(g, "v"), tk(g, "alpha"), scale=0.9, **gk)
+        s16 = state.clone()
+        o = gdn.gdn_decode_step(state, tk(g, "q"), tk(g, "k"), tk(g, "v"), tk(g, "alpha"), scale=0.9,
+                                out_f32=True, **gk)
         o_ref, ref_state = oracle.decode_step(ref_state, tk(x, "q"), tk(x, "k"), tk(x, "v"),
                                               tk(x, "alpha"), scale=0.9, **xk)
         assert_parity(o, o_ref, kind, f"o step {t}")
+        if kind == "bf16":
+            o16 = gdn.gdn_decode_step(s16, tk(g, "q"), tk(g, "k"), tk(g, "v"), tk(g, "alpha"),
+                                      scale=0.9, **gk)
+            assert_bf16_is_rounding(o16, o, f"o step {t}")
+            assert torch.equal(s16, state)
     assert_parity(state, ref_state, kind, "state")
 
 
@@ -58,7 +65,7 @@ def test_decode_with_conv_and_swish_gate():
         tk = lambda src, key: src[key][:, t].contiguous()
         o = gdn.gdn_decode_step(state, tk(g, "q"), tk(g, "k"), tk(g, "v"), tk(g, "alpha"),
                                 b=tk(g, "b"), w=tk(g, "w"), conv_state=conv_state,
-                                conv_w=g["conv_w"], z=tk(g, "z"))
+                                conv_w=g["conv_w"], z=tk(g, "z"), out_f32=True)
         # Oracle: conv (kernel 4) + SiLU over [history, new input], L2 on q, k, then the step.
         raw = np.concatenate([npf(tk(x, "q")).reshape(N, -1), npf(tk(x, "k")).reshape(N, -1),
                               npf(tk(x, "v")).reshape(N, -1)], axis=1)[:, None, :]
@@ -82,8 +89,10 @@ def test_layer_core_matches_oracle(apc, gpc):
     g = to_cuda(x)
     gk = dict(beta=g["beta"]) if not gpc else dict(b=g["b"], w=g["w"])
     y, ht, cs = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"],
-                                       want_conv_state=True, **gk)
+                                       want_conv_state=True, out_f32=True, **gk)
+    y16, _, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], **gk)
     torch.cuda.synchronize()
+    assert_bf16_is_rounding(y16, y, "y")
     xk = dict(beta=x["beta"]) if not gpc else dict(b=x["b"], w=x["w"])
     if gpc:
         # layer_core_fwd of the oracle takes scalar beta; compose by hand for channel gates

@@ -31,6 +31,16 @@ def test_header_declares_the_binding_names():
     assert declared_functions() == sorted(gdn.EXPORTED)
 
 
+def test_selftest_library_exports_its_header(lib):
+    text = open(os.path.join(ROOT, "include", "gdn_selftest.h")).read()
+    declared = sorted(set(re.findall(r"\b(gdn_selftest_\w+)\s*\(", text)))
+    assert declared
+    out = subprocess.run(["nm", "-D", "--defined-only", gbuild.SELFTEST_LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (gdn_\w+)", out))
+    assert set(declared) <= exported, set(declared) - exported
+
+
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
