@@ -10,33 +10,34 @@ namespace gdn {
 
 struct ConvParams {
     const void *xq, *xk, *xv, *conv_w;
-    void *q, *k, *v;      // outputs [B,T,Hk,d], [B,T,Hk,d], [B,T,Hv,d]
+    void *q, *k, *v;      // outputs [B,T,Hk,d], [B,T,Hk,d], [B,T,Hv,d] in TOut
     void* conv_state_out; // [B, Cch, 3] or null
     int B, T, Hk, Hv, d;
 };
 
-template <class TIn, int D>
+template <class TIn, class TOut, int D>
 __global__ void __launch_bounds__(256) conv_silu_l2_kernel(ConvParams p) {
     constexpr int PER = D / 32;  // channels per lane
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
     const int rows_per_tok = 2 * p.Hk + p.Hv;
     const long nrows = (long)p.B * p.T * rows_per_tok;
     if (warp >= nrows) return;
-    const int hrow = warp % rows_per_tok;
+    const int hrow = (int)(warp % rows_per_tok);
     const long bt = warp / rows_per_tok;
-    const int t = bt % p.T;
+    const int t = (int)(bt % p.T);
     const TIn* x;
-    TIn* out;
+    TOut* out;
     int H, h, ch0;
     bool norm;
     if (hrow < p.Hk) {
-        x = static_cast<const TIn*>(p.xq); out = static_cast<TIn*>(p.q); H = p.Hk; h = hrow;
+        x = static_cast<const TIn*>(p.xq); out = static_cast<TOut*>(p.q); H = p.Hk; h = hrow;
         ch0 = h * D; norm = true;
     } else if (hrow < 2 * p.Hk) {
-        x = static_cast<const TIn*>(p.xk); out = static_cast<TIn*>(p.k); H = p.Hk; h = hrow - p.Hk;
+        x = static_cast<const TIn*>(p.xk); out = static_cast<TOut*>(p.k); H = p.Hk; h = hrow - p.Hk;
         ch0 = p.Hk * D + h * D; norm = true;
     } else {
-        x = static_cast<const TIn*>(p.xv); out = static_cast<TIn*>(p.v); H = p.Hv; h = hrow - 2 * p.Hk;
+        x = static_cast<const TIn*>(p.xv); out = static_cast<TOut*>(p.v); H = p.Hv; h = hrow - 2 * p.Hk;
         ch0 = 2 * p.Hk * D + h * D; norm = false;
     }
     const TIn* cw = static_cast<const TIn*>(p.conv_w);
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(256) conv_silu_l2_kernel(ConvParams p) {
         scale = rsqrtf(ss + 1e-6f);
     }
 #pragma unroll
-    for (int i = 0; i < PER; ++i) out[(bt * H + h) * D + lane + 32 * i] = from_f32<TIn>(y[i] * scale);
+    for (int i = 0; i < PER; ++i) out[(bt * H + h) * D + lane + 32 * i] = from_f32<TOut>(y[i] * scale);
     // The last three raw inputs of each channel, for a decode that continues this sequence.
     if (p.conv_state_out && t == p.T - 1) {
         const long cch = 2L * p.Hk * D + (long)p.Hv * D;

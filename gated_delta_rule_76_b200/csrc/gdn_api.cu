@@ -239,7 +239,8 @@ gdn_status check_workspace(void* ws, size_t have, size_t need) {
 ChunkIO io_from(const gdn_fwd_args* a) {
     ChunkIO io{};
     io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
-    io.z = a->z; io.h0 = a->h0; io.o = a->o; io.ht = a->ht; io.o_f32 = a->out_f32;
+    io.z = a->z; io.h0 = a->h0; io.o = a->o; io.ht = a->ht; io.o_type = a->out_f32 ? 1 : 0;
+    io.z_bf16 = 0;
     return io;
 }
 
@@ -248,6 +249,7 @@ cudaError_t run_fwd(int var, const Problem& pb, const ChunkIO& io, const ChunkWs
     switch (var) {
         case 0: return bf16_chunk_fwd(pb, io, ws, f, st);
         case 1: return bf16_f32g_chunk_fwd(pb, io, ws, f, st);
+        case 3: return f32_bf16g_chunk_fwd(pb, io, ws, f, st);
         default: return f32_chunk_fwd(pb, io, ws, f, st);
     }
 }
@@ -367,8 +369,8 @@ gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
 size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    const size_t es = elem_size(a->dtype);
-    const size_t conv = align256((size_t)(a->B * a->T) * (2 * a->Hk * a->dk + a->Hv * a->dv) * es);
+    // q, k, v after the convolution are kept in fp32 between the two kernels.
+    const size_t conv = align256((size_t)(a->B * a->T) * (2 * a->Hk * a->dk + a->Hv * a->dv) * 4);
     return conv + plan_chunk_ws(pb, false, false).bytes;
 }
 
@@ -412,9 +414,9 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
     char* base = static_cast<char*>(workspace);
     void* qc = base;
-    void* kc = base + BT * a->Hk * a->dk * es;
-    void* vc = base + 2 * BT * a->Hk * a->dk * es;
-    const size_t conv_bytes = align256(BT * cch * es);
+    void* kc = base + BT * a->Hk * a->dk * 4;
+    void* vc = base + 2 * BT * a->Hk * a->dk * 4;
+    const size_t conv_bytes = align256(BT * cch * 4);
     ConvParams cp{};
     cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
     cp.q = qc; cp.k = kc; cp.v = vc; cp.conv_state_out = a->conv_state_out;
@@ -426,9 +428,12 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     WsPlan plan = plan_chunk_ws(pb, false, false);
     ChunkIO io{};
     io.q = qc; io.k = kc; io.v = vc; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.z = a->z;
-    io.h0 = a->h0; io.o = a->y; io.ht = a->ht; io.o_f32 = a->out_f32;
+    io.h0 = a->h0; io.o = a->y; io.ht = a->ht;
+    // fp32 intermediates: y is written in dtype (bf16 -> o_type 2) unless out_f32.
+    io.o_type = a->out_f32 || a->dtype == GDN_F32 ? 1 : 2;
+    io.z_bf16 = a->dtype == GDN_BF16;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
-    e = run_fwd(var, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
+    e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
 }
 

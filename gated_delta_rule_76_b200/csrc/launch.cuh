@@ -124,9 +124,11 @@ cudaError_t conv_impl(const ConvParams& p, cudaStream_t st) {
     const long rows = (long)p.B * p.T * (2L * p.Hk + p.Hv);
     const long blocks = (rows * 32 + 255) / 256;
     if (p.d == 128)
-        return launch_kernel(conv_silu_l2_kernel<TIn, 128>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p);
+        return launch_kernel(conv_silu_l2_kernel<TIn, float, 128>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                             st, p);
     if (p.d == 64)
-        return launch_kernel(conv_silu_l2_kernel<TIn, 64>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p);
+        return launch_kernel(conv_silu_l2_kernel<TIn, float, 64>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                             st, p);
     return cudaErrorInvalidValue;
 }
 

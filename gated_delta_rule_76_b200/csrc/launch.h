@@ -41,5 +41,6 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates
 GDN_DECLARE_LAUNCHERS(f32)        // fp32 tensors, fp32 gates
+GDN_DECLARE_LAUNCHERS(f32_bf16g)  // fp32 tensors, bf16 gates (layer-core intermediates)
 
 }  // namespace gdn

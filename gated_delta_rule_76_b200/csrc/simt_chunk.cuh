@@ -37,7 +37,8 @@ struct ChunkIO {
     const void *q, *k, *v, *alpha, *b, *w, *z;
     const float* h0;
     void* o;
-    int o_f32;  // o written in fp32 instead of TIn
+    int o_type;  // 0: o in TIn, 1: fp32, 2: bf16
+    int z_bf16;  // z stored as bf16 (else as TIn)
     float* ht;
     const void* dout;
     const float* dht;
@@ -247,10 +248,12 @@ chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int sav
                         const long off = pb.v_row(b, t0 + r, hv) + j0 + c;
                         float ov = pb.scale * g.acc[i][j];
                         if (GATE) {
-                            const float zz = to_f32(static_cast<const TIn*>(io.z)[off]);
+                            const float zz = io.z_bf16 ? to_f32(static_cast<const __nv_bfloat16*>(io.z)[off])
+                                                       : to_f32(static_cast<const TIn*>(io.z)[off]);
                             ov *= zz * sigmoidf_(zz);
                         }
-                        if (io.o_f32) static_cast<float*>(io.o)[off] = ov;
+                        if (io.o_type == 1) static_cast<float*>(io.o)[off] = ov;
+                        else if (io.o_type == 2) static_cast<__nv_bfloat16*>(io.o)[off] = from_f32<__nv_bfloat16>(ov);
                         else o[off] = from_f32<TIn>(ov);
                     }
                 }
