@@ -117,7 +117,7 @@ bool identity_heads(const Problem& pb) { return pb.Hk == pb.Hv && pb.head_map ==
 WsPlan plan_chunk_ws(const Problem& pb, bool bwd, bool gqa_partials) {
     WsPlan w{};
     const size_t nch = (size_t)pb.B * pb.Hv * pb.NT, C = kChunk, dk = pb.dk, dv = pb.dv;
-    size_t off = 0;
+    size_t off = 256;  // bytes [0, 256): device status word
     auto take = [&](size_t floats) {
         size_t o = off;
         off = align256(off + floats * sizeof(float));
@@ -244,6 +244,9 @@ ChunkIO io_from(const gdn_fwd_args* a) {
     return io;
 }
 
+// Status word at the start of every workspace, cleared at the start of each call.
+int* ws_status(void* ws) { return static_cast<int*>(ws); }
+
 cudaError_t run_fwd(int var, const Problem& pb, const ChunkIO& io, const ChunkWs& ws, Flags f,
                     cudaStream_t st) {
     switch (var) {
@@ -266,9 +269,15 @@ gdn_status copy_state(float* dst, const float* src, size_t bytes, cudaStream_t s
 
 extern "C" {
 
+static bool fwd_uses_tensor_cores(const gdn_fwd_args* a, const Problem& pb) {
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
+    return tc_fwd_eligible(pb, a->dtype == GDN_BF16, a->gate_dtype == GDN_BF16, f);
+}
+
 size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    if (fwd_uses_tensor_cores(a, pb)) return 256;
     return plan_chunk_ws(pb, false, false).bytes;
 }
 
@@ -280,11 +289,15 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
     const size_t sbytes = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
     if (a->T == 0) return copy_state(a->ht, a->h0, sbytes, st, "gdn_chunk_fwd");
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    WsPlan plan = plan_chunk_ws(pb, false, false);
-    if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
-    cudaError_t e = run_fwd(variant(a->dtype, a->gate_dtype), pb, io_from(a),
-                            carve_chunk_ws(plan, workspace), f, st);
+    const bool tc = fwd_uses_tensor_cores(a, pb);
+    WsPlan plan = plan_chunk_ws(pb, false, false);
+    if ((s = check_workspace(workspace, workspace_bytes, tc ? 256 : plan.bytes))) return s;
+    cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
+    if (e == cudaSuccess) {
+        if (tc) e = tc_chunk_fwd(pb, io_from(a), f, a->gate_dtype == GDN_BF16, ws_status(workspace), st);
+        else e = run_fwd(variant(a->dtype, a->gate_dtype), pb, io_from(a), carve_chunk_ws(plan, workspace), f, st);
+    }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_fwd");
 }
 
@@ -312,7 +325,8 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     io.dh0 = a->grad_h0;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
     ChunkWs ws = carve_chunk_ws(plan, workspace);
-    cudaError_t e;
+    cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_bwd");
     switch (variant(a->dtype, a->gate_dtype)) {
         case 0: e = bf16_chunk_bwd(pb, io, ws, f, direct, st); break;
         case 1: e = bf16_f32g_chunk_bwd(pb, io, ws, f, direct, st); break;
@@ -371,7 +385,7 @@ size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     // q, k, v after the convolution are kept in fp32 between the two kernels.
     const size_t conv = align256((size_t)(a->B * a->T) * (2 * a->Hk * a->dk + a->Hv * a->dv) * 4);
-    return conv + plan_chunk_ws(pb, false, false).bytes;
+    return 256 + conv + plan_chunk_ws(pb, false, false).bytes;
 }
 
 gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t workspace_bytes,
@@ -412,7 +426,9 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     }
     const size_t need = gdn_layer_core_fwd_workspace_size(a);
     if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
-    char* base = static_cast<char*>(workspace);
+    cudaError_t e0 = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
+    if (e0 != cudaSuccess) return cuda_fail(e0, "gdn_layer_core_fwd");
+    char* base = static_cast<char*>(workspace) + 256;
     void* qc = base;
     void* kc = base + BT * a->Hk * a->dk * 4;
     void* vc = base + 2 * BT * a->Hk * a->dk * 4;
@@ -435,6 +451,17 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
     e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
+}
+
+gdn_status gdn_workspace_status(const void* workspace, gdn_stream stream) {
+    if (!workspace) return fail(GDN_ERR_INVALID_ARG, "workspace is NULL");
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost,
+                                    static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_workspace_status");
+    if (word != 0) return fail(GDN_ERR_TIMEOUT, "a bounded wait inside a kernel expired (status %d)", word);
+    return GDN_OK;
 }
 
 const char* gdn_last_error(void) { return g_last_error.c_str(); }

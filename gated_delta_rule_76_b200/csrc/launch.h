@@ -38,6 +38,11 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
     cudaError_t NAME##_decode(const DecodeParams&, Flags, cudaStream_t);                       \
     cudaError_t NAME##_conv(const ConvParams&, cudaStream_t);
 
+// Tensor-core chunk forward (tc_fwd.cu): bf16 q/k/v with dk = dv = 128.
+bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags f);
+cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
+                         cudaStream_t st);
+
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates
 GDN_DECLARE_LAUNCHERS(f32)        // fp32 tensors, fp32 gates

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgdn.so")
 
 GDN_BF16, GDN_F32 = 0, 1
 _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
-           4: "GDN_ERR_WORKSPACE"}
+           4: "GDN_ERR_WORKSPACE", 5: "GDN_ERR_TIMEOUT"}
 
 P = ctypes.c_void_p
 I64 = ctypes.c_int64
@@ -61,7 +61,8 @@ class LayerArgs(ctypes.Structure):
 
 EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
-            "gdn_layer_core_fwd", "gdn_last_error", "gdn_kernel_launches", "gdn_version"]
+            "gdn_layer_core_fwd", "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches",
+            "gdn_version"]
 
 _lib = None
 
@@ -92,6 +93,8 @@ def load(path: str = LIB_PATH):
     lib.gdn_layer_core_fwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_layer_core_fwd.argtypes = [ctypes.POINTER(LayerArgs), P, ctypes.c_size_t, P]
     lib.gdn_layer_core_fwd.restype = ctypes.c_int
+    lib.gdn_workspace_status.argtypes = [P, P]
+    lib.gdn_workspace_status.restype = ctypes.c_int
     lib.gdn_last_error.argtypes = []
     lib.gdn_last_error.restype = ctypes.c_char_p
     lib.gdn_kernel_launches.argtypes = []

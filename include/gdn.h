@@ -64,6 +64,7 @@ typedef int gdn_status;
 #define GDN_ERR_UNSUPPORTED 2 /* valid but not implemented here: dk/dv outside {64,128}, dtype */
 #define GDN_ERR_CUDA 3        /* a CUDA call or kernel launch failed (message has the CUDA error) */
 #define GDN_ERR_WORKSPACE 4   /* workspace NULL or smaller than *_workspace_size() */
+#define GDN_ERR_TIMEOUT 5     /* a bounded wait inside a kernel expired (see gdn_workspace_status) */
 
 typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
 
@@ -212,6 +213,13 @@ typedef struct gdn_layer_args {
 GDN_API size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* args);
 GDN_API gdn_status gdn_layer_core_fwd(const gdn_layer_args* args, void* workspace, size_t workspace_bytes,
                               gdn_stream stream);
+
+/* Device-side status of the last call that used `workspace` (a chunk forward, backward or layer
+ * core).  The tensor-core kernels bound every internal wait; when one expires the kernel records
+ * it in the workspace, stops issuing work, releases its tensor memory and returns.  This call
+ * synchronises `stream`, returns GDN_ERR_TIMEOUT if such an expiry was recorded (GDN_OK
+ * otherwise) and does not clear the record (the next call on the workspace does). */
+GDN_API gdn_status gdn_workspace_status(const void* workspace, gdn_stream stream);
 
 /* Thread-local description of the calling thread's last failure ("" if none). */
 GDN_API const char* gdn_last_error(void);
