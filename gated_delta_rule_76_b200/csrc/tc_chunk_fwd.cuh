@@ -13,17 +13,26 @@
 //   X3 = Y^T T^T   with Y^T = Z^T - (Ehat S0)^T  (M = dv, N = 64, K = 64; A in tensor memory)
 //   X4 = V'^T P^T  accumulated onto (Qhat S0)^T  (M = dv, N = 64, K = 64)
 //   X5 = V'^T Kbar (B = Kbar^T, K-major)  (M = dv, N = dk, K = 64)
-// Thread j of the two scan warpgroups owns TMEM lane j (= value column j) and keeps its column
-// of the fp32 state in registers, split between the warpgroups by halves of dk.
 //
+// Precision.  A bf16 operand carries a relative rounding of up to 2^-9, and with seven rounded
+// operand families the output error reaches ~4% of its RMS at the largest entry.  Every derived
+// operand x is therefore carried as a pair hi = bf16(x), lo = bf16(x - hi) and the products take
+// the cross terms that matter (hi*hi + lo*hi + hi*lo), each in fp32 in tensor memory:
+//   X1: Ehat, Qhat and Ktil split (3 MMAs);  X2: S0 split, and Qhat split in Qhat S0 (2 + 3 MMAs);
+//   X3: Y split (2);  X4: V' and P split (3);  X5: V' and Kbar split (3).  T stays bf16.
+// This keeps the output within ~0.2% of its RMS of the exact result at the largest entry.
+//
+// Thread j of the two scan warpgroups owns TMEM lane j (= value column j) and keeps its column of
+// the fp32 state in registers, split between the warpgroups by halves of dk.
 // Roles (384 threads):
 //   warps 0-7  (scan)     : the sequential chain X2 -> Y -> X3 -> V' -> X4, X5 -> output, state;
-//                           thread 0 issues the scan's MMAs and the TMA loads.
-//   warps 8-11 (prologue) : for the next chunk, the cumulative decay and in-place scaling of the
-//                           TMA tiles, X1, the triangular solve T = (I + A)^-1, and Kbar^T.
-// Shared memory (~226 KB): two slots of raw tiles (q, k, alpha, b) that are transformed in place
-// into the MMA operands, two slots of v/w tiles, Kbar^T, a fp32 scratch for A.
-// Tensor memory: 480 of 512 columns.  Every mbarrier wait is bounded: on expiry the kernel sets
+//                           thread 0 issues the scan's MMAs and the v/w TMA loads.
+//   warps 8-11 (prologue) : for the next chunk, the cumulative decay and the split operands, X1,
+//                           the triangular solve T = (I + A)^-1, P and Kbar^T; thread 256 issues
+//                           X1 and the q/k/alpha/b TMA loads.
+// Operand tiles are single-buffered: each has a "ready" barrier (prologue -> scan) and a "free"
+// barrier (the scan's MMA that read it has completed -> prologue); the raw TMA stage is reloaded as
+// soon as X1 (its last reader) completes.  Every mbarrier wait is bounded: on expiry the kernel sets
 // an error word, stops issuing work and frees its tensor memory.
 #pragma once
 #include <cuda.h>
@@ -42,42 +51,48 @@ constexpr int kThreads = 384;
 constexpr uint64_t kWaitNs = 4000000000ull;
 
 // tensor memory columns
-constexpr uint32_t TM_X1 = 0;    // 64:  A (lanes 0-63), P (lanes 64-127), fp32
-constexpr uint32_t TM_X2 = 64;   // 128: (Ehat S0)^T | (Qhat S0 + P V')^T
-constexpr uint32_t TM_X3 = 192;  // 64:  V'^T fp32
-constexpr uint32_t TM_X5 = 256;  // 128: (Kbar^T V')^T
-constexpr uint32_t TM_S0 = 384;  // 64:  S0^T as bf16 pairs (A operand of X2)
-constexpr uint32_t TM_Y = 448;   // 32:  Y^T, then V'^T, as bf16 pairs (A operand of X3, X4, X5)
+constexpr uint32_t TM_X1 = 0;     // 64:  A (lanes 0-63), P (lanes 64-127), fp32
+constexpr uint32_t TM_X2 = 64;    // 128: (Ehat S0)^T | (Qhat S0 + P V')^T
+constexpr uint32_t TM_X5 = 192;   // 128: first V'^T = (Y^T T^T) in cols 0-63, then (Kbar^T V')^T
+constexpr uint32_t TM_S0H = 320;  // 64:  S0^T hi, bf16 pairs
+constexpr uint32_t TM_S0L = 384;  // 64:  S0^T lo
+constexpr uint32_t TM_YH = 448;   // 32:  Y^T (then V'^T) hi
+constexpr uint32_t TM_YL = 480;   // 32:  Y^T (then V'^T) lo
 constexpr uint32_t TM_COLS = 512;
 
-// shared memory offsets from the 1024-byte-aligned base
-constexpr uint32_t SLOT_BYTES = 65536;
-constexpr uint32_t OFF_EQ = 0;       // [2 atoms][128 rows][128 B]: rows 0-63 b -> Ehat, 64-127 q -> Qhat
-constexpr uint32_t OFF_KT = 32768;   // [2][64][128 B]: k -> Ktil
-constexpr uint32_t OFF_AL = 49152;   // [2][64][128 B]: alpha; later T (first 8 KB) and P (next 8 KB)
-constexpr uint32_t SM_VW = 131072;   // 2 slots x 32 KB: v [2][64][128B], w [2][64][128B]
-constexpr uint32_t VW_BYTES = 32768;
-constexpr uint32_t SM_KB = 196608;   // Kbar^T [1 atom][128 rows][128 B]
-constexpr uint32_t SM_ASCR = 212992; // A fp32 [64][64], float4 columns XOR-swizzled by row
-constexpr uint32_t SM_GAM = 229376;  // gamma, 3 slots x 128 floats (slot n % 3: the prologue runs at most
-                                     // two chunks ahead of the scan's last read of gamma)
-constexpr uint32_t SM_BAR = 230912;  // mbarriers, tensor memory base, abort flag
+// shared memory offsets from the 1024-byte-aligned base (K-major 128-byte-swizzled bf16 tiles)
+constexpr uint32_t SM_RQB = 0;        // 32 KB [2 atoms][128 rows]: TMA b (rows 0-63), q (64-127) -> [Ehat;Qhat] lo
+constexpr uint32_t SM_RK = 32768;     // 16 KB [2][64]: TMA k -> Ktil hi
+constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo
+constexpr uint32_t SM_EQ = 65536;     // 32 KB [2][128]: [Ehat;Qhat] hi
+constexpr uint32_t SM_QLO = 98304;    // 16 KB [2][64]: Qhat lo (for X2)
+constexpr uint32_t SM_T = 114688;     // 8 KB [1][64]: T
+constexpr uint32_t SM_P = 122880;     // 16 KB: P hi [1][64], P lo [1][64]
+constexpr uint32_t SM_KB = 139264;    // 32 KB: Kbar^T hi [1][128], Kbar^T lo [1][128]
+constexpr uint32_t SM_VW = 172032;    // 32 KB: v [2][64], w [2][64]
+constexpr uint32_t SM_ASCR = 204800;  // 16 KB: A fp32 [64][64], float4 columns XOR-swizzled by row
+constexpr uint32_t SM_GAM = 221184;   // gamma, 3 slots x 128 floats (chunk n uses slot n % 3)
+constexpr uint32_t SM_BAR = 222720;   // mbarriers, tensor memory base, abort flag
 constexpr uint32_t SM_END = SM_BAR + 256;
 constexpr size_t kSmemBytes = SM_END + 1024;
 
 enum Bar {
-    B_FULL = 0,     // +slot: raw q, k, alpha, b tiles landed
-    B_VWFULL = 2,   // +slot: v, w tiles landed
-    B_X1 = 4,
-    B_READY = 5,    // +slot: Ehat, Qhat, Ktil written (operands of X2)
-    B_TREADY = 7,   // +slot: T and P written
-    B_KBREADY = 9,
-    B_KBFREE = 10,
-    B_X2A = 11,
-    B_X2B = 12,
-    B_X3 = 13,
-    B_X45 = 14,
-    B_COUNT = 15
+    B_RAW = 0,      // q, k, alpha, b tiles of the prologue's chunk landed
+    B_VW,           // v, w tiles of the scan's chunk landed
+    B_X1,           // X1 complete
+    B_EQ_READY,     // [Ehat;Qhat] hi and Qhat lo written
+    B_EQ_FREE,      // X2 complete
+    B_T_READY,
+    B_T_FREE,       // X3 complete
+    B_P_READY,
+    B_P_FREE,       // X4 complete
+    B_KB_READY,
+    B_KB_FREE,      // X5 complete
+    B_X2A,
+    B_X2B,
+    B_X3,
+    B_X45,
+    B_COUNT
 };
 
 struct Params {
@@ -95,8 +110,18 @@ struct Params {
 __device__ __forceinline__ float bf(const uint8_t* tile, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
 }
-__device__ __forceinline__ void put_bf(uint8_t* tile, uint32_t off, float v) {
-    *reinterpret_cast<__nv_bfloat16*>(tile + off) = __float2bfloat16_rn(v);
+__device__ __forceinline__ void put_raw(uint8_t* tile, uint32_t off, __nv_bfloat16 v) {
+    *reinterpret_cast<__nv_bfloat16*>(tile + off) = v;
+}
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi).
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+    hi = __float2bfloat16_rn(x);
+    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16x2(x0, x1);
+    const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
+    lo = pack_bf16x2(x0 - h0, x1 - h1);
 }
 __device__ __forceinline__ uint32_t ascr_index(int r, int c) {  // fp32 element index
     return (uint32_t)r * 64u + ((uint32_t)((c >> 2) ^ (r & 15)) << 2) + (uint32_t)(c & 3);
@@ -135,33 +160,38 @@ __device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint6
 }
 
 template <bool APC, bool GPC>
-__device__ __forceinline__ void issue_tma(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
-                                          const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* ta,
-                                          const CUtensorMap* tb_, const CUtensorMap* tw) {
-    const int s = n & 1, t0 = n * C;
-    const uint32_t slot = smem_u32(cx.sm) + s * SLOT_BYTES;
-    uint64_t* full = cx.bars + B_FULL + s;
-    mbar_arrive_expect_tx(full, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
-    tma4(slot + OFF_EQ + 8192, tq, full, 0, hk, t0, b);           // q -> rows 64-127, channels 0-63
-    tma4(slot + OFF_EQ + 16384 + 8192, tq, full, 64, hk, t0, b);  // channels 64-127
-    tma4(slot + OFF_KT, tk, full, 0, hk, t0, b);
-    tma4(slot + OFF_KT + 8192, tk, full, 64, hk, t0, b);
+__device__ __forceinline__ void load_raw(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
+                                         const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_) {
+    const int t0 = n * C;
+    const uint32_t base = smem_u32(cx.sm);
+    uint64_t* bar = cx.bars + B_RAW;
+    mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
+    tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);           // q -> rows 64-127, channels 0-63
+    tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);  // channels 64-127
+    tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
+    tma4(base + SM_RK + 8192, tk, bar, 64, hk, t0, b);
     if (GPC) {
-        tma4(slot + OFF_EQ, tb_, full, 0, hv, t0, b);              // b -> rows 0-63
-        tma4(slot + OFF_EQ + 16384, tb_, full, 64, hv, t0, b);
+        tma4(base + SM_RQB, tb_, bar, 0, hv, t0, b);              // b -> rows 0-63
+        tma4(base + SM_RQB + 16384, tb_, bar, 64, hv, t0, b);
     }
     if (APC) {
-        tma4(slot + OFF_AL, ta, full, 0, hv, t0, b);
-        tma4(slot + OFF_AL + 8192, ta, full, 64, hv, t0, b);
+        tma4(base + SM_RA, ta, bar, 0, hv, t0, b);
+        tma4(base + SM_RA + 8192, ta, bar, 64, hv, t0, b);
     }
-    uint64_t* vwf = cx.bars + B_VWFULL + s;
-    const uint32_t vw = smem_u32(cx.sm) + SM_VW + s * VW_BYTES;
-    mbar_arrive_expect_tx(vwf, GPC ? 32768u : 16384u);
-    tma4(vw, tv, vwf, 0, hv, t0, b);
-    tma4(vw + 8192, tv, vwf, 64, hv, t0, b);
+}
+
+template <bool GPC>
+__device__ __forceinline__ void load_vw(const Ctx& cx, int n, int b, int hv, const CUtensorMap* tv,
+                                        const CUtensorMap* tw) {
+    const int t0 = n * C;
+    const uint32_t vw = smem_u32(cx.sm) + SM_VW;
+    uint64_t* bar = cx.bars + B_VW;
+    mbar_arrive_expect_tx(bar, GPC ? 32768u : 16384u);
+    tma4(vw, tv, bar, 0, hv, t0, b);
+    tma4(vw + 8192, tv, bar, 64, hv, t0, b);
     if (GPC) {
-        tma4(vw + 16384, tw, vwf, 0, hv, t0, b);
-        tma4(vw + 16384 + 8192, tw, vwf, 64, hv, t0, b);
+        tma4(vw + 16384, tw, bar, 0, hv, t0, b);
+        tma4(vw + 16384 + 8192, tw, bar, 64, hv, t0, b);
     }
 }
 
@@ -185,6 +215,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int b = blockIdx.x / pb.Hv, hv = blockIdx.x % pb.Hv;
     const int hk = pb.key_head(hv);
     const int NT = pb.NT;
+    const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) mbar_init(cx.bars + i, 1);
@@ -199,61 +230,61 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    int issued = 0;  // chunks whose TMA loads thread 0 has issued
     if (tid == 0) {
-        for (; issued < 2 && issued < NT; ++issued)
-            issue_tma<APC, GPC>(cx, issued, b, hk, hv, &tm_q, &tm_k, &tm_v, &tm_a, &tm_b, &tm_w);
+        load_raw<APC, GPC>(cx, 0, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+        load_vw<GPC>(cx, 0, b, hv, &tm_v, &tm_w);
     }
+    int raw_issued = 1, vw_issued = 1;  // meaningful in the issuing threads only
 
     if (warp < 8) {
         // =================================== state scan ===================================
         const int j = tid & 127, h = tid >> 7;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tl = tbase + lane_base;
+        const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
         const long soff = pb.state_off(b, hv);
+        const TG* beta = static_cast<const TG*>(p.b);
+        const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
         float S[64];  // S[c'] = state[64h + c'][j]
 #pragma unroll
         for (int c = 0; c < 64; ++c) S[c] = p.h0 ? p.h0[soff + (long)(64 * h + c) * D + j] : 0.f;
-        {
-            uint32_t pk[16];
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
+        for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(S[32 * q2 + 2 * i], S[32 * q2 + 2 * i + 1]);
-                tmem_st16(tl + TM_S0 + 32 * h + 16 * q2, pk);
-            }
-            tmem_st_wait();
+            for (int i = 0; i < 16; ++i) split_pack(S[32 * q2 + 2 * i], S[32 * q2 + 2 * i + 1], hi[i], lo[i]);
+            tmem_st16(tl + TM_S0H + 32 * h + 16 * q2, hi);
+            tmem_st16(tl + TM_S0L + 32 * h + 16 * q2, lo);
         }
+        tmem_st_wait();
         tc_fence_before();
         named_bar(1, 256);
 
-        const TG* beta = static_cast<const TG*>(p.b);
         for (int n = 0; n < NT; ++n) {
-            const int s = n & 1;
-            const uint32_t par = (n >> 1) & 1, pn = n & 1;
+            const uint32_t pn = n & 1;
             const int t0 = n * C, L = min(C, pb.T - t0);
-            const uint32_t slot = smem_u32(sm) + s * SLOT_BYTES;
-            // ---- X2 = S0^T [Ehat;Qhat]^T ------------------------------------------------------
+            // ---- X2 = S0^T [Ehat;Qhat]^T  (S0 split; Qhat split in the Qhat half) ------------------
             if (tid == 0) {
                 tc_fence_after();
-                if (wait_bar(cx, B_READY + s, par) && !*cx.abort_flag) {
-                    const uint32_t id64 = idesc_bf16_f32(128, 64);
-                    mma_ts_k(tbase + TM_X2, tbase + TM_S0, slot + OFF_EQ, 128, 128, id64, false);
+                if (wait_bar(cx, B_EQ_READY, pn) && !*cx.abort_flag) {
+                    mma_ts_k(tbase + TM_X2, tbase + TM_S0H, sbase + SM_EQ, 128, 128, id64, false);
+                    mma_ts_k(tbase + TM_X2, tbase + TM_S0L, sbase + SM_EQ, 128, 128, id64, true);
                     mma_commit(cx.bars + B_X2A);
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0, slot + OFF_EQ + 8192, 128, 128, id64, false);
+                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_EQ + 8192, 128, 128, id64, false);
+                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0L, sbase + SM_EQ + 8192, 128, 128, id64, true);
+                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_QLO, 64, 128, id64, true);
                     mma_commit(cx.bars + B_X2B);
+                    mma_commit(cx.bars + B_EQ_FREE);
                 }
             }
-            // ---- Y^T = Z^T - (Ehat S0)^T  (tensor memory, bf16) -----------------------------
+            // ---- Y^T = Z^T - (Ehat S0)^T  (tensor memory, split) -----------------------------------
             wait_bar(cx, B_X2A, pn);
-            wait_bar(cx, B_VWFULL + s, par);
+            wait_bar(cx, B_VW, pn);
             tc_fence_after();
             {
                 uint32_t r[32];
                 tmem_ld32(tl + TM_X2 + 32 * h, r);
                 tmem_ld_wait();
-                const uint8_t* vt = sm + SM_VW + s * VW_BYTES;
-                uint32_t pk[16];
+                const uint8_t* vt = sm + SM_VW;
+                uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float y2[2];
@@ -267,54 +298,63 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         else ww = rr < L ? to_f32(beta[pb.gate_row(b, t0 + rr, hv, 1)]) : 0.f;
                         y2[e] = vv * ww - __uint_as_float(r[2 * i + e]);
                     }
-                    pk[i] = pack_bf16x2(y2[0], y2[1]);
+                    split_pack(y2[0], y2[1], hi[i], lo[i]);
                 }
-                tmem_st16(tl + TM_Y + 16 * h, pk);
+                tmem_st16(tl + TM_YH + 16 * h, hi);
+                tmem_st16(tl + TM_YL + 16 * h, lo);
                 tmem_st_wait();
             }
             tc_fence_before();
             named_bar(1, 256);
-            // ---- X3 = Y^T T^T = V'^T -----------------------------------------------------------
+            // ---- X3 = Y^T T^T = V'^T; v/w of the next chunk --------------------------------------
             if (tid == 0) {
                 tc_fence_after();
-                if (wait_bar(cx, B_TREADY + s, par) && !*cx.abort_flag) {
-                    mma_ts_k(tbase + TM_X3, tbase + TM_Y, slot + OFF_AL, 64, 64, idesc_bf16_f32(128, 64), false);
+                if (vw_issued < NT && !*cx.abort_flag) {
+                    load_vw<GPC>(cx, vw_issued, b, hv, &tm_v, &tm_w);
+                    ++vw_issued;
+                }
+                if (wait_bar(cx, B_T_READY, pn) && !*cx.abort_flag) {
+                    mma_ts_k(tbase + TM_X5, tbase + TM_YH, sbase + SM_T, 64, 64, id64, false);
+                    mma_ts_k(tbase + TM_X5, tbase + TM_YL, sbase + SM_T, 64, 64, id64, true);
                     mma_commit(cx.bars + B_X3);
+                    mma_commit(cx.bars + B_T_FREE);
                 }
             }
             wait_bar(cx, B_X3, pn);
             tc_fence_after();
             {
-                uint32_t r[32], pk[16];
-                tmem_ld32(tl + TM_X3 + 32 * h, r);
+                uint32_t r[32], hi[16], lo[16];
+                tmem_ld32(tl + TM_X5 + 32 * h, r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                tmem_st16(tl + TM_Y + 16 * h, pk);
+                    split_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), hi[i], lo[i]);
+                tmem_st16(tl + TM_YH + 16 * h, hi);
+                tmem_st16(tl + TM_YL + 16 * h, lo);
                 tmem_st_wait();
             }
             tc_fence_before();
             named_bar(1, 256);
-            // ---- X4 (O += V'^T P^T), X5 (dS^T = V'^T Kbar) --------------------------------------
+            // ---- X4 (O += V'^T P^T), X5 (dS^T = V'^T Kbar) ---------------------------------------
             if (tid == 0) {
                 tc_fence_after();
-                if (wait_bar(cx, B_KBREADY, pn) && !*cx.abort_flag) {
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_Y, slot + OFF_AL + 8192, 64, 64, idesc_bf16_f32(128, 64),
-                             true);
-                    mma_ts_k(tbase + TM_X5, tbase + TM_Y, smem_u32(sm) + SM_KB, 128, 64, idesc_bf16_f32(128, 128),
-                             false);
+                const bool okp = wait_bar(cx, B_P_READY, pn);
+                const bool okk = wait_bar(cx, B_KB_READY, pn);
+                if (okp && okk && !*cx.abort_flag) {
+                    const uint32_t P = sbase + SM_P, KB = sbase + SM_KB;
+                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_YH, P, 64, 64, id64, true);
+                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_YL, P, 64, 64, id64, true);
+                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_YH, P + 8192, 64, 64, id64, true);
+                    mma_ts_k(tbase + TM_X5, tbase + TM_YH, KB, 128, 64, id128, false);
+                    mma_ts_k(tbase + TM_X5, tbase + TM_YL, KB, 128, 64, id128, true);
+                    mma_ts_k(tbase + TM_X5, tbase + TM_YH, KB + 16384, 128, 64, id128, true);
                     mma_commit(cx.bars + B_X45);
-                    mma_commit(cx.bars + B_KBFREE);
+                    mma_commit(cx.bars + B_P_FREE);
+                    mma_commit(cx.bars + B_KB_FREE);
                 }
             }
-            const bool done45 = wait_bar(cx, B_X45, pn);
+            wait_bar(cx, B_X45, pn);
             tc_fence_after();
-            if (tid == 0 && done45 && issued < NT && !*cx.abort_flag) {
-                // slot s and its v/w slot are free again: prefetch chunk n + 2
-                issue_tma<APC, GPC>(cx, issued, b, hk, hv, &tm_q, &tm_k, &tm_v, &tm_a, &tm_b, &tm_w);
-                ++issued;
-            }
             // ---- output rows 32h .. 32h+31 of column j -----------------------------------------
             {
                 uint32_t r[32];
@@ -335,20 +375,22 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
             }
-            // ---- state: S = Diag(gamma) S0 + Kbar^T V'; S0^T (bf16) for the next chunk --------------
+            // ---- state: S = Diag(gamma) S0 + Kbar^T V'; split S0^T for the next chunk -------------
             {
                 const float* g = gam + (n % 3) * 128 + 64 * h;
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2) {
-                    uint32_t r[32], pk[16];
+                    uint32_t r[32], hi[16], lo[16];
                     tmem_ld32(tl + TM_X5 + 64 * h + 32 * q2, r);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         S[32 * q2 + i] = fmaf(g[32 * q2 + i], S[32 * q2 + i], __uint_as_float(r[i]));
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(S[32 * q2 + 2 * i], S[32 * q2 + 2 * i + 1]);
-                    tmem_st16(tl + TM_S0 + 32 * h + 16 * q2, pk);
+                    for (int i = 0; i < 16; ++i)
+                        split_pack(S[32 * q2 + 2 * i], S[32 * q2 + 2 * i + 1], hi[i], lo[i]);
+                    tmem_st16(tl + TM_S0H + 32 * h + 16 * q2, hi);
+                    tmem_st16(tl + TM_S0L + 32 * h + 16 * q2, lo);
                 }
                 tmem_st_wait();
             }
@@ -364,101 +406,103 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
     } else {
         // =================================== chunk prologue ===================================
-        const int c = tid - 256;              // key channel; also TMEM lane of X1
+        const int c = tid - 256;  // key channel; also TMEM lane of X1
         const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
         const TG* alpha_g = static_cast<const TG*>(p.alpha);
         const TG* beta_g = static_cast<const TG*>(p.b);
         float* ascr = reinterpret_cast<float*>(sm + SM_ASCR);
+        uint8_t* RQB = sm + SM_RQB;
+        uint8_t* RK = sm + SM_RK;
+        uint8_t* RA = sm + SM_RA;
+        uint8_t* EQ = sm + SM_EQ;
+        uint8_t* QLO = sm + SM_QLO;
         float kr[64];
         for (int m = 0; m < NT; ++m) {
-            const int s = m & 1;
-            const uint32_t par = (m >> 1) & 1, pm = m & 1;
+            const uint32_t pm = m & 1, pprev = (m - 1) & 1;
             const int t0 = m * C, L = min(C, pb.T - t0);
-            uint8_t* slot = sm + s * SLOT_BYTES;
-            uint8_t* EQ = slot + OFF_EQ;
-            uint8_t* KT = slot + OFF_KT;
-            uint8_t* AL = slot + OFF_AL;
-            wait_bar(cx, B_FULL + s, par);
-            // ---- cumulative decay, gated and decayed factors, in place ------------------------
+            wait_bar(cx, B_RAW, pm);
+            if (m > 0) wait_bar(cx, B_EQ_FREE, pprev);
+            // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA / QLO) ----------
             float G = 1.f;
 #pragma unroll
             for (int r = 0; r < C; ++r) {
+                const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
+                const uint32_t ok = sw128_offset(r, c, 64);
                 float a = 1.f;
                 if (r < L) {
-                    if (APC) a = bf(AL, sw128_offset(r, c, 64));
+                    if (APC) a = bf(RA, ok);
                     else a = to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]);
                 }
                 G *= a;
-                const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
-                const uint32_t ok = sw128_offset(r, c, 64);
-                const float kv = bf(KT, ok), qv = bf(EQ, oq);
+                const float kv = bf(RK, ok), qv = bf(RQB, oq);
                 float bv;
-                if (GPC) bv = bf(EQ, oe);
+                if (GPC) bv = bf(RQB, oe);
                 else bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
-                const float inv = 1.f / G;
-                put_bf(EQ, oe, bv * kv * G);
-                put_bf(EQ, oq, qv * G);
-                kr[r] = kv * inv;
-                put_bf(KT, ok, kr[r]);
+                __nv_bfloat16 hi, lo;
+                split_bf16(bv * kv * G, hi, lo);
+                put_raw(EQ, oe, hi);
+                put_raw(RQB, oe, lo);
+                split_bf16(qv * G, hi, lo);
+                put_raw(EQ, oq, hi);
+                put_raw(RQB, oq, lo);
+                put_raw(QLO, ok, lo);
+                kr[r] = kv / G;
+                split_bf16(kr[r], hi, lo);
+                put_raw(RK, ok, hi);
+                put_raw(RA, ok, lo);
             }
             gam[(m % 3) * 128 + c] = G;
             fence_async_shared();
             named_bar(2, 128);
-            // ---- X1 = [Ehat;Qhat] Ktil^T --------------------------------------------------------
+            // ---- X1 = [Ehat;Qhat] Ktil^T with the split operands ----------------------------------
             if (c == 0) {
                 tc_fence_after();
                 if (!*cx.abort_flag) {
-                    mma_ss_k(tbase + TM_X1, smem_u32(EQ), 128, smem_u32(KT), 64, 128, idesc_bf16_f32(128, 64), false);
+                    const uint32_t id = idesc_bf16_f32(128, 64);
+                    mma_ss_k(tbase + TM_X1, sbase + SM_EQ, 128, sbase + SM_RK, 64, 128, id, false);
+                    mma_ss_k(tbase + TM_X1, sbase + SM_EQ, 128, sbase + SM_RA, 64, 128, id, true);
+                    mma_ss_k(tbase + TM_X1, sbase + SM_RQB, 128, sbase + SM_RK, 64, 128, id, true);
                     mma_commit(cx.bars + B_X1);
                 }
-                mbar_arrive(cx.bars + B_READY + s);
+                mbar_arrive(cx.bars + B_EQ_READY);
             }
             wait_bar(cx, B_X1, pm);
             tc_fence_after();
-            {
-                uint32_t r[64];
-                tmem_ld32(tl + TM_X1, *reinterpret_cast<uint32_t(*)[32]>(r));
-                tmem_ld32(tl + TM_X1 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-                tmem_ld_wait();
-                if (c >= 64) {
-                    // P row (c - 64), lower triangle with the diagonal, bf16, K-major
-                    const int rr = c - 64;
-                    uint8_t* Pt = AL + 8192;
+            if (c == 0 && raw_issued < NT && !*cx.abort_flag) {
+                // X1 was the last reader of the raw stage: load the next chunk's q, k, alpha, b
+                load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                ++raw_issued;
+            }
+            if (c < 64) {
+                // A row c (lanes 0-63 of X1), strictly lower, into the fp32 scratch; warp-uniform
+                // branch: warps 8-9 hold lanes 0-63.
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint32_t w4[4];
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + TM_X1 + 32 * half, r);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s0 = 8 * ch + 2 * e;
-                            const float x0 = s0 <= rr ? __uint_as_float(r[s0]) : 0.f;
-                            const float x1 = s0 + 1 <= rr ? __uint_as_float(r[s0 + 1]) : 0.f;
-                            w4[e] = pack_bf16x2(x0, x1);
-                        }
-                        *reinterpret_cast<uint4*>(Pt + sw128_offset(rr, 8 * ch, 64)) =
-                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                    }
-                } else {
-                    // A row c, strictly lower, fp32 scratch
-#pragma unroll
-                    for (int q4 = 0; q4 < 16; ++q4) {
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const int s0 = 32 * half + 4 * q4;
                         float4 v4;
-                        v4.x = 4 * q4 + 0 < c ? __uint_as_float(r[4 * q4 + 0]) : 0.f;
-                        v4.y = 4 * q4 + 1 < c ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
-                        v4.z = 4 * q4 + 2 < c ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
-                        v4.w = 4 * q4 + 3 < c ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
-                        *reinterpret_cast<float4*>(ascr + ascr_index(c, 4 * q4)) = v4;
+                        v4.x = s0 + 0 < c ? __uint_as_float(r[4 * q4 + 0]) : 0.f;
+                        v4.y = s0 + 1 < c ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
+                        v4.z = s0 + 2 < c ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
+                        v4.w = s0 + 3 < c ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
+                        *reinterpret_cast<float4*>(ascr + ascr_index(c, s0)) = v4;
                     }
                 }
             }
             tc_fence_before();
             named_bar(2, 128);
-            // ---- T = (I + A)^-1, column jj by the lane pair (jj, parity pp) ----------------------
+            // ---- T = (I + A)^-1, column jj by the lane pair (jj, parity pp) -----------------------
+            if (m > 0) wait_bar(cx, B_T_FREE, pprev);
             {
                 const int jj = c >> 1, pp = c & 1;
                 float x[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = 0.f;
-                uint8_t* Tt = AL;
+                uint8_t* Tt = sm + SM_T;
 #pragma unroll
                 for (int i = 0; i < C; ++i) {
                     float acc = 0.f;
@@ -472,44 +516,79 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const float xi = i == jj ? 1.f : (i > jj ? -acc : 0.f);
                     if ((i & 1) == pp) {
                         x[i >> 1] = xi;
-                        put_bf(Tt, sw128_offset(i, jj, 64), xi);
+                        put_raw(Tt, sw128_offset(i, jj, 64), __float2bfloat16_rn(xi));
                     }
                 }
             }
             fence_async_shared();
             named_bar(2, 128);
-            if (c == 0) mbar_arrive(cx.bars + B_TREADY + s);
-            // ---- Kbar^T row c: k * gamma / Gamma_r --------------------------------------------
-            if (m > 0) wait_bar(cx, B_KBFREE, (m - 1) & 1);
+            if (c == 0) mbar_arrive(cx.bars + B_T_READY);
+            // ---- P (lower triangle with the diagonal), split, from lanes 64-127 -------------------
+            if (m > 0) wait_bar(cx, B_P_FREE, pprev);
+            tc_fence_after();
+            if (c >= 64) {
+                // P row c - 64 (lanes 64-127 of X1, still intact: the next X1 is issued by the next
+                // chunk's prologue); warps 10-11.
+                const int rr = c - 64;
+                uint8_t* Ph = sm + SM_P;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + TM_X1 + 32 * half, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t wh[4], wl[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = 8 * ch + 2 * e, s0 = 32 * half + i0;
+                            const float x0 = s0 <= rr ? __uint_as_float(r[i0]) : 0.f;
+                            const float x1 = s0 + 1 <= rr ? __uint_as_float(r[i0 + 1]) : 0.f;
+                            split_pack(x0, x1, wh[e], wl[e]);
+                        }
+                        const uint32_t off = sw128_offset(rr, 32 * half + 8 * ch, 64);
+                        *reinterpret_cast<uint4*>(Ph + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                        *reinterpret_cast<uint4*>(Ph + 8192 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_async_shared();
+            named_bar(2, 128);
+            if (c == 0) mbar_arrive(cx.bars + B_P_READY);
+            // ---- Kbar^T row c = k * gamma / Gamma_r, split -----------------------------------------
+            if (m > 0) wait_bar(cx, B_KB_FREE, pprev);
             {
                 uint8_t* KB = sm + SM_KB;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t w4[4];
+                    uint32_t wh[4], wl[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) w4[e] = pack_bf16x2(kr[8 * ch + 2 * e] * G, kr[8 * ch + 2 * e + 1] * G);
-                    *reinterpret_cast<uint4*>(KB + sw128_offset(c, 8 * ch, 128)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    for (int e = 0; e < 4; ++e)
+                        split_pack(kr[8 * ch + 2 * e] * G, kr[8 * ch + 2 * e + 1] * G, wh[e], wl[e]);
+                    const uint32_t off = sw128_offset(c, 8 * ch, 128);
+                    *reinterpret_cast<uint4*>(KB + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                    *reinterpret_cast<uint4*>(KB + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
                 }
             }
             fence_async_shared();
             named_bar(2, 128);
-            if (c == 0) mbar_arrive(cx.bars + B_KBREADY);
+            if (c == 0) mbar_arrive(cx.bars + B_KB_READY);
             const int stop = *cx.abort_flag;
             named_bar(2, 128);
             if (stop) break;
         }
     }
 
-    // ---- teardown: loads still in flight after an abort are waited for (bounded) ----------------
+    // ---- teardown: TMA loads still in flight after an abort are waited for (bounded) -----------
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *cx.abort_flag) {
+    if (*cx.abort_flag && (tid == 0 || tid == 256)) {
         const uint64_t t0 = globaltimer_ns();
-        for (int n = issued - 2 < 0 ? 0 : issued - 2; n < issued; ++n) {
-            while (!mbar_try_wait(cx.bars + B_FULL + (n & 1), (n >> 1) & 1) && globaltimer_ns() - t0 < kWaitNs) {
-            }
-            while (!mbar_try_wait(cx.bars + B_VWFULL + (n & 1), (n >> 1) & 1) && globaltimer_ns() - t0 < kWaitNs) {
-            }
+        const int bar = tid == 0 ? B_VW : B_RAW;
+        const int issued = tid == 0 ? vw_issued : raw_issued;
+        // the last issued load completes phase (issued - 1)
+        while (!mbar_try_wait(cx.bars + bar, (uint32_t)((issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
         }
     }
     __syncthreads();

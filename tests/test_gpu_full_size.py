@@ -1,0 +1,127 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the benchmark times.
+
+The GPU computes every (sequence, head) of the workload; the fp64 oracle recomputes a seeded
+sample of (sequence, head) pairs one by one (each pair is independent), and the outputs, final
+states and gradients of those pairs are compared at the stated tolerances:
+  * GDN-2 forward + backward, B=8 T=4096 H=16 d=128 (bf16 inputs, fp32 state);
+  * Gated DeltaNet forward with scalar gates, B=8 T=4096 H=16 d=128;
+  * GQA layer core, B=2 T=16384, 16 key / 128 value heads (conv + SiLU + L2 + swish gate);
+  * GDN-2 decode, 256 sequences x 1024 steps, H=16 d=128 (every step's output of the sampled
+    sequences, and their final states).
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_76_b200 import gdn
+from gated_delta_rule_76_b200.inputs import (WORKLOADS, decode_initial_state, decode_inputs,
+                                             workload_inputs)
+from oracle import oracle
+from parity import assert_bf16_is_rounding, assert_parity, npf
+
+pytestmark = pytest.mark.gpu
+
+
+def sample_pairs(B, H, n, seed):
+    rng = np.random.default_rng(seed)
+    flat = rng.choice(B * H, size=n, replace=False)
+    return sorted((int(f) // H, int(f) % H) for f in flat)
+
+
+def gate_kw(x, sl=slice(None)):
+    if "beta" in x:
+        return dict(beta=x["beta"][sl])
+    return dict(b=x["b"][sl], w=x["w"][sl])
+
+
+def test_gdn2_forward_backward_full_size():
+    name = "gdn2_fwd_bwd_bf16"
+    wl = WORKLOADS[name]
+    x = workload_inputs(name, with_dout=True)
+    g = {k: v.cuda() for k, v in x.items()}
+    o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], out_f32=True, **gate_kw(g))
+    o16, _ = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], **gate_kw(g))
+    grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], **gate_kw(g))
+    torch.cuda.synchronize()
+    assert_bf16_is_rounding(o16, o, "o")
+    for b, h in sample_pairs(wl.B, wl.Hv, 4, seed=3):
+        sl = slice(b, b + 1)
+        xs = {k: v[sl] for k, v in x.items()}
+        o_ref, ht_ref = oracle.fwd(xs["q"], xs["k"], xs["v"], xs["alpha"], h0=xs["h0"], pairs=[h],
+                                   **gate_kw(xs))
+        assert_parity(o[b, :, h], o_ref[0, :, h], "bf16", f"o ({b},{h})")
+        assert_parity(ht[b, h], ht_ref[0, h], "bf16", f"ht ({b},{h})")
+        ref = oracle.bwd(xs["q"], xs["k"], xs["v"], xs["alpha"], h0=xs["h0"], dout=xs["dout"], pairs=[h],
+                         **gate_kw(xs))
+        # identity head map: per-value-head q/k gradients are the q/k gradients of that head
+        assert_parity(grads["dq"][b, :, h], ref["dq_v"][0, :, h], "bf16", f"dq ({b},{h})")
+        assert_parity(grads["dk"][b, :, h], ref["dk_v"][0, :, h], "bf16", f"dk ({b},{h})")
+        for key in ("dv", "dalpha", "db", "dw"):
+            assert_parity(grads[key][b, :, h], ref[key][0, :, h], "bf16", f"{key} ({b},{h})")
+        assert_parity(grads["dh0"][b, h], ref["dh0"][0, h], "bf16", f"dh0 ({b},{h})")
+
+
+def test_gated_deltanet_scalar_forward_full_size():
+    name = "gdn_fwd_scalar_bf16"
+    wl = WORKLOADS[name]
+    x = workload_inputs(name)
+    g = {k: v.cuda() for k, v in x.items()}
+    o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], beta=g["beta"], out_f32=True)
+    torch.cuda.synchronize()
+    for b, h in sample_pairs(wl.B, wl.Hv, 4, seed=4):
+        sl = slice(b, b + 1)
+        o_ref, ht_ref = oracle.fwd(x["q"][sl], x["k"][sl], x["v"][sl], x["alpha"][sl],
+                                   beta=x["beta"][sl], pairs=[h])
+        assert_parity(o[b, :, h], o_ref[0, :, h], "bf16", f"o ({b},{h})")
+        assert_parity(ht[b, h], ht_ref[0, h], "bf16", f"ht ({b},{h})")
+
+
+def test_gqa_layer_core_full_size():
+    name = "gqa_layer_core_bf16"
+    wl = WORKLOADS[name]
+    x = workload_inputs(name)
+    g = {k: v.cuda() for k, v in x.items()}
+    y, ht, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"],
+                                      beta=g["beta"], out_f32=True)
+    torch.cuda.synchronize()
+    d, Hk, Hv = wl.dk, wl.Hk, wl.Hv
+    w = npf(x["conv_w"])
+    group = Hv // Hk
+    for b, hv in sample_pairs(wl.B, wl.Hv, 3, seed=5):
+        hk = hv // group
+        sl = slice(b, b + 1)
+        cq = slice(hk * d, (hk + 1) * d)
+        ck = slice(Hk * d + hk * d, Hk * d + (hk + 1) * d)
+        cv = slice(2 * Hk * d + hv * d, 2 * Hk * d + (hv + 1) * d)
+        q, _ = oracle.conv_silu(npf(x["q"][sl, :, hk]), w[cq])
+        k, _ = oracle.conv_silu(npf(x["k"][sl, :, hk]), w[ck])
+        v, _ = oracle.conv_silu(npf(x["v"][sl, :, hv]), w[cv])
+        q = oracle.l2norm(q)[:, :, None]
+        k = oracle.l2norm(k)[:, :, None]
+        o_ref, ht_ref = oracle.fwd(q, k, v[:, :, None], npf(x["alpha"][sl, :, hv:hv + 1]),
+                                   beta=npf(x["beta"][sl, :, hv:hv + 1]), head_map=[0])
+        y_ref = oracle.swish_gate(o_ref[0, :, 0], npf(x["z"][b, :, hv]))
+        assert_parity(y[b, :, hv], y_ref, "bf16", f"y ({b},{hv})")
+        assert_parity(ht[b, hv], ht_ref[0, 0], "bf16", f"ht ({b},{hv})")
+
+
+def test_gdn2_decode_1024_steps_full_size():
+    name = "gdn2_decode_bf16"
+    wl = WORKLOADS[name]
+    steps = wl.decode_steps
+    xs = decode_inputs(name, steps)
+    s0 = decode_initial_state(name)
+    g = {k: v.cuda() for k, v in xs.items()}
+    state = s0.cuda()
+    o = torch.empty((steps, wl.B, wl.Hv, wl.dv), dtype=torch.float32, device="cuda")
+    for s in range(steps):
+        gdn.gdn_decode_step(state, g["q"][s], g["k"][s], g["v"][s], g["alpha"][s], b=g["b"][s], w=g["w"][s],
+                            o=o[s])
+    torch.cuda.synchronize()
+    for n, h in sample_pairs(wl.B, wl.Hv, 6, seed=6):
+        # The sampled sequence's 1024 steps as one sequence (T decode steps == one forward).
+        seq = {k: v[:, n:n + 1].transpose(0, 1).contiguous() for k, v in xs.items()}
+        o_ref, st_ref = oracle.fwd(seq["q"], seq["k"], seq["v"], seq["alpha"], b=seq["b"], w=seq["w"],
+                                   h0=s0[n:n + 1], pairs=[h])
+        assert_parity(o[:, n, h], o_ref[0, :, h], "bf16", f"o ({n},{h})")
+        assert_parity(state[n, h], st_ref[0, h], "bf16", f"state ({n},{h})")
