@@ -200,8 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w, Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // Offset arithmetic on the shared array keeps the pointer in the shared state space, so the
+    // compiler emits shared loads/stores and knows they cannot alias global memory.
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
     cx.sm = sm;
     cx.bars = reinterpret_cast<uint64_t*>(sm + SM_BAR);
@@ -425,31 +427,40 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA / QLO) ----------
             float G = 1.f;
 #pragma unroll
-            for (int r = 0; r < C; ++r) {
-                const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
-                const uint32_t ok = sw128_offset(r, c, 64);
-                float a = 1.f;
-                if (r < L) {
-                    if (APC) a = bf(RA, ok);
-                    else a = to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]);
+            for (int r0 = 0; r0 < C; r0 += 8) {
+                // loads of 8 rows first (independent of this block's stores), then compute/store
+                float av[8], kv[8], qv[8], bv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = r0 + u;
+                    const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
+                    const uint32_t ok = sw128_offset(r, c, 64);
+                    if (APC) av[u] = r < L ? bf(RA, ok) : 1.f;
+                    else av[u] = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+                    kv[u] = bf(RK, ok);
+                    qv[u] = bf(RQB, oq);
+                    if (GPC) bv[u] = bf(RQB, oe);
+                    else bv[u] = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
                 }
-                G *= a;
-                const float kv = bf(RK, ok), qv = bf(RQB, oq);
-                float bv;
-                if (GPC) bv = bf(RQB, oe);
-                else bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
-                __nv_bfloat16 hi, lo;
-                split_bf16(bv * kv * G, hi, lo);
-                put_raw(EQ, oe, hi);
-                put_raw(RQB, oe, lo);
-                split_bf16(qv * G, hi, lo);
-                put_raw(EQ, oq, hi);
-                put_raw(RQB, oq, lo);
-                put_raw(QLO, ok, lo);
-                kr[r] = kv / G;
-                split_bf16(kr[r], hi, lo);
-                put_raw(RK, ok, hi);
-                put_raw(RA, ok, lo);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = r0 + u;
+                    const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
+                    const uint32_t ok = sw128_offset(r, c, 64);
+                    G *= av[u];
+                    __nv_bfloat16 hi, lo;
+                    split_bf16(bv[u] * kv[u] * G, hi, lo);
+                    put_raw(EQ, oe, hi);
+                    put_raw(RQB, oe, lo);
+                    split_bf16(qv[u] * G, hi, lo);
+                    put_raw(EQ, oq, hi);
+                    put_raw(RQB, oq, lo);
+                    put_raw(QLO, ok, lo);
+                    kr[r] = kv[u] / G;
+                    split_bf16(kr[r], hi, lo);
+                    put_raw(RK, ok, hi);
+                    put_raw(RA, ok, lo);
+                }
             }
             gam[(m % 3) * 128 + c] = G;
             fence_async_shared();
@@ -502,23 +513,24 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float x[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = 0.f;
-                uint8_t* Tt = sm + SM_T;
 #pragma unroll
                 for (int i = 0; i < C; ++i) {
-                    float acc = 0.f;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int mm = 0; mm < (i + 1) / 2; ++mm) {
                         const int s0 = 2 * mm + pp;  // rows of this lane's parity below i
                         const float aval = ascr[ascr_index(i, s0 < C ? s0 : 0)];
-                        acc = fmaf(s0 < i ? aval : 0.f, x[mm], acc);
+                        acc[mm & 3] = fmaf(s0 < i ? aval : 0.f, x[mm], acc[mm & 3]);
                     }
-                    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                    const float xi = i == jj ? 1.f : (i > jj ? -acc : 0.f);
-                    if ((i & 1) == pp) {
-                        x[i >> 1] = xi;
-                        put_raw(Tt, sw128_offset(i, jj, 64), __float2bfloat16_rn(xi));
-                    }
+                    float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                    const float xi = i == jj ? 1.f : (i > jj ? -sum : 0.f);
+                    if ((i & 1) == pp) x[i >> 1] = xi;
                 }
+                uint8_t* Tt = sm + SM_T;
+#pragma unroll
+                for (int mm = 0; mm < 32; ++mm)
+                    put_raw(Tt, sw128_offset(2 * mm + pp, jj, 64), __float2bfloat16_rn(x[mm]));
             }
             fence_async_shared();
             named_bar(2, 128);
