@@ -73,7 +73,8 @@ constexpr uint32_t SM_VW = 172032;    // 32 KB: v [2][64], w [2][64]
 constexpr uint32_t SM_ASCR = 204800;  // 16 KB: A fp32 [64][64], float4 columns XOR-swizzled by row
 constexpr uint32_t SM_GAM = 221184;   // gamma, 3 slots x 128 floats (chunk n uses slot n % 3)
 constexpr uint32_t SM_BAR = 222720;   // mbarriers, tensor memory base, abort flag
-constexpr uint32_t SM_END = SM_BAR + 256;
+constexpr uint32_t SM_RS = SM_BAR + 256;  // 3 KB fp32 [16][48]: block-row products of the solve
+constexpr uint32_t SM_END = SM_RS + 3072;
 constexpr size_t kSmemBytes = SM_END + 1024;
 
 enum Bar {
@@ -135,7 +136,7 @@ struct Ctx {
 };
 
 // Bounded wait that also gives up as soon as another thread has aborted.
-__device__ __forceinline__ bool wait_bar(const Ctx& cx, int bar, uint32_t parity) {
+__device__ __noinline__ bool wait_bar(const Ctx& cx, int bar, uint32_t parity) {
     uint64_t* b = cx.bars + bar;
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -413,12 +414,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const TG* alpha_g = static_cast<const TG*>(p.alpha);
         const TG* beta_g = static_cast<const TG*>(p.b);
         float* ascr = reinterpret_cast<float*>(sm + SM_ASCR);
+        float* rs = reinterpret_cast<float*>(sm + SM_RS);
         uint8_t* RQB = sm + SM_RQB;
         uint8_t* RK = sm + SM_RK;
         uint8_t* RA = sm + SM_RA;
         uint8_t* EQ = sm + SM_EQ;
         uint8_t* QLO = sm + SM_QLO;
-        float kr[64];
         for (int m = 0; m < NT; ++m) {
             const uint32_t pm = m & 1, pprev = (m - 1) & 1;
             const int t0 = m * C, L = min(C, pb.T - t0);
@@ -426,7 +427,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (m > 0) wait_bar(cx, B_EQ_FREE, pprev);
             // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA / QLO) ----------
             float G = 1.f;
-#pragma unroll
+#pragma unroll 1
             for (int r0 = 0; r0 < C; r0 += 8) {
                 // loads of 8 rows first (independent of this block's stores), then compute/store
                 float av[8], kv[8], qv[8], bv[8];
@@ -456,8 +457,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     put_raw(EQ, oq, hi);
                     put_raw(RQB, oq, lo);
                     put_raw(QLO, ok, lo);
-                    kr[r] = kv[u] / G;
-                    split_bf16(kr[r], hi, lo);
+                    split_bf16(kv[u] / G, hi, lo);
                     put_raw(RK, ok, hi);
                     put_raw(RA, ok, lo);
                 }
@@ -479,14 +479,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             wait_bar(cx, B_X1, pm);
             tc_fence_after();
-            if (c == 0 && raw_issued < NT && !*cx.abort_flag) {
-                // X1 was the last reader of the raw stage: load the next chunk's q, k, alpha, b
-                load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
-                ++raw_issued;
-            }
             if (c < 64) {
-                // A row c (lanes 0-63 of X1), strictly lower, into the fp32 scratch; warp-uniform
-                // branch: warps 8-9 hold lanes 0-63.
+                // A row c (lanes 0-63 of X1), strictly lower, into the fp32 scratch; warps 8-9.
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t r[32];
@@ -506,31 +500,76 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             tc_fence_before();
             named_bar(2, 128);
-            // ---- T = (I + A)^-1, column jj by the lane pair (jj, parity pp) -----------------------
+            // ---- T = (I + A)^-1 by 16 x 16 blocks, in place in the fp32 scratch ------------------
+            // (1) diagonal blocks D_i = (I + A_ii)^-1: thread c < 64 solves column c & 15 of block c >> 4.
+            if (c < 64) {
+                const int base = 16 * (c >> 4), jc = c & 15;
+                float x[16];
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int u = 0; u < s2; ++u) acc = fmaf(ascr[ascr_index(base + s2, base + u)], x[u], acc);
+                    x[s2] = s2 == jc ? 1.f : (s2 > jc ? -acc : 0.f);
+                }
+                named_bar(3, 64);
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) ascr[ascr_index(base + s2, base + jc)] = x[s2];
+            }
+            named_bar(2, 128);
+            // (2) block rows ib = 1..3:  T_{ib, 0:ib} = -D_ib (A_{ib, 0:ib} T_{0:ib, 0:ib}).
+            //     Thread c: row rho = c >> 3 of the block row, columns (c & 7) + 8 mm, mm < 2 ib.
+            {
+                const int rho = c >> 3, g0 = c & 7;
+#pragma unroll 1
+                for (int ib = 1; ib < 4; ++ib) {
+                    const int row = 16 * ib + rho, ncol = 16 * ib;
+                    float acc[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+                    for (int kk = 0; kk < ncol; ++kk) {
+                        const float a = ascr[ascr_index(row, kk)];
+#pragma unroll
+                        for (int mm = 0; mm < 6; ++mm) {
+                            const int gcol = g0 + 8 * mm;
+                            // T_{0:ib,0:ib} is block lower triangular: rows below the column's block
+                            if (mm < 2 * ib && kk >= (gcol & ~15))
+                                acc[mm] = fmaf(a, ascr[ascr_index(kk, gcol)], acc[mm]);
+                        }
+                    }
+#pragma unroll
+                    for (int mm = 0; mm < 6; ++mm)
+                        if (mm < 2 * ib) rs[rho * 48 + g0 + 8 * mm] = acc[mm];
+                    named_bar(2, 128);
+                    float t6[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int sg = 0; sg < 16; ++sg) {
+                        const float d = ascr[ascr_index(row, ncol + sg)];  // D_ib[rho][sg]
+#pragma unroll
+                        for (int mm = 0; mm < 6; ++mm)
+                            if (mm < 2 * ib) t6[mm] = fmaf(d, rs[sg * 48 + g0 + 8 * mm], t6[mm]);
+                    }
+#pragma unroll
+                    for (int mm = 0; mm < 6; ++mm)
+                        if (mm < 2 * ib) ascr[ascr_index(row, g0 + 8 * mm)] = -t6[mm];
+                    named_bar(2, 128);
+                }
+            }
+            // (3) T (fp32) -> bf16 K-major tile: thread c converts 32 entries of row c >> 1.
             if (m > 0) wait_bar(cx, B_T_FREE, pprev);
             {
-                const int jj = c >> 1, pp = c & 1;
-                float x[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = 0.f;
-#pragma unroll
-                for (int i = 0; i < C; ++i) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int mm = 0; mm < (i + 1) / 2; ++mm) {
-                        const int s0 = 2 * mm + pp;  // rows of this lane's parity below i
-                        const float aval = ascr[ascr_index(i, s0 < C ? s0 : 0)];
-                        acc[mm & 3] = fmaf(s0 < i ? aval : 0.f, x[mm], acc[mm & 3]);
-                    }
-                    float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                    const float xi = i == jj ? 1.f : (i > jj ? -sum : 0.f);
-                    if ((i & 1) == pp) x[i >> 1] = xi;
-                }
+                const int row = c >> 1, col0 = 32 * (c & 1);
                 uint8_t* Tt = sm + SM_T;
 #pragma unroll
-                for (int mm = 0; mm < 32; ++mm)
-                    put_raw(Tt, sw128_offset(2 * mm + pp, jj, 64), __float2bfloat16_rn(x[mm]));
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int cc = col0 + 8 * ch + 2 * e;
+                        w4[e] = pack_bf16x2(ascr[ascr_index(row, cc)], ascr[ascr_index(row, cc + 1)]);
+                    }
+                    *reinterpret_cast<uint4*>(Tt + sw128_offset(row, col0 + 8 * ch, 64)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
             }
             fence_async_shared();
             named_bar(2, 128);
@@ -539,8 +578,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (m > 0) wait_bar(cx, B_P_FREE, pprev);
             tc_fence_after();
             if (c >= 64) {
-                // P row c - 64 (lanes 64-127 of X1, still intact: the next X1 is issued by the next
-                // chunk's prologue); warps 10-11.
+                // P row c - 64 (lanes 64-127 of X1, intact until the next chunk's X1); warps 10-11.
                 const int rr = c - 64;
                 uint8_t* Ph = sm + SM_P;
 #pragma unroll
@@ -568,16 +606,20 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_async_shared();
             named_bar(2, 128);
             if (c == 0) mbar_arrive(cx.bars + B_P_READY);
-            // ---- Kbar^T row c = k * gamma / Gamma_r, split -----------------------------------------
+            // ---- Kbar^T row c = (Ktil hi + lo) * gamma, split; then reload the raw stage -----------
             if (m > 0) wait_bar(cx, B_KB_FREE, pprev);
             {
                 uint8_t* KB = sm + SM_KB;
-#pragma unroll
+#pragma unroll 1
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t wh[4], wl[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        split_pack(kr[8 * ch + 2 * e] * G, kr[8 * ch + 2 * e + 1] * G, wh[e], wl[e]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = 8 * ch + 2 * e;
+                        const uint32_t o0 = sw128_offset(r, c, 64), o1 = sw128_offset(r + 1, c, 64);
+                        const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
+                        split_pack(k0, k1, wh[e], wl[e]);
+                    }
                     const uint32_t off = sw128_offset(c, 8 * ch, 128);
                     *reinterpret_cast<uint4*>(KB + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
                     *reinterpret_cast<uint4*>(KB + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
@@ -585,7 +627,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             fence_async_shared();
             named_bar(2, 128);
-            if (c == 0) mbar_arrive(cx.bars + B_KB_READY);
+            if (c == 0) {
+                mbar_arrive(cx.bars + B_KB_READY);
+                // X1 and the Kbar^T pass were the last readers of the raw stage.
+                if (raw_issued < NT && !*cx.abort_flag) {
+                    load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                    ++raw_issued;
+                }
+            }
             const int stop = *cx.abort_flag;
             named_bar(2, 128);
             if (stop) break;

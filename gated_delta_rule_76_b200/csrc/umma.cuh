@@ -180,6 +180,7 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // column), B: N rows (b_rows per atom column); K in multiples of 16.
 __device__ __forceinline__ void mma_ss_k(uint32_t d_tmem, uint32_t a_smem, int a_rows, uint32_t b_smem,
                                          int b_rows, int K, uint32_t idesc, bool accumulate) {
+#pragma unroll 1
     for (int k = 0; k < K; k += 16) {
         const uint32_t a = a_smem + (uint32_t)(k >> 6) * (uint32_t)a_rows * 128u + (uint32_t)(k & 63) * 2u;
         const uint32_t b = b_smem + (uint32_t)(k >> 6) * (uint32_t)b_rows * 128u + (uint32_t)(k & 63) * 2u;
@@ -189,6 +190,7 @@ __device__ __forceinline__ void mma_ss_k(uint32_t d_tmem, uint32_t a_smem, int a
 // Same with A in tensor memory (bf16 pairs packed per 32-bit column: 8 columns per K = 16).
 __device__ __forceinline__ void mma_ts_k(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, int b_rows, int K,
                                          uint32_t idesc, bool accumulate) {
+#pragma unroll 1
     for (int k = 0; k < K; k += 16) {
         const uint32_t b = b_smem + (uint32_t)(k >> 6) * (uint32_t)b_rows * 128u + (uint32_t)(k & 63) * 2u;
         mma_ts(d_tmem, a_tmem + (uint32_t)(k >> 1), sdesc_k_sw128(b), idesc, (accumulate || k > 0) ? 1u : 0u);
