@@ -45,6 +45,20 @@ namespace tcfwd {
 
 using namespace gdn::tc;
 
+// Optional phase timestamps of CTA 0 (compiled only with -DGDN_FWD_TRACE, for profiling builds):
+// g_fwd_trace[chunk][point] = %globaltimer.
+#ifdef GDN_FWD_TRACE
+__device__ unsigned long long g_fwd_trace[64][32];
+#define GDN_TRACE(chunk, point)                                                   \
+    do {                                                                          \
+        if (blockIdx.x == 0 && (chunk) < 64) g_fwd_trace[(chunk)][(point)] = globaltimer_ns(); \
+    } while (0)
+#else
+#define GDN_TRACE(chunk, point) \
+    do {                        \
+    } while (0)
+#endif
+
 constexpr int C = 64;
 constexpr int D = 128;
 constexpr int kThreads = 384;
@@ -135,13 +149,13 @@ struct Ctx {
     int* err;
 };
 
-// Bounded wait that also gives up as soon as another thread has aborted.
-__device__ __noinline__ bool wait_bar(const Ctx& cx, int bar, uint32_t parity) {
+// Bounded wait by a single thread (the others sleep in a named barrier meanwhile).  Polls sleep in
+// hardware between attempts; gives up when another thread has aborted or after kWaitNs.
+__device__ __forceinline__ bool wait1(const Ctx& cx, int bar, uint32_t parity) {
     uint64_t* b = cx.bars + bar;
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (mbar_try_wait(b, parity)) return true;
+    while (!mbar_try_wait_sleep(b, parity, 1000u)) {
         if (*cx.abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitNs) {
             *cx.abort_flag = 1;
@@ -149,6 +163,7 @@ __device__ __noinline__ bool wait_bar(const Ctx& cx, int bar, uint32_t parity) {
             return false;
         }
     }
+    return true;
 }
 
 __device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
@@ -242,10 +257,17 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (warp < 8) {
         // =================================== state scan ===================================
         const int j = tid & 127, h = tid >> 7;
+        volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 136);
         const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
         const long soff = pb.state_off(b, hv);
         const TG* beta = static_cast<const TG*>(p.b);
         const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
+        // swizzled byte offsets of column j in a 64-row tile: row r -> base + r*128 + xo[r & 7]
+        const uint32_t vbase = (uint32_t)(j >> 6) * 64u * 128u;
+        uint32_t xo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) xo[u] = ((uint32_t)(j & 63) * 2u) ^ ((uint32_t)u << 4);
+        const long orow = (long)pb.Hv * D;  // element stride between tokens of o / z
         float S[64];  // S[c'] = state[64h + c'][j]
 #pragma unroll
         for (int c = 0; c < 64; ++c) S[c] = p.h0 ? p.h0[soff + (long)(64 * h + c) * D + j] : 0.f;
@@ -266,40 +288,42 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int t0 = n * C, L = min(C, pb.T - t0);
             // ---- X2 = S0^T [Ehat;Qhat]^T  (S0 split; Qhat split in the Qhat half) ------------------
             if (tid == 0) {
+                GDN_TRACE(n, 0);
                 tc_fence_after();
-                if (wait_bar(cx, B_EQ_READY, pn) && !*cx.abort_flag) {
-                    mma_ts_k(tbase + TM_X2, tbase + TM_S0H, sbase + SM_EQ, 128, 128, id64, false);
-                    mma_ts_k(tbase + TM_X2, tbase + TM_S0L, sbase + SM_EQ, 128, 128, id64, true);
+                if (wait1(cx, B_EQ_READY, pn) && !*cx.abort_flag) {
+                    GDN_TRACE(n, 1);
+                    mma_ts_u<128, 128>(tbase + TM_X2, tbase + TM_S0H, sbase + SM_EQ, id128, false);
+                    mma_ts_u<128, 128>(tbase + TM_X2, tbase + TM_S0L, sbase + SM_EQ, id128, true);
                     mma_commit(cx.bars + B_X2A);
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_EQ + 8192, 128, 128, id64, false);
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0L, sbase + SM_EQ + 8192, 128, 128, id64, true);
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_QLO, 64, 128, id64, true);
-                    mma_commit(cx.bars + B_X2B);
+                    mma_ts_u<128, 64>(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_QLO, id64, true);
                     mma_commit(cx.bars + B_EQ_FREE);
+                    wait1(cx, B_X2A, pn);
+                    GDN_TRACE(n, 2);
                 }
+                wait1(cx, B_VW, pn);
+                GDN_TRACE(n, 3);
             }
-            // ---- Y^T = Z^T - (Ehat S0)^T  (tensor memory, split) -----------------------------------
-            wait_bar(cx, B_X2A, pn);
-            wait_bar(cx, B_VW, pn);
+            named_bar(1, 256);
             tc_fence_after();
+            // ---- Y^T = Z^T - (Ehat S0)^T  (tensor memory, split) -----------------------------------
             {
                 uint32_t r[32];
                 tmem_ld32(tl + TM_X2 + 32 * h, r);
                 tmem_ld_wait();
-                const uint8_t* vt = sm + SM_VW;
+                const uint8_t* vt = sm + SM_VW + vbase + 32u * h * 128u;
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float y2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int rr = 32 * h + 2 * i + e;
-                        const uint32_t off = sw128_offset(rr, j, 64);
+                        const int ii = 2 * i + e, rr = 32 * h + ii;
+                        const uint32_t off = (uint32_t)ii * 128u + xo[ii & 7];
                         const float vv = bf(vt, off);
                         float ww;
                         if (GPC) ww = bf(vt + 16384, off);
                         else ww = rr < L ? to_f32(beta[pb.gate_row(b, t0 + rr, hv, 1)]) : 0.f;
-                        y2[e] = vv * ww - __uint_as_float(r[2 * i + e]);
+                        y2[e] = vv * ww - __uint_as_float(r[ii]);
                     }
                     split_pack(y2[0], y2[1], hi[i], lo[i]);
                 }
@@ -311,19 +335,23 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             named_bar(1, 256);
             // ---- X3 = Y^T T^T = V'^T; v/w of the next chunk --------------------------------------
             if (tid == 0) {
+                GDN_TRACE(n, 4);
                 tc_fence_after();
                 if (vw_issued < NT && !*cx.abort_flag) {
                     load_vw<GPC>(cx, vw_issued, b, hv, &tm_v, &tm_w);
                     ++vw_issued;
                 }
-                if (wait_bar(cx, B_T_READY, pn) && !*cx.abort_flag) {
-                    mma_ts_k(tbase + TM_X5, tbase + TM_YH, sbase + SM_T, 64, 64, id64, false);
-                    mma_ts_k(tbase + TM_X5, tbase + TM_YL, sbase + SM_T, 64, 64, id64, true);
+                if (wait1(cx, B_T_READY, pn) && !*cx.abort_flag) {
+                    GDN_TRACE(n, 5);
+                    mma_ts_u<64, 64>(tbase + TM_X5, tbase + TM_YH, sbase + SM_T, id64, false);
+                    mma_ts_u<64, 64>(tbase + TM_X5, tbase + TM_YL, sbase + SM_T, id64, true);
                     mma_commit(cx.bars + B_X3);
                     mma_commit(cx.bars + B_T_FREE);
+                    wait1(cx, B_X3, pn);
+                    GDN_TRACE(n, 6);
                 }
             }
-            wait_bar(cx, B_X3, pn);
+            named_bar(1, 256);
             tc_fence_after();
             {
                 uint32_t r[32], hi[16], lo[16];
@@ -340,55 +368,77 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             named_bar(1, 256);
             // ---- X4 (O += V'^T P^T), X5 (dS^T = V'^T Kbar) ---------------------------------------
             if (tid == 0) {
+                GDN_TRACE(n, 7);
                 tc_fence_after();
-                const bool okp = wait_bar(cx, B_P_READY, pn);
-                const bool okk = wait_bar(cx, B_KB_READY, pn);
-                if (okp && okk && !*cx.abort_flag) {
+                const bool okp = wait1(cx, B_P_READY, pn);
+                GDN_TRACE(n, 8);
+                const bool okk = okp && wait1(cx, B_KB_READY, pn);
+                GDN_TRACE(n, 9);
+                if (okk && !*cx.abort_flag) {
                     const uint32_t P = sbase + SM_P, KB = sbase + SM_KB;
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_YH, P, 64, 64, id64, true);
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_YL, P, 64, 64, id64, true);
-                    mma_ts_k(tbase + TM_X2 + 64, tbase + TM_YH, P + 8192, 64, 64, id64, true);
-                    mma_ts_k(tbase + TM_X5, tbase + TM_YH, KB, 128, 64, id128, false);
-                    mma_ts_k(tbase + TM_X5, tbase + TM_YL, KB, 128, 64, id128, true);
-                    mma_ts_k(tbase + TM_X5, tbase + TM_YH, KB + 16384, 128, 64, id128, true);
+                    mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P, id64, true);
+                    mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YL, P, id64, true);
+                    mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P + 8192, id64, true);
+                    mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB, id128, false);
+                    mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YL, KB, id128, true);
+                    mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB + 16384, id128, true);
                     mma_commit(cx.bars + B_X45);
                     mma_commit(cx.bars + B_P_FREE);
                     mma_commit(cx.bars + B_KB_FREE);
+                    wait1(cx, B_X45, pn);
+                    GDN_TRACE(n, 10);
                 }
             }
-            wait_bar(cx, B_X45, pn);
+            named_bar(1, 256);
             tc_fence_after();
             // ---- output rows 32h .. 32h+31 of column j -----------------------------------------
             {
                 uint32_t r[32];
                 tmem_ld32(tl + TM_X2 + 64 + 32 * h, r);
                 tmem_ld_wait();
+                const long obase = pb.v_row(b, t0 + 32 * h, hv) + j;
+                const int nrow = min(32, L - 32 * h);
+                float ov[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int rr = 32 * h + i;
-                    if (rr < L) {
-                        const long off = pb.v_row(b, t0 + rr, hv) + j;
-                        float ov = pb.scale * __uint_as_float(r[i]);
-                        if (GATE) {
-                            const float zz = __bfloat162float(static_cast<const __nv_bfloat16*>(p.z)[off]);
-                            ov *= zz * sigmoidf_(zz);
+                for (int i = 0; i < 32; ++i) ov[i] = pb.scale * __uint_as_float(r[i]);
+                if (GATE) {
+                    const __nv_bfloat16* zp = static_cast<const __nv_bfloat16*>(p.z) + obase;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < nrow) {
+                            const float zz = __bfloat162float(zp[i * orow]);
+                            ov[i] *= zz * sigmoidf_(zz);
                         }
-                        if (p.o_type == 1) static_cast<float*>(p.o)[off] = ov;
-                        else static_cast<__nv_bfloat16*>(p.o)[off] = __float2bfloat16_rn(ov);
-                    }
+                }
+                if (p.o_type == 1) {
+                    float* op = static_cast<float*>(p.o) + obase;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < nrow) op[i * orow] = ov[i];
+                } else {
+                    __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + obase;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < nrow) op[i * orow] = __float2bfloat16_rn(ov[i]);
                 }
             }
             // ---- state: S = Diag(gamma) S0 + Kbar^T V'; split S0^T for the next chunk -------------
             {
-                const float* g = gam + (n % 3) * 128 + 64 * h;
+                const float4* g4 = reinterpret_cast<const float4*>(gam + (n % 3) * 128 + 64 * h);
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2) {
                     uint32_t r[32], hi[16], lo[16];
                     tmem_ld32(tl + TM_X5 + 64 * h + 32 * q2, r);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        S[32 * q2 + i] = fmaf(g[32 * q2 + i], S[32 * q2 + i], __uint_as_float(r[i]));
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 g = g4[8 * q2 + i4];
+                        const int i = 4 * i4;
+                        S[32 * q2 + i + 0] = fmaf(g.x, S[32 * q2 + i + 0], __uint_as_float(r[i + 0]));
+                        S[32 * q2 + i + 1] = fmaf(g.y, S[32 * q2 + i + 1], __uint_as_float(r[i + 1]));
+                        S[32 * q2 + i + 2] = fmaf(g.z, S[32 * q2 + i + 2], __uint_as_float(r[i + 2]));
+                        S[32 * q2 + i + 3] = fmaf(g.w, S[32 * q2 + i + 3], __uint_as_float(r[i + 3]));
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         split_pack(S[32 * q2 + 2 * i], S[32 * q2 + 2 * i + 1], hi[i], lo[i]);
@@ -397,11 +447,15 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 tmem_st_wait();
             }
+            // One thread samples the abort flag (another group may set it at any time) and the
+            // group leaves the loop together.
+            if (tid == 0) {
+                GDN_TRACE(n, 11);
+                *stop_slot = *cx.abort_flag;
+            }
             tc_fence_before();
             named_bar(1, 256);
-            const int stop = *cx.abort_flag;
-            named_bar(1, 256);
-            if (stop) break;
+            if (*stop_slot) break;
         }
         if (p.ht && !*cx.abort_flag) {
 #pragma unroll
@@ -410,6 +464,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     } else {
         // =================================== chunk prologue ===================================
         const int c = tid - 256;  // key channel; also TMEM lane of X1
+        volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 140);
         const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
         const TG* alpha_g = static_cast<const TG*>(p.alpha);
         const TG* beta_g = static_cast<const TG*>(p.b);
@@ -420,64 +475,75 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint8_t* RA = sm + SM_RA;
         uint8_t* EQ = sm + SM_EQ;
         uint8_t* QLO = sm + SM_QLO;
+        // swizzled byte offsets of channel c: 64-row tiles base64 + r*128 + xo[r&7], 128-row tiles base128 + ...
+        const uint32_t base64 = (uint32_t)(c >> 6) * 64u * 128u, base128 = (uint32_t)(c >> 6) * 128u * 128u;
+        uint32_t xo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) xo[u] = ((uint32_t)(c & 63) * 2u) ^ ((uint32_t)u << 4);
+        const uint32_t id64 = idesc_bf16_f32(128, 64);
         for (int m = 0; m < NT; ++m) {
             const uint32_t pm = m & 1, pprev = (m - 1) & 1;
             const int t0 = m * C, L = min(C, pb.T - t0);
-            wait_bar(cx, B_RAW, pm);
-            if (m > 0) wait_bar(cx, B_EQ_FREE, pprev);
+            if (c == 0) {
+                GDN_TRACE(m, 16);
+                wait1(cx, B_RAW, pm);
+                GDN_TRACE(m, 17);
+                if (m > 0) wait1(cx, B_EQ_FREE, pprev);
+                GDN_TRACE(m, 18);
+            }
+            named_bar(2, 128);
             // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA / QLO) ----------
             float G = 1.f;
 #pragma unroll 1
             for (int r0 = 0; r0 < C; r0 += 8) {
-                // loads of 8 rows first (independent of this block's stores), then compute/store
+                const uint32_t ob64 = base64 + (uint32_t)r0 * 128u, ob128 = base128 + (uint32_t)r0 * 128u;
                 float av[8], kv[8], qv[8], bv[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int r = r0 + u;
-                    const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
-                    const uint32_t ok = sw128_offset(r, c, 64);
+                    const uint32_t ok = ob64 + u * 128u + xo[u], oe = ob128 + u * 128u + xo[u];
                     if (APC) av[u] = r < L ? bf(RA, ok) : 1.f;
                     else av[u] = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
                     kv[u] = bf(RK, ok);
-                    qv[u] = bf(RQB, oq);
+                    qv[u] = bf(RQB, oe + 8192u);
                     if (GPC) bv[u] = bf(RQB, oe);
                     else bv[u] = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
                 }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const int r = r0 + u;
-                    const uint32_t oe = sw128_offset(r, c, 128), oq = sw128_offset(64 + r, c, 128);
-                    const uint32_t ok = sw128_offset(r, c, 64);
+                    const uint32_t ok = ob64 + u * 128u + xo[u], oe = ob128 + u * 128u + xo[u];
                     G *= av[u];
                     __nv_bfloat16 hi, lo;
                     split_bf16(bv[u] * kv[u] * G, hi, lo);
                     put_raw(EQ, oe, hi);
                     put_raw(RQB, oe, lo);
                     split_bf16(qv[u] * G, hi, lo);
-                    put_raw(EQ, oq, hi);
-                    put_raw(RQB, oq, lo);
+                    put_raw(EQ, oe + 8192u, hi);
+                    put_raw(RQB, oe + 8192u, lo);
                     put_raw(QLO, ok, lo);
-                    split_bf16(kv[u] / G, hi, lo);
+                    split_bf16(__fdividef(kv[u], G), hi, lo);
                     put_raw(RK, ok, hi);
                     put_raw(RA, ok, lo);
                 }
             }
             gam[(m % 3) * 128 + c] = G;
+            if (c == 0) GDN_TRACE(m, 19);
             fence_async_shared();
             named_bar(2, 128);
             // ---- X1 = [Ehat;Qhat] Ktil^T with the split operands ----------------------------------
             if (c == 0) {
                 tc_fence_after();
                 if (!*cx.abort_flag) {
-                    const uint32_t id = idesc_bf16_f32(128, 64);
-                    mma_ss_k(tbase + TM_X1, sbase + SM_EQ, 128, sbase + SM_RK, 64, 128, id, false);
-                    mma_ss_k(tbase + TM_X1, sbase + SM_EQ, 128, sbase + SM_RA, 64, 128, id, true);
-                    mma_ss_k(tbase + TM_X1, sbase + SM_RQB, 128, sbase + SM_RK, 64, 128, id, true);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RK, id64, false);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RA, id64, true);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_RQB, sbase + SM_RK, id64, true);
                     mma_commit(cx.bars + B_X1);
                 }
                 mbar_arrive(cx.bars + B_EQ_READY);
+                wait1(cx, B_X1, pm);
+                GDN_TRACE(m, 20);
             }
-            wait_bar(cx, B_X1, pm);
+            named_bar(2, 128);
             tc_fence_after();
             if (c < 64) {
                 // A row c (lanes 0-63 of X1), strictly lower, into the fp32 scratch; warps 8-9.
@@ -507,10 +573,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float x[16];
 #pragma unroll
                 for (int s2 = 0; s2 < 16; ++s2) {
-                    float acc = 0.f;
+                    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                    for (int u = 0; u < s2; ++u) acc = fmaf(ascr[ascr_index(base + s2, base + u)], x[u], acc);
-                    x[s2] = s2 == jc ? 1.f : (s2 > jc ? -acc : 0.f);
+                    for (int u = 0; u < s2; ++u) {
+                        const float a = ascr[ascr_index(base + s2, base + u)];
+                        if (u & 1) a1 = fmaf(a, x[u], a1);
+                        else a0 = fmaf(a, x[u], a0);
+                    }
+                    x[s2] = s2 == jc ? 1.f : (s2 > jc ? -(a0 + a1) : 0.f);
                 }
                 named_bar(3, 64);
 #pragma unroll
@@ -518,65 +588,84 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             named_bar(2, 128);
             // (2) block rows ib = 1..3:  T_{ib, 0:ib} = -D_ib (A_{ib, 0:ib} T_{0:ib, 0:ib}).
-            //     Thread c: row rho = c >> 3 of the block row, columns (c & 7) + 8 mm, mm < 2 ib.
+            //     Thread c: rows 2 (c >> 4) and 2 (c >> 4) + 1 of the block row, column (c & 15) of
+            //     every column block jb < ib.
             {
-                const int rho = c >> 3, g0 = c & 7;
+                const int rp = 2 * (c >> 4), cl = c & 15;
 #pragma unroll 1
                 for (int ib = 1; ib < 4; ++ib) {
-                    const int row = 16 * ib + rho, ncol = 16 * ib;
-                    float acc[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+                    const int row0 = 16 * ib + rp, ncol = 16 * ib;
+                    float acc0[3] = {0.f, 0.f, 0.f}, acc1[3] = {0.f, 0.f, 0.f};
+#pragma unroll 4
                     for (int kk = 0; kk < ncol; ++kk) {
-                        const float a = ascr[ascr_index(row, kk)];
+                        const float a0 = ascr[ascr_index(row0, kk)], a1 = ascr[ascr_index(row0 + 1, kk)];
 #pragma unroll
-                        for (int mm = 0; mm < 6; ++mm) {
-                            const int gcol = g0 + 8 * mm;
-                            // T_{0:ib,0:ib} is block lower triangular: rows below the column's block
-                            if (mm < 2 * ib && kk >= (gcol & ~15))
-                                acc[mm] = fmaf(a, ascr[ascr_index(kk, gcol)], acc[mm]);
+                        for (int jb = 0; jb < 3; ++jb) {
+                            // T_{0:ib,0:ib} is block lower triangular: rows kk >= 16 jb of column block jb
+                            if (jb < ib && kk >= 16 * jb) {
+                                const float t = ascr[ascr_index(kk, cl + 16 * jb)];
+                                acc0[jb] = fmaf(a0, t, acc0[jb]);
+                                acc1[jb] = fmaf(a1, t, acc1[jb]);
+                            }
                         }
                     }
 #pragma unroll
-                    for (int mm = 0; mm < 6; ++mm)
-                        if (mm < 2 * ib) rs[rho * 48 + g0 + 8 * mm] = acc[mm];
+                    for (int jb = 0; jb < 3; ++jb)
+                        if (jb < ib) {
+                            rs[rp * 48 + cl + 16 * jb] = acc0[jb];
+                            rs[(rp + 1) * 48 + cl + 16 * jb] = acc1[jb];
+                        }
                     named_bar(2, 128);
-                    float t6[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    float t0v[3] = {0.f, 0.f, 0.f}, t1v[3] = {0.f, 0.f, 0.f};
 #pragma unroll 4
                     for (int sg = 0; sg < 16; ++sg) {
-                        const float d = ascr[ascr_index(row, ncol + sg)];  // D_ib[rho][sg]
+                        // D_ib[rho][sg] (lower triangular with unit diagonal)
+                        const float d0 = ascr[ascr_index(row0, ncol + sg)], d1 = ascr[ascr_index(row0 + 1, ncol + sg)];
 #pragma unroll
-                        for (int mm = 0; mm < 6; ++mm)
-                            if (mm < 2 * ib) t6[mm] = fmaf(d, rs[sg * 48 + g0 + 8 * mm], t6[mm]);
+                        for (int jb = 0; jb < 3; ++jb)
+                            if (jb < ib) {
+                                const float rv = rs[sg * 48 + cl + 16 * jb];
+                                t0v[jb] = fmaf(d0, rv, t0v[jb]);
+                                t1v[jb] = fmaf(d1, rv, t1v[jb]);
+                            }
                     }
 #pragma unroll
-                    for (int mm = 0; mm < 6; ++mm)
-                        if (mm < 2 * ib) ascr[ascr_index(row, g0 + 8 * mm)] = -t6[mm];
+                    for (int jb = 0; jb < 3; ++jb)
+                        if (jb < ib) {
+                            ascr[ascr_index(row0, cl + 16 * jb)] = -t0v[jb];
+                            ascr[ascr_index(row0 + 1, cl + 16 * jb)] = -t1v[jb];
+                        }
                     named_bar(2, 128);
                 }
             }
             // (3) T (fp32) -> bf16 K-major tile: thread c converts 32 entries of row c >> 1.
-            if (m > 0) wait_bar(cx, B_T_FREE, pprev);
+            if (c == 0) GDN_TRACE(m, 21);
+            if (c == 0 && m > 0) wait1(cx, B_T_FREE, pprev);
+            if (c == 0) GDN_TRACE(m, 22);
+            named_bar(2, 128);
             {
                 const int row = c >> 1, col0 = 32 * (c & 1);
                 uint8_t* Tt = sm + SM_T;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int cc = col0 + 8 * ch + 2 * e;
-                        w4[e] = pack_bf16x2(ascr[ascr_index(row, cc)], ascr[ascr_index(row, cc + 1)]);
-                    }
+                    const float4 f0 = *reinterpret_cast<const float4*>(ascr + ascr_index(row, col0 + 8 * ch));
+                    const float4 f1 = *reinterpret_cast<const float4*>(ascr + ascr_index(row, col0 + 8 * ch + 4));
                     *reinterpret_cast<uint4*>(Tt + sw128_offset(row, col0 + 8 * ch, 64)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                                   pack_bf16x2(f1.z, f1.w));
                 }
             }
             fence_async_shared();
             named_bar(2, 128);
-            if (c == 0) mbar_arrive(cx.bars + B_T_READY);
-            // ---- P (lower triangle with the diagonal), split, from lanes 64-127 -------------------
-            if (m > 0) wait_bar(cx, B_P_FREE, pprev);
+            if (c == 0) {
+                mbar_arrive(cx.bars + B_T_READY);
+                GDN_TRACE(m, 23);
+                if (m > 0) wait1(cx, B_P_FREE, pprev);
+                GDN_TRACE(m, 24);
+            }
+            named_bar(2, 128);
             tc_fence_after();
+            // ---- P (lower triangle with the diagonal), split, from lanes 64-127 -------------------
             if (c >= 64) {
                 // P row c - 64 (lanes 64-127 of X1, intact until the next chunk's X1); warps 10-11.
                 const int rr = c - 64;
@@ -605,18 +694,23 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tc_fence_before();
             fence_async_shared();
             named_bar(2, 128);
-            if (c == 0) mbar_arrive(cx.bars + B_P_READY);
+            if (c == 0) {
+                mbar_arrive(cx.bars + B_P_READY);
+                GDN_TRACE(m, 25);
+                if (m > 0) wait1(cx, B_KB_FREE, pprev);
+                GDN_TRACE(m, 26);
+            }
+            named_bar(2, 128);
             // ---- Kbar^T row c = (Ktil hi + lo) * gamma, split; then reload the raw stage -----------
-            if (m > 0) wait_bar(cx, B_KB_FREE, pprev);
             {
                 uint8_t* KB = sm + SM_KB;
-#pragma unroll 1
+#pragma unroll 2
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t wh[4], wl[4];
+                    const uint32_t ob = base64 + (uint32_t)ch * 1024u;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int r = 8 * ch + 2 * e;
-                        const uint32_t o0 = sw128_offset(r, c, 64), o1 = sw128_offset(r + 1, c, 64);
+                        const uint32_t o0 = ob + (2 * e) * 128u + xo[2 * e], o1 = ob + (2 * e + 1) * 128u + xo[2 * e + 1];
                         const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
                         split_pack(k0, k1, wh[e], wl[e]);
                     }
@@ -629,15 +723,16 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             named_bar(2, 128);
             if (c == 0) {
                 mbar_arrive(cx.bars + B_KB_READY);
+                GDN_TRACE(m, 27);
                 // X1 and the Kbar^T pass were the last readers of the raw stage.
                 if (raw_issued < NT && !*cx.abort_flag) {
                     load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
                     ++raw_issued;
                 }
+                *stop_slot = *cx.abort_flag;
             }
-            const int stop = *cx.abort_flag;
             named_bar(2, 128);
-            if (stop) break;
+            if (*stop_slot) break;
         }
     }
 

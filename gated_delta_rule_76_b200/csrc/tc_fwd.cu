@@ -96,3 +96,10 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
 }
 
 }  // namespace gdn
+
+#ifdef GDN_FWD_TRACE
+// Profiling builds only: copy the phase timestamps of CTA 0 of the last forward to the host.
+extern "C" __attribute__((visibility("default"))) int gdn_fwd_trace_read(unsigned long long* host) {
+    return (int)cudaMemcpyFromSymbol(host, gdn::tcfwd::g_fwd_trace, sizeof(unsigned long long) * 64 * 32);
+}
+#endif

@@ -176,6 +176,44 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// Unrolled K-loops with the shared-memory descriptors computed once: the start-address field
+// (bits [0,14), 16-byte units) advances by the K offset; tiles stay below 256 KB, so the field never
+// carries into the next one.  A_ROWS / B_ROWS: rows per 128-byte-wide atom column of the tile.
+template <int K, int A_ROWS, int B_ROWS>
+__device__ __forceinline__ void mma_ss_u(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc,
+                                         bool accumulate) {
+    const uint64_t da = sdesc_k_sw128(a_smem), db = sdesc_k_sw128(b_smem);
+#pragma unroll
+    for (int k = 0; k < K; k += 16) {
+        const uint32_t ao = ((uint32_t)(k >> 6) * A_ROWS * 128u + (uint32_t)(k & 63) * 2u) >> 4;
+        const uint32_t bo = ((uint32_t)(k >> 6) * B_ROWS * 128u + (uint32_t)(k & 63) * 2u) >> 4;
+        mma_ss(d_tmem, da + ao, db + bo, idesc, (accumulate || k > 0) ? 1u : 0u);
+    }
+}
+template <int K, int B_ROWS>
+__device__ __forceinline__ void mma_ts_u(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
+                                         bool accumulate) {
+    const uint64_t db = sdesc_k_sw128(b_smem);
+#pragma unroll
+    for (int k = 0; k < K; k += 16) {
+        const uint32_t bo = ((uint32_t)(k >> 6) * B_ROWS * 128u + (uint32_t)(k & 63) * 2u) >> 4;
+        mma_ts(d_tmem, a_tmem + (uint32_t)(k >> 1), db + bo, idesc, (accumulate || k > 0) ? 1u : 0u);
+    }
+}
+
+// Wait for the phase of the given parity, sleeping in hardware between polls (suspend hint in ns).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Issue a K-loop of MMAs for operands in K-major SW128 tiles.  A: M rows (a_rows rows per atom
 // column), B: N rows (b_rows per atom column); K in multiples of 16.
 __device__ __forceinline__ void mma_ss_k(uint32_t d_tmem, uint32_t a_smem, int a_rows, uint32_t b_smem,
