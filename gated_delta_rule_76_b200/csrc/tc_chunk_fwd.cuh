@@ -84,11 +84,14 @@ constexpr uint32_t SM_T = 114688;     // 8 KB [1][64]: T
 constexpr uint32_t SM_P = 122880;     // 16 KB: P hi [1][64], P lo [1][64]
 constexpr uint32_t SM_KB = 139264;    // 32 KB: Kbar^T hi [1][128], Kbar^T lo [1][128]
 constexpr uint32_t SM_VW = 172032;    // 32 KB: v [2][64], w [2][64]
-constexpr uint32_t SM_ASCR = 204800;  // 16 KB: A fp32 [64][64], float4 columns XOR-swizzled by row
-constexpr uint32_t SM_GAM = 221184;   // gamma, 3 slots x 128 floats (chunk n uses slot n % 3)
-constexpr uint32_t SM_BAR = 222720;   // mbarriers, tensor memory base, abort flag
-constexpr uint32_t SM_RS = SM_BAR + 256;  // 3 KB fp32 [16][48]: block-row products of the solve
-constexpr uint32_t SM_END = SM_RS + 3072;
+constexpr uint32_t SM_ASCR = 204800;  // 17 KB: A, then T, fp32 [64][LDA] row-major
+constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats (chunk n uses slot n % 3)
+constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, abort flag
+constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: alpha products per row group [8][128], then the
+                                          // block-row products of the solve [16][LDR]
+constexpr uint32_t SM_END = SM_RS + 4096;
+constexpr int LDA = 68;  // fp32 row stride of the A/T scratch: float4 rows, rows 16 B apart in bank
+constexpr int LDR = 52;  // fp32 row stride of the block-row products
 constexpr size_t kSmemBytes = SM_END + 1024;
 
 enum Bar {
@@ -138,8 +141,74 @@ __device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uin
     const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
     lo = pack_bf16x2(x0 - h0, x1 - h1);
 }
-__device__ __forceinline__ uint32_t ascr_index(int r, int c) {  // fp32 element index
-    return (uint32_t)r * 64u + ((uint32_t)((c >> 2) ^ (r & 15)) << 2) + (uint32_t)(c & 3);
+// 8 bf16 (one 16-byte chunk of a swizzled row) <-> 8 floats.
+__device__ __forceinline__ void unpack8(const uint4 v, float (&x)[8]) {
+    x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    x[4] = __uint_as_float(v.z << 16); x[5] = __uint_as_float(v.z & 0xFFFF0000u);
+    x[6] = __uint_as_float(v.w << 16); x[7] = __uint_as_float(v.w & 0xFFFF0000u);
+}
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+    split_pack(x[0], x[1], hi.x, lo.x);
+    split_pack(x[2], x[3], hi.y, lo.y);
+    split_pack(x[4], x[5], hi.z, lo.z);
+    split_pack(x[6], x[7], hi.w, lo.w);
+}
+__device__ __forceinline__ uint4 ld16(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void st16(uint8_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+__device__ __forceinline__ float4 ldf4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void fma4(float (&acc)[4], float a, const float4 t) {
+    acc[0] = fmaf(a, t.x, acc[0]);
+    acc[1] = fmaf(a, t.y, acc[1]);
+    acc[2] = fmaf(a, t.z, acc[2]);
+    acc[3] = fmaf(a, t.w, acc[3]);
+}
+
+// One block row IB (rows 16 IB .. 16 IB + 15) of T = (I + A)^-1, given the diagonal blocks
+// D_i = (I + A_ii)^-1 and the block rows above it, in place in the fp32 scratch t (row stride LDA):
+//   R = A_{IB, 0:IB} T_{0:IB, 0:IB},   T_{IB, 0:IB} = -D_IB R.
+// Thread c < 32 IB computes rows 2 rp, 2 rp + 1 of the block row and columns 4 cg .. 4 cg + 3.
+template <int IB>
+__device__ __forceinline__ void solve_block_row(float* t, float* rsb, int c) {
+    constexpr int NCG = 4 * IB;
+    const bool act = c < 8 * NCG;
+    const int cg = c % NCG, rp = c / NCG;
+    const int row = 16 * IB + 2 * rp, col = 4 * cg;
+    if (act) {
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* a0p = t + row * LDA;
+        // T_{0:IB, jb} is zero above its diagonal block: start at row 16 jb of the column block.
+#pragma unroll 1
+        for (int kk = 16 * (col >> 4); kk < 16 * IB; kk += 4) {
+            const float4 a0 = ldf4(a0p + kk), a1 = ldf4(a0p + LDA + kk);
+            const float4 t0 = ldf4(t + (kk + 0) * LDA + col), t1 = ldf4(t + (kk + 1) * LDA + col);
+            const float4 t2 = ldf4(t + (kk + 2) * LDA + col), t3 = ldf4(t + (kk + 3) * LDA + col);
+            fma4(acc0, a0.x, t0); fma4(acc1, a1.x, t0);
+            fma4(acc0, a0.y, t1); fma4(acc1, a1.y, t1);
+            fma4(acc0, a0.z, t2); fma4(acc1, a1.z, t2);
+            fma4(acc0, a0.w, t3); fma4(acc1, a1.w, t3);
+        }
+        *reinterpret_cast<float4*>(rsb + (2 * rp) * LDR + col) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
+        *reinterpret_cast<float4*>(rsb + (2 * rp + 1) * LDR + col) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
+    }
+    named_bar(2, 128);
+    if (act) {
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* d0p = t + row * LDA + 16 * IB;
+#pragma unroll
+        for (int sg = 0; sg < 16; sg += 4) {
+            const float4 d0 = ldf4(d0p + sg), d1 = ldf4(d0p + LDA + sg);
+            const float4 r0 = ldf4(rsb + (sg + 0) * LDR + col), r1 = ldf4(rsb + (sg + 1) * LDR + col);
+            const float4 r2 = ldf4(rsb + (sg + 2) * LDR + col), r3 = ldf4(rsb + (sg + 3) * LDR + col);
+            fma4(acc0, d0.x, r0); fma4(acc1, d1.x, r0);
+            fma4(acc0, d0.y, r1); fma4(acc1, d1.y, r1);
+            fma4(acc0, d0.z, r2); fma4(acc1, d1.z, r2);
+            fma4(acc0, d0.w, r3); fma4(acc1, d1.w, r3);
+        }
+        *reinterpret_cast<float4*>(t + row * LDA + col) = make_float4(-acc0[0], -acc0[1], -acc0[2], -acc0[3]);
+        *reinterpret_cast<float4*>(t + (row + 1) * LDA + col) = make_float4(-acc1[0], -acc1[1], -acc1[2], -acc1[3]);
+    }
+    named_bar(2, 128);
 }
 
 struct Ctx {
@@ -493,40 +562,103 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             named_bar(2, 128);
             // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA / QLO) ----------
-            float G = 1.f;
-#pragma unroll 1
-            for (int r0 = 0; r0 < C; r0 += 8) {
-                const uint32_t ob64 = base64 + (uint32_t)r0 * 128u, ob128 = base128 + (uint32_t)r0 * 128u;
-                float av[8], kv[8], qv[8], bv[8];
+            // Thread c: channels 8 cg .. 8 cg + 7 (one 16-byte chunk of a swizzled row) of rows
+            // 8 rg .. 8 rg + 7.  Gamma over the chunk is the product of the row groups' products.
+            {
+                const int cg = c & 15, rg = c >> 4, r0 = 8 * rg;
+                const uint32_t a64 = (uint32_t)(cg >> 3) * 64u * 128u + (uint32_t)r0 * 128u;
+                const uint32_t a128 = (uint32_t)(cg >> 3) * 128u * 128u + (uint32_t)r0 * 128u;
+                const uint32_t ch = (uint32_t)(cg & 7);
+                float* part = rs;  // [8][128]
+                float Gl[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) Gl[i] = 1.f;
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int r = r0 + u;
-                    const uint32_t ok = ob64 + u * 128u + xo[u], oe = ob128 + u * 128u + xo[u];
-                    if (APC) av[u] = r < L ? bf(RA, ok) : 1.f;
-                    else av[u] = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
-                    kv[u] = bf(RK, ok);
-                    qv[u] = bf(RQB, oe + 8192u);
-                    if (GPC) bv[u] = bf(RQB, oe);
-                    else bv[u] = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
-                }
+                    float a8[8];
+                    if (APC) {
+                        unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+                        if (r >= L) {
 #pragma unroll
+                            for (int i = 0; i < 8; ++i) a8[i] = 1.f;
+                        }
+                    } else {
+                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) a8[i] = av;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) Gl[i] *= a8[i];
+                }
+                *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg) = make_float4(Gl[0], Gl[1], Gl[2], Gl[3]);
+                *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg + 4) = make_float4(Gl[4], Gl[5], Gl[6], Gl[7]);
+                named_bar(2, 128);
+                float G[8], gm[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) G[i] = gm[i] = 1.f;
+#pragma unroll
+                for (int g2 = 0; g2 < 8; ++g2) {
+                    const float4 p0 = ldf4(part + g2 * 128 + 8 * cg), p1 = ldf4(part + g2 * 128 + 8 * cg + 4);
+                    const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (g2 < rg) G[i] *= pv[i];
+                        gm[i] *= pv[i];
+                    }
+                }
+                if (rg == 0) {
+                    float* gs = gam + (m % 3) * 128 + 8 * cg;
+                    *reinterpret_cast<float4*>(gs) = make_float4(gm[0], gm[1], gm[2], gm[3]);
+                    *reinterpret_cast<float4*>(gs + 4) = make_float4(gm[4], gm[5], gm[6], gm[7]);
+                }
+#pragma unroll 2
                 for (int u = 0; u < 8; ++u) {
-                    const uint32_t ok = ob64 + u * 128u + xo[u], oe = ob128 + u * 128u + xo[u];
-                    G *= av[u];
-                    __nv_bfloat16 hi, lo;
-                    split_bf16(bv[u] * kv[u] * G, hi, lo);
-                    put_raw(EQ, oe, hi);
-                    put_raw(RQB, oe, lo);
-                    split_bf16(qv[u] * G, hi, lo);
-                    put_raw(EQ, oe + 8192u, hi);
-                    put_raw(RQB, oe + 8192u, lo);
-                    put_raw(QLO, ok, lo);
-                    split_bf16(__fdividef(kv[u], G), hi, lo);
-                    put_raw(RK, ok, hi);
-                    put_raw(RA, ok, lo);
+                    const int r = r0 + u;
+                    const uint32_t sw = (ch ^ (uint32_t)u) << 4;
+                    const uint32_t o64 = a64 + u * 128u + sw, oe = a128 + u * 128u + sw, oq = oe + 64u * 128u;
+                    float a8[8], k8[8], q8[8], b8[8];
+                    if (APC) {
+                        unpack8(ld16(RA + o64), a8);
+                        if (r >= L) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) a8[i] = 1.f;
+                        }
+                    } else {
+                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) a8[i] = av;
+                    }
+                    unpack8(ld16(RK + o64), k8);
+                    unpack8(ld16(RQB + oq), q8);
+                    if (GPC) {
+                        unpack8(ld16(RQB + oe), b8);
+                    } else {
+                        const float bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) b8[i] = bv;
+                    }
+                    float e8[8], qq[8], kt[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        G[i] *= a8[i];
+                        e8[i] = b8[i] * k8[i] * G[i];
+                        qq[i] = q8[i] * G[i];
+                        kt[i] = __fdividef(k8[i], G[i]);
+                    }
+                    uint4 hi, lo;
+                    split8(e8, hi, lo);
+                    st16(EQ + oe, hi);
+                    st16(RQB + oe, lo);
+                    split8(qq, hi, lo);
+                    st16(EQ + oq, hi);
+                    st16(RQB + oq, lo);
+                    st16(QLO + o64, lo);
+                    split8(kt, hi, lo);
+                    st16(RK + o64, hi);
+                    st16(RA + o64, lo);
                 }
             }
-            gam[(m % 3) * 128 + c] = G;
             if (c == 0) GDN_TRACE(m, 19);
             fence_async_shared();
             named_bar(2, 128);
@@ -560,99 +692,65 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         v4.y = s0 + 1 < c ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
                         v4.z = s0 + 2 < c ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
                         v4.w = s0 + 3 < c ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
-                        *reinterpret_cast<float4*>(ascr + ascr_index(c, s0)) = v4;
+                        *reinterpret_cast<float4*>(ascr + c * LDA + s0) = v4;
                     }
                 }
             }
             tc_fence_before();
             named_bar(2, 128);
+            if (c == 0) GDN_TRACE(m, 31);
             // ---- T = (I + A)^-1 by 16 x 16 blocks, in place in the fp32 scratch ------------------
-            // (1) diagonal blocks D_i = (I + A_ii)^-1: thread c < 64 solves column c & 15 of block c >> 4.
+            // (1) diagonal blocks D_i = (I + A_ii)^-1: thread c < 64 solves column c & 15 of block
+            //     c >> 4 by forward substitution.
             if (c < 64) {
                 const int base = 16 * (c >> 4), jc = c & 15;
                 float x[16];
 #pragma unroll
                 for (int s2 = 0; s2 < 16; ++s2) {
+                    const float* arow = ascr + (base + s2) * LDA + base;
                     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                    for (int u = 0; u < s2; ++u) {
-                        const float a = ascr[ascr_index(base + s2, base + u)];
-                        if (u & 1) a1 = fmaf(a, x[u], a1);
-                        else a0 = fmaf(a, x[u], a0);
+                    for (int u4 = 0; u4 < (s2 + 3) / 4; ++u4) {
+                        const float4 a4 = ldf4(arow + 4 * u4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int u = 4 * u4 + e;
+                            if (u < s2) {
+                                if (u & 1) a1 = fmaf(av[e], x[u], a1);
+                                else a0 = fmaf(av[e], x[u], a0);
+                            }
+                        }
                     }
                     x[s2] = s2 == jc ? 1.f : (s2 > jc ? -(a0 + a1) : 0.f);
                 }
                 named_bar(3, 64);
 #pragma unroll
-                for (int s2 = 0; s2 < 16; ++s2) ascr[ascr_index(base + s2, base + jc)] = x[s2];
+                for (int s2 = 0; s2 < 16; ++s2) ascr[(base + s2) * LDA + base + jc] = x[s2];
             }
             named_bar(2, 128);
-            // (2) block rows ib = 1..3:  T_{ib, 0:ib} = -D_ib (A_{ib, 0:ib} T_{0:ib, 0:ib}).
-            //     Thread c: rows 2 (c >> 4) and 2 (c >> 4) + 1 of the block row, column (c & 15) of
-            //     every column block jb < ib.
-            {
-                const int rp = 2 * (c >> 4), cl = c & 15;
-#pragma unroll 1
-                for (int ib = 1; ib < 4; ++ib) {
-                    const int row0 = 16 * ib + rp, ncol = 16 * ib;
-                    float acc0[3] = {0.f, 0.f, 0.f}, acc1[3] = {0.f, 0.f, 0.f};
-#pragma unroll 4
-                    for (int kk = 0; kk < ncol; ++kk) {
-                        const float a0 = ascr[ascr_index(row0, kk)], a1 = ascr[ascr_index(row0 + 1, kk)];
-#pragma unroll
-                        for (int jb = 0; jb < 3; ++jb) {
-                            // T_{0:ib,0:ib} is block lower triangular: rows kk >= 16 jb of column block jb
-                            if (jb < ib && kk >= 16 * jb) {
-                                const float t = ascr[ascr_index(kk, cl + 16 * jb)];
-                                acc0[jb] = fmaf(a0, t, acc0[jb]);
-                                acc1[jb] = fmaf(a1, t, acc1[jb]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int jb = 0; jb < 3; ++jb)
-                        if (jb < ib) {
-                            rs[rp * 48 + cl + 16 * jb] = acc0[jb];
-                            rs[(rp + 1) * 48 + cl + 16 * jb] = acc1[jb];
-                        }
-                    named_bar(2, 128);
-                    float t0v[3] = {0.f, 0.f, 0.f}, t1v[3] = {0.f, 0.f, 0.f};
-#pragma unroll 4
-                    for (int sg = 0; sg < 16; ++sg) {
-                        // D_ib[rho][sg] (lower triangular with unit diagonal)
-                        const float d0 = ascr[ascr_index(row0, ncol + sg)], d1 = ascr[ascr_index(row0 + 1, ncol + sg)];
-#pragma unroll
-                        for (int jb = 0; jb < 3; ++jb)
-                            if (jb < ib) {
-                                const float rv = rs[sg * 48 + cl + 16 * jb];
-                                t0v[jb] = fmaf(d0, rv, t0v[jb]);
-                                t1v[jb] = fmaf(d1, rv, t1v[jb]);
-                            }
-                    }
-#pragma unroll
-                    for (int jb = 0; jb < 3; ++jb)
-                        if (jb < ib) {
-                            ascr[ascr_index(row0, cl + 16 * jb)] = -t0v[jb];
-                            ascr[ascr_index(row0 + 1, cl + 16 * jb)] = -t1v[jb];
-                        }
-                    named_bar(2, 128);
-                }
-            }
-            // (3) T (fp32) -> bf16 K-major tile: thread c converts 32 entries of row c >> 1.
+            if (c == 0) GDN_TRACE(m, 28);
+            // (2) block rows 1..3 below the diagonal.
+            solve_block_row<1>(ascr, rs, c);
+            if (c == 0) GDN_TRACE(m, 29);
+            solve_block_row<2>(ascr, rs, c);
+            if (c == 0) GDN_TRACE(m, 30);
+            solve_block_row<3>(ascr, rs, c);
+            // (3) T (fp32) -> bf16 K-major tile: thread c converts half c >> 6 of row c & 63.
             if (c == 0) GDN_TRACE(m, 21);
             if (c == 0 && m > 0) wait1(cx, B_T_FREE, pprev);
             if (c == 0) GDN_TRACE(m, 22);
             named_bar(2, 128);
             {
-                const int row = c >> 1, col0 = 32 * (c & 1);
+                const int row = c & 63, col0 = 32 * (c >> 6);
                 uint8_t* Tt = sm + SM_T;
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const float4 f0 = *reinterpret_cast<const float4*>(ascr + ascr_index(row, col0 + 8 * ch));
-                    const float4 f1 = *reinterpret_cast<const float4*>(ascr + ascr_index(row, col0 + 8 * ch + 4));
-                    *reinterpret_cast<uint4*>(Tt + sw128_offset(row, col0 + 8 * ch, 64)) =
-                        make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
-                                   pack_bf16x2(f1.z, f1.w));
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const float4 f0 = ldf4(ascr + row * LDA + col0 + 8 * q8);
+                    const float4 f1 = ldf4(ascr + row * LDA + col0 + 8 * q8 + 4);
+                    st16(Tt + sw128_offset(row, col0 + 8 * q8, 64),
+                         make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                                    pack_bf16x2(f1.z, f1.w)));
                 }
             }
             fence_async_shared();
@@ -704,6 +802,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ---- Kbar^T row c = (Ktil hi + lo) * gamma, split; then reload the raw stage -----------
             {
                 uint8_t* KB = sm + SM_KB;
+                const float G = gam[(m % 3) * 128 + c];
 #pragma unroll 2
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t wh[4], wl[4];
