@@ -267,6 +267,12 @@ gdn_status copy_state(float* dst, const float* src, size_t bytes, cudaStream_t s
 
 }  // namespace
 
+namespace gdn {
+// For the other translation units of the C ABI.
+gdn_status check_fwd_args(const gdn_fwd_args* a) { return check_fwd(a); }
+gdn_status record_error(gdn_status code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace gdn
+
 extern "C" {
 
 static bool fwd_uses_tensor_cores(const gdn_fwd_args* a, const Problem& pb) {

@@ -59,7 +59,7 @@ class LayerArgs(ctypes.Structure):
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
 
 
-EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_bwd_workspace_size",
+EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
             "gdn_layer_core_fwd", "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches",
             "gdn_version"]
@@ -83,6 +83,8 @@ def load(path: str = LIB_PATH):
     lib.gdn_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(FwdArgs), P, ctypes.c_size_t, P]
     lib.gdn_chunk_fwd.restype = ctypes.c_int
+    lib.gdn_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdArgs), P]
+    lib.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.gdn_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
     lib.gdn_chunk_bwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_chunk_bwd.argtypes = [ctypes.POINTER(BwdArgs), P, ctypes.c_size_t, P]
@@ -205,6 +207,23 @@ def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, he
     need = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, q.device, workspace)
     check(lib.gdn_chunk_fwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_fwd")
+    return o, ht
+
+
+def gdn_chunk_fwd_noalloc(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
+                          scale: float = 1.0, *, o=None, ht=None, want_ht: bool = True, out_f32: bool = False,
+                          stream=None):
+    """gdn_chunk_fwd with the library's built-in 16 MiB scratch instead of a workspace (calls on one
+    device must not overlap in time).  Returns (o, ht)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
+    if ht is None and want_ht:
+        ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    lib = load()
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht)
+    check(lib.gdn_chunk_fwd_noalloc(ctypes.byref(a), _stream(stream)), "gdn_chunk_fwd_noalloc")
     return o, ht
 
 

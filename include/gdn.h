@@ -103,6 +103,25 @@ GDN_API size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args);
 GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size_t workspace_bytes,
                          gdn_stream stream);
 
+/* Chunkwise forward without a caller workspace.  The source pages have no counterpart: this is a
+ * convenience of the library for callers that cannot hand out device memory.  Arguments, results,
+ * validation and errors are those of gdn_chunk_fwd; the scratch memory is a fixed 16 MiB device
+ * array inside the library (one per device), used as gdn_chunk_fwd's workspace.
+ *  - Limit: a problem whose gdn_chunk_fwd_workspace_size() exceeds 16 MiB is rejected with
+ *    GDN_ERR_WORKSPACE before anything is launched (the tensor-core path needs 256 bytes, so
+ *    bf16 problems with dk = dv = 128 always fit; the CUDA-core path needs per-chunk factors).
+ *  - Set-up: the first call on a device resolves the array's address on that (current) device
+ *    with cudaGetSymbolAddress, which may load the library's device code; make the first call on
+ *    each device before any stream capture.  Later calls only launch work on `stream`.
+ *  - Nothing is allocated (no cudaMalloc, no host or device allocation by any library).  The
+ *    status word at the start of the scratch is cleared on `stream` at the start of every call;
+ *    nothing else in the scratch needs to start at zero.  The status word is not readable by the
+ *    caller: an expired bounded wait inside a kernel is not reported by this call.
+ *  - Concurrency: every call on a device uses the same scratch array.  Calls whose execution can
+ *    overlap (different streams, or different host threads without ordering) race on it; the
+ *    caller must order them, e.g. by issuing them all on one stream. */
+GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, gdn_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Chunkwise backward.  Reverse mode of gdn_chunk_fwd (without z): the chunk-boundary states are
  * recomputed, the state gradient is scanned from the last chunk to the first, and per chunk the
