@@ -188,18 +188,28 @@ class ClockSampler:
 # distributed plumbing
 # --------------------------------------------------------------------------------------------
 class Dist:
-    def __init__(self, ngpus):
+    """One process per GPU: NCCL for the timing reduction (gloo on CPU, for the host-logic tests).
+    Every rank takes the same collective steps: one barrier on each side of a timed region and one
+    max-reduction of its elapsed time."""
+
+    def __init__(self, ngpus, backend=None):
         import torch
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cuda"
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                    device_id=torch.device("cuda", self.local))
+            backend = backend or "nccl"
+            kw = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            else:
+                self.device = "cpu"
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600), **kw)
             self.pg = dist
         elif torch.cuda.is_available():
             torch.cuda.set_device(0)
@@ -212,7 +222,7 @@ class Dist:
         if not self.pg:
             return x
         import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 

@@ -26,7 +26,7 @@
  * differences for the backward, split/decode carry).  Parity unpinned: none of the functions
  * below; the L2-norm epsilon (1e-6) is a reading, the pages give none.
  *
- * Build: g++ -O2 -std=c++17 -fPIC -shared -pthread (no -ffast-math), see oracle/build.py.
+ * Build: g++ -O2 -std=c++17 -fPIC -shared -pthread (no -ffast-math), see build() in oracle/oracle.py.
  */
 #include <atomic>
 #include <cmath>
