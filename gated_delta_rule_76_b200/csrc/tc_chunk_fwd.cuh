@@ -26,14 +26,16 @@
 // the fp32 state in registers, split between the warpgroups by halves of dk.
 // Roles (384 threads):
 //   warps 0-7  (scan)     : the sequential chain X2 -> Y -> X3 -> V' -> X4, X5 -> output, state;
-//                           thread 0 issues the scan's MMAs and the v/w TMA loads.
+//                           while the prologue solves for T they also build P (from X1) and
+//                           Kbar^T (from the split Ktil).  Thread 0 issues the scan's MMAs and all
+//                           TMA loads.
 //   warps 8-11 (prologue) : for the next chunk, the cumulative decay and the split operands, X1,
-//                           the triangular solve T = (I + A)^-1, P and Kbar^T; thread 256 issues
-//                           X1 and the q/k/alpha/b TMA loads.
-// Operand tiles are single-buffered: each has a "ready" barrier (prologue -> scan) and a "free"
-// barrier (the scan's MMA that read it has completed -> prologue); the raw TMA stage is reloaded as
-// soon as X1 (its last reader) completes.  Every mbarrier wait is bounded: on expiry the kernel sets
-// an error word, stops issuing work and frees its tensor memory.
+//                           and the triangular solve T = (I + A)^-1; thread 256 issues X1.
+// Operand tiles are single-buffered.  [Ehat;Qhat] and T each have a "ready" barrier (prologue ->
+// scan) and a "free" barrier (the scan's MMA that read it has completed -> prologue); the raw TMA
+// stage is reloaded once X1 and the Kbar^T pass (its last readers) are done.  Every mbarrier wait
+// is bounded: on expiry the kernel sets an error word, stops issuing work and frees its tensor
+// memory.
 #pragma once
 #include <cuda.h>
 
@@ -102,12 +104,7 @@ enum Bar {
     B_EQ_FREE,      // X2 complete
     B_T_READY,
     B_T_FREE,       // X3 complete
-    B_P_READY,
-    B_P_FREE,       // X4 complete
-    B_KB_READY,
-    B_KB_FREE,      // X5 complete
     B_X2A,
-    B_X2B,
     B_X3,
     B_X45,
     B_COUNT
@@ -400,8 +397,69 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tmem_st16(tl + TM_YL + 16 * h, lo);
                 tmem_st_wait();
             }
+            // ---- P and Kbar^T of this chunk (operands of X4, X5) while the prologue solves for T ----
+            if (tid == 0) {
+                tc_fence_after();
+                wait1(cx, B_X1, pn);
+                GDN_TRACE(n, 8);
+            }
             tc_fence_before();
             named_bar(1, 256);
+            tc_fence_after();
+            if (j >= 64) {
+                // P row j - 64 (lanes 64-127 of X1), columns 32 h .. 32 h + 31, lower with diagonal.
+                const int rr = j - 64;
+                uint8_t* Ph = sm + SM_P;
+                uint32_t r[32];
+                tmem_ld32(tl + TM_X1 + 32 * h, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t wh[4], wl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i0 = 8 * ch + 2 * e, s0 = 32 * h + i0;
+                        const float x0 = s0 <= rr ? __uint_as_float(r[i0]) : 0.f;
+                        const float x1 = s0 + 1 <= rr ? __uint_as_float(r[i0 + 1]) : 0.f;
+                        split_pack(x0, x1, wh[e], wl[e]);
+                    }
+                    const uint32_t off = sw128_offset(rr, 32 * h + 8 * ch, 64);
+                    st16(Ph + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                    st16(Ph + 8192 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                }
+            }
+            {
+                // Kbar^T row j, tokens 32 h .. 32 h + 31: (Ktil hi + lo) * gamma, split.
+                uint8_t* KB = sm + SM_KB;
+                const uint8_t* RK = sm + SM_RK;
+                const uint8_t* RA = sm + SM_RA;
+                const float G = gam[(n % 3) * 128 + j];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int ch = 4 * h + cc;
+                    uint32_t wh[4], wl[4];
+                    const uint32_t ob = vbase + (uint32_t)ch * 1024u;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t o0 = ob + (2 * e) * 128u + xo[2 * e];
+                        const uint32_t o1 = ob + (2 * e + 1) * 128u + xo[2 * e + 1];
+                        const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
+                        split_pack(k0, k1, wh[e], wl[e]);
+                    }
+                    const uint32_t off = sw128_offset(j, 8 * ch, 128);
+                    st16(KB + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                    st16(KB + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                }
+            }
+            tc_fence_before();
+            fence_async_shared();
+            named_bar(1, 256);
+            // X1 and the Kbar^T pass were the last readers of the raw stage: load the next chunk's.
+            if (tid == 0) GDN_TRACE(n, 9);
+            if (tid == 0 && raw_issued < NT && !*cx.abort_flag) {
+                load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                ++raw_issued;
+            }
             // ---- X3 = Y^T T^T = V'^T; v/w of the next chunk --------------------------------------
             if (tid == 0) {
                 GDN_TRACE(n, 4);
@@ -439,11 +497,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (tid == 0) {
                 GDN_TRACE(n, 7);
                 tc_fence_after();
-                const bool okp = wait1(cx, B_P_READY, pn);
-                GDN_TRACE(n, 8);
-                const bool okk = okp && wait1(cx, B_KB_READY, pn);
-                GDN_TRACE(n, 9);
-                if (okk && !*cx.abort_flag) {
+                if (!*cx.abort_flag) {
                     const uint32_t P = sbase + SM_P, KB = sbase + SM_KB;
                     mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P, id64, true);
                     mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YL, P, id64, true);
@@ -452,8 +506,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YL, KB, id128, true);
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB + 16384, id128, true);
                     mma_commit(cx.bars + B_X45);
-                    mma_commit(cx.bars + B_P_FREE);
-                    mma_commit(cx.bars + B_KB_FREE);
                     wait1(cx, B_X45, pn);
                     GDN_TRACE(n, 10);
                 }
@@ -544,11 +596,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint8_t* RA = sm + SM_RA;
         uint8_t* EQ = sm + SM_EQ;
         uint8_t* QLO = sm + SM_QLO;
-        // swizzled byte offsets of channel c: 64-row tiles base64 + r*128 + xo[r&7], 128-row tiles base128 + ...
-        const uint32_t base64 = (uint32_t)(c >> 6) * 64u * 128u, base128 = (uint32_t)(c >> 6) * 128u * 128u;
-        uint32_t xo[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) xo[u] = ((uint32_t)(c & 63) * 2u) ^ ((uint32_t)u << 4);
         const uint32_t id64 = idesc_bf16_f32(128, 64);
         for (int m = 0; m < NT; ++m) {
             const uint32_t pm = m & 1, pprev = (m - 1) & 1;
@@ -758,76 +805,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (c == 0) {
                 mbar_arrive(cx.bars + B_T_READY);
                 GDN_TRACE(m, 23);
-                if (m > 0) wait1(cx, B_P_FREE, pprev);
-                GDN_TRACE(m, 24);
-            }
-            named_bar(2, 128);
-            tc_fence_after();
-            // ---- P (lower triangle with the diagonal), split, from lanes 64-127 -------------------
-            if (c >= 64) {
-                // P row c - 64 (lanes 64-127 of X1, intact until the next chunk's X1); warps 10-11.
-                const int rr = c - 64;
-                uint8_t* Ph = sm + SM_P;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tl + TM_X1 + 32 * half, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t wh[4], wl[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i0 = 8 * ch + 2 * e, s0 = 32 * half + i0;
-                            const float x0 = s0 <= rr ? __uint_as_float(r[i0]) : 0.f;
-                            const float x1 = s0 + 1 <= rr ? __uint_as_float(r[i0 + 1]) : 0.f;
-                            split_pack(x0, x1, wh[e], wl[e]);
-                        }
-                        const uint32_t off = sw128_offset(rr, 32 * half + 8 * ch, 64);
-                        *reinterpret_cast<uint4*>(Ph + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                        *reinterpret_cast<uint4*>(Ph + 8192 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                    }
-                }
-            }
-            tc_fence_before();
-            fence_async_shared();
-            named_bar(2, 128);
-            if (c == 0) {
-                mbar_arrive(cx.bars + B_P_READY);
-                GDN_TRACE(m, 25);
-                if (m > 0) wait1(cx, B_KB_FREE, pprev);
-                GDN_TRACE(m, 26);
-            }
-            named_bar(2, 128);
-            // ---- Kbar^T row c = (Ktil hi + lo) * gamma, split; then reload the raw stage -----------
-            {
-                uint8_t* KB = sm + SM_KB;
-                const float G = gam[(m % 3) * 128 + c];
-#pragma unroll 2
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t wh[4], wl[4];
-                    const uint32_t ob = base64 + (uint32_t)ch * 1024u;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t o0 = ob + (2 * e) * 128u + xo[2 * e], o1 = ob + (2 * e + 1) * 128u + xo[2 * e + 1];
-                        const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
-                        split_pack(k0, k1, wh[e], wl[e]);
-                    }
-                    const uint32_t off = sw128_offset(c, 8 * ch, 128);
-                    *reinterpret_cast<uint4*>(KB + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                    *reinterpret_cast<uint4*>(KB + 16384 + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-                }
-            }
-            fence_async_shared();
-            named_bar(2, 128);
-            if (c == 0) {
-                mbar_arrive(cx.bars + B_KB_READY);
-                GDN_TRACE(m, 27);
-                // X1 and the Kbar^T pass were the last readers of the raw stage.
-                if (raw_issued < NT && !*cx.abort_flag) {
-                    load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
-                    ++raw_issued;
-                }
                 *stop_slot = *cx.abort_flag;
             }
             named_bar(2, 128);
@@ -838,12 +815,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ---- teardown: TMA loads still in flight after an abort are waited for (bounded) -----------
     tc_fence_before();
     __syncthreads();
-    if (*cx.abort_flag && (tid == 0 || tid == 256)) {
+    if (*cx.abort_flag && tid == 0) {
+        // thread 0 issued every load; the last one of each stage completes phase (issued - 1)
         const uint64_t t0 = globaltimer_ns();
-        const int bar = tid == 0 ? B_VW : B_RAW;
-        const int issued = tid == 0 ? vw_issued : raw_issued;
-        // the last issued load completes phase (issued - 1)
-        while (!mbar_try_wait(cx.bars + bar, (uint32_t)((issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+        while (!mbar_try_wait(cx.bars + B_VW, (uint32_t)((vw_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+        }
+        while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
         }
     }
     __syncthreads();
