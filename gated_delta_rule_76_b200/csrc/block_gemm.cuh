@@ -2,7 +2,7 @@
 //
 // acc(m, n) += alpha * sum_k A(m, k) * B(k, n), with A(m, k) = A.p[m * A.sm + k * A.sk] and
 // B(k, n) = B.p[k * B.sk + n * B.sn]: any operand may be transposed or live in global or shared
-// memory.  Thread t owns rows m = t / NTC + i * (NTH / NTC) and columns n = t % NTC + j * NTC.
+// memory.  Thread t owns a TM x TN register tile of consecutive rows and columns.
 // Used by the fp32 (FFMA) chunk kernels; the bf16 forward uses tensor cores instead.
 #pragma once
 #include "common.cuh"
@@ -21,15 +21,20 @@ struct BlockGemm {
     static constexpr int TM = M / MTR;
     static constexpr int TN = N / NTC;
     static_assert(NTH % NTC == 0 && M % MTR == 0 && N % NTC == 0, "bad GEMM tiling");
-    static constexpr int LA = M + 1;  // odd leading dimensions: conflict-free strided stores
-    static constexpr int LB = N + 1;
-    // Shared scratch needed by mma(), in floats.
+    static_assert(TM % 4 == 0 && (TN == 2 || TN % 4 == 0), "register tile must be float4 / float2 loadable");
+    // Leading dimensions are multiples of 4 floats so that a thread's TM rows / TN columns of one
+    // k are read with 16-byte (8-byte) shared loads.
+    static constexpr int LA = M + 4;
+    static constexpr int LB = N + 4;
+    // Shared scratch needed by mma(), in floats (its base must be 16-byte aligned).
     static constexpr int kScratch = KS * (LA + LB);
 
     float acc[TM][TN];
 
-    __device__ __forceinline__ int row(int i) const { return threadIdx.x / NTC + i * MTR; }
-    __device__ __forceinline__ int col(int j) const { return threadIdx.x % NTC + j * NTC; }
+    // Thread t owns the TM consecutive rows starting at (t / NTC) * TM and the TN consecutive
+    // columns starting at (t % NTC) * TN.
+    __device__ __forceinline__ int row(int i) const { return (threadIdx.x / NTC) * TM + i; }
+    __device__ __forceinline__ int col(int j) const { return (threadIdx.x % NTC) * TN + j; }
 
     __device__ __forceinline__ void zero() {
 #pragma unroll
@@ -38,19 +43,19 @@ struct BlockGemm {
             for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
     }
 
-    // Stage A (M x ks) and B (ks x N) slices; both loops walk the operand's contiguous axis.
-    __device__ __forceinline__ void stage(const View& A, const View& B, int k0, int ks,
+    // Stage alpha * A (M x ks) and B (ks x N) slices; both loops walk the operand's contiguous axis.
+    __device__ __forceinline__ void stage(const View& A, const View& B, int k0, int ks, float alpha,
                                           float* As, float* Bs) {
         const int tid = threadIdx.x;
         if (A.sk == 1) {
             for (int idx = tid; idx < M * KS; idx += NTH) {
                 const int m = idx / KS, kk = idx % KS;
-                As[kk * LA + m] = kk < ks ? A.p[m * A.sm + (long)(k0 + kk)] : 0.f;
+                As[kk * LA + m] = kk < ks ? alpha * A.p[m * A.sm + (long)(k0 + kk)] : 0.f;
             }
         } else {
             for (int idx = tid; idx < M * KS; idx += NTH) {
                 const int m = idx % M, kk = idx / M;
-                As[kk * LA + m] = kk < ks ? A.p[m * A.sm + (long)(k0 + kk) * A.sk] : 0.f;
+                As[kk * LA + m] = kk < ks ? alpha * A.p[m * A.sm + (long)(k0 + kk) * A.sk] : 0.f;
             }
         }
         if (B.sk == 1) {
@@ -72,23 +77,42 @@ struct BlockGemm {
     __device__ void mma(const View& A, const View& B, int K, float* scratch, float alpha = 1.f) {
         float* As = scratch;
         float* Bs = scratch + KS * LA;
-        const int tm = threadIdx.x / NTC, tn = threadIdx.x % NTC;
+        const float* ap = As + (threadIdx.x / NTC) * TM;
+        const float* bp = Bs + (threadIdx.x % NTC) * TN;
         for (int k0 = 0; k0 < K; k0 += KS) {
             const int ks = K - k0 < KS ? K - k0 : KS;
             __syncthreads();
-            stage(A, B, k0, ks, As, Bs);
+            stage(A, B, k0, ks, alpha, As, Bs);
             __syncthreads();
 #pragma unroll 4
             for (int kk = 0; kk < ks; ++kk) {
                 float a[TM], b[TN];
 #pragma unroll
-                for (int i = 0; i < TM; ++i) a[i] = As[kk * LA + tm + i * MTR];
+                for (int i4 = 0; i4 < TM / 4; ++i4) {
+                    const float4 v = *reinterpret_cast<const float4*>(ap + kk * LA + 4 * i4);
+                    a[4 * i4 + 0] = v.x;
+                    a[4 * i4 + 1] = v.y;
+                    a[4 * i4 + 2] = v.z;
+                    a[4 * i4 + 3] = v.w;
+                }
+                if constexpr (TN == 2) {
+                    const float2 v = *reinterpret_cast<const float2*>(bp + kk * LB);
+                    b[0] = v.x;
+                    b[1] = v.y;
+                } else {
 #pragma unroll
-                for (int j = 0; j < TN; ++j) b[j] = Bs[kk * LB + tn + j * NTC];
+                    for (int j4 = 0; j4 < TN / 4; ++j4) {
+                        const float4 v = *reinterpret_cast<const float4*>(bp + kk * LB + 4 * j4);
+                        b[4 * j4 + 0] = v.x;
+                        b[4 * j4 + 1] = v.y;
+                        b[4 * j4 + 2] = v.z;
+                        b[4 * j4 + 3] = v.w;
+                    }
+                }
 #pragma unroll
                 for (int i = 0; i < TM; ++i)
 #pragma unroll
-                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(alpha * a[i], b[j], acc[i][j]);
+                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
             }
         }
         __syncthreads();
