@@ -43,49 +43,65 @@ struct BlockGemm {
             for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
     }
 
-    // Stage alpha * A (M x ks) and B (ks x N) slices; both loops walk the operand's contiguous axis.
-    __device__ __forceinline__ void stage(const View& A, const View& B, int k0, int ks, float alpha,
-                                          float* As, float* Bs) {
+    static constexpr int NA = M * KS / NTH;  // staged A elements per thread and K slice
+    static constexpr int NB = N * KS / NTH;  // staged B elements per thread and K slice
+    static_assert(M * KS % NTH == 0 && N * KS % NTH == 0, "staging must divide evenly");
+
+    // Read one K slice of A (M x KS) and B (KS x N) into registers; both walk the operand's
+    // contiguous axis.  Entries past K read as 0.
+    __device__ __forceinline__ void fetch(const View& A, const View& B, int k0, int K, float (&ra)[NA],
+                                          float (&rb)[NB]) const {
         const int tid = threadIdx.x;
-        if (A.sk == 1) {
-            for (int idx = tid; idx < M * KS; idx += NTH) {
-                const int m = idx / KS, kk = idx % KS;
-                As[kk * LA + m] = kk < ks ? alpha * A.p[m * A.sm + (long)(k0 + kk)] : 0.f;
-            }
-        } else {
-            for (int idx = tid; idx < M * KS; idx += NTH) {
-                const int m = idx % M, kk = idx / M;
-                As[kk * LA + m] = kk < ks ? alpha * A.p[m * A.sm + (long)(k0 + kk) * A.sk] : 0.f;
-            }
+#pragma unroll
+        for (int it = 0; it < NA; ++it) {
+            const int idx = tid + it * NTH;
+            const int m = A.sk == 1 ? idx / KS : idx % M, kk = A.sk == 1 ? idx % KS : idx / M;
+            ra[it] = k0 + kk < K ? A.p[m * A.sm + (long)(k0 + kk) * A.sk] : 0.f;
         }
-        if (B.sk == 1) {
-            for (int idx = tid; idx < N * KS; idx += NTH) {
-                const int n = idx % N, kk = idx / N;
-                Bs[kk * LB + n] = kk < ks ? B.p[(long)(k0 + kk) * B.sm + n] : 0.f;
-            }
-        } else {
-            for (int idx = tid; idx < N * KS; idx += NTH) {
-                const int n = idx / KS, kk = idx % KS;
-                Bs[kk * LB + n] = kk < ks ? B.p[(long)(k0 + kk) * B.sm + n * B.sk] : 0.f;
-            }
+#pragma unroll
+        for (int it = 0; it < NB; ++it) {
+            const int idx = tid + it * NTH;
+            const int n = B.sk == 1 ? idx % N : idx / KS, kk = B.sk == 1 ? idx / N : idx % KS;
+            rb[it] = k0 + kk < K ? B.p[(long)(k0 + kk) * B.sm + n * B.sk] : 0.f;
+        }
+    }
+    // Write the fetched slice (A scaled by alpha) to the shared staging tiles As[k][m], Bs[k][n].
+    __device__ __forceinline__ void put(const View& A, const View& B, const float (&ra)[NA],
+                                        const float (&rb)[NB], float alpha, float* As, float* Bs) const {
+        const int tid = threadIdx.x;
+#pragma unroll
+        for (int it = 0; it < NA; ++it) {
+            const int idx = tid + it * NTH;
+            const int m = A.sk == 1 ? idx / KS : idx % M, kk = A.sk == 1 ? idx % KS : idx / M;
+            As[kk * LA + m] = alpha * ra[it];
+        }
+#pragma unroll
+        for (int it = 0; it < NB; ++it) {
+            const int idx = tid + it * NTH;
+            const int n = B.sk == 1 ? idx % N : idx / KS, kk = B.sk == 1 ? idx / N : idx % KS;
+            Bs[kk * LB + n] = rb[it];
         }
     }
 
     // acc += alpha * A * B over K.  Starts and ends with a CTA barrier, so operands written by
     // any thread before the call are visible and shared operands may be overwritten after it.
-    // For B, View::sm is the stride of k and View::sk the stride of n.
+    // For B, View::sm is the stride of k and View::sk the stride of n.  The next K slice is read
+    // into registers while the current one is multiplied, so its load latency is hidden.
     __device__ void mma(const View& A, const View& B, int K, float* scratch, float alpha = 1.f) {
         float* As = scratch;
         float* Bs = scratch + KS * LA;
         const float* ap = As + (threadIdx.x / NTC) * TM;
         const float* bp = Bs + (threadIdx.x % NTC) * TN;
+        float ra[NA], rb[NB];
+        __syncthreads();  // operands written before the call are visible to fetch()
+        fetch(A, B, 0, K, ra, rb);
         for (int k0 = 0; k0 < K; k0 += KS) {
-            const int ks = K - k0 < KS ? K - k0 : KS;
             __syncthreads();
-            stage(A, B, k0, ks, alpha, As, Bs);
+            put(A, B, ra, rb, alpha, As, Bs);
             __syncthreads();
+            if (k0 + KS < K) fetch(A, B, k0 + KS, K, ra, rb);
 #pragma unroll 4
-            for (int kk = 0; kk < ks; ++kk) {
+            for (int kk = 0; kk < KS; ++kk) {
                 float a[TM], b[TN];
 #pragma unroll
                 for (int i4 = 0; i4 < TM / 4; ++i4) {
