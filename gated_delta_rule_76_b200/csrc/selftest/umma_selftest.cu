@@ -4,6 +4,8 @@
 //  gdn_selftest_mma: D1 = A * B1^T      (A 128x128 from shared memory, B1 64x128), then
 //                    D1 += A2 * B3^T    (A2 128x64, B3 64x64; accumulate into the same TMEM),
 //                    D2 = A * B2^T      (A from tensor memory, B2 128x128).
+//  gdn_selftest_mma_mn: MN-major operands (a token-major tile read with M or N = channel):
+//                    D1 = Ak X, D2 = X^T B2^T, D3 = Ak X with Ak in tensor memory.
 //  gdn_selftest_tma: one 4-D TMA box (64 channels x 1 head x 64 tokens x 1 batch, 128-byte
 //                    swizzle) of a [B,T,H,D] bf16 tensor copied to shared memory and read back
 //                    through sw128_offset(); tokens past T must read as zero.
@@ -111,6 +113,104 @@ __global__ void __launch_bounds__(128) mma_selftest_kernel(const __nv_bfloat16* 
     if (warp == 0) tmem_dealloc(tb, 256);
 }
 
+// MN-major operands.  Ak [128 x 64] (K-major), X [64 x 128] (token-major: row k, 128 MN values),
+// B2 [64 x 64] (K-major).  D1 = Ak X (B MN-major from a 64-row tile), D2 = X^T B2^T (A MN-major
+// from rows 64-127 of a 128-row tile), D3 = Ak X with Ak taken from tensor memory.
+__global__ void __launch_bounds__(128) mma_mn_selftest_kernel(const __nv_bfloat16* Ak, const __nv_bfloat16* X,
+                                                              const __nv_bfloat16* B2, float* D1, float* D2,
+                                                              float* D3, int* err) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sAk = smem;             // 128 x 64 K-major  (16 KB)
+    uint8_t* sX64 = sAk + 16384;     // X as a 64-row tile (16 KB)
+    uint8_t* sX128 = sX64 + 16384;   // X in rows 64-127 of a 128-row tile (32 KB)
+    uint8_t* sB2 = sX128 + 32768;    // 64 x 64 K-major   (8 KB)
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tbase;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    for (int i = tid; i < 128 * 64; i += 128) {
+        const int r = i / 64, c = i % 64;
+        *reinterpret_cast<__nv_bfloat16*>(sAk + sw128_offset(r, c, 128)) = Ak[i];
+    }
+    for (int i = tid; i < 64 * 128; i += 128) {
+        const int r = i / 128, c = i % 128;
+        *reinterpret_cast<__nv_bfloat16*>(sX64 + sw128_offset(r, c, 64)) = X[i];
+        *reinterpret_cast<__nv_bfloat16*>(sX128 + sw128_offset(64 + r, c, 128)) = X[i];
+    }
+    for (int i = tid; i < 64 * 64; i += 128) {
+        const int r = i / 64, c = i % 64;
+        *reinterpret_cast<__nv_bfloat16*>(sB2 + sw128_offset(r, c, 64)) = B2[i];
+    }
+    fence_async_shared();
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tbase, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = tbase;
+    const uint32_t c1 = 0, c2 = 128, c3 = 192, ca = 320;  // D1 128, D2 64, D3 128, A copy 32 columns
+    {
+        const int m = tid;
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+            uint32_t r[16];
+            for (int i = 0; i < 16; ++i) {
+                const int k = 2 * (c0 + i);
+                r[i] = pack_bf16x2(__bfloat162float(Ak[m * 64 + k]), __bfloat162float(Ak[m * 64 + k + 1]));
+            }
+            tmem_st16(tmem_addr(tb, warp * 32, ca + c0), r);
+        }
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+        const uint32_t id1 = idesc_bf16_f32_mn(128, 128, false, true);
+        const uint32_t id2 = idesc_bf16_f32_mn(128, 64, true, false);
+        for (int k = 0; k < 64; k += 16) {
+            const uint32_t acc = k > 0 ? 1u : 0u;
+            mma_ss(tb + c1, sdesc_k_sw128(smem_u32(sAk) + (uint32_t)k * 2u),
+                   sdesc_mn_sw128(smem_u32(sX64) + (uint32_t)k * 128u, 8192u), id1, acc);
+            mma_ss(tb + c2, sdesc_mn_sw128(smem_u32(sX128) + 8192u + (uint32_t)k * 128u, 16384u),
+                   sdesc_k_sw128(smem_u32(sB2) + (uint32_t)k * 2u), id2, acc);
+            mma_ts(tb + c3, tb + ca + (uint32_t)(k >> 1), sdesc_mn_sw128(smem_u32(sX64) + (uint32_t)k * 128u, 8192u),
+                   id1, acc);
+        }
+        mma_commit(&bar);
+    }
+    __syncwarp();
+    const bool ok = __syncthreads_and(mbar_wait(&bar, 0, kWaitNs) ? 1 : 0) != 0;
+    if (!ok && tid == 0) atomicExch(err, 1);
+    tc_fence_after();
+    if (ok) {
+        const int m = warp * 32 + (tid & 31);
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem_addr(tb, warp * 32, c1 + c0), r);
+            tmem_ld_wait();
+            for (int i = 0; i < 32; ++i) D1[m * 128 + c0 + i] = __uint_as_float(r[i]);
+            tmem_ld32(tmem_addr(tb, warp * 32, c3 + c0), r);
+            tmem_ld_wait();
+            for (int i = 0; i < 32; ++i) D3[m * 128 + c0 + i] = __uint_as_float(r[i]);
+        }
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem_addr(tb, warp * 32, c2 + c0), r);
+            tmem_ld_wait();
+            for (int i = 0; i < 32; ++i) D2[m * 64 + c0 + i] = __uint_as_float(r[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, 512);
+}
+
 __global__ void __launch_bounds__(128) tma_selftest_kernel(const __grid_constant__ CUtensorMap tmap, int c0,
                                                            int hh, int t0, int bb, __nv_bfloat16* out,
                                                            int* err) {
@@ -157,6 +257,17 @@ SELFTEST_API int gdn_selftest_mma(const void* A, const void* B1, const void* A2,
     mma_selftest_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(
         (const __nv_bfloat16*)A, (const __nv_bfloat16*)B1, (const __nv_bfloat16*)A2, (const __nv_bfloat16*)B3,
         (const __nv_bfloat16*)B2, D1, D2, err);
+    return (int)cudaGetLastError();
+}
+
+SELFTEST_API int gdn_selftest_mma_mn(const void* Ak, const void* X, const void* B2, float* D1, float* D2,
+                                     float* D3, int* err, void* stream) {
+    const size_t smem = 16384 + 16384 + 32768 + 8192 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(mma_mn_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return (int)e;
+    mma_mn_selftest_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(
+        (const __nv_bfloat16*)Ak, (const __nv_bfloat16*)X, (const __nv_bfloat16*)B2, D1, D2, D3, err);
     return (int)cudaGetLastError();
 }
 

@@ -148,6 +148,25 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Same, with A (bit 15) and/or B (bit 16) MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
+}
+// Shared-memory descriptor of an MN-major bf16 operand with the 128-byte swizzle: one 128-byte
+// row holds 64 consecutive MN elements of one k, 8 rows (k .. k + 7) form a 1024-byte swizzle
+// atom; `lbo_bytes` is the distance between consecutive 64-element MN groups and the next 8
+// k-rows start 1024 bytes further.  This is the layout of a token-major tile loaded by TMA in
+// boxes of 64 channels (MN = channel, K = token, lbo = box size).  Advance the start address by
+// 2048 bytes per K = 16 step.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t smem_addr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
 
 // D[tmem] (+)= A[smem] * B[smem]^T for one K = 16 slice.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,

@@ -18,6 +18,12 @@ extern "C" {
 int gdn_selftest_mma(const void* A, const void* B1, const void* A2, const void* B3, const void* B2,
                      float* D1, float* D2, int* err, void* stream);
 
+/* MN-major operands.  Ak [128x64], X [64x128], B2 [64x64] bf16 row-major.
+ * D1 [128x128] = Ak X (B MN-major: X as a 64-row token-major tile), D2 [128x64] = X^T B2^T (A
+ * MN-major: X in rows 64-127 of a 128-row tile), D3 [128x128] = Ak X with Ak in tensor memory. */
+int gdn_selftest_mma_mn(const void* Ak, const void* X, const void* B2, float* D1, float* D2, float* D3,
+                        int* err, void* stream);
+
 /* x: [B,T,H,128] bf16.  out [64x64] bf16 receives x[bb, t0 + r, hh, c0 + c] (zero where
  * t0 + r >= T), loaded by one TMA box with the 128-byte swizzle and read back in shared memory
  * through the swizzled address map. */

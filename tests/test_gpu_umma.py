@@ -19,6 +19,8 @@ def lib():
     P = ctypes.c_void_p
     L.gdn_selftest_mma.argtypes = [P] * 9
     L.gdn_selftest_mma.restype = ctypes.c_int
+    L.gdn_selftest_mma_mn.argtypes = [P] * 8
+    L.gdn_selftest_mma_mn.restype = ctypes.c_int
     L.gdn_selftest_tma.argtypes = [P] + [ctypes.c_int] * 7 + [P, P, P]
     L.gdn_selftest_tma.restype = ctypes.c_int
     return L
@@ -43,6 +45,27 @@ def test_tcgen05_mma_shared_and_tensor_memory_operands(lib):
     ref1 = A.double() @ B1.double().T + A2.double() @ B3.double().T
     ref2 = A.double() @ B2.double().T
     for got, ref, name in ((D1, ref1, "ss + accumulate"), (D2, ref2, "A from tensor memory")):
+        e = (got.cpu().double() - ref).abs().max() / ref.abs().max()
+        assert e < 1e-5, f"{name}: relative error {e:.2e}"
+
+
+def test_tcgen05_mma_mn_major_operands(lib):
+    g = torch.Generator().manual_seed(2)
+    mk = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16)
+    Ak, X, B2 = mk(128, 64), mk(64, 128), mk(64, 64)
+    dev = [t.cuda() for t in (Ak, X, B2)]
+    D1 = torch.full((128, 128), float("nan"), device="cuda")
+    D2 = torch.full((128, 64), float("nan"), device="cuda")
+    D3 = torch.full((128, 128), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = lib.gdn_selftest_mma_mn(*[p(t) for t in dev], p(D1), p(D2), p(D3), p(err),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 0 and int(err.item()) == 0
+    ref1 = Ak.double() @ X.double()
+    ref2 = X.double().T @ B2.double().T
+    for got, ref, name in ((D1, ref1, "B MN-major"), (D2, ref2, "A MN-major, 128-row tile"),
+                           (D3, ref1, "A in tensor memory, B MN-major")):
         e = (got.cpu().double() - ref).abs().max() / ref.abs().max()
         assert e < 1e-5, f"{name}: relative error {e:.2e}"
 
