@@ -25,6 +25,19 @@ namespace gdn {
 constexpr int kSimtThreads = 256;
 constexpr int kDvTile = 32;  // dv columns per scan CTA
 
+// CTA-wide element loop over N = IT * kSimtThreads indices: every load of a thread is issued before
+// any of its stores, so their latencies overlap (load(idx) -> float, store(idx, value)).
+template <int N, class Load, class Store>
+__device__ __forceinline__ void cta_load(Load load, Store store) {
+    static_assert(N % kSimtThreads == 0, "N must be a multiple of the CTA size");
+    constexpr int IT = N / kSimtThreads;
+    float v[IT];
+#pragma unroll
+    for (int it = 0; it < IT; ++it) v[it] = load((int)threadIdx.x + it * kSimtThreads);
+#pragma unroll
+    for (int it = 0; it < IT; ++it) store((int)threadIdx.x + it * kSimtThreads, v[it]);
+}
+
 struct ChunkWs {
     float *T, *P, *Eh, *Qh, *Kb, *Kt, *Gm, *gam;  // per chunk factors
     float *S0, *dSC;                              // per chunk states / state gradients
@@ -78,20 +91,26 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
     for (int c = tid; c < DK; c += kSimtThreads) {
         float G = 1.f;
         float* gm = ws.Gm ? ws.Gm + ci * C * DK : nullptr;
-        for (int r = 0; r < C; ++r) {
-            float kv = 0.f, qv = 0.f, bv = 0.f, av = 1.f;
-            if (r < L) {
-                const int t = t0 + r;
-                kv = to_f32(k[pb.qk_row(b, t, hk) + c]);
-                qv = to_f32(q[pb.qk_row(b, t, hk) + c]);
-                av = to_f32(al[pb.gate_row(b, t, hv, APC ? DK : 1) + (APC ? c : 0)]);
-                bv = to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]);
+        for (int r0 = 0; r0 < C; r0 += 8) {
+            float kv[8], qv[8], bv[8], av[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = r0 + u, t = t0 + r;
+                const bool in = r < L;
+                kv[u] = in ? to_f32(k[pb.qk_row(b, t, hk) + c]) : 0.f;
+                qv[u] = in ? to_f32(q[pb.qk_row(b, t, hk) + c]) : 0.f;
+                av[u] = in ? to_f32(al[pb.gate_row(b, t, hv, APC ? DK : 1) + (APC ? c : 0)]) : 1.f;
+                bv[u] = in ? to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]) : 0.f;
             }
-            G *= av;
-            Eh[r * LD + c] = bv * kv * G;
-            Qh[r * LD + c] = qv * G;
-            Kt[r * LD + c] = kv / G;
-            if (save_bwd) gm[r * DK + c] = G;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = r0 + u;
+                G *= av[u];
+                Eh[r * LD + c] = bv[u] * kv[u] * G;
+                Qh[r * LD + c] = qv[u] * G;
+                Kt[r * LD + c] = kv[u] / G;
+                if (save_bwd) gm[r * DK + c] = G;
+            }
         }
         ws.gam[ci * DK + c] = G;
         for (int r = 0; r < C; ++r) {
@@ -176,10 +195,9 @@ chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int sav
     const TG* wg = static_cast<const TG*>(GPC ? io.w : io.b);
     const long soff = pb.state_off(b, hv);
 
-    for (int idx = tid; idx < DK * W; idx += kSimtThreads) {
-        const int c = idx / W, j = idx % W;
-        S[idx] = io.h0 ? io.h0[soff + (long)c * dv + j0 + j] : 0.f;
-    }
+    cta_load<DK * W>(
+        [&](int idx) { return io.h0 ? io.h0[soff + (long)(idx / W) * dv + j0 + idx % W] : 0.f; },
+        [&](int idx, float v) { S[idx] = v; });
 
     using GCW = BlockGemm<C, W, kSimtThreads, 16>;   // [C x 32] outputs
     using GKW = BlockGemm<DK, W, kSimtThreads, 16>;  // [DK x 32] outputs
@@ -193,17 +211,14 @@ chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int sav
         const float* Pm = ws.P + ci * C * C;
         const float* gam = ws.gam + ci * DK;
         __syncthreads();
-        for (int idx = tid; idx < C * W; idx += kSimtThreads) {
-            const int r = idx / W, j = idx % W;
-            float zv = 0.f;
-            if (r < L) {
-                const int t = t0 + r;
-                const float vv = to_f32(vin[pb.v_row(b, t, hv) + j0 + j]);
-                const float ww = to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
-                zv = vv * ww;
-            }
-            Z[idx] = zv;
-        }
+        cta_load<C * W>(
+            [&](int idx) {
+                const int r = idx / W, j = idx % W, t = t0 + r;
+                if (r >= L) return 0.f;
+                return to_f32(vin[pb.v_row(b, t, hv) + j0 + j]) *
+                       to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
+            },
+            [&](int idx, float v) { Z[idx] = v; });
         if (save_states)
             for (int idx = tid; idx < DK * W; idx += kSimtThreads) {
                 const int c = idx / W, j = idx % W;
@@ -314,10 +329,9 @@ chunk_scan_bwd_kernel(Problem pb, ChunkIO io, ChunkWs ws) {
     const TG* wg = static_cast<const TG*>(GPC ? io.w : io.b);
     const long soff = pb.state_off(b, hv);
 
-    for (int idx = tid; idx < DK * W; idx += kSimtThreads) {
-        const int c = idx / W, j = idx % W;
-        dS[idx] = io.dht ? io.dht[soff + (long)c * dv + j0 + j] : 0.f;
-    }
+    cta_load<DK * W>(
+        [&](int idx) { return io.dht ? io.dht[soff + (long)(idx / W) * dv + j0 + idx % W] : 0.f; },
+        [&](int idx, float v) { dS[idx] = v; });
 
     using GCW = BlockGemm<C, W, kSimtThreads, 16>;
     using GKW = BlockGemm<DK, W, kSimtThreads, 16>;
@@ -331,25 +345,27 @@ chunk_scan_bwd_kernel(Problem pb, ChunkIO io, ChunkWs ws) {
         const float* Pm = ws.P + ci * C * C;
         const float* gam = ws.gam + ci * DK;
         __syncthreads();
-        for (int idx = tid; idx < DK * W; idx += kSimtThreads) {
-            const int c = idx / W, j = idx % W;
-            const long off = ci * DK * dv + (long)c * dv + j0 + j;
-            ws.dSC[off] = dS[idx];
-            S0[idx] = ws.S0[off];
-        }
-        for (int idx = tid; idx < C * W; idx += kSimtThreads) {
-            const int r = idx / W, j = idx % W;
-            float zv = 0.f, go = 0.f;
-            if (r < L) {
-                const int t = t0 + r;
-                const long off = pb.v_row(b, t, hv) + j0 + j;
-                zv = to_f32(vin[off]) *
-                     to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
-                go = pb.scale * to_f32(gout[off]);
-            }
-            Z[idx] = zv;
-            dO[idx] = go;
-        }
+        cta_load<DK * W>(
+            [&](int idx) {
+                const long off = ci * DK * dv + (long)(idx / W) * dv + j0 + idx % W;
+                ws.dSC[off] = dS[idx];
+                return ws.S0[off];
+            },
+            [&](int idx, float v) { S0[idx] = v; });
+        cta_load<C * W>(
+            [&](int idx) {
+                const int r = idx / W, j = idx % W, t = t0 + r;
+                if (r >= L) return 0.f;
+                return to_f32(vin[pb.v_row(b, t, hv) + j0 + j]) *
+                       to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
+            },
+            [&](int idx, float v) { Z[idx] = v; });
+        cta_load<C * W>(
+            [&](int idx) {
+                const int r = idx / W, j = idx % W;
+                return r < L ? pb.scale * to_f32(gout[pb.v_row(b, t0 + r, hv) + j0 + j]) : 0.f;
+            },
+            [&](int idx, float v) { dO[idx] = v; });
         // Y = Z - Ehat S0 ; V' = T Y
         {
             GCW g;
@@ -490,10 +506,12 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
     const TG* al = static_cast<const TG*>(io.alpha);
     const TG* bg = static_cast<const TG*>(io.b);
 
-    for (int idx = tid; idx < C * DV; idx += kSimtThreads) {
-        const int r = idx / DV, j = idx % DV;
-        dO[r * LDV + j] = r < L ? pb.scale * to_f32(static_cast<const TIn*>(io.dout)[pb.v_row(b, t0 + r, hv) + j]) : 0.f;
-    }
+    cta_load<C * DV>(
+        [&](int idx) {
+            const int r = idx / DV, j = idx % DV;
+            return r < L ? pb.scale * to_f32(static_cast<const TIn*>(io.dout)[pb.v_row(b, t0 + r, hv) + j]) : 0.f;
+        },
+        [&](int idx, float v) { dO[(idx / DV) * LDV + idx % DV] = v; });
 
     using GCC = BlockGemm<C, C, kSimtThreads, 32>;
     {   // dP = lower(scale dO V'^T)
