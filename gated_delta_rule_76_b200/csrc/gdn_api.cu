@@ -307,9 +307,15 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_fwd");
 }
 
+static bool bwd_uses_tensor_cores(const gdn_bwd_args* a, const Problem& pb) {
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
+    return tc_fwd_eligible(pb, a->dtype == GDN_BF16, a->gate_dtype == GDN_BF16, f);
+}
+
 size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    if (bwd_uses_tensor_cores(a, pb)) return plan_tc_bwd_ws(pb, !identity_heads(pb)).bytes;
     return plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
 }
 
@@ -322,17 +328,23 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     if (a->T == 0) return copy_state(a->grad_h0, a->grad_ht, sbytes, st, "gdn_chunk_bwd");
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     const bool direct = identity_heads(pb);
+    const bool tc = bwd_uses_tensor_cores(a, pb);
     WsPlan plan = plan_chunk_ws(pb, true, !direct);
-    if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
+    TcBwdWs tplan = tc ? plan_tc_bwd_ws(pb, !direct) : TcBwdWs{};
+    if ((s = check_workspace(workspace, workspace_bytes, tc ? tplan.bytes : plan.bytes))) return s;
     ChunkIO io{};
     io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
     io.h0 = a->h0; io.dout = a->grad_o; io.dht = a->grad_ht; io.dq = a->grad_q; io.dk = a->grad_k;
     io.dv = a->grad_v; io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = a->grad_w;
     io.dh0 = a->grad_h0;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
-    ChunkWs ws = carve_chunk_ws(plan, workspace);
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_bwd");
+    if (tc) {
+        e = tc_chunk_bwd(pb, io, f, a->gate_dtype == GDN_BF16, direct, tplan, workspace, st);
+        return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_bwd");
+    }
+    ChunkWs ws = carve_chunk_ws(plan, workspace);
     switch (variant(a->dtype, a->gate_dtype)) {
         case 0: e = bf16_chunk_bwd(pb, io, ws, f, direct, st); break;
         case 1: e = bf16_f32g_chunk_bwd(pb, io, ws, f, direct, st); break;

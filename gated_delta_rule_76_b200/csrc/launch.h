@@ -38,10 +38,25 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
     cudaError_t NAME##_decode(const DecodeParams&, Flags, cudaStream_t);                       \
     cudaError_t NAME##_conv(const ConvParams&, cudaStream_t);
 
-// Tensor-core chunk forward (tc_fwd.cu): bf16 q/k/v with dk = dv = 128.
+// Tensor-core chunk forward (tc_fwd.cu): bf16 q/k/v with dk = dv = 128.  With `save`, the state
+// entering every chunk and V' of every token are written for the backward (o and ht may be NULL).
+struct TcFwdSave {
+    float* s0;               // [B*Hv][NT][dk][dv]
+    __nv_bfloat16* vp_hi;    // [B,T,Hv,dv]
+    __nv_bfloat16* vp_lo;
+};
 bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags f);
 cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
-                         cudaStream_t st);
+                         cudaStream_t st, const TcFwdSave* save = nullptr);
+
+// Tensor-core chunk backward (tc_bwd.cu): same eligibility as the forward, without z.
+struct TcBwdWs {
+    size_t bytes = 0;  // total, including the 256-byte status word at offset 0
+    size_t s0, dsc, vp_hi, vp_lo, ny_hi, ny_lo, dq_v, dk_v;  // byte offsets (dq_v, dk_v: GQA only)
+};
+TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials);
+cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, bool direct,
+                         const TcBwdWs& plan, void* ws, cudaStream_t st);
 
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates

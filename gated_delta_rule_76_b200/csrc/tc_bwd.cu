@@ -1,0 +1,158 @@
+// Host side of the tensor-core chunk backward: workspace plan, TMA descriptors, launches.
+// One call runs the forward kernel in saving mode, the reverse state-gradient scan, the
+// chunk-parallel gradient kernel and, when value heads share key heads, the GQA reduction.
+#include <cuda.h>
+
+#include "launch.cuh"
+#include "tc_chunk_bwd.cuh"
+#include "tma_host.h"
+
+namespace gdn {
+
+namespace {
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <bool APC, bool GPC, class TG>
+cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cudaStream_t st) {
+    auto kernel = tcbwd::scan::chunk_bwd_scan_kernel<APC, GPC, TG>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcbwd::scan::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kernel<<<p.pb.B * p.pb.Hv, tcbwd::scan::kThreads, tcbwd::scan::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                                    p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <bool APC, bool GPC, class TG>
+cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cudaStream_t st) {
+    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcbwd::grad::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long nch = (long)p.pb.B * p.pb.Hv * p.pb.NT;
+    kernel<<<(unsigned)nch, tcbwd::grad::kThreads, tcbwd::grad::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                                 m[5], m[6], m[7], m[8], p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <bool APC, bool GPC, class TG>
+cudaError_t launch_both(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
+                        const tcbwd::grad::Params& gp, cudaStream_t st) {
+    cudaError_t e = launch_scan<APC, GPC, TG>(ms, sp, st);
+    if (e != cudaSuccess) return e;
+    return launch_grad<APC, GPC, TG>(mg, gp, st);
+}
+
+}  // namespace
+
+TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials) {
+    TcBwdWs w;
+    const size_t nch = (size_t)pb.B * pb.Hv * pb.NT;
+    const size_t st = nch * pb.dk * pb.dv * sizeof(float);
+    const size_t tok = (size_t)pb.B * pb.T * pb.Hv * pb.dv * 2;
+    const size_t part = (size_t)pb.B * pb.T * pb.Hv * pb.dk * sizeof(float);
+    size_t off = 256;  // bytes [0, 256): device status word
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = al256(off + bytes);
+        return o;
+    };
+    w.s0 = take(st);
+    w.dsc = take(st);
+    w.vp_hi = take(tok);
+    w.vp_lo = take(tok);
+    w.ny_hi = take(tok);
+    w.ny_lo = take(tok);
+    w.dq_v = gqa_partials ? take(part) : ~size_t(0);
+    w.dk_v = gqa_partials ? take(part) : ~size_t(0);
+    w.bytes = off;
+    return w;
+}
+
+cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, bool direct,
+                         const TcBwdWs& plan, void* ws, cudaStream_t st) {
+    char* base = static_cast<char*>(ws);
+    int* err = static_cast<int*>(ws);
+    float* s0 = reinterpret_cast<float*>(base + plan.s0);
+    float* dsc = reinterpret_cast<float*>(base + plan.dsc);
+    auto* vph = reinterpret_cast<__nv_bfloat16*>(base + plan.vp_hi);
+    auto* vpl = reinterpret_cast<__nv_bfloat16*>(base + plan.vp_lo);
+    auto* nyh = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_hi);
+    auto* nyl = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_lo);
+    float* dq_v = direct ? static_cast<float*>(io.dq) : reinterpret_cast<float*>(base + plan.dq_v);
+    float* dk_v = direct ? static_cast<float*>(io.dk) : reinterpret_cast<float*>(base + plan.dk_v);
+
+    // 1. forward in saving mode (no output, no final state)
+    ChunkIO fio = io;
+    fio.o = nullptr;
+    fio.ht = nullptr;
+    fio.z = nullptr;
+    Flags ff = f;
+    ff.gate = false;
+    const TcFwdSave save{s0, vph, vpl};
+    cudaError_t e = tc_chunk_fwd(pb, fio, ff, bf16_gates, err, st, &save);
+    if (e != cudaSuccess) return e;
+
+    // 2. maps: q, k, alpha, b, dO, -dY hi/lo, V' hi/lo (unused gate maps copy a valid one)
+    CUtensorMap m[9];
+    bool ok = make_map(&m[0], io.q, pb.B, pb.T, pb.Hk) && make_map(&m[1], io.k, pb.B, pb.T, pb.Hk) &&
+              make_map(&m[4], io.dout, pb.B, pb.T, pb.Hv) && make_map(&m[5], nyh, pb.B, pb.T, pb.Hv) &&
+              make_map(&m[6], nyl, pb.B, pb.T, pb.Hv) && make_map(&m[7], vph, pb.B, pb.T, pb.Hv) &&
+              make_map(&m[8], vpl, pb.B, pb.T, pb.Hv);
+    m[2] = m[4];
+    m[3] = m[4];
+    if (ok && f.apc) ok = make_map(&m[2], io.alpha, pb.B, pb.T, pb.Hv);
+    if (ok && f.gpc) ok = make_map(&m[3], io.b, pb.B, pb.T, pb.Hv);
+    if (!ok) return cudaErrorInvalidValue;
+    const CUtensorMap ms[5] = {m[0], m[1], m[2], m[3], m[4]};
+
+    tcbwd::scan::Params sp{};
+    sp.pb = pb;
+    sp.alpha = io.alpha;
+    sp.b = io.b;
+    sp.dht = io.dht;
+    sp.dh0 = io.dh0;
+    sp.dsc = dsc;
+    sp.ny_hi = nyh;
+    sp.ny_lo = nyl;
+    sp.err = err;
+
+    tcbwd::grad::Params gp{};
+    gp.pb = pb;
+    gp.alpha = io.alpha;
+    gp.b = io.b;
+    gp.w = io.w;
+    gp.q = static_cast<const __nv_bfloat16*>(io.q);
+    gp.k = static_cast<const __nv_bfloat16*>(io.k);
+    gp.v = static_cast<const __nv_bfloat16*>(io.v);
+    gp.s0 = s0;
+    gp.dsc = dsc;
+    gp.dq = dq_v;
+    gp.dk = dk_v;
+    gp.dv = static_cast<float*>(io.dv);
+    gp.dalpha = static_cast<float*>(io.dalpha);
+    gp.db = static_cast<float*>(io.db);
+    gp.dw = static_cast<float*>(io.dw);
+    gp.direct = direct ? 1 : 0;
+    gp.err = err;
+
+    if (f.apc && f.gpc) e = launch_both<true, true, __nv_bfloat16>(ms, sp, m, gp, st);
+    else if (f.apc) e = launch_both<true, false, __nv_bfloat16>(ms, sp, m, gp, st);
+    else if (f.gpc) e = launch_both<false, true, __nv_bfloat16>(ms, sp, m, gp, st);
+    else if (bf16_gates) e = launch_both<false, false, __nv_bfloat16>(ms, sp, m, gp, st);
+    else e = launch_both<false, false, float>(ms, sp, m, gp, st);
+    if (e != cudaSuccess || direct) return e;
+
+    // 3. GQA: sum the per-value-head dq, dk over the value heads of each key head
+    const long total = (long)pb.B * pb.T * pb.Hk * pb.dk;
+    const int blocks = (int)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
+    GDN_TRY(launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb, (const float*)dq_v,
+                          static_cast<float*>(io.dq)));
+    return launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb, (const float*)dk_v,
+                         static_cast<float*>(io.dk));
+}
+
+}  // namespace gdn

@@ -1,0 +1,1221 @@
+// Chunkwise backward on the 5th-generation tensor cores (sm_100a), dk = dv = 128, bf16 inputs.
+//
+// Reverse mode of the chunk form (Gated DeltaNet-2 summary, «Entraînement Parallèle Efficace par
+// Blocs» for the forward it differentiates, «Passage Arrière Conscient des Portes» for the gated
+// backward).  Per chunk, with the forward's factors Gamma, Ehat = (b.*k).*Gamma,
+// Qhat = scale q.*Gamma (the readout scale is folded into Qhat, hence into P), Ktil = k./Gamma,
+// Kbar = Ktil.*gamma, T = (I + A)^-1, P = lower(Qhat Ktil^T), W = T Ehat, and the forward's
+// V' = T (Z - Ehat S0):
+//   dV' = P^T dO + Kbar dS_end,   dY = T^T dV'   (dZ = dY: dv = w.*dY, dw = v.*dY)
+//   dS0 = Qhat^T dO - W^T dV' + Diag(gamma) dS_end          (= Qhat^T dO - Ehat^T dY + ...)
+//   dP = lower(dO V'^T),  dA = strict_lower(-dY V'^T)        (= -T^T (dV' Y^T) T^T)
+//   dQhat = dO S0^T + dP Ktil,   dEhat = -dY S0^T + dA Ktil
+//   dKtil = dA^T Ehat + dP^T Qhat,   dKbar = V' dS_end^T
+// and through the factors to q, k, b (e = b.*k) and the cumulative log decay, whose gradient is
+// a reverse cumulative sum over the chunk.  The derivative of gamma collects
+// sum_r dKbar.*Kbar + gamma .* rowsum(dS_end .* S0).
+//
+// Kernels of one backward call:
+//   1. the forward kernel (tc_chunk_fwd.cuh) in saving mode: the state entering every chunk
+//      (fp32) and V' of every token (bf16 hi/lo);
+//   2. chunk_bwd_scan_kernel (this file): one CTA per (batch, value head), chunks in reverse;
+//      the state gradient dS is carried in registers (thread j: column j), its chain per chunk
+//      is  XA = dO^T P + dS^T Kbar^T (= dV'^T)  ->  XC = dO^T Qhat - dV'^T W (= dS0^T without
+//      the decay term)  ->  dS = Diag(gamma) dS + XC^T;  off the chain it forms -dY^T = -dV'^T T.
+//      It saves dS_end of every chunk (fp32) and -dY of every token (bf16 hi/lo), and writes dh0;
+//   3. chunk_bwd_grad_kernel (this file): one CTA per chunk, every gradient of the chunk's inputs.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_chunk_fwd.cuh"
+#include "umma.cuh"
+
+namespace gdn {
+namespace tcbwd {
+
+using namespace gdn::tc;
+using tcfwd::bf;
+using tcfwd::Ctx;
+using tcfwd::fma4;
+using tcfwd::ld16;
+using tcfwd::ldf4;
+using tcfwd::solve_block_row;
+using tcfwd::split8;
+using tcfwd::split_pack;
+using tcfwd::st16;
+using tcfwd::tma4;
+using tcfwd::unpack8;
+using tcfwd::wait1;
+
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr int LDA = tcfwd::LDA;
+constexpr uint64_t kWaitNs = tcfwd::kWaitNs;
+
+// =========================================== scan ===========================================
+namespace scan {
+
+constexpr int kThreads = 384;
+
+// tensor memory columns
+constexpr uint32_t TM_X1 = 0;     // 64:  A (lanes 0-63), P (lanes 64-127) of the prologue's chunk
+constexpr uint32_t TM_XA = 64;    // 64:  dV'^T, then -dY^T
+constexpr uint32_t TM_XC = 128;   // 128: dO^T Qhat - dV'^T W
+constexpr uint32_t TM_DSH = 256;  // 64:  dS^T hi (bf16 pairs)
+constexpr uint32_t TM_DSL = 320;  // 64:  dS^T lo
+constexpr uint32_t TM_DVH = 384;  // 32:  -dV'^T hi
+constexpr uint32_t TM_DVL = 416;  // 32:  -dV'^T lo
+constexpr uint32_t TM_WT = 448;   // 64:  W^T = Ehat^T T^T of the prologue's chunk
+constexpr uint32_t TM_COLS = 512;
+
+// shared memory (1024-byte-aligned base; bf16 tiles with the 128-byte swizzle)
+constexpr uint32_t SM_RQB = 0;        // 32 KB [2][128]: TMA b (rows 0-63), q (64-127) -> [Ehat;Qhat] lo
+constexpr uint32_t SM_RK = 32768;     // 16 KB [2][64]: TMA k -> Ktil hi
+constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo
+constexpr uint32_t SM_EQ = 65536;     // 32 KB [2][128]: [Ehat;Qhat] hi
+constexpr uint32_t SM_KB = 98304;     // 32 KB: Kbar hi [2][64], Kbar lo [2][64] (token rows)
+constexpr uint32_t SM_P = 131072;     // 16 KB: P hi [1][64], P lo [1][64] (row s, columns r)
+constexpr uint32_t SM_T = 147456;     // 8 KB [1][64]: T (row r, columns s)
+constexpr uint32_t SM_WT = 155648;    // 32 KB: W^T hi [1][128], W^T lo [1][128] (row c, columns r)
+constexpr uint32_t SM_DO = 188416;    // 16 KB: dO, two boxes of 64 channels x 64 tokens
+constexpr uint32_t SM_ASCR = 204800;  // 17 KB: A, then T, fp32 [64][LDA]
+constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats
+constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, flags
+constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: row-group products, then solve block rows
+constexpr uint32_t SM_END = SM_RS + 4096;
+constexpr size_t kSmemBytes = SM_END + 1024;
+
+enum Bar {
+    B_RAW = 0,   // q, k, alpha, b of the prologue's chunk landed
+    B_DO,        // dO of the scan's chunk landed
+    B_X1,        // X1 complete
+    B_WT,        // W^T complete
+    B_PREADY,    // prologue -> scan: P, Kbar, [Ehat;Qhat] written
+    B_WREADY,    // prologue -> scan: T, W^T written
+    B_XA,        // XA complete
+    B_XCPRE,     // dO^T Qhat complete: [Ehat;Qhat] and dO may be overwritten
+    B_XC,        // XC complete
+    B_DY,        // -dY^T complete: T and W^T may be overwritten
+    B_COUNT
+};
+
+struct Params {
+    Problem pb;
+    const void* alpha;     // scalar-gate reads
+    const void* b;
+    const float* dht;      // [B,Hv,dk,dv] or NULL
+    float* dh0;            // [B,Hv,dk,dv] or NULL
+    float* dsc;            // [B*Hv][NT][dk][dv]: dS_end of every chunk
+    __nv_bfloat16* ny_hi;  // [B,T,Hv,dv]: -dY of every token, hi / lo
+    __nv_bfloat16* ny_lo;
+    int* err;
+};
+
+
+template <bool APC, bool GPC>
+__device__ __forceinline__ void scan_load_raw(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
+                                         const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_) {
+    const int t0 = n * C;
+    const uint32_t base = smem_u32(cx.sm);
+    uint64_t* bar = cx.bars + B_RAW;
+    mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
+    tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);  // q -> rows 64-127
+    tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);
+    tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
+    tma4(base + SM_RK + 8192, tk, bar, 64, hk, t0, b);
+    if (GPC) {
+        tma4(base + SM_RQB, tb_, bar, 0, hv, t0, b);  // b -> rows 0-63
+        tma4(base + SM_RQB + 16384, tb_, bar, 64, hv, t0, b);
+    }
+    if (APC) {
+        tma4(base + SM_RA, ta, bar, 0, hv, t0, b);
+        tma4(base + SM_RA + 8192, ta, bar, 64, hv, t0, b);
+    }
+}
+
+__device__ __forceinline__ void scan_load_do(const Ctx& cx, int n, int b, int hv, const CUtensorMap* tdo) {
+    const uint32_t dst = smem_u32(cx.sm) + SM_DO;
+    uint64_t* bar = cx.bars + B_DO;
+    mbar_arrive_expect_tx(bar, 16384u);
+    tma4(dst, tdo, bar, 0, hv, n * C, b);
+    tma4(dst + 8192, tdo, bar, 64, hv, n * C, b);
+}
+
+template <bool APC, bool GPC, class TG>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_do, Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Ctx cx;
+    cx.sm = sm;
+    cx.bars = reinterpret_cast<uint64_t*>(sm + SM_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_BAR + 128);
+    cx.abort_flag = reinterpret_cast<volatile int*>(sm + SM_BAR + 132);
+    cx.err = p.err;
+    float* gam = reinterpret_cast<float*>(sm + SM_GAM);
+
+    const Problem& pb = p.pb;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int b = blockIdx.x / pb.Hv, hv = blockIdx.x % pb.Hv;
+    const int hk = pb.key_head(hv);
+    const int NT = pb.NT;
+    const uint32_t sbase = smem_u32(sm);
+
+    if (tid == 0) {
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(cx.bars + i, 1);
+        *cx.abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    // Chunks are processed in reverse: iteration i works on chunk NT - 1 - i.
+    int raw_issued = 0, do_issued = 0;  // meaningful in the issuing threads (256 and 0)
+    if (tid == 256) {
+        scan_load_raw<APC, GPC>(cx, NT - 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+        raw_issued = 1;
+    }
+    if (tid == 0) {
+        scan_load_do(cx, NT - 1, b, hv, &tm_do);
+        do_issued = 1;
+    }
+
+    if (warp < 8) {
+        // ================================ state-gradient scan ================================
+        const int j = tid & 127, h = tid >> 7;
+        volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 136);
+        const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+        const long soff = pb.state_off(b, hv);
+        const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
+        const uint32_t id_dop = idesc_bf16_f32_mn(128, 64, true, true);    // dO^T P
+        const uint32_t id_doq = idesc_bf16_f32_mn(128, 128, true, true);   // dO^T Qhat
+        const uint32_t id_dy = idesc_bf16_f32_mn(128, 64, false, true);    // (-dV'^T) T
+        float S[64];  // S[c'] = dS[64h + c'][j]
+#pragma unroll
+        for (int c = 0; c < 64; ++c) S[c] = p.dht ? p.dht[soff + (long)(64 * h + c) * D + j] : 0.f;
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) split_pack(S[32 * q2 + 2 * i], S[32 * q2 + 2 * i + 1], hi[i], lo[i]);
+            tmem_st16(tl + TM_DSH + 32 * h + 16 * q2, hi);
+            tmem_st16(tl + TM_DSL + 32 * h + 16 * q2, lo);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar(1, 256);
+
+        for (int i = 0; i < NT; ++i) {
+            const int n = NT - 1 - i;
+            const uint32_t pi = i & 1;
+            const int t0 = n * C, L = min(C, pb.T - t0);
+            // ---- XA = dS^T Kbar^T + dO^T P (= dV'^T);  XC = dO^T Qhat ----------------------------
+            if (tid == 0) {
+                tc_fence_after();
+                if (wait1(cx, B_PREADY, pi) && wait1(cx, B_DO, pi) && !*cx.abort_flag) {
+                    mma_ts_u<128, 64>(tbase + TM_XA, tbase + TM_DSH, sbase + SM_KB, id64, false);
+                    mma_ts_u<128, 64>(tbase + TM_XA, tbase + TM_DSL, sbase + SM_KB, id64, true);
+                    mma_ts_u<128, 64>(tbase + TM_XA, tbase + TM_DSH, sbase + SM_KB + 16384, id64, true);
+#pragma unroll
+                    for (int k = 0; k < 64; k += 16) {
+                        const uint64_t da = sdesc_mn_sw128(sbase + SM_DO + (uint32_t)k * 128u, 8192u);
+                        mma_ss(tbase + TM_XA, da, sdesc_mn_sw128(sbase + SM_P + (uint32_t)k * 128u, 8192u), id_dop, 1u);
+                        mma_ss(tbase + TM_XA, da, sdesc_mn_sw128(sbase + SM_P + 8192u + (uint32_t)k * 128u, 8192u),
+                               id_dop, 1u);
+                    }
+                    mma_commit(cx.bars + B_XA);
+#pragma unroll
+                    for (int k = 0; k < 64; k += 16) {
+                        const uint64_t da = sdesc_mn_sw128(sbase + SM_DO + (uint32_t)k * 128u, 8192u);
+                        mma_ss(tbase + TM_XC, da, sdesc_mn_sw128(sbase + SM_EQ + 8192u + (uint32_t)k * 128u, 16384u),
+                               id_doq, k > 0 ? 1u : 0u);
+                        mma_ss(tbase + TM_XC, da, sdesc_mn_sw128(sbase + SM_RQB + 8192u + (uint32_t)k * 128u, 16384u),
+                               id_doq, 1u);
+                    }
+                    mma_commit(cx.bars + B_XCPRE);
+                    wait1(cx, B_XA, pi);
+                }
+            }
+            named_bar(1, 256);
+            tc_fence_after();
+            // ---- -dV'^T, split, as the A operand of XC and -dY ------------------------------------
+            {
+                uint32_t r[32], hi[16], lo[16];
+                tmem_ld32(tl + TM_XA + 32 * h, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i2 = 0; i2 < 16; ++i2)
+                    split_pack(-__uint_as_float(r[2 * i2]), -__uint_as_float(r[2 * i2 + 1]), hi[i2], lo[i2]);
+                tmem_st16(tl + TM_DVH + 16 * h, hi);
+                tmem_st16(tl + TM_DVL + 16 * h, lo);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            named_bar(1, 256);
+            // ---- XC += (-dV'^T) W;  XA = (-dV'^T) T (= -dY^T);  next dO ----------------------------
+            if (tid == 0) {
+                tc_fence_after();
+                if (wait1(cx, B_WREADY, pi) && !*cx.abort_flag) {
+                    mma_ts_u<64, 128>(tbase + TM_XC, tbase + TM_DVH, sbase + SM_WT, id128, true);
+                    mma_ts_u<64, 128>(tbase + TM_XC, tbase + TM_DVL, sbase + SM_WT, id128, true);
+                    mma_ts_u<64, 128>(tbase + TM_XC, tbase + TM_DVH, sbase + SM_WT + 16384, id128, true);
+                    mma_commit(cx.bars + B_XC);
+#pragma unroll
+                    for (int k = 0; k < 64; k += 16) {
+                        const uint64_t dt = sdesc_mn_sw128(sbase + SM_T + (uint32_t)k * 128u, 8192u);
+                        mma_ts(tbase + TM_XA, tbase + TM_DVH + (uint32_t)(k >> 1), dt, id_dy, k > 0 ? 1u : 0u);
+                        mma_ts(tbase + TM_XA, tbase + TM_DVL + (uint32_t)(k >> 1), dt, id_dy, 1u);
+                    }
+                    mma_commit(cx.bars + B_DY);
+                }
+                if (do_issued < NT && wait1(cx, B_XCPRE, pi) && !*cx.abort_flag) {
+                    scan_load_do(cx, NT - 1 - do_issued, b, hv, &tm_do);
+                    ++do_issued;
+                }
+                wait1(cx, B_XC, pi);
+            }
+            if (p.dsc) {
+                // dS_end of chunk n, rows 64h .. 64h + 63 of column j (coalesced over j)
+                float* dst = p.dsc + ((long)blockIdx.x * NT + n) * (D * D) + (long)(64 * h) * D + j;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) dst[c * D] = S[c];
+            }
+            named_bar(1, 256);
+            tc_fence_after();
+            // ---- dS <- Diag(gamma) dS + XC^T; split for the next chunk ----------------------------
+            {
+                const float4* g4 = reinterpret_cast<const float4*>(gam + (i % 3) * 128 + 64 * h);
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    uint32_t r[32], hi[16], lo[16];
+                    tmem_ld32(tl + TM_XC + 64 * h + 32 * q2, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 g = g4[8 * q2 + i4];
+                        const int e = 32 * q2 + 4 * i4;
+                        S[e + 0] = fmaf(g.x, S[e + 0], __uint_as_float(r[4 * i4 + 0]));
+                        S[e + 1] = fmaf(g.y, S[e + 1], __uint_as_float(r[4 * i4 + 1]));
+                        S[e + 2] = fmaf(g.z, S[e + 2], __uint_as_float(r[4 * i4 + 2]));
+                        S[e + 3] = fmaf(g.w, S[e + 3], __uint_as_float(r[4 * i4 + 3]));
+                    }
+#pragma unroll
+                    for (int i2 = 0; i2 < 16; ++i2)
+                        split_pack(S[32 * q2 + 2 * i2], S[32 * q2 + 2 * i2 + 1], hi[i2], lo[i2]);
+                    tmem_st16(tl + TM_DSH + 32 * h + 16 * q2, hi);
+                    tmem_st16(tl + TM_DSL + 32 * h + 16 * q2, lo);
+                }
+                tmem_st_wait();
+            }
+            // ---- -dY of chunk n, token-major hi / lo ----------------------------------------------
+            if (tid == 0) {
+                tc_fence_after();
+                wait1(cx, B_DY, pi);
+            }
+            tc_fence_before();
+            named_bar(1, 256);
+            tc_fence_after();
+            {
+                uint32_t r[32];
+                tmem_ld32(tl + TM_XA + 32 * h, r);
+                tmem_ld_wait();
+                const long vrow = (long)pb.Hv * D;
+                const long vb = pb.v_row(b, t0 + 32 * h, hv) + j;
+                const int nrow = min(32, L - 32 * h);
+#pragma unroll
+                for (int ii = 0; ii < 32; ++ii) {
+                    if (ii < nrow) {
+                        const float x = __uint_as_float(r[ii]);
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                        p.ny_hi[vb + ii * vrow] = hi;
+                        p.ny_lo[vb + ii * vrow] = __float2bfloat16_rn(x - __bfloat162float(hi));
+                    }
+                }
+            }
+            if (tid == 0) *stop_slot = *cx.abort_flag;
+            tc_fence_before();
+            named_bar(1, 256);
+            if (*stop_slot) break;
+        }
+        if (p.dh0 && !*cx.abort_flag) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) p.dh0[soff + (long)(64 * h + c) * D + j] = S[c];
+        }
+    } else {
+        // ====================================== prologue ======================================
+        const int c = tid - 256;  // key channel; also the tensor-memory lane of X1 and W^T
+        volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 140);
+        const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+        const TG* alpha_g = static_cast<const TG*>(p.alpha);
+        const TG* beta_g = static_cast<const TG*>(p.b);
+        float* ascr = reinterpret_cast<float*>(sm + SM_ASCR);
+        float* rs = reinterpret_cast<float*>(sm + SM_RS);
+        uint8_t* RQB = sm + SM_RQB;
+        uint8_t* RK = sm + SM_RK;
+        uint8_t* RA = sm + SM_RA;
+        uint8_t* EQ = sm + SM_EQ;
+        uint8_t* KB = sm + SM_KB;
+        const uint32_t id64 = idesc_bf16_f32(128, 64);
+        const uint32_t id_wt = idesc_bf16_f32_mn(128, 64, true, false);  // Ehat^T (MN-major) x T
+        const float scale = pb.scale;
+        for (int i = 0; i < NT; ++i) {
+            const int n = NT - 1 - i;
+            const uint32_t pi = i & 1;
+            const int t0 = n * C, L = min(C, pb.T - t0);
+            if (c == 0) wait1(cx, B_RAW, pi);
+            named_bar(2, 128);
+            // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA), split Kbar -----
+            // Thread c: channels 8 cg .. 8 cg + 7 of rows 8 rg .. 8 rg + 7; Gamma over the chunk is
+            // the product of the row groups' products.
+            {
+                const int cg = c & 15, rg = c >> 4, r0 = 8 * rg;
+                const uint32_t a64 = (uint32_t)(cg >> 3) * 64u * 128u + (uint32_t)r0 * 128u;
+                const uint32_t a128 = (uint32_t)(cg >> 3) * 128u * 128u + (uint32_t)r0 * 128u;
+                const uint32_t ch = (uint32_t)(cg & 7);
+                float* part = rs;  // [8][128]
+                float Gl[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Gl[e] = 1.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = r0 + u;
+                    float a8[8];
+                    if (APC) {
+                        unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+                        if (r >= L) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) a8[e] = 1.f;
+                        }
+                    } else {
+                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) a8[e] = av;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) Gl[e] *= a8[e];
+                }
+                *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg) = make_float4(Gl[0], Gl[1], Gl[2], Gl[3]);
+                *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg + 4) = make_float4(Gl[4], Gl[5], Gl[6], Gl[7]);
+                named_bar(2, 128);
+                float G[8], gm[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) G[e] = gm[e] = 1.f;
+#pragma unroll
+                for (int g2 = 0; g2 < 8; ++g2) {
+                    const float4 p0 = ldf4(part + g2 * 128 + 8 * cg), p1 = ldf4(part + g2 * 128 + 8 * cg + 4);
+                    const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (g2 < rg) G[e] *= pv[e];
+                        gm[e] *= pv[e];
+                    }
+                }
+                if (rg == 0) {
+                    float* gs = gam + (i % 3) * 128 + 8 * cg;
+                    *reinterpret_cast<float4*>(gs) = make_float4(gm[0], gm[1], gm[2], gm[3]);
+                    *reinterpret_cast<float4*>(gs + 4) = make_float4(gm[4], gm[5], gm[6], gm[7]);
+                }
+#pragma unroll 2
+                for (int u = 0; u < 8; ++u) {
+                    const int r = r0 + u;
+                    const uint32_t sw = (ch ^ (uint32_t)u) << 4;
+                    const uint32_t o64 = a64 + u * 128u + sw, oe = a128 + u * 128u + sw, oq = oe + 64u * 128u;
+                    float a8[8], k8[8], q8[8], b8[8];
+                    if (APC) {
+                        unpack8(ld16(RA + o64), a8);
+                        if (r >= L) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) a8[e] = 1.f;
+                        }
+                    } else {
+                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) a8[e] = av;
+                    }
+                    unpack8(ld16(RK + o64), k8);
+                    unpack8(ld16(RQB + oq), q8);
+                    if (GPC) {
+                        unpack8(ld16(RQB + oe), b8);
+                    } else {
+                        const float bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) b8[e] = bv;
+                    }
+                    float e8[8], qq[8], kt[8], kb[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        G[e] *= a8[e];
+                        e8[e] = b8[e] * k8[e] * G[e];
+                        qq[e] = scale * q8[e] * G[e];
+                        kt[e] = __fdividef(k8[e], G[e]);
+                        kb[e] = kt[e] * gm[e];
+                    }
+                    uint4 hi, lo;
+                    split8(e8, hi, lo);
+                    st16(EQ + oe, hi);
+                    st16(RQB + oe, lo);
+                    split8(qq, hi, lo);
+                    st16(EQ + oq, hi);
+                    st16(RQB + oq, lo);
+                    split8(kt, hi, lo);
+                    st16(RK + o64, hi);
+                    st16(RA + o64, lo);
+                    split8(kb, hi, lo);
+                    st16(KB + o64, hi);
+                    st16(KB + 16384 + o64, lo);
+                }
+            }
+            fence_async_shared();
+            named_bar(2, 128);
+            // ---- X1 = [Ehat;Qhat] Ktil^T ----------------------------------------------------------
+            if (c == 0) {
+                tc_fence_after();
+                if (!*cx.abort_flag) {
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RK, id64, false);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RA, id64, true);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_RQB, sbase + SM_RK, id64, true);
+                    mma_commit(cx.bars + B_X1);
+                }
+                wait1(cx, B_X1, pi);
+            }
+            named_bar(2, 128);
+            tc_fence_after();
+            if (c < 64) {
+                // A row c (lanes 0-63), strictly lower, into the fp32 scratch.
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + TM_X1 + 32 * half, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const int s0 = 32 * half + 4 * q4;
+                        float4 v4;
+                        v4.x = s0 + 0 < c ? __uint_as_float(r[4 * q4 + 0]) : 0.f;
+                        v4.y = s0 + 1 < c ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
+                        v4.z = s0 + 2 < c ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
+                        v4.w = s0 + 3 < c ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
+                        *reinterpret_cast<float4*>(ascr + c * LDA + s0) = v4;
+                    }
+                }
+            } else {
+                // P row s = c - 64 (lanes 64-127), lower with the diagonal, split: row s, columns r.
+                const int rr = c - 64;
+                uint8_t* Ph = sm + SM_P;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + TM_X1 + 32 * half, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t wh[4], wl[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = 8 * ch + 2 * e, s0 = 32 * half + i0;
+                            const float x0 = s0 <= rr ? __uint_as_float(r[i0]) : 0.f;
+                            const float x1 = s0 + 1 <= rr ? __uint_as_float(r[i0 + 1]) : 0.f;
+                            split_pack(x0, x1, wh[e], wl[e]);
+                        }
+                        const uint32_t off = sw128_offset(rr, 32 * half + 8 * ch, 64);
+                        st16(Ph + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                        st16(Ph + 8192 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                    }
+                }
+            }
+            fence_async_shared();
+            tc_fence_before();
+            named_bar(2, 128);
+            if (c == 0) mbar_arrive(cx.bars + B_PREADY);
+            // ---- T = (I + A)^-1 by 16 x 16 blocks, in place in the fp32 scratch ------------------
+            if (c < 64) {
+                const int base = 16 * (c >> 4), jc = c & 15;
+                float x[16];
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) {
+                    const float* arow = ascr + (base + s2) * LDA + base;
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int u4 = 0; u4 < (s2 + 3) / 4; ++u4) {
+                        const float4 a4 = ldf4(arow + 4 * u4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int u = 4 * u4 + e;
+                            if (u < s2) {
+                                if (u & 1) a1 = fmaf(av[e], x[u], a1);
+                                else a0 = fmaf(av[e], x[u], a0);
+                            }
+                        }
+                    }
+                    x[s2] = s2 == jc ? 1.f : (s2 > jc ? -(a0 + a1) : 0.f);
+                }
+                named_bar(3, 64);
+#pragma unroll
+                for (int s2 = 0; s2 < 16; ++s2) ascr[(base + s2) * LDA + base + jc] = x[s2];
+            }
+            named_bar(2, 128);
+            solve_block_row<1>(ascr, rs, c);
+            solve_block_row<2>(ascr, rs, c);
+            solve_block_row<3>(ascr, rs, c);
+            // ---- T (fp32) -> bf16 tile once the scan has finished with the previous T and W^T ------
+            if (c == 0 && i > 0) wait1(cx, B_DY, pi ^ 1u);
+            named_bar(2, 128);
+            {
+                const int row = c & 63, col0 = 32 * (c >> 6);
+                uint8_t* Tt = sm + SM_T;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const float4 f0 = ldf4(ascr + row * LDA + col0 + 8 * q8);
+                    const float4 f1 = ldf4(ascr + row * LDA + col0 + 8 * q8 + 4);
+                    st16(Tt + sw128_offset(row, col0 + 8 * q8, 64),
+                         make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                                    pack_bf16x2(f1.z, f1.w)));
+                }
+            }
+            fence_async_shared();
+            named_bar(2, 128);
+            // ---- W^T = Ehat^T T^T; then the raw stage is free for the next chunk ------------------
+            if (c == 0) {
+                tc_fence_after();
+                if (!*cx.abort_flag) {
+#pragma unroll
+                    for (int k = 0; k < 64; k += 16) {
+                        const uint64_t dt = sdesc_k_sw128(sbase + SM_T + (uint32_t)k * 2u);
+                        mma_ss(tbase + TM_WT, sdesc_mn_sw128(sbase + SM_EQ + (uint32_t)k * 128u, 16384u), dt, id_wt,
+                               k > 0 ? 1u : 0u);
+                        mma_ss(tbase + TM_WT, sdesc_mn_sw128(sbase + SM_RQB + (uint32_t)k * 128u, 16384u), dt, id_wt, 1u);
+                    }
+                    mma_commit(cx.bars + B_WT);
+                }
+                wait1(cx, B_WT, pi);
+                if (raw_issued < NT && wait1(cx, B_XCPRE, pi) && !*cx.abort_flag) {
+                    scan_load_raw<APC, GPC>(cx, NT - 1 - raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                    ++raw_issued;
+                }
+            }
+            named_bar(2, 128);
+            tc_fence_after();
+            {
+                // W^T row c, split: row c, columns r (K-major B operand of XC).
+                uint8_t* WT = sm + SM_WT;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + TM_WT + 32 * half, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t wh[4], wl[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = 8 * ch + 2 * e;
+                            split_pack(__uint_as_float(r[i0]), __uint_as_float(r[i0 + 1]), wh[e], wl[e]);
+                        }
+                        const uint32_t off = sw128_offset(c, 32 * half + 8 * ch, 128);
+                        st16(WT + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                        st16(WT + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                    }
+                }
+            }
+            fence_async_shared();
+            tc_fence_before();
+            named_bar(2, 128);
+            if (c == 0) {
+                mbar_arrive(cx.bars + B_WREADY);
+                *stop_slot = *cx.abort_flag;
+            }
+            named_bar(2, 128);
+            if (*stop_slot) break;
+        }
+    }
+
+    // ---- teardown: TMA loads still in flight after an abort are waited for (bounded) -----------
+    tc_fence_before();
+    __syncthreads();
+    if (*cx.abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        if (tid == 0 && do_issued > 0)
+            while (!mbar_try_wait(cx.bars + B_DO, (uint32_t)((do_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+            }
+        if (tid == 256 && raw_issued > 0)
+            while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) &&
+                   globaltimer_ns() - t0 < kWaitNs) {
+            }
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+}  // namespace scan
+
+// ======================================== gradients ========================================
+// One CTA per chunk (grid = B * Hv * NT, blockIdx.x = (b * Hv + hv) * NT + n), 256 threads.
+//   P6 = G V'^T,  G = [dO; -dY]                      -> [dP; dA] after the masks (lanes: rows)
+//   P7 = S0 G^T + Ktil^T [dP; dA]^T                  -> [dQhat^T | dEhat^T]   (lanes: channels)
+//   P8 = [Qhat^T | Ehat^T] [dP; dA]                  -> dKtil^T
+//   P9 = dS_end V'^T                                 -> dKbar^T
+// S0 and dS_end are A operands in tensor memory (lane c holds row c); every other operand is a
+// bf16 hi/lo pair of 128-byte-swizzled shared-memory tiles.  The epilogue thread of lane c walks
+// the tokens of its half of the chunk: the cumulative decay and the reverse cumulative sum of the
+// log-decay gradient are sequential per thread.
+namespace grad {
+
+constexpr int kThreads = 256;
+
+constexpr uint32_t TM_S0H = 0;    // 64: S0 hi (lane c, bf16 pairs along j)
+constexpr uint32_t TM_S0L = 64;   // 64: S0 lo
+constexpr uint32_t TM_DSH = 128;  // 64: dS_end hi
+constexpr uint32_t TM_DSL = 192;  // 64: dS_end lo
+constexpr uint32_t TM_P6 = 256;   // 64: P6 (lanes = rows of G), then P8
+constexpr uint32_t TM_P7 = 320;   // 128: P7
+constexpr uint32_t TM_P9 = 448;   // 64: P9
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t SM_RQB = 0;        // 32 KB [2][128]: TMA b (rows 0-63), q (64-127) -> [Ehat;Qhat] lo
+constexpr uint32_t SM_RK = 32768;     // 16 KB [2][64]: TMA k -> Ktil hi
+constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo
+constexpr uint32_t SM_EQ = 65536;     // 32 KB [2][128]: [Ehat;Qhat] hi
+constexpr uint32_t SM_GH = 98304;     // 32 KB [2][128]: dO (rows 0-63), -dY hi (rows 64-127)
+constexpr uint32_t SM_GL = 131072;    // 32 KB [2][128]: zeros (rows 0-63), -dY lo (rows 64-127)
+constexpr uint32_t SM_VP = 163840;    // 32 KB: V' hi [2][64], V' lo [2][64]
+constexpr uint32_t SM_DPA = 196608;   // 32 KB: [dP;dA] hi [1][128], lo [1][128]
+constexpr uint32_t SM_BAR = 229376;   // mbarriers, tensor memory base
+constexpr uint32_t SM_DBV = SM_BAR + 256;  // 64 floats: sum_j dY v per token (scalar beta)
+constexpr uint32_t SM_END = SM_DBV + 256;
+constexpr size_t kSmemBytes = SM_END + 1024;
+// epilogue exchange, in the [Ehat;Qhat] lo tile once the products are complete
+constexpr uint32_t SX_PROD = 0;      // [2][128] products of alpha over each half of the chunk
+constexpr uint32_t SX_PART = 1024;   // [128] lower half: sum_r gamma dKbar Ktil + gamma rowsum(dS .* S0)
+constexpr uint32_t SX_SUF = 1536;    // [128] upper half: sum of its log-decay gradients
+constexpr uint32_t SX_RED = 2048;    // [8][32] per-warp row sums (scalar gates)
+constexpr uint32_t SX_RED2 = 3072;   // [8][32]
+
+enum Bar { B_RAW = 0, B_GV, B_P6, B_P789, B_COUNT };
+
+struct Params {
+    Problem pb;
+    const void* alpha;   // global reads of the gates, q, k, v, w in the epilogue
+    const void* b;
+    const void* w;
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    const float* s0;     // [B*Hv][NT][dk][dv]
+    const float* dsc;    // [B*Hv][NT][dk][dv]
+    float* dq;           // [B,T,Hk,dk] (direct) or [B,T,Hv,dk] per value head
+    float* dk;
+    float* dv;           // [B,T,Hv,dv]
+    float* dalpha;
+    float* db;
+    float* dw;
+    int direct;          // dq, dk written per key head (no head sharing)
+    int* err;
+};
+
+template <bool APC, bool GPC>
+__device__ __forceinline__ void grad_load_all(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
+                                         const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_,
+                                         const CUtensorMap* tdo, const CUtensorMap* tyh, const CUtensorMap* tyl,
+                                         const CUtensorMap* tvh, const CUtensorMap* tvl) {
+    const int t0 = n * C;
+    const uint32_t base = smem_u32(cx.sm);
+    uint64_t* bar = cx.bars + B_RAW;
+    mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
+    tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);
+    tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);
+    tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
+    tma4(base + SM_RK + 8192, tk, bar, 64, hk, t0, b);
+    if (GPC) {
+        tma4(base + SM_RQB, tb_, bar, 0, hv, t0, b);
+        tma4(base + SM_RQB + 16384, tb_, bar, 64, hv, t0, b);
+    }
+    if (APC) {
+        tma4(base + SM_RA, ta, bar, 0, hv, t0, b);
+        tma4(base + SM_RA + 8192, ta, bar, 64, hv, t0, b);
+    }
+    bar = cx.bars + B_GV;
+    mbar_arrive_expect_tx(bar, 5u * 16384u);
+    tma4(base + SM_GH, tdo, bar, 0, hv, t0, b);
+    tma4(base + SM_GH + 16384, tdo, bar, 64, hv, t0, b);
+    tma4(base + SM_GH + 8192, tyh, bar, 0, hv, t0, b);
+    tma4(base + SM_GH + 16384 + 8192, tyh, bar, 64, hv, t0, b);
+    tma4(base + SM_GL + 8192, tyl, bar, 0, hv, t0, b);
+    tma4(base + SM_GL + 16384 + 8192, tyl, bar, 64, hv, t0, b);
+    tma4(base + SM_VP, tvh, bar, 0, hv, t0, b);
+    tma4(base + SM_VP + 8192, tvh, bar, 64, hv, t0, b);
+    tma4(base + SM_VP + 16384, tvl, bar, 0, hv, t0, b);
+    tma4(base + SM_VP + 16384 + 8192, tvl, bar, 64, hv, t0, b);
+}
+
+// Sum of v over the 32 lanes of a warp.
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <bool APC, bool GPC, class TG>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_yh,
+                      const __grid_constant__ CUtensorMap tm_yl, const __grid_constant__ CUtensorMap tm_vh,
+                      const __grid_constant__ CUtensorMap tm_vl, Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Ctx cx;
+    cx.sm = sm;
+    cx.bars = reinterpret_cast<uint64_t*>(sm + SM_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_BAR + 128);
+    cx.abort_flag = reinterpret_cast<volatile int*>(sm + SM_BAR + 132);
+    cx.err = p.err;
+
+    const Problem& pb = p.pb;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const long ci = blockIdx.x;  // (b * Hv + hv) * NT + n
+    const int n = (int)(ci % pb.NT);
+    const int bh = (int)(ci / pb.NT);
+    const int b = bh / pb.Hv, hv = bh % pb.Hv;
+    const int hk = pb.key_head(hv);
+    const int t0 = n * C, L = min(C, pb.T - t0);
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t tl_lane = (uint32_t)((warp & 3) * 32) << 16;
+
+    if (tid == 0) {
+        for (int i = 0; i < B_COUNT; ++i) mbar_init(cx.bars + i, 1);
+        *cx.abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + tl_lane;
+    if (tid == 0)
+        grad_load_all<APC, GPC>(cx, n, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b, &tm_do, &tm_yh, &tm_yl, &tm_vh, &tm_vl);
+    {
+        // zero rows 0-63 of the G lo tile (dO is exact in bf16)
+        uint8_t* gl = sm + SM_GL;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx = tid + u * kThreads;  // 1024 chunks of 16 bytes: 2 atoms x 512
+            st16(gl + (uint32_t)(idx >> 9) * 16384u + (uint32_t)(idx & 511) * 16u, make_uint4(0u, 0u, 0u, 0u));
+        }
+    }
+
+    float dot_c = 0.f;  // lanes c (warps 0-3): sum_j dS_end[c][j] S0[c][j]
+    if (warp < 4) {
+        // ---- S0 and dS_end rows into tensor memory (split), row dot product ------------------
+        const int c = tid;
+        const float4* s0r = reinterpret_cast<const float4*>(p.s0 + (ci * D + c) * D);
+        const float4* dsr = reinterpret_cast<const float4*>(p.dsc + (ci * D + c) * D);
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float4 a[8], d[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                a[u] = s0r[8 * q4 + u];
+                d[u] = dsr[8 * q4 + u];
+            }
+            uint32_t ah[16], al[16], dh[16], dl[16];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                dot_c = fmaf(d[u].x, a[u].x, dot_c);
+                dot_c = fmaf(d[u].y, a[u].y, dot_c);
+                dot_c = fmaf(d[u].z, a[u].z, dot_c);
+                dot_c = fmaf(d[u].w, a[u].w, dot_c);
+                split_pack(a[u].x, a[u].y, ah[2 * u], al[2 * u]);
+                split_pack(a[u].z, a[u].w, ah[2 * u + 1], al[2 * u + 1]);
+                split_pack(d[u].x, d[u].y, dh[2 * u], dl[2 * u]);
+                split_pack(d[u].z, d[u].w, dh[2 * u + 1], dl[2 * u + 1]);
+            }
+            tmem_st16(tl + TM_S0H + 16 * q4, ah);
+            tmem_st16(tl + TM_S0L + 16 * q4, al);
+            tmem_st16(tl + TM_DSH + 16 * q4, dh);
+            tmem_st16(tl + TM_DSL + 16 * q4, dl);
+        }
+        tmem_st_wait();
+    } else {
+        // ---- cumulative decay; split [Ehat;Qhat], Ktil ----------------------------------------
+        const int c = tid - 128;
+        if (c == 0) wait1(cx, B_RAW, 0);
+        named_bar(2, 128);
+        const TG* alpha_g = static_cast<const TG*>(p.alpha);
+        const TG* beta_g = static_cast<const TG*>(p.b);
+        uint8_t* RQB = sm + SM_RQB;
+        uint8_t* RK = sm + SM_RK;
+        uint8_t* RA = sm + SM_RA;
+        uint8_t* EQ = sm + SM_EQ;
+        float* part = reinterpret_cast<float*>(sm + SM_DPA);  // [8][128], before [dP;dA] is written
+        const float scale = pb.scale;
+        const int cg = c & 15, rg = c >> 4, r0 = 8 * rg;
+        const uint32_t a64 = (uint32_t)(cg >> 3) * 64u * 128u + (uint32_t)r0 * 128u;
+        const uint32_t a128 = (uint32_t)(cg >> 3) * 128u * 128u + (uint32_t)r0 * 128u;
+        const uint32_t ch = (uint32_t)(cg & 7);
+        float Gl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) Gl[e] = 1.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int r = r0 + u;
+            float a8[8];
+            if (APC) {
+                unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+                if (r >= L) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a8[e] = 1.f;
+                }
+            } else {
+                const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a8[e] = av;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) Gl[e] *= a8[e];
+        }
+        *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg) = make_float4(Gl[0], Gl[1], Gl[2], Gl[3]);
+        *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg + 4) = make_float4(Gl[4], Gl[5], Gl[6], Gl[7]);
+        named_bar(2, 128);
+        float G[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) G[e] = 1.f;
+#pragma unroll
+        for (int g2 = 0; g2 < 8; ++g2) {
+            if (g2 < rg) {
+                const float4 p0 = ldf4(part + g2 * 128 + 8 * cg), p1 = ldf4(part + g2 * 128 + 8 * cg + 4);
+                G[0] *= p0.x; G[1] *= p0.y; G[2] *= p0.z; G[3] *= p0.w;
+                G[4] *= p1.x; G[5] *= p1.y; G[6] *= p1.z; G[7] *= p1.w;
+            }
+        }
+#pragma unroll 2
+        for (int u = 0; u < 8; ++u) {
+            const int r = r0 + u;
+            const uint32_t sw = (ch ^ (uint32_t)u) << 4;
+            const uint32_t o64 = a64 + u * 128u + sw, oe = a128 + u * 128u + sw, oq = oe + 64u * 128u;
+            float a8[8], k8[8], q8[8], b8[8];
+            if (APC) {
+                unpack8(ld16(RA + o64), a8);
+                if (r >= L) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a8[e] = 1.f;
+                }
+            } else {
+                const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a8[e] = av;
+            }
+            unpack8(ld16(RK + o64), k8);
+            unpack8(ld16(RQB + oq), q8);
+            if (GPC) {
+                unpack8(ld16(RQB + oe), b8);
+            } else {
+                const float bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) b8[e] = bv;
+            }
+            float e8[8], qq[8], kt[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                G[e] *= a8[e];
+                e8[e] = b8[e] * k8[e] * G[e];
+                qq[e] = scale * q8[e] * G[e];
+                kt[e] = __fdividef(k8[e], G[e]);
+            }
+            uint4 hi, lo;
+            split8(e8, hi, lo);
+            st16(EQ + oe, hi);
+            st16(RQB + oe, lo);
+            split8(qq, hi, lo);
+            st16(EQ + oq, hi);
+            st16(RQB + oq, lo);
+            split8(kt, hi, lo);
+            st16(RK + o64, hi);
+            st16(RA + o64, lo);
+        }
+    }
+    fence_async_shared();
+    tc_fence_before();
+    __syncthreads();
+    // ---- P6 = G V'^T ----------------------------------------------------------------------------
+    if (tid == 0) {
+        tc_fence_after();
+        if (wait1(cx, B_GV, 0) && !*cx.abort_flag) {
+            const uint32_t id64 = idesc_bf16_f32(128, 64);
+            mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP, id64, false);
+            mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GL, sbase + SM_VP, id64, true);
+            mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP + 16384, id64, true);
+            mma_commit(cx.bars + B_P6);
+            wait1(cx, B_P6, 0);
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    const bool ok = !*cx.abort_flag;
+    if (warp < 4) {
+        // ---- [dP; dA]: row r' of P6, masked (dP: s <= r', dA: s < r' - 64), split -------------
+        if (ok) {
+            const int rp = tid;
+            const int lim = rp < 64 ? rp : rp - 65;  // keep s <= lim
+            uint8_t* dpa = sm + SM_DPA;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[32];
+                tmem_ld32(tl + TM_P6 + 32 * half, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t wh[4], wl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i0 = 8 * ch + 2 * e, s0 = 32 * half + i0;
+                        const float x0 = s0 <= lim ? __uint_as_float(r[i0]) : 0.f;
+                        const float x1 = s0 + 1 <= lim ? __uint_as_float(r[i0 + 1]) : 0.f;
+                        split_pack(x0, x1, wh[e], wl[e]);
+                    }
+                    const uint32_t off = sw128_offset(rp, 32 * half + 8 * ch, 128);
+                    st16(dpa + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                    st16(dpa + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                }
+            }
+        }
+    } else {
+        // ---- dv = w .* dY, dw = v .* dY (or sum_j v dY for a scalar beta) -----------------------
+        const int tt = tid - 128, r = tt >> 1, jh = tt & 1;
+        float* dbv = reinterpret_cast<float*>(sm + SM_DBV);
+        float bsum = 0.f;
+        if (r < L) {
+            const long row = pb.v_row(b, t0 + r, hv);
+            const uint8_t* gh = sm + SM_GH;
+            const uint8_t* gl = sm + SM_GL;
+            float bscal = 0.f;
+            if (!GPC) bscal = to_f32(static_cast<const TG*>(p.b)[pb.gate_row(b, t0 + r, hv, 1)]);
+#pragma unroll 2
+            for (int cc = 0; cc < 8; ++cc) {
+                const int j = 64 * jh + 8 * cc;
+                const uint32_t off = sw128_offset(64 + r, j, 128);
+                float yh[8], yl[8], v8[8], w8[8];
+                unpack8(ld16(gh + off), yh);
+                unpack8(ld16(gl + off), yl);
+                unpack8(*reinterpret_cast<const uint4*>(p.v + row + j), v8);
+                if (GPC) unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.w) + row + j), w8);
+                float dvv[8], dww[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float dy = -(yh[e] + yl[e]);
+                    dvv[e] = (GPC ? w8[e] : bscal) * dy;
+                    dww[e] = v8[e] * dy;
+                    if (!GPC) bsum = fmaf(v8[e], dy, bsum);
+                }
+                float4* dvp = reinterpret_cast<float4*>(p.dv + row + j);
+                dvp[0] = make_float4(dvv[0], dvv[1], dvv[2], dvv[3]);
+                dvp[1] = make_float4(dvv[4], dvv[5], dvv[6], dvv[7]);
+                if (GPC) {
+                    float4* dwp = reinterpret_cast<float4*>(p.dw + row + j);
+                    dwp[0] = make_float4(dww[0], dww[1], dww[2], dww[3]);
+                    dwp[1] = make_float4(dww[4], dww[5], dww[6], dww[7]);
+                }
+            }
+        }
+        if (!GPC) {
+            bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
+            if (jh == 0) dbv[r] = bsum;
+        }
+    }
+    fence_async_shared();
+    tc_fence_before();
+    __syncthreads();
+    // ---- P7 = S0 G^T + Ktil^T [dP;dA]^T,  P8 = [Qhat^T|Ehat^T] [dP;dA],  P9 = dS V'^T --------------
+    if (tid == 0) {
+        tc_fence_after();
+        if (ok) {
+            const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
+            mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0H, sbase + SM_GH, id128, false);
+            mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0L, sbase + SM_GH, id128, true);
+            mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0H, sbase + SM_GL, id128, true);
+            const uint32_t id_kt = idesc_bf16_f32_mn(128, 128, true, false);
+#pragma unroll
+            for (int k = 0; k < 64; k += 16) {
+                const uint64_t akh = sdesc_mn_sw128(sbase + SM_RK + (uint32_t)k * 128u, 8192u);
+                const uint64_t akl = sdesc_mn_sw128(sbase + SM_RA + (uint32_t)k * 128u, 8192u);
+                const uint64_t bdh = sdesc_k_sw128(sbase + SM_DPA + (uint32_t)k * 2u);
+                const uint64_t bdl = sdesc_k_sw128(sbase + SM_DPA + 16384u + (uint32_t)k * 2u);
+                mma_ss(tbase + TM_P7, akh, bdh, id_kt, 1u);
+                mma_ss(tbase + TM_P7, akl, bdh, id_kt, 1u);
+                mma_ss(tbase + TM_P7, akh, bdl, id_kt, 1u);
+            }
+            const uint32_t id_k8 = idesc_bf16_f32_mn(128, 64, true, true);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t s0 = 16u * (uint32_t)kk;
+                const uint32_t arow = s0 < 64u ? 64u + s0 : s0 - 64u;  // Qhat rows, then Ehat rows
+                const uint64_t ah = sdesc_mn_sw128(sbase + SM_EQ + arow * 128u, 16384u);
+                const uint64_t al = sdesc_mn_sw128(sbase + SM_RQB + arow * 128u, 16384u);
+                const uint64_t bh_ = sdesc_mn_sw128(sbase + SM_DPA + s0 * 128u, 8192u);
+                const uint64_t bl_ = sdesc_mn_sw128(sbase + SM_DPA + 16384u + s0 * 128u, 8192u);
+                mma_ss(tbase + TM_P6, ah, bh_, id_k8, kk > 0 ? 1u : 0u);
+                mma_ss(tbase + TM_P6, al, bh_, id_k8, 1u);
+                mma_ss(tbase + TM_P6, ah, bl_, id_k8, 1u);
+            }
+            mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSH, sbase + SM_VP, id64, false);
+            mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSL, sbase + SM_VP, id64, true);
+            mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSH, sbase + SM_VP + 16384, id64, true);
+            mma_commit(cx.bars + B_P789);
+            wait1(cx, B_P789, 0);
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    // ---- epilogue: lane c, tokens 32 half .. 32 half + 31 ------------------------------------------
+    if (!*cx.abort_flag) {
+        const int c = tid & 127, half = tid >> 7;
+        float* X = reinterpret_cast<float*>(sm + SM_RQB);
+        const float* dbv = reinterpret_cast<const float*>(sm + SM_DBV);
+        const TG* alpha_g = static_cast<const TG*>(p.alpha);
+        const TG* b_g = static_cast<const TG*>(p.b);
+        const float scale = pb.scale;
+        float al[32];
+        float prod = 1.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int r = 32 * half + i;
+            float a = 1.f;
+            if (r < L) a = APC ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, D) + c])
+                               : to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]);
+            al[i] = a;
+            prod *= a;
+        }
+        X[SX_PROD / 4 + half * 128 + c] = prod;
+        __syncthreads();
+        const float pL = X[SX_PROD / 4 + c], pU = X[SX_PROD / 4 + 128 + c];
+        const float gam = pL * pU;
+        float G = half ? pL : 1.f;
+        float dg[32];
+        float part = 0.f;
+        float* red = X + SX_RED / 4;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+            uint32_t rq[16], re[16], rk[16], rb[16];
+            tmem_ld16(tl + TM_P7 + 32 * half + 16 * sub, rq);
+            tmem_ld16(tl + TM_P7 + 64 + 32 * half + 16 * sub, re);
+            tmem_ld16(tl + TM_P6 + 32 * half + 16 * sub, rk);
+            tmem_ld16(tl + TM_P9 + 32 * half + 16 * sub, rb);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int il = 16 * sub + i, r = 32 * half + il, t = t0 + r;
+                const bool in = r < L;
+                G *= al[il];
+                float qv = 0.f, kv = 0.f, bv = 0.f;
+                if (in) {
+                    const long qk = pb.qk_row(b, t, hk) + c;
+                    qv = __bfloat162float(p.q[qk]);
+                    kv = __bfloat162float(p.k[qk]);
+                    bv = GPC ? to_f32(b_g[pb.gate_row(b, t, hv, D) + c]) : to_f32(b_g[pb.gate_row(b, t, hv, 1)]);
+                }
+                const float Qh = scale * qv * G, Eh = bv * kv * G, Kt = __fdividef(kv, G);
+                const float dQh = __uint_as_float(rq[i]), dEh = __uint_as_float(re[i]);
+                const float dKb = __uint_as_float(rb[i]);
+                const float dkc = fmaf(gam, dKb, __uint_as_float(rk[i]));
+                const float de = G * dEh;
+                dg[il] = dQh * Qh + dEh * Eh - dkc * Kt;
+                part = fmaf(gam * dKb, Kt, part);
+                if (in) {
+                    const long o = p.direct ? pb.qk_row(b, t, hk) + c : pb.gate_row(b, t, hv, D) + c;
+                    p.dq[o] = scale * G * dQh;
+                    p.dk[o] = fmaf(de, bv, __fdividef(dkc, G));
+                    if (GPC) p.db[pb.gate_row(b, t, hv, D) + c] = de * kv;
+                }
+                if (!GPC) {
+                    const float s = warp_sum(de * kv);
+                    if ((tid & 31) == 0) red[warp * 32 + il] = s;
+                }
+            }
+        }
+        if (half == 0) X[SX_PART / 4 + c] = fmaf(gam, dot_c, part);
+        __syncthreads();
+        float* red2 = X + SX_RED2 / 4;
+        float run = 0.f;
+        if (half == 1) {
+            dg[31] += part + X[SX_PART / 4 + c];
+#pragma unroll
+            for (int il = 31; il >= 0; --il) {
+                run += dg[il];
+                const int r = 32 + il;
+                if (APC) {
+                    if (r < L) p.dalpha[pb.gate_row(b, t0 + r, hv, D) + c] = run / al[il];
+                } else {
+                    const float s = warp_sum(run);
+                    if ((tid & 31) == 0) red2[warp * 32 + il] = s;
+                }
+            }
+            X[SX_SUF / 4 + c] = run;
+        }
+        __syncthreads();
+        if (half == 0) {
+            run = X[SX_SUF / 4 + c];
+#pragma unroll
+            for (int il = 31; il >= 0; --il) {
+                run += dg[il];
+                const int r = il;
+                if (APC) {
+                    if (r < L) p.dalpha[pb.gate_row(b, t0 + r, hv, D) + c] = run / al[il];
+                } else {
+                    const float s = warp_sum(run);
+                    if ((tid & 31) == 0) red2[warp * 32 + il] = s;
+                }
+            }
+        }
+        if (!APC || !GPC) {
+            __syncthreads();
+            if (tid < 64) {
+                const int r = tid, hh = r >> 5, il = r & 31;
+                if (r < L) {
+                    const long g1 = pb.gate_row(b, t0 + r, hv, 1);
+                    if (!APC) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) s += red2[(4 * hh + w) * 32 + il];
+                        p.dalpha[g1] = s / to_f32(alpha_g[g1]);
+                    }
+                    if (!GPC) {
+                        float s = dbv[r];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) s += red[(4 * hh + w) * 32 + il];
+                        p.db[g1] = s;
+                    }
+                }
+            }
+        }
+    }
+    // ---- teardown ----------------------------------------------------------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (*cx.abort_flag && tid == 0) {
+        const uint64_t tw = globaltimer_ns();
+        while (!mbar_try_wait(cx.bars + B_RAW, 0) && globaltimer_ns() - tw < kWaitNs) {
+        }
+        while (!mbar_try_wait(cx.bars + B_GV, 0) && globaltimer_ns() - tw < kWaitNs) {
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+}  // namespace grad
+}  // namespace tcbwd
+}  // namespace gdn

@@ -120,6 +120,10 @@ struct Params {
     int o_type;  // 0: bf16, 1: fp32
     float* ht;
     int* err;    // device error word (bit 0: a bounded wait expired)
+    // Backward support (all NULL in a plain forward).  o may be NULL then: no output is formed.
+    float* s0_out;               // [B*Hv][NT][dk][dv] fp32: the state entering every chunk
+    __nv_bfloat16* vp_hi;        // [B,T,Hv,dv]: V' = T (Z - Ehat S0) of every token, split
+    __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
 };
 
 __device__ __forceinline__ float bf(const uint8_t* tile, uint32_t off) {
@@ -352,6 +356,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int n = 0; n < NT; ++n) {
             const uint32_t pn = n & 1;
             const int t0 = n * C, L = min(C, pb.T - t0);
+            if (p.s0_out) {
+                // state entering chunk n, rows 64h .. 64h + 63 of column j (coalesced over j)
+                float* dst = p.s0_out + ((long)blockIdx.x * NT + n) * (D * D) + (long)(64 * h) * D + j;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) dst[c * D] = S[c];
+            }
             // ---- X2 = S0^T [Ehat;Qhat]^T  (S0 split; Qhat split in the Qhat half) ------------------
             if (tid == 0) {
                 GDN_TRACE(n, 0);
@@ -489,6 +499,24 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     split_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), hi[i], lo[i]);
                 tmem_st16(tl + TM_YH + 16 * h, hi);
                 tmem_st16(tl + TM_YL + 16 * h, lo);
+                if (p.vp_hi) {
+                    // V' rows 32h .. 32h + 31 of column j, token-major (coalesced over j)
+                    const long vrow = (long)pb.Hv * D;
+                    const long vb = pb.v_row(b, t0 + 32 * h, hv) + j;
+                    const int nrow = min(32, L - 32 * h);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int r0 = 2 * i;
+                        if (r0 < nrow) {
+                            p.vp_hi[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(hi[i] & 0xFFFFu));
+                            p.vp_lo[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(lo[i] & 0xFFFFu));
+                        }
+                        if (r0 + 1 < nrow) {
+                            p.vp_hi[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(hi[i] >> 16));
+                            p.vp_lo[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(lo[i] >> 16));
+                        }
+                    }
+                }
                 tmem_st_wait();
             }
             tc_fence_before();
@@ -499,9 +527,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tc_fence_after();
                 if (!*cx.abort_flag) {
                     const uint32_t P = sbase + SM_P, KB = sbase + SM_KB;
-                    mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P, id64, true);
-                    mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YL, P, id64, true);
-                    mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P + 8192, id64, true);
+                    if (p.o) {
+                        mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P, id64, true);
+                        mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YL, P, id64, true);
+                        mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P + 8192, id64, true);
+                    }
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB, id128, false);
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YL, KB, id128, true);
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB + 16384, id128, true);
@@ -513,7 +543,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             named_bar(1, 256);
             tc_fence_after();
             // ---- output rows 32h .. 32h+31 of column j -----------------------------------------
-            {
+            if (p.o) {
                 uint32_t r[32];
                 tmem_ld32(tl + TM_X2 + 64 + 32 * h, r);
                 tmem_ld_wait();

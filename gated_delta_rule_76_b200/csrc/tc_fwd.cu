@@ -5,40 +5,11 @@
 
 #include "launch.h"
 #include "tc_chunk_fwd.cuh"
+#include "tma_host.h"
 
 namespace gdn {
 
 namespace {
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// [B, T, H, 128] bf16, boxes of 64 channels x 1 head x 64 tokens x 1 sequence, 128-byte swizzle.
-// Tokens past T are zero-filled by the hardware.
-bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn || !base) return false;
-    const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)T * H * 256};
-    const cuuint32_t box[4] = {64, 1, 64, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <bool APC, bool GPC, bool GATE, class TG>
 cudaError_t launch_tc(const CUtensorMap* maps, const tcfwd::Params& p, cudaStream_t st) {
@@ -66,7 +37,7 @@ bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags
 }
 
 cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
-                         cudaStream_t st) {
+                         cudaStream_t st, const TcFwdSave* save) {
     CUtensorMap maps[6];
     bool ok = make_map(&maps[0], io.q, pb.B, pb.T, pb.Hk) && make_map(&maps[1], io.k, pb.B, pb.T, pb.Hk) &&
               make_map(&maps[2], io.v, pb.B, pb.T, pb.Hv);
@@ -77,7 +48,7 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     if (ok && f.apc) ok = make_map(&maps[3], io.alpha, pb.B, pb.T, pb.Hv);
     if (ok && f.gpc) ok = make_map(&maps[4], io.b, pb.B, pb.T, pb.Hv) && make_map(&maps[5], io.w, pb.B, pb.T, pb.Hv);
     if (!ok) return cudaErrorInvalidValue;
-    tcfwd::Params p;
+    tcfwd::Params p{};
     p.pb = pb;
     p.alpha = io.alpha;
     p.b = io.b;
@@ -87,6 +58,11 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     p.o_type = io.o_type == 1 ? 1 : 0;
     p.ht = io.ht;
     p.err = err;
+    if (save) {
+        p.s0_out = save->s0;
+        p.vp_hi = save->vp_hi;
+        p.vp_lo = save->vp_lo;
+    }
     const bool gate = f.gate;
     if (f.apc && f.gpc) return launch_tc_g<true, true, __nv_bfloat16>(gate, maps, p, st);
     if (f.apc) return launch_tc_g<true, false, __nv_bfloat16>(gate, maps, p, st);
