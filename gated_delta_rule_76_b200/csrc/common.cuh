@@ -46,4 +46,15 @@ struct Problem {
     }
 };
 
+// Scalar gate of token t0 + r of value head hv (one value per token), or `fill` for a row r >= L
+// past the end of the sequence.  The load itself is unconditional, from the row clamped to the
+// last token: a load under a branch is waited for where the branch ends, which would serialise
+// the loads of an unrolled loop.
+template <class TG>
+__device__ __forceinline__ float gate_or(const TG* g, const Problem& pb, int b, int t0, int r, int L, int hv,
+                                         float fill) {
+    const float x = to_f32(__ldg(g + pb.gate_row(b, t0 + (r < L ? r : L - 1), hv, 1)));
+    return r < L ? x : fill;
+}
+
 }  // namespace gdn

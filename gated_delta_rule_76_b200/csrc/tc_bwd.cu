@@ -32,7 +32,10 @@ cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cuda
                                          (int)tcbwd::grad::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long nch = (long)p.pb.B * p.pb.Hv * p.pb.NT;
-    kernel<<<(unsigned)nch, tcbwd::grad::kThreads, tcbwd::grad::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const long grid = nch < nsm ? nch : nsm;  // persistent: one CTA per SM walks the chunks
+    kernel<<<(unsigned)grid, tcbwd::grad::kThreads, tcbwd::grad::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
                                                                                  m[5], m[6], m[7], m[8], p);
     count_launch();
     return cudaGetLastError();
@@ -52,6 +55,7 @@ TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials) {
     TcBwdWs w;
     const size_t nch = (size_t)pb.B * pb.Hv * pb.NT;
     const size_t st = nch * pb.dk * pb.dv * sizeof(float);
+    const size_t st1 = (size_t)pb.B * pb.Hv * (pb.NT + 1) * pb.dk * pb.dv * sizeof(float);
     const size_t tok = (size_t)pb.B * pb.T * pb.Hv * pb.dv * 2;
     const size_t part = (size_t)pb.B * pb.T * pb.Hv * pb.dk * sizeof(float);
     size_t off = 256;  // bytes [0, 256): device status word
@@ -60,7 +64,7 @@ TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials) {
         off = al256(off + bytes);
         return o;
     };
-    w.s0 = take(st);
+    w.s0 = take(st1);  // entering state of every chunk, then the final state
     w.dsc = take(st);
     w.vp_hi = take(tok);
     w.vp_lo = take(tok);
@@ -156,3 +160,10 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
 }
 
 }  // namespace gdn
+
+#ifdef GDN_BWD_TRACE
+// Profiling builds only: copy the phase timestamps of CTA 0 of the last gradient kernel to the host.
+extern "C" __attribute__((visibility("default"))) int gdn_bwd_trace_read(unsigned long long* host) {
+    return (int)cudaMemcpyFromSymbol(host, gdn::tcbwd::g_bwd_trace, sizeof(unsigned long long) * 16 * 16);
+}
+#endif

@@ -34,6 +34,20 @@
 namespace gdn {
 namespace tcbwd {
 
+// Optional phase timestamps of CTA 0 of the gradient kernel (compiled only with -DGDN_BWD_TRACE,
+// for profiling builds): g_bwd_trace[iteration][point] = %globaltimer.
+#ifdef GDN_BWD_TRACE
+__device__ unsigned long long g_bwd_trace[16][16];
+#define GDN_BTRACE(it, point)                                                            \
+    do {                                                                                 \
+        if (blockIdx.x == 0 && (it) < 16) g_bwd_trace[(it)][(point)] = globaltimer_ns(); \
+    } while (0)
+#else
+#define GDN_BTRACE(it, point) \
+    do {                      \
+    } while (0)
+#endif
+
 using namespace gdn::tc;
 using tcfwd::bf;
 using tcfwd::Ctx;
@@ -106,7 +120,7 @@ struct Params {
     const void* b;
     const float* dht;      // [B,Hv,dk,dv] or NULL
     float* dh0;            // [B,Hv,dk,dv] or NULL
-    float* dsc;            // [B*Hv][NT][dk][dv]: dS_end of every chunk
+    float* dsc;            // [B*Hv][NT][dv/4][dk][4]: dS_end of every chunk
     __nv_bfloat16* ny_hi;  // [B,T,Hv,dv]: -dY of every token, hi / lo
     __nv_bfloat16* ny_lo;
     int* err;
@@ -283,10 +297,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 wait1(cx, B_XC, pi);
             }
             if (p.dsc) {
-                // dS_end of chunk n, rows 64h .. 64h + 63 of column j (coalesced over j)
-                float* dst = p.dsc + ((long)blockIdx.x * NT + n) * (D * D) + (long)(64 * h) * D + j;
+                // dS_end of chunk n, rows 64h .. 64h + 63 of column j, layout [j / 4][row][j % 4]
+                float* dst = p.dsc + ((long)blockIdx.x * NT + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
 #pragma unroll
-                for (int c = 0; c < 64; ++c) dst[c * D] = S[c];
+                for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
             }
             named_bar(1, 256);
             tc_fence_after();
@@ -395,7 +409,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             for (int e = 0; e < 8; ++e) a8[e] = 1.f;
                         }
                     } else {
-                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a8[e] = av;
                     }
@@ -436,7 +450,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             for (int e = 0; e < 8; ++e) a8[e] = 1.f;
                         }
                     } else {
-                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a8[e] = av;
                     }
@@ -445,7 +459,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
                     } else {
-                        const float bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
+                        const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) b8[e] = bv;
                     }
@@ -659,15 +673,18 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 }  // namespace scan
 
 // ======================================== gradients ========================================
-// One CTA per chunk (grid = B * Hv * NT, blockIdx.x = (b * Hv + hv) * NT + n), 256 threads.
+// Persistent: one CTA per SM walks the chunks ci = blockIdx.x, blockIdx.x + gridDim.x, ...
+// (ci = (b * Hv + hv) * NT + n), 256 threads in two groups of four warps.  Per chunk:
 //   P6 = G V'^T,  G = [dO; -dY]                      -> [dP; dA] after the masks (lanes: rows)
 //   P7 = S0 G^T + Ktil^T [dP; dA]^T                  -> [dQhat^T | dEhat^T]   (lanes: channels)
 //   P8 = [Qhat^T | Ehat^T] [dP; dA]                  -> dKtil^T
 //   P9 = dS_end V'^T                                 -> dKbar^T
 // S0 and dS_end are A operands in tensor memory (lane c holds row c); every other operand is a
-// bf16 hi/lo pair of 128-byte-swizzled shared-memory tiles.  The epilogue thread of lane c walks
-// the tokens of its half of the chunk: the cumulative decay and the reverse cumulative sum of the
-// log-decay gradient are sequential per thread.
+// bf16 hi/lo pair of 128-byte-swizzled shared-memory tiles.  Once P7-P9 of chunk i are complete,
+// the epilogue group (warps 0-3, lane c = channel c) writes dv, dw and then every other gradient
+// of chunk i, walking the tokens from last to first so that the reverse cumulative sum of the
+// log-decay gradient is a running sum per thread, while the staging group (warps 4-7) loads
+// chunk i + 1: S0 and dS_end into tensor memory, the TMA tiles, the split factors.
 namespace grad {
 
 constexpr int kThreads = 256;
@@ -689,16 +706,17 @@ constexpr uint32_t SM_GH = 98304;     // 32 KB [2][128]: dO (rows 0-63), -dY hi 
 constexpr uint32_t SM_GL = 131072;    // 32 KB [2][128]: zeros (rows 0-63), -dY lo (rows 64-127)
 constexpr uint32_t SM_VP = 163840;    // 32 KB: V' hi [2][64], V' lo [2][64]
 constexpr uint32_t SM_DPA = 196608;   // 32 KB: [dP;dA] hi [1][128], lo [1][128]
-constexpr uint32_t SM_BAR = 229376;   // mbarriers, tensor memory base
-constexpr uint32_t SM_DBV = SM_BAR + 256;  // 64 floats: sum_j dY v per token (scalar beta)
-constexpr uint32_t SM_END = SM_DBV + 256;
+constexpr uint32_t SM_BAR = 229376;   // mbarriers, tensor memory base, flags
+constexpr uint32_t SM_XSLOT = SM_BAR + 256;   // [128] rowsum(dS_end .* S0) of the staged chunk
+constexpr uint32_t SM_GSLOT = SM_BAR + 768;   // [128] gamma (the chunk's total decay) of the staged chunk
+constexpr uint32_t SM_END = SM_BAR + 1280;
 constexpr size_t kSmemBytes = SM_END + 1024;
-// epilogue exchange, in the [Ehat;Qhat] lo tile once the products are complete
-constexpr uint32_t SX_PROD = 0;      // [2][128] products of alpha over each half of the chunk
-constexpr uint32_t SX_PART = 1024;   // [128] lower half: sum_r gamma dKbar Ktil + gamma rowsum(dS .* S0)
-constexpr uint32_t SX_SUF = 1536;    // [128] upper half: sum of its log-decay gradients
-constexpr uint32_t SX_RED = 2048;    // [8][32] per-warp row sums (scalar gates)
-constexpr uint32_t SX_RED2 = 3072;   // [8][32]
+// Epilogue scratch: the zero rows 0-63 of the G lo tile (first atom column, 8 KB) are free while
+// the epilogue runs; the epilogue zeroes what it used before the next chunk's P6.
+constexpr uint32_t SX_DBV = 0;      // [64] sum_j dY v per token (scalar beta)
+constexpr uint32_t SX_RA = 256;     // [4][64] per-warp sums over channels of d log alpha
+constexpr uint32_t SX_RB = 1280;    // [4][64] per-warp sums over channels of de .* k
+constexpr uint32_t SX_BYTES = 2304;
 
 enum Bar { B_RAW = 0, B_GV, B_P6, B_P789, B_COUNT };
 
@@ -710,8 +728,8 @@ struct Params {
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
-    const float* s0;     // [B*Hv][NT][dk][dv]
-    const float* dsc;    // [B*Hv][NT][dk][dv]
+    const float* s0;     // [B*Hv][NT][dv/4][dk][4]: row c, columns 4q..4q+3 at float4 (q * dk + c)
+    const float* dsc;    // same layout
     float* dq;           // [B,T,Hk,dk] (direct) or [B,T,Hv,dk] per value head
     float* dk;
     float* dv;           // [B,T,Hv,dv]
@@ -722,39 +740,61 @@ struct Params {
     int* err;
 };
 
+struct ChunkPos {
+    long ci;
+    int n, b, hv, hk, t0, L;
+};
+
+__device__ __forceinline__ ChunkPos chunk_pos(const Problem& pb, long ci) {
+    ChunkPos cp;
+    cp.ci = ci;
+    cp.n = (int)(ci % pb.NT);
+    const int bh = (int)(ci / pb.NT);
+    cp.b = bh / pb.Hv;
+    cp.hv = bh % pb.Hv;
+    cp.hk = pb.key_head(cp.hv);
+    cp.t0 = cp.n * C;
+    cp.L = min(C, pb.T - cp.t0);
+    return cp;
+}
+
+struct Maps {
+    const CUtensorMap *q, *k, *a, *b, *dO, *yh, *yl, *vh, *vl;
+};
+
 template <bool APC, bool GPC>
-__device__ __forceinline__ void grad_load_all(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
-                                         const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_,
-                                         const CUtensorMap* tdo, const CUtensorMap* tyh, const CUtensorMap* tyl,
-                                         const CUtensorMap* tvh, const CUtensorMap* tvl) {
-    const int t0 = n * C;
+__device__ __forceinline__ void load_raw_g(const Ctx& cx, const ChunkPos& cp, const Maps& m) {
     const uint32_t base = smem_u32(cx.sm);
     uint64_t* bar = cx.bars + B_RAW;
     mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
-    tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);
-    tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);
-    tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
-    tma4(base + SM_RK + 8192, tk, bar, 64, hk, t0, b);
+    tma4(base + SM_RQB + 8192, m.q, bar, 0, cp.hk, cp.t0, cp.b);
+    tma4(base + SM_RQB + 16384 + 8192, m.q, bar, 64, cp.hk, cp.t0, cp.b);
+    tma4(base + SM_RK, m.k, bar, 0, cp.hk, cp.t0, cp.b);
+    tma4(base + SM_RK + 8192, m.k, bar, 64, cp.hk, cp.t0, cp.b);
     if (GPC) {
-        tma4(base + SM_RQB, tb_, bar, 0, hv, t0, b);
-        tma4(base + SM_RQB + 16384, tb_, bar, 64, hv, t0, b);
+        tma4(base + SM_RQB, m.b, bar, 0, cp.hv, cp.t0, cp.b);
+        tma4(base + SM_RQB + 16384, m.b, bar, 64, cp.hv, cp.t0, cp.b);
     }
     if (APC) {
-        tma4(base + SM_RA, ta, bar, 0, hv, t0, b);
-        tma4(base + SM_RA + 8192, ta, bar, 64, hv, t0, b);
+        tma4(base + SM_RA, m.a, bar, 0, cp.hv, cp.t0, cp.b);
+        tma4(base + SM_RA + 8192, m.a, bar, 64, cp.hv, cp.t0, cp.b);
     }
-    bar = cx.bars + B_GV;
+}
+
+__device__ __forceinline__ void load_gv(const Ctx& cx, const ChunkPos& cp, const Maps& m) {
+    const uint32_t base = smem_u32(cx.sm);
+    uint64_t* bar = cx.bars + B_GV;
     mbar_arrive_expect_tx(bar, 5u * 16384u);
-    tma4(base + SM_GH, tdo, bar, 0, hv, t0, b);
-    tma4(base + SM_GH + 16384, tdo, bar, 64, hv, t0, b);
-    tma4(base + SM_GH + 8192, tyh, bar, 0, hv, t0, b);
-    tma4(base + SM_GH + 16384 + 8192, tyh, bar, 64, hv, t0, b);
-    tma4(base + SM_GL + 8192, tyl, bar, 0, hv, t0, b);
-    tma4(base + SM_GL + 16384 + 8192, tyl, bar, 64, hv, t0, b);
-    tma4(base + SM_VP, tvh, bar, 0, hv, t0, b);
-    tma4(base + SM_VP + 8192, tvh, bar, 64, hv, t0, b);
-    tma4(base + SM_VP + 16384, tvl, bar, 0, hv, t0, b);
-    tma4(base + SM_VP + 16384 + 8192, tvl, bar, 64, hv, t0, b);
+    tma4(base + SM_GH, m.dO, bar, 0, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_GH + 16384, m.dO, bar, 64, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_GH + 8192, m.yh, bar, 0, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_GH + 16384 + 8192, m.yh, bar, 64, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_GL + 8192, m.yl, bar, 0, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_GL + 16384 + 8192, m.yl, bar, 64, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_VP, m.vh, bar, 0, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_VP + 8192, m.vh, bar, 64, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_VP + 16384, m.vl, bar, 0, cp.hv, cp.t0, cp.b);
+    tma4(base + SM_VP + 16384 + 8192, m.vl, bar, 64, cp.hv, cp.t0, cp.b);
 }
 
 // Sum of v over the 32 lanes of a warp.
@@ -762,6 +802,392 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// Staging group (128 threads, c = lane = channel): S0 and dS_end rows of the chunk into tensor
+// memory as split A operands and rowsum(dS_end .* S0) into xslot[c]; then, once the raw TMA tiles
+// have landed, the cumulative decay (gamma into gslot[c]) and the split [Ehat;Qhat], Ktil tiles.
+template <bool APC, bool GPC, class TG>
+__device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, const ChunkPos& cp, uint32_t tl, int c,
+                                            float* xslot, float* gslot, uint32_t raw_parity, int it = 15) {
+    const Problem& pb = p.pb;
+    {
+        // row c: columns 4u .. 4u + 3 are the float4 u * D (coalesced over the group's rows)
+        const long bh = cp.ci / pb.NT;
+        const float4* s0r = reinterpret_cast<const float4*>(p.s0 + (bh * (pb.NT + 1) + cp.n) * D * D) + c;
+        const float4* dsr = reinterpret_cast<const float4*>(p.dsc + cp.ci * D * D) + c;
+        float dot = 0.f;
+#pragma unroll 1
+        for (int q8 = 0; q8 < 2; ++q8) {
+            float4 a[16], d[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                a[u] = __ldg(s0r + (16 * q8 + u) * D);
+                d[u] = __ldg(dsr + (16 * q8 + u) * D);
+            }
+#pragma unroll
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t ah[16], al[16], dh[16], dl[16];
+#pragma unroll
+                for (int u8 = 0; u8 < 8; ++u8) {
+                    const int u = 8 * hq + u8;
+                    dot = fmaf(d[u].x, a[u].x, dot);
+                    dot = fmaf(d[u].y, a[u].y, dot);
+                    dot = fmaf(d[u].z, a[u].z, dot);
+                    dot = fmaf(d[u].w, a[u].w, dot);
+                    split_pack(a[u].x, a[u].y, ah[2 * u8], al[2 * u8]);
+                    split_pack(a[u].z, a[u].w, ah[2 * u8 + 1], al[2 * u8 + 1]);
+                    split_pack(d[u].x, d[u].y, dh[2 * u8], dl[2 * u8]);
+                    split_pack(d[u].z, d[u].w, dh[2 * u8 + 1], dl[2 * u8 + 1]);
+                }
+                const int q4 = 2 * q8 + hq;
+                tmem_st16(tl + TM_S0H + 16 * q4, ah);
+                tmem_st16(tl + TM_S0L + 16 * q4, al);
+                tmem_st16(tl + TM_DSH + 16 * q4, dh);
+                tmem_st16(tl + TM_DSL + 16 * q4, dl);
+            }
+        }
+        xslot[c] = dot;
+        tmem_st_wait();
+    }
+    if (c == 0) wait1(cx, B_RAW, raw_parity);
+    if (c == 0) GDN_BTRACE(it, 7);
+    named_bar(2, 128);
+    const TG* alpha_g = static_cast<const TG*>(p.alpha);
+    const TG* beta_g = static_cast<const TG*>(p.b);
+    uint8_t* RQB = cx.sm + SM_RQB;
+    uint8_t* RK = cx.sm + SM_RK;
+    uint8_t* RA = cx.sm + SM_RA;
+    uint8_t* EQ = cx.sm + SM_EQ;
+    float* part = reinterpret_cast<float*>(cx.sm + SM_DPA);  // [8][128], before [dP;dA] is written
+    const float scale = pb.scale;
+    const int b = cp.b, hv = cp.hv, t0 = cp.t0, L = cp.L;
+    const int cg = c & 15, rg = c >> 4, r0 = 8 * rg;
+    const uint32_t a64 = (uint32_t)(cg >> 3) * 64u * 128u + (uint32_t)r0 * 128u;
+    const uint32_t a128 = (uint32_t)(cg >> 3) * 128u * 128u + (uint32_t)r0 * 128u;
+    const uint32_t ch = (uint32_t)(cg & 7);
+    float Gl[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) Gl[e] = 1.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int r = r0 + u;
+        float a8[8];
+        if (APC) {
+            unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+            if (r >= L) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a8[e] = 1.f;
+            }
+        } else {
+            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a8[e] = av;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) Gl[e] *= a8[e];
+    }
+    *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg) = make_float4(Gl[0], Gl[1], Gl[2], Gl[3]);
+    *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg + 4) = make_float4(Gl[4], Gl[5], Gl[6], Gl[7]);
+    named_bar(2, 128);
+    float G[8], gm[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) G[e] = gm[e] = 1.f;
+#pragma unroll
+    for (int g2 = 0; g2 < 8; ++g2) {
+        const float4 p0 = ldf4(part + g2 * 128 + 8 * cg), p1 = ldf4(part + g2 * 128 + 8 * cg + 4);
+        const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (g2 < rg) G[e] *= pv[e];
+            gm[e] *= pv[e];
+        }
+    }
+    if (rg == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gslot[8 * cg + e] = gm[e];
+    }
+
+#pragma unroll 2
+    for (int u = 0; u < 8; ++u) {
+        const int r = r0 + u;
+        const uint32_t sw = (ch ^ (uint32_t)u) << 4;
+        const uint32_t o64 = a64 + u * 128u + sw, oe = a128 + u * 128u + sw, oq = oe + 64u * 128u;
+        float a8[8], k8[8], q8[8], b8[8];
+        if (APC) {
+            unpack8(ld16(RA + o64), a8);
+            if (r >= L) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a8[e] = 1.f;
+            }
+        } else {
+            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a8[e] = av;
+        }
+        unpack8(ld16(RK + o64), k8);
+        unpack8(ld16(RQB + oq), q8);
+        if (GPC) {
+            unpack8(ld16(RQB + oe), b8);
+        } else {
+            const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) b8[e] = bv;
+        }
+        float e8[8], qq[8], kt[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            G[e] *= a8[e];
+            e8[e] = b8[e] * k8[e] * G[e];
+            qq[e] = scale * q8[e] * G[e];
+            kt[e] = __fdividef(k8[e], G[e]);
+        }
+        uint4 hi, lo;
+        split8(e8, hi, lo);
+        st16(EQ + oe, hi);
+        st16(RQB + oe, lo);
+        split8(qq, hi, lo);
+        st16(EQ + oq, hi);
+        st16(RQB + oq, lo);
+        split8(kt, hi, lo);
+        st16(RK + o64, hi);
+        st16(RA + o64, lo);
+    }
+    fence_async_shared();
+    tc_fence_before();
+}
+
+// dv = w .* dY, dw = v .* dY (a scalar beta: sum_j v dY per token into scr[SX_DBV]); run by the
+// staging group after its staging, warp w: tokens w, w + 4, ..., lane l: value channels 4l .. 4l + 3.
+
+template <bool GPC, class TG>
+__device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const ChunkPos& cp, int tt, float* scr) {
+    const Problem& pb = p.pb;
+    const int w = tt >> 5, l = tt & 31, j = 4 * l;
+    const uint8_t* gh = cx.sm + SM_GH;
+    const uint8_t* gl = cx.sm + SM_GL;
+    // loads are unconditional (a row past the sequence reads its last token); stores are guarded
+    uint2 vr[16], wr[16];
+    float bs[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = w + 4 * i;
+        const long row = pb.v_row(cp.b, cp.t0 + min(r, cp.L - 1), cp.hv);
+        vr[i] = __ldg(reinterpret_cast<const uint2*>(p.v + row + j));
+        if (GPC) wr[i] = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.w) + row + j));
+        else bs[i] = gate_or(static_cast<const TG*>(p.b), pb, cp.b, cp.t0, r, cp.L, cp.hv, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int r = w + 4 * i;
+        const uint32_t off = sw128_offset(64 + r, j, 128);
+        const uint2 yh = *reinterpret_cast<const uint2*>(gh + off), yl = *reinterpret_cast<const uint2*>(gl + off);
+        float dy[4], v4[4], w4[4];
+        dy[0] = -(__uint_as_float(yh.x << 16) + __uint_as_float(yl.x << 16));
+        dy[1] = -(__uint_as_float(yh.x & 0xFFFF0000u) + __uint_as_float(yl.x & 0xFFFF0000u));
+        dy[2] = -(__uint_as_float(yh.y << 16) + __uint_as_float(yl.y << 16));
+        dy[3] = -(__uint_as_float(yh.y & 0xFFFF0000u) + __uint_as_float(yl.y & 0xFFFF0000u));
+        v4[0] = __uint_as_float(vr[i].x << 16); v4[1] = __uint_as_float(vr[i].x & 0xFFFF0000u);
+        v4[2] = __uint_as_float(vr[i].y << 16); v4[3] = __uint_as_float(vr[i].y & 0xFFFF0000u);
+        if (GPC) {
+            w4[0] = __uint_as_float(wr[i].x << 16); w4[1] = __uint_as_float(wr[i].x & 0xFFFF0000u);
+            w4[2] = __uint_as_float(wr[i].y << 16); w4[3] = __uint_as_float(wr[i].y & 0xFFFF0000u);
+        } else {
+            w4[0] = w4[1] = w4[2] = w4[3] = bs[i];
+        }
+        const long row = pb.v_row(cp.b, cp.t0 + min(r, cp.L - 1), cp.hv);
+        if (r < cp.L) {
+            *reinterpret_cast<float4*>(p.dv + row + j) =
+                make_float4(w4[0] * dy[0], w4[1] * dy[1], w4[2] * dy[2], w4[3] * dy[3]);
+            if (GPC)
+                *reinterpret_cast<float4*>(p.dw + row + j) =
+                    make_float4(v4[0] * dy[0], v4[1] * dy[1], v4[2] * dy[2], v4[3] * dy[3]);
+        }
+        if (!GPC) {
+            const float sum = warp_sum(fmaf(v4[0], dy[0], fmaf(v4[1], dy[1], fmaf(v4[2], dy[2], v4[3] * dy[3]))));
+            if (l == 0) scr[SX_DBV / 4 + r] = sum;
+        }
+    }
+}
+
+// Epilogue of one chunk once P7-P9 are complete (epilogue group, lane c = channel c).  Per token r
+// (Gamma_r the cumulative decay, gamma = Gamma_63):
+//   dq = scale Gamma dQhat,  de = Gamma dEhat,  db = de k,  dk = de b + (dKtil + gamma dKbar) / Gamma,
+//   dg_r = dQhat Qhat + dEhat Ehat - (dKtil + gamma dKbar) Ktil   (derivative w.r.t. log Gamma_r),
+//   d log alpha_r = sum_{r' >= r} dg_r' + X,   X = gamma (sum_r dKbar_r Ktil_r + rowsum(dS .* S0))
+// (X: the chunk's total decay gamma enters S_end = Diag(gamma) S0 + Kbar^T V' and Kbar).  The tokens
+// are walked from last to first (Gamma_{r-1} = Gamma_r / alpha_r) with the running sum.
+constexpr int RB = 8;  // tokens per block
+
+struct RowIn {
+    float q[RB], k[RB], b[RB], a[RB];
+};
+
+// sum_r dKbar[r][c] Ktil[r][c], from P9 and the Ktil hi/lo tiles still in shared memory (before the
+// next chunk's raw tiles are loaded over them).
+__device__ __forceinline__ float grad_xs(const Ctx& cx, uint32_t tl, int c) {
+    const uint8_t* RK = cx.sm + SM_RK;
+    const uint8_t* RA = cx.sm + SM_RA;
+    float xs = 0.f;
+    // column c of a 64-row K-major tile: row r at cbase + 128 r + xo[r & 7]
+    const uint32_t cbase = (uint32_t)(c >> 6) * 64u * 128u;
+    uint32_t xo[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) xo[u] = ((uint32_t)(c & 63) * 2u) ^ ((uint32_t)u << 4);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        uint32_t rb[32];
+        tmem_ld32(tl + TM_P9 + 32 * hf, rb);
+        float kt[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t off = cbase + (uint32_t)(32 * hf + i) * 128u + xo[i & 7];
+            kt[i] = bf(RK, off) + bf(RA, off);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) xs = fmaf(__uint_as_float(rb[i]), kt[i], xs);
+    }
+    return xs;
+}
+
+// Row addressing of one chunk for lane c: element offsets of token t0 + r are base + r * stride.
+struct RowPtrs {
+    long qk, qk_s;   // q, k (and dq, dk when direct) rows: [B,T,Hk,dk]
+    long g, g_s;     // per-channel gate rows and per-value-head rows: [B,T,Hv,dk]
+    long s1, s1_s;   // scalar gate rows: [B,T,Hv]
+    long o, o_s;     // dq, dk rows (direct: the q/k rows; else per value head)
+};
+
+__device__ __forceinline__ RowPtrs row_ptrs(const Params& p, const ChunkPos& cp, int c) {
+    const Problem& pb = p.pb;
+    RowPtrs rp;
+    rp.qk = pb.qk_row(cp.b, cp.t0, cp.hk) + c;
+    rp.qk_s = (long)pb.Hk * D;
+    rp.g = pb.gate_row(cp.b, cp.t0, cp.hv, D) + c;
+    rp.g_s = (long)pb.Hv * D;
+    rp.s1 = pb.gate_row(cp.b, cp.t0, cp.hv, 1);
+    rp.s1_s = pb.Hv;
+    rp.o = p.direct ? rp.qk : rp.g;
+    rp.o_s = p.direct ? rp.qk_s : rp.g_s;
+    return rp;
+}
+
+// Inputs of tokens r0 .. r0 + RB - 1.  FULL: every row of the chunk is inside the sequence; else rows
+// past the sequence read its last token and are then replaced (a load under a branch would be waited
+// for where the branch ends).
+template <bool APC, bool GPC, bool FULL, class TG>
+__device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, const RowPtrs& rp, int r0, RowIn& x) {
+    const TG* ag = static_cast<const TG*>(p.alpha);
+    const TG* bg = static_cast<const TG*>(p.b);
+#pragma unroll
+    for (int i = 0; i < RB; ++i) {
+        const int r = r0 + i, rr = FULL ? r : min(r, cp.L - 1);
+        const float q0 = __bfloat162float(__ldg(p.q + rp.qk + rr * rp.qk_s));
+        const float k0 = __bfloat162float(__ldg(p.k + rp.qk + rr * rp.qk_s));
+        const float b0 = GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s));
+        const float a0 = APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s)) : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s));
+        const bool in = FULL || r < cp.L;
+        x.q[i] = in ? q0 : 0.f;
+        x.k[i] = in ? k0 : 0.f;
+        x.b[i] = in ? b0 : 0.f;
+        x.a[i] = in ? a0 : 1.f;
+    }
+}
+
+template <bool APC, bool GPC, bool FULL, class TG>
+__device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
+                                                float gam, float xtot, float* scr, int it) {
+    const float scale = p.pb.scale;
+    const RowPtrs rp = row_ptrs(p, cp, c);
+    float G = gam, run = 0.f;
+    auto do_block = [&](int blk, const RowIn& x) {
+        uint32_t rq[RB], re[RB], rk[RB], rb[RB];
+        tmem_ld8(tl + TM_P7 + RB * blk, rq);
+        tmem_ld8(tl + TM_P7 + 64 + RB * blk, re);
+        tmem_ld8(tl + TM_P6 + RB * blk, rk);
+        tmem_ld8(tl + TM_P9 + RB * blk, rb);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = RB - 1; i >= 0; --i) {
+            const int r = RB * blk + i;
+            const float qv = x.q[i], kv = x.k[i], bv = x.b[i];
+            const float ra = __fdividef(1.f, x.a[i]), rg = __fdividef(1.f, G);
+            const float dQh = __uint_as_float(rq[i]), dEh = __uint_as_float(re[i]);
+            const float dkc = fmaf(gam, __uint_as_float(rb[i]), __uint_as_float(rk[i]));
+            const float de = G * dEh;
+            run += fmaf(dQh, scale * qv * G, fmaf(dEh, bv * kv * G, -dkc * kv * rg));
+            const float dla = run + xtot;
+            if (FULL || r < cp.L) {
+                p.dq[rp.o + r * rp.o_s] = scale * G * dQh;
+                p.dk[rp.o + r * rp.o_s] = fmaf(de, bv, dkc * rg);
+                if (GPC) p.db[rp.g + r * rp.g_s] = de * kv;
+                if (APC) p.dalpha[rp.g + r * rp.g_s] = dla * ra;
+            }
+            if (!GPC) {
+                const float sum = warp_sum(de * kv);
+                if ((c & 31) == 0) scr[SX_RB / 4 + warp * 64 + r] = sum;
+            }
+            if (!APC) {
+                const float sum = warp_sum(dla);
+                if ((c & 31) == 0) scr[SX_RA / 4 + warp * 64 + r] = sum;
+            }
+            G *= ra;  // Gamma_{r-1} = Gamma_r / alpha_r
+        }
+    };
+    // two input buffers: a block's loads are in flight while the previous block is formed
+    RowIn x0, x1;
+    load_rows<APC, GPC, FULL, TG>(p, cp, rp, 7 * RB, x0);
+#pragma unroll 1
+    for (int blk = C / RB - 1; blk > 0; blk -= 2) {
+        load_rows<APC, GPC, FULL, TG>(p, cp, rp, (blk - 1) * RB, x1);
+        do_block(blk, x0);
+        if (blk > 1) load_rows<APC, GPC, FULL, TG>(p, cp, rp, (blk - 2) * RB, x0);
+        do_block(blk - 1, x1);
+        if (c == 0) GDN_BTRACE(it, 10 + (C / RB - 1 - blk) / 2);
+    }
+}
+
+// Full chunks (every chunk but a ragged last one) take the variant without per-token guards.
+template <bool APC, bool GPC, class TG>
+__device__ __forceinline__ void grad_epilogue(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
+                                              float gam, float xtot, float* scr, int it = 15) {
+    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    else grad_epilogue_t<APC, GPC, false, TG>(p, cp, tl, c, warp, gam, xtot, scr, it);
+}
+
+// Scalar gates: per-token sums over the channels (the epilogue group's per-warp partials, the
+// dv/dw pass's sum_j v dY), then rows 0-63 of the G lo tile are zeroed again for the next P6.
+template <bool APC, bool GPC, class TG>
+__device__ __forceinline__ void scalar_gate_finish(const Params& p, const ChunkPos& cp, int c, float* scr) {
+    const Problem& pb = p.pb;
+    if (c < cp.L) {
+        const long g1 = pb.gate_row(cp.b, cp.t0 + c, cp.hv, 1);
+        if (!APC) {
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) sum += scr[SX_RA / 4 + w * 64 + c];
+            p.dalpha[g1] = sum / to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1));
+        }
+        if (!GPC) {
+            float sum = scr[SX_DBV / 4 + c];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) sum += scr[SX_RB / 4 + w * 64 + c];
+            p.db[g1] = sum;
+        }
+    }
+    named_bar(2, 128);
+    uint4* z = reinterpret_cast<uint4*>(scr);
+    for (int i = c; i < (int)(SX_BYTES / 16); i += 128) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_shared();
+}
+
+// Barrier 3 of all 256 threads: the epilogue group arrives (does not wait), the staging group waits.
+__device__ __forceinline__ void bar_arrive_all(uint32_t id) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
+}
+__device__ __forceinline__ void bar_sync_all(uint32_t id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
 template <bool APC, bool GPC, class TG>
@@ -778,22 +1204,22 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     cx.bars = reinterpret_cast<uint64_t*>(sm + SM_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_BAR + 128);
     cx.abort_flag = reinterpret_cast<volatile int*>(sm + SM_BAR + 132);
+    volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 136);
     cx.err = p.err;
+    float* xslot = reinterpret_cast<float*>(sm + SM_XSLOT);
+    float* gslot = reinterpret_cast<float*>(sm + SM_GSLOT);
+    float* scr = reinterpret_cast<float*>(sm + SM_GL);
 
     const Problem& pb = p.pb;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const long ci = blockIdx.x;  // (b * Hv + hv) * NT + n
-    const int n = (int)(ci % pb.NT);
-    const int bh = (int)(ci / pb.NT);
-    const int b = bh / pb.Hv, hv = bh % pb.Hv;
-    const int hk = pb.key_head(hv);
-    const int t0 = n * C, L = min(C, pb.T - t0);
+    const long nch = (long)pb.B * pb.Hv * pb.NT;
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t tl_lane = (uint32_t)((warp & 3) * 32) << 16;
+    const Maps m{&tm_q, &tm_k, &tm_a, &tm_b, &tm_do, &tm_yh, &tm_yl, &tm_vh, &tm_vl};
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) mbar_init(cx.bars + i, 1);
         *cx.abort_flag = 0;
+        *stop_slot = 0;
         mbar_fence_init();
     }
     if (warp == 0) {
@@ -804,244 +1230,86 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t tl = tbase + tl_lane;
-    if (tid == 0)
-        grad_load_all<APC, GPC>(cx, n, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b, &tm_do, &tm_yh, &tm_yl, &tm_vh, &tm_vl);
-    {
-        // zero rows 0-63 of the G lo tile (dO is exact in bf16)
-        uint8_t* gl = sm + SM_GL;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int idx = tid + u * kThreads;  // 1024 chunks of 16 bytes: 2 atoms x 512
-            st16(gl + (uint32_t)(idx >> 9) * 16384u + (uint32_t)(idx & 511) * 16u, make_uint4(0u, 0u, 0u, 0u));
+    const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+    int raw_issued = 0, gv_issued = 0;  // raw tiles: thread 0;  G and V' tiles: thread 128
+    long ci = blockIdx.x;
+    if (ci < nch) {
+        const ChunkPos c0 = chunk_pos(pb, ci);
+        if (tid == 0) {
+            load_raw_g<APC, GPC>(cx, c0, m);
+            raw_issued = 1;
         }
-    }
-
-    float dot_c = 0.f;  // lanes c (warps 0-3): sum_j dS_end[c][j] S0[c][j]
-    if (warp < 4) {
-        // ---- S0 and dS_end rows into tensor memory (split), row dot product ------------------
-        const int c = tid;
-        const float4* s0r = reinterpret_cast<const float4*>(p.s0 + (ci * D + c) * D);
-        const float4* dsr = reinterpret_cast<const float4*>(p.dsc + (ci * D + c) * D);
-#pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
-            float4 a[8], d[8];
+        if (tid == 128) {
+            load_gv(cx, c0, m);
+            gv_issued = 1;
+        }
+        if (warp < 4) {
+            uint8_t* gl = sm + SM_GL;  // rows 0-63 of the G lo tile: zeros (dO is exact in bf16)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                a[u] = s0r[8 * q4 + u];
-                d[u] = dsr[8 * q4 + u];
+                const int idx = tid + 128 * u;
+                st16(gl + (uint32_t)(idx >> 9) * 16384u + (uint32_t)(idx & 511) * 16u, make_uint4(0u, 0u, 0u, 0u));
             }
-            uint32_t ah[16], al[16], dh[16], dl[16];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                dot_c = fmaf(d[u].x, a[u].x, dot_c);
-                dot_c = fmaf(d[u].y, a[u].y, dot_c);
-                dot_c = fmaf(d[u].z, a[u].z, dot_c);
-                dot_c = fmaf(d[u].w, a[u].w, dot_c);
-                split_pack(a[u].x, a[u].y, ah[2 * u], al[2 * u]);
-                split_pack(a[u].z, a[u].w, ah[2 * u + 1], al[2 * u + 1]);
-                split_pack(d[u].x, d[u].y, dh[2 * u], dl[2 * u]);
-                split_pack(d[u].z, d[u].w, dh[2 * u + 1], dl[2 * u + 1]);
-            }
-            tmem_st16(tl + TM_S0H + 16 * q4, ah);
-            tmem_st16(tl + TM_S0L + 16 * q4, al);
-            tmem_st16(tl + TM_DSH + 16 * q4, dh);
-            tmem_st16(tl + TM_DSL + 16 * q4, dl);
-        }
-        tmem_st_wait();
-    } else {
-        // ---- cumulative decay; split [Ehat;Qhat], Ktil ----------------------------------------
-        const int c = tid - 128;
-        if (c == 0) wait1(cx, B_RAW, 0);
-        named_bar(2, 128);
-        const TG* alpha_g = static_cast<const TG*>(p.alpha);
-        const TG* beta_g = static_cast<const TG*>(p.b);
-        uint8_t* RQB = sm + SM_RQB;
-        uint8_t* RK = sm + SM_RK;
-        uint8_t* RA = sm + SM_RA;
-        uint8_t* EQ = sm + SM_EQ;
-        float* part = reinterpret_cast<float*>(sm + SM_DPA);  // [8][128], before [dP;dA] is written
-        const float scale = pb.scale;
-        const int cg = c & 15, rg = c >> 4, r0 = 8 * rg;
-        const uint32_t a64 = (uint32_t)(cg >> 3) * 64u * 128u + (uint32_t)r0 * 128u;
-        const uint32_t a128 = (uint32_t)(cg >> 3) * 128u * 128u + (uint32_t)r0 * 128u;
-        const uint32_t ch = (uint32_t)(cg & 7);
-        float Gl[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) Gl[e] = 1.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int r = r0 + u;
-            float a8[8];
-            if (APC) {
-                unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
-                if (r >= L) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) a8[e] = 1.f;
-                }
-            } else {
-                const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) a8[e] = av;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) Gl[e] *= a8[e];
-        }
-        *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg) = make_float4(Gl[0], Gl[1], Gl[2], Gl[3]);
-        *reinterpret_cast<float4*>(part + rg * 128 + 8 * cg + 4) = make_float4(Gl[4], Gl[5], Gl[6], Gl[7]);
-        named_bar(2, 128);
-        float G[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) G[e] = 1.f;
-#pragma unroll
-        for (int g2 = 0; g2 < 8; ++g2) {
-            if (g2 < rg) {
-                const float4 p0 = ldf4(part + g2 * 128 + 8 * cg), p1 = ldf4(part + g2 * 128 + 8 * cg + 4);
-                G[0] *= p0.x; G[1] *= p0.y; G[2] *= p0.z; G[3] *= p0.w;
-                G[4] *= p1.x; G[5] *= p1.y; G[6] *= p1.z; G[7] *= p1.w;
-            }
-        }
-#pragma unroll 2
-        for (int u = 0; u < 8; ++u) {
-            const int r = r0 + u;
-            const uint32_t sw = (ch ^ (uint32_t)u) << 4;
-            const uint32_t o64 = a64 + u * 128u + sw, oe = a128 + u * 128u + sw, oq = oe + 64u * 128u;
-            float a8[8], k8[8], q8[8], b8[8];
-            if (APC) {
-                unpack8(ld16(RA + o64), a8);
-                if (r >= L) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) a8[e] = 1.f;
-                }
-            } else {
-                const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) a8[e] = av;
-            }
-            unpack8(ld16(RK + o64), k8);
-            unpack8(ld16(RQB + oq), q8);
-            if (GPC) {
-                unpack8(ld16(RQB + oe), b8);
-            } else {
-                const float bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) b8[e] = bv;
-            }
-            float e8[8], qq[8], kt[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                G[e] *= a8[e];
-                e8[e] = b8[e] * k8[e] * G[e];
-                qq[e] = scale * q8[e] * G[e];
-                kt[e] = __fdividef(k8[e], G[e]);
-            }
-            uint4 hi, lo;
-            split8(e8, hi, lo);
-            st16(EQ + oe, hi);
-            st16(RQB + oe, lo);
-            split8(qq, hi, lo);
-            st16(EQ + oq, hi);
-            st16(RQB + oq, lo);
-            split8(kt, hi, lo);
-            st16(RK + o64, hi);
-            st16(RA + o64, lo);
+        } else {
+            stage_chunk<APC, GPC, TG>(p, cx, c0, tl, tid - 128, xslot, gslot, 0u);
         }
     }
-    fence_async_shared();
-    tc_fence_before();
-    __syncthreads();
-    // ---- P6 = G V'^T ----------------------------------------------------------------------------
-    if (tid == 0) {
+    for (int it = 0; ci < nch; ++it, ci += gridDim.x) {
+        const ChunkPos cp = chunk_pos(pb, ci);
+        const uint32_t par = (uint32_t)it & 1u;
+        fence_async_shared();
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
-        if (wait1(cx, B_GV, 0) && !*cx.abort_flag) {
-            const uint32_t id64 = idesc_bf16_f32(128, 64);
-            mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP, id64, false);
-            mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GL, sbase + SM_VP, id64, true);
-            mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP + 16384, id64, true);
-            mma_commit(cx.bars + B_P6);
-            wait1(cx, B_P6, 0);
+        if (tid == 0) GDN_BTRACE(it, 0);
+        const long nx = ci + gridDim.x;
+        // rowsum(dS_end .* S0) and gamma of this chunk (the staging group overwrites the slots with
+        // the next chunk's after the next barrier)
+        const float dot_c = xslot[tid & 127], gam_c = gslot[tid & 127];
+        // ---- P6 = G V'^T --------------------------------------------------------------------------
+        if (tid == 0) {
+            if (wait1(cx, B_GV, par) && !*cx.abort_flag) {
+                const uint32_t id64 = idesc_bf16_f32(128, 64);
+                mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP, id64, false);
+                mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GL, sbase + SM_VP, id64, true);
+                mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP + 16384, id64, true);
+                mma_commit(cx.bars + B_P6);
+                wait1(cx, B_P6, par);
+            }
+            GDN_BTRACE(it, 1);
         }
-    }
-    __syncthreads();
-    tc_fence_after();
-    const bool ok = !*cx.abort_flag;
-    if (warp < 4) {
-        // ---- [dP; dA]: row r' of P6, masked (dP: s <= r', dA: s < r' - 64), split -------------
-        if (ok) {
-            const int rp = tid;
+        __syncthreads();
+        tc_fence_after();
+        // ---- [dP; dA]: row r' of P6, masked (dP: s <= r', dA: s < r' - 64), split ------------------
+        if (!*cx.abort_flag) {
+            const int rp = tid & 127, hc = tid >> 7;
             const int lim = rp < 64 ? rp : rp - 65;  // keep s <= lim
             uint8_t* dpa = sm + SM_DPA;
+            uint32_t r[32];
+            tmem_ld32(tl + TM_P6 + 32 * hc, r);
+            tmem_ld_wait();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tmem_ld32(tl + TM_P6 + 32 * half, r);
-                tmem_ld_wait();
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t wh[4], wl[4];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t wh[4], wl[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i0 = 8 * ch + 2 * e, s0 = 32 * half + i0;
-                        const float x0 = s0 <= lim ? __uint_as_float(r[i0]) : 0.f;
-                        const float x1 = s0 + 1 <= lim ? __uint_as_float(r[i0 + 1]) : 0.f;
-                        split_pack(x0, x1, wh[e], wl[e]);
-                    }
-                    const uint32_t off = sw128_offset(rp, 32 * half + 8 * ch, 128);
-                    st16(dpa + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
-                    st16(dpa + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                for (int e = 0; e < 4; ++e) {
+                    const int i0 = 8 * ch + 2 * e, s0 = 32 * hc + i0;
+                    const float x0 = s0 <= lim ? __uint_as_float(r[i0]) : 0.f;
+                    const float x1 = s0 + 1 <= lim ? __uint_as_float(r[i0 + 1]) : 0.f;
+                    split_pack(x0, x1, wh[e], wl[e]);
                 }
+                const uint32_t off = sw128_offset(rp, 32 * hc + 8 * ch, 128);
+                st16(dpa + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                st16(dpa + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
             }
         }
-    } else {
-        // ---- dv = w .* dY, dw = v .* dY (or sum_j v dY for a scalar beta) -----------------------
-        const int tt = tid - 128, r = tt >> 1, jh = tt & 1;
-        float* dbv = reinterpret_cast<float*>(sm + SM_DBV);
-        float bsum = 0.f;
-        if (r < L) {
-            const long row = pb.v_row(b, t0 + r, hv);
-            const uint8_t* gh = sm + SM_GH;
-            const uint8_t* gl = sm + SM_GL;
-            float bscal = 0.f;
-            if (!GPC) bscal = to_f32(static_cast<const TG*>(p.b)[pb.gate_row(b, t0 + r, hv, 1)]);
-#pragma unroll 2
-            for (int cc = 0; cc < 8; ++cc) {
-                const int j = 64 * jh + 8 * cc;
-                const uint32_t off = sw128_offset(64 + r, j, 128);
-                float yh[8], yl[8], v8[8], w8[8];
-                unpack8(ld16(gh + off), yh);
-                unpack8(ld16(gl + off), yl);
-                unpack8(*reinterpret_cast<const uint4*>(p.v + row + j), v8);
-                if (GPC) unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.w) + row + j), w8);
-                float dvv[8], dww[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float dy = -(yh[e] + yl[e]);
-                    dvv[e] = (GPC ? w8[e] : bscal) * dy;
-                    dww[e] = v8[e] * dy;
-                    if (!GPC) bsum = fmaf(v8[e], dy, bsum);
-                }
-                float4* dvp = reinterpret_cast<float4*>(p.dv + row + j);
-                dvp[0] = make_float4(dvv[0], dvv[1], dvv[2], dvv[3]);
-                dvp[1] = make_float4(dvv[4], dvv[5], dvv[6], dvv[7]);
-                if (GPC) {
-                    float4* dwp = reinterpret_cast<float4*>(p.dw + row + j);
-                    dwp[0] = make_float4(dww[0], dww[1], dww[2], dww[3]);
-                    dwp[1] = make_float4(dww[4], dww[5], dww[6], dww[7]);
-                }
-            }
-        }
-        if (!GPC) {
-            bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
-            if (jh == 0) dbv[r] = bsum;
-        }
-    }
-    fence_async_shared();
-    tc_fence_before();
-    __syncthreads();
-    // ---- P7 = S0 G^T + Ktil^T [dP;dA]^T,  P8 = [Qhat^T|Ehat^T] [dP;dA],  P9 = dS V'^T --------------
-    if (tid == 0) {
+        fence_async_shared();
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
-        if (ok) {
+        // ---- P7 = S0 G^T + Ktil^T [dP;dA]^T,  P8 = [Qhat^T|Ehat^T] [dP;dA],  P9 = dS V'^T ----------
+        if (tid == 0) GDN_BTRACE(it, 2);
+        if (tid == 0 && !*cx.abort_flag) {
             const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
             mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0H, sbase + SM_GH, id128, false);
             mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0L, sbase + SM_GH, id128, true);
@@ -1074,148 +1342,61 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSL, sbase + SM_VP, id64, true);
             mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSH, sbase + SM_VP + 16384, id64, true);
             mma_commit(cx.bars + B_P789);
-            wait1(cx, B_P789, 0);
+            wait1(cx, B_P789, par);
+            GDN_BTRACE(it, 3);
         }
+        __syncthreads();
+        tc_fence_after();
+        // ---- chunk ci: dv, dw, then the epilogue;  chunk ci + gridDim.x: staging -------------------
+        if (warp < 4) {
+            const float xs = grad_xs(cx, tl, tid);
+            named_bar(1, 128);  // Ktil read: the next chunk's raw tiles may land
+            if (tid == 0 && nx < nch && !*cx.abort_flag) {
+                load_raw_g<APC, GPC>(cx, chunk_pos(pb, nx), m);
+                ++raw_issued;
+            }
+            if (tid == 0) GDN_BTRACE(it, 9);
+            if (!*cx.abort_flag)
+                grad_epilogue<APC, GPC, TG>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
+            if (tid == 0) GDN_BTRACE(it, 5);
+            if (!APC || !GPC) bar_arrive_all(3);  // per-warp partials of the scalar gates written
+        } else {
+            if (nx < nch)
+                stage_chunk<APC, GPC, TG>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
+            if (tid == 128) GDN_BTRACE(it, 8);
+            grad_dv_dw<GPC, TG>(p, cx, cp, tid - 128, scr);
+            named_bar(2, 128);
+            if (tid == 128) GDN_BTRACE(it, 4);
+            // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land
+            if (tid == 128 && nx < nch && !*cx.abort_flag) {
+                load_gv(cx, chunk_pos(pb, nx), m);
+                ++gv_issued;
+            }
+            if (!APC || !GPC) {
+                bar_sync_all(3);
+                if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG>(p, cp, tid - 128, scr);
+            }
+        }
+        if (tid == 0) *stop_slot = *cx.abort_flag;
+        __syncthreads();
+        if (*stop_slot) break;
     }
-    __syncthreads();
-    tc_fence_after();
-    // ---- epilogue: lane c, tokens 32 half .. 32 half + 31 ------------------------------------------
-    if (!*cx.abort_flag) {
-        const int c = tid & 127, half = tid >> 7;
-        float* X = reinterpret_cast<float*>(sm + SM_RQB);
-        const float* dbv = reinterpret_cast<const float*>(sm + SM_DBV);
-        const TG* alpha_g = static_cast<const TG*>(p.alpha);
-        const TG* b_g = static_cast<const TG*>(p.b);
-        const float scale = pb.scale;
-        float al[32];
-        float prod = 1.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * half + i;
-            float a = 1.f;
-            if (r < L) a = APC ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, D) + c])
-                               : to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]);
-            al[i] = a;
-            prod *= a;
-        }
-        X[SX_PROD / 4 + half * 128 + c] = prod;
-        __syncthreads();
-        const float pL = X[SX_PROD / 4 + c], pU = X[SX_PROD / 4 + 128 + c];
-        const float gam = pL * pU;
-        float G = half ? pL : 1.f;
-        float dg[32];
-        float part = 0.f;
-        float* red = X + SX_RED / 4;
-#pragma unroll
-        for (int sub = 0; sub < 2; ++sub) {
-            uint32_t rq[16], re[16], rk[16], rb[16];
-            tmem_ld16(tl + TM_P7 + 32 * half + 16 * sub, rq);
-            tmem_ld16(tl + TM_P7 + 64 + 32 * half + 16 * sub, re);
-            tmem_ld16(tl + TM_P6 + 32 * half + 16 * sub, rk);
-            tmem_ld16(tl + TM_P9 + 32 * half + 16 * sub, rb);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int il = 16 * sub + i, r = 32 * half + il, t = t0 + r;
-                const bool in = r < L;
-                G *= al[il];
-                float qv = 0.f, kv = 0.f, bv = 0.f;
-                if (in) {
-                    const long qk = pb.qk_row(b, t, hk) + c;
-                    qv = __bfloat162float(p.q[qk]);
-                    kv = __bfloat162float(p.k[qk]);
-                    bv = GPC ? to_f32(b_g[pb.gate_row(b, t, hv, D) + c]) : to_f32(b_g[pb.gate_row(b, t, hv, 1)]);
-                }
-                const float Qh = scale * qv * G, Eh = bv * kv * G, Kt = __fdividef(kv, G);
-                const float dQh = __uint_as_float(rq[i]), dEh = __uint_as_float(re[i]);
-                const float dKb = __uint_as_float(rb[i]);
-                const float dkc = fmaf(gam, dKb, __uint_as_float(rk[i]));
-                const float de = G * dEh;
-                dg[il] = dQh * Qh + dEh * Eh - dkc * Kt;
-                part = fmaf(gam * dKb, Kt, part);
-                if (in) {
-                    const long o = p.direct ? pb.qk_row(b, t, hk) + c : pb.gate_row(b, t, hv, D) + c;
-                    p.dq[o] = scale * G * dQh;
-                    p.dk[o] = fmaf(de, bv, __fdividef(dkc, G));
-                    if (GPC) p.db[pb.gate_row(b, t, hv, D) + c] = de * kv;
-                }
-                if (!GPC) {
-                    const float s = warp_sum(de * kv);
-                    if ((tid & 31) == 0) red[warp * 32 + il] = s;
-                }
-            }
-        }
-        if (half == 0) X[SX_PART / 4 + c] = fmaf(gam, dot_c, part);
-        __syncthreads();
-        float* red2 = X + SX_RED2 / 4;
-        float run = 0.f;
-        if (half == 1) {
-            dg[31] += part + X[SX_PART / 4 + c];
-#pragma unroll
-            for (int il = 31; il >= 0; --il) {
-                run += dg[il];
-                const int r = 32 + il;
-                if (APC) {
-                    if (r < L) p.dalpha[pb.gate_row(b, t0 + r, hv, D) + c] = run / al[il];
-                } else {
-                    const float s = warp_sum(run);
-                    if ((tid & 31) == 0) red2[warp * 32 + il] = s;
-                }
-            }
-            X[SX_SUF / 4 + c] = run;
-        }
-        __syncthreads();
-        if (half == 0) {
-            run = X[SX_SUF / 4 + c];
-#pragma unroll
-            for (int il = 31; il >= 0; --il) {
-                run += dg[il];
-                const int r = il;
-                if (APC) {
-                    if (r < L) p.dalpha[pb.gate_row(b, t0 + r, hv, D) + c] = run / al[il];
-                } else {
-                    const float s = warp_sum(run);
-                    if ((tid & 31) == 0) red2[warp * 32 + il] = s;
-                }
-            }
-        }
-        if (!APC || !GPC) {
-            __syncthreads();
-            if (tid < 64) {
-                const int r = tid, hh = r >> 5, il = r & 31;
-                if (r < L) {
-                    const long g1 = pb.gate_row(b, t0 + r, hv, 1);
-                    if (!APC) {
-                        float s = 0.f;
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) s += red2[(4 * hh + w) * 32 + il];
-                        p.dalpha[g1] = s / to_f32(alpha_g[g1]);
-                    }
-                    if (!GPC) {
-                        float s = dbv[r];
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) s += red[(4 * hh + w) * 32 + il];
-                        p.db[g1] = s;
-                    }
-                }
-            }
-        }
-    }
-    // ---- teardown ----------------------------------------------------------------------------------
+    // ---- teardown: TMA loads still in flight after an abort are waited for (bounded) -----------
     tc_fence_before();
     __syncthreads();
-    if (*cx.abort_flag && tid == 0) {
+    if (*cx.abort_flag && (tid == 0 || tid == 128)) {
         const uint64_t tw = globaltimer_ns();
-        while (!mbar_try_wait(cx.bars + B_RAW, 0) && globaltimer_ns() - tw < kWaitNs) {
-        }
-        while (!mbar_try_wait(cx.bars + B_GV, 0) && globaltimer_ns() - tw < kWaitNs) {
-        }
+        if (raw_issued > 0)
+            while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - tw < kWaitNs) {
+            }
+        if (gv_issued > 0)
+            while (!mbar_try_wait(cx.bars + B_GV, (uint32_t)((gv_issued - 1) & 1)) && globaltimer_ns() - tw < kWaitNs) {
+            }
     }
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
 }
-
 }  // namespace grad
 }  // namespace tcbwd
 }  // namespace gdn

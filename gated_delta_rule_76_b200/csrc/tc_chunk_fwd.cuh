@@ -121,7 +121,8 @@ struct Params {
     float* ht;
     int* err;    // device error word (bit 0: a bounded wait expired)
     // Backward support (all NULL in a plain forward).  o may be NULL then: no output is formed.
-    float* s0_out;               // [B*Hv][NT][dk][dv] fp32: the state entering every chunk
+    float* s0_out;               // [B*Hv][NT + 1][dv/4][dk][4] fp32: the state entering every chunk, then
+                                 //   the final state
     __nv_bfloat16* vp_hi;        // [B,T,Hv,dv]: V' = T (Z - Ehat S0) of every token, split
     __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
 };
@@ -357,10 +358,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t pn = n & 1;
             const int t0 = n * C, L = min(C, pb.T - t0);
             if (p.s0_out) {
-                // state entering chunk n, rows 64h .. 64h + 63 of column j (coalesced over j)
-                float* dst = p.s0_out + ((long)blockIdx.x * NT + n) * (D * D) + (long)(64 * h) * D + j;
+                // state entering chunk n, rows 64h .. 64h + 63 of column j, in the layout
+                // [j / 4][row][j % 4] (a reader holding one row per thread loads it as float4s)
+                float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
 #pragma unroll
-                for (int c = 0; c < 64; ++c) dst[c * D] = S[c];
+                for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
             }
             // ---- X2 = S0^T [Ehat;Qhat]^T  (S0 split; Qhat split in the Qhat half) ------------------
             if (tid == 0) {
@@ -398,7 +400,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const float vv = bf(vt, off);
                         float ww;
                         if (GPC) ww = bf(vt + 16384, off);
-                        else ww = rr < L ? to_f32(beta[pb.gate_row(b, t0 + rr, hv, 1)]) : 0.f;
+                        else ww = gate_or(beta, pb, b, t0, rr, L, hv, 0.f);
                         y2[e] = vv * ww - __uint_as_float(r[ii]);
                     }
                     split_pack(y2[0], y2[1], hi[i], lo[i]);
@@ -612,6 +614,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int c = 0; c < 64; ++c) p.ht[soff + (long)(64 * h + c) * D + j] = S[c];
         }
+        if (p.s0_out && !*cx.abort_flag) {
+            // the final state follows the last chunk's entering state
+            float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + NT) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
+        }
     } else {
         // =================================== chunk prologue ===================================
         const int c = tid - 256;  // key channel; also TMEM lane of X1
@@ -661,7 +669,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             for (int i = 0; i < 8; ++i) a8[i] = 1.f;
                         }
                     } else {
-                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) a8[i] = av;
                     }
@@ -702,7 +710,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             for (int i = 0; i < 8; ++i) a8[i] = 1.f;
                         }
                     } else {
-                        const float av = r < L ? to_f32(alpha_g[pb.gate_row(b, t0 + r, hv, 1)]) : 1.f;
+                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) a8[i] = av;
                     }
@@ -711,7 +719,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
                     } else {
-                        const float bv = r < L ? to_f32(beta_g[pb.gate_row(b, t0 + r, hv, 1)]) : 0.f;
+                        const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) b8[i] = bv;
                     }

@@ -131,6 +131,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
+// 32 lanes x 8 consecutive 32-bit columns per warp (same lane mapping as tmem_ld32).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7])
+                 : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -274,6 +281,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void* tmap,
         "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst_smem),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// Bulk prefetch of the global range [gaddr, gaddr + bytes) into L2 (16-byte aligned start, bytes a
+// multiple of 16).  Nothing is written; the issuing thread does not wait.
+__device__ __forceinline__ void prefetch_l2(const void* gaddr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)), "r"(bytes)
+                 : "memory");
+}
+
+// Prefetch of the 128-byte line holding gaddr into L2 (load/store path; the thread does not wait).
+__device__ __forceinline__ void prefetch_line_l2(const void* gaddr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(gaddr)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
