@@ -274,14 +274,19 @@ def bench_headline(args, dist, peaks, peak_kind, stream, device):
     B, T = wl.B, wl.T
     o = torch.empty_like(g["v"])
     ht = torch.empty((B, wl.Hv, wl.dk, wl.dv), dtype=torch.float32, device=device)
-    fa, _ = gdn.fwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], o=o, ht=ht, **gates(g))
     import ctypes
     lib = gdn.load()
+    # the forward keeps what the backward needs (chunk states, V') in a cache: training's forward +
+    # backward, without recomputing the forward inside the backward
+    cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], **gates(g)),
+                        dtype=torch.uint8, device=device)
+    fa, _ = gdn.fwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], o=o, ht=ht, bwd_cache=cache, **gates(g))
     ws_f = torch.empty(lib.gdn_chunk_fwd_workspace_size(ctypes.byref(fa)), dtype=torch.uint8, device=device)
     f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=device)
     grads = {"dq": f32(g["q"]), "dk": f32(g["k"]), "dv": f32(g["v"]), "dalpha": f32(g["alpha"]),
              "db": f32(g["b"]), "dw": f32(g["w"]), "dh0": f32(g["h0"])}
-    ba, _ = gdn.bwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], grads=grads, **gates(g))
+    ba, _ = gdn.bwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], grads=grads,
+                         fwd_cache=cache, **gates(g))
     ws_b = torch.empty(lib.gdn_chunk_bwd_workspace_size(ctypes.byref(ba)), dtype=torch.uint8, device=device)
     sptr = ctypes.c_void_p(stream.cuda_stream)
 
@@ -342,14 +347,16 @@ def bench_headline_e2e(args, dist, x, stream, device):
     dev = {n: torch.empty_like(host[n], device=device) for n in names_in}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     out_host = {}
+    cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"],
+                                                     w=dev["w"], h0=dev["h0"]), dtype=torch.uint8, device=device)
 
     def step():
         for n in names_in:
             dev[n].copy_(host[n], non_blocking=True)
         o, ht = gdn.gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
-                                  h0=dev["h0"], stream=stream)
+                                  h0=dev["h0"], bwd_cache=cache, stream=stream)
         gr = gdn.gdn_chunk_bwd(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
-                               h0=dev["h0"], grad_o=dev["dout"], stream=stream)
+                               h0=dev["h0"], grad_o=dev["dout"], fwd_cache=cache, stream=stream)
         res = {"o": o, "ht": ht, **gr}
         for n, t in res.items():
             if n not in out_host:
@@ -577,7 +584,7 @@ def main():
                    "chunk": 64, "state": "fp32", "gates": "channel alpha, b, w (bf16)",
                    "parallelism": f"dp{dist.world} (independent replicas of the workload)",
                    "l2": "inputs larger than L2 (~0.9 GB read per step); no flush needed",
-                   "step": "gdn_chunk_fwd + gdn_chunk_bwd"},
+                   "step": "gdn_chunk_fwd (keeping the backward cache) + gdn_chunk_bwd (from the cache)"},
         "roofline": head["roofline"],
         "step_roofline": head["step_roofline"],
         "fwd_ms": round(head["fwd_ms"], 4), "bwd_ms": round(head["bwd_ms"], 4),

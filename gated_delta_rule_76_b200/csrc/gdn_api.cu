@@ -192,8 +192,11 @@ gdn_status check_fwd(const gdn_fwd_args* a) {
     const Buf out[] = {
         {a->o, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "o"},
         {a->ht, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "ht"},
+        {a->bwd_cache, a->bwd_cache ? a->bwd_cache_bytes : 0, "bwd_cache"},
     };
-    return check_buffers(in, 9, out, 2);
+    if (a->bwd_cache && (reinterpret_cast<uintptr_t>(a->bwd_cache) & 255u))
+        return fail(GDN_ERR_INVALID_ARG, "bwd_cache is not 256-byte aligned");
+    return check_buffers(in, 9, out, 3);
 }
 
 gdn_status check_bwd(const gdn_bwd_args* a) {
@@ -218,14 +221,17 @@ gdn_status check_bwd(const gdn_bwd_args* a) {
         {a->v, BT * a->Hv * a->dv * es, "v"}, {a->alpha, na, "alpha"}, {a->b, nb, "b"},
         {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_o, BT * a->Hv * a->dv * es, "grad_o"}, {a->grad_ht, st, "grad_ht"},
+        {a->fwd_cache, a->fwd_cache ? a->fwd_cache_bytes : 0, "fwd_cache"},
     };
+    if (a->fwd_cache && (reinterpret_cast<uintptr_t>(a->fwd_cache) & 255u))
+        return fail(GDN_ERR_INVALID_ARG, "fwd_cache is not 256-byte aligned");
     const size_t na4 = na / gs * 4, nb4 = nb / gs * 4;
     const Buf out[] = {
         {a->grad_q, BT * a->Hk * a->dk * 4, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * 4, "grad_k"},
         {a->grad_v, BT * a->Hv * a->dv * 4, "grad_v"}, {a->grad_alpha, na4, "grad_alpha"},
         {a->grad_b, nb4, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * 4, "grad_w"}, {a->grad_h0, st, "grad_h0"},
     };
-    return check_buffers(in, 10, out, 7);
+    return check_buffers(in, 11, out, 7);
 }
 
 gdn_status check_workspace(void* ws, size_t have, size_t need) {
@@ -280,6 +286,12 @@ static bool fwd_uses_tensor_cores(const gdn_fwd_args* a, const Problem& pb) {
     return tc_fwd_eligible(pb, a->dtype == GDN_BF16, a->gate_dtype == GDN_BF16, f);
 }
 
+size_t gdn_chunk_fwd_cache_size(const gdn_fwd_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    return fwd_uses_tensor_cores(a, pb) ? plan_tc_cache(pb).bytes : 0;
+}
+
 size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
@@ -297,11 +309,28 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
     const bool tc = fwd_uses_tensor_cores(a, pb);
+    if (a->bwd_cache) {
+        if (!tc)
+            return fail(GDN_ERR_UNSUPPORTED, "bwd_cache: only the tensor-core path (bf16, dk = dv = 128) keeps a cache");
+        if (a->bwd_cache_bytes < plan_tc_cache(pb).bytes)
+            return fail(GDN_ERR_WORKSPACE, "bwd_cache has %zu bytes, %zu needed", a->bwd_cache_bytes,
+                        plan_tc_cache(pb).bytes);
+    }
     WsPlan plan = plan_chunk_ws(pb, false, false);
     if ((s = check_workspace(workspace, workspace_bytes, tc ? 256 : plan.bytes))) return s;
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
     if (e == cudaSuccess) {
-        if (tc) e = tc_chunk_fwd(pb, io_from(a), f, a->gate_dtype == GDN_BF16, ws_status(workspace), st);
+        TcFwdSave save{};
+        if (a->bwd_cache) {
+            const TcCache cp = plan_tc_cache(pb);
+            char* cb = static_cast<char*>(a->bwd_cache);
+            save.s0 = reinterpret_cast<float*>(cb + cp.s0);
+            save.vp_hi = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_hi);
+            save.vp_lo = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_lo);
+        }
+        if (tc)
+            e = tc_chunk_fwd(pb, io_from(a), f, a->gate_dtype == GDN_BF16, ws_status(workspace), st,
+                             a->bwd_cache ? &save : nullptr);
         else e = run_fwd(variant(a->dtype, a->gate_dtype), pb, io_from(a), carve_chunk_ws(plan, workspace), f, st);
     }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_fwd");
@@ -315,7 +344,7 @@ static bool bwd_uses_tensor_cores(const gdn_bwd_args* a, const Problem& pb) {
 size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    if (bwd_uses_tensor_cores(a, pb)) return plan_tc_bwd_ws(pb, !identity_heads(pb)).bytes;
+    if (bwd_uses_tensor_cores(a, pb)) return plan_tc_bwd_ws(pb, !identity_heads(pb), a->fwd_cache != nullptr).bytes;
     return plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
 }
 
@@ -330,7 +359,13 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     const bool direct = identity_heads(pb);
     const bool tc = bwd_uses_tensor_cores(a, pb);
     WsPlan plan = plan_chunk_ws(pb, true, !direct);
-    TcBwdWs tplan = tc ? plan_tc_bwd_ws(pb, !direct) : TcBwdWs{};
+    if (a->fwd_cache) {
+        if (!tc) return fail(GDN_ERR_UNSUPPORTED, "fwd_cache: only the tensor-core path keeps a forward cache");
+        if (a->fwd_cache_bytes < plan_tc_cache(pb).bytes)
+            return fail(GDN_ERR_INVALID_ARG, "fwd_cache has %zu bytes, %zu needed", a->fwd_cache_bytes,
+                        plan_tc_cache(pb).bytes);
+    }
+    TcBwdWs tplan = tc ? plan_tc_bwd_ws(pb, !direct, a->fwd_cache != nullptr) : TcBwdWs{};
     if ((s = check_workspace(workspace, workspace_bytes, tc ? tplan.bytes : plan.bytes))) return s;
     ChunkIO io{};
     io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
@@ -341,7 +376,7 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_bwd");
     if (tc) {
-        e = tc_chunk_bwd(pb, io, f, a->gate_dtype == GDN_BF16, direct, tplan, workspace, st);
+        e = tc_chunk_bwd(pb, io, f, a->gate_dtype == GDN_BF16, direct, tplan, workspace, a->fwd_cache, st);
         return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_bwd");
     }
     ChunkWs ws = carve_chunk_ws(plan, workspace);

@@ -50,13 +50,21 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
                          cudaStream_t st, const TcFwdSave* save = nullptr);
 
 // Tensor-core chunk backward (tc_bwd.cu): same eligibility as the forward, without z.
+// The forward cache (what the backward needs from the forward): byte offsets from its start.
+struct TcCache {
+    size_t bytes = 0;
+    size_t s0, vp_hi, vp_lo;  // states [B*Hv][NT+1][dv/4][dk][4] fp32; V' hi, lo [B,T,Hv,dv] bf16
+};
+TcCache plan_tc_cache(const Problem& pb);
 struct TcBwdWs {
     size_t bytes = 0;  // total, including the 256-byte status word at offset 0
-    size_t s0, dsc, vp_hi, vp_lo, ny_hi, ny_lo, dq_v, dk_v;  // byte offsets (dq_v, dk_v: GQA only)
+    size_t cache;      // a forward cache inside the workspace (~0 when the caller passes one)
+    size_t dsc, ny_hi, ny_lo, dq_v, dk_v;  // byte offsets (dq_v, dk_v: GQA only)
 };
-TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials);
+TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials, bool caller_cache);
+// cache: the caller's forward cache (the forward is not recomputed), or NULL.
 cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, bool direct,
-                         const TcBwdWs& plan, void* ws, cudaStream_t st);
+                         const TcBwdWs& plan, void* ws, const void* cache, cudaStream_t st);
 
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates

@@ -51,11 +51,27 @@ cudaError_t launch_both(const CUtensorMap* ms, const tcbwd::scan::Params& sp, co
 
 }  // namespace
 
-TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials) {
+TcCache plan_tc_cache(const Problem& pb) {
+    TcCache c;
+    const size_t st1 = (size_t)pb.B * pb.Hv * (pb.NT + 1) * pb.dk * pb.dv * sizeof(float);
+    const size_t tok = (size_t)pb.B * pb.T * pb.Hv * pb.dv * 2;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = al256(off + bytes);
+        return o;
+    };
+    c.s0 = take(st1);  // entering state of every chunk, then the final state
+    c.vp_hi = take(tok);
+    c.vp_lo = take(tok);
+    c.bytes = off;
+    return c;
+}
+
+TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials, bool caller_cache) {
     TcBwdWs w;
     const size_t nch = (size_t)pb.B * pb.Hv * pb.NT;
     const size_t st = nch * pb.dk * pb.dv * sizeof(float);
-    const size_t st1 = (size_t)pb.B * pb.Hv * (pb.NT + 1) * pb.dk * pb.dv * sizeof(float);
     const size_t tok = (size_t)pb.B * pb.T * pb.Hv * pb.dv * 2;
     const size_t part = (size_t)pb.B * pb.T * pb.Hv * pb.dk * sizeof(float);
     size_t off = 256;  // bytes [0, 256): device status word
@@ -64,10 +80,8 @@ TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials) {
         off = al256(off + bytes);
         return o;
     };
-    w.s0 = take(st1);  // entering state of every chunk, then the final state
+    w.cache = caller_cache ? ~size_t(0) : take(plan_tc_cache(pb).bytes);
     w.dsc = take(st);
-    w.vp_hi = take(tok);
-    w.vp_lo = take(tok);
     w.ny_hi = take(tok);
     w.ny_lo = take(tok);
     w.dq_v = gqa_partials ? take(part) : ~size_t(0);
@@ -77,28 +91,33 @@ TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials) {
 }
 
 cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, bool direct,
-                         const TcBwdWs& plan, void* ws, cudaStream_t st) {
+                         const TcBwdWs& plan, void* ws, const void* cache, cudaStream_t st) {
     char* base = static_cast<char*>(ws);
     int* err = static_cast<int*>(ws);
-    float* s0 = reinterpret_cast<float*>(base + plan.s0);
+    const TcCache cp = plan_tc_cache(pb);
+    char* cb = cache ? static_cast<char*>(const_cast<void*>(cache)) : base + plan.cache;
+    float* s0 = reinterpret_cast<float*>(cb + cp.s0);
+    auto* vph = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_hi);
+    auto* vpl = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_lo);
     float* dsc = reinterpret_cast<float*>(base + plan.dsc);
-    auto* vph = reinterpret_cast<__nv_bfloat16*>(base + plan.vp_hi);
-    auto* vpl = reinterpret_cast<__nv_bfloat16*>(base + plan.vp_lo);
     auto* nyh = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_hi);
     auto* nyl = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_lo);
     float* dq_v = direct ? static_cast<float*>(io.dq) : reinterpret_cast<float*>(base + plan.dq_v);
     float* dk_v = direct ? static_cast<float*>(io.dk) : reinterpret_cast<float*>(base + plan.dk_v);
 
-    // 1. forward in saving mode (no output, no final state)
-    ChunkIO fio = io;
-    fio.o = nullptr;
-    fio.ht = nullptr;
-    fio.z = nullptr;
-    Flags ff = f;
-    ff.gate = false;
-    const TcFwdSave save{s0, vph, vpl};
-    cudaError_t e = tc_chunk_fwd(pb, fio, ff, bf16_gates, err, st, &save);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (!cache) {
+        // 1. forward in saving mode (no output, no final state)
+        ChunkIO fio = io;
+        fio.o = nullptr;
+        fio.ht = nullptr;
+        fio.z = nullptr;
+        Flags ff = f;
+        ff.gate = false;
+        const TcFwdSave save{s0, vph, vpl};
+        e = tc_chunk_fwd(pb, fio, ff, bf16_gates, err, st, &save);
+        if (e != cudaSuccess) return e;
+    }
 
     // 2. maps: q, k, alpha, b, dO, -dY hi/lo, V' hi/lo (unused gate maps copy a valid one)
     CUtensorMap m[9];

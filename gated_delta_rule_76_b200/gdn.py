@@ -31,7 +31,8 @@ class FwdArgs(ctypes.Structure):
                 ("z", P), ("o", P), ("ht", P), ("head_map", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32),
+                ("bwd_cache", P), ("bwd_cache_bytes", ctypes.c_size_t)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -40,7 +41,8 @@ class BwdArgs(ctypes.Structure):
                 ("grad_v", P), ("grad_alpha", P), ("grad_b", P), ("grad_w", P), ("grad_h0", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32)]
+                ("dtype", I32), ("gate_dtype", I32),
+                ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -59,7 +61,7 @@ class LayerArgs(ctypes.Structure):
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
 
 
-EXPORTED = ["gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
+EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
             "gdn_layer_core_fwd", "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches",
             "gdn_version"]
@@ -79,6 +81,8 @@ def load(path: str = LIB_PATH):
     if not os.path.exists(path):
         raise GdnError(f"{path} is missing: build it with `python -m gated_delta_rule_76_b200.build`")
     lib = ctypes.CDLL(path)
+    lib.gdn_chunk_fwd_cache_size.argtypes = [ctypes.POINTER(FwdArgs)]
+    lib.gdn_chunk_fwd_cache_size.restype = ctypes.c_size_t
     lib.gdn_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
     lib.gdn_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_chunk_fwd.argtypes = [ctypes.POINTER(FwdArgs), P, ctypes.c_size_t, P]
@@ -176,7 +180,7 @@ def _head_map(head_map, device):
 # public calls
 # ---------------------------------------------------------------------------------------------
 def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
-             scale: float = 1.0, o=None, ht=None) -> Tuple[FwdArgs, list]:
+             scale: float = 1.0, o=None, ht=None, bwd_cache=None) -> Tuple[FwdArgs, list]:
     """Build the gdn_fwd_args struct (the returned list keeps referenced tensors alive)."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
@@ -187,15 +191,30 @@ def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_ma
                 B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                 alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
                 dtype=_dt(q), gate_dtype=_dt(alpha),
-                out_f32=int(o is not None and o.dtype == torch.float32 and q.dtype != torch.float32))
-    return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm]
+                out_f32=int(o is not None and o.dtype == torch.float32 and q.dtype != torch.float32),
+                bwd_cache=_ptr(bwd_cache),
+                bwd_cache_bytes=0 if bwd_cache is None else bwd_cache.numel() * bwd_cache.element_size())
+    return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm, bwd_cache]
+
+
+def gdn_chunk_fwd_cache_size(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
+                             scale: float = 1.0) -> int:
+    """Bytes of the forward cache gdn_chunk_fwd(..., bwd_cache=) can fill for a later backward
+    (0: this problem runs on the CUDA-core path, which keeps none)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, None, head_map, scale)
+    return int(load().gdn_chunk_fwd_cache_size(ctypes.byref(a)))
 
 
 def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
                   scale: float = 1.0, *, o=None, ht=None, want_ht: bool = True, out_f32: bool = False,
-                  workspace: Optional[torch.Tensor] = None, stream=None):
+                  bwd_cache: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None):
     """Chunkwise forward.  Returns (o [B,T,Hv,dv], ht [B,Hv,dk,dv] or None).
-    ``out_f32`` writes o in fp32 (the unrounded accumulator) instead of the input dtype."""
+    ``out_f32`` writes o in fp32 (the unrounded accumulator) instead of the input dtype.
+    ``bwd_cache``: a device byte tensor of gdn_chunk_fwd_cache_size() bytes that the forward fills
+    for gdn_chunk_bwd(..., fwd_cache=) over the same inputs."""
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     if o is None:
@@ -203,7 +222,7 @@ def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, he
     if ht is None and want_ht:
         ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
     lib = load()
-    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht)
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht, bwd_cache)
     need = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, q.device, workspace)
     check(lib.gdn_chunk_fwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_fwd")
@@ -228,7 +247,7 @@ def gdn_chunk_fwd_noalloc(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=
 
 
 def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, scale=1.0,
-             grad_o=None, grad_ht=None, grads=None) -> Tuple[BwdArgs, list]:
+             grad_o=None, grad_ht=None, grads=None, fwd_cache=None) -> Tuple[BwdArgs, list]:
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
@@ -241,14 +260,18 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
                 grad_w=_ptr(g.get("dw")), grad_h0=_ptr(g.get("dh0")),
                 B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                 alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
-                dtype=_dt(q), gate_dtype=_dt(alpha))
-    return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g]
+                dtype=_dt(q), gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
+                fwd_cache_bytes=0 if fwd_cache is None else fwd_cache.numel() * fwd_cache.element_size())
+    return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g, fwd_cache]
 
 
 def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
                   scale: float = 1.0, *, grad_o, grad_ht=None, want_dh0: bool = True,
-                  workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """Chunkwise backward.  Returns fp32 dq, dk, dv, dalpha and db/dw (or dbeta), dh0."""
+                  fwd_cache: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> Dict[str, torch.Tensor]:
+    """Chunkwise backward.  Returns fp32 dq, dk, dv, dalpha and db/dw (or dbeta), dh0.
+    ``fwd_cache``: the cache a gdn_chunk_fwd(..., bwd_cache=) call filled with these same inputs
+    (the forward is then not recomputed)."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=t.device)
     grads = {"dq": f32(q), "dk": f32(k), "dv": f32(v), "dalpha": f32(alpha)}
@@ -262,7 +285,7 @@ def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=N
         Hv, dv = v.shape[2], v.shape[3]
         grads["dh0"] = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
     lib = load()
-    a, keep = bwd_args(q, k, v, alpha, b, w, beta, h0, head_map, scale, grad_o, grad_ht, grads)
+    a, keep = bwd_args(q, k, v, alpha, b, w, beta, h0, head_map, scale, grad_o, grad_ht, grads, fwd_cache)
     need = lib.gdn_chunk_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, q.device, workspace)
     check(lib.gdn_chunk_bwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_bwd")

@@ -97,8 +97,18 @@ typedef struct gdn_fwd_args {
     int32_t dtype;        /* gdn_dtype of q, k, v, z, o */
     int32_t gate_dtype;   /* gdn_dtype of alpha, b, w */
     int32_t out_f32;      /* 1: o is written in fp32 (unrounded accumulator) instead of dtype */
+    /* Optional cache for a later gdn_chunk_bwd over the same inputs (training): when not NULL the
+     * forward also writes the state entering every chunk, the final state and V' = T (Z - Ehat S0)
+     * of every token into this caller buffer, and a backward given it skips recomputing them.
+     * Needs bwd_cache_bytes >= gdn_chunk_fwd_cache_size(args) and a 256-byte-aligned start; only
+     * the tensor-core path (bf16 q/k/v, dk = dv = 128) keeps a cache: elsewhere the size is 0 and
+     * bwd_cache must be NULL.  The cache is independent of z. */
+    void* bwd_cache;
+    size_t bwd_cache_bytes;
 } gdn_fwd_args;
 
+/* Bytes of the optional forward cache (0 where the problem cannot keep one). */
+GDN_API size_t gdn_chunk_fwd_cache_size(const gdn_fwd_args* args);
 GDN_API size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* args);
 GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size_t workspace_bytes,
                          gdn_stream stream);
@@ -154,6 +164,12 @@ typedef struct gdn_bwd_args {
     int32_t gates_per_channel;
     int32_t dtype;
     int32_t gate_dtype;
+    /* Optional: the cache a gdn_chunk_fwd call wrote with exactly these inputs (q, k, v, alpha, b,
+     * w, h0, head_map, scale, sizes).  The backward then reads the saved chunk states and V' instead
+     * of recomputing the forward.  The library cannot check that the cache belongs to these
+     * inputs: a stale cache gives wrong gradients.  NULL: the forward is recomputed. */
+    const void* fwd_cache;
+    size_t fwd_cache_bytes;
 } gdn_bwd_args;
 
 GDN_API size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args);

@@ -146,3 +146,39 @@ def test_invalid_arguments_raise_on_gpu():
                           o=g["v"])
     with pytest.raises(gdn.GdnError):
         gdn.gdn_chunk_fwd(g["q"].cpu(), g["k"], g["v"], g["alpha"], b=g["b"], w=g["w"])
+
+
+@pytest.mark.parametrize("name", ["gdn2_bf16_ragged", "gdn_scalar_bf16_f32gates_gqa", "one_token",
+                                  "chunk_minus_one"])
+def test_bwd_from_forward_cache_matches_recompute(name):
+    """A forward that fills the cache gives the same o, ht; a backward given the cache gives the
+    same gradients as one that recomputes the forward (the same kernels on the same inputs)."""
+    x, scale = make(name, with_dout=True)
+    g = to_cuda(x)
+    kw = dict(h0=g.get("h0"), scale=scale, **gate_kw(g))
+    nbytes = gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], **kw)
+    assert nbytes > 0
+    cache = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], out_f32=True, bwd_cache=cache, **kw)
+    o_ref, ht_ref = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], out_f32=True, **kw)
+    assert torch.equal(o, o_ref) and torch.equal(ht, ht_ref)
+    with_cache = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], grad_ht=g["dht"],
+                                   fwd_cache=cache, **kw)
+    recompute = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], grad_ht=g["dht"], **kw)
+    torch.cuda.synchronize()
+    for key in with_cache:
+        assert torch.equal(with_cache[key], recompute[key]), key
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["alpha"], h0=x.get("h0"), scale=scale, dout=x["dout"],
+                     dht=x["dht"], **gate_kw(x))
+    for key in ["dq", "dk", "dv", "dalpha", "dh0"] + (["dbeta"] if "beta" in x else ["db", "dw"]):
+        assert_parity(with_cache[key], ref[key], "bf16", key)
+
+
+def test_forward_cache_is_refused_off_the_tensor_core_path():
+    x, scale = make("kda_f32_d128", with_dout=True)
+    g = to_cuda(x)
+    kw = dict(h0=g.get("h0"), scale=scale, **gate_kw(g))
+    assert gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], **kw) == 0
+    cache = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(gdn.GdnError, match="UNSUPPORTED"):
+        gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)

@@ -125,3 +125,17 @@ def test_workspace_size_scales_with_chunks(lib):
     big = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(_fwd(T=65)))
     assert big > small  # a ragged tail adds a chunk
     assert lib.gdn_chunk_fwd_workspace_size(None) == 0
+
+
+def test_forward_cache_validation_on_the_host(lib):
+    # fp32 tensors run on the CUDA-core path, which keeps no cache: size 0, a cache is refused
+    a = _fwd(dtype=1, gate_dtype=1)
+    assert lib.gdn_chunk_fwd_cache_size(ctypes.byref(a)) == 0
+    a = _fwd(dtype=1, gate_dtype=1, bwd_cache=1 << 24, bwd_cache_bytes=1 << 20)
+    rc = lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), 1 << 30, None)
+    assert rc == 2, lib.gdn_last_error()
+    # a cache must start on a 256-byte boundary and may not overlap an output
+    a = _fwd(bwd_cache=(1 << 24) + 16, bwd_cache_bytes=1 << 20)
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), 1 << 30, None) == 1
+    a = _fwd(bwd_cache=1 << 20, bwd_cache_bytes=1 << 20)
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), 1 << 30, None) == 1
