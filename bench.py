@@ -107,7 +107,15 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False):
+# DRAM bytes (read + write) of one gdn_chunk_bwd call on the headline workload, from one ncu capture
+# of its two kernels (reverse scan, gradients) on B=2 T=2048 (an eighth of the workload's tokens:
+# the per-chunk traffic is fixed, so it scales with the tokens); see
+# profiles/chunk_bwd_kernels_gdn2_b2_t2048.md.  To be set to None whenever those kernels change.
+BWD_CALL_TRAFFIC_BYTES = (84.06 + 55.49 + 360.23 + 154.44) * 1e6 * 8
+
+
+def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False,
+             traffic=None):
     t_mem = bytes_per_launch / (peaks["hbm_gbs"] * 1e9)
     fpk = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     t_flop = flops_per_launch / (fpk * 1e12)
@@ -119,7 +127,7 @@ def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scop
         achieved = flops_per_launch / seconds / 1e12
         out = {"bound": "tensor", "achieved": round(achieved, 2), "peak": fpk, "unit": "TFLOP/s",
                "frac": round(achieved / fpk, 4)}
-    out.update({"traffic": None, "peak_source": peak_kind, "scope": scope,
+    out.update({"traffic": None if traffic is None else int(traffic), "peak_source": peak_kind, "scope": scope,
                 "algorithmic_bytes": int(bytes_per_launch), "algorithmic_flops": int(flops_per_launch)})
     return out
 
@@ -329,7 +337,8 @@ def bench_headline(args, dist, peaks, peak_kind, stream, device):
     dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
     dom = {"fwd": (bytes_f, flops_f, fwd_ms), "bwd": (bytes_b, flops_b, bwd_ms)}[dominant]
     roof = roofline(dom[0], dom[1], dom[2] * 1e-3, peaks, peak_kind,
-                    f"gdn_chunk_{dominant} call (dominant call of the step; its kernels back to back)")
+                    f"gdn_chunk_{dominant} call (dominant call of the step; its kernels back to back)",
+                    traffic=BWD_CALL_TRAFFIC_BYTES if dominant == "bwd" else None)
     step_roof = roofline(bytes_f + bytes_b, flops_f + flops_b, ms * 1e-3, peaks, peak_kind,
                          "whole fwd+bwd step")
     return {"ms": ms, "tokens": tokens, "launches_per_step": launches_per_step, "fwd_ms": fwd_ms,
@@ -517,6 +526,44 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------------------------
+def _profile_train_b2_t2048():
+    """GDN-2 training step on B=2 T=2048 H=16 d=128 bf16 (seed 21), twice: the forward keeping the
+    backward cache, then the backward from it."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import draw
+    x = draw(2, 2048, 16, 16, 128, 128, alpha_per_channel=True, gates_per_channel=True, dtype="bf16",
+             gate_dtype="bf16", seed=21, has_h0=True, with_dout=True)
+    g = {k: v.cuda() for k, v in x.items()}
+    kw = dict(b=g["b"], w=g["w"], h0=g["h0"])
+    cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], **kw),
+                        dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
+        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache, **kw)
+    torch.cuda.synchronize()
+    print("ok", float(grads["dq"].abs().mean()))
+    return 0
+
+
+def _profile_fwd_b8_t1024():
+    """GDN-2 forward on B=8 T=1024 H=16 d=128 bf16 (seed 21), twice, without a cache."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import draw
+    x = draw(8, 1024, 16, 16, 128, 128, alpha_per_channel=True, gates_per_channel=True, dtype="bf16",
+             gate_dtype="bf16", seed=21, has_h0=True)
+    g = {k: v.cuda() for k, v in x.items()}
+    for _ in range(2):
+        o, _ = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], b=g["b"], w=g["w"], h0=g["h0"])
+    torch.cuda.synchronize()
+    print("ok", float(o.float().abs().mean()))
+    return 0
+
+
+PROFILE_CASES = {"train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -525,7 +572,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--parts", default="all", help="all | headline | comma list of: decode,fwd,gdn,layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None, choices=sorted(PROFILE_CASES),
+                    help="run one small untimed case for an ncu capture (prints 'ok') and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        return PROFILE_CASES[args.profile_case]()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
@@ -562,9 +613,13 @@ def main():
         torch.cuda.empty_cache()
     sub = {}
     if "fwd" in parts:
-        sub["gdn2_fwd"] = {"workload": HEADLINE, "value": head["tokens"] / (head["fwd_ms"] * 1e-3) * dist.world,
-                           "unit": "tokens/s", "ms_per_step": round(head["fwd_ms"], 4),
-                           "roofline": head["fwd_roofline"]}
+        # the forward alone (inference: no backward cache), then the training step's forward
+        sub["gdn2_fwd"] = bench_part_fwd(HEADLINE, args, dist, peaks, peak_kind, stream, device)
+        torch.cuda.empty_cache()
+        sub["gdn2_fwd_keeping_cache"] = {"workload": HEADLINE,
+                                         "value": head["tokens"] / (head["fwd_ms"] * 1e-3) * dist.world,
+                                         "unit": "tokens/s", "ms_per_step": round(head["fwd_ms"], 4),
+                                         "roofline": head["fwd_roofline"]}
     if "gdn" in parts:
         sub["gdn_fwd_scalar"] = bench_part_fwd("gdn_fwd_scalar_bf16", args, dist, peaks, peak_kind, stream, device)
         torch.cuda.empty_cache()
