@@ -1100,7 +1100,7 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
                                                 float gam, float xtot, float* scr, int it) {
     const float scale = p.pb.scale;
     const RowPtrs rp = row_ptrs(p, cp, c);
-    float G = gam, run = 0.f;
+    float G = gam, rg = __fdividef(1.f, gam), run = 0.f;
     auto do_block = [&](int blk, const RowIn& x) {
         uint32_t rq[RB], re[RB], rk[RB], rb[RB];
         tmem_ld8(tl + TM_P7 + RB * blk, rq);
@@ -1112,7 +1112,7 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
         for (int i = RB - 1; i >= 0; --i) {
             const int r = RB * blk + i;
             const float qv = x.q[i], kv = x.k[i], bv = x.b[i];
-            const float ra = __fdividef(1.f, x.a[i]), rg = __fdividef(1.f, G);
+            const float ra = __fdividef(1.f, x.a[i]);
             const float dQh = __uint_as_float(rq[i]), dEh = __uint_as_float(re[i]);
             const float dkc = fmaf(gam, __uint_as_float(rb[i]), __uint_as_float(rk[i]));
             const float de = G * dEh;
@@ -1132,7 +1132,8 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
                 const float sum = warp_sum(dla);
                 if ((c & 31) == 0) scr[SX_RA / 4 + warp * 64 + r] = sum;
             }
-            G *= ra;  // Gamma_{r-1} = Gamma_r / alpha_r
+            G *= ra;       // Gamma_{r-1} = Gamma_r / alpha_r
+            rg *= x.a[i];  // 1 / Gamma_{r-1}
         }
     };
     // two input buffers: a block's loads are in flight while the previous block is formed
