@@ -482,27 +482,42 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     cudaError_t e0 = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
     if (e0 != cudaSuccess) return cuda_fail(e0, "gdn_layer_core_fwd");
     char* base = static_cast<char*>(workspace) + 256;
-    void* qc = base;
-    void* kc = base + BT * a->Hk * a->dk * 4;
-    void* vc = base + 2 * BT * a->Hk * a->dk * 4;
     const size_t conv_bytes = align256(BT * cch * 4);
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
+    // The conv outputs are fp32 values.  With scalar gates and bf16 tensors they go to the
+    // tensor-core forward as bf16 hi/lo pairs (same bytes); otherwise they stay fp32 for the
+    // CUDA-core forward.
+    const bool split = a->dtype == GDN_BF16 && !f.apc && !f.gpc &&
+                       tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
+    const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
     ConvParams cp{};
     cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
-    cp.q = qc; cp.k = kc; cp.v = vc; cp.conv_state_out = a->conv_state_out;
+    if (split) {
+        cp.q = base; cp.q_lo = base + qn * 2;
+        cp.k = base + qn * 4; cp.k_lo = base + qn * 6;
+        cp.v = base + qn * 8; cp.v_lo = base + qn * 8 + vn * 2;
+    } else {
+        cp.q = base; cp.k = base + qn * 4; cp.v = base + qn * 8;
+    }
+    cp.conv_state_out = a->conv_state_out;
     cp.B = (int)a->B; cp.T = (int)a->T; cp.Hk = (int)a->Hk; cp.Hv = (int)a->Hv; cp.d = (int)a->dk;
     const int var = variant(a->dtype, a->gate_dtype);
     cudaError_t e = var == 2 ? f32_conv(cp, sm) : bf16_conv(cp, sm);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_fwd (conv)");
-    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    WsPlan plan = plan_chunk_ws(pb, false, false);
     ChunkIO io{};
-    io.q = qc; io.k = kc; io.v = vc; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.z = a->z;
+    io.q = cp.q; io.k = cp.k; io.v = cp.v; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.z = a->z;
     io.h0 = a->h0; io.o = a->y; io.ht = a->ht;
-    // fp32 intermediates: y is written in dtype (bf16 -> o_type 2) unless out_f32.
+    // y is written in dtype (bf16 -> o_type 2) unless out_f32.
     io.o_type = a->out_f32 || a->dtype == GDN_F32 ? 1 : 2;
     io.z_bf16 = a->dtype == GDN_BF16;
-    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
-    e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
+    if (split) {
+        io.q_lo = cp.q_lo; io.k_lo = cp.k_lo; io.v_lo = cp.v_lo;
+        e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm);
+    } else {
+        WsPlan plan = plan_chunk_ws(pb, false, false);
+        e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
+    }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
 }
 

@@ -121,14 +121,11 @@ cudaError_t decode_conv_shift(const DecodeParams& p, cudaStream_t st) {
 
 template <class TIn>
 cudaError_t conv_impl(const ConvParams& p, cudaStream_t st) {
-    const long rows = (long)p.B * p.T * (2L * p.Hk + p.Hv);
-    const long blocks = (rows * 32 + 255) / 256;
-    if (p.d == 128)
-        return launch_kernel(conv_silu_l2_kernel<TIn, float, 128>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
-                             st, p);
-    if (p.d == 64)
-        return launch_kernel(conv_silu_l2_kernel<TIn, float, 64>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
-                             st, p);
+    const dim3 grid((unsigned)((p.T + kConvTile - 1) / kConvTile), (unsigned)((2 * p.Hk + p.Hv + 3) / 4), (unsigned)p.B);
+    if (p.d == 128 && p.q_lo)
+        return launch_kernel(conv_silu_l2_kernel<TIn, __nv_bfloat16, 128, true>, grid, dim3(128), 0, st, p);
+    if (p.d == 128) return launch_kernel(conv_silu_l2_kernel<TIn, float, 128>, grid, dim3(128), 0, st, p);
+    if (p.d == 64) return launch_kernel(conv_silu_l2_kernel<TIn, float, 64>, grid, dim3(128), 0, st, p);
     return cudaErrorInvalidValue;
 }
 

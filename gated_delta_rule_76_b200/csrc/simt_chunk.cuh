@@ -48,6 +48,8 @@ struct ChunkWs {
 
 struct ChunkIO {
     const void *q, *k, *v, *alpha, *b, *w, *z;
+    // Tensor-core forward only: fp32 q, k, v given as bf16 pairs, q = q + q_lo etc. (NULL: plain)
+    const void *q_lo, *k_lo, *v_lo;
     const float* h0;
     void* o;
     int o_type;  // 0: o in TIn, 1: fp32, 2: bf16

@@ -91,7 +91,8 @@ constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats (chunk n us
 constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, abort flag
 constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: alpha products per row group [8][128], then the
                                           // block-row products of the solve [16][LDR]
-constexpr uint32_t SM_END = SM_RS + 4096;
+constexpr uint32_t SM_SG = SM_RS + 4096;  // scalar gates of a chunk: [2 slots][alpha, beta][64] fp32
+constexpr uint32_t SM_END = SM_SG + 1024;
 constexpr int LDA = 68;  // fp32 row stride of the A/T scratch: float4 rows, rows 16 B apart in bank
 constexpr int LDR = 52;  // fp32 row stride of the block-row products
 constexpr size_t kSmemBytes = SM_END + 1024;
@@ -179,9 +180,10 @@ __device__ __forceinline__ void solve_block_row(float* t, float* rsb, int c) {
     if (act) {
         float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
         const float* a0p = t + row * LDA;
-        // T_{0:IB, jb} is zero above its diagonal block: start at row 16 jb of the column block.
-#pragma unroll 1
-        for (int kk = 16 * (col >> 4); kk < 16 * IB; kk += 4) {
+        // T_{0:IB, 0:IB} is lower triangular and the scratch holds zeros above it, so the sum runs
+        // over all 16 IB rows with compile-time bounds: fully unrolled, every load is issued early.
+#pragma unroll
+        for (int kk = 0; kk < 16 * IB; kk += 4) {
             const float4 a0 = ldf4(a0p + kk), a1 = ldf4(a0p + LDA + kk);
             const float4 t0 = ldf4(t + (kk + 0) * LDA + col), t1 = ldf4(t + (kk + 1) * LDA + col);
             const float4 t2 = ldf4(t + (kk + 2) * LDA + col), t3 = ldf4(t + (kk + 3) * LDA + col);
@@ -246,43 +248,70 @@ __device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint6
         : "memory");
 }
 
-template <bool APC, bool GPC>
+// Raw tiles of chunk n.  With SPLIT (scalar gates only) q, k, v arrive as bf16 hi + lo pairs of
+// fp32 values; the lo halves take the tiles that scalar gates leave free: q lo the b rows of RQB,
+// k lo the alpha tile, v lo the w tile (the maps in the tb_, ta and tw slots point at them).
+template <bool APC, bool GPC, bool SPLIT>
 __device__ __forceinline__ void load_raw(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
                                          const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_) {
+    static_assert(!SPLIT || (!APC && !GPC), "split inputs use the gate tiles");
     const int t0 = n * C;
     const uint32_t base = smem_u32(cx.sm);
     uint64_t* bar = cx.bars + B_RAW;
-    mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
+    mbar_arrive_expect_tx(bar, 32768u + (GPC || SPLIT ? 16384u : 0u) + (APC || SPLIT ? 16384u : 0u));
     tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);           // q -> rows 64-127, channels 0-63
     tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);  // channels 64-127
     tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
     tma4(base + SM_RK + 8192, tk, bar, 64, hk, t0, b);
-    if (GPC) {
-        tma4(base + SM_RQB, tb_, bar, 0, hv, t0, b);              // b -> rows 0-63
-        tma4(base + SM_RQB + 16384, tb_, bar, 64, hv, t0, b);
+    if (GPC || SPLIT) {
+        const int hb = SPLIT ? hk : hv;
+        tma4(base + SM_RQB, tb_, bar, 0, hb, t0, b);              // b (or q lo) -> rows 0-63
+        tma4(base + SM_RQB + 16384, tb_, bar, 64, hb, t0, b);
     }
-    if (APC) {
-        tma4(base + SM_RA, ta, bar, 0, hv, t0, b);
-        tma4(base + SM_RA + 8192, ta, bar, 64, hv, t0, b);
+    if (APC || SPLIT) {
+        const int ha = SPLIT ? hk : hv;
+        tma4(base + SM_RA, ta, bar, 0, ha, t0, b);                // alpha (or k lo)
+        tma4(base + SM_RA + 8192, ta, bar, 64, ha, t0, b);
     }
 }
 
-template <bool GPC>
+// L2 prefetch of the tiles load_raw reads for chunk n (no shared memory, no barrier), issued one
+// chunk ahead so that the load, which waits for the previous chunk's readers, finds them in L2.
+__device__ __forceinline__ void tma_prefetch4(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+template <bool APC, bool GPC, bool SPLIT>
+__device__ __forceinline__ void prefetch_raw(int n, int b, int hk, int hv, const CUtensorMap* tq,
+                                             const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_) {
+    const int t0 = n * C;
+#pragma unroll
+    for (int c0 = 0; c0 < 128; c0 += 64) {
+        tma_prefetch4(tq, c0, hk, t0, b);
+        tma_prefetch4(tk, c0, hk, t0, b);
+        if (GPC || SPLIT) tma_prefetch4(tb_, c0, SPLIT ? hk : hv, t0, b);
+        if (APC || SPLIT) tma_prefetch4(ta, c0, SPLIT ? hk : hv, t0, b);
+    }
+}
+
+template <bool GPC, bool SPLIT>
 __device__ __forceinline__ void load_vw(const Ctx& cx, int n, int b, int hv, const CUtensorMap* tv,
                                         const CUtensorMap* tw) {
     const int t0 = n * C;
     const uint32_t vw = smem_u32(cx.sm) + SM_VW;
     uint64_t* bar = cx.bars + B_VW;
-    mbar_arrive_expect_tx(bar, GPC ? 32768u : 16384u);
+    mbar_arrive_expect_tx(bar, GPC || SPLIT ? 32768u : 16384u);
     tma4(vw, tv, bar, 0, hv, t0, b);
     tma4(vw + 8192, tv, bar, 64, hv, t0, b);
-    if (GPC) {
-        tma4(vw + 16384, tw, bar, 0, hv, t0, b);
+    if (GPC || SPLIT) {
+        tma4(vw + 16384, tw, bar, 0, hv, t0, b);                  // w (or v lo)
         tma4(vw + 16384 + 8192, tw, bar, 64, hv, t0, b);
     }
 }
 
-template <bool APC, bool GPC, bool GATE, class TG>
+template <bool APC, bool GPC, bool GATE, class TG, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -320,8 +349,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     if (tid == 0) {
-        load_raw<APC, GPC>(cx, 0, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
-        load_vw<GPC>(cx, 0, b, hv, &tm_v, &tm_w);
+        load_raw<APC, GPC, SPLIT>(cx, 0, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+        load_vw<GPC, SPLIT>(cx, 0, b, hv, &tm_v, &tm_w);
     }
     int raw_issued = 1, vw_issued = 1;  // meaningful in the issuing threads only
 
@@ -364,6 +393,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
             }
+            if (GATE && tid < 128 && t0 + (tid >> 1) < pb.T) {
+                // the output epilogue's z rows of this chunk into L2 (two 128-byte lines a token)
+                prefetch_line_l2(static_cast<const __nv_bfloat16*>(p.z) + pb.v_row(b, t0 + (tid >> 1), hv) +
+                                 64 * (tid & 1));
+            }
             // ---- X2 = S0^T [Ehat;Qhat]^T  (S0 split; Qhat split in the Qhat half) ------------------
             if (tid == 0) {
                 GDN_TRACE(n, 0);
@@ -389,6 +423,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tmem_ld32(tl + TM_X2 + 32 * h, r);
                 tmem_ld_wait();
                 const uint8_t* vt = sm + SM_VW + vbase + 32u * h * 128u;
+                const float* sgb = reinterpret_cast<const float*>(sm + SM_SG) + pn * 128 + 64;
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -397,10 +432,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int e = 0; e < 2; ++e) {
                         const int ii = 2 * i + e, rr = 32 * h + ii;
                         const uint32_t off = (uint32_t)ii * 128u + xo[ii & 7];
-                        const float vv = bf(vt, off);
+                        const float vv = SPLIT ? bf(vt, off) + bf(vt + 16384, off) : bf(vt, off);
                         float ww;
                         if (GPC) ww = bf(vt + 16384, off);
-                        else ww = gate_or(beta, pb, b, t0, rr, L, hv, 0.f);
+                        else ww = sgb[rr];
                         y2[e] = vv * ww - __uint_as_float(r[ii]);
                     }
                     split_pack(y2[0], y2[1], hi[i], lo[i]);
@@ -469,7 +504,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // X1 and the Kbar^T pass were the last readers of the raw stage: load the next chunk's.
             if (tid == 0) GDN_TRACE(n, 9);
             if (tid == 0 && raw_issued < NT && !*cx.abort_flag) {
-                load_raw<APC, GPC>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                load_raw<APC, GPC, SPLIT>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
                 ++raw_issued;
             }
             // ---- X3 = Y^T T^T = V'^T; v/w of the next chunk --------------------------------------
@@ -477,7 +512,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 GDN_TRACE(n, 4);
                 tc_fence_after();
                 if (vw_issued < NT && !*cx.abort_flag) {
-                    load_vw<GPC>(cx, vw_issued, b, hv, &tm_v, &tm_w);
+                    load_vw<GPC, SPLIT>(cx, vw_issued, b, hv, &tm_v, &tm_w);
                     ++vw_issued;
                 }
                 if (wait1(cx, B_T_READY, pn) && !*cx.abort_flag) {
@@ -554,14 +589,15 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float ov[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] = pb.scale * __uint_as_float(r[i]);
-                if (GATE) {
+                if (GATE && nrow > 0) {
+                    // Clamped, branch-free loads (a load under a per-token branch would be waited
+                    // for at the end of that branch, one token at a time).
                     const __nv_bfloat16* zp = static_cast<const __nv_bfloat16*>(p.z) + obase;
+                    float zz[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < nrow) {
-                            const float zz = __bfloat162float(zp[i * orow]);
-                            ov[i] *= zz * sigmoidf_(zz);
-                        }
+                    for (int i = 0; i < 32; ++i) zz[i] = __bfloat162float(zp[(long)min(i, nrow - 1) * orow]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] *= zz[i] * sigmoidf_(zz[i]);
                 }
                 if (p.o_type == 1) {
                     float* op = static_cast<float*>(p.o) + obase;
@@ -635,12 +671,33 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint8_t* EQ = sm + SM_EQ;
         uint8_t* QLO = sm + SM_QLO;
         const uint32_t id64 = idesc_bf16_f32(128, 64);
+        float ga_next = 1.f, gb_next = 0.f;  // scalar gates of the next chunk (threads c < 64)
+        const float* sga = reinterpret_cast<const float*>(sm + SM_SG);
         for (int m = 0; m < NT; ++m) {
             const uint32_t pm = m & 1, pprev = (m - 1) & 1;
             const int t0 = m * C, L = min(C, pb.T - t0);
+            if (!APC || !GPC) {
+                // Scalar gates of chunk m into slot m & 1 (the scan reads beta there); the next
+                // chunk's are loaded now and held in registers, so their latency is hidden.
+                float* sg = reinterpret_cast<float*>(sm + SM_SG) + pm * 128;
+                if (c < 64) {
+                    if (m == 0) {
+                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t0, c, L, hv, 1.f);
+                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t0, c, L, hv, 0.f);
+                    }
+                    sg[c] = ga_next;
+                    sg[64 + c] = gb_next;
+                    if (m + 1 < NT) {
+                        const int t1 = t0 + C, L1 = min(C, pb.T - t1);
+                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t1, c, L1, hv, 1.f);
+                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t1, c, L1, hv, 0.f);
+                    }
+                }
+            }
             if (c == 0) {
                 GDN_TRACE(m, 16);
                 wait1(cx, B_RAW, pm);
+                if (m + 1 < NT) prefetch_raw<APC, GPC, SPLIT>(m + 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
                 GDN_TRACE(m, 17);
                 if (m > 0) wait1(cx, B_EQ_FREE, pprev);
                 GDN_TRACE(m, 18);
@@ -669,7 +726,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             for (int i = 0; i < 8; ++i) a8[i] = 1.f;
                         }
                     } else {
-                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+                        const float av = sga[pm * 128 + r];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) a8[i] = av;
                     }
@@ -710,16 +767,26 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             for (int i = 0; i < 8; ++i) a8[i] = 1.f;
                         }
                     } else {
-                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+                        const float av = sga[pm * 128 + r];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) a8[i] = av;
                     }
                     unpack8(ld16(RK + o64), k8);
                     unpack8(ld16(RQB + oq), q8);
+                    if (SPLIT) {
+                        float kl[8], ql[8];
+                        unpack8(ld16(RA + o64), kl);
+                        unpack8(ld16(RQB + oe), ql);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            k8[i] += kl[i];
+                            q8[i] += ql[i];
+                        }
+                    }
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
                     } else {
-                        const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f);
+                        const float bv = sga[pm * 128 + 64 + r];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) b8[i] = bv;
                     }

@@ -11,9 +11,9 @@ namespace gdn {
 
 namespace {
 
-template <bool APC, bool GPC, bool GATE, class TG>
+template <bool APC, bool GPC, bool GATE, class TG, bool SPLIT = false>
 cudaError_t launch_tc(const CUtensorMap* maps, const tcfwd::Params& p, cudaStream_t st) {
-    auto kernel = tcfwd::chunk_fwd_kernel<APC, GPC, GATE, TG>;
+    auto kernel = tcfwd::chunk_fwd_kernel<APC, GPC, GATE, TG, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcfwd::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -39,6 +39,8 @@ bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags
 cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
                          cudaStream_t st, const TcFwdSave* save) {
     CUtensorMap maps[6];
+    const bool split = io.q_lo != nullptr;
+    if (split && (f.apc || f.gpc || !io.k_lo || !io.v_lo)) return cudaErrorInvalidValue;
     bool ok = make_map(&maps[0], io.q, pb.B, pb.T, pb.Hk) && make_map(&maps[1], io.k, pb.B, pb.T, pb.Hk) &&
               make_map(&maps[2], io.v, pb.B, pb.T, pb.Hv);
     // Unused maps are copies of a valid one (never dereferenced).
@@ -47,6 +49,10 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     maps[5] = maps[2];
     if (ok && f.apc) ok = make_map(&maps[3], io.alpha, pb.B, pb.T, pb.Hv);
     if (ok && f.gpc) ok = make_map(&maps[4], io.b, pb.B, pb.T, pb.Hv) && make_map(&maps[5], io.w, pb.B, pb.T, pb.Hv);
+    // Split inputs: the lo halves take the gate slots (k lo: alpha, q lo: b, v lo: w).
+    if (ok && split)
+        ok = make_map(&maps[3], io.k_lo, pb.B, pb.T, pb.Hk) && make_map(&maps[4], io.q_lo, pb.B, pb.T, pb.Hk) &&
+             make_map(&maps[5], io.v_lo, pb.B, pb.T, pb.Hv);
     if (!ok) return cudaErrorInvalidValue;
     tcfwd::Params p{};
     p.pb = pb;
@@ -64,6 +70,12 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
         p.vp_lo = save->vp_lo;
     }
     const bool gate = f.gate;
+    if (split) {
+        // the layer core's form: scalar gates and the swish output gate
+        if (!gate) return cudaErrorInvalidValue;
+        return bf16_gates ? launch_tc<false, false, true, __nv_bfloat16, true>(maps, p, st)
+                          : launch_tc<false, false, true, float, true>(maps, p, st);
+    }
     if (f.apc && f.gpc) return launch_tc_g<true, true, __nv_bfloat16>(gate, maps, p, st);
     if (f.apc) return launch_tc_g<true, false, __nv_bfloat16>(gate, maps, p, st);
     if (f.gpc) return launch_tc_g<false, true, __nv_bfloat16>(gate, maps, p, st);

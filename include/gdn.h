@@ -221,6 +221,9 @@ GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, gdn_stream strea
  * Convolution channels are ordered q (Hk*dk), k (Hk*dk), v (Hv*dv); conv_w is [Cch, 4] with
  * conv_w[ch][3] weighting the current token.  conv_state_out, if not NULL, receives the last
  * three raw inputs of every channel ([B, Cch, 3], dtype) so that decoding can continue.
+ * The convolution outputs are fp32 values kept in the workspace.  With bf16 tensors, dk = dv =
+ * 128 and scalar gates they are stored as bf16 hi/lo pairs (x = hi + lo to 16 mantissa bits) and
+ * the tensor-core chunk forward consumes them; otherwise they stay fp32 for the CUDA-core forward.
  * ------------------------------------------------------------------------------------------ */
 typedef struct gdn_layer_args {
     const void* xq;       /* [B,T,Hk,dk] dtype (pre-convolution projections) */

@@ -112,3 +112,26 @@ def test_layer_core_matches_oracle(apc, gpc):
     assert_parity(ht, ht_ref, "bf16", "ht")
     raw = torch.cat([x["q"].reshape(B, T, -1), x["k"].reshape(B, T, -1), x["v"].reshape(B, T, -1)], 2)
     assert torch.equal(cs.cpu(), raw[:, -3:].permute(0, 2, 1).contiguous())
+
+
+@pytest.mark.parametrize("B,T,Hk,Hv,gdt", [(1, 200, 2, 8, "f32"), (2, 129, 1, 2, "bf16"), (1, 64, 1, 1, "f32")])
+def test_layer_core_tensor_core_path(B, T, Hk, Hv, gdt):
+    """d = 128 with scalar gates: the conv kernel hands the tensor-core forward its fp32 outputs as
+    bf16 hi/lo pairs (two launches: conv, chunk forward).  Several chunks, a ragged tail, GQA."""
+    d = 128
+    x = draw(B, T, Hk, Hv, d, d, alpha_per_channel=False, gates_per_channel=False, dtype="bf16",
+             gate_dtype=gdt, seed=37, has_h0=True, conv=True, swish_gate=True)
+    g = to_cuda(x)
+    n0 = gdn.kernel_launches()
+    y, ht, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], beta=g["beta"],
+                                      h0=g["h0"], scale=0.8, out_f32=True)
+    torch.cuda.synchronize()
+    assert gdn.kernel_launches() - n0 == 2, "conv + tensor-core forward"
+    y16, _, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], beta=g["beta"],
+                                       h0=g["h0"], scale=0.8)
+    torch.cuda.synchronize()
+    assert_bf16_is_rounding(y16, y, "y")
+    y_ref, ht_ref = oracle.layer_core_fwd(x["q"], x["k"], x["v"], x["conv_w"], x["alpha"], x["beta"], x["z"],
+                                          scale=0.8, h0=x["h0"])
+    assert_parity(y, y_ref, "bf16", "y")
+    assert_parity(ht, ht_ref, "bf16", "ht")
