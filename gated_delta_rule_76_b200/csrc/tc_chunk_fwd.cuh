@@ -81,7 +81,7 @@ constexpr uint32_t SM_RQB = 0;        // 32 KB [2 atoms][128 rows]: TMA b (rows 
 constexpr uint32_t SM_RK = 32768;     // 16 KB [2][64]: TMA k -> Ktil hi
 constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo
 constexpr uint32_t SM_EQ = 65536;     // 32 KB [2][128]: [Ehat;Qhat] hi
-constexpr uint32_t SM_QLO = 98304;    // 16 KB [2][64]: Qhat lo (for X2)
+constexpr uint32_t SM_Z = 98304;      // 16 KB [2][64]: TMA z tile of the scan's chunk (gated output)
 constexpr uint32_t SM_T = 114688;     // 8 KB [1][64]: T
 constexpr uint32_t SM_P = 122880;     // 16 KB: P hi [1][64], P lo [1][64]
 constexpr uint32_t SM_KB = 139264;    // 32 KB: Kbar^T hi [1][128], Kbar^T lo [1][128]
@@ -108,6 +108,7 @@ enum Bar {
     B_X2A,
     B_X3,
     B_X45,
+    B_Z,            // z tile of the scan's chunk landed (gated output)
     B_COUNT
 };
 
@@ -315,7 +316,8 @@ template <bool APC, bool GPC, bool GATE, class TG, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w, Params p) {
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_w,
+                 const __grid_constant__ CUtensorMap tm_z, Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // Offset arithmetic on the shared array keeps the pointer in the shared state space, so the
     // compiler emits shared loads/stores and knows they cannot alias global memory.
@@ -352,7 +354,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         load_raw<APC, GPC, SPLIT>(cx, 0, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
         load_vw<GPC, SPLIT>(cx, 0, b, hv, &tm_v, &tm_w);
     }
-    int raw_issued = 1, vw_issued = 1;  // meaningful in the issuing threads only
+    int raw_issued = 1, vw_issued = 1, z_issued = 0;  // meaningful in thread 0 only
 
     if (warp < 8) {
         // =================================== state scan ===================================
@@ -393,10 +395,13 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
             }
-            if (GATE && tid < 128 && t0 + (tid >> 1) < pb.T) {
-                // the output epilogue's z rows of this chunk into L2 (two 128-byte lines a token)
-                prefetch_line_l2(static_cast<const __nv_bfloat16*>(p.z) + pb.v_row(b, t0 + (tid >> 1), hv) +
-                                 64 * (tid & 1));
+            if (GATE && tid == 0 && !*cx.abort_flag) {
+                // z of this chunk for the output epilogue (the previous chunk's reads are done)
+                const uint32_t zd = sbase + SM_Z;
+                mbar_arrive_expect_tx(cx.bars + B_Z, 16384u);
+                tma4(zd, &tm_z, cx.bars + B_Z, 0, hv, t0, b);
+                tma4(zd + 8192, &tm_z, cx.bars + B_Z, 64, hv, t0, b);
+                ++z_issued;
             }
             // ---- X2 = S0^T [Ehat;Qhat]^T  (S0 split; Qhat split in the Qhat half) ------------------
             if (tid == 0) {
@@ -407,11 +412,51 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_ts_u<128, 128>(tbase + TM_X2, tbase + TM_S0H, sbase + SM_EQ, id128, false);
                     mma_ts_u<128, 128>(tbase + TM_X2, tbase + TM_S0L, sbase + SM_EQ, id128, true);
                     mma_commit(cx.bars + B_X2A);
-                    mma_ts_u<128, 64>(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_QLO, id64, true);
+                    // Qhat lo: rows 64-127 of the [Ehat;Qhat] lo tile
+                    mma_ts_u<128, 128>(tbase + TM_X2 + 64, tbase + TM_S0H, sbase + SM_RQB + 8192, id64, true);
                     mma_commit(cx.bars + B_EQ_FREE);
-                    wait1(cx, B_X2A, pn);
-                    GDN_TRACE(n, 2);
                 }
+            }
+            // The prologue's Ktil and gamma of this chunk are in shared memory (EQ_READY).
+            named_bar(1, 256);
+            // ---- Kbar^T of this chunk (operand of X5), while X2 runs --------------------------------
+            {
+                // Kbar^T row j, tokens 32 h .. 32 h + 31: (Ktil hi + lo) * gamma, split.
+                uint8_t* KB = sm + SM_KB;
+                const uint8_t* RK = sm + SM_RK;
+                const uint8_t* RA = sm + SM_RA;
+                const float G = gam[(n % 3) * 128 + j];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int ch = 4 * h + cc;
+                    uint32_t wh[4], wl[4];
+                    const uint32_t ob = vbase + (uint32_t)ch * 1024u;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t o0 = ob + (2 * e) * 128u + xo[2 * e];
+                        const uint32_t o1 = ob + (2 * e + 1) * 128u + xo[2 * e + 1];
+                        const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
+                        split_pack(k0, k1, wh[e], wl[e]);
+                    }
+                    const uint32_t off = sw128_offset(j, 8 * ch, 128);
+                    st16(KB + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                    st16(KB + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                }
+            }
+            tc_fence_before();
+            fence_async_shared();
+            named_bar(1, 256);
+            if (tid == 0) {
+                tc_fence_after();
+                // X1 and the Kbar^T pass were the last readers of the raw stage: load the next chunk's.
+                wait1(cx, B_X1, pn);
+                GDN_TRACE(n, 8);
+                if (raw_issued < NT && !*cx.abort_flag) {
+                    load_raw<APC, GPC, SPLIT>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                    ++raw_issued;
+                }
+                wait1(cx, B_X2A, pn);
+                GDN_TRACE(n, 2);
                 wait1(cx, B_VW, pn);
                 GDN_TRACE(n, 3);
             }
@@ -444,15 +489,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tmem_st16(tl + TM_YL + 16 * h, lo);
                 tmem_st_wait();
             }
-            // ---- P and Kbar^T of this chunk (operands of X4, X5) while the prologue solves for T ----
-            if (tid == 0) {
-                tc_fence_after();
-                wait1(cx, B_X1, pn);
-                GDN_TRACE(n, 8);
-            }
-            tc_fence_before();
-            named_bar(1, 256);
-            tc_fence_after();
+            // ---- P of this chunk (operand of X4); X1 completed before the Y step --------------------
             if (j >= 64) {
                 // P row j - 64 (lanes 64-127 of X1), columns 32 h .. 32 h + 31, lower with diagonal.
                 const int rr = j - 64;
@@ -475,38 +512,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     st16(Ph + 8192 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
                 }
             }
-            {
-                // Kbar^T row j, tokens 32 h .. 32 h + 31: (Ktil hi + lo) * gamma, split.
-                uint8_t* KB = sm + SM_KB;
-                const uint8_t* RK = sm + SM_RK;
-                const uint8_t* RA = sm + SM_RA;
-                const float G = gam[(n % 3) * 128 + j];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int ch = 4 * h + cc;
-                    uint32_t wh[4], wl[4];
-                    const uint32_t ob = vbase + (uint32_t)ch * 1024u;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t o0 = ob + (2 * e) * 128u + xo[2 * e];
-                        const uint32_t o1 = ob + (2 * e + 1) * 128u + xo[2 * e + 1];
-                        const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
-                        split_pack(k0, k1, wh[e], wl[e]);
-                    }
-                    const uint32_t off = sw128_offset(j, 8 * ch, 128);
-                    st16(KB + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
-                    st16(KB + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
-                }
-            }
             tc_fence_before();
             fence_async_shared();
             named_bar(1, 256);
-            // X1 and the Kbar^T pass were the last readers of the raw stage: load the next chunk's.
-            if (tid == 0) GDN_TRACE(n, 9);
-            if (tid == 0 && raw_issued < NT && !*cx.abort_flag) {
-                load_raw<APC, GPC, SPLIT>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
-                ++raw_issued;
-            }
             // ---- X3 = Y^T T^T = V'^T; v/w of the next chunk --------------------------------------
             if (tid == 0) {
                 GDN_TRACE(n, 4);
@@ -576,6 +584,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     wait1(cx, B_X45, pn);
                     GDN_TRACE(n, 10);
                 }
+                if (GATE) wait1(cx, B_Z, pn);
             }
             named_bar(1, 256);
             tc_fence_after();
@@ -589,15 +598,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float ov[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] = pb.scale * __uint_as_float(r[i]);
-                if (GATE && nrow > 0) {
-                    // Clamped, branch-free loads (a load under a per-token branch would be waited
-                    // for at the end of that branch, one token at a time).
-                    const __nv_bfloat16* zp = static_cast<const __nv_bfloat16*>(p.z) + obase;
-                    float zz[32];
+                if (GATE) {
+                    // z column j, rows 32h .. 32h + 31, from the TMA tile (zero past the end)
+                    const uint8_t* zt = sm + SM_Z + vbase + 32u * h * 128u;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) zz[i] = __bfloat162float(zp[(long)min(i, nrow - 1) * orow]);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] *= zz[i] * sigmoidf_(zz[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        const float zz = bf(zt, (uint32_t)i * 128u + xo[i & 7]);
+                        ov[i] *= zz * __fdividef(1.f, 1.f + __expf(-zz));
+                    }
                 }
                 if (p.o_type == 1) {
                     float* op = static_cast<float*>(p.o) + obase;
@@ -612,6 +620,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             // ---- state: S = Diag(gamma) S0 + Kbar^T V'; split S0^T for the next chunk -------------
+            if (tid == 0) GDN_TRACE(n, 13);
             {
                 const float4* g4 = reinterpret_cast<const float4*>(gam + (n % 3) * 128 + 64 * h);
 #pragma unroll
@@ -669,7 +678,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint8_t* RK = sm + SM_RK;
         uint8_t* RA = sm + SM_RA;
         uint8_t* EQ = sm + SM_EQ;
-        uint8_t* QLO = sm + SM_QLO;
         const uint32_t id64 = idesc_bf16_f32(128, 64);
         float ga_next = 1.f, gb_next = 0.f;  // scalar gates of the next chunk (threads c < 64)
         const float* sga = reinterpret_cast<const float*>(sm + SM_SG);
@@ -703,7 +711,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 GDN_TRACE(m, 18);
             }
             named_bar(2, 128);
-            // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA / QLO) ----------
+            // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA) -----------------
             // Thread c: channels 8 cg .. 8 cg + 7 (one 16-byte chunk of a swizzled row) of rows
             // 8 rg .. 8 rg + 7.  Gamma over the chunk is the product of the row groups' products.
             {
@@ -805,7 +813,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     split8(qq, hi, lo);
                     st16(EQ + oq, hi);
                     st16(RQB + oq, lo);
-                    st16(QLO + o64, lo);
                     split8(kt, hi, lo);
                     st16(RK + o64, hi);
                     st16(RA + o64, lo);
@@ -926,6 +933,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         while (!mbar_try_wait(cx.bars + B_VW, (uint32_t)((vw_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
         }
         while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+        }
+        while (z_issued > 0 && !mbar_try_wait(cx.bars + B_Z, (uint32_t)((z_issued - 1) & 1)) &&
+               globaltimer_ns() - t0 < kWaitNs) {
         }
     }
     __syncthreads();

@@ -18,7 +18,7 @@ cudaError_t launch_tc(const CUtensorMap* maps, const tcfwd::Params& p, cudaStrea
                                          (int)tcfwd::kSmemBytes);
     if (e != cudaSuccess) return e;
     kernel<<<p.pb.B * p.pb.Hv, tcfwd::kThreads, tcfwd::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3],
-                                                                        maps[4], maps[5], p);
+                                                                        maps[4], maps[5], maps[6], p);
     count_launch();
     return cudaGetLastError();
 }
@@ -38,7 +38,7 @@ bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags
 
 cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
                          cudaStream_t st, const TcFwdSave* save) {
-    CUtensorMap maps[6];
+    CUtensorMap maps[7];
     const bool split = io.q_lo != nullptr;
     if (split && (f.apc || f.gpc || !io.k_lo || !io.v_lo)) return cudaErrorInvalidValue;
     bool ok = make_map(&maps[0], io.q, pb.B, pb.T, pb.Hk) && make_map(&maps[1], io.k, pb.B, pb.T, pb.Hk) &&
@@ -47,6 +47,8 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     maps[3] = maps[2];
     maps[4] = maps[2];
     maps[5] = maps[2];
+    maps[6] = maps[2];
+    if (ok && f.gate) ok = make_map(&maps[6], io.z, pb.B, pb.T, pb.Hv);  // z [B,T,Hv,dv] bf16
     if (ok && f.apc) ok = make_map(&maps[3], io.alpha, pb.B, pb.T, pb.Hv);
     if (ok && f.gpc) ok = make_map(&maps[4], io.b, pb.B, pb.T, pb.Hv) && make_map(&maps[5], io.w, pb.B, pb.T, pb.Hv);
     // Split inputs: the lo halves take the gate slots (k lo: alpha, q lo: b, v lo: w).
