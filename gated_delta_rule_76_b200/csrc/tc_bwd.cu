@@ -185,4 +185,8 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
 extern "C" __attribute__((visibility("default"))) int gdn_bwd_trace_read(unsigned long long* host) {
     return (int)cudaMemcpyFromSymbol(host, gdn::tcbwd::g_bwd_trace, sizeof(unsigned long long) * 16 * 16);
 }
+// ... and those of CTA 0 of the last reverse scan.
+extern "C" __attribute__((visibility("default"))) int gdn_scan_trace_read(unsigned long long* host) {
+    return (int)cudaMemcpyFromSymbol(host, gdn::tcbwd::g_scan_trace, sizeof(unsigned long long) * 64 * 32);
+}
 #endif

@@ -42,8 +42,17 @@ __device__ unsigned long long g_bwd_trace[16][16];
     do {                                                                                 \
         if (blockIdx.x == 0 && (it) < 16) g_bwd_trace[(it)][(point)] = globaltimer_ns(); \
     } while (0)
+// The reverse scan's CTA 0: g_scan_trace[iteration][point].
+__device__ unsigned long long g_scan_trace[64][32];
+#define GDN_STRACE(it, point)                                                              \
+    do {                                                                                   \
+        if (blockIdx.x == 0 && (it) < 64) g_scan_trace[(it)][(point)] = globaltimer_ns(); \
+    } while (0)
 #else
 #define GDN_BTRACE(it, point) \
+    do {                      \
+    } while (0)
+#define GDN_STRACE(it, point) \
     do {                      \
     } while (0)
 #endif
@@ -106,7 +115,7 @@ enum Bar {
     B_X1,        // X1 complete
     B_WT,        // W^T complete
     B_PREADY,    // prologue -> scan: P, Kbar, [Ehat;Qhat] written
-    B_WREADY,    // prologue -> scan: T, W^T written
+    B_TREADY,    // prologue -> scan: T written
     B_XA,        // XA complete
     B_XCPRE,     // dO^T Qhat complete: [Ehat;Qhat] and dO may be overwritten
     B_XC,        // XC complete
@@ -192,12 +201,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     // Chunks are processed in reverse: iteration i works on chunk NT - 1 - i.
-    int raw_issued = 0, do_issued = 0;  // meaningful in the issuing threads (256 and 0)
-    if (tid == 256) {
+    int raw_issued = 0, do_issued = 0;  // meaningful in thread 0, which issues every load
+    if (tid == 0) {
         scan_load_raw<APC, GPC>(cx, NT - 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
         raw_issued = 1;
-    }
-    if (tid == 0) {
         scan_load_do(cx, NT - 1, b, hv, &tm_do);
         do_issued = 1;
     }
@@ -212,6 +219,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const uint32_t id_dop = idesc_bf16_f32_mn(128, 64, true, true);    // dO^T P
         const uint32_t id_doq = idesc_bf16_f32_mn(128, 128, true, true);   // dO^T Qhat
         const uint32_t id_dy = idesc_bf16_f32_mn(128, 64, false, true);    // (-dV'^T) T
+        const uint32_t id_wt = idesc_bf16_f32_mn(128, 64, true, false);    // Ehat^T (MN-major) x T
         float S[64];  // S[c'] = dS[64h + c'][j]
 #pragma unroll
         for (int c = 0; c < 64; ++c) S[c] = p.dht ? p.dht[soff + (long)(64 * h + c) * D + j] : 0.f;
@@ -233,8 +241,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int t0 = n * C, L = min(C, pb.T - t0);
             // ---- XA = dS^T Kbar^T + dO^T P (= dV'^T);  XC = dO^T Qhat ----------------------------
             if (tid == 0) {
+                GDN_STRACE(i, 0);
                 tc_fence_after();
                 if (wait1(cx, B_PREADY, pi) && wait1(cx, B_DO, pi) && !*cx.abort_flag) {
+                    GDN_STRACE(i, 1);
                     mma_ts_u<128, 64>(tbase + TM_XA, tbase + TM_DSH, sbase + SM_KB, id64, false);
                     mma_ts_u<128, 64>(tbase + TM_XA, tbase + TM_DSL, sbase + SM_KB, id64, true);
                     mma_ts_u<128, 64>(tbase + TM_XA, tbase + TM_DSH, sbase + SM_KB + 16384, id64, true);
@@ -256,6 +266,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     mma_commit(cx.bars + B_XCPRE);
                     wait1(cx, B_XA, pi);
+                    GDN_STRACE(i, 2);
                 }
             }
             named_bar(1, 256);
@@ -274,10 +285,56 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             tc_fence_before();
             named_bar(1, 256);
+            // ---- W^T = Ehat^T T^T once the prologue has written T; then the raw stage is free ------
+            if (tid == 0) {
+                tc_fence_after();
+                GDN_STRACE(i, 3);
+                if (wait1(cx, B_TREADY, pi) && !*cx.abort_flag) {
+#pragma unroll
+                    for (int k = 0; k < 64; k += 16) {
+                        const uint64_t dt = sdesc_k_sw128(sbase + SM_T + (uint32_t)k * 2u);
+                        mma_ss(tbase + TM_WT, sdesc_mn_sw128(sbase + SM_EQ + (uint32_t)k * 128u, 16384u), dt, id_wt,
+                               k > 0 ? 1u : 0u);
+                        mma_ss(tbase + TM_WT, sdesc_mn_sw128(sbase + SM_RQB + (uint32_t)k * 128u, 16384u), dt, id_wt, 1u);
+                    }
+                    mma_commit(cx.bars + B_WT);
+                    wait1(cx, B_WT, pi);
+                    // X1, XC's dO^T Qhat and W^T were the last readers of the raw stage.
+                    if (raw_issued < NT && wait1(cx, B_XCPRE, pi) && !*cx.abort_flag) {
+                        scan_load_raw<APC, GPC>(cx, NT - 1 - raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                        ++raw_issued;
+                    }
+                }
+                GDN_STRACE(i, 4);
+            }
+            named_bar(1, 256);
+            tc_fence_after();
+            {
+                // W^T row j, columns 32 h .. 32 h + 31, split (K-major B operand of XC).
+                uint8_t* WT = sm + SM_WT;
+                uint32_t r[32];
+                tmem_ld32(tl + TM_WT + 32 * h, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t wh[4], wl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i0 = 8 * ch + 2 * e;
+                        split_pack(__uint_as_float(r[i0]), __uint_as_float(r[i0 + 1]), wh[e], wl[e]);
+                    }
+                    const uint32_t off = sw128_offset(j, 32 * h + 8 * ch, 128);
+                    st16(WT + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
+                    st16(WT + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
+                }
+            }
+            fence_async_shared();
+            tc_fence_before();
+            named_bar(1, 256);
             // ---- XC += (-dV'^T) W;  XA = (-dV'^T) T (= -dY^T);  next dO ----------------------------
             if (tid == 0) {
                 tc_fence_after();
-                if (wait1(cx, B_WREADY, pi) && !*cx.abort_flag) {
+                if (!*cx.abort_flag) {
                     mma_ts_u<64, 128>(tbase + TM_XC, tbase + TM_DVH, sbase + SM_WT, id128, true);
                     mma_ts_u<64, 128>(tbase + TM_XC, tbase + TM_DVL, sbase + SM_WT, id128, true);
                     mma_ts_u<64, 128>(tbase + TM_XC, tbase + TM_DVH, sbase + SM_WT + 16384, id128, true);
@@ -295,6 +352,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     ++do_issued;
                 }
                 wait1(cx, B_XC, pi);
+                GDN_STRACE(i, 5);
             }
             if (p.dsc) {
                 // dS_end of chunk n, rows 64h .. 64h + 63 of column j, layout [j / 4][row][j % 4]
@@ -331,8 +389,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             // ---- -dY of chunk n, token-major hi / lo ----------------------------------------------
             if (tid == 0) {
+                GDN_STRACE(i, 6);
                 tc_fence_after();
                 wait1(cx, B_DY, pi);
+                GDN_STRACE(i, 7);
             }
             tc_fence_before();
             named_bar(1, 256);
@@ -354,7 +414,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                 }
             }
-            if (tid == 0) *stop_slot = *cx.abort_flag;
+            if (tid == 0) {
+                GDN_STRACE(i, 8);
+                *stop_slot = *cx.abort_flag;
+            }
             tc_fence_before();
             named_bar(1, 256);
             if (*stop_slot) break;
@@ -378,13 +441,16 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         uint8_t* EQ = sm + SM_EQ;
         uint8_t* KB = sm + SM_KB;
         const uint32_t id64 = idesc_bf16_f32(128, 64);
-        const uint32_t id_wt = idesc_bf16_f32_mn(128, 64, true, false);  // Ehat^T (MN-major) x T
         const float scale = pb.scale;
         for (int i = 0; i < NT; ++i) {
             const int n = NT - 1 - i;
             const uint32_t pi = i & 1;
             const int t0 = n * C, L = min(C, pb.T - t0);
-            if (c == 0) wait1(cx, B_RAW, pi);
+            if (c == 0) {
+                GDN_STRACE(i, 16);
+                wait1(cx, B_RAW, pi);
+                GDN_STRACE(i, 17);
+            }
             named_bar(2, 128);
             // ---- cumulative decay; split operands (hi -> EQ / RK, lo -> RQB / RA), split Kbar -----
             // Thread c: channels 8 cg .. 8 cg + 7 of rows 8 rg .. 8 rg + 7; Gamma over the chunk is
@@ -491,6 +557,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             named_bar(2, 128);
             // ---- X1 = [Ehat;Qhat] Ktil^T ----------------------------------------------------------
             if (c == 0) {
+                GDN_STRACE(i, 18);
                 tc_fence_after();
                 if (!*cx.abort_flag) {
                     mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RK, id64, false);
@@ -548,7 +615,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fence_async_shared();
             tc_fence_before();
             named_bar(2, 128);
-            if (c == 0) mbar_arrive(cx.bars + B_PREADY);
+            if (c == 0) {
+                GDN_STRACE(i, 19);
+                mbar_arrive(cx.bars + B_PREADY);
+            }
             // ---- T = (I + A)^-1 by 16 x 16 blocks, in place in the fp32 scratch ------------------
             if (c < 64) {
                 const int base = 16 * (c >> 4), jc = c & 15;
@@ -581,6 +651,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             solve_block_row<2>(ascr, rs, c);
             solve_block_row<3>(ascr, rs, c);
             // ---- T (fp32) -> bf16 tile once the scan has finished with the previous T and W^T ------
+            if (c == 0) GDN_STRACE(i, 20);
             if (c == 0 && i > 0) wait1(cx, B_DY, pi ^ 1u);
             named_bar(2, 128);
             {
@@ -597,54 +668,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             fence_async_shared();
             named_bar(2, 128);
-            // ---- W^T = Ehat^T T^T; then the raw stage is free for the next chunk ------------------
             if (c == 0) {
-                tc_fence_after();
-                if (!*cx.abort_flag) {
-#pragma unroll
-                    for (int k = 0; k < 64; k += 16) {
-                        const uint64_t dt = sdesc_k_sw128(sbase + SM_T + (uint32_t)k * 2u);
-                        mma_ss(tbase + TM_WT, sdesc_mn_sw128(sbase + SM_EQ + (uint32_t)k * 128u, 16384u), dt, id_wt,
-                               k > 0 ? 1u : 0u);
-                        mma_ss(tbase + TM_WT, sdesc_mn_sw128(sbase + SM_RQB + (uint32_t)k * 128u, 16384u), dt, id_wt, 1u);
-                    }
-                    mma_commit(cx.bars + B_WT);
-                }
-                wait1(cx, B_WT, pi);
-                if (raw_issued < NT && wait1(cx, B_XCPRE, pi) && !*cx.abort_flag) {
-                    scan_load_raw<APC, GPC>(cx, NT - 1 - raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
-                    ++raw_issued;
-                }
-            }
-            named_bar(2, 128);
-            tc_fence_after();
-            {
-                // W^T row c, split: row c, columns r (K-major B operand of XC).
-                uint8_t* WT = sm + SM_WT;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tl + TM_WT + 32 * half, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t wh[4], wl[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i0 = 8 * ch + 2 * e;
-                            split_pack(__uint_as_float(r[i0]), __uint_as_float(r[i0 + 1]), wh[e], wl[e]);
-                        }
-                        const uint32_t off = sw128_offset(c, 32 * half + 8 * ch, 128);
-                        st16(WT + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
-                        st16(WT + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
-                    }
-                }
-            }
-            fence_async_shared();
-            tc_fence_before();
-            named_bar(2, 128);
-            if (c == 0) {
-                mbar_arrive(cx.bars + B_WREADY);
+                // T is in shared memory: the scan forms W^T and splits it.
+                mbar_arrive(cx.bars + B_TREADY);
+                GDN_STRACE(i, 22);
                 *stop_slot = *cx.abort_flag;
             }
             named_bar(2, 128);
@@ -660,7 +687,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (tid == 0 && do_issued > 0)
             while (!mbar_try_wait(cx.bars + B_DO, (uint32_t)((do_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
             }
-        if (tid == 256 && raw_issued > 0)
+        if (tid == 0 && raw_issued > 0)
             while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) &&
                    globaltimer_ns() - t0 < kWaitNs) {
             }

@@ -362,7 +362,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 136);
         const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
         const long soff = pb.state_off(b, hv);
-        const TG* beta = static_cast<const TG*>(p.b);
         const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
         // swizzled byte offsets of column j in a 64-row tile: row r -> base + r*128 + xo[r & 7]
         const uint32_t vbase = (uint32_t)(j >> 6) * 64u * 128u;
