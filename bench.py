@@ -111,7 +111,7 @@ def load_peaks():
 # of its two kernels (reverse scan, gradients) on B=2 T=2048 (an eighth of the workload's tokens:
 # the per-chunk traffic is fixed, so it scales with the tokens); see
 # profiles/chunk_bwd_kernels_gdn2_b2_t2048.md.  To be set to None whenever those kernels change.
-BWD_CALL_TRAFFIC_BYTES = (84.06 + 55.49 + 360.23 + 154.44) * 1e6 * 8
+BWD_CALL_TRAFFIC_BYTES = (84.07 + 54.87 + 360.25 + 155.14) * 1e6 * 8
 
 
 def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False,
@@ -561,7 +561,23 @@ def _profile_fwd_b8_t1024():
     return 0
 
 
-PROFILE_CASES = {"train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024}
+def _profile_layer_b2_t16384():
+    """GQA layer core (conv k=4 + SiLU + L2, chunk forward, swish gate) on its full workload
+    (B=2 T=16384, 16 key / 128 value heads, d=128 bf16, seed of the workload), twice."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import workload_inputs
+    x = workload_inputs("gqa_layer_core_bf16")
+    g = {k: v.cuda() for k, v in x.items()}
+    for _ in range(2):
+        y, _, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], beta=g["beta"])
+    torch.cuda.synchronize()
+    print("ok", float(y.float().abs().mean()))
+    return 0
+
+
+PROFILE_CASES = {"train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024,
+                 "layer_b2_t16384": _profile_layer_b2_t16384}
 
 
 def main():
