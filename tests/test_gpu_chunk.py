@@ -16,6 +16,9 @@ CASES = {
     "gdn2_bf16_ragged": (2, 200, 2, 2, 128, True, True, "bf16", "bf16", True, 1.0),
     "gdn_scalar_bf16_f32gates_gqa": (1, 130, 1, 4, 128, False, False, "bf16", "f32", True, 1.0),
     "kda_f32_d128": (1, 65, 2, 2, 128, True, False, "f32", "f32", True, 0.5),
+    # tensor-core path, the two mixed gate forms (channel alpha + scalar beta; scalar alpha + b, w)
+    "kda_bf16_d128": (1, 140, 2, 2, 128, True, False, "bf16", "bf16", True, 0.8),
+    "gdn2_scalar_alpha_bf16_d128_gqa": (1, 100, 1, 2, 128, False, True, "bf16", "bf16", True, 1.0),
     "gdn2_scalar_alpha_bf16_d64": (3, 97, 2, 2, 64, False, True, "bf16", "bf16", False, 1.0),
     "gdn2_f32_d64_gqa": (2, 150, 1, 2, 64, True, True, "f32", "f32", True, 1.0),
     "one_token": (2, 1, 1, 1, 128, True, True, "bf16", "bf16", True, 1.0),
