@@ -131,8 +131,13 @@ def draw(B: int, T: int, Hk: int, Hv: int, dk: int, dv: int, *,
          alpha_per_channel: bool, gates_per_channel: bool, dtype: str = "bf16",
          gate_dtype: Optional[str] = None, seed: int = 0, has_h0: bool = True,
          conv: bool = False, swish_gate: bool = False, with_dout: bool = False,
-         with_dht: bool = False, normalise_qk: Optional[bool] = None) -> Dict[str, object]:
+         with_dht: bool = False, normalise_qk: Optional[bool] = None,
+         erase_scale: float = 1.0) -> Dict[str, object]:
     """Draw one batch of chunkwise-forward/backward inputs.
+
+    erase_scale multiplies the erase gate b (or the scalar beta): 2 gives the negative-eigenvalue
+    range b, beta in [0, 2] of the explainer's «Réunir les deux» note (the transition's eigenvalue
+    along k is then 1 - beta in [-1, 1]); the write gate w stays in [0, 1].
 
     Returns a dict of torch CPU tensors in token-major layouts:
       q, k [B,T,Hk,dk]; v [B,T,Hv,dv]; alpha [B,T,Hv,dk] or [B,T,Hv];
@@ -157,10 +162,10 @@ def draw(B: int, T: int, Hk: int, Hv: int, dk: int, dv: int, *,
     a_shape = (B, T, Hv, dk) if alpha_per_channel else (B, T, Hv)
     out["alpha"] = _cast(_decay(_normal(rng, a_shape)), gate_dtype)
     if gates_per_channel:
-        out["b"] = _cast(_sigmoid(_normal(rng, (B, T, Hv, dk))), gate_dtype)
+        out["b"] = _cast(erase_scale * _sigmoid(_normal(rng, (B, T, Hv, dk))), gate_dtype)
         out["w"] = _cast(_sigmoid(_normal(rng, (B, T, Hv, dv))), gate_dtype)
     else:
-        out["beta"] = _cast(_sigmoid(_normal(rng, (B, T, Hv))), gate_dtype)
+        out["beta"] = _cast(erase_scale * _sigmoid(_normal(rng, (B, T, Hv))), gate_dtype)
     if swish_gate:
         out["z"] = _cast(_normal(rng, (B, T, Hv, dv)), dtype)
     if conv:

@@ -9,7 +9,9 @@
  *
  * with S_t in R^{dk x dv} (dk rows, dv contiguous columns), the erase gate b_t in [0,1]^dk on the
  * key axis, the write gate w_t in [0,1]^dv on the value axis and the channel decay alpha_t in
- * (0,1)^dk.  With b = w = beta (one scalar per token and head) and a scalar alpha this is Gated
+ * (0,1)^dk.  Erase gates (b or the scalar beta) up to 2 are accepted as well: the negative-
+ * eigenvalue variant of the Gated DeltaNet explainer's note under «Réunir les deux» (for a unit
+ * key the transition's eigenvalue along k is 1 - beta in [-1, 1]); every kernel is unchanged.  With b = w = beta (one scalar per token and head) and a scalar alpha this is Gated
  * DeltaNet (Gated DeltaNet explainer, docsaid.org, «Réunir les deux»); with alpha = 1 as well it
  * is DeltaNet («DeltaNet : ne corriger que l'entrée visée»).  Channel alpha with scalar beta is
  * the KDA case named on the same GDN-2 page.

@@ -185,3 +185,29 @@ def test_forward_cache_is_refused_off_the_tensor_core_path():
     cache = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     with pytest.raises(gdn.GdnError, match="UNSUPPORTED"):
         gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
+
+
+@pytest.mark.parametrize("B,T,Hk,Hv,d,apc,gpc,dt", [
+    (1, 150, 2, 2, 128, True, True, "bf16"),     # tensor-core path, channel gates
+    (1, 130, 1, 2, 128, False, False, "bf16"),   # tensor-core path, scalar beta
+    (1, 100, 1, 1, 64, True, True, "f32"),       # CUDA-core path
+])
+def test_negative_eigenvalue_gates(B, T, Hk, Hv, d, apc, gpc, dt):
+    """Erase gates b, beta in [0, 2] (the explainer's note under «Réunir les deux»): forward and
+    backward against the oracle, the kernels unchanged."""
+    x = draw(B, T, Hk, Hv, d, d, alpha_per_channel=apc, gates_per_channel=gpc, dtype=dt, gate_dtype=dt,
+             seed=41, has_h0=True, with_dout=True, with_dht=True, erase_scale=2.0)
+    gk = gate_kw(x)
+    assert float((gk["b"] if gpc else gk["beta"]).float().max()) > 1.5
+    g = to_cuda(x)
+    kind = kind_of(x["q"])
+    o, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], out_f32=True, **gate_kw(g))
+    o_ref, ht_ref = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=x["h0"], **gk)
+    assert_parity(o, o_ref, kind, "o")
+    assert_parity(ht, ht_ref, kind, "ht")
+    grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"],
+                              grad_ht=g["dht"], **gate_kw(g))
+    torch.cuda.synchronize()
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["alpha"], h0=x["h0"], dout=x["dout"], dht=x["dht"], **gk)
+    for key in ["dq", "dk", "dv", "dalpha", "dh0"] + (["db", "dw"] if gpc else ["dbeta"]):
+        assert_parity(grads[key], ref[key], kind, key)

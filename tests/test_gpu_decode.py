@@ -135,3 +135,23 @@ def test_layer_core_tensor_core_path(B, T, Hk, Hv, gdt):
                                           scale=0.8, h0=x["h0"])
     assert_parity(y, y_ref, "bf16", "y")
     assert_parity(ht, ht_ref, "bf16", "ht")
+
+
+def test_decode_negative_eigenvalue_gates():
+    """Erase gates in [0, 2] (the explainer's note under «Réunir les deux») through the decode
+    step, each side carrying its own state."""
+    N, Hk, Hv, d, steps = 3, 1, 2, 128, 6
+    x = draw(N, steps, Hk, Hv, d, d, alpha_per_channel=True, gates_per_channel=True, dtype="bf16",
+             gate_dtype="bf16", seed=43, has_h0=True, erase_scale=2.0)
+    assert float(x["b"].float().max()) > 1.5
+    g = to_cuda(x)
+    state = g["h0"].clone()
+    ref_state = npf(x["h0"])
+    for t in range(steps):
+        tk = lambda src, key: src[key][:, t].contiguous()
+        o = gdn.gdn_decode_step(state, tk(g, "q"), tk(g, "k"), tk(g, "v"), tk(g, "alpha"), b=tk(g, "b"),
+                                w=tk(g, "w"), out_f32=True)
+        o_ref, ref_state = oracle.decode_step(ref_state, tk(x, "q"), tk(x, "k"), tk(x, "v"), tk(x, "alpha"),
+                                              b=tk(x, "b"), w=tk(x, "w"))
+        assert_parity(o, o_ref, "bf16", f"o step {t}")
+    assert_parity(state, ref_state, "bf16", "state")

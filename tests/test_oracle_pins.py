@@ -191,6 +191,43 @@ def test_edit_invariant():
         assert np.allclose(S.T @ e, (1 - kappa) * (Sbar.T @ e) + kappa * z, atol=1e-13)
 
 
+def test_reflection_at_beta_two_is_an_involution():
+    """Negative-eigenvalue range (explainer, «Réunir les deux», note on beta in [0, 2]): with
+    alpha = 1, a unit key, beta = 2 and no write (v = 0) the step is the Householder reflection
+    S -> (I - 2 k k^T) S, so the same step twice returns the state, and once negates the read
+    at k while sparing every direction orthogonal to k."""
+    rng = np.random.default_rng(31)
+    dk, dv = 6, 5
+    k = rng.standard_normal(dk)
+    k /= np.linalg.norm(k)
+    h0 = rng.standard_normal((1, 1, dk, dv))
+    kk = np.broadcast_to(k, (1, 2, 1, dk)).copy()
+    ones = np.ones((1, 2, 1))
+    v0 = np.zeros((1, 2, 1, dv))
+    _, once = oracle.fwd(kk[:, :1], kk[:, :1], v0[:, :1], ones[:, :1], beta=2 * ones[:, :1], h0=h0)
+    _, twice = oracle.fwd(kk, kk, v0, ones, beta=2 * ones, h0=h0)
+    assert np.allclose(twice[0, 0], h0[0, 0], atol=1e-13)
+    assert np.allclose(once[0, 0].T @ k, -(h0[0, 0].T @ k), atol=1e-13)
+    u = rng.standard_normal(dk)
+    u -= (u @ k) * k
+    assert np.allclose(u @ once[0, 0], u @ h0[0, 0], atol=1e-13)
+
+
+def test_edit_invariant_over_the_negative_eigenvalue_range():
+    """The edit invariant S_t^T e_t = (1 - kappa) Sbar^T e_t + kappa z_t holds unchanged for erase
+    gates b in [0, 2] (kappa = k . e up to 2 for a unit key)."""
+    rng = np.random.default_rng(32)
+    for _ in range(5):
+        x = rand_inputs(rng, 1, 1, 1, 1, 7, 5)
+        x["b"] = 2.0 * x["b"]
+        _, hT = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], b=x["b"], w=x["w"], h0=x["h0"])
+        k, b_, w_ = x["k"][0, 0, 0], x["b"][0, 0, 0], x["w"][0, 0, 0]
+        e, z = b_ * k, w_ * x["v"][0, 0, 0]
+        Sbar = x["alpha"][0, 0, 0][:, None] * x["h0"][0, 0]
+        kappa = k @ e
+        assert np.allclose(hT[0, 0].T @ e, (1 - kappa) * (Sbar.T @ e) + kappa * z, atol=1e-13)
+
+
 def test_orthogonal_keys_spared():
     """For u orthogonal to k_t: u^T S_t = u^T D_t S_{t-1} (explainer, «DeltaNet»)."""
     rng = np.random.default_rng(17)
