@@ -387,13 +387,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int n = 0; n < NT; ++n) {
             const uint32_t pn = n & 1;
             const int t0 = n * C, L = min(C, pb.T - t0);
-            if (p.s0_out) {
-                // state entering chunk n, rows 64h .. 64h + 63 of column j, in the layout
-                // [j / 4][row][j % 4] (a reader holding one row per thread loads it as float4s)
-                float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
-#pragma unroll
-                for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
-            }
             if (GATE && tid == 0 && !*cx.abort_flag) {
                 // z of this chunk for the output epilogue (the previous chunk's reads are done)
                 const uint32_t zd = sbase + SM_Z;
@@ -441,6 +434,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     st16(KB + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
                     st16(KB + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
                 }
+            }
+            if (p.s0_out) {
+                // state entering chunk n (saving mode), stored while X2 runs: rows 64h .. 64h + 63
+                // of column j, in the layout [j / 4][row][j % 4] (a reader holding one row per
+                // thread loads it as float4s)
+                float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
+#pragma unroll
+                for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
             }
             tc_fence_before();
             fence_async_shared();
@@ -534,33 +535,16 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             named_bar(1, 256);
             tc_fence_after();
+            uint32_t vhi[16], vlo[16];  // V' of rows 32h .. 32h + 31, column j (stored after X4/X5 issue)
             {
-                uint32_t r[32], hi[16], lo[16];
+                uint32_t r[32];
                 tmem_ld32(tl + TM_X5 + 32 * h, r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    split_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), hi[i], lo[i]);
-                tmem_st16(tl + TM_YH + 16 * h, hi);
-                tmem_st16(tl + TM_YL + 16 * h, lo);
-                if (p.vp_hi) {
-                    // V' rows 32h .. 32h + 31 of column j, token-major (coalesced over j)
-                    const long vrow = (long)pb.Hv * D;
-                    const long vb = pb.v_row(b, t0 + 32 * h, hv) + j;
-                    const int nrow = min(32, L - 32 * h);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int r0 = 2 * i;
-                        if (r0 < nrow) {
-                            p.vp_hi[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(hi[i] & 0xFFFFu));
-                            p.vp_lo[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(lo[i] & 0xFFFFu));
-                        }
-                        if (r0 + 1 < nrow) {
-                            p.vp_hi[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(hi[i] >> 16));
-                            p.vp_lo[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(lo[i] >> 16));
-                        }
-                    }
-                }
+                    split_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), vhi[i], vlo[i]);
+                tmem_st16(tl + TM_YH + 16 * h, vhi);
+                tmem_st16(tl + TM_YL + 16 * h, vlo);
                 tmem_st_wait();
             }
             tc_fence_before();
@@ -580,6 +564,29 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YL, KB, id128, true);
                     mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB + 16384, id128, true);
                     mma_commit(cx.bars + B_X45);
+                }
+            }
+            if (p.vp_hi) {
+                // V' (saving mode), stored while X4 / X5 run: rows 32h .. 32h + 31 of column j,
+                // token-major (coalesced over j)
+                const long vrow = (long)pb.Hv * D;
+                const long vb = pb.v_row(b, t0 + 32 * h, hv) + j;
+                const int nrow = min(32, L - 32 * h);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r0 = 2 * i;
+                    if (r0 < nrow) {
+                        p.vp_hi[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(vhi[i] & 0xFFFFu));
+                        p.vp_lo[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(vlo[i] & 0xFFFFu));
+                    }
+                    if (r0 + 1 < nrow) {
+                        p.vp_hi[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(vhi[i] >> 16));
+                        p.vp_lo[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(vlo[i] >> 16));
+                    }
+                }
+            }
+            if (tid == 0) {
+                if (!*cx.abort_flag) {
                     wait1(cx, B_X45, pn);
                     GDN_TRACE(n, 10);
                 }
