@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(128) conv_silu_l2_kernel(ConvParams p) {
             acc += wt[i][1] * x2[i];
             acc += wt[i][2] * x1[i];
             acc += wt[i][3] * x0[i];
-            y[i] = acc / (1.0f + __expf(-acc));
+            y[i] = acc * __fdividef(1.0f, 1.0f + __expf(-acc));  // SiLU (fast reciprocal: a few ulp)
             ss += y[i] * y[i];
         }
         float scale = 1.f;
