@@ -260,3 +260,93 @@ def layer_core_fwd(xq, xk, xv, conv_w, alpha, beta, z, head_map=None, scale=1.0,
     v = v.reshape(B, T, Hv, dv)
     o, hT = fwd(q, k, v, alpha, beta=beta, h0=h0, head_map=head_map, scale=scale, pairs=pairs)
     return swish_gate(o, z), hT
+
+
+# ---- layer-core backward (reverse mode of layer_core_fwd, fp64 numpy) ---------------------------
+# The layer of the explainer's «Architecture et versions hybrides» (Figure 1 caption) and the mkdocs
+# chapter «Gated DeltaNet»: per channel a causal depthwise convolution of kernel 4 (zero history,
+# conv_w[ch][3] weighting the current token), SiLU, then the L2 norm of each q and k head row; the
+# recurrence; the swish(z) output gate.  Each reverse step below is the derivative of one forward
+# step, written out; the finite-difference pin in tests/ checks the composition.
+
+def _conv_pre(x, w):
+    """Causal depthwise conv, kernel 4, zero history: u[:, t, c] = sum_tap w[c, tap] x[:, t-3+tap, c]."""
+    B, T, C = x.shape
+    u = np.zeros_like(x)
+    for tap in range(4):
+        sh = 3 - tap
+        if sh == 0:
+            u += w[:, tap] * x
+        elif sh < T:
+            u[:, sh:] += w[:, tap] * x[:, :T - sh]
+    return u
+
+
+def _conv_pre_bwd(x, w, du):
+    """Reverse of _conv_pre: dx[:, s] = sum_tap w[tap] du[:, s+3-tap]; dw[c, tap] = sum du[t] x[t-3+tap]."""
+    B, T, C = x.shape
+    dx = np.zeros_like(x)
+    dw = np.zeros((C, 4))
+    for tap in range(4):
+        sh = 3 - tap
+        if sh == 0:
+            dx += w[:, tap] * du
+            dw[:, tap] = np.sum(du * x, axis=(0, 1))
+        elif sh < T:
+            dx[:, :T - sh] += w[:, tap] * du[:, sh:]
+            dw[:, tap] = np.sum(du[:, sh:] * x[:, :T - sh], axis=(0, 1))
+    return dx, dw
+
+
+def _sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def layer_core_bwd(xq, xk, xv, conv_w, alpha, z, dy, b=None, w=None, beta=None, head_map=None,
+                   scale=1.0, h0=None, dht=None) -> Dict[str, np.ndarray]:
+    """Reverse mode of the GQA layer core for loss gradients dy (of y) and dht (of the final
+    state).  Returns dxq, dxk, dxv, dconv_w, dz, dalpha, db/dw or dbeta, dh0."""
+    xq, xk, xv, W = f64(xq), f64(xk), f64(xv), f64(conv_w)
+    zz, g = f64(z), f64(dy)
+    B, T, Hk, dk = xq.shape
+    Hv, dv = xv.shape[2], xv.shape[3]
+    cq = Hk * dk
+    parts = {}
+    for name, x, wsl, H, d, norm in (("q", xq, W[:cq], Hk, dk, True), ("k", xk, W[cq:2 * cq], Hk, dk, True),
+                                     ("v", xv, W[2 * cq:], Hv, dv, False)):
+        xf = x.reshape(B, T, H * d)
+        u = _conv_pre(xf, wsl)
+        a = u * _sigmoid(u)                          # SiLU
+        if norm:
+            a4 = a.reshape(B, T, H, d)
+            n = np.sqrt(np.sum(a4 * a4, axis=-1, keepdims=True) + L2_EPS)
+            out = a4 / n                             # L2 norm of each head row
+        else:
+            n, out = None, a.reshape(B, T, H, d)
+        parts[name] = (xf, wsl, u, a, n, out)
+    q, k, v = parts["q"][5], parts["k"][5], parts["v"][5]
+    gk = dict(beta=beta) if beta is not None else dict(b=b, w=w)
+    o, _ = fwd(q, k, v, alpha, head_map=head_map, scale=scale, h0=h0, **gk)
+    sg = _sigmoid(zz)
+    do = g * zz * sg                                 # y = o * z * sigmoid(z)
+    dz = g * o * (sg + zz * sg * (1.0 - sg))
+    core = bwd(q, k, v, alpha, head_map=head_map, scale=scale, h0=h0, dout=do, dht=dht, **gk)
+    res = {"dz": dz, "dalpha": core["dalpha"], "dh0": core["dh0"]}
+    for key in ("dbeta", "db", "dw"):
+        if key in core:
+            res[key] = core[key]
+    dconv = []
+    for name, gout in (("q", core["dq"]), ("k", core["dk"]), ("v", core["dv"])):
+        xf, wsl, u, a, n, out = parts[name]
+        if n is not None:                            # out = a / n,  n = sqrt(sum a^2 + eps)
+            dot = np.sum(out * gout, axis=-1, keepdims=True)
+            da = ((gout - out * dot) / n).reshape(a.shape)
+        else:
+            da = gout.reshape(a.shape)
+        s = _sigmoid(u)
+        du = da * (s + u * s * (1.0 - s))            # d/du of u * sigmoid(u)
+        dx, dwc = _conv_pre_bwd(xf, wsl, du)
+        res["dx" + name] = dx.reshape(parts[name][5].shape)
+        dconv.append(dwc)
+    res["dconv_w"] = np.concatenate(dconv, axis=0)
+    return res

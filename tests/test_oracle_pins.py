@@ -410,3 +410,59 @@ def test_l2norm_and_swish_gate():
     z = rng.standard_normal(100) * 4
     from scipy.special import expit
     assert np.allclose(oracle.swish_gate(o, z), o * z * expit(z), atol=1e-14)
+
+
+@pytest.mark.parametrize("channel_gates", [False, True])
+def test_layer_backward_finite_differences(channel_gates):
+    """The layer core's reverse mode (conv k=4, SiLU, L2 norm, the recurrence, the swish gate)
+    against central differences of sum(y * dy) + sum(hT * dht), for every input, on a tiny GQA
+    layer.  The forward here is composed from the oracle's own conv_silu / l2norm / fwd /
+    swish_gate, so the pin ties the hand-written reverse steps to their forward definitions."""
+    rng = np.random.default_rng(55)
+    B, T, Hk, Hv, d = 1, 6, 1, 2, 4
+    cq = Hk * d
+    x = dict(xq=rng.standard_normal((B, T, Hk, d)), xk=rng.standard_normal((B, T, Hk, d)),
+             xv=rng.standard_normal((B, T, Hv, d)), conv_w=0.5 * rng.standard_normal((2 * cq + Hv * d, 4)),
+             alpha=np.exp(-0.1 * np.logaddexp(0.0, rng.standard_normal((B, T, Hv)))),
+             z=rng.standard_normal((B, T, Hv, d)), h0=0.3 * rng.standard_normal((B, Hv, d, d)))
+    if channel_gates:
+        x["b"] = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, Hv, d))))
+        x["w"] = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, Hv, d))))
+        gnames = ["b", "w"]
+    else:
+        x["beta"] = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, Hv))))
+        gnames = ["beta"]
+    dy = rng.standard_normal((B, T, Hv, d))
+    dht = rng.standard_normal((B, Hv, d, d))
+    scale = 0.8
+
+    def loss(vals):
+        W = vals["conv_w"]
+        q, _ = oracle.conv_silu(vals["xq"].reshape(B, T, cq), W[:cq])
+        k, _ = oracle.conv_silu(vals["xk"].reshape(B, T, cq), W[cq:2 * cq])
+        v, _ = oracle.conv_silu(vals["xv"].reshape(B, T, Hv * d), W[2 * cq:])
+        q = oracle.l2norm(q.reshape(B, T, Hk, d))
+        k = oracle.l2norm(k.reshape(B, T, Hk, d))
+        o, hT = oracle.fwd(q, k, v.reshape(B, T, Hv, d), vals["alpha"], h0=vals["h0"], scale=scale,
+                           nthreads=1, **{n: vals[n] for n in gnames})
+        return np.sum(oracle.swish_gate(o, vals["z"]) * dy) + np.sum(hT * dht)
+
+    g = oracle.layer_core_bwd(x["xq"], x["xk"], x["xv"], x["conv_w"], x["alpha"], x["z"], dy, h0=x["h0"],
+                              dht=dht, scale=scale, **{n: x[n] for n in gnames})
+    key = {"xq": "dxq", "xk": "dxk", "xv": "dxv", "conv_w": "dconv_w", "alpha": "dalpha", "z": "dz",
+           "h0": "dh0", "b": "db", "w": "dw", "beta": "dbeta"}
+    names = list(x)
+    h = 1e-6
+    for n in names:
+        base = x[n]
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = {m: x[m].copy() for m in names}
+            minus = {m: x[m].copy() for m in names}
+            plus[n][idx] += h
+            minus[n][idx] -= h
+            fd[idx] = (loss(plus) - loss(minus)) / (2 * h)
+        err = np.max(np.abs(g[key[n]] - fd)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-6, (n, err)
