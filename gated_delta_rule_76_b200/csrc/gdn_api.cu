@@ -521,6 +521,122 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
 }
 
+// Workspace of the layer backward: the recomputed conv results (fp32), the recurrence's output o
+// and its gradient, the gradients of q, k, v from the recurrence, the conv-weight partials, then
+// the CUDA-core chunk backward's own workspace.  Offsets from the start, 256-byte aligned.
+struct LayerBwdPlan {
+    size_t q, k, v, o, dout, gq, gk, gv, wpart, chunk, bytes;
+};
+static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& pb) {
+    LayerBwdPlan w{};
+    const size_t BT = (size_t)(a->B * a->T), qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
+    size_t off = 256;
+    auto take = [&](size_t floats) {
+        const size_t o = off;
+        off = align256(off + floats * sizeof(float));
+        return o;
+    };
+    w.q = take(qn); w.k = take(qn); w.v = take(vn); w.o = take(vn); w.dout = take(vn);
+    w.gq = take(qn); w.gk = take(qn); w.gv = take(vn);
+    w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk));
+    w.chunk = off;
+    w.bytes = off + plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
+    return w;
+}
+
+size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    return plan_layer_bwd(a, pb).bytes;
+}
+
+gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size_t workspace_bytes,
+                              gdn_stream stream) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    gdn_status s = check_common(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->head_map,
+                                a->alpha_per_channel, a->gates_per_channel, a->dtype, a->gate_dtype);
+    if (s) return s;
+    if (a->dk != a->dv) return fail(GDN_ERR_UNSUPPORTED, "the layer core needs dk == dv");
+    if (a->T > 0 && (!a->xq || !a->xk || !a->xv || !a->conv_w || !a->alpha || !a->b || !a->z || !a->grad_y ||
+                     !a->grad_xq || !a->grad_xk || !a->grad_xv || !a->grad_alpha || !a->grad_b || !a->grad_z))
+        return fail(GDN_ERR_INVALID_ARG, "inputs, grad_y and the gradients of xq, xk, xv, alpha, b, z are required");
+    if (!a->grad_conv_w) return fail(GDN_ERR_INVALID_ARG, "grad_conv_w is required");
+    if (a->gates_per_channel ? (a->T > 0 && (!a->w || !a->grad_w)) : (a->w != nullptr || a->grad_w != nullptr))
+        return fail(GDN_ERR_INVALID_ARG, "w and grad_w are required with channel gates and must be NULL otherwise");
+    const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
+    const size_t BT = (size_t)(a->B * a->T);
+    const size_t cch = (size_t)(2 * a->Hk * a->dk + a->Hv * a->dv);
+    const size_t st = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
+    const size_t na = BT * a->Hv * (a->alpha_per_channel ? a->dk : 1), nb = BT * a->Hv * (a->gates_per_channel ? a->dk : 1);
+    const size_t nw = a->gates_per_channel ? BT * a->Hv * a->dv : 0;
+    const Buf in[] = {
+        {a->xq, BT * a->Hk * a->dk * es, "xq"}, {a->xk, BT * a->Hk * a->dk * es, "xk"},
+        {a->xv, BT * a->Hv * a->dv * es, "xv"}, {a->conv_w, cch * 4 * es, "conv_w"},
+        {a->alpha, na * gs, "alpha"}, {a->b, nb * gs, "b"}, {a->w, nw * gs, "w"},
+        {a->z, BT * a->Hv * a->dv * es, "z"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        {a->grad_y, BT * a->Hv * a->dv * es, "grad_y"}, {a->grad_ht, st, "grad_ht"},
+    };
+    const Buf out[] = {
+        {a->grad_xq, BT * a->Hk * a->dk * 4, "grad_xq"}, {a->grad_xk, BT * a->Hk * a->dk * 4, "grad_xk"},
+        {a->grad_xv, BT * a->Hv * a->dv * 4, "grad_xv"}, {a->grad_conv_w, cch * 4 * 4, "grad_conv_w"},
+        {a->grad_alpha, na * 4, "grad_alpha"}, {a->grad_b, nb * 4, "grad_b"}, {a->grad_w, nw * 4, "grad_w"},
+        {a->grad_z, BT * a->Hv * a->dv * 4, "grad_z"}, {a->grad_h0, st, "grad_h0"},
+    };
+    if ((s = check_buffers(in, 12, out, 9))) return s;
+    cudaStream_t sm = static_cast<cudaStream_t>(stream);
+    if (a->T == 0) {
+        cudaError_t e = cudaMemsetAsync(a->grad_conv_w, 0, cch * 4 * 4, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd");
+        return copy_state(a->grad_h0, a->grad_ht, st, sm, "gdn_layer_core_bwd");
+    }
+    Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    const LayerBwdPlan plan = plan_layer_bwd(a, pb);
+    if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
+    char* wsb = static_cast<char*>(workspace);
+    auto at = [&](size_t o) { return reinterpret_cast<float*>(wsb + o); };
+    cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd");
+    // 1. conv + SiLU + L2, fp32 results
+    ConvParams cp{};
+    cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
+    cp.q = at(plan.q); cp.k = at(plan.k); cp.v = at(plan.v);
+    cp.B = (int)a->B; cp.T = (int)a->T; cp.Hk = (int)a->Hk; cp.Hv = (int)a->Hv; cp.d = (int)a->dk;
+    const bool bf16 = a->dtype == GDN_BF16;
+    e = bf16 ? bf16_conv(cp, sm) : f32_conv(cp, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
+    // 2. the recurrence's output o (fp32, no gate) on the CUDA-core forward
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
+    const WsPlan cplan = plan_chunk_ws(pb, true, !identity_heads(pb));
+    const ChunkWs cws = carve_chunk_ws(cplan, wsb + plan.chunk);
+    ChunkIO io{};
+    io.q = cp.q; io.k = cp.k; io.v = cp.v; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.h0 = a->h0;
+    io.o = at(plan.o); io.o_type = 1;
+    const int var = a->gate_dtype == GDN_F32 ? 2 : 3;
+    e = run_fwd(var, pb, io, cws, f, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+    // 3. swish gate
+    LayerBwdIO lio{};
+    lio.xq = a->xq; lio.xk = a->xk; lio.xv = a->xv; lio.conv_w = a->conv_w; lio.z = a->z; lio.dy = a->grad_y;
+    lio.o = at(plan.o); lio.gq = at(plan.gq); lio.gk = at(plan.gk); lio.gv = at(plan.gv);
+    lio.dout = at(plan.dout); lio.dz = a->grad_z;
+    lio.dxq = a->grad_xq; lio.dxk = a->grad_xk; lio.dxv = a->grad_xv;
+    lio.wpart = at(plan.wpart); lio.dconv_w = a->grad_conv_w;
+    lio.B = (int)a->B; lio.T = (int)a->T; lio.Hk = (int)a->Hk; lio.Hv = (int)a->Hv; lio.d = (int)a->dk;
+    e = layer_gate_bwd(lio, bf16, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (gate)");
+    // 4. the recurrence's backward on the fp32 conv results
+    io.o = nullptr;
+    io.dout = at(plan.dout); io.dht = a->grad_ht;
+    io.dq = at(plan.gq); io.dk = at(plan.gk); io.dv = at(plan.gv);
+    io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = a->grad_w; io.dh0 = a->grad_h0;
+    e = var == 2 ? f32_chunk_bwd(pb, io, cws, f, identity_heads(pb), sm)
+                 : f32_bf16g_chunk_bwd(pb, io, cws, f, identity_heads(pb), sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence)");
+    // 5. L2 norm, SiLU and conv backward, conv-weight gradient
+    e = layer_conv_bwd(lio, bf16, sm);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_bwd (conv)");
+}
+
 gdn_status gdn_workspace_status(const void* workspace, gdn_stream stream) {
     if (!workspace) return fail(GDN_ERR_INVALID_ARG, "workspace is NULL");
     int word = 0;

@@ -66,6 +66,21 @@ TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials, bool caller_cache);
 cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, bool direct,
                          const TcBwdWs& plan, void* ws, const void* cache, cudaStream_t st);
 
+// Layer-core backward pieces (layer_bwd.cu).
+struct LayerBwdIO {
+    const void *xq, *xk, *xv, *conv_w;  // layer inputs (dtype)
+    const void *z, *dy;                 // [B,T,Hv,d] (dtype)
+    const float* o;                     // [B,T,Hv,d] the recurrence's output, before the gate
+    const float *gq, *gk, *gv;          // gradients of the L2-normalised q, k and of v
+    float *dout, *dz;                   // out: gradient of o (fp32), of z
+    float *dxq, *dxk, *dxv;             // out: gradients of the conv inputs
+    float *wpart, *dconv_w;             // per-tile partial sums of the conv-weight gradient; out
+    int B, T, Hk, Hv, d;
+};
+size_t layer_bwd_wpart_floats(int B, int T, int Hk, int Hv, int d);
+cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
+cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
+
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates
 GDN_DECLARE_LAUNCHERS(f32)        // fp32 tensors, fp32 gates

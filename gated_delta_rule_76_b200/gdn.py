@@ -61,10 +61,20 @@ class LayerArgs(ctypes.Structure):
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
 
 
+class LayerBwdArgs(ctypes.Structure):
+    _fields_ = [("xq", P), ("xk", P), ("xv", P), ("conv_w", P), ("alpha", P), ("b", P), ("w", P),
+                ("z", P), ("h0", P), ("head_map", P), ("grad_y", P), ("grad_ht", P),
+                ("grad_xq", P), ("grad_xk", P), ("grad_xv", P), ("grad_conv_w", P), ("grad_alpha", P),
+                ("grad_b", P), ("grad_w", P), ("grad_z", P), ("grad_h0", P),
+                ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
+                ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
+                ("dtype", I32), ("gate_dtype", I32)]
+
+
 EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
-            "gdn_layer_core_fwd", "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches",
-            "gdn_version"]
+            "gdn_layer_core_fwd", "gdn_layer_core_bwd_workspace_size", "gdn_layer_core_bwd",
+            "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches", "gdn_version"]
 
 _lib = None
 
@@ -99,6 +109,10 @@ def load(path: str = LIB_PATH):
     lib.gdn_layer_core_fwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_layer_core_fwd.argtypes = [ctypes.POINTER(LayerArgs), P, ctypes.c_size_t, P]
     lib.gdn_layer_core_fwd.restype = ctypes.c_int
+    lib.gdn_layer_core_bwd_workspace_size.argtypes = [ctypes.POINTER(LayerBwdArgs)]
+    lib.gdn_layer_core_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_layer_core_bwd.argtypes = [ctypes.POINTER(LayerBwdArgs), P, ctypes.c_size_t, P]
+    lib.gdn_layer_core_bwd.restype = ctypes.c_int
     lib.gdn_workspace_status.argtypes = [P, P]
     lib.gdn_workspace_status.restype = ctypes.c_int
     lib.gdn_last_error.argtypes = []
@@ -338,3 +352,40 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
     check(lib.gdn_layer_core_fwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)),
           "gdn_layer_core_fwd")
     return y, ht, cs
+
+
+def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, beta=None, h0=None,
+                       grad_ht=None, head_map=None, scale: float = 1.0, *, want_h0_grad: bool = True,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """GQA layer core backward (reverse mode of gdn_layer_core_fwd).  Returns a dict of fp32
+    gradients: dxq, dxk, dxv, dconv_w, dalpha, dz, dh0 (or None) and db/dw or dbeta."""
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    B, T, Hk, dk = xq.shape
+    Hv, dv = xv.shape[2], xv.shape[3]
+    dev = xq.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dxq": torch.empty((B, T, Hk, dk), **f32), "dxk": torch.empty((B, T, Hk, dk), **f32),
+           "dxv": torch.empty((B, T, Hv, dv), **f32), "dconv_w": torch.empty(tuple(conv_w.shape), **f32),
+           "dalpha": torch.empty(tuple(alpha.shape), **f32), "dz": torch.empty((B, T, Hv, dv), **f32),
+           "dh0": torch.empty((B, Hv, dk, dv), **f32) if want_h0_grad else None}
+    if gpc:
+        out["db"] = torch.empty(tuple(bb.shape), **f32)
+        out["dw"] = torch.empty(tuple(ww.shape), **f32)
+        gb, gw = out["db"], out["dw"]
+    else:
+        out["dbeta"] = torch.empty(tuple(bb.shape), **f32)
+        gb, gw = out["dbeta"], None
+    hm = _head_map(head_map, dev)
+    a = LayerBwdArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
+                     b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), head_map=_ptr(hm), grad_y=_ptr(grad_y),
+                     grad_ht=_ptr(grad_ht), grad_xq=_ptr(out["dxq"]), grad_xk=_ptr(out["dxk"]),
+                     grad_xv=_ptr(out["dxv"]), grad_conv_w=_ptr(out["dconv_w"]), grad_alpha=_ptr(out["dalpha"]),
+                     grad_b=_ptr(gb), grad_w=_ptr(gw), grad_z=_ptr(out["dz"]), grad_h0=_ptr(out["dh0"]),
+                     B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
+                     alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc, dtype=_dt(xq),
+                     gate_dtype=_dt(alpha))
+    lib = load()
+    need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
+    ws = _workspace(need, dev, workspace)
+    check(lib.gdn_layer_core_bwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_layer_core_bwd")
+    return out

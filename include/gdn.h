@@ -254,6 +254,55 @@ GDN_API size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* args);
 GDN_API gdn_status gdn_layer_core_fwd(const gdn_layer_args* args, void* workspace, size_t workspace_bytes,
                               gdn_stream stream);
 
+/* ------------------------------------------------------------------------------------------
+ * GQA layer core (backward): the reverse mode of gdn_layer_core_fwd for the gradients dy of y
+ * and (optionally) dht of the final state.  The explainer's «Architecture et versions hybrides»
+ * (Figure 1 caption) and the mkdocs chapter «Gated DeltaNet» give the layer; each reverse step is
+ * the derivative of its forward step:
+ *   swish gate  y = o * z * sigmoid(z):  do = dy * z s,  dz = dy * o * (s + z s (1 - s)), s = sigmoid(z)
+ *   recurrence  the chunk backward (gdn_chunk_bwd) on the fp32 conv results, with do and dht
+ *   L2 norm     q = a / sqrt(|a|^2 + 1e-6):  da = (dq - q (q . dq)) / sqrt(|a|^2 + 1e-6)
+ *   SiLU        a = u sigmoid(u):  du = da * (s + u s (1 - s))
+ *   conv        u_t = sum_tap w[tap] x_{t-3+tap}:  dx_s = sum_tap w[tap] du_{s+3-tap},
+ *               dconv_w[ch][tap] = sum over tokens of du_t x_{t-3+tap}
+ * The forward parts it needs (conv results, the recurrence's output o) are recomputed in the
+ * workspace.  The recurrence runs on the CUDA-core chunk kernels (fp32 conv results), so the
+ * workspace is large: gdn_layer_core_bwd_workspace_size() says how large.  dk must equal dv.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct gdn_layer_bwd_args {
+    const void* xq;       /* the forward's inputs, as in gdn_layer_args */
+    const void* xk;
+    const void* xv;
+    const void* conv_w;
+    const void* alpha;
+    const void* b;
+    const void* w;
+    const void* z;
+    const float* h0;      /* NULL = zeros */
+    const int32_t* head_map;
+    const void* grad_y;   /* [B,T,Hv,dv] dtype, required */
+    const float* grad_ht; /* [B,Hv,dk,dv] fp32, NULL = zeros */
+    float* grad_xq;       /* out [B,T,Hk,dk] fp32 */
+    float* grad_xk;       /* out [B,T,Hk,dk] fp32 */
+    float* grad_xv;       /* out [B,T,Hv,dv] fp32 */
+    float* grad_conv_w;   /* out [Cch, 4] fp32 */
+    float* grad_alpha;    /* out, shape of alpha, fp32 */
+    float* grad_b;        /* out, shape of b (grad of beta [B,T,Hv] when gates are scalar), fp32 */
+    float* grad_w;        /* out, shape of w with channel gates; NULL otherwise */
+    float* grad_z;        /* out [B,T,Hv,dv] fp32 */
+    float* grad_h0;       /* out [B,Hv,dk,dv] fp32, may be NULL */
+    int64_t B, T, Hk, Hv, dk, dv;
+    float scale;
+    int32_t alpha_per_channel;
+    int32_t gates_per_channel;
+    int32_t dtype;
+    int32_t gate_dtype;
+} gdn_layer_bwd_args;
+
+GDN_API size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* args);
+GDN_API gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* args, void* workspace, size_t workspace_bytes,
+                                      gdn_stream stream);
+
 /* Device-side status of the last call that used `workspace` (a chunk forward, backward or layer
  * core).  The tensor-core kernels bound every internal wait; when one expires the kernel records
  * it in the workspace, stops issuing work, releases its tensor memory and returns.  This call

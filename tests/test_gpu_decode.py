@@ -155,3 +155,27 @@ def test_decode_negative_eigenvalue_gates():
                                               b=tk(x, "b"), w=tk(x, "w"))
         assert_parity(o, o_ref, "bf16", f"o step {t}")
     assert_parity(state, ref_state, "bf16", "state")
+
+
+@pytest.mark.parametrize("B,T,Hk,Hv,d,gpc,gdt,dt", [
+    (2, 150, 2, 4, 64, False, "f32", "bf16"),    # GQA, scalar gates, ragged tail
+    (1, 130, 1, 2, 128, False, "bf16", "bf16"),  # d = 128, bf16 gates
+    (1, 100, 1, 2, 64, True, "bf16", "bf16"),    # channel gates
+    (1, 70, 1, 1, 64, False, "f32", "f32"),      # fp32 tensors
+])
+def test_layer_core_backward_matches_oracle(B, T, Hk, Hv, d, gpc, gdt, dt):
+    """gdn_layer_core_bwd against the oracle's reverse mode of the layer (itself pinned by finite
+    differences): gradients of the conv inputs, the conv weights, the gates, z and h0."""
+    x = draw(B, T, Hk, Hv, d, d, alpha_per_channel=gpc, gates_per_channel=gpc, dtype=dt,
+             gate_dtype=gdt, seed=61, has_h0=True, conv=True, swish_gate=True, with_dout=True, with_dht=True)
+    g = to_cuda(x)
+    gk = dict(beta=g["beta"]) if not gpc else dict(b=g["b"], w=g["w"])
+    xk = dict(beta=x["beta"]) if not gpc else dict(b=x["b"], w=x["w"])
+    got = gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"], h0=g["h0"],
+                                 grad_ht=g["dht"], scale=0.8, **gk)
+    torch.cuda.synchronize()
+    ref = oracle.layer_core_bwd(x["q"], x["k"], x["v"], x["conv_w"], x["alpha"], x["z"], x["dout"], h0=x["h0"],
+                                dht=x["dht"], scale=0.8, **xk)
+    kind = "f32" if dt == "f32" else "bf16"
+    for key in ["dxq", "dxk", "dxv", "dconv_w", "dalpha", "dz", "dh0"] + (["db", "dw"] if gpc else ["dbeta"]):
+        assert_parity(got[key], ref[key], kind, key)

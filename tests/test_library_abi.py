@@ -53,7 +53,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 STRUCTS = {"gdn_fwd_args": gdn.FwdArgs, "gdn_bwd_args": gdn.BwdArgs,
-           "gdn_decode_args": gdn.DecodeArgs, "gdn_layer_args": gdn.LayerArgs}
+           "gdn_decode_args": gdn.DecodeArgs, "gdn_layer_args": gdn.LayerArgs,
+           "gdn_layer_bwd_args": gdn.LayerBwdArgs}
 
 
 def test_ctypes_structs_match_c_layout():
