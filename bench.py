@@ -467,6 +467,36 @@ def bench_part_fwd(name, args, dist, peaks, peak_kind, stream, device):
                        "gates": "channel" if wl.gates_per_channel else "scalar beta"}}
 
 
+def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
+    """The GQA layer core's training step: gdn_layer_core_fwd then gdn_layer_core_bwd (the
+    recurrence's backward on the CUDA-core kernels), inputs resident, gradients of every input."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import WORKLOADS
+    name = "gqa_layer_core_bf16"
+    wl = WORKLOADS[name]
+    x, g = chunk_inputs(name, device, with_dout=True)
+    y = torch.empty_like(g["v"])
+    with torch.cuda.stream(stream):
+        def fn():
+            gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], y=y, want_ht=False,
+                                   stream=stream, **gates(g))
+            gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"],
+                                   stream=stream, **gates(g))
+        ms = timed(fn, max(2, args.steps // 4), args.warmup, dist, stream)
+    tokens = wl.B * wl.T
+    by = (fwd_bytes_per_token(wl, gate=True) + bwd_bytes_per_token(wl)
+          + wl.Hv * wl.dv * (_es(wl.dtype) + 4)) * tokens               # + z read, fp32 dz written
+    fl = (fwd_flops_per_token(wl) + bwd_flops_per_token(wl)) * tokens
+    del x, g
+    return {"workload": name + " (training step: layer forward + backward)",
+            "value": tokens / (ms * 1e-3) * dist.world, "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "roofline": roofline(by, fl, ms * 1e-3, peaks, peak_kind,
+                                 "gdn_layer_core_fwd + gdn_layer_core_bwd calls"),
+            "config": {"B": wl.B, "T": wl.T, "Hk": wl.Hk, "Hv": wl.Hv, "dk": wl.dk, "dv": wl.dv,
+                       "backward": "recurrence on the CUDA-core chunk kernels (fp32 conv results)"}}
+
+
 # --------------------------------------------------------------------------------------------
 # CPU oracle timings (baseline and reference arm)
 # --------------------------------------------------------------------------------------------
@@ -641,6 +671,8 @@ def main():
         torch.cuda.empty_cache()
     if "layer" in parts:
         sub["gqa_layer_core"] = bench_part_fwd("gqa_layer_core_bf16", args, dist, peaks, peak_kind, stream, device)
+        torch.cuda.empty_cache()
+        sub["gqa_layer_train"] = bench_part_layer_train(args, dist, peaks, peak_kind, stream, device)
         torch.cuda.empty_cache()
     clk = clocks.stop()
 
