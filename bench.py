@@ -346,31 +346,59 @@ def bench_headline(args, dist, peaks, peak_kind, stream, device):
             "fwd_roofline": roofline(bytes_f, flops_f, fwd_ms * 1e-3, peaks, peak_kind, "gdn_chunk_fwd call")}, (x, g, o, ht, grads)
 
 
-def bench_headline_e2e(args, dist, x, stream, device):
+def bench_headline_e2e(args, dist, x, stream, device, slices=8):
     """Same metric through the public API with host buffers: H2D of the step's inputs from pinned
-    memory, forward + backward, D2H of every result, all inside the timed region."""
+    memory, forward + backward, D2H of every result, all inside the timed region.  The batch's
+    sequences are independent, so the step runs as `slices` slices of the batch on three streams
+    (copy in, compute, copy out): the copies of one slice overlap the compute and the
+    other-direction copies of the others, and the PCIe link carries both directions at once."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     names_in = ["q", "k", "v", "alpha", "b", "w", "h0", "dout"]
     host = {n: x[n].pin_memory() for n in names_in}
     dev = {n: torch.empty_like(host[n], device=device) for n in names_in}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
+    B = host["q"].shape[0]
+    ns = slices if B % slices == 0 else 1
+    sb = B // ns
+    cut = lambda t, i: t[i * sb:(i + 1) * sb]
+    caches = [torch.empty(gdn.gdn_chunk_fwd_cache_size(cut(dev["q"], i), cut(dev["k"], i), cut(dev["v"], i),
+                                                       cut(dev["alpha"], i), b=cut(dev["b"], i), w=cut(dev["w"], i),
+                                                       h0=cut(dev["h0"], i)), dtype=torch.uint8, device=device)
+              for i in range(ns)]
+    s_in, s_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
     out_host = {}
-    cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"],
-                                                     w=dev["w"], h0=dev["h0"]), dtype=torch.uint8, device=device)
 
     def step():
-        for n in names_in:
-            dev[n].copy_(host[n], non_blocking=True)
-        o, ht = gdn.gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
-                                  h0=dev["h0"], bwd_cache=cache, stream=stream)
-        gr = gdn.gdn_chunk_bwd(dev["q"], dev["k"], dev["v"], dev["alpha"], b=dev["b"], w=dev["w"],
-                               h0=dev["h0"], grad_o=dev["dout"], fwd_cache=cache, stream=stream)
-        res = {"o": o, "ht": ht, **gr}
-        for n, t in res.items():
-            if n not in out_host:
-                out_host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-            out_host[n].copy_(t, non_blocking=True)
+        s_in.wait_stream(stream)
+        ev_in = []
+        with torch.cuda.stream(s_in):
+            for i in range(ns):
+                for n in names_in:
+                    cut(dev[n], i).copy_(cut(host[n], i), non_blocking=True)
+                ev_in.append(torch.cuda.Event())
+                ev_in[-1].record(s_in)
+        res, ev_c = [], []
+        for i in range(ns):
+            stream.wait_event(ev_in[i])
+            d = {n: cut(dev[n], i) for n in names_in}
+            o, ht = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], b=d["b"], w=d["w"], h0=d["h0"],
+                                      bwd_cache=caches[i], stream=stream)
+            gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], b=d["b"], w=d["w"], h0=d["h0"],
+                                   grad_o=d["dout"], fwd_cache=caches[i], stream=stream)
+            res.append({"o": o, "ht": ht, **gr})
+            ev_c.append(torch.cuda.Event())
+            ev_c[-1].record(stream)
+        with torch.cuda.stream(s_out):
+            for i in range(ns):
+                s_out.wait_event(ev_c[i])
+                for n, t in res[i].items():
+                    if n not in out_host:
+                        out_host[n] = torch.empty((B,) + tuple(t.shape[1:]), dtype=t.dtype, pin_memory=True)
+                    cut(out_host[n], i).copy_(t, non_blocking=True)
+        # the timing stream ends after the last copy; the slices' device outputs are released
+        # only after that point in stream order
+        stream.wait_stream(s_out)
 
     with torch.cuda.stream(stream):
         ms = timed(step, max(2, args.steps // 4), 1, dist, stream)
