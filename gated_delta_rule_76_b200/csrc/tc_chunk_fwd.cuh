@@ -132,14 +132,7 @@ struct Params {
 __device__ __forceinline__ float bf(const uint8_t* tile, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
 }
-__device__ __forceinline__ void put_raw(uint8_t* tile, uint32_t off, __nv_bfloat16 v) {
-    *reinterpret_cast<__nv_bfloat16*>(tile + off) = v;
-}
-// x = hi + lo with hi = bf16(x), lo = bf16(x - hi).
-__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-    hi = __float2bfloat16_rn(x);
-    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-}
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi), for two values at once (bf16x2 pairs).
 __device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     hi = pack_bf16x2(x0, x1);
     const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);

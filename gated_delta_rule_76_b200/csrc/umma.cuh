@@ -121,22 +121,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
-// 32 lanes x 16 consecutive 32-bit columns per warp (same lane mapping as tmem_ld32).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-// 32 lanes x 4 consecutive 32-bit columns per warp (same lane mapping as tmem_ld32).
-__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(taddr));
-}
 // 32 lanes x 8 consecutive 32-bit columns per warp (same lane mapping as tmem_ld32).
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -275,25 +259,6 @@ __device__ __forceinline__ void mma_ts_k(uint32_t d_tmem, uint32_t a_tmem, uint3
         const uint32_t b = b_smem + (uint32_t)(k >> 6) * (uint32_t)b_rows * 128u + (uint32_t)(k & 63) * 2u;
         mma_ts(d_tmem, a_tmem + (uint32_t)(k >> 1), sdesc_k_sw128(b), idesc, (accumulate || k > 0) ? 1u : 0u);
     }
-}
-
-// ---- TMA ------------------------------------------------------------------------------------------
-// Tiled bulk tensor load into shared memory, completion signalled on an mbarrier (bytes counted
-// via expect_tx).  No multicast.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void* tmap, uint64_t* bar, int c0, int c1,
-                                            int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst_smem),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// Bulk prefetch of the global range [gaddr, gaddr + bytes) into L2 (16-byte aligned start, bytes a
-// multiple of 16).  Nothing is written; the issuing thread does not wait.
-__device__ __forceinline__ void prefetch_l2(const void* gaddr, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)), "r"(bytes)
-                 : "memory");
 }
 
 // Prefetch of the 128-byte line holding gaddr into L2 (load/store path; the thread does not wait).
