@@ -140,3 +140,39 @@ def test_forward_cache_validation_on_the_host(lib):
     assert lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), 1 << 30, None) == 1
     a = _fwd(bwd_cache=1 << 20, bwd_cache_bytes=1 << 20)
     assert lib.gdn_chunk_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), 1 << 30, None) == 1
+
+
+def _layer_bwd(**kw):
+    M = 1 << 16
+    base = dict(xq=16, xk=32, xv=48, conv_w=64, alpha=80, b=96, w=None, z=112, h0=None, head_map=None,
+                grad_y=128, grad_ht=None, grad_xq=16 * M, grad_xk=17 * M, grad_xv=18 * M, grad_conv_w=19 * M,
+                grad_alpha=20 * M, grad_b=21 * M, grad_w=None, grad_z=22 * M, grad_h0=None,
+                B=1, T=64, Hk=1, Hv=1, dk=64, dv=64, scale=1.0, alpha_per_channel=0, gates_per_channel=0,
+                dtype=0, gate_dtype=1)
+    base.update(kw)
+    return gdn.LayerBwdArgs(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=64, dv=128), 2),                 # the layer needs dk == dv
+    (dict(grad_y=None), 1),                   # missing gradient of y
+    (dict(grad_conv_w=None), 1),              # missing output
+    (dict(grad_w=23 << 16), 1),               # scalar gates but grad_w given
+    (dict(gates_per_channel=1, alpha_per_channel=1), 1),  # channel gates without w / grad_w
+    (dict(grad_xq=16), 1),                    # output overlaps an input
+    (dict(grad_z=(22 << 16) + 8), 1),         # misaligned output
+])
+def test_layer_backward_host_validation(lib, kw, code):
+    a = _layer_bwd(**kw)
+    rc = lib.gdn_layer_core_bwd(ctypes.byref(a), ctypes.c_void_p(1 << 34), 1 << 34, None)
+    assert rc == code, lib.gdn_last_error()
+    assert lib.gdn_last_error().decode()
+
+
+def test_layer_backward_workspace(lib):
+    a = _layer_bwd()
+    need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
+    assert need > 0
+    assert lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(_layer_bwd(T=65))) > need
+    assert lib.gdn_layer_core_bwd(ctypes.byref(a), ctypes.c_void_p(1 << 34), need - 1, None) == 4
+    assert lib.gdn_layer_core_bwd(None, None, 0, None) == 1
