@@ -1127,20 +1127,6 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
                                                 float gam, float xtot, float* scr, int it) {
     const float scale = p.pb.scale;
     const RowPtrs rp = row_ptrs(p, cp, c);
-    {
-        // The walk reads the chunk's q, k, b, alpha rows 8 tokens at a time, one block ahead; most
-        // of them have left L2 since the staging group's load a chunk ago.  Request every line
-        // now (thread c: token c / 2, 128-byte half c % 2 of each 256-byte row).
-        const int r = c >> 1;
-        if (FULL || r < cp.L) {
-            const long hq = rp.qk - c + r * rp.qk_s + 64 * (c & 1);
-            prefetch_line_l2(p.q + hq);
-            prefetch_line_l2(p.k + hq);
-            const long hg = rp.g - c + r * rp.g_s + 64 * (c & 1);
-            if (GPC) prefetch_line_l2(static_cast<const TG*>(p.b) + hg);
-            if (APC) prefetch_line_l2(static_cast<const TG*>(p.alpha) + hg);
-        }
-    }
     float G = gam, rg = __fdividef(1.f, gam), run = 0.f;
     auto do_block = [&](int blk, const RowIn& x) {
         uint32_t rq[RB], re[RB], rk[RB], rb[RB];

@@ -261,11 +261,6 @@ __device__ __forceinline__ void mma_ts_k(uint32_t d_tmem, uint32_t a_tmem, uint3
     }
 }
 
-// Prefetch of the 128-byte line holding gaddr into L2 (load/store path; the thread does not wait).
-__device__ __forceinline__ void prefetch_line_l2(const void* gaddr) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(gaddr)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
