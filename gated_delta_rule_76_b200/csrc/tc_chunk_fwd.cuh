@@ -26,16 +26,19 @@
 // the fp32 state in registers, split between the warpgroups by halves of dk.
 // Roles (384 threads):
 //   warps 0-7  (scan)     : the sequential chain X2 -> Y -> X3 -> V' -> X4, X5 -> output, state;
-//                           while the prologue solves for T they also build P (from X1) and
-//                           Kbar^T (from the split Ktil).  Thread 0 issues the scan's MMAs and all
-//                           TMA loads.
+//                           while X2 runs they build Kbar^T (from the split Ktil and gamma), and
+//                           while the prologue solves for T they build P (from X1).  Thread 0
+//                           issues the scan's MMAs and all TMA loads (the z tile of a gated output
+//                           at the top of each chunk).
 //   warps 8-11 (prologue) : for the next chunk, the cumulative decay and the split operands, X1,
 //                           and the triangular solve T = (I + A)^-1; thread 256 issues X1.
 // Operand tiles are single-buffered.  [Ehat;Qhat] and T each have a "ready" barrier (prologue ->
 // scan) and a "free" barrier (the scan's MMA that read it has completed -> prologue); the raw TMA
-// stage is reloaded once X1 and the Kbar^T pass (its last readers) are done.  Every mbarrier wait
-// is bounded: on expiry the kernel sets an error word, stops issuing work and frees its tensor
-// memory.
+// stage is reloaded as soon as X1 and the Kbar^T pass (its last readers) are done.  Saving mode
+// (the backward cache) stores the entering state and V' while the MMAs run.  Split inputs (fp32
+// q, k, v as bf16 hi/lo pairs, scalar gates only) take the lo tiles in the gate slots.  Every
+// mbarrier wait is bounded: on expiry the kernel sets an error word, stops issuing work and frees
+// its tensor memory.
 #pragma once
 #include <cuda.h>
 
