@@ -22,8 +22,11 @@
 //      the state gradient dS is carried in registers (thread j: column j), its chain per chunk
 //      is  XA = dO^T P + dS^T Kbar^T (= dV'^T)  ->  XC = dO^T Qhat - dV'^T W (= dS0^T without
 //      the decay term)  ->  dS = Diag(gamma) dS + XC^T;  off the chain it forms -dY^T = -dV'^T T.
-//      It saves dS_end of every chunk (fp32) and -dY of every token (bf16 hi/lo), and writes dh0;
-//   3. chunk_bwd_grad_kernel (this file): one CTA per chunk, every gradient of the chunk's inputs.
+//      The prologue warps build the chunk's factors, X1, P and T; the chain warps form W^T from
+//      T and the split Ehat tiles and request the next chunk's raw tiles.  It saves dS_end of
+//      every chunk (fp32) and -dY of every token (bf16 hi/lo), and writes dh0;
+//   3. chunk_bwd_grad_kernel (this file): persistent, one CTA per SM walking the chunks; every
+//      gradient of a chunk's inputs.
 #pragma once
 #include <cuda.h>
 
@@ -89,7 +92,7 @@ constexpr uint32_t TM_DSH = 256;  // 64:  dS^T hi (bf16 pairs)
 constexpr uint32_t TM_DSL = 320;  // 64:  dS^T lo
 constexpr uint32_t TM_DVH = 384;  // 32:  -dV'^T hi
 constexpr uint32_t TM_DVL = 416;  // 32:  -dV'^T lo
-constexpr uint32_t TM_WT = 448;   // 64:  W^T = Ehat^T T^T of the prologue's chunk
+constexpr uint32_t TM_WT = 448;   // 64:  W^T = Ehat^T T^T of the chain's chunk
 constexpr uint32_t TM_COLS = 512;
 
 // shared memory (1024-byte-aligned base; bf16 tiles with the 128-byte swizzle)
