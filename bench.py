@@ -111,7 +111,7 @@ def load_peaks():
 # of its two kernels (reverse scan, gradients) on B=2 T=2048 (an eighth of the workload's tokens:
 # the per-chunk traffic is fixed, so it scales with the tokens); see
 # profiles/chunk_bwd_kernels_gdn2_b2_t2048.md.  To be set to None whenever those kernels change.
-BWD_CALL_TRAFFIC_BYTES = (84.07 + 54.87 + 360.25 + 155.14) * 1e6 * 8
+BWD_CALL_TRAFFIC_BYTES = (84.17 + 54.30 + 360.25 + 154.68) * 1e6 * 8
 
 
 def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False,
@@ -634,8 +634,25 @@ def _profile_layer_b2_t16384():
     return 0
 
 
+def _profile_train_b8_t4096():
+    """The headline training step (gdn_chunk_fwd keeping the cache, gdn_chunk_bwd from it) on its
+    full workload, three times."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    x, g = chunk_inputs(HEADLINE, torch.device("cuda"), with_dout=True)
+    kw = dict(b=g["b"], w=g["w"], h0=g["h0"])
+    cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], **kw),
+                        dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
+        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache, **kw)
+    torch.cuda.synchronize()
+    print("ok", float(grads["dq"].abs().mean()))
+    return 0
+
+
 PROFILE_CASES = {"train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024,
-                 "layer_b2_t16384": _profile_layer_b2_t16384}
+                 "layer_b2_t16384": _profile_layer_b2_t16384, "train_b8_t4096": _profile_train_b8_t4096}
 
 
 def main():
