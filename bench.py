@@ -651,8 +651,25 @@ def _profile_train_b8_t4096():
     return 0
 
 
+def _profile_layer_train_b2_t16384():
+    """GQA layer core's training step (gdn_layer_core_fwd, then gdn_layer_core_bwd) on its full
+    workload, once."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import workload_inputs
+    x = workload_inputs("gqa_layer_core_bf16", with_dout=True)
+    g = {k: v.cuda() for k, v in x.items()}
+    y, _, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], beta=g["beta"])
+    grads = gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"],
+                                   beta=g["beta"])
+    torch.cuda.synchronize()
+    print("ok", float(y.float().abs().mean()), float(grads["dxq"].abs().mean()))
+    return 0
+
+
 PROFILE_CASES = {"train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024,
-                 "layer_b2_t16384": _profile_layer_b2_t16384, "train_b8_t4096": _profile_train_b8_t4096}
+                 "layer_b2_t16384": _profile_layer_b2_t16384, "train_b8_t4096": _profile_train_b8_t4096,
+                 "layer_train_b2_t16384": _profile_layer_train_b2_t16384}
 
 
 def main():

@@ -604,8 +604,10 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     const bool bf16 = a->dtype == GDN_BF16;
     e = bf16 ? bf16_conv(cp, sm) : f32_conv(cp, sm);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
-    // 2. the recurrence's output o (fp32, no gate) on the CUDA-core forward
+    // 2. the recurrence's output o (fp32, no gate) on the CUDA-core forward, which also keeps
+    //    the chunk states for step 4 (paired: the backward does not run the forward again)
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
+    f.paired = true;
     const WsPlan cplan = plan_chunk_ws(pb, true, !identity_heads(pb));
     const ChunkWs cws = carve_chunk_ws(cplan, wsb + plan.chunk);
     ChunkIO io{};

@@ -18,6 +18,14 @@ cudaError_t launch_kernel(K kernel, dim3 grid, dim3 block, size_t smem, cudaStre
     return cudaGetLastError();
 }
 
+// dq or dk of the key heads from the per-value-head partials [B,T,Hv,dk] (gqa_reduce_kernel).
+inline cudaError_t gqa_reduce(const Problem& pb, const float* part, float* out, cudaStream_t st) {
+    const long rows = (long)pb.B * pb.T;
+    const int blocks = (int)(rows < 148L * 8 ? rows : 148L * 8);
+    return launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), (size_t)(pb.Hv + pb.Hk + 1) * sizeof(int), st,
+                         pb, part, out);
+}
+
 #define GDN_TRY(expr)                         \
     do {                                      \
         cudaError_t e_ = (expr);              \
@@ -30,7 +38,7 @@ cudaError_t chunk_fwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
     const dim3 block(kSimtThreads);
     GDN_TRY(launch_kernel(chunk_prep_kernel<TIn, TG, APC, GPC, DK>, dim3(pb.NT, pb.Hv, pb.B),
                           block, chunk_prep_smem<DK>(), st, pb, io, ws, save_states ? 1 : 0));
-    const dim3 sgrid(pb.dv / kDvTile, pb.Hv, pb.B);
+    const dim3 sgrid(pb.dv / kDvTileFwd, pb.Hv, pb.B);
     if (gate)
         return launch_kernel(chunk_scan_fwd_kernel<TIn, TG, GPC, DK, true>, sgrid, block,
                              chunk_scan_fwd_smem<DK>(), st, pb, io, ws, write_out ? 1 : 0,
@@ -42,20 +50,16 @@ cudaError_t chunk_fwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
 
 template <class TIn, class TG, bool APC, bool GPC, int DK>
 cudaError_t chunk_bwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws, bool direct_qk,
-                        cudaStream_t st) {
+                        bool paired, cudaStream_t st) {
     const dim3 block(kSimtThreads);
-    GDN_TRY((chunk_fwd_t<TIn, TG, APC, GPC, DK>(pb, io, ws, false, true, false, st)));
+    if (!paired) GDN_TRY((chunk_fwd_t<TIn, TG, APC, GPC, DK>(pb, io, ws, false, true, false, st)));
     GDN_TRY(launch_kernel(chunk_scan_bwd_kernel<TIn, TG, GPC, DK>, dim3(pb.dv / kDvTile, pb.Hv, pb.B),
                           block, chunk_scan_bwd_smem<DK>(), st, pb, io, ws));
     GDN_TRY(launch_kernel(chunk_grad_kernel<TIn, TG, APC, GPC, DK, DK>, dim3(pb.NT, pb.Hv, pb.B),
                           block, chunk_grad_smem<DK, DK>(), st, pb, io, ws, direct_qk ? 1 : 0));
     if (!direct_qk) {
-        const long total = (long)pb.B * pb.T * pb.Hk * pb.dk;
-        const int blocks = static_cast<int>((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
-        GDN_TRY(launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb,
-                              (const float*)ws.dq_v, static_cast<float*>(io.dq)));
-        GDN_TRY(launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb,
-                              (const float*)ws.dk_v, static_cast<float*>(io.dk)));
+        GDN_TRY(gqa_reduce(pb, (const float*)ws.dq_v, static_cast<float*>(io.dq), st));
+        GDN_TRY(gqa_reduce(pb, (const float*)ws.dk_v, static_cast<float*>(io.dk), st));
     }
     return cudaSuccess;
 }
@@ -79,7 +83,7 @@ cudaError_t chunk_fwd_impl(const Problem& pb, const ChunkIO& io, const ChunkWs& 
                            cudaStream_t st) {
     return dispatch_chunk<TIn, TG>(pb, f, [&](auto apc, auto gpc, auto dk) {
         return chunk_fwd_t<TIn, TG, decltype(apc)::value, decltype(gpc)::value, decltype(dk)::value>(
-            pb, io, ws, f.gate, false, true, st);
+            pb, io, ws, f.gate, f.paired, true, st);
     });
 }
 
@@ -88,7 +92,7 @@ cudaError_t chunk_bwd_impl(const Problem& pb, const ChunkIO& io, const ChunkWs& 
                            bool direct_qk, cudaStream_t st) {
     return dispatch_chunk<TIn, TG>(pb, f, [&](auto apc, auto gpc, auto dk) {
         return chunk_bwd_t<TIn, TG, decltype(apc)::value, decltype(gpc)::value, decltype(dk)::value>(
-            pb, io, ws, direct_qk, st);
+            pb, io, ws, direct_qk, f.paired, st);
     });
 }
 

@@ -19,6 +19,9 @@ struct Flags {
     bool apc;   // alpha per channel
     bool gpc;   // b, w per channel (else scalar beta)
     bool gate;  // swish(z) output gate in the forward
+    // CUDA-core path, a forward and a backward on one workspace: the forward also saves what the
+    // backward needs (chunk states, Kt, G), and the backward does not run the forward again.
+    bool paired = false;
 };
 
 // Workspace carving.  Every array is 256-byte aligned.

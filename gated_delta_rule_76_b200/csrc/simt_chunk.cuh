@@ -23,7 +23,8 @@
 namespace gdn {
 
 constexpr int kSimtThreads = 256;
-constexpr int kDvTile = 32;  // dv columns per scan CTA
+constexpr int kDvTile = 32;     // dv columns per backward scan CTA
+constexpr int kDvTileFwd = 64;  // dv columns per forward scan CTA (4 x 4 register tiles)
 
 // CTA-wide element loop over N = IT * kSimtThreads indices: every load of a thread is issued before
 // any of its stores, so their latencies overlap (load(idx) -> float, store(idx, value)).
@@ -76,9 +77,11 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
     float* Eh = smem;                 // [C][LD]
     float* Qh = Eh + C * LD;          // [C][LD]
     float* Kt = Qh + C * LD;          // [C][LD]
-    float* A = Kt + C * LD;           // [C][LC]
-    float* Tm = A + C * LC;           // [C][LC]
-    float* scratch = Tm + C * LC;
+    float* scratch = Kt + C * LD;
+    // A [C][LC] takes Eh's space once the first product has read it, T [C][LC] takes Qh's once the
+    // second has (each product ends with a CTA barrier): two CTAs fit on an SM.
+    float* A = Eh;
+    float* Tm = Qh;
 
     const int n = blockIdx.x, hv = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
     const int hk = pb.key_head(hv);
@@ -126,7 +129,7 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
     __syncthreads();
 
     // A = strict_lower(Ehat Ktil^T), P = lower(Qhat Ktil^T).
-    using G64 = BlockGemm<C, C, kSimtThreads, 32>;
+    using G64 = BlockGemm<C, C, kSimtThreads, 32, 16>;
     {
         G64 g;
         g.zero();
@@ -172,8 +175,8 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
 
 template <int DK>
 constexpr size_t chunk_prep_smem() {
-    return sizeof(float) * (3 * kChunk * (DK + 1) + 2 * kChunk * (kChunk + 1) +
-                            BlockGemm<kChunk, kChunk, kSimtThreads, 32>::kScratch);
+    static_assert(DK >= kChunk, "A and T reuse the space of Ehat and Qhat");
+    return sizeof(float) * (3 * kChunk * (DK + 1) + BlockGemm<kChunk, kChunk, kSimtThreads, 32, 16>::kScratch);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -182,7 +185,7 @@ constexpr size_t chunk_prep_smem() {
 template <class TIn, class TG, bool GPC, int DK, bool GATE>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int save_states) {
-    constexpr int C = kChunk, W = kDvTile;
+    constexpr int C = kChunk, W = kDvTileFwd;
     extern __shared__ float smem[];
     float* S = smem;            // [DK][W]
     float* Z = S + DK * W;      // [C][W]
@@ -299,8 +302,8 @@ chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int sav
 
 template <int DK>
 constexpr size_t chunk_scan_fwd_smem() {
-    return sizeof(float) * (DK * kDvTile + 3 * kChunk * kDvTile +
-                            BlockGemm<DK, kDvTile, kSimtThreads, 16>::kScratch);
+    return sizeof(float) * (DK * kDvTileFwd + 3 * kChunk * kDvTileFwd +
+                            BlockGemm<DK, kDvTileFwd, kSimtThreads, 16>::kScratch);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -732,19 +735,36 @@ constexpr size_t chunk_grad_smem() {
 }
 
 // Sum per-value-head dq/dk [B,T,Hv,dk] over the value heads of each key head, ascending hv
-// (fixed order: deterministic).
-static __global__ void gqa_reduce_kernel(Problem pb, const float* part, float* out) {
-    const long total = (long)pb.B * pb.T * pb.Hk * pb.dk;
-    for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total;
-         idx += (long)gridDim.x * blockDim.x) {
-        const int c = idx % pb.dk;
-        const long row = idx / pb.dk;
-        const int hk = row % pb.Hk;
-        const long bt = row / pb.Hk;
-        float s = 0.f;
-        for (int hv = 0; hv < pb.Hv; ++hv)
-            if (pb.key_head(hv) == hk) s += part[(bt * pb.Hv + hv) * pb.dk + c];
-        out[idx] = s;
+// (fixed order: deterministic).  The block first lists the value heads of every key head in
+// shared memory (dynamic: Hv + Hk + 1 ints); then each thread sums float4 columns of one token
+// row at a time.  dk is a multiple of 4 and every row starts 16-byte aligned.
+static __global__ void __launch_bounds__(256) gqa_reduce_kernel(Problem pb, const float* part, float* out) {
+    extern __shared__ int heads[];  // heads[0 .. Hv): value heads grouped by key head; then Hk + 1 starts
+    int* beg = heads + pb.Hv;
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int hk = 0; hk < pb.Hk; ++hk) {
+            beg[hk] = n;
+            for (int hv = 0; hv < pb.Hv; ++hv)
+                if (pb.key_head(hv) == hk) heads[n++] = hv;
+        }
+        beg[pb.Hk] = n;
+    }
+    __syncthreads();
+    const int q4 = pb.dk / 4, per_row = pb.Hk * q4;
+    const long rows = (long)pb.B * pb.T;
+    const float4* src = reinterpret_cast<const float4*>(part);
+    float4* dst = reinterpret_cast<float4*>(out);
+    for (long bt = blockIdx.x; bt < rows; bt += gridDim.x) {
+        for (int i = threadIdx.x; i < per_row; i += blockDim.x) {
+            const int hk = i / q4, c = i - hk * q4;
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = beg[hk]; j < beg[hk + 1]; ++j) {
+                const float4 x = __ldg(src + (bt * pb.Hv + heads[j]) * q4 + c);
+                s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
+            }
+            dst[bt * per_row + i] = s;
+        }
     }
 }
 

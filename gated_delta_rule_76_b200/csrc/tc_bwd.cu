@@ -170,12 +170,8 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     if (e != cudaSuccess || direct) return e;
 
     // 3. GQA: sum the per-value-head dq, dk over the value heads of each key head
-    const long total = (long)pb.B * pb.T * pb.Hk * pb.dk;
-    const int blocks = (int)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
-    GDN_TRY(launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb, (const float*)dq_v,
-                          static_cast<float*>(io.dq)));
-    return launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), 0, st, pb, (const float*)dk_v,
-                         static_cast<float*>(io.dk));
+    GDN_TRY(gqa_reduce(pb, (const float*)dq_v, static_cast<float*>(io.dq), st));
+    return gqa_reduce(pb, (const float*)dk_v, static_cast<float*>(io.dk), st);
 }
 
 }  // namespace gdn
