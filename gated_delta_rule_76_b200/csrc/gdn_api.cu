@@ -522,11 +522,17 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
 }
 
 // Workspace of the layer backward: the recomputed conv results (fp32), the recurrence's output o
-// and its gradient, the gradients of q, k, v from the recurrence, the conv-weight partials, then
-// the CUDA-core chunk backward's own workspace.  Offsets from the start, 256-byte aligned.
+// and its gradient, the gradients of q, k, v from the recurrence, the conv-weight partials, the
+// tensor-core forward's chunk states (bf16 tensors with d = 128 and scalar gates), then the
+// CUDA-core chunk backward's own workspace.  Offsets from the start, 256-byte aligned.
 struct LayerBwdPlan {
-    size_t q, k, v, o, dout, gq, gk, gv, wpart, chunk, bytes;
+    size_t q, k, v, o, dout, gq, gk, gv, wpart, s0tc, chunk, bytes;
 };
+// The layer backward's forward (o and the chunk states) runs on the tensor cores, from the conv
+// results as bf16 hi/lo pairs, when the layer forward would.
+static bool layer_bwd_tc_form(const gdn_layer_bwd_args* a) {
+    return a->dtype == GDN_BF16 && a->dk == 128 && a->dv == 128 && !a->alpha_per_channel && !a->gates_per_channel;
+}
 static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& pb) {
     LayerBwdPlan w{};
     const size_t BT = (size_t)(a->B * a->T), qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
@@ -539,6 +545,7 @@ static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& p
     w.q = take(qn); w.k = take(qn); w.v = take(vn); w.o = take(vn); w.dout = take(vn);
     w.gq = take(qn); w.gk = take(qn); w.gv = take(vn);
     w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk));
+    w.s0tc = layer_bwd_tc_form(a) ? take((size_t)a->B * a->Hv * (pb.NT + 1) * a->dk * a->dv) : ~size_t(0);
     w.chunk = off;
     w.bytes = off + plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
     return w;
@@ -604,8 +611,8 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     const bool bf16 = a->dtype == GDN_BF16;
     e = bf16 ? bf16_conv(cp, sm) : f32_conv(cp, sm);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
-    // 2. the recurrence's output o (fp32, no gate) on the CUDA-core forward, which also keeps
-    //    the chunk states for step 4 (paired: the backward does not run the forward again)
+    // 2. the recurrence's output o (fp32, no gate) and the chunk states for step 4 (paired: the
+    //    backward does not run the forward again)
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
     f.paired = true;
     const WsPlan cplan = plan_chunk_ws(pb, true, !identity_heads(pb));
@@ -614,8 +621,33 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     io.q = cp.q; io.k = cp.k; io.v = cp.v; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.h0 = a->h0;
     io.o = at(plan.o); io.o_type = 1;
     const int var = a->gate_dtype == GDN_F32 ? 2 : 3;
-    e = run_fwd(var, pb, io, cws, f, sm);
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+    const bool tc = layer_bwd_tc_form(a) && tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
+    if (tc) {
+        // 2a. the conv results again, as bf16 hi/lo pairs, into the space of the q, k, v gradients
+        //     (written only in step 4); 2b. the tensor-core forward on them, saving the states;
+        //     2c. the states into the CUDA-core layout; 2d. the CUDA-core prep (the factors and T
+        //     the backward reads)
+        const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
+        ConvParams sp = cp;
+        char* gq = reinterpret_cast<char*>(at(plan.gq));
+        char* gk = reinterpret_cast<char*>(at(plan.gk));
+        char* gv = reinterpret_cast<char*>(at(plan.gv));
+        sp.q = gq; sp.q_lo = gq + qn * 2; sp.k = gk; sp.k_lo = gk + qn * 2; sp.v = gv; sp.v_lo = gv + vn * 2;
+        e = bf16_conv(sp, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (split conv)");
+        ChunkIO tio = io;
+        tio.q = sp.q; tio.k = sp.k; tio.v = sp.v; tio.q_lo = sp.q_lo; tio.k_lo = sp.k_lo; tio.v_lo = sp.v_lo;
+        TcFwdSave save{at(plan.s0tc), nullptr, nullptr};
+        e = tc_chunk_fwd(pb, tio, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, &save);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+        e = layer_states_to_rows(at(plan.s0tc), cws.S0, (int)(a->B * a->Hv), pb.NT, (int)a->dk, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (states)");
+        e = var == 2 ? f32_chunk_prep(pb, io, cws, f, sm) : f32_bf16g_chunk_prep(pb, io, cws, f, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (prep)");
+    } else {
+        e = run_fwd(var, pb, io, cws, f, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+    }
     // 3. swish gate
     LayerBwdIO lio{};
     lio.xq = a->xq; lio.xk = a->xk; lio.xv = a->xv; lio.conv_w = a->conv_w; lio.z = a->z; lio.dy = a->grad_y;

@@ -38,6 +38,8 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
                                  cudaStream_t);                                              \
     cudaError_t NAME##_chunk_bwd(const Problem&, const ChunkIO&, const ChunkWs&, Flags, bool, \
                                  cudaStream_t);                                              \
+    cudaError_t NAME##_chunk_prep(const Problem&, const ChunkIO&, const ChunkWs&, Flags,      \
+                                  cudaStream_t);                                             \
     cudaError_t NAME##_decode(const DecodeParams&, Flags, cudaStream_t);                       \
     cudaError_t NAME##_conv(const ConvParams&, cudaStream_t);
 
@@ -83,6 +85,9 @@ struct LayerBwdIO {
 size_t layer_bwd_wpart_floats(int B, int T, int Hk, int Hv, int d);
 cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
 cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
+// Chunk states from the tensor-core forward's saving layout [BH][NT + 1][D/4][D][4] to the CUDA-core
+// kernels' [BH * NT][D][D] (row = key channel; the final state, slot NT, is not copied).
+cudaError_t layer_states_to_rows(const float* src, float* dst, int BH, int NT, int D, cudaStream_t st);
 
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates

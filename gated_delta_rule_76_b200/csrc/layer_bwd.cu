@@ -172,6 +172,22 @@ __global__ void __launch_bounds__(256) dconv_reduce_kernel(const float* __restri
     dw[j] = s;
 }
 
+// One float4 of a state per thread.  A warp covers 8 rows x 4 float4 column groups, so its reads
+// (consecutive rows of one column group) and its writes (consecutive column groups of one row)
+// both touch contiguous runs.
+__global__ void __launch_bounds__(256) states_to_rows_kernel(const float4* __restrict__ src, float4* __restrict__ dst,
+                                                             long nchunk, int NT, int D) {
+    const int q4 = D / 4, cblocks = q4 / 4;
+    const long per = (long)D * q4;
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < nchunk * per; i += (long)gridDim.x * blockDim.x) {
+        const long ci = i / per;
+        const int e = (int)(i - ci * per), lane = e & 31, grp = e >> 5;
+        const int r = (grp / cblocks) * 8 + (lane & 7), j4 = (grp % cblocks) * 4 + (lane >> 3);
+        const long bh = ci / NT, n = ci - bh * NT;
+        dst[ci * per + (long)r * q4 + j4] = src[(bh * (NT + 1) + n) * per + (long)j4 * D + r];
+    }
+}
+
 template <class TIn>
 cudaError_t conv_bwd_t(const LayerBwdIO& io, cudaStream_t st) {
     const int ntile = (io.T + kTile - 1) / kTile;
@@ -215,6 +231,14 @@ cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st) {
 
 cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st) {
     return bf16 ? conv_bwd_t<__nv_bfloat16>(io, st) : conv_bwd_t<float>(io, st);
+}
+
+cudaError_t layer_states_to_rows(const float* src, float* dst, int BH, int NT, int D, cudaStream_t st) {
+    if (D % 16 != 0) return cudaErrorInvalidValue;
+    const long total = (long)BH * NT * D * (D / 4);
+    const long blocks = (total + 255) / 256 < 148L * 16 ? (total + 255) / 256 : 148L * 16;
+    return launch_kernel(states_to_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                         reinterpret_cast<const float4*>(src), reinterpret_cast<float4*>(dst), (long)BH * NT, NT, D);
 }
 
 }  // namespace gdn

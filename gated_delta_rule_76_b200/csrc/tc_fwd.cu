@@ -73,10 +73,13 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     }
     const bool gate = f.gate;
     if (split) {
-        // the layer core's form: scalar gates and the swish output gate
-        if (!gate) return cudaErrorInvalidValue;
-        return bf16_gates ? launch_tc<false, false, true, __nv_bfloat16, true>(maps, p, st)
-                          : launch_tc<false, false, true, float, true>(maps, p, st);
+        // the layer core's form (scalar gates): with the swish output gate (its forward), or
+        // without it (the raw o and the chunk states for its backward)
+        if (gate)
+            return bf16_gates ? launch_tc<false, false, true, __nv_bfloat16, true>(maps, p, st)
+                              : launch_tc<false, false, true, float, true>(maps, p, st);
+        return bf16_gates ? launch_tc<false, false, false, __nv_bfloat16, true>(maps, p, st)
+                          : launch_tc<false, false, false, float, true>(maps, p, st);
     }
     if (f.apc && f.gpc) return launch_tc_g<true, true, __nv_bfloat16>(gate, maps, p, st);
     if (f.apc) return launch_tc_g<true, false, __nv_bfloat16>(gate, maps, p, st);

@@ -159,7 +159,8 @@ def test_decode_negative_eigenvalue_gates():
 
 @pytest.mark.parametrize("B,T,Hk,Hv,d,gpc,gdt,dt", [
     (2, 150, 2, 4, 64, False, "f32", "bf16"),    # GQA, scalar gates, ragged tail
-    (1, 130, 1, 2, 128, False, "bf16", "bf16"),  # d = 128, bf16 gates
+    (1, 130, 1, 2, 128, False, "bf16", "bf16"),  # d = 128, bf16 gates (tensor-core forward inside)
+    (2, 200, 2, 4, 128, False, "f32", "bf16"),   # d = 128, GQA, fp32 gates, ragged tail (same)
     (1, 100, 1, 2, 64, True, "bf16", "bf16"),    # channel gates
     (1, 70, 1, 1, 64, False, "f32", "f32"),      # fp32 tensors
 ])
