@@ -497,7 +497,8 @@ def bench_part_fwd(name, args, dist, peaks, peak_kind, stream, device):
 
 def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
     """The GQA layer core's training step: gdn_layer_core_fwd then gdn_layer_core_bwd (the
-    recurrence's backward on the CUDA-core kernels), inputs resident, gradients of every input."""
+    recurrence's backward on the tensor cores, once per bf16 half of do), inputs resident,
+    gradients of every input."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     from gated_delta_rule_76_b200.inputs import WORKLOADS
@@ -522,7 +523,8 @@ def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
             "roofline": roofline(by, fl, ms * 1e-3, peaks, peak_kind,
                                  "gdn_layer_core_fwd + gdn_layer_core_bwd calls"),
             "config": {"B": wl.B, "T": wl.T, "Hk": wl.Hk, "Hv": wl.Hv, "dk": wl.dk, "dv": wl.dv,
-                       "backward": "recurrence on the CUDA-core chunk kernels (fp32 conv results)"}}
+                       "backward": "recurrence on the tensor-core backward kernels, once per bf16 half of do "
+                                   "(conv results as bf16 hi/lo pairs)"}}
 
 
 # --------------------------------------------------------------------------------------------

@@ -521,33 +521,54 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
 }
 
-// Workspace of the layer backward: the recomputed conv results (fp32), the recurrence's output o
-// and its gradient, the gradients of q, k, v from the recurrence, the conv-weight partials, the
-// tensor-core forward's chunk states (bf16 tensors with d = 128 and scalar gates), then the
-// CUDA-core chunk backward's own workspace.  Offsets from the start, 256-byte aligned.
+// Workspace of the layer backward, offsets from its start, 256-byte aligned.
+// Tensor-core form (bf16 tensors, d = 128, scalar gates, no initial state): the tensor-core
+// backward's own workspace
+// first (its status word is the call's, at offset 0), then the conv results as bf16 hi/lo pairs,
+// the recurrence's output o, the gradient of o (bf16 hi/lo), the q, k, v gradients from the
+// recurrence, the conv-weight partials, the forward cache (states, V'), and the second set of
+// recurrence gradients (those of the lo half of the gradient of o).
+// CUDA-core form (everything else): the status word, the fp32 conv results, o, the gradient of o
+// (fp32), the q, k, v gradients, the conv-weight partials, then the CUDA-core chunk workspace.
 struct LayerBwdPlan {
-    size_t q, k, v, o, dout, gq, gk, gv, wpart, s0tc, chunk, bytes;
+    bool tc;
+    size_t q, k, v, o, dout, gq, gk, gv, wpart, cache, chunk, bytes;
+    size_t gq2, gk2, gv2, ga2, gb2, gh2;  // tensor-core form: gradients from the lo half of do
 };
-// The layer backward's forward (o and the chunk states) runs on the tensor cores, from the conv
-// results as bf16 hi/lo pairs, when the layer forward would.
+// With an initial state h0 the first tokens' dxk is tens of times its RMS (the conv sees one tap
+// there, and the L2 norm's backward divides by a small norm): the tensor-core backward's ~1e-3
+// relative error there exceeds the 2e-2-of-RMS budget, so such calls keep the fp32 CUDA-core form.
 static bool layer_bwd_tc_form(const gdn_layer_bwd_args* a) {
-    return a->dtype == GDN_BF16 && a->dk == 128 && a->dv == 128 && !a->alpha_per_channel && !a->gates_per_channel;
+    return a->dtype == GDN_BF16 && a->dk == 128 && a->dv == 128 && !a->alpha_per_channel && !a->gates_per_channel &&
+           a->h0 == nullptr;
 }
 static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& pb) {
     LayerBwdPlan w{};
+    w.tc = layer_bwd_tc_form(a);
     const size_t BT = (size_t)(a->B * a->T), qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
-    size_t off = 256;
-    auto take = [&](size_t floats) {
+    size_t off = w.tc ? align256(plan_tc_bwd_ws(pb, !identity_heads(pb), true).bytes) : 256;
+    auto take = [&](size_t bytes) {
         const size_t o = off;
-        off = align256(off + floats * sizeof(float));
+        off = align256(off + bytes);
         return o;
     };
-    w.q = take(qn); w.k = take(qn); w.v = take(vn); w.o = take(vn); w.dout = take(vn);
-    w.gq = take(qn); w.gk = take(qn); w.gv = take(vn);
-    w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk));
-    w.s0tc = layer_bwd_tc_form(a) ? take((size_t)a->B * a->Hv * (pb.NT + 1) * a->dk * a->dv) : ~size_t(0);
-    w.chunk = off;
-    w.bytes = off + plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
+    w.chunk = w.tc ? 0 : ~size_t(0);
+    w.q = take(qn * 4); w.k = take(qn * 4); w.v = take(vn * 4); w.o = take(vn * 4);
+    w.dout = take(vn * 4);  // fp32, or bf16 hi then lo
+    w.gq = take(qn * 4); w.gk = take(qn * 4); w.gv = take(vn * 4);
+    w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk) * 4);
+    if (w.tc) {
+        w.cache = take(plan_tc_cache(pb).bytes);
+        const size_t ng = BT * a->Hv;  // scalar gates
+        w.gq2 = take(qn * 4); w.gk2 = take(qn * 4); w.gv2 = take(vn * 4);
+        w.ga2 = take(ng * 4); w.gb2 = take(ng * 4);
+        w.gh2 = take((size_t)a->B * a->Hv * a->dk * a->dv * 4);
+    } else {
+        w.cache = ~size_t(0);
+        w.chunk = off;
+        off += plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
+    }
+    w.bytes = off;
     return w;
 }
 
@@ -603,69 +624,96 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     auto at = [&](size_t o) { return reinterpret_cast<float*>(wsb + o); };
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd");
-    // 1. conv + SiLU + L2, fp32 results
+    const bool bf16 = a->dtype == GDN_BF16, bf16g = a->gate_dtype == GDN_BF16;
+    const bool direct = identity_heads(pb);
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
     ConvParams cp{};
     cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
-    cp.q = at(plan.q); cp.k = at(plan.k); cp.v = at(plan.v);
     cp.B = (int)a->B; cp.T = (int)a->T; cp.Hk = (int)a->Hk; cp.Hv = (int)a->Hv; cp.d = (int)a->dk;
-    const bool bf16 = a->dtype == GDN_BF16;
-    e = bf16 ? bf16_conv(cp, sm) : f32_conv(cp, sm);
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
-    // 2. the recurrence's output o (fp32, no gate) and the chunk states for step 4 (paired: the
-    //    backward does not run the forward again)
-    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
-    f.paired = true;
-    const WsPlan cplan = plan_chunk_ws(pb, true, !identity_heads(pb));
-    const ChunkWs cws = carve_chunk_ws(cplan, wsb + plan.chunk);
-    ChunkIO io{};
-    io.q = cp.q; io.k = cp.k; io.v = cp.v; io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.h0 = a->h0;
-    io.o = at(plan.o); io.o_type = 1;
-    const int var = a->gate_dtype == GDN_F32 ? 2 : 3;
-    const bool tc = layer_bwd_tc_form(a) && tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
-    if (tc) {
-        // 2a. the conv results again, as bf16 hi/lo pairs, into the space of the q, k, v gradients
-        //     (written only in step 4); 2b. the tensor-core forward on them, saving the states;
-        //     2c. the states into the CUDA-core layout; 2d. the CUDA-core prep (the factors and T
-        //     the backward reads)
-        const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
-        ConvParams sp = cp;
-        char* gq = reinterpret_cast<char*>(at(plan.gq));
-        char* gk = reinterpret_cast<char*>(at(plan.gk));
-        char* gv = reinterpret_cast<char*>(at(plan.gv));
-        sp.q = gq; sp.q_lo = gq + qn * 2; sp.k = gk; sp.k_lo = gk + qn * 2; sp.v = gv; sp.v_lo = gv + vn * 2;
-        e = bf16_conv(sp, sm);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (split conv)");
-        ChunkIO tio = io;
-        tio.q = sp.q; tio.k = sp.k; tio.v = sp.v; tio.q_lo = sp.q_lo; tio.k_lo = sp.k_lo; tio.v_lo = sp.v_lo;
-        TcFwdSave save{at(plan.s0tc), nullptr, nullptr};
-        e = tc_chunk_fwd(pb, tio, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, &save);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
-        e = layer_states_to_rows(at(plan.s0tc), cws.S0, (int)(a->B * a->Hv), pb.NT, (int)a->dk, sm);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (states)");
-        e = var == 2 ? f32_chunk_prep(pb, io, cws, f, sm) : f32_bf16g_chunk_prep(pb, io, cws, f, sm);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (prep)");
-    } else {
-        e = run_fwd(var, pb, io, cws, f, sm);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
-    }
-    // 3. swish gate
     LayerBwdIO lio{};
     lio.xq = a->xq; lio.xk = a->xk; lio.xv = a->xv; lio.conv_w = a->conv_w; lio.z = a->z; lio.dy = a->grad_y;
     lio.o = at(plan.o); lio.gq = at(plan.gq); lio.gk = at(plan.gk); lio.gv = at(plan.gv);
-    lio.dout = at(plan.dout); lio.dz = a->grad_z;
+    lio.dz = a->grad_z;
     lio.dxq = a->grad_xq; lio.dxk = a->grad_xk; lio.dxv = a->grad_xv;
     lio.wpart = at(plan.wpart); lio.dconv_w = a->grad_conv_w;
     lio.B = (int)a->B; lio.T = (int)a->T; lio.Hk = (int)a->Hk; lio.Hv = (int)a->Hv; lio.d = (int)a->dk;
-    e = layer_gate_bwd(lio, bf16, sm);
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (gate)");
-    // 4. the recurrence's backward on the fp32 conv results
-    io.o = nullptr;
-    io.dout = at(plan.dout); io.dht = a->grad_ht;
-    io.dq = at(plan.gq); io.dk = at(plan.gk); io.dv = at(plan.gv);
-    io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = a->grad_w; io.dh0 = a->grad_h0;
-    e = var == 2 ? f32_chunk_bwd(pb, io, cws, f, identity_heads(pb), sm)
-                 : f32_bf16g_chunk_bwd(pb, io, cws, f, identity_heads(pb), sm);
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence)");
+    ChunkIO io{};
+    io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.h0 = a->h0;
+    if (plan.tc) {
+        if (!tc_fwd_eligible(pb, true, bf16g, f))
+            return fail(GDN_ERR_UNSUPPORTED, "the tensor-map encoder of the CUDA driver is unavailable");
+        // 1. conv + SiLU + L2, fp32 results stored as bf16 hi/lo pairs
+        const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
+        char* q = wsb + plan.q;
+        char* k = wsb + plan.k;
+        char* v = wsb + plan.v;
+        cp.q = q; cp.q_lo = q + qn * 2; cp.k = k; cp.k_lo = k + qn * 2; cp.v = v; cp.v_lo = v + vn * 2;
+        e = bf16_conv(cp, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
+        // 2. the tensor-core forward in saving mode: o (fp32, no gate), the chunk states and V'
+        io.q = cp.q; io.k = cp.k; io.v = cp.v; io.q_lo = cp.q_lo; io.k_lo = cp.k_lo; io.v_lo = cp.v_lo;
+        io.o = at(plan.o); io.o_type = 1;
+        const TcCache cc = plan_tc_cache(pb);
+        char* cb = wsb + plan.cache;
+        const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
+                             reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo)};
+        e = tc_chunk_fwd(pb, io, f, bf16g, ws_status(workspace), sm, &save);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+        // 3. swish gate; the gradient of o as bf16 hi/lo pairs (tensor-core operands)
+        lio.dout16 = reinterpret_cast<__nv_bfloat16*>(wsb + plan.dout);
+        lio.dout16_lo = lio.dout16 + vn;
+        e = layer_gate_bwd(lio, bf16, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (gate)");
+        // 4. the tensor-core backward from the cache, once per half of do.  The backward is linear
+        //    in its cotangents (do, dht), so the gradients of (hi, dht) and of (lo, 0) add up to
+        //    those of (do, dht); a single bf16 do would move dq by ~5% of its RMS on this layer.
+        const TcBwdWs tplan = plan_tc_bwd_ws(pb, !direct, true);
+        io.o = nullptr;
+        io.dout = lio.dout16; io.dht = a->grad_ht;
+        io.dq = at(plan.gq); io.dk = at(plan.gk); io.dv = at(plan.gv);
+        io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = nullptr; io.dh0 = a->grad_h0;
+        e = tc_chunk_bwd(pb, io, f, bf16g, direct, tplan, workspace, cb, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence)");
+        io.dout = lio.dout16_lo; io.dht = nullptr;
+        io.dq = at(plan.gq2); io.dk = at(plan.gk2); io.dv = at(plan.gv2);
+        io.dalpha = at(plan.ga2); io.db = at(plan.gb2); io.dh0 = a->grad_h0 ? at(plan.gh2) : nullptr;
+        e = tc_chunk_bwd(pb, io, f, bf16g, direct, tplan, workspace, cb, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence, lo half)");
+        const long ng = (long)BT * a->Hv;
+        const struct { float* dst; const float* src; long n; } acc[] = {
+            {at(plan.gq), at(plan.gq2), (long)qn}, {at(plan.gk), at(plan.gk2), (long)qn},
+            {at(plan.gv), at(plan.gv2), (long)vn}, {a->grad_alpha, at(plan.ga2), ng}, {a->grad_b, at(plan.gb2), ng},
+            {a->grad_h0, at(plan.gh2), a->grad_h0 ? (long)(st / 4) : 0}};
+        for (const auto& x : acc) {
+            e = layer_accumulate(x.dst, x.src, x.n, sm);
+            if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (accumulate)");
+        }
+    } else {
+        // 1. conv + SiLU + L2, fp32 results
+        cp.q = at(plan.q); cp.k = at(plan.k); cp.v = at(plan.v);
+        e = bf16 ? bf16_conv(cp, sm) : f32_conv(cp, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
+        // 2. o (fp32, no gate) on the CUDA-core forward, which also keeps the chunk states for step 4
+        //    (paired: the backward does not run the forward again)
+        f.paired = true;
+        const ChunkWs cws = carve_chunk_ws(plan_chunk_ws(pb, true, !direct), wsb + plan.chunk);
+        io.q = cp.q; io.k = cp.k; io.v = cp.v;
+        io.o = at(plan.o); io.o_type = 1;
+        const int var = a->gate_dtype == GDN_F32 ? 2 : 3;
+        e = run_fwd(var, pb, io, cws, f, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+        // 3. swish gate
+        lio.dout = at(plan.dout);
+        e = layer_gate_bwd(lio, bf16, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (gate)");
+        // 4. the recurrence's backward on the fp32 conv results
+        io.o = nullptr;
+        io.dout = at(plan.dout); io.dht = a->grad_ht;
+        io.dq = at(plan.gq); io.dk = at(plan.gk); io.dv = at(plan.gv);
+        io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = a->grad_w; io.dh0 = a->grad_h0;
+        e = var == 2 ? f32_chunk_bwd(pb, io, cws, f, direct, sm) : f32_bf16g_chunk_bwd(pb, io, cws, f, direct, sm);
+        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence)");
+    }
     // 5. L2 norm, SiLU and conv backward, conv-weight gradient
     e = layer_conv_bwd(lio, bf16, sm);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_bwd (conv)");

@@ -87,17 +87,6 @@ cudaError_t chunk_fwd_impl(const Problem& pb, const ChunkIO& io, const ChunkWs& 
     });
 }
 
-// prep alone, saving what the backward reads (the chunk states come from another forward)
-template <class TIn, class TG>
-cudaError_t chunk_prep_impl(const Problem& pb, const ChunkIO& io, const ChunkWs& ws, Flags f, cudaStream_t st) {
-    return dispatch_chunk<TIn, TG>(pb, f, [&](auto apc, auto gpc, auto dk) {
-        constexpr bool APC = decltype(apc)::value, GPC = decltype(gpc)::value;
-        constexpr int DK = decltype(dk)::value;
-        return launch_kernel(chunk_prep_kernel<TIn, TG, APC, GPC, DK>, dim3(pb.NT, pb.Hv, pb.B), dim3(kSimtThreads),
-                             chunk_prep_smem<DK>(), st, pb, io, ws, 1);
-    });
-}
-
 template <class TIn, class TG>
 cudaError_t chunk_bwd_impl(const Problem& pb, const ChunkIO& io, const ChunkWs& ws, Flags f,
                            bool direct_qk, cudaStream_t st) {
@@ -152,10 +141,6 @@ cudaError_t conv_impl(const ConvParams& p, cudaStream_t st) {
     cudaError_t NAME##_chunk_bwd(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,         \
                                  Flags f, bool direct_qk, cudaStream_t st) {                     \
         return chunk_bwd_impl<TIN, TG>(pb, io, ws, f, direct_qk, st);                            \
-    }                                                                                            \
-    cudaError_t NAME##_chunk_prep(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,        \
-                                  Flags f, cudaStream_t st) {                                    \
-        return chunk_prep_impl<TIN, TG>(pb, io, ws, f, st);                                      \
     }                                                                                            \
     cudaError_t NAME##_decode(const DecodeParams& p, Flags f, cudaStream_t st) {                 \
         GDN_TRY((decode_impl<TIN, TG>(p, f, st)));                                               \

@@ -38,15 +38,13 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
                                  cudaStream_t);                                              \
     cudaError_t NAME##_chunk_bwd(const Problem&, const ChunkIO&, const ChunkWs&, Flags, bool, \
                                  cudaStream_t);                                              \
-    cudaError_t NAME##_chunk_prep(const Problem&, const ChunkIO&, const ChunkWs&, Flags,      \
-                                  cudaStream_t);                                             \
     cudaError_t NAME##_decode(const DecodeParams&, Flags, cudaStream_t);                       \
     cudaError_t NAME##_conv(const ConvParams&, cudaStream_t);
 
 // Tensor-core chunk forward (tc_fwd.cu): bf16 q/k/v with dk = dv = 128.  With `save`, the state
 // entering every chunk and V' of every token are written for the backward (o and ht may be NULL).
 struct TcFwdSave {
-    float* s0;               // [B*Hv][NT][dk][dv]
+    float* s0;               // [B*Hv][NT + 1][dv/4][dk][4]
     __nv_bfloat16* vp_hi;    // [B,T,Hv,dv]
     __nv_bfloat16* vp_lo;
 };
@@ -78,6 +76,7 @@ struct LayerBwdIO {
     const float* o;                     // [B,T,Hv,d] the recurrence's output, before the gate
     const float *gq, *gk, *gv;          // gradients of the L2-normalised q, k and of v
     float *dout, *dz;                   // out: gradient of o (fp32), of z
+    __nv_bfloat16 *dout16, *dout16_lo;  // out instead of dout when set: the gradient of o as bf16 hi/lo
     float *dxq, *dxk, *dxv;             // out: gradients of the conv inputs
     float *wpart, *dconv_w;             // per-tile partial sums of the conv-weight gradient; out
     int B, T, Hk, Hv, d;
@@ -85,9 +84,8 @@ struct LayerBwdIO {
 size_t layer_bwd_wpart_floats(int B, int T, int Hk, int Hv, int d);
 cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
 cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
-// Chunk states from the tensor-core forward's saving layout [BH][NT + 1][D/4][D][4] to the CUDA-core
-// kernels' [BH * NT][D][D] (row = key channel; the final state, slot NT, is not copied).
-cudaError_t layer_states_to_rows(const float* src, float* dst, int BH, int NT, int D, cudaStream_t st);
+// dst[i] += src[i], i < n (the two halves of a gradient computed from hi and lo cotangents).
+cudaError_t layer_accumulate(float* dst, const float* src, long n, cudaStream_t st);
 
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates

@@ -16,14 +16,18 @@ namespace {
 __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 // y = o * z * sigmoid(z):  do = dy * z * sigmoid(z),  dz = dy * o * (s + z s (1 - s)).
-template <class T>
+// With dout_lo (bf16 outputs only), do is stored as hi = bf16(do) and lo = bf16(do - hi).
+template <class T, class TO>
 __global__ void __launch_bounds__(256) swish_gate_bwd_kernel(const float* __restrict__ o, const T* __restrict__ z,
-                                                             const T* __restrict__ dy, float* __restrict__ dout,
-                                                             float* __restrict__ dz, long n) {
+                                                             const T* __restrict__ dy, TO* __restrict__ dout,
+                                                             TO* __restrict__ dout_lo, float* __restrict__ dz, long n) {
     for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
         const float zz = to_f32(z[i]), g = to_f32(dy[i]);
         const float s = sigmoid_fast(zz);
-        dout[i] = g * zz * s;
+        const float d = g * zz * s;
+        const TO hi = from_f32<TO>(d);
+        dout[i] = hi;
+        if (dout_lo) dout_lo[i] = from_f32<TO>(d - to_f32(hi));
         dz[i] = g * o[i] * (s + zz * s * (1.f - s));
     }
 }
@@ -162,6 +166,20 @@ __global__ void __launch_bounds__(128) conv_silu_l2_bwd_kernel(const TIn* __rest
     }
 }
 
+__global__ void __launch_bounds__(256) accumulate_kernel(float4* __restrict__ dst, const float4* __restrict__ src,
+                                                         float* __restrict__ dst1, const float* __restrict__ src1,
+                                                         long n4, long n) {
+    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+        float4 a = dst[i];
+        const float4 b = src[i];
+        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        dst[i] = a;
+    }
+    // what the float4 body leaves (n % 4 elements, or all of them when the pointers are unaligned)
+    for (long t = 4 * n4 + (long)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += (long)gridDim.x * blockDim.x)
+        dst1[t] += src1[t];
+}
+
 // dconv_w[j] = sum over partials p of wpart[p][j]  (j = channel * 4 + tap), one thread per j.
 __global__ void __launch_bounds__(256) dconv_reduce_kernel(const float* __restrict__ wpart, float* __restrict__ dw,
                                                            long nj, int np) {
@@ -170,22 +188,6 @@ __global__ void __launch_bounds__(256) dconv_reduce_kernel(const float* __restri
     float s = 0.f;
     for (int p = 0; p < np; ++p) s += wpart[(long)p * nj + j];
     dw[j] = s;
-}
-
-// One float4 of a state per thread.  A warp covers 8 rows x 4 float4 column groups, so its reads
-// (consecutive rows of one column group) and its writes (consecutive column groups of one row)
-// both touch contiguous runs.
-__global__ void __launch_bounds__(256) states_to_rows_kernel(const float4* __restrict__ src, float4* __restrict__ dst,
-                                                             long nchunk, int NT, int D) {
-    const int q4 = D / 4, cblocks = q4 / 4;
-    const long per = (long)D * q4;
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < nchunk * per; i += (long)gridDim.x * blockDim.x) {
-        const long ci = i / per;
-        const int e = (int)(i - ci * per), lane = e & 31, grp = e >> 5;
-        const int r = (grp / cblocks) * 8 + (lane & 7), j4 = (grp % cblocks) * 4 + (lane >> 3);
-        const long bh = ci / NT, n = ci - bh * NT;
-        dst[ci * per + (long)r * q4 + j4] = src[(bh * (NT + 1) + n) * per + (long)j4 * D + r];
-    }
 }
 
 template <class TIn>
@@ -215,8 +217,12 @@ template <class T>
 cudaError_t gate_bwd_t(const LayerBwdIO& io, cudaStream_t st) {
     const long n = (long)io.B * io.T * io.Hv * io.d;
     const long blocks = (n + 255) / 256 < 148L * 32 ? (n + 255) / 256 : 148L * 32;
-    return launch_kernel(swish_gate_bwd_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, st, (const float*)io.o,
-                         static_cast<const T*>(io.z), static_cast<const T*>(io.dy), io.dout, io.dz, n);
+    if (io.dout16)
+        return launch_kernel(swish_gate_bwd_kernel<T, __nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, st,
+                             (const float*)io.o, static_cast<const T*>(io.z), static_cast<const T*>(io.dy), io.dout16,
+                             io.dout16_lo, io.dz, n);
+    return launch_kernel(swish_gate_bwd_kernel<T, float>, dim3((unsigned)blocks), dim3(256), 0, st, (const float*)io.o,
+                         static_cast<const T*>(io.z), static_cast<const T*>(io.dy), io.dout, (float*)nullptr, io.dz, n);
 }
 
 }  // namespace
@@ -233,12 +239,15 @@ cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st) {
     return bf16 ? conv_bwd_t<__nv_bfloat16>(io, st) : conv_bwd_t<float>(io, st);
 }
 
-cudaError_t layer_states_to_rows(const float* src, float* dst, int BH, int NT, int D, cudaStream_t st) {
-    if (D % 16 != 0) return cudaErrorInvalidValue;
-    const long total = (long)BH * NT * D * (D / 4);
-    const long blocks = (total + 255) / 256 < 148L * 16 ? (total + 255) / 256 : 148L * 16;
-    return launch_kernel(states_to_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
-                         reinterpret_cast<const float4*>(src), reinterpret_cast<float4*>(dst), (long)BH * NT, NT, D);
+cudaError_t layer_accumulate(float* dst, const float* src, long n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    // float4 body only when both pointers are 16-byte aligned
+    const bool v4 = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15u) == 0;
+    const long n4 = v4 ? n / 4 : 0;
+    const long work = n4 > n - 4 * n4 ? n4 : n - 4 * n4;
+    const long blocks = (work + 255) / 256 < 148L * 16 ? (work + 255) / 256 : 148L * 16;
+    return launch_kernel(accumulate_kernel, dim3((unsigned)(blocks > 0 ? blocks : 1)), dim3(256), 0, st,
+                         reinterpret_cast<float4*>(dst), reinterpret_cast<const float4*>(src), dst, src, n4, n);
 }
 
 }  // namespace gdn

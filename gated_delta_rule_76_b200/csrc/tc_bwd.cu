@@ -13,9 +13,9 @@ namespace {
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT>
 cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cudaStream_t st) {
-    auto kernel = tcbwd::scan::chunk_bwd_scan_kernel<APC, GPC, TG>;
+    auto kernel = tcbwd::scan::chunk_bwd_scan_kernel<APC, GPC, TG, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcbwd::scan::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -25,9 +25,9 @@ cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cuda
     return cudaGetLastError();
 }
 
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT>
 cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cudaStream_t st) {
-    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG>;
+    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcbwd::grad::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -41,12 +41,12 @@ cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cuda
     return cudaGetLastError();
 }
 
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT = false>
 cudaError_t launch_both(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
                         const tcbwd::grad::Params& gp, cudaStream_t st) {
-    cudaError_t e = launch_scan<APC, GPC, TG>(ms, sp, st);
+    cudaError_t e = launch_scan<APC, GPC, TG, SPLIT>(ms, sp, st);
     if (e != cudaSuccess) return e;
-    return launch_grad<APC, GPC, TG>(mg, gp, st);
+    return launch_grad<APC, GPC, TG, SPLIT>(mg, gp, st);
 }
 
 }  // namespace
@@ -105,6 +105,8 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     float* dq_v = direct ? static_cast<float*>(io.dq) : reinterpret_cast<float*>(base + plan.dq_v);
     float* dk_v = direct ? static_cast<float*>(io.dk) : reinterpret_cast<float*>(base + plan.dk_v);
 
+    const bool split = io.q_lo != nullptr;
+    if (split && (f.apc || f.gpc || !io.k_lo || !io.v_lo)) return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (!cache) {
         // 1. forward in saving mode (no output, no final state)
@@ -129,6 +131,8 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     m[3] = m[4];
     if (ok && f.apc) ok = make_map(&m[2], io.alpha, pb.B, pb.T, pb.Hv);
     if (ok && f.gpc) ok = make_map(&m[3], io.b, pb.B, pb.T, pb.Hv);
+    // split inputs: the lo halves of k and q take the alpha and b slots
+    if (ok && split) ok = make_map(&m[2], io.k_lo, pb.B, pb.T, pb.Hk) && make_map(&m[3], io.q_lo, pb.B, pb.T, pb.Hk);
     if (!ok) return cudaErrorInvalidValue;
     const CUtensorMap ms[5] = {m[0], m[1], m[2], m[3], m[4]};
 
@@ -151,6 +155,9 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     gp.q = static_cast<const __nv_bfloat16*>(io.q);
     gp.k = static_cast<const __nv_bfloat16*>(io.k);
     gp.v = static_cast<const __nv_bfloat16*>(io.v);
+    gp.q_lo = static_cast<const __nv_bfloat16*>(io.q_lo);
+    gp.k_lo = static_cast<const __nv_bfloat16*>(io.k_lo);
+    gp.v_lo = static_cast<const __nv_bfloat16*>(io.v_lo);
     gp.s0 = s0;
     gp.dsc = dsc;
     gp.dq = dq_v;
@@ -162,7 +169,9 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     gp.direct = direct ? 1 : 0;
     gp.err = err;
 
-    if (f.apc && f.gpc) e = launch_both<true, true, __nv_bfloat16>(ms, sp, m, gp, st);
+    if (split) e = bf16_gates ? launch_both<false, false, __nv_bfloat16, true>(ms, sp, m, gp, st)
+                              : launch_both<false, false, float, true>(ms, sp, m, gp, st);
+    else if (f.apc && f.gpc) e = launch_both<true, true, __nv_bfloat16>(ms, sp, m, gp, st);
     else if (f.apc) e = launch_both<true, false, __nv_bfloat16>(ms, sp, m, gp, st);
     else if (f.gpc) e = launch_both<false, true, __nv_bfloat16>(ms, sp, m, gp, st);
     else if (bf16_gates) e = launch_both<false, false, __nv_bfloat16>(ms, sp, m, gp, st);

@@ -139,13 +139,21 @@ struct Params {
 };
 
 
-template <bool APC, bool GPC>
+// SPLIT (scalar gates only): q and k arrive as bf16 hi/lo pairs; ta maps k lo (into the alpha
+// slot) and tb_ maps q lo (into the b rows), both indexed by the key head.
+template <bool APC, bool GPC, bool SPLIT>
 __device__ __forceinline__ void scan_load_raw(const Ctx& cx, int n, int b, int hk, int hv, const CUtensorMap* tq,
                                          const CUtensorMap* tk, const CUtensorMap* ta, const CUtensorMap* tb_) {
     const int t0 = n * C;
     const uint32_t base = smem_u32(cx.sm);
     uint64_t* bar = cx.bars + B_RAW;
-    mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
+    mbar_arrive_expect_tx(bar, 32768u + (GPC || SPLIT ? 16384u : 0u) + (APC || SPLIT ? 16384u : 0u));
+    if (SPLIT) {
+        tma4(base + SM_RQB, tb_, bar, 0, hk, t0, b);  // q lo -> rows 0-63
+        tma4(base + SM_RQB + 16384, tb_, bar, 64, hk, t0, b);
+        tma4(base + SM_RA, ta, bar, 0, hk, t0, b);    // k lo
+        tma4(base + SM_RA + 8192, ta, bar, 64, hk, t0, b);
+    }
     tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);  // q -> rows 64-127
     tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);
     tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
@@ -168,7 +176,7 @@ __device__ __forceinline__ void scan_load_do(const Ctx& cx, int n, int b, int hv
     tma4(dst + 8192, tdo, bar, 64, hv, n * C, b);
 }
 
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -206,7 +214,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // Chunks are processed in reverse: iteration i works on chunk NT - 1 - i.
     int raw_issued = 0, do_issued = 0;  // meaningful in thread 0, which issues every load
     if (tid == 0) {
-        scan_load_raw<APC, GPC>(cx, NT - 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+        scan_load_raw<APC, GPC, SPLIT>(cx, NT - 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
         raw_issued = 1;
         scan_load_do(cx, NT - 1, b, hv, &tm_do);
         do_issued = 1;
@@ -304,7 +312,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     wait1(cx, B_WT, pi);
                     // X1, XC's dO^T Qhat and W^T were the last readers of the raw stage.
                     if (raw_issued < NT && wait1(cx, B_XCPRE, pi) && !*cx.abort_flag) {
-                        scan_load_raw<APC, GPC>(cx, NT - 1 - raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
+                        scan_load_raw<APC, GPC, SPLIT>(cx, NT - 1 - raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
                         ++raw_issued;
                     }
                 }
@@ -525,6 +533,16 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     unpack8(ld16(RK + o64), k8);
                     unpack8(ld16(RQB + oq), q8);
+                    if (SPLIT) {  // + the lo halves (read before this thread overwrites them below)
+                        float kl[8], ql[8];
+                        unpack8(ld16(RA + o64), kl);
+                        unpack8(ld16(RQB + oe), ql);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            k8[e] += kl[e];
+                            q8[e] += ql[e];
+                        }
+                    }
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
                     } else {
@@ -758,6 +776,9 @@ struct Params {
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
+    const __nv_bfloat16* q_lo;  // SPLIT: lo halves of q, k, v (hi in q, k, v)
+    const __nv_bfloat16* k_lo;
+    const __nv_bfloat16* v_lo;
     const float* s0;     // [B*Hv][NT][dv/4][dk][4]: row c, columns 4q..4q+3 at float4 (q * dk + c)
     const float* dsc;    // same layout
     float* dq;           // [B,T,Hk,dk] (direct) or [B,T,Hv,dk] per value head
@@ -792,11 +813,18 @@ struct Maps {
     const CUtensorMap *q, *k, *a, *b, *dO, *yh, *yl, *vh, *vl;
 };
 
-template <bool APC, bool GPC>
+// SPLIT: as in the scan, m.a maps k lo and m.b maps q lo.
+template <bool APC, bool GPC, bool SPLIT>
 __device__ __forceinline__ void load_raw_g(const Ctx& cx, const ChunkPos& cp, const Maps& m) {
     const uint32_t base = smem_u32(cx.sm);
     uint64_t* bar = cx.bars + B_RAW;
-    mbar_arrive_expect_tx(bar, 32768u + (GPC ? 16384u : 0u) + (APC ? 16384u : 0u));
+    mbar_arrive_expect_tx(bar, 32768u + (GPC || SPLIT ? 16384u : 0u) + (APC || SPLIT ? 16384u : 0u));
+    if (SPLIT) {
+        tma4(base + SM_RQB, m.b, bar, 0, cp.hk, cp.t0, cp.b);  // q lo -> rows 0-63
+        tma4(base + SM_RQB + 16384, m.b, bar, 64, cp.hk, cp.t0, cp.b);
+        tma4(base + SM_RA, m.a, bar, 0, cp.hk, cp.t0, cp.b);    // k lo
+        tma4(base + SM_RA + 8192, m.a, bar, 64, cp.hk, cp.t0, cp.b);
+    }
     tma4(base + SM_RQB + 8192, m.q, bar, 0, cp.hk, cp.t0, cp.b);
     tma4(base + SM_RQB + 16384 + 8192, m.q, bar, 64, cp.hk, cp.t0, cp.b);
     tma4(base + SM_RK, m.k, bar, 0, cp.hk, cp.t0, cp.b);
@@ -837,7 +865,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Staging group (128 threads, c = lane = channel): S0 and dS_end rows of the chunk into tensor
 // memory as split A operands and rowsum(dS_end .* S0) into xslot[c]; then, once the raw TMA tiles
 // have landed, the cumulative decay (gamma into gslot[c]) and the split [Ehat;Qhat], Ktil tiles.
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT>
 __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, const ChunkPos& cp, uint32_t tl, int c,
                                             float* xslot, float* gslot, uint32_t raw_parity, int it = 15) {
     const Problem& pb = p.pb;
@@ -957,6 +985,16 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         }
         unpack8(ld16(RK + o64), k8);
         unpack8(ld16(RQB + oq), q8);
+        if (SPLIT) {  // + the lo halves (read before this thread overwrites them below)
+            float kl[8], ql[8];
+            unpack8(ld16(RA + o64), kl);
+            unpack8(ld16(RQB + oe), ql);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                k8[e] += kl[e];
+                q8[e] += ql[e];
+            }
+        }
         if (GPC) {
             unpack8(ld16(RQB + oe), b8);
         } else {
@@ -990,20 +1028,21 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
 // dv = w .* dY, dw = v .* dY (a scalar beta: sum_j v dY per token into scr[SX_DBV]); run by the
 // staging group after its staging, warp w: tokens w, w + 4, ..., lane l: value channels 4l .. 4l + 3.
 
-template <bool GPC, class TG>
+template <bool GPC, class TG, bool SPLIT>
 __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const ChunkPos& cp, int tt, float* scr) {
     const Problem& pb = p.pb;
     const int w = tt >> 5, l = tt & 31, j = 4 * l;
     const uint8_t* gh = cx.sm + SM_GH;
     const uint8_t* gl = cx.sm + SM_GL;
     // loads are unconditional (a row past the sequence reads its last token); stores are guarded
-    uint2 vr[16], wr[16];
+    uint2 vr[16], wr[16], vl[16];
     float bs[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int r = w + 4 * i;
         const long row = pb.v_row(cp.b, cp.t0 + min(r, cp.L - 1), cp.hv);
         vr[i] = __ldg(reinterpret_cast<const uint2*>(p.v + row + j));
+        if (SPLIT) vl[i] = __ldg(reinterpret_cast<const uint2*>(p.v_lo + row + j));
         if (GPC) wr[i] = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.w) + row + j));
         else bs[i] = gate_or(static_cast<const TG*>(p.b), pb, cp.b, cp.t0, r, cp.L, cp.hv, 0.f);
     }
@@ -1019,6 +1058,10 @@ __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const
         dy[3] = -(__uint_as_float(yh.y & 0xFFFF0000u) + __uint_as_float(yl.y & 0xFFFF0000u));
         v4[0] = __uint_as_float(vr[i].x << 16); v4[1] = __uint_as_float(vr[i].x & 0xFFFF0000u);
         v4[2] = __uint_as_float(vr[i].y << 16); v4[3] = __uint_as_float(vr[i].y & 0xFFFF0000u);
+        if (SPLIT) {
+            v4[0] += __uint_as_float(vl[i].x << 16); v4[1] += __uint_as_float(vl[i].x & 0xFFFF0000u);
+            v4[2] += __uint_as_float(vl[i].y << 16); v4[3] += __uint_as_float(vl[i].y & 0xFFFF0000u);
+        }
         if (GPC) {
             w4[0] = __uint_as_float(wr[i].x << 16); w4[1] = __uint_as_float(wr[i].x & 0xFFFF0000u);
             w4[2] = __uint_as_float(wr[i].y << 16); w4[3] = __uint_as_float(wr[i].y & 0xFFFF0000u);
@@ -1106,15 +1149,19 @@ __device__ __forceinline__ RowPtrs row_ptrs(const Params& p, const ChunkPos& cp,
 // Inputs of tokens r0 .. r0 + RB - 1.  FULL: every row of the chunk is inside the sequence; else rows
 // past the sequence read its last token and are then replaced (a load under a branch would be waited
 // for where the branch ends).
-template <bool APC, bool GPC, bool FULL, class TG>
+template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT>
 __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, const RowPtrs& rp, int r0, RowIn& x) {
     const TG* ag = static_cast<const TG*>(p.alpha);
     const TG* bg = static_cast<const TG*>(p.b);
 #pragma unroll
     for (int i = 0; i < RB; ++i) {
         const int r = r0 + i, rr = FULL ? r : min(r, cp.L - 1);
-        const float q0 = __bfloat162float(__ldg(p.q + rp.qk + rr * rp.qk_s));
-        const float k0 = __bfloat162float(__ldg(p.k + rp.qk + rr * rp.qk_s));
+        float q0 = __bfloat162float(__ldg(p.q + rp.qk + rr * rp.qk_s));
+        float k0 = __bfloat162float(__ldg(p.k + rp.qk + rr * rp.qk_s));
+        if (SPLIT) {
+            q0 += __bfloat162float(__ldg(p.q_lo + rp.qk + rr * rp.qk_s));
+            k0 += __bfloat162float(__ldg(p.k_lo + rp.qk + rr * rp.qk_s));
+        }
         const float b0 = GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s));
         const float a0 = APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s)) : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s));
         const bool in = FULL || r < cp.L;
@@ -1125,7 +1172,7 @@ __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, c
     }
 }
 
-template <bool APC, bool GPC, bool FULL, class TG>
+template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT>
 __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
                                                 float gam, float xtot, float* scr, int it) {
     const float scale = p.pb.scale;
@@ -1168,23 +1215,23 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
     };
     // two input buffers: a block's loads are in flight while the previous block is formed
     RowIn x0, x1;
-    load_rows<APC, GPC, FULL, TG>(p, cp, rp, 7 * RB, x0);
+    load_rows<APC, GPC, FULL, TG, SPLIT>(p, cp, rp, 7 * RB, x0);
 #pragma unroll 1
     for (int blk = C / RB - 1; blk > 0; blk -= 2) {
-        load_rows<APC, GPC, FULL, TG>(p, cp, rp, (blk - 1) * RB, x1);
+        load_rows<APC, GPC, FULL, TG, SPLIT>(p, cp, rp, (blk - 1) * RB, x1);
         do_block(blk, x0);
-        if (blk > 1) load_rows<APC, GPC, FULL, TG>(p, cp, rp, (blk - 2) * RB, x0);
+        if (blk > 1) load_rows<APC, GPC, FULL, TG, SPLIT>(p, cp, rp, (blk - 2) * RB, x0);
         do_block(blk - 1, x1);
         if (c == 0) GDN_BTRACE(it, 10 + (C / RB - 1 - blk) / 2);
     }
 }
 
 // Full chunks (every chunk but a ragged last one) take the variant without per-token guards.
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT>
 __device__ __forceinline__ void grad_epilogue(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
                                               float gam, float xtot, float* scr, int it = 15) {
-    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG>(p, cp, tl, c, warp, gam, xtot, scr, it);
-    else grad_epilogue_t<APC, GPC, false, TG>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    else grad_epilogue_t<APC, GPC, false, TG, SPLIT>(p, cp, tl, c, warp, gam, xtot, scr, it);
 }
 
 // Scalar gates: per-token sums over the channels (the epilogue group's per-warp partials, the
@@ -1221,7 +1268,7 @@ __device__ __forceinline__ void bar_sync_all(uint32_t id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -1267,7 +1314,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (ci < nch) {
         const ChunkPos c0 = chunk_pos(pb, ci);
         if (tid == 0) {
-            load_raw_g<APC, GPC>(cx, c0, m);
+            load_raw_g<APC, GPC, SPLIT>(cx, c0, m);
             raw_issued = 1;
         }
         if (tid == 128) {
@@ -1282,7 +1329,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 st16(gl + (uint32_t)(idx >> 9) * 16384u + (uint32_t)(idx & 511) * 16u, make_uint4(0u, 0u, 0u, 0u));
             }
         } else {
-            stage_chunk<APC, GPC, TG>(p, cx, c0, tl, tid - 128, xslot, gslot, 0u);
+            stage_chunk<APC, GPC, TG, SPLIT>(p, cx, c0, tl, tid - 128, xslot, gslot, 0u);
         }
     }
     for (int it = 0; ci < nch; ++it, ci += gridDim.x) {
@@ -1383,19 +1430,19 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float xs = grad_xs(cx, tl, tid);
             named_bar(1, 128);  // Ktil read: the next chunk's raw tiles may land
             if (tid == 0 && nx < nch && !*cx.abort_flag) {
-                load_raw_g<APC, GPC>(cx, chunk_pos(pb, nx), m);
+                load_raw_g<APC, GPC, SPLIT>(cx, chunk_pos(pb, nx), m);
                 ++raw_issued;
             }
             if (tid == 0) GDN_BTRACE(it, 9);
             if (!*cx.abort_flag)
-                grad_epilogue<APC, GPC, TG>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
+                grad_epilogue<APC, GPC, TG, SPLIT>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
             if (tid == 0) GDN_BTRACE(it, 5);
             if (!APC || !GPC) bar_arrive_all(3);  // per-warp partials of the scalar gates written
         } else {
             if (nx < nch)
-                stage_chunk<APC, GPC, TG>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
+                stage_chunk<APC, GPC, TG, SPLIT>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
             if (tid == 128) GDN_BTRACE(it, 8);
-            grad_dv_dw<GPC, TG>(p, cx, cp, tid - 128, scr);
+            grad_dv_dw<GPC, TG, SPLIT>(p, cx, cp, tid - 128, scr);
             named_bar(2, 128);
             if (tid == 128) GDN_BTRACE(it, 4);
             // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land

@@ -266,8 +266,13 @@ GDN_API gdn_status gdn_layer_core_fwd(const gdn_layer_args* args, void* workspac
  *   conv        u_t = sum_tap w[tap] x_{t-3+tap}:  dx_s = sum_tap w[tap] du_{s+3-tap},
  *               dconv_w[ch][tap] = sum over tokens of du_t x_{t-3+tap}
  * The forward parts it needs (conv results, the recurrence's output o) are recomputed in the
- * workspace.  The recurrence runs on the CUDA-core chunk kernels (fp32 conv results), so the
- * workspace is large: gdn_layer_core_bwd_workspace_size() says how large.  dk must equal dv.
+ * workspace.  With bf16 tensors, d = 128, scalar gates and no h0 the recurrence runs on the
+ * tensor cores: the conv results as bf16 hi/lo pairs, do as bf16 hi/lo pairs, the backward once
+ * per half of do (it is linear in do and dht) with the two sets of gradients added.  Otherwise
+ * (h0 given, channel gates, d = 64, fp32 tensors) it runs on the fp32 CUDA-core chunk kernels,
+ * whose workspace is large.  gdn_layer_core_bwd_workspace_size() says how large; dk must equal
+ * dv.  With h0 the first tokens' dxk reaches tens of times its RMS, where the tensor-core path's
+ * ~1e-3 relative error would exceed the 2e-2-of-RMS budget: hence the fp32 kernels there.
  * ------------------------------------------------------------------------------------------ */
 typedef struct gdn_layer_bwd_args {
     const void* xq;       /* the forward's inputs, as in gdn_layer_args */

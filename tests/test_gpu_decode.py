@@ -157,26 +157,28 @@ def test_decode_negative_eigenvalue_gates():
     assert_parity(state, ref_state, "bf16", "state")
 
 
-@pytest.mark.parametrize("B,T,Hk,Hv,d,gpc,gdt,dt", [
-    (2, 150, 2, 4, 64, False, "f32", "bf16"),    # GQA, scalar gates, ragged tail
-    (1, 130, 1, 2, 128, False, "bf16", "bf16"),  # d = 128, bf16 gates (tensor-core forward inside)
-    (2, 200, 2, 4, 128, False, "f32", "bf16"),   # d = 128, GQA, fp32 gates, ragged tail (same)
-    (1, 100, 1, 2, 64, True, "bf16", "bf16"),    # channel gates
-    (1, 70, 1, 1, 64, False, "f32", "f32"),      # fp32 tensors
+@pytest.mark.parametrize("B,T,Hk,Hv,d,gpc,gdt,dt,h0", [
+    (2, 150, 2, 4, 64, False, "f32", "bf16", True),    # GQA, scalar gates, ragged tail
+    (1, 130, 1, 2, 128, False, "bf16", "bf16", True),  # d = 128 with h0: CUDA-core recurrence backward
+    (2, 200, 2, 4, 128, False, "f32", "bf16", True),   # same, GQA, fp32 gates, ragged tail
+    (1, 130, 1, 2, 128, False, "bf16", "bf16", False),  # d = 128 without h0: tensor-core backward (hi/lo)
+    (2, 200, 2, 4, 128, False, "f32", "bf16", False),   # same, GQA, fp32 gates, ragged tail, dht given
+    (1, 100, 1, 2, 64, True, "bf16", "bf16", True),    # channel gates
+    (1, 70, 1, 1, 64, False, "f32", "f32", True),      # fp32 tensors
 ])
-def test_layer_core_backward_matches_oracle(B, T, Hk, Hv, d, gpc, gdt, dt):
+def test_layer_core_backward_matches_oracle(B, T, Hk, Hv, d, gpc, gdt, dt, h0):
     """gdn_layer_core_bwd against the oracle's reverse mode of the layer (itself pinned by finite
     differences): gradients of the conv inputs, the conv weights, the gates, z and h0."""
     x = draw(B, T, Hk, Hv, d, d, alpha_per_channel=gpc, gates_per_channel=gpc, dtype=dt,
-             gate_dtype=gdt, seed=61, has_h0=True, conv=True, swish_gate=True, with_dout=True, with_dht=True)
+             gate_dtype=gdt, seed=61, has_h0=h0, conv=True, swish_gate=True, with_dout=True, with_dht=True)
     g = to_cuda(x)
     gk = dict(beta=g["beta"]) if not gpc else dict(b=g["b"], w=g["w"])
     xk = dict(beta=x["beta"]) if not gpc else dict(b=x["b"], w=x["w"])
-    got = gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"], h0=g["h0"],
-                                 grad_ht=g["dht"], scale=0.8, **gk)
+    got = gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"],
+                                 h0=g.get("h0"), grad_ht=g["dht"], scale=0.8, **gk)
     torch.cuda.synchronize()
-    ref = oracle.layer_core_bwd(x["q"], x["k"], x["v"], x["conv_w"], x["alpha"], x["z"], x["dout"], h0=x["h0"],
-                                dht=x["dht"], scale=0.8, **xk)
+    ref = oracle.layer_core_bwd(x["q"], x["k"], x["v"], x["conv_w"], x["alpha"], x["z"], x["dout"],
+                                h0=x.get("h0"), dht=x["dht"], scale=0.8, **xk)
     kind = "f32" if dt == "f32" else "bf16"
     for key in ["dxq", "dxk", "dxv", "dconv_w", "dalpha", "dz", "dh0"] + (["db", "dw"] if gpc else ["dbeta"]):
         assert_parity(got[key], ref[key], kind, key)
