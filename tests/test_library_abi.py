@@ -169,6 +169,16 @@ def test_layer_backward_host_validation(lib, kw, code):
     assert lib.gdn_last_error().decode()
 
 
+def test_layer_backward_workspace_forms(lib):
+    """bf16, d = 128, scalar gates and no h0 take the tensor-core form, whose workspace (states, V',
+    two sets of recurrence gradients) is smaller than the CUDA-core form's per-chunk factors; an h0,
+    fp32 tensors or d = 64 take the CUDA-core form."""
+    size = lambda **kw: lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(_layer_bwd(T=4096, **kw)))
+    tc = size(dk=128, dv=128)
+    assert 0 < tc < size(dk=128, dv=128, h0=144)
+    assert tc < size(dk=128, dv=128, dtype=1)
+
+
 def test_layer_backward_workspace(lib):
     a = _layer_bwd()
     need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
