@@ -496,9 +496,9 @@ def bench_part_fwd(name, args, dist, peaks, peak_kind, stream, device):
 
 
 def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
-    """The GQA layer core's training step: gdn_layer_core_fwd then gdn_layer_core_bwd (the
-    recurrence's backward on the tensor cores, once per bf16 half of do), inputs resident,
-    gradients of every input."""
+    """The GQA layer core's training step: gdn_layer_core_fwd keeping its cache, then
+    gdn_layer_core_bwd reading it (the recurrence's backward on the tensor cores, once per bf16
+    half of do), inputs resident, gradients of every input."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     from gated_delta_rule_76_b200.inputs import WORKLOADS
@@ -506,12 +506,12 @@ def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
     wl = WORKLOADS[name]
     x, g = chunk_inputs(name, device, with_dout=True)
     y = torch.empty_like(g["v"])
+    lin = (g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"])
+    cache = torch.empty(gdn.gdn_layer_core_fwd_cache_size(*lin, **gates(g)), dtype=torch.uint8, device=device)
     with torch.cuda.stream(stream):
         def fn():
-            gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], y=y, want_ht=False,
-                                   stream=stream, **gates(g))
-            gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"],
-                                   stream=stream, **gates(g))
+            gdn.gdn_layer_core_fwd(*lin, y=y, want_ht=False, bwd_cache=cache, stream=stream, **gates(g))
+            gdn.gdn_layer_core_bwd(*lin, g["dout"], fwd_cache=cache, stream=stream, **gates(g))
         ms = timed(fn, max(2, args.steps // 4), args.warmup, dist, stream)
     tokens = wl.B * wl.T
     by = (fwd_bytes_per_token(wl, gate=True) + bwd_bytes_per_token(wl)
@@ -523,8 +523,8 @@ def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
             "roofline": roofline(by, fl, ms * 1e-3, peaks, peak_kind,
                                  "gdn_layer_core_fwd + gdn_layer_core_bwd calls"),
             "config": {"B": wl.B, "T": wl.T, "Hk": wl.Hk, "Hv": wl.Hv, "dk": wl.dk, "dv": wl.dv,
-                       "backward": "recurrence on the tensor-core backward kernels, once per bf16 half of do "
-                                   "(conv results as bf16 hi/lo pairs)"}}
+                       "backward": "from the forward's cache (conv results as bf16 hi/lo pairs, o, states, V'); "
+                                   "recurrence on the tensor-core backward kernels, once per bf16 half of do"}}
 
 
 # --------------------------------------------------------------------------------------------
@@ -661,9 +661,10 @@ def _profile_layer_train_b2_t16384():
     from gated_delta_rule_76_b200.inputs import workload_inputs
     x = workload_inputs("gqa_layer_core_bf16", with_dout=True)
     g = {k: v.cuda() for k, v in x.items()}
-    y, _, _ = gdn.gdn_layer_core_fwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], beta=g["beta"])
-    grads = gdn.gdn_layer_core_bwd(g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"], g["dout"],
-                                   beta=g["beta"])
+    lin = (g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"])
+    cache = torch.empty(gdn.gdn_layer_core_fwd_cache_size(*lin, beta=g["beta"]), dtype=torch.uint8, device="cuda")
+    y, _, _ = gdn.gdn_layer_core_fwd(*lin, beta=g["beta"], bwd_cache=cache)
+    grads = gdn.gdn_layer_core_bwd(*lin, g["dout"], beta=g["beta"], fwd_cache=cache)
     torch.cuda.synchronize()
     print("ok", float(y.float().abs().mean()), float(grads["dxq"].abs().mean()))
     return 0

@@ -433,6 +433,41 @@ gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_decode_step");
 }
 
+// The layer backward's tensor-core form: bf16 tensors, d = 128, scalar gates, no initial state.
+// With an initial state h0 the first tokens' dxk is tens of times its RMS (the conv sees one tap
+// there, and the L2 norm's backward divides by a small norm): the tensor-core backward's ~1e-3
+// relative error there exceeds the 2e-2-of-RMS budget, so such calls keep the fp32 CUDA-core form.
+static bool layer_tc_form(int32_t dtype, int64_t dk, int64_t dv, int32_t apc, int32_t gpc, const float* h0) {
+    return dtype == GDN_BF16 && dk == 128 && dv == 128 && !apc && !gpc && h0 == nullptr;
+}
+
+// The layer forward's backward cache (tensor-core form only), byte offsets from its start: the
+// conv results as bf16 hi/lo pairs (q, k, v), the recurrence's output before the gate (fp32),
+// then the chunk forward cache (states, V').
+struct LayerCache {
+    size_t q, k, v, o, tc, bytes;
+};
+static LayerCache plan_layer_cache(const Problem& pb) {
+    LayerCache c{};
+    const size_t BT = (size_t)pb.B * pb.T, qn = BT * pb.Hk * pb.dk, vn = BT * pb.Hv * pb.dv;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    c.q = take(qn * 4); c.k = take(qn * 4); c.v = take(vn * 4); c.o = take(vn * 4);
+    c.tc = take(plan_tc_cache(pb).bytes);
+    c.bytes = off;
+    return c;
+}
+
+size_t gdn_layer_core_fwd_cache_size(const gdn_layer_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hk < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    if (!layer_tc_form(a->dtype, a->dk, a->dv, a->alpha_per_channel, a->gates_per_channel, a->h0)) return 0;
+    return plan_layer_cache(make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map)).bytes;
+}
+
 size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
@@ -467,8 +502,19 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     const Buf out[] = {
         {a->y, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "y"}, {a->ht, st, "ht"},
         {a->conv_state_out, (size_t)a->B * cch * 3 * es, "conv_state_out"},
+        {a->bwd_cache, a->bwd_cache ? a->bwd_cache_bytes : 0, "bwd_cache"},
     };
-    if ((s = check_buffers(in, 10, out, 3))) return s;
+    if ((s = check_buffers(in, 10, out, 4))) return s;
+    if (a->bwd_cache) {
+        if (!layer_tc_form(a->dtype, a->dk, a->dv, a->alpha_per_channel, a->gates_per_channel, a->h0))
+            return fail(GDN_ERR_UNSUPPORTED, "bwd_cache: only the tensor-core form (bf16, d = 128, scalar gates, no h0) "
+                                             "keeps a layer cache");
+        if (reinterpret_cast<uintptr_t>(a->bwd_cache) & 255u)
+            return fail(GDN_ERR_INVALID_ARG, "bwd_cache is not 256-byte aligned");
+        if (a->bwd_cache_bytes < gdn_layer_core_fwd_cache_size(a))
+            return fail(GDN_ERR_WORKSPACE, "bwd_cache has %zu bytes, %zu needed", a->bwd_cache_bytes,
+                        gdn_layer_core_fwd_cache_size(a));
+    }
     cudaStream_t sm = static_cast<cudaStream_t>(stream);
     if (a->T == 0) {
         if (a->conv_state_out) {
@@ -490,7 +536,12 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     // CUDA-core forward.
     const bool split = a->dtype == GDN_BF16 && !f.apc && !f.gpc &&
                        tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
+    if (a->bwd_cache && !split)
+        return fail(GDN_ERR_UNSUPPORTED, "bwd_cache: the tensor-map encoder of the CUDA driver is unavailable");
     const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
+    const LayerCache lc = a->bwd_cache ? plan_layer_cache(pb) : LayerCache{};
+    char* cache = static_cast<char*>(a->bwd_cache);
+    if (cache) base = cache;  // the conv results are kept in the cache (same layout as below)
     ConvParams cp{};
     cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
     if (split) {
@@ -513,7 +564,15 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     io.z_bf16 = a->dtype == GDN_BF16;
     if (split) {
         io.q_lo = cp.q_lo; io.k_lo = cp.k_lo; io.v_lo = cp.v_lo;
-        e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm);
+        if (cache) {
+            const TcCache cc = plan_tc_cache(pb);
+            char* cb = cache + lc.tc;
+            const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
+                                 reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo), reinterpret_cast<float*>(cache + lc.o)};
+            e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, &save);
+        } else {
+            e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm);
+        }
     } else {
         WsPlan plan = plan_chunk_ws(pb, false, false);
         e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
@@ -535,12 +594,8 @@ struct LayerBwdPlan {
     size_t q, k, v, o, dout, gq, gk, gv, wpart, cache, chunk, bytes;
     size_t gq2, gk2, gv2, ga2, gb2, gh2;  // tensor-core form: gradients from the lo half of do
 };
-// With an initial state h0 the first tokens' dxk is tens of times its RMS (the conv sees one tap
-// there, and the L2 norm's backward divides by a small norm): the tensor-core backward's ~1e-3
-// relative error there exceeds the 2e-2-of-RMS budget, so such calls keep the fp32 CUDA-core form.
 static bool layer_bwd_tc_form(const gdn_layer_bwd_args* a) {
-    return a->dtype == GDN_BF16 && a->dk == 128 && a->dv == 128 && !a->alpha_per_channel && !a->gates_per_channel &&
-           a->h0 == nullptr;
+    return layer_tc_form(a->dtype, a->dk, a->dv, a->alpha_per_channel, a->gates_per_channel, a->h0);
 }
 static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& pb) {
     LayerBwdPlan w{};
@@ -553,12 +608,16 @@ static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& p
         return o;
     };
     w.chunk = w.tc ? 0 : ~size_t(0);
-    w.q = take(qn * 4); w.k = take(qn * 4); w.v = take(vn * 4); w.o = take(vn * 4);
+    // with the forward's cache the conv results, o, the states and V' are read from it
+    const bool cached = w.tc && a->fwd_cache != nullptr;
+    if (!cached) {
+        w.q = take(qn * 4); w.k = take(qn * 4); w.v = take(vn * 4); w.o = take(vn * 4);
+    }
     w.dout = take(vn * 4);  // fp32, or bf16 hi then lo
     w.gq = take(qn * 4); w.gk = take(qn * 4); w.gv = take(vn * 4);
     w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk) * 4);
     if (w.tc) {
-        w.cache = take(plan_tc_cache(pb).bytes);
+        w.cache = cached ? ~size_t(0) : take(plan_tc_cache(pb).bytes);
         const size_t ng = BT * a->Hv;  // scalar gates
         w.gq2 = take(qn * 4); w.gk2 = take(qn * 4); w.gv2 = take(vn * 4);
         w.ga2 = take(ng * 4); w.gb2 = take(ng * 4);
@@ -603,6 +662,7 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
         {a->alpha, na * gs, "alpha"}, {a->b, nb * gs, "b"}, {a->w, nw * gs, "w"},
         {a->z, BT * a->Hv * a->dv * es, "z"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_y, BT * a->Hv * a->dv * es, "grad_y"}, {a->grad_ht, st, "grad_ht"},
+        {a->fwd_cache, a->fwd_cache ? a->fwd_cache_bytes : 0, "fwd_cache"},
     };
     const Buf out[] = {
         {a->grad_xq, BT * a->Hk * a->dk * 4, "grad_xq"}, {a->grad_xk, BT * a->Hk * a->dk * 4, "grad_xk"},
@@ -610,7 +670,18 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
         {a->grad_alpha, na * 4, "grad_alpha"}, {a->grad_b, nb * 4, "grad_b"}, {a->grad_w, nw * 4, "grad_w"},
         {a->grad_z, BT * a->Hv * a->dv * 4, "grad_z"}, {a->grad_h0, st, "grad_h0"},
     };
-    if ((s = check_buffers(in, 12, out, 9))) return s;
+    if ((s = check_buffers(in, 13, out, 9))) return s;
+    if (a->fwd_cache) {
+        if (!layer_bwd_tc_form(a))
+            return fail(GDN_ERR_UNSUPPORTED, "fwd_cache: only the tensor-core form (bf16, d = 128, scalar gates, no h0) "
+                                             "keeps a layer cache");
+        if (reinterpret_cast<uintptr_t>(a->fwd_cache) & 255u)
+            return fail(GDN_ERR_INVALID_ARG, "fwd_cache is not 256-byte aligned");
+        const size_t need = plan_layer_cache(make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale,
+                                                          a->head_map)).bytes;
+        if (a->fwd_cache_bytes < need)
+            return fail(GDN_ERR_INVALID_ARG, "fwd_cache has %zu bytes, %zu needed", a->fwd_cache_bytes, need);
+    }
     cudaStream_t sm = static_cast<cudaStream_t>(stream);
     if (a->T == 0) {
         cudaError_t e = cudaMemsetAsync(a->grad_conv_w, 0, cch * 4 * 4, sm);
@@ -642,23 +713,30 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     if (plan.tc) {
         if (!tc_fwd_eligible(pb, true, bf16g, f))
             return fail(GDN_ERR_UNSUPPORTED, "the tensor-map encoder of the CUDA driver is unavailable");
-        // 1. conv + SiLU + L2, fp32 results stored as bf16 hi/lo pairs
+        // 1. conv + SiLU + L2, fp32 results stored as bf16 hi/lo pairs; 2. the tensor-core forward
+        //    in saving mode: o (fp32, no gate), the chunk states and V'.  Both come from the
+        //    forward's cache when the caller passes one.
         const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
-        char* q = wsb + plan.q;
-        char* k = wsb + plan.k;
-        char* v = wsb + plan.v;
+        char* fc = static_cast<char*>(const_cast<void*>(a->fwd_cache));
+        const LayerCache lc = fc ? plan_layer_cache(pb) : LayerCache{};
+        char* q = fc ? fc + lc.q : wsb + plan.q;
+        char* k = fc ? fc + lc.k : wsb + plan.k;
+        char* v = fc ? fc + lc.v : wsb + plan.v;
+        float* o = fc ? reinterpret_cast<float*>(fc + lc.o) : at(plan.o);
+        char* cb = fc ? fc + lc.tc : wsb + plan.cache;
         cp.q = q; cp.q_lo = q + qn * 2; cp.k = k; cp.k_lo = k + qn * 2; cp.v = v; cp.v_lo = v + vn * 2;
-        e = bf16_conv(cp, sm);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
-        // 2. the tensor-core forward in saving mode: o (fp32, no gate), the chunk states and V'
         io.q = cp.q; io.k = cp.k; io.v = cp.v; io.q_lo = cp.q_lo; io.k_lo = cp.k_lo; io.v_lo = cp.v_lo;
-        io.o = at(plan.o); io.o_type = 1;
-        const TcCache cc = plan_tc_cache(pb);
-        char* cb = wsb + plan.cache;
-        const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
-                             reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo)};
-        e = tc_chunk_fwd(pb, io, f, bf16g, ws_status(workspace), sm, &save);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+        lio.o = o;
+        if (!fc) {
+            e = bf16_conv(cp, sm);
+            if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
+            io.o = o; io.o_type = 1;
+            const TcCache cc = plan_tc_cache(pb);
+            const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
+                                 reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo), nullptr};
+            e = tc_chunk_fwd(pb, io, f, bf16g, ws_status(workspace), sm, &save);
+            if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
+        }
         // 3. swish gate; the gradient of o as bf16 hi/lo pairs (tensor-core operands)
         lio.dout16 = reinterpret_cast<__nv_bfloat16*>(wsb + plan.dout);
         lio.dout16_lo = lio.dout16 + vn;

@@ -47,6 +47,7 @@ struct TcFwdSave {
     float* s0;               // [B*Hv][NT + 1][dv/4][dk][4]
     __nv_bfloat16* vp_hi;    // [B,T,Hv,dv]
     __nv_bfloat16* vp_lo;
+    float* o_raw;            // with the swish gate, may be NULL: the output before the gate (fp32)
 };
 bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags f);
 cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,

@@ -130,6 +130,7 @@ struct Params {
                                  //   the final state
     __nv_bfloat16* vp_hi;        // [B,T,Hv,dv]: V' = T (Z - Ehat S0) of every token, split
     __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
+    float* o_raw;                // GATE only, may be NULL: the output before the gate, fp32 [B,T,Hv,dv]
 };
 
 __device__ __forceinline__ float bf(const uint8_t* tile, uint32_t off) {
@@ -600,6 +601,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float ov[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] = pb.scale * __uint_as_float(r[i]);
+                if (GATE && p.o_raw) {
+                    float* rp = p.o_raw + obase;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < nrow) rp[i * orow] = ov[i];
+                }
                 if (GATE) {
                     // z column j, rows 32h .. 32h + 31, from the TMA tile (zero past the end)
                     const uint8_t* zt = sm + SM_Z + vbase + 32u * h * 128u;

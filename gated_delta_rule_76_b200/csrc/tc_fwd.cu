@@ -70,6 +70,7 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
         p.s0_out = save->s0;
         p.vp_hi = save->vp_hi;
         p.vp_lo = save->vp_lo;
+        p.o_raw = save->o_raw;
     }
     const bool gate = f.gate;
     if (split) {

@@ -58,7 +58,8 @@ class LayerArgs(ctypes.Structure):
                 ("z", P), ("h0", P), ("y", P), ("ht", P), ("conv_state_out", P), ("head_map", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32), ("bwd_cache", P),
+                ("bwd_cache_bytes", ctypes.c_size_t)]
 
 
 class LayerBwdArgs(ctypes.Structure):
@@ -68,11 +69,11 @@ class LayerBwdArgs(ctypes.Structure):
                 ("grad_b", P), ("grad_w", P), ("grad_z", P), ("grad_h0", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t)]
 
 
 EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
-            "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_workspace_size",
+            "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_cache_size", "gdn_layer_core_fwd_workspace_size",
             "gdn_layer_core_fwd", "gdn_layer_core_bwd_workspace_size", "gdn_layer_core_bwd",
             "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches", "gdn_version"]
 
@@ -105,6 +106,8 @@ def load(path: str = LIB_PATH):
     lib.gdn_chunk_bwd.restype = ctypes.c_int
     lib.gdn_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), P]
     lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_layer_core_fwd_cache_size.argtypes = [ctypes.POINTER(LayerArgs)]
+    lib.gdn_layer_core_fwd_cache_size.restype = ctypes.c_size_t
     lib.gdn_layer_core_fwd_workspace_size.argtypes = [ctypes.POINTER(LayerArgs)]
     lib.gdn_layer_core_fwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_layer_core_fwd.argtypes = [ctypes.POINTER(LayerArgs), P, ctypes.c_size_t, P]
@@ -326,12 +329,36 @@ def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=N
     return o
 
 
+def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y=None, ht=None, cs=None,
+                out_f32=0, bwd_cache=None):
+    bb, ww, gpc = _gates(alpha, b, w, beta)
+    B, T, Hk, dk = xq.shape
+    Hv, dv = xv.shape[2], xv.shape[3]
+    hm = _head_map(head_map, xq.device)
+    a = LayerArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
+                  b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
+                  conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
+                  dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
+                  gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha), out_f32=out_f32,
+                  bwd_cache=_ptr(bwd_cache), bwd_cache_bytes=bwd_cache.numel() if bwd_cache is not None else 0)
+    return a, hm
+
+
+def gdn_layer_core_fwd_cache_size(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, h0=None,
+                                  head_map=None, scale: float = 1.0) -> int:
+    """Bytes of the layer forward's optional backward cache (0 where it cannot keep one)."""
+    a, _ = _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale)
+    return int(load().gdn_layer_core_fwd_cache_size(ctypes.byref(a)))
+
+
 def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, h0=None,
                        head_map=None, scale: float = 1.0, *, want_ht: bool = True,
                        want_conv_state: bool = False, y=None, out_f32: bool = False,
+                       bwd_cache: Optional[torch.Tensor] = None,
                        workspace: Optional[torch.Tensor] = None, stream=None):
-    """GQA layer core forward.  Returns (y, ht or None, conv_state or None)."""
-    bb, ww, gpc = _gates(alpha, b, w, beta)
+    """GQA layer core forward.  Returns (y, ht or None, conv_state or None).  ``bwd_cache``: a
+    uint8 device tensor of gdn_layer_core_fwd_cache_size() bytes that a later
+    gdn_layer_core_bwd(..., fwd_cache=) over the same inputs reads."""
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
     if y is None:
@@ -339,13 +366,8 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
     ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=xq.device) if want_ht else None
     cs = (torch.empty((B, 2 * Hk * dk + Hv * dv, 3), dtype=xq.dtype, device=xq.device)
           if want_conv_state else None)
-    hm = _head_map(head_map, xq.device)
-    a = LayerArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
-                  b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
-                  conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
-                  dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
-                  gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha),
-                  out_f32=int(y.dtype == torch.float32 and xq.dtype != torch.float32))
+    a, hm = _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y=y, ht=ht, cs=cs,
+                        out_f32=int(y.dtype == torch.float32 and xq.dtype != torch.float32), bwd_cache=bwd_cache)
     lib = load()
     need = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, xq.device, workspace)
@@ -356,9 +378,11 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
 
 def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, beta=None, h0=None,
                        grad_ht=None, head_map=None, scale: float = 1.0, *, want_h0_grad: bool = True,
+                       fwd_cache: Optional[torch.Tensor] = None,
                        workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
     """GQA layer core backward (reverse mode of gdn_layer_core_fwd).  Returns a dict of fp32
-    gradients: dxq, dxk, dxv, dconv_w, dalpha, dz, dh0 (or None) and db/dw or dbeta."""
+    gradients: dxq, dxk, dxv, dconv_w, dalpha, dz, dh0 (or None) and db/dw or dbeta.
+    ``fwd_cache``: the cache a gdn_layer_core_fwd(..., bwd_cache=) call filled with these inputs."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
@@ -383,7 +407,8 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
                      grad_b=_ptr(gb), grad_w=_ptr(gw), grad_z=_ptr(out["dz"]), grad_h0=_ptr(out["dh0"]),
                      B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                      alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc, dtype=_dt(xq),
-                     gate_dtype=_dt(alpha))
+                     gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
+                     fwd_cache_bytes=fwd_cache.numel() if fwd_cache is not None else 0)
     lib = load()
     need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, dev, workspace)

@@ -248,8 +248,19 @@ typedef struct gdn_layer_args {
     int32_t dtype;
     int32_t gate_dtype;
     int32_t out_f32;      /* 1: y is written in fp32 instead of dtype */
+    /* Optional cache for a later gdn_layer_core_bwd over the same inputs (training): when not NULL
+     * the forward also keeps its conv results (bf16 hi/lo pairs), the recurrence's output before
+     * the gate (fp32), the state entering every chunk and V' of every token in this caller
+     * buffer, and a backward given it skips recomputing them.  Needs bwd_cache_bytes >=
+     * gdn_layer_core_fwd_cache_size(args) and a 256-byte-aligned start.  Only the layer's
+     * tensor-core backward form keeps one (bf16 tensors, dk = dv = 128, scalar gates, no h0):
+     * elsewhere the size is 0 and bwd_cache must be NULL. */
+    void* bwd_cache;
+    size_t bwd_cache_bytes;
 } gdn_layer_args;
 
+/* Bytes of the optional layer forward cache (0 where the layer backward cannot use one). */
+GDN_API size_t gdn_layer_core_fwd_cache_size(const gdn_layer_args* args);
 GDN_API size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* args);
 GDN_API gdn_status gdn_layer_core_fwd(const gdn_layer_args* args, void* workspace, size_t workspace_bytes,
                               gdn_stream stream);
@@ -302,6 +313,12 @@ typedef struct gdn_layer_bwd_args {
     int32_t gates_per_channel;
     int32_t dtype;
     int32_t gate_dtype;
+    /* Optional: the cache a gdn_layer_core_fwd call wrote with exactly these inputs.  The backward
+     * then reads the conv results, o, the chunk states and V' from it instead of recomputing them.
+     * The library cannot check that the cache belongs to these inputs: a stale cache gives wrong
+     * gradients.  NULL: the forward parts are recomputed. */
+    const void* fwd_cache;
+    size_t fwd_cache_bytes;
 } gdn_layer_bwd_args;
 
 GDN_API size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* args);

@@ -182,3 +182,30 @@ def test_layer_core_backward_matches_oracle(B, T, Hk, Hv, d, gpc, gdt, dt, h0):
     kind = "f32" if dt == "f32" else "bf16"
     for key in ["dxq", "dxk", "dxv", "dconv_w", "dalpha", "dz", "dh0"] + (["db", "dw"] if gpc else ["dbeta"]):
         assert_parity(got[key], ref[key], kind, key)
+
+
+@pytest.mark.parametrize("B,T,Hk,Hv,gdt", [(2, 200, 2, 4, "f32"), (1, 64, 1, 1, "bf16")])
+def test_layer_core_backward_from_forward_cache(B, T, Hk, Hv, gdt):
+    """A layer forward keeping its cache, then a backward reading it: y and every gradient are
+    bit for bit those of the calls without a cache (the same kernels on the same values), and the
+    gradients match the oracle."""
+    x = draw(B, T, Hk, Hv, 128, 128, alpha_per_channel=False, gates_per_channel=False, dtype="bf16",
+             gate_dtype=gdt, seed=67, has_h0=False, conv=True, swish_gate=True, with_dout=True, with_dht=True)
+    g = to_cuda(x)
+    args = (g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"])
+    n = gdn.gdn_layer_core_fwd_cache_size(*args, beta=g["beta"], scale=0.8)
+    assert n > 0
+    cache = torch.empty(n, dtype=torch.uint8, device="cuda")
+    y_c, ht_c, _ = gdn.gdn_layer_core_fwd(*args, beta=g["beta"], scale=0.8, out_f32=True, bwd_cache=cache)
+    y, ht, _ = gdn.gdn_layer_core_fwd(*args, beta=g["beta"], scale=0.8, out_f32=True)
+    got_c = gdn.gdn_layer_core_bwd(*args, g["dout"], beta=g["beta"], grad_ht=g["dht"], scale=0.8, fwd_cache=cache)
+    got = gdn.gdn_layer_core_bwd(*args, g["dout"], beta=g["beta"], grad_ht=g["dht"], scale=0.8)
+    torch.cuda.synchronize()
+    assert torch.equal(y_c, y) and torch.equal(ht_c, ht)
+    keys = ["dxq", "dxk", "dxv", "dconv_w", "dalpha", "dz", "dh0", "dbeta"]
+    for key in keys:
+        assert torch.equal(got_c[key], got[key]), key
+    ref = oracle.layer_core_bwd(x["q"], x["k"], x["v"], x["conv_w"], x["alpha"], x["z"], x["dout"],
+                                dht=x["dht"], scale=0.8, beta=x["beta"])
+    for key in keys:
+        assert_parity(got_c[key], ref[key], "bf16", key)

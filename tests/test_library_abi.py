@@ -169,6 +169,39 @@ def test_layer_backward_host_validation(lib, kw, code):
     assert lib.gdn_last_error().decode()
 
 
+def _layer_fwd(**kw):
+    M = 1 << 16
+    base = dict(xq=16, xk=32, xv=48, conv_w=64, alpha=80, b=96, w=None, z=112, h0=None, y=16 * M, ht=None,
+                conv_state_out=None, head_map=None, B=1, T=64, Hk=1, Hv=1, dk=128, dv=128, scale=1.0,
+                alpha_per_channel=0, gates_per_channel=0, dtype=0, gate_dtype=1, out_f32=0, bwd_cache=None,
+                bwd_cache_bytes=0)
+    base.update(kw)
+    return gdn.LayerArgs(**base)
+
+
+def test_layer_forward_cache_on_the_host(lib):
+    """Only the tensor-core form (bf16, d = 128, scalar gates, no h0) keeps a layer cache; a cache
+    elsewhere, misaligned, overlapping an output or too small is refused before any launch."""
+    size = lambda **kw: lib.gdn_layer_core_fwd_cache_size(ctypes.byref(_layer_fwd(**kw)))
+    need = size()
+    assert need > 0 and size(T=65) > need
+    assert size(h0=144) == 0 and size(dtype=1) == 0 and size(dk=64, dv=64) == 0
+    assert size(alpha_per_channel=1, gates_per_channel=1, w=128, gate_dtype=0) == 0
+    ws = ctypes.c_void_p(1 << 34)
+    run = lambda **kw: lib.gdn_layer_core_fwd(ctypes.byref(_layer_fwd(**kw)), ws, 1 << 34, None)
+    assert run(h0=144, bwd_cache=1 << 30, bwd_cache_bytes=need) == 2
+    assert run(bwd_cache=(1 << 30) + 16, bwd_cache_bytes=need) == 1
+    assert run(bwd_cache=16 << 16, bwd_cache_bytes=need) == 1      # overlaps y
+    assert run(bwd_cache=1 << 30, bwd_cache_bytes=need - 1) == 4
+    bwd = lambda **kw: lib.gdn_layer_core_bwd(ctypes.byref(_layer_bwd(dk=128, dv=128, **kw)), ws, 1 << 34, None)
+    assert bwd(h0=144, fwd_cache=1 << 30, fwd_cache_bytes=need) == 2
+    assert bwd(fwd_cache=(1 << 30) + 16, fwd_cache_bytes=need) == 1
+    assert bwd(fwd_cache=1 << 30, fwd_cache_bytes=need - 1) == 1
+    # with a cache the backward's workspace leaves out the conv results, o, the states and V'
+    wsz = lambda **kw: lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(_layer_bwd(dk=128, dv=128, T=4096, **kw)))
+    assert 0 < wsz(fwd_cache=1 << 30, fwd_cache_bytes=1 << 40) < wsz()
+
+
 def test_layer_backward_workspace_forms(lib):
     """bf16, d = 128, scalar gates and no h0 take the tensor-core form, whose workspace (states, V',
     two sets of recurrence gradients) is smaller than the CUDA-core form's per-chunk factors; an h0,
