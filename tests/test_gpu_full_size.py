@@ -5,7 +5,8 @@ sample of (sequence, head) pairs one by one (each pair is independent), and the 
 states and gradients of those pairs are compared at the stated tolerances:
   * GDN-2 forward + backward, B=8 T=4096 H=16 d=128 (bf16 inputs, fp32 state);
   * Gated DeltaNet forward with scalar gates, B=8 T=4096 H=16 d=128;
-  * GQA layer core, B=2 T=16384, 16 key / 128 value heads (conv + SiLU + L2 + swish gate);
+  * GQA layer core, B=2 T=16384, 16 key / 128 value heads (conv + SiLU + L2 + swish gate), and its
+    training step (forward keeping the cache, backward) for one key head and its 8 value heads;
   * GDN-2 decode, 256 sequences x 1024 steps, H=16 d=128 (every step's output of the sampled
     sequences, and their final states).
 """
@@ -103,6 +104,39 @@ def test_gqa_layer_core_full_size():
         y_ref = oracle.swish_gate(o_ref[0, :, 0], npf(x["z"][b, :, hv]))
         assert_parity(y[b, :, hv], y_ref, "bf16", f"y ({b},{hv})")
         assert_parity(ht[b, hv], ht_ref[0, 0], "bf16", f"ht ({b},{hv})")
+
+
+def test_gqa_layer_training_step_full_size():
+    """The layer's training step as the benchmark times it (forward keeping its cache, backward
+    reading it) on the full workload.  The conv is depthwise and the key heads are independent, so
+    the oracle recomputes one key head with its 8 value heads over both sequences exactly: every
+    gradient of those channels, heads and conv weights is compared."""
+    name = "gqa_layer_core_bf16"
+    wl = WORKLOADS[name]
+    x = workload_inputs(name, with_dout=True)
+    g = {k: v.cuda() for k, v in x.items()}
+    lin = (g["q"], g["k"], g["v"], g["conv_w"], g["alpha"], g["z"])
+    cache = torch.empty(gdn.gdn_layer_core_fwd_cache_size(*lin, beta=g["beta"]), dtype=torch.uint8, device="cuda")
+    gdn.gdn_layer_core_fwd(*lin, beta=g["beta"], bwd_cache=cache, want_ht=False)
+    got = gdn.gdn_layer_core_bwd(*lin, g["dout"], beta=g["beta"], fwd_cache=cache)
+    torch.cuda.synchronize()
+    del cache
+    d, Hk, Hv = wl.dk, wl.Hk, wl.Hv
+    group = Hv // Hk
+    hk = int(np.random.default_rng(7).integers(Hk))
+    hv = slice(hk * group, (hk + 1) * group)
+    w = npf(x["conv_w"])
+    rows = np.r_[hk * d:(hk + 1) * d, Hk * d + hk * d:Hk * d + (hk + 1) * d,
+                 2 * Hk * d + hv.start * d:2 * Hk * d + hv.stop * d]
+    ref = oracle.layer_core_bwd(npf(x["q"][:, :, hk:hk + 1]), npf(x["k"][:, :, hk:hk + 1]), npf(x["v"][:, :, hv]),
+                                w[rows], npf(x["alpha"][:, :, hv]), npf(x["z"][:, :, hv]), npf(x["dout"][:, :, hv]),
+                                beta=npf(x["beta"][:, :, hv]))
+    assert_parity(got["dxq"][:, :, hk:hk + 1], ref["dxq"], "bf16", f"dxq (key head {hk})")
+    assert_parity(got["dxk"][:, :, hk:hk + 1], ref["dxk"], "bf16", f"dxk (key head {hk})")
+    for key in ("dxv", "dz", "dalpha", "dbeta"):
+        assert_parity(got[key][:, :, hv], ref[key], "bf16", key)
+    assert_parity(got["dh0"][:, hv], ref["dh0"], "bf16", "dh0")
+    assert_parity(got["dconv_w"].cpu()[torch.as_tensor(rows)], ref["dconv_w"], "bf16", "dconv_w")
 
 
 def test_gdn2_decode_1024_steps_full_size():
