@@ -1,5 +1,6 @@
-"""The pins must bite: plausible mistakes planted in a copy of the oracle (compiled on the CPU)
-each make at least one pin of test_oracle_pins.py fail."""
+"""The pins must bite: plausible mistakes planted in a copy of the oracle (the compiled recurrence,
+and the numpy reverse mode of the layer core) each make at least one pin of test_oracle_pins.py
+fail."""
 import os
 import shutil
 import subprocess
@@ -102,3 +103,52 @@ def test_planted_mistake_is_caught(name, edits, workdir):
     finally:
         oracle._lib = saved
     assert failed, f"no pin caught the planted mistake: {name}"
+
+
+# The layer core's reverse mode is numpy code in oracle.py: (name, original text, planted mistake).
+# Each lives in the backward only (the layer pin's forward runs through the compiled conv and
+# recurrence), so the finite-difference pin must catch it.
+PY = os.path.join(os.path.dirname(oracle.__file__), "oracle.py")
+LAYER_MUTANTS = [
+    ("swish gate: dz without its z s (1 - s) term",
+     "dz = g * o * (sg + zz * sg * (1.0 - sg))", "dz = g * o * sg"),
+    ("swish gate: do without the factor z", "do = g * zz * sg", "do = g * sg"),
+    ("L2 norm backward without the projection",
+     "da = ((gout - out * dot) / n).reshape(a.shape)", "da = (gout / n).reshape(a.shape)"),
+    ("SiLU backward: the sigmoid's derivative instead of SiLU's",
+     "du = da * (s + u * s * (1.0 - s))", "du = da * s * (1.0 - s)"),
+    ("conv input gradient: taps reversed",
+     "dx[:, :T - sh] += w[:, tap] * du[:, sh:]", "dx[:, :T - sh] += w[:, 3 - tap] * du[:, sh:]"),
+    ("conv weight gradient: current tap shifted by one token",
+     "dw[:, tap] = np.sum(du * x, axis=(0, 1))", "dw[:, tap] = np.sum(du[:, 1:] * x[:, :-1], axis=(0, 1))"),
+    ("recomputed conv: history taps shifted the wrong way",
+     "u[:, sh:] += w[:, tap] * x[:, :T - sh]", "u[:, :T - sh] += w[:, tap] * x[:, sh:]"),
+]
+
+
+def _oracle_copy(src):
+    import types
+    mod = types.ModuleType("oracle_mutant")
+    mod.__file__ = oracle.__file__
+    exec(compile(src, PY, "exec"), mod.__dict__)
+    return mod
+
+
+def test_unmutated_layer_oracle_copy_passes_its_pin(monkeypatch):
+    monkeypatch.setattr(pins, "oracle", _oracle_copy(open(PY).read()))
+    for channel_gates in (False, True):
+        pins.test_layer_backward_finite_differences(channel_gates)
+
+
+@pytest.mark.parametrize("name,old,new", LAYER_MUTANTS, ids=[m[0] for m in LAYER_MUTANTS])
+def test_planted_layer_backward_mistake_is_caught(name, old, new, monkeypatch):
+    src = open(PY).read()
+    assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+    monkeypatch.setattr(pins, "oracle", _oracle_copy(src.replace(old, new)))
+    caught = []
+    for channel_gates in (False, True):
+        try:
+            pins.test_layer_backward_finite_differences(channel_gates)
+        except AssertionError:
+            caught.append(channel_gates)
+    assert caught, f"no pin caught the planted mistake: {name}"
