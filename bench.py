@@ -111,8 +111,8 @@ def load_peaks():
 # of its two kernels (reverse scan, gradients) on B=2 T=2048 (an eighth of the workload's tokens:
 # the per-chunk traffic is fixed, so it scales with the tokens); see
 # profiles/chunk_bwd_kernels_gdn2_b2_t2048.md.  To be set to None whenever those kernels change.
-# (The split-input template flag added later is false in the measured instantiations and compiles
-# out of them: same registers, same shared memory, same instructions on that path.)
+# (The split-input template flag added later is false in the measured instantiations; its code sits
+# under `if (SPLIT)` and compiles out of them: ptxas reports the same registers and shared memory.)
 BWD_CALL_TRAFFIC_BYTES = (84.17 + 54.30 + 360.25 + 154.68) * 1e6 * 8
 
 
