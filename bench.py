@@ -62,16 +62,20 @@ def fwd_bytes_per_token(wl, T=None, with_h0=None, gate=False):
     return b
 
 
-def bwd_bytes_per_token(wl, T=None):
-    """Reads q, k, v, alpha, b, w, dO (+ h0); writes fp32 dq, dk, dv, dalpha, db, dw (+ dh0)."""
+def bwd_bytes_per_token(wl, T=None, grad_bytes=None):
+    """API-level bytes of one backward token: q, k, v, alpha, b, w and dO read; the gradients of
+    q, k, v, alpha, b, w written (+ h0 read, dh0 written).  The algorithmic count sizes every
+    gradient like its input (bf16 here); `grad_bytes=4` gives the bytes the library actually
+    writes (its gradients are fp32)."""
     T = T or wl.T
     es, gs = _es(wl.dtype), _es(wl.gate_dtype)
+    ges, ggs = (grad_bytes or es), (grad_bytes or gs)
     n_qk = wl.Hk * 2 * wl.dk
     n_v = wl.Hv * wl.dv
     n_a = wl.Hv * (wl.dk if wl.alpha_per_channel else 1)
     n_g = wl.Hv * ((wl.dk + wl.dv) if wl.gates_per_channel else 1)
     b = (n_qk + n_v) * es + (n_a + n_g) * gs + n_v * es           # inputs and dO read
-    b += (n_qk + n_v + n_a + n_g) * 4                              # fp32 gradients written
+    b += (n_qk + n_v) * ges + (n_a + n_g) * ggs                    # gradients written
     b += (2 if wl.has_h0 else 1) * wl.Hv * wl.dk * wl.dv * 4 / T   # h0 read, dh0 written
     return b
 
@@ -107,13 +111,11 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-# DRAM bytes (read + write) of one gdn_chunk_bwd call on the headline workload, from one ncu capture
-# of its two kernels (reverse scan, gradients) on B=2 T=2048 (an eighth of the workload's tokens:
-# the per-chunk traffic is fixed, so it scales with the tokens); see
-# profiles/chunk_bwd_kernels_gdn2_b2_t2048.md.  To be set to None whenever those kernels change.
-# (The split-input template flag added later is false in the measured instantiations; its code sits
-# under `if (SPLIT)` and compiles out of them: ptxas reports the same registers and shared memory.)
-BWD_CALL_TRAFFIC_BYTES = (84.17 + 54.30 + 360.25 + 154.68) * 1e6 * 8
+# DRAM bytes (read + write) of one gdn_chunk_bwd call on the headline workload, summed over its two
+# kernels (reverse scan, gradients) from one ncu capture per kernel of the full-size call with
+# dram__bytes_read.sum and dram__bytes_write.sum.  None until such a capture exists for the
+# kernels as they are now; to be reset to None whenever those kernels change.
+BWD_CALL_TRAFFIC_BYTES = None
 
 
 def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False,
@@ -341,6 +343,9 @@ def bench_headline(args, dist, peaks, peak_kind, stream, device):
     roof = roofline(dom[0], dom[1], dom[2] * 1e-3, peaks, peak_kind,
                     f"gdn_chunk_{dominant} call (dominant call of the step; its kernels back to back)",
                     traffic=BWD_CALL_TRAFFIC_BYTES if dominant == "bwd" else None)
+    if dominant == "bwd":
+        # the gradients leave as fp32: what the call writes, beside the algorithmic (bf16) count
+        roof["written_bytes_fp32_grads"] = int(bwd_bytes_per_token(wl, grad_bytes=4) * tokens)
     step_roof = roofline(bytes_f + bytes_b, flops_f + flops_b, ms * 1e-3, peaks, peak_kind,
                          "whole fwd+bwd step")
     return {"ms": ms, "tokens": tokens, "launches_per_step": launches_per_step, "fwd_ms": fwd_ms,
@@ -517,7 +522,7 @@ def bench_part_layer_train(args, dist, peaks, peak_kind, stream, device):
         ms = timed(fn, max(2, args.steps // 4), args.warmup, dist, stream)
     tokens = wl.B * wl.T
     by = (fwd_bytes_per_token(wl, gate=True) + bwd_bytes_per_token(wl)
-          + wl.Hv * wl.dv * (_es(wl.dtype) + 4)) * tokens               # + z read, fp32 dz written
+          + wl.Hv * wl.dv * 2 * _es(wl.dtype)) * tokens                 # + z read, dz written
     fl = (fwd_flops_per_token(wl) + bwd_flops_per_token(wl)) * tokens
     del x, g
     return {"workload": name + " (training step: layer forward + backward)",
@@ -672,7 +677,24 @@ def _profile_layer_train_b2_t16384():
     return 0
 
 
-PROFILE_CASES = {"train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024,
+def _profile_decode_b256():
+    """GDN-2 decode on its full workload shape (256 sequences, 16 heads, d=128, fp32 state of
+    268 MB), 8 consecutive steps."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import WORKLOADS, decode_initial_state, decode_inputs
+    wl = WORKLOADS[DECODE]
+    xs = decode_inputs(DECODE, 8)
+    g = {k: v.cuda() for k, v in xs.items()}
+    state = decode_initial_state(DECODE).cuda()
+    for s in range(8):
+        o = gdn.gdn_decode_step(state, g["q"][s], g["k"][s], g["v"][s], g["alpha"][s], b=g["b"][s], w=g["w"][s])
+    torch.cuda.synchronize()
+    print("ok", float(o.float().abs().mean()), wl.B)
+    return 0
+
+
+PROFILE_CASES = {"decode_b256": _profile_decode_b256, "train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024,
                  "layer_b2_t16384": _profile_layer_b2_t16384, "train_b8_t4096": _profile_train_b8_t4096,
                  "layer_train_b2_t16384": _profile_layer_train_b2_t16384}
 
@@ -763,11 +785,22 @@ def main():
         "gpu_launches": int(head["launches_per_step"] * args.steps),
         "clocks": clk,
     }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, wl)
+    # the other workloads last: a reader that keeps only the line's tail still sees them, and
+    # the line ends with a compact summary of every workload's rate and roofline fraction
     line.update(extra)
     if sub:
         line["parts"] = sub
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(x, wl)
+    summary = {"step_frac": head["step_roofline"]["frac"], "bwd_frac": head["roofline"]["frac"],
+               "fwd_keeping_cache_frac": head["fwd_roofline"]["frac"]}
+    if "decode" in extra:
+        summary["decode_tokens_s"] = round(extra["decode"]["value"], 1)
+        summary["decode_frac"] = extra["decode"]["roofline"]["frac"]
+    for key, part in sub.items():
+        summary[key + "_tokens_s"] = round(part["value"], 1)
+        summary[key + "_frac"] = part["roofline"]["frac"]
+    line["summary"] = summary
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

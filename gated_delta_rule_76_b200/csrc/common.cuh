@@ -28,8 +28,12 @@ struct Problem {
     float scale;
     const int32_t* head_map;  // may be null: hv / (Hv / Hk)
 
+    // An explicit map entry outside [0, Hk) breaks the interface's precondition; it is clamped
+    // into range so that no kernel reads outside q or k (the result is then unspecified).
     __device__ __forceinline__ int key_head(int hv) const {
-        return head_map ? head_map[hv] : hv / (Hv / Hk);
+        if (!head_map) return hv / (Hv / Hk);
+        const int h = __ldg(head_map + hv);
+        return h < 0 ? 0 : (h >= Hk ? Hk - 1 : h);
     }
     // Element offsets of one token row in the token-major layouts.
     __device__ __forceinline__ long qk_row(int b, int t, int hk) const {

@@ -37,7 +37,8 @@ decode_step_kernel(DecodeParams p) {
     __shared__ float nrm[2];
 
     const int hv = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
-    const int hk = p.head_map ? p.head_map[hv] : hv / (p.Hv / p.Hk);
+    // a map entry outside [0, Hk) breaks the precondition: clamped, so no read leaves q or k
+    const int hk = p.head_map ? min(max(__ldg(p.head_map + hv), 0), p.Hk - 1) : hv / (p.Hv / p.Hk);
     const TIn* q = static_cast<const TIn*>(p.q) + ((long)n * p.Hk + hk) * DK;
     const TIn* k = static_cast<const TIn*>(p.k) + ((long)n * p.Hk + hk) * DK;
     const TIn* v = static_cast<const TIn*>(p.v) + ((long)n * p.Hv + hv) * DV;

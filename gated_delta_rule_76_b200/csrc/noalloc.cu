@@ -1,7 +1,6 @@
 // gdn_chunk_fwd_noalloc: the chunkwise forward with its scratch memory taken from a fixed device
 // array inside this library instead of a caller workspace.  Nothing here allocates memory.
 #include <cstdio>
-#include <mutex>
 
 #include "gdn.h"
 #include "launch.h"
@@ -19,28 +18,20 @@ namespace {
 constexpr size_t kScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_scratch on the current device, resolved once per device (with that device
-// current, as cudaGetSymbolAddress requires).
+// Device address of g_scratch in the current context, looked up on every call with
+// cudaGetSymbolAddress (with the device current, as that call requires).  It is not cached: after a
+// cudaDeviceReset the module is loaded again and the array may sit at another address.  Once the
+// module is loaded the lookup is a host-side table read.
 gdn_status scratch_of_current_device(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return gdn::record_error(GDN_ERR_CUDA, "gdn_chunk_fwd_noalloc: cudaGetDevice failed");
-    if (dev < 0 || dev >= kMaxDevices)
-        return gdn::record_error(GDN_ERR_UNSUPPORTED, "gdn_chunk_fwd_noalloc: device index out of range");
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_scratch);
-        if (e != cudaSuccess || !p)
-            return gdn::record_error(GDN_ERR_CUDA,
-                                     "gdn_chunk_fwd_noalloc: cudaGetSymbolAddress of the scratch array failed");
-        g_scratch_ptr[dev] = p;
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess || !p) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "gdn_chunk_fwd_noalloc: cudaGetSymbolAddress of the scratch array failed (%s)",
+                 cudaGetErrorName(e));
+        return gdn::record_error(GDN_ERR_CUDA, msg);
     }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return GDN_OK;
 }
 

@@ -6,6 +6,9 @@
 //                    D2 = A * B2^T      (A from tensor memory, B2 128x128).
 //  gdn_selftest_mma_mn: MN-major operands (a token-major tile read with M or N = channel):
 //                    D1 = Ak X, D2 = X^T B2^T, D3 = Ak X with Ak in tensor memory.
+//  gdn_selftest_wait_expiry: the tensor-core kernels' failure path (their bounded wait, the error
+//                    word and the release of tensor memory) driven by a barrier that nothing
+//                    arrives at, with a short limit.
 //  gdn_selftest_tma: one 4-D TMA box (64 channels x 1 head x 64 tokens x 1 batch, 128-byte
 //                    swizzle) of a [B,T,H,D] bf16 tensor copied to shared memory and read back
 //                    through sw128_offset(); tokens past T must read as zero.
@@ -16,6 +19,7 @@
 #include <stdint.h>
 
 #include "../umma.cuh"
+#include "../tc_chunk_fwd.cuh"
 
 using namespace gdn::tc;
 
@@ -246,6 +250,49 @@ typedef CUresult (*EncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, v
                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The failure path of the tensor-core kernels on a barrier that completes only if `arrive`:
+// thread 0 waits on it with the kernels' own bounded wait (gdn::tcfwd::wait1) and the given limit
+// while the other threads hold tensor memory, as a kernel's roles do.  On expiry the wait sets the
+// CTA's abort flag and bit 0 of *status (a workspace status word); every thread then sees the
+// abort, and the CTA releases its tensor memory and returns.  out[0] = 1 if the wait succeeded,
+// out[1] = number of threads that saw the abort flag.
+__global__ void __launch_bounds__(128) wait_expiry_selftest_kernel(int* status, int* out, unsigned long long limit_ns,
+                                                                   int arrive) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    __shared__ uint32_t tbase;
+    __shared__ int seen;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    gdn::tcfwd::Ctx cx;
+    cx.sm = nullptr;
+    cx.bars = &bar;
+    cx.abort_flag = reinterpret_cast<volatile int*>(&abort_flag);
+    cx.err = status;
+    cx.wait_ns = limit_ns;
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        seen = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&tbase, 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (arrive && tid == 32) mbar_arrive(&bar);
+    if (tid == 0) out[0] = gdn::tcfwd::wait1(cx, 0, 0) ? 1 : 0;
+    __syncthreads();
+    if (*cx.abort_flag) atomicAdd(&seen, 1);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) out[1] = seen;
+    if (warp == 0) tmem_dealloc(tbase, 32);
+}
+
 }  // namespace
 
 SELFTEST_API int gdn_selftest_mma(const void* A, const void* B1, const void* A2, const void* B3,
@@ -290,5 +337,12 @@ SELFTEST_API int gdn_selftest_tma(const void* x, int B, int T, int H, int c0, in
     if (r != CUDA_SUCCESS) return 2000 + (int)r;
     const size_t smem = 8192 + 1024;
     tma_selftest_kernel<<<1, 128, smem, (cudaStream_t)stream>>>(map, c0, hh, t0, bb, (__nv_bfloat16*)out, err);
+    return (int)cudaGetLastError();
+}
+
+// status: a workspace status word (device int); out: 2 device ints.
+SELFTEST_API int gdn_selftest_wait_expiry(int* status, int* out, unsigned long long limit_ns, int arrive,
+                                          void* stream) {
+    wait_expiry_selftest_kernel<<<1, 128, 0, (cudaStream_t)stream>>>(status, out, limit_ns, arrive);
     return (int)cudaGetLastError();
 }

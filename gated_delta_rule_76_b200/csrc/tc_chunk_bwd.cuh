@@ -136,6 +136,7 @@ struct Params {
     __nv_bfloat16* ny_hi;  // [B,T,Hv,dv]: -dY of every token, hi / lo
     __nv_bfloat16* ny_lo;
     int* err;
+    uint64_t wait_ns;      // limit of every bounded wait; 0 = kWaitNs
 };
 
 
@@ -189,6 +190,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_BAR + 128);
     cx.abort_flag = reinterpret_cast<volatile int*>(sm + SM_BAR + 132);
     cx.err = p.err;
+    cx.wait_ns = p.wait_ns ? p.wait_ns : kWaitNs;
     float* gam = reinterpret_cast<float*>(sm + SM_GAM);
 
     const Problem& pb = p.pb;
@@ -706,11 +708,11 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (*cx.abort_flag) {
         const uint64_t t0 = globaltimer_ns();
         if (tid == 0 && do_issued > 0)
-            while (!mbar_try_wait(cx.bars + B_DO, (uint32_t)((do_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+            while (!mbar_try_wait(cx.bars + B_DO, (uint32_t)((do_issued - 1) & 1)) && globaltimer_ns() - t0 < cx.wait_ns) {
             }
         if (tid == 0 && raw_issued > 0)
             while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) &&
-                   globaltimer_ns() - t0 < kWaitNs) {
+                   globaltimer_ns() - t0 < cx.wait_ns) {
             }
     }
     __syncthreads();
@@ -789,6 +791,7 @@ struct Params {
     float* dw;
     int direct;          // dq, dk written per key head (no head sharing)
     int* err;
+    uint64_t wait_ns;    // limit of every bounded wait; 0 = kWaitNs
 };
 
 struct ChunkPos {
@@ -1284,6 +1287,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     cx.abort_flag = reinterpret_cast<volatile int*>(sm + SM_BAR + 132);
     volatile int* stop_slot = reinterpret_cast<volatile int*>(sm + SM_BAR + 136);
     cx.err = p.err;
+    cx.wait_ns = p.wait_ns ? p.wait_ns : kWaitNs;
     float* xslot = reinterpret_cast<float*>(sm + SM_XSLOT);
     float* gslot = reinterpret_cast<float*>(sm + SM_GSLOT);
     float* scr = reinterpret_cast<float*>(sm + SM_GL);
@@ -1465,10 +1469,10 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (*cx.abort_flag && (tid == 0 || tid == 128)) {
         const uint64_t tw = globaltimer_ns();
         if (raw_issued > 0)
-            while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - tw < kWaitNs) {
+            while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - tw < cx.wait_ns) {
             }
         if (gv_issued > 0)
-            while (!mbar_try_wait(cx.bars + B_GV, (uint32_t)((gv_issued - 1) & 1)) && globaltimer_ns() - tw < kWaitNs) {
+            while (!mbar_try_wait(cx.bars + B_GV, (uint32_t)((gv_issued - 1) & 1)) && globaltimer_ns() - tw < cx.wait_ns) {
             }
     }
     __syncthreads();

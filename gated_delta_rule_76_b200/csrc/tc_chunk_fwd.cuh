@@ -125,6 +125,7 @@ struct Params {
     int o_type;  // 0: bf16, 1: fp32
     float* ht;
     int* err;    // device error word (bit 0: a bounded wait expired)
+    uint64_t wait_ns;  // limit of every bounded wait; 0 = kWaitNs
     // Backward support (all NULL in a plain forward).  o may be NULL then: no output is formed.
     float* s0_out;               // [B*Hv][NT + 1][dv/4][dk][4] fp32: the state entering every chunk, then
                                  //   the final state
@@ -218,17 +219,18 @@ struct Ctx {
     uint64_t* bars;
     volatile int* abort_flag;
     int* err;
+    uint64_t wait_ns;  // limit of one bounded wait (kWaitNs unless a caller asks for another)
 };
 
 // Bounded wait by a single thread (the others sleep in a named barrier meanwhile).  Polls sleep in
-// hardware between attempts; gives up when another thread has aborted or after kWaitNs.
+// hardware between attempts; gives up when another thread has aborted or after cx.wait_ns.
 __device__ __forceinline__ bool wait1(const Ctx& cx, int bar, uint32_t parity) {
     uint64_t* b = cx.bars + bar;
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_sleep(b, parity, 1000u)) {
         if (*cx.abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitNs) {
+        if (globaltimer_ns() - t0 > cx.wait_ns) {
             *cx.abort_flag = 1;
             atomicOr(cx.err, 1);
             return false;
@@ -325,6 +327,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SM_BAR + 128);
     cx.abort_flag = reinterpret_cast<volatile int*>(sm + SM_BAR + 132);
     cx.err = p.err;
+    cx.wait_ns = p.wait_ns ? p.wait_ns : kWaitNs;
     float* gam = reinterpret_cast<float*>(sm + SM_GAM);
 
     const Problem& pb = p.pb;
@@ -939,12 +942,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (*cx.abort_flag && tid == 0) {
         // thread 0 issued every load; the last one of each stage completes phase (issued - 1)
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(cx.bars + B_VW, (uint32_t)((vw_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+        while (!mbar_try_wait(cx.bars + B_VW, (uint32_t)((vw_issued - 1) & 1)) && globaltimer_ns() - t0 < cx.wait_ns) {
         }
-        while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - t0 < kWaitNs) {
+        while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) && globaltimer_ns() - t0 < cx.wait_ns) {
         }
         while (z_issued > 0 && !mbar_try_wait(cx.bars + B_Z, (uint32_t)((z_issued - 1) & 1)) &&
-               globaltimer_ns() - t0 < kWaitNs) {
+               globaltimer_ns() - t0 < cx.wait_ns) {
         }
     }
     __syncthreads();

@@ -185,11 +185,18 @@ def _gates(alpha, b, w, beta):
     return b, w, 1
 
 
-def _head_map(head_map, device):
+def _head_map(head_map, device, Hk: int):
+    """The value-head -> key-head map as an int32 device array.  A map given on the host (a list
+    or a CPU tensor) is checked before it is uploaded: every entry must be in [0, Hk).  A map
+    already on the device is passed through unchecked (checking it would synchronise)."""
     if head_map is None:
         return None
     if not torch.is_tensor(head_map):
         head_map = torch.tensor(head_map, dtype=torch.int32)
+    if head_map.device.type == "cpu" and head_map.numel():
+        lo, hi = int(head_map.min()), int(head_map.max())
+        if lo < 0 or hi >= Hk:
+            raise GdnError(f"head_map entries must be in [0, {Hk}); got [{lo}, {hi}]")
     return head_map.to(device=device, dtype=torch.int32).contiguous()
 
 
@@ -202,7 +209,7 @@ def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_ma
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
-    hm = _head_map(head_map, q.device)
+    hm = _head_map(head_map, q.device, q.shape[-2])
     a = FwdArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
                 h0=_ptr(h0), z=_ptr(z), o=_ptr(o), ht=_ptr(ht), head_map=_ptr(hm),
                 B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
@@ -268,7 +275,7 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
-    hm = _head_map(head_map, q.device)
+    hm = _head_map(head_map, q.device, q.shape[-2])
     g = grads
     a = BwdArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
                 h0=_ptr(h0), head_map=_ptr(hm), grad_o=_ptr(grad_o), grad_ht=_ptr(grad_ht),
@@ -318,7 +325,7 @@ def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=N
     Hv, dv = v.shape[1], v.shape[2]
     if o is None:
         o = torch.empty((N, Hv, dv), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
-    hm = _head_map(head_map, q.device)
+    hm = _head_map(head_map, q.device, q.shape[-2])
     a = DecodeArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
                    state=_ptr(state), o=_ptr(o), head_map=_ptr(hm), conv_state=_ptr(conv_state),
                    conv_w=_ptr(conv_w), z=_ptr(z), N=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
@@ -334,7 +341,7 @@ def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
-    hm = _head_map(head_map, xq.device)
+    hm = _head_map(head_map, xq.device, xq.shape[-2])
     a = LayerArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
                   b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
                   conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
@@ -399,7 +406,7 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
     else:
         out["dbeta"] = torch.empty(tuple(bb.shape), **f32)
         gb, gw = out["dbeta"], None
-    hm = _head_map(head_map, dev)
+    hm = _head_map(head_map, dev, Hk)
     a = LayerBwdArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
                      b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), head_map=_ptr(hm), grad_y=_ptr(grad_y),
                      grad_ht=_ptr(grad_ht), grad_xq=_ptr(out["dxq"]), grad_xk=_ptr(out["dxk"]),

@@ -28,7 +28,10 @@
  *  - Layouts: token-major.  q, k: [B,T,Hk,dk]; v, o, z: [B,T,Hv,dv]; channel gates alpha, b:
  *    [B,T,Hv,dk], w: [B,T,Hv,dv]; scalar gates alpha, beta: [B,T,Hv]; states: [B,Hv,dk,dv] fp32.
  *  - GQA: value head hv reads key head head_map[hv] (int32 device array of Hv entries).  NULL
- *    means contiguous groups hv / (Hv / Hk) (Hv must then be a multiple of Hk).  Several value
+ *    means contiguous groups hv / (Hv / Hk) (Hv must then be a multiple of Hk).  Every entry
+ *    must lie in [0, Hk); the map lives on the device, so the host cannot check it: kernels clamp
+ *    an entry outside that range into it (no read falls outside q or k) and the results are then
+ *    unspecified.  The Python binding checks the map before uploading it.  Several value
  *    heads share each key head in the 16-key / 128-value layer of the mkdocs chapter «Gated
  *    DeltaNet», «Les projections d'entrée».
  *  - Sizes: dk, dv in {64, 128}; B, T, Hk, Hv >= 1 (T = 0 is accepted and does nothing but copy
@@ -122,9 +125,10 @@ GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size
  *  - Limit: a problem whose gdn_chunk_fwd_workspace_size() exceeds 16 MiB is rejected with
  *    GDN_ERR_WORKSPACE before anything is launched (the tensor-core path needs 256 bytes, so
  *    bf16 problems with dk = dv = 128 always fit; the CUDA-core path needs per-chunk factors).
- *  - Set-up: the first call on a device resolves the array's address on that (current) device
- *    with cudaGetSymbolAddress, which may load the library's device code; make the first call on
- *    each device before any stream capture.  Later calls only launch work on `stream`.
+ *  - Set-up: every call looks up the array's address on the current device with
+ *    cudaGetSymbolAddress (so a device reset between calls is harmless).  The first call on a
+ *    device may load the library's device code there; make it before any stream capture.  Later
+ *    lookups are host-side; each call then launches work on `stream` only.
  *  - Nothing is allocated (no cudaMalloc, no host or device allocation by any library).  The
  *    status word at the start of the scratch is cleared on `stream` at the start of every call;
  *    nothing else in the scratch needs to start at zero.  The status word is not readable by the

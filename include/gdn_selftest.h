@@ -30,6 +30,14 @@ int gdn_selftest_mma_mn(const void* Ak, const void* X, const void* B2, float* D1
 int gdn_selftest_tma(const void* x, int B, int T, int H, int c0, int hh, int t0, int bb, void* out,
                      int* err, void* stream);
 
+/* The tensor-core kernels' failure path: thread 0 of one 128-thread CTA holding tensor memory
+ * waits on an mbarrier with the kernels' bounded wait and a limit of limit_ns; the barrier
+ * completes only if `arrive` is non-zero.  On expiry bit 0 of *status is set (status is meant to
+ * be the first word of a libgdn workspace, so that gdn_workspace_status reports it), every
+ * thread sees the CTA's abort flag, and the CTA releases its tensor memory and returns.
+ * out[0] = 1 if the wait succeeded, else 0; out[1] = number of threads that saw the abort. */
+int gdn_selftest_wait_expiry(int* status, int* out, unsigned long long limit_ns, int arrive, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

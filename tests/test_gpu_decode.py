@@ -49,8 +49,11 @@ def test_decode_steps_match_oracle(N, Hk, Hv, d, apc, gpc, dtype, gdt):
     assert_parity(state, ref_state, kind, "state")
 
 
-def test_decode_with_conv_and_swish_gate():
-    N, Hk, Hv, d, steps = 3, 2, 4, 64, 5
+@pytest.mark.parametrize("N,Hk,Hv,d,steps", [
+    (3, 2, 4, 64, 5),
+    (8, 2, 16, 128, 8),  # the layer's head width and an 8-value-head group per key head
+])
+def test_decode_with_conv_and_swish_gate(N, Hk, Hv, d, steps):
     cch = 2 * Hk * d + Hv * d
     x = draw(N, steps, Hk, Hv, d, d, alpha_per_channel=True, gates_per_channel=True, dtype="bf16",
              gate_dtype="bf16", seed=21, has_h0=True, conv=True, swish_gate=True)

@@ -219,3 +219,12 @@ def test_layer_backward_workspace(lib):
     assert lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(_layer_bwd(T=65))) > need
     assert lib.gdn_layer_core_bwd(ctypes.byref(a), ctypes.c_void_p(1 << 34), need - 1, None) == 4
     assert lib.gdn_layer_core_bwd(None, None, 0, None) == 1
+
+
+def test_binding_checks_a_host_head_map():
+    """Entries outside [0, Hk) are refused before the map is uploaded (the kernels only clamp)."""
+    from gated_delta_rule_76_b200 import gdn
+    assert gdn._head_map([0, 1, 1, 0], "cpu", 2).tolist() == [0, 1, 1, 0]
+    for bad in ([0, 2], [-1, 0]):
+        with pytest.raises(gdn.GdnError):
+            gdn._head_map(bad, "cpu", 2)
