@@ -142,6 +142,8 @@ WsPlan plan_chunk_ws(const Problem& pb, bool bwd, bool gqa_partials) {
     const size_t part = (size_t)pb.B * pb.T * pb.Hv * dk;
     w.dq_v = (bwd && gqa_partials) ? take(part) : none;
     w.dk_v = (bwd && gqa_partials) ? take(part) : none;
+    w.flags = take((size_t)pb.B * pb.Hv);  // ints: pairs outside the decay range
+    w.sbuf = bwd ? take(seq_sbuf_floats(pb)) : none;
     w.bytes = off;
     return w;
 }
@@ -155,6 +157,8 @@ ChunkWs carve_chunk_ws(const WsPlan& w, void* base) {
     ws.Kt = at(w.Kt); ws.Gm = at(w.Gm); ws.gam = at(w.gam); ws.S0 = at(w.S0); ws.dSC = at(w.dSC);
     ws.V = at(w.V); ws.Y = at(w.Y); ws.dV = at(w.dV); ws.dY = at(w.dY); ws.dbw = at(w.dbw);
     ws.dq_v = at(w.dq_v); ws.dk_v = at(w.dk_v);
+    ws.flags = reinterpret_cast<int*>(at(w.flags));
+    ws.sbuf = at(w.sbuf);
     return ws;
 }
 
@@ -253,6 +257,15 @@ ChunkIO io_from(const gdn_fwd_args* a) {
 // Status word at the start of every workspace, cleared at the start of each call.
 int* ws_status(void* ws) { return static_cast<int*>(ws); }
 
+// The flag array of the pairs outside the chunk form's decay range, cleared at the start of a call.
+cudaError_t clear_flags(int* flags, const Problem& pb, cudaStream_t st) {
+    return cudaMemsetAsync(flags, 0, (size_t)pb.B * pb.Hv * sizeof(int), st);
+}
+
+// The tensor-core forward's workspace: the status word, then the flag array.
+size_t tc_fwd_ws_bytes(const Problem& pb) { return 256 + align256((size_t)pb.B * pb.Hv * sizeof(int)); }
+int* tc_fwd_flags(void* ws) { return reinterpret_cast<int*>(static_cast<char*>(ws) + 256); }
+
 cudaError_t run_fwd(int var, const Problem& pb, const ChunkIO& io, const ChunkWs& ws, Flags f,
                     cudaStream_t st) {
     switch (var) {
@@ -295,7 +308,7 @@ size_t gdn_chunk_fwd_cache_size(const gdn_fwd_args* a) {
 size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    if (fwd_uses_tensor_cores(a, pb)) return 256;
+    if (fwd_uses_tensor_cores(a, pb)) return tc_fwd_ws_bytes(pb);
     return plan_chunk_ws(pb, false, false).bytes;
 }
 
@@ -317,8 +330,10 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
                         plan_tc_cache(pb).bytes);
     }
     WsPlan plan = plan_chunk_ws(pb, false, false);
-    if ((s = check_workspace(workspace, workspace_bytes, tc ? 256 : plan.bytes))) return s;
+    if ((s = check_workspace(workspace, workspace_bytes, tc ? tc_fwd_ws_bytes(pb) : plan.bytes))) return s;
+    int* flags = tc ? tc_fwd_flags(workspace) : carve_chunk_ws(plan, workspace).flags;
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
+    if (e == cudaSuccess) e = clear_flags(flags, pb, st);
     if (e == cudaSuccess) {
         TcFwdSave save{};
         if (a->bwd_cache) {
@@ -330,7 +345,7 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
         }
         if (tc)
             e = tc_chunk_fwd(pb, io_from(a), f, a->gate_dtype == GDN_BF16, ws_status(workspace), st,
-                             a->bwd_cache ? &save : nullptr);
+                             a->bwd_cache ? &save : nullptr, flags);
         else e = run_fwd(variant(a->dtype, a->gate_dtype), pb, io_from(a), carve_chunk_ws(plan, workspace), f, st);
     }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_fwd");
@@ -374,6 +389,9 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     io.dh0 = a->grad_h0;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
+    if (e == cudaSuccess)
+        e = clear_flags(tc ? reinterpret_cast<int*>(static_cast<char*>(workspace) + tplan.flags)
+                           : carve_chunk_ws(plan, workspace).flags, pb, st);
     if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_bwd");
     if (tc) {
         e = tc_chunk_bwd(pb, io, f, a->gate_dtype == GDN_BF16, direct, tplan, workspace, a->fwd_cache, st);
@@ -525,11 +543,15 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     }
     const size_t need = gdn_layer_core_fwd_workspace_size(a);
     if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
-    cudaError_t e0 = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
-    if (e0 != cudaSuccess) return cuda_fail(e0, "gdn_layer_core_fwd");
     char* base = static_cast<char*>(workspace) + 256;
     const size_t conv_bytes = align256(BT * cch * 4);
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    // the chunk part of the workspace (after the conv results) holds the flag array in both forms
+    const WsPlan chunk_plan = plan_chunk_ws(pb, false, false);
+    int* flags = carve_chunk_ws(chunk_plan, base + conv_bytes).flags;
+    cudaError_t e0 = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
+    if (e0 == cudaSuccess) e0 = clear_flags(flags, pb, sm);
+    if (e0 != cudaSuccess) return cuda_fail(e0, "gdn_layer_core_fwd");
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
     // The conv outputs are fp32 values.  With scalar gates and bf16 tensors they go to the
     // tensor-core forward as bf16 hi/lo pairs (same bytes); otherwise they stay fp32 for the
@@ -569,13 +591,12 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
             char* cb = cache + lc.tc;
             const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
                                  reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo), reinterpret_cast<float*>(cache + lc.o)};
-            e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, &save);
+            e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, &save, flags);
         } else {
-            e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm);
+            e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, nullptr, flags);
         }
     } else {
-        WsPlan plan = plan_chunk_ws(pb, false, false);
-        e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(plan, base + conv_bytes), f, sm);
+        e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(chunk_plan, base + conv_bytes), f, sm);
     }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_fwd");
 }
@@ -693,10 +714,15 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
     char* wsb = static_cast<char*>(workspace);
     auto at = [&](size_t o) { return reinterpret_cast<float*>(wsb + o); };
-    cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
-    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd");
     const bool bf16 = a->dtype == GDN_BF16, bf16g = a->gate_dtype == GDN_BF16;
     const bool direct = identity_heads(pb);
+    // the flag array of the pairs outside the decay range: in the tensor-core backward's workspace
+    // (at offset 0) or in the CUDA-core chunk workspace
+    int* flags = plan.tc ? reinterpret_cast<int*>(wsb + plan_tc_bwd_ws(pb, !direct, true).flags)
+                         : carve_chunk_ws(plan_chunk_ws(pb, true, !direct), wsb + plan.chunk).flags;
+    cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
+    if (e == cudaSuccess) e = clear_flags(flags, pb, sm);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd");
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
     ConvParams cp{};
     cp.xq = a->xq; cp.xk = a->xk; cp.xv = a->xv; cp.conv_w = a->conv_w;
@@ -734,7 +760,7 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
             const TcCache cc = plan_tc_cache(pb);
             const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
                                  reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo), nullptr};
-            e = tc_chunk_fwd(pb, io, f, bf16g, ws_status(workspace), sm, &save);
+            e = tc_chunk_fwd(pb, io, f, bf16g, ws_status(workspace), sm, &save, flags);
             if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
         }
         // 3. swish gate; the gradient of o as bf16 hi/lo pairs (tensor-core operands)

@@ -1,5 +1,7 @@
 // Templated launchers, instantiated once per (tensor dtype, gate dtype) in inst_*.cu.
 #pragma once
+#include <type_traits>
+
 #include "launch.h"
 
 namespace gdn {
@@ -40,12 +42,17 @@ cudaError_t chunk_fwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
                           block, chunk_prep_smem<DK>(), st, pb, io, ws, save_states ? 1 : 0));
     const dim3 sgrid(pb.dv / kDvTileFwd, pb.Hv, pb.B);
     if (gate)
-        return launch_kernel(chunk_scan_fwd_kernel<TIn, TG, GPC, DK, true>, sgrid, block,
-                             chunk_scan_fwd_smem<DK>(), st, pb, io, ws, write_out ? 1 : 0,
-                             save_states ? 1 : 0);
-    return launch_kernel(chunk_scan_fwd_kernel<TIn, TG, GPC, DK, false>, sgrid, block,
-                         chunk_scan_fwd_smem<DK>(), st, pb, io, ws, write_out ? 1 : 0,
-                         save_states ? 1 : 0);
+        GDN_TRY(launch_kernel(chunk_scan_fwd_kernel<TIn, TG, GPC, DK, true>, sgrid, block,
+                              chunk_scan_fwd_smem<DK>(), st, pb, io, ws, write_out ? 1 : 0,
+                              save_states ? 1 : 0));
+    else
+        GDN_TRY(launch_kernel(chunk_scan_fwd_kernel<TIn, TG, GPC, DK, false>, sgrid, block,
+                              chunk_scan_fwd_smem<DK>(), st, pb, io, ws, write_out ? 1 : 0,
+                              save_states ? 1 : 0));
+    // pairs whose decay left the factors' range (marked by prep): their outputs again, exactly
+    if (!ws.flags || !write_out) return cudaSuccess;
+    return seq_fwd(pb, io, Flags{APC, GPC, gate}, std::is_same<TIn, float>::value, std::is_same<TG, float>::value,
+                   ws.flags, nullptr, st);
 }
 
 template <class TIn, class TG, bool APC, bool GPC, int DK>
@@ -57,6 +64,13 @@ cudaError_t chunk_bwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
                           block, chunk_scan_bwd_smem<DK>(), st, pb, io, ws));
     GDN_TRY(launch_kernel(chunk_grad_kernel<TIn, TG, APC, GPC, DK, DK>, dim3(pb.NT, pb.Hv, pb.B),
                           block, chunk_grad_smem<DK, DK>(), st, pb, io, ws, direct_qk ? 1 : 0));
+    // pairs whose decay left the factors' range (marked by prep): every gradient again, exactly;
+    // the pair's slice of the chunk-state array holds its checkpoints
+    if (ws.flags && ws.sbuf)
+        GDN_TRY(seq_bwd(pb, io, Flags{APC, GPC, false}, std::is_same<TIn, float>::value, std::is_same<TG, float>::value,
+                        ws.flags, direct_qk ? static_cast<float*>(io.dq) : ws.dq_v,
+                        direct_qk ? static_cast<float*>(io.dk) : ws.dk_v, direct_qk, ws.S0,
+                        (long)pb.NT * DK * DK, ws.sbuf, st));
     if (!direct_qk) {
         GDN_TRY(gqa_reduce(pb, (const float*)ws.dq_v, static_cast<float*>(io.dq), st));
         GDN_TRY(gqa_reduce(pb, (const float*)ws.dk_v, static_cast<float*>(io.dk), st));

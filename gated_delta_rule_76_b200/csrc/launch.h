@@ -28,6 +28,7 @@ struct Flags {
 struct WsPlan {
     size_t bytes = 0;
     size_t T, P, Eh, Qh, Kb, Kt, Gm, gam, S0, dSC, V, Y, dV, dY, dbw, dq_v, dk_v;
+    size_t flags, sbuf;  // pairs outside the chunk form's decay range; the sequential backward's states
 };
 WsPlan plan_chunk_ws(const Problem& pb, bool bwd, bool gqa_partials);
 ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
@@ -50,8 +51,20 @@ struct TcFwdSave {
     float* o_raw;            // with the swish gate, may be NULL: the output before the gate (fp32)
 };
 bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags f);
+// flags: [B*Hv] ints, zero on entry (or NULL): the kernel marks the pairs whose decay leaves the
+// chunk form's range, and the exact sequential kernel then recomputes their outputs.
 cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
-                         cudaStream_t st, const TcFwdSave* save = nullptr);
+                         cudaStream_t st, const TcFwdSave* save = nullptr, int* flags = nullptr);
+
+// Exact sequential recurrence (seq.cu) for the pairs marked in flags: the forward (o, the output
+// before the gate, ht) and the backward (every gradient; ck: per pair ck_stride floats for the
+// states entering chunks 1..NT-1, sbuf: seq_sbuf_floats()).  dq, dk are per key head when direct,
+// else per value head.
+size_t seq_sbuf_floats(const Problem& pb);
+cudaError_t seq_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
+                    float* o_raw, cudaStream_t st);
+cudaError_t seq_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
+                    float* dq, float* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st);
 
 // Tensor-core chunk backward (tc_bwd.cu): same eligibility as the forward, without z.
 // The forward cache (what the backward needs from the forward): byte offsets from its start.
@@ -64,6 +77,7 @@ struct TcBwdWs {
     size_t bytes = 0;  // total, including the 256-byte status word at offset 0
     size_t cache;      // a forward cache inside the workspace (~0 when the caller passes one)
     size_t dsc, ny_hi, ny_lo, dq_v, dk_v;  // byte offsets (dq_v, dk_v: GQA only)
+    size_t flags, sbuf;                    // pairs outside the decay range; sequential backward states
 };
 TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials, bool caller_cache);
 // cache: the caller's forward cache (the forward is not recomputed), or NULL.

@@ -19,6 +19,7 @@
 #pragma once
 #include "block_gemm.cuh"
 #include "common.cuh"
+#include "seq.cuh"
 
 namespace gdn {
 
@@ -45,6 +46,8 @@ struct ChunkWs {
     float *V, *Y, *dV, *dY;                       // per chunk [C][dv] intermediates (backward)
     float* dbw;                                   // [BH][NT][dv/32][C] scalar-beta partials
     float *dq_v, *dk_v;                           // [B,T,Hv,dk] per value head (GQA)
+    int* flags;                                   // [B*Hv]: pairs outside the decay range (seq.cuh)
+    float* sbuf;                                  // the sequential backward's states (seq.cuh)
 };
 
 struct ChunkIO {
@@ -118,6 +121,8 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
             }
         }
         ws.gam[ci * DK + c] = G;
+        // a chunk product below the factors' range: the pair goes to the sequential kernels
+        if (ws.flags && seq::decay_out_of_range(G)) ws.flags[(long)b * pb.Hv + hv] = 1;
         for (int r = 0; r < C; ++r) {
             ws.Eh[(ci * C + r) * DK + c] = Eh[r * LD + c];
             ws.Qh[(ci * C + r) * DK + c] = Qh[r * LD + c];

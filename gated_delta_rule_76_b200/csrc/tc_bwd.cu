@@ -1,6 +1,8 @@
 // Host side of the tensor-core chunk backward: workspace plan, TMA descriptors, launches.
 // One call runs the forward kernel in saving mode, the reverse state-gradient scan, the
-// chunk-parallel gradient kernel and, when value heads share key heads, the GQA reduction.
+// chunk-parallel gradient kernel, the exact sequential backward for the pairs outside the decay
+// range (a launch that returns at once for the others) and, when value heads share key heads, the
+// GQA reduction.
 #include <cuda.h>
 
 #include "launch.cuh"
@@ -86,6 +88,8 @@ TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials, bool caller_cache) 
     w.ny_lo = take(tok);
     w.dq_v = gqa_partials ? take(part) : ~size_t(0);
     w.dk_v = gqa_partials ? take(part) : ~size_t(0);
+    w.flags = take((size_t)pb.B * pb.Hv * sizeof(int));
+    w.sbuf = take(seq_sbuf_floats(pb) * sizeof(float));
     w.bytes = off;
     return w;
 }
@@ -104,6 +108,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     auto* nyl = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_lo);
     float* dq_v = direct ? static_cast<float*>(io.dq) : reinterpret_cast<float*>(base + plan.dq_v);
     float* dk_v = direct ? static_cast<float*>(io.dk) : reinterpret_cast<float*>(base + plan.dk_v);
+    int* flags = reinterpret_cast<int*>(base + plan.flags);  // zeroed by the caller
 
     const bool split = io.q_lo != nullptr;
     if (split && (f.apc || f.gpc || !io.k_lo || !io.v_lo)) return cudaErrorInvalidValue;
@@ -117,7 +122,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
         Flags ff = f;
         ff.gate = false;
         const TcFwdSave save{s0, vph, vpl};
-        e = tc_chunk_fwd(pb, fio, ff, bf16_gates, err, st, &save);
+        e = tc_chunk_fwd(pb, fio, ff, bf16_gates, err, st, &save, flags);
         if (e != cudaSuccess) return e;
     }
 
@@ -146,6 +151,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     sp.ny_hi = nyh;
     sp.ny_lo = nyl;
     sp.err = err;
+    sp.flags = flags;
 
     tcbwd::grad::Params gp{};
     gp.pb = pb;
@@ -176,9 +182,14 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     else if (f.gpc) e = launch_both<false, true, __nv_bfloat16>(ms, sp, m, gp, st);
     else if (bf16_gates) e = launch_both<false, false, __nv_bfloat16>(ms, sp, m, gp, st);
     else e = launch_both<false, false, float>(ms, sp, m, gp, st);
+    if (e != cudaSuccess) return e;
+    // 3. pairs whose decay left the factors' range (marked by the scan): every gradient again,
+    //    exactly; the pair's slice of the dS array holds its checkpoints
+    e = seq_bwd(pb, io, f, false, !bf16_gates, flags, dq_v, dk_v, direct, dsc, (long)pb.NT * pb.dk * pb.dv,
+                reinterpret_cast<float*>(base + plan.sbuf), st);
     if (e != cudaSuccess || direct) return e;
 
-    // 3. GQA: sum the per-value-head dq, dk over the value heads of each key head
+    // 4. GQA: sum the per-value-head dq, dk over the value heads of each key head
     GDN_TRY(gqa_reduce(pb, (const float*)dq_v, static_cast<float*>(io.dq), st));
     return gqa_reduce(pb, (const float*)dk_v, static_cast<float*>(io.dk), st);
 }

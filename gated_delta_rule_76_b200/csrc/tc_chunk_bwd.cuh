@@ -137,6 +137,7 @@ struct Params {
     __nv_bfloat16* ny_lo;
     int* err;
     uint64_t wait_ns;      // limit of every bounded wait; 0 = kWaitNs
+    int* flags;            // [B*Hv] or NULL: set for a pair with a chunk outside the decay range
 };
 
 
@@ -515,6 +516,12 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float* gs = gam + (i % 3) * 128 + 8 * cg;
                     *reinterpret_cast<float4*>(gs) = make_float4(gm[0], gm[1], gm[2], gm[3]);
                     *reinterpret_cast<float4*>(gs + 4) = make_float4(gm[4], gm[5], gm[6], gm[7]);
+                    if (p.flags) {
+                        bool out = false;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) out |= seq::decay_out_of_range(gm[e]);
+                        if (out) p.flags[blockIdx.x] = 1;  // the pair is recomputed exactly
+                    }
                 }
 #pragma unroll 2
                 for (int u = 0; u < 8; ++u) {

@@ -19,8 +19,9 @@
 // operand x is therefore carried as a pair hi = bf16(x), lo = bf16(x - hi) and the products take
 // the cross terms that matter (hi*hi + lo*hi + hi*lo), each in fp32 in tensor memory:
 //   X1: Ehat, Qhat and Ktil split (3 MMAs);  X2: S0 split, and Qhat split in Qhat S0 (2 + 3 MMAs);
-//   X3: Y split (2);  X4: V' and P split (3);  X5: V' and Kbar split (3).  T stays bf16.
-// This keeps the output within ~0.2% of its RMS of the exact result at the largest entry.
+//   X3: Y and T split (3);  X4: V' and P split (3);  X5: V' and Kbar split (3).
+// T lo shares the fp32 scratch of the solve: the next chunk's A is written there only after X3 of
+// this chunk has completed.
 //
 // Thread j of the two scan warpgroups owns TMEM lane j (= value column j) and keeps its column of
 // the fp32 state in registers, split between the warpgroups by halves of dk.
@@ -43,6 +44,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "seq.cuh"
 #include "umma.cuh"
 
 namespace gdn {
@@ -89,7 +91,8 @@ constexpr uint32_t SM_T = 114688;     // 8 KB [1][64]: T
 constexpr uint32_t SM_P = 122880;     // 16 KB: P hi [1][64], P lo [1][64]
 constexpr uint32_t SM_KB = 139264;    // 32 KB: Kbar^T hi [1][128], Kbar^T lo [1][128]
 constexpr uint32_t SM_VW = 172032;    // 32 KB: v [2][64], w [2][64]
-constexpr uint32_t SM_ASCR = 204800;  // 17 KB: A, then T, fp32 [64][LDA] row-major
+constexpr uint32_t SM_ASCR = 204800;  // 17 KB: A, then T, fp32 [64][LDA] row-major; then T lo
+constexpr uint32_t SM_TLO = SM_ASCR;   // 8 KB [1][64]: T lo (bf16), from the solve until X3 has read it
 constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats (chunk n uses slot n % 3)
 constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, abort flag
 constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: alpha products per row group [8][128], then the
@@ -132,6 +135,7 @@ struct Params {
     __nv_bfloat16* vp_hi;        // [B,T,Hv,dv]: V' = T (Z - Ehat S0) of every token, split
     __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
     float* o_raw;                // GATE only, may be NULL: the output before the gate, fp32 [B,T,Hv,dv]
+    int* flags;                  // [B*Hv] or NULL: set for a pair with a chunk outside the decay range
 };
 
 __device__ __forceinline__ float bf(const uint8_t* tile, uint32_t off) {
@@ -527,6 +531,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     GDN_TRACE(n, 5);
                     mma_ts_u<64, 64>(tbase + TM_X5, tbase + TM_YH, sbase + SM_T, id64, false);
                     mma_ts_u<64, 64>(tbase + TM_X5, tbase + TM_YL, sbase + SM_T, id64, true);
+                    mma_ts_u<64, 64>(tbase + TM_X5, tbase + TM_YH, sbase + SM_TLO, id64, true);
                     mma_commit(cx.bars + B_X3);
                     mma_commit(cx.bars + B_T_FREE);
                     wait1(cx, B_X3, pn);
@@ -773,6 +778,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float* gs = gam + (m % 3) * 128 + 8 * cg;
                     *reinterpret_cast<float4*>(gs) = make_float4(gm[0], gm[1], gm[2], gm[3]);
                     *reinterpret_cast<float4*>(gs + 4) = make_float4(gm[4], gm[5], gm[6], gm[7]);
+                    if (p.flags) {
+                        bool out = false;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) out |= seq::decay_out_of_range(gm[i]);
+                        if (out) p.flags[blockIdx.x] = 1;  // the pair is recomputed exactly
+                    }
                 }
 #pragma unroll 2
                 for (int u = 0; u < 8; ++u) {
@@ -846,6 +857,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 wait1(cx, B_X1, pm);
                 GDN_TRACE(m, 20);
             }
+            // The fp32 scratch holds the previous chunk's T lo until X3 has read it.
+            if (c == 0 && m > 0) wait1(cx, B_T_FREE, pprev);
             named_bar(2, 128);
             tc_fence_after();
             if (c < 64) {
@@ -907,7 +920,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             solve_block_row<2>(ascr, rs, c);
             if (c == 0) GDN_TRACE(m, 30);
             solve_block_row<3>(ascr, rs, c);
-            // (3) T (fp32) -> bf16 K-major tile: thread c converts half c >> 6 of row c & 63.
+            // (3) T (fp32) -> K-major bf16 tiles T hi (SM_T) and T lo (the first 8 KB of the scratch,
+            //     once every thread holds its values): thread c converts half c >> 6 of row c & 63.
             if (c == 0) GDN_TRACE(m, 21);
             if (c == 0 && m > 0) wait1(cx, B_T_FREE, pprev);
             if (c == 0) GDN_TRACE(m, 22);
@@ -915,13 +929,24 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             {
                 const int row = c & 63, col0 = 32 * (c >> 6);
                 uint8_t* Tt = sm + SM_T;
+                uint8_t* Tl = sm + SM_TLO;
+                float tv[32];
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 f = ldf4(ascr + row * LDA + col0 + 4 * q4);
+                    tv[4 * q4] = f.x; tv[4 * q4 + 1] = f.y; tv[4 * q4 + 2] = f.z; tv[4 * q4 + 3] = f.w;
+                }
+                named_bar(2, 128);
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
-                    const float4 f0 = ldf4(ascr + row * LDA + col0 + 8 * q8);
-                    const float4 f1 = ldf4(ascr + row * LDA + col0 + 8 * q8 + 4);
-                    st16(Tt + sw128_offset(row, col0 + 8 * q8, 64),
-                         make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
-                                    pack_bf16x2(f1.z, f1.w)));
+                    uint4 hi, lo;
+                    float x8[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x8[i] = tv[8 * q8 + i];
+                    split8(x8, hi, lo);
+                    const uint32_t off = sw128_offset(row, col0 + 8 * q8, 64);
+                    st16(Tt + off, hi);
+                    st16(Tl + off, lo);
                 }
             }
             fence_async_shared();

@@ -36,8 +36,9 @@ bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags
     return encode_fn() != nullptr;
 }
 
-cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
-                         cudaStream_t st, const TcFwdSave* save) {
+namespace {
+cudaError_t tc_chunk_fwd_kernel(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
+                                cudaStream_t st, const TcFwdSave* save, int* flags) {
     CUtensorMap maps[7];
     const bool split = io.q_lo != nullptr;
     if (split && (f.apc || f.gpc || !io.k_lo || !io.v_lo)) return cudaErrorInvalidValue;
@@ -66,6 +67,7 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     p.o_type = io.o_type == 1 ? 1 : 0;
     p.ht = io.ht;
     p.err = err;
+    p.flags = flags;
     if (save) {
         p.s0_out = save->s0;
         p.vp_hi = save->vp_hi;
@@ -87,6 +89,18 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     if (f.gpc) return launch_tc_g<false, true, __nv_bfloat16>(gate, maps, p, st);
     if (bf16_gates) return launch_tc_g<false, false, __nv_bfloat16>(gate, maps, p, st);
     return launch_tc_g<false, false, float>(gate, maps, p, st);
+}
+}  // namespace
+
+cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf16_gates, int* err,
+                         cudaStream_t st, const TcFwdSave* save, int* flags) {
+    cudaError_t e = tc_chunk_fwd_kernel(pb, io, f, bf16_gates, err, st, save, flags);
+    if (e != cudaSuccess || !flags) return e;
+    // Pairs whose decay left the factors' range: their outputs again, exactly (the backward's
+    // saving-only forward asks for no output, and its backward recomputes such pairs itself).
+    float* o_raw = save ? save->o_raw : nullptr;
+    if (!io.o && !io.ht && !o_raw) return cudaSuccess;
+    return seq_fwd(pb, io, f, false, !bf16_gates, flags, o_raw, st);
 }
 
 }  // namespace gdn

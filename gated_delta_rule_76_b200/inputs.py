@@ -115,11 +115,11 @@ def _l2_rows(x: np.ndarray) -> np.ndarray:
     return out.reshape(x.shape)
 
 
-def _decay(x: np.ndarray) -> np.ndarray:
-    """alpha = exp(-softplus(x) * 0.1), evaluated in float64 (input recipe)."""
+def _decay(x: np.ndarray, scale: float = 0.1) -> np.ndarray:
+    """alpha = exp(-softplus(x) * scale), evaluated in float64 (input recipe: scale 0.1)."""
     x = x.astype(np.float64)
     sp = np.logaddexp(0.0, x)
-    return np.exp(-0.1 * sp)
+    return np.exp(-scale * sp)
 
 
 def _sigmoid(x: np.ndarray) -> np.ndarray:
@@ -132,8 +132,12 @@ def draw(B: int, T: int, Hk: int, Hv: int, dk: int, dv: int, *,
          gate_dtype: Optional[str] = None, seed: int = 0, has_h0: bool = True,
          conv: bool = False, swish_gate: bool = False, with_dout: bool = False,
          with_dht: bool = False, normalise_qk: Optional[bool] = None,
-         erase_scale: float = 1.0) -> Dict[str, object]:
+         erase_scale: float = 1.0, decay_scale: float = 0.1) -> Dict[str, object]:
     """Draw one batch of chunkwise-forward/backward inputs.
+
+    decay_scale replaces the recipe's 0.1 in alpha = exp(-softplus(x) * 0.1): larger values give
+    fast-forgetting gates (3 puts the typical alpha near 0.1 and the smallest near 1e-3), the range
+    where a chunk's decay product leaves the chunk kernels' factorised range.
 
     erase_scale multiplies the erase gate b (or the scalar beta): 2 gives the negative-eigenvalue
     range b, beta in [0, 2] of the explainer's «Réunir les deux» note (the transition's eigenvalue
@@ -160,7 +164,7 @@ def draw(B: int, T: int, Hk: int, Hv: int, dk: int, dv: int, *,
     del q, k
     out["v"] = _cast(_normal(rng, (B, T, Hv, dv)), dtype)
     a_shape = (B, T, Hv, dk) if alpha_per_channel else (B, T, Hv)
-    out["alpha"] = _cast(_decay(_normal(rng, a_shape)), gate_dtype)
+    out["alpha"] = _cast(_decay(_normal(rng, a_shape), decay_scale), gate_dtype)
     if gates_per_channel:
         out["b"] = _cast(erase_scale * _sigmoid(_normal(rng, (B, T, Hv, dk))), gate_dtype)
         out["w"] = _cast(_sigmoid(_normal(rng, (B, T, Hv, dv))), gate_dtype)

@@ -39,10 +39,13 @@
  *  - Dtypes: q, k, v, o, z in `dtype`; alpha, b, w, beta in `gate_dtype`; states and every
  *    gradient are fp32 (gradients leave the fp32 accumulators unrounded: several of them are
  *    heavy-tailed, and a bf16 store alone would cost up to half an ulp of their largest entry).
- *  - Range: the chunked kernels factor the decay as exp(g_r) * exp(-g_s) inside a chunk of 64
- *    tokens (g = cumulative log alpha).  The product of alpha over one chunk must stay above
- *    1e-30 per channel, otherwise the factors overflow and the result is NaN/Inf (never a
- *    silently clamped number).  The single-token decode step has no such limit.
+ *  - Range: every alpha in [0, 1] is supported.  The chunked kernels carry the decay inside a
+ *    chunk of 64 tokens as a ratio Gamma_r / Gamma_s of running products of alpha, which fp32
+ *    holds while the product over a chunk stays at or above 2^-100 (~7.9e-31) on every channel.
+ *    Each chunk kernel checks that bound on every chunk; a (sequence, head) pair with a chunk
+ *    below it is recomputed by an exact sequential kernel in the same call (token by token, no
+ *    ratio of decays), which overwrites that pair's results.  Such pairs cost several times more
+ *    than the chunk form.  The single-token decode step has no ratio and no such bound.
  *  - Errors: every call returns a gdn_status.  Invalid arguments are detected on the host before
  *    any launch and nothing is written.  gdn_last_error() returns a thread-local message about
  *    the last failure of the calling thread.  No C++ exception crosses this interface.
@@ -123,8 +126,9 @@ GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size
  * validation and errors are those of gdn_chunk_fwd; the scratch memory is a fixed 16 MiB device
  * array inside the library (one per device), used as gdn_chunk_fwd's workspace.
  *  - Limit: a problem whose gdn_chunk_fwd_workspace_size() exceeds 16 MiB is rejected with
- *    GDN_ERR_WORKSPACE before anything is launched (the tensor-core path needs 256 bytes, so
- *    bf16 problems with dk = dv = 128 always fit; the CUDA-core path needs per-chunk factors).
+ *    GDN_ERR_WORKSPACE before anything is launched (the tensor-core path needs 256 bytes plus
+ *    4 bytes per (sequence, value head), so bf16 problems with dk = dv = 128 fit up to ~4 million
+ *    pairs; the CUDA-core path needs per-chunk factors).
  *  - Set-up: every call looks up the array's address on the current device with
  *    cudaGetSymbolAddress (so a device reset between calls is harmless).  The first call on a
  *    device may load the library's device code there; make it before any stream capture.  Later
