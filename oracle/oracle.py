@@ -198,6 +198,41 @@ def chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
     return o, hT
 
 
+def segment_map(q, k, v, alpha, b=None, w=None, beta=None, head_map=None):
+    """The affine map by which one segment of a sequence acts on the state.
+
+    For the state S_in entering the segment, the state after it is M S_in + N (per (batch, value
+    head)), because each token's update is affine in the state (GDN-2 summary, «Méthodologie» §1):
+        S_t = A_t S_{t-1} + k_t z_t^T,   A_t = (I - k_t e_t^T) Diag(alpha_t),  e = b .* k,  z = w .* v
+    so M = A_T ... A_1 (dk x dk, the transitions multiplied out here one token at a time) and N is
+    the state after the segment entered with zeros (fwd() from a zero state).
+    Returns (M [B,Hv,dk,dk], N [B,Hv,dk,dv])."""
+    a = _Args(q, k, v, alpha, b, w, beta, None, head_map, 1.0)
+    B, T, Hk, Hv, dk, dv = a.dims
+    M = np.empty((B, Hv, dk, dk))
+    for bb in range(B):
+        for hv in range(Hv):
+            hk = a.map[hv]
+            m = np.eye(dk)
+            for t in range(T):
+                kk = a.k[bb, t, hk]
+                al = np.broadcast_to(a.alpha[bb, t, hv], (dk,))
+                e = np.broadcast_to(a.bg[bb, t, hv], (dk,)) * kk
+                m = al[:, None] * m                # Diag(alpha_t) M
+                m = m - np.outer(kk, e @ m)       # (I - k e^T) Diag(alpha_t) M
+            M[bb, hv] = m
+    _, N = fwd(q, k, v, alpha, b=b, w=w, beta=beta, head_map=head_map)
+    return M, N
+
+
+def compose(M, N, S, transpose: bool = False):
+    """M S + N (or M^T S + N) for every (batch, head): the state after a segment given the state
+    entering it, or, transposed, a state gradient carried back across a segment."""
+    M, N, S = f64(M), f64(N), f64(S)
+    Mt = np.swapaxes(M, -1, -2) if transpose else M
+    return np.einsum("bhij,bhjk->bhik", Mt, S) + N
+
+
 def decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=None, scale=1.0,
                 pairs: Optional[Sequence[int]] = None):
     """One token for N sequences: q,k [N,Hk,dk], v [N,Hv,dv], gates [N,Hv,(d)], state

@@ -466,3 +466,75 @@ def test_layer_backward_finite_differences(channel_gates):
             fd[idx] = (loss(plus) - loss(minus)) / (2 * h)
         err = np.max(np.abs(g[key[n]] - fd)) / max(np.max(np.abs(fd)), 1e-12)
         assert err < 1e-6, (n, err)
+
+
+# ---- segment maps (sequence split along time) --------------------------------------------------
+def _gates(x):
+    return dict(beta=x["beta"]) if "beta" in x else dict(b=x["b"], w=x["w"])
+
+
+@pytest.mark.parametrize("channel", [True, False])
+def test_segment_map_is_the_state_map(channel):
+    """M S + N equals the recurrence run from S, for any entering state S (the update is affine in
+    the state): checked against fwd() from two random states."""
+    rng = np.random.default_rng(71)
+    x = rand_inputs(rng, 2, 37, 1, 2, 8, 8, channel_alpha=channel, channel_gates=channel, h0=False)
+    M, N = oracle.segment_map(x["q"], x["k"], x["v"], x["alpha"], **_gates(x))
+    for _ in range(2):
+        S = rng.standard_normal((2, 2, 8, 8))
+        _, hT = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=S, **_gates(x))
+        assert relerr(oracle.compose(M, N, S), hT) < 1e-12
+
+
+def test_segment_maps_compose_over_a_split_sequence():
+    """Two segments: (M2 M1, M2 N1 + N2) is the map of the whole, and the exclusive composition
+    gives the state entering the second segment."""
+    rng = np.random.default_rng(72)
+    x = rand_inputs(rng, 1, 50, 2, 4, 8, 8, h0=True)
+    cut = 21
+    seg = lambda lo, hi: {k: (v[:, lo:hi] if v.ndim >= 3 and k != "h0" else v) for k, v in x.items()}
+    a, b = seg(0, cut), seg(cut, 50)
+    M1, N1 = oracle.segment_map(a["q"], a["k"], a["v"], a["alpha"], **_gates(a))
+    M2, N2 = oracle.segment_map(b["q"], b["k"], b["v"], b["alpha"], **_gates(b))
+    M, N = oracle.segment_map(x["q"], x["k"], x["v"], x["alpha"], **_gates(x))
+    assert relerr(np.einsum("bhij,bhjk->bhik", M2, M1), M) < 1e-12
+    assert relerr(oracle.compose(M2, N2, N1), N) < 1e-12
+    _, h_mid = oracle.fwd(a["q"], a["k"], a["v"], a["alpha"], h0=x["h0"], **_gates(a))
+    assert relerr(oracle.compose(M1, N1, x["h0"]), h_mid) < 1e-12
+
+
+def test_segment_map_closed_forms():
+    """No erase (b = 0): M = Diag(prod alpha) (decay only), N = sum_t (prod_{s>t} alpha_s) k_t z_t^T;
+    with alpha = 1 as well, M = I and N = K^T Z (linear attention's running sum)."""
+    rng = np.random.default_rng(73)
+    x = rand_inputs(rng, 1, 30, 1, 1, 6, 6, h0=False)
+    x["b"] = np.zeros_like(x["b"])
+    M, N = oracle.segment_map(x["q"], x["k"], x["v"], x["alpha"], **_gates(x))
+    a = x["alpha"][0, :, 0]                      # [T, dk]
+    assert relerr(M[0, 0], np.diag(np.prod(a, axis=0))) < 1e-14
+    tail = np.array([np.prod(a[t + 1:], axis=0) for t in range(30)])  # [T, dk]
+    z = x["w"][0, :, 0] * x["v"][0, :, 0]
+    N_ref = np.einsum("tc,tc,tj->cj", tail, x["k"][0, :, 0], z)
+    assert relerr(N[0, 0], N_ref) < 1e-12
+    x["alpha"] = np.ones_like(x["alpha"])
+    M, N = oracle.segment_map(x["q"], x["k"], x["v"], x["alpha"], **_gates(x))
+    assert np.array_equal(M[0, 0], np.eye(6))
+    assert relerr(N[0, 0], x["k"][0, :, 0].T @ z) < 1e-12
+
+
+def test_transposed_composition_carries_a_state_gradient_back():
+    """For L = <G, S_out> with S_out = M S_in + N, dL/dS_in = M^T G: the transposed composition,
+    checked by finite differences of the oracle's own forward."""
+    rng = np.random.default_rng(74)
+    x = rand_inputs(rng, 1, 12, 1, 1, 4, 4, h0=True)
+    M, N = oracle.segment_map(x["q"], x["k"], x["v"], x["alpha"], **_gates(x))
+    G = rng.standard_normal((1, 1, 4, 4))
+    grad = oracle.compose(M, np.zeros_like(G), G, transpose=True)
+    eps = 1e-6
+    for (i, j) in [(0, 0), (1, 3), (3, 2)]:
+        d = np.zeros_like(x["h0"])
+        d[0, 0, i, j] = eps
+        _, hp = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=x["h0"] + d, **_gates(x))
+        _, hm = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=x["h0"] - d, **_gates(x))
+        fd = np.sum(G * (hp - hm)) / (2 * eps)
+        assert abs(fd - grad[0, 0, i, j]) < 1e-7 * max(1.0, abs(fd))
