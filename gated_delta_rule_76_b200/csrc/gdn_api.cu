@@ -168,13 +168,14 @@ using namespace gdn;
 
 namespace {
 
-gdn_status check_fwd(const gdn_fwd_args* a) {
+gdn_status check_fwd(const gdn_fwd_args* a, bool need_o = true) {
     if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
     gdn_status s = check_common(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->head_map,
                                 a->alpha_per_channel, a->gates_per_channel, a->dtype, a->gate_dtype);
     if (s) return s;
-    if (a->T > 0 && (!a->q || !a->k || !a->v || !a->alpha || !a->b || !a->o))
-        return fail(GDN_ERR_INVALID_ARG, "q, k, v, alpha, b and o are required");
+    if (a->T > 0 && (!a->q || !a->k || !a->v || !a->alpha || !a->b || (need_o && !a->o)))
+        return fail(GDN_ERR_INVALID_ARG, need_o ? "q, k, v, alpha, b and o are required"
+                                                : "q, k, v, alpha and b are required");
     if (a->gates_per_channel && a->T > 0 && !a->w)
         return fail(GDN_ERR_INVALID_ARG, "w is required when gates_per_channel = 1");
     if (!a->gates_per_channel && a->w)
@@ -312,10 +313,12 @@ size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
     return plan_chunk_ws(pb, false, false).bytes;
 }
 
-gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspace_bytes,
-                         gdn_stream stream) {
-    gdn_status s = check_fwd(a);
-    if (s) return s;
+}  // extern "C"
+
+// The chunk forward on validated arguments (o may be NULL: no output is written).
+static gdn_status chunk_fwd_core(const gdn_fwd_args* a, void* workspace, size_t workspace_bytes,
+                                 gdn_stream stream) {
+    gdn_status s = GDN_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t sbytes = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
     if (a->T == 0) return copy_state(a->ht, a->h0, sbytes, st, "gdn_chunk_fwd");
@@ -349,6 +352,88 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
         else e = run_fwd(variant(a->dtype, a->gate_dtype), pb, io_from(a), carve_chunk_ws(plan, workspace), f, st);
     }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_fwd");
+}
+
+extern "C" {
+
+gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspace_bytes,
+                         gdn_stream stream) {
+    gdn_status s = check_fwd(a);
+    if (s) return s;
+    return chunk_fwd_core(a, workspace, workspace_bytes, stream);
+}
+
+// Segment map: the forward from a zero state (N = ht, o optional), then the forward from the
+// identity with the writes zeroed (v = 0), whose final state is M.
+size_t gdn_segment_map_workspace_size(const gdn_fwd_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    const size_t es = elem_size(a->dtype);
+    return align256(gdn_chunk_fwd_workspace_size(a)) + align256((size_t)(a->B * a->Hv * a->dk * a->dk) * 4) +
+           align256((size_t)(a->B * a->T * a->Hv * a->dv) * es);
+}
+
+gdn_status gdn_segment_map(const gdn_fwd_args* a, float* M, void* workspace, size_t workspace_bytes,
+                           gdn_stream stream) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    if (a->h0 || a->z || a->bwd_cache)
+        return fail(GDN_ERR_INVALID_ARG, "gdn_segment_map: h0, z and bwd_cache must be NULL");
+    if (!a->ht || !M) return fail(GDN_ERR_INVALID_ARG, "gdn_segment_map: ht (receives N) and M are required");
+    // validated as a forward whose o is optional; M must not overlap any input or output
+    gdn_status s = check_fwd(a, false);
+    if (s) return s;
+    const gdn_fwd_args x = *a;
+    const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype), BT = (size_t)(a->B * a->T);
+    const size_t mbytes = (size_t)(a->B * a->Hv * a->dk * a->dk) * 4;
+    const Buf in[] = {{a->q, BT * a->Hk * a->dk * es, "q"}, {a->k, BT * a->Hk * a->dk * es, "k"},
+                      {a->v, BT * a->Hv * a->dv * es, "v"},
+                      {a->alpha, BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
+                      {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
+                      {a->w, a->w ? BT * a->Hv * a->dv * gs : 0, "w"}, {a->head_map, (size_t)a->Hv * 4, "head_map"}};
+    const Buf out[] = {{M, mbytes, "M"}, {a->ht, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "ht"},
+                       {a->o, a->o ? BT * a->Hv * a->dv * (a->out_f32 ? 4 : es) : 0, "o"}};
+    if ((s = check_buffers(in, 7, out, 3))) return s;
+    const size_t need = gdn_segment_map_workspace_size(a);
+    if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (a->T == 0) {
+        cudaError_t e = cudaMemsetAsync(a->ht, 0, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, st);
+        if (e == cudaSuccess) e = identity_states(M, a->B * a->Hv, (int)a->dk, st);
+        return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_segment_map");
+    }
+    char* base = static_cast<char*>(workspace);
+    const size_t fw = align256(gdn_chunk_fwd_workspace_size(a));
+    float* ident = reinterpret_cast<float*>(base + fw);
+    void* zero_v = base + fw + align256(mbytes);
+    // N: the segment from a zero state
+    if ((s = chunk_fwd_core(&x, workspace, fw, stream))) return s;
+    // M: from the identity, with nothing written (z = w .* v = 0)
+    cudaError_t e = identity_states(ident, a->B * a->Hv, (int)a->dk, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(zero_v, 0, BT * a->Hv * a->dv * es, st);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_segment_map");
+    gdn_fwd_args y = x;
+    y.v = zero_v;
+    y.h0 = ident;
+    y.ht = M;
+    y.o = nullptr;
+    return chunk_fwd_core(&y, workspace, fw, stream);
+}
+
+gdn_status gdn_state_compose(const float* M, const float* N, const float* S_in, float* S_out, int64_t pairs,
+                             int64_t dk, int64_t dv, int32_t transpose, gdn_stream stream) {
+    if (!M || !S_out) return fail(GDN_ERR_INVALID_ARG, "gdn_state_compose: M and S_out are required");
+    if (pairs < 1) return fail(GDN_ERR_INVALID_ARG, "gdn_state_compose: pairs must be >= 1");
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128))
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_state_compose: dk, dv must be 64 or 128");
+    if (transpose != 0 && transpose != 1) return fail(GDN_ERR_INVALID_ARG, "transpose must be 0 or 1");
+    if (transpose && dk != dv) return fail(GDN_ERR_INVALID_ARG, "gdn_state_compose: M^T needs dk == dv");
+    const size_t st = (size_t)(pairs * dk * dv) * 4;
+    const Buf in[] = {{M, (size_t)(pairs * dk * dk) * 4, "M"}, {N, N ? st : 0, "N"}, {S_in, S_in ? st : 0, "S_in"}};
+    const Buf out[] = {{S_out, st, "S_out"}};
+    gdn_status s = check_buffers(in, 3, out, 1);
+    if (s) return s;
+    cudaError_t e = compose_states(M, N, S_in, S_out, (long)pairs, (int)dk, (int)dv, transpose != 0,
+                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_state_compose");
 }
 
 static bool bwd_uses_tensor_cores(const gdn_bwd_args* a, const Problem& pb) {

@@ -50,7 +50,7 @@ cudaError_t chunk_fwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
                               chunk_scan_fwd_smem<DK>(), st, pb, io, ws, write_out ? 1 : 0,
                               save_states ? 1 : 0));
     // pairs whose decay left the factors' range (marked by prep): their outputs again, exactly
-    if (!ws.flags || !write_out) return cudaSuccess;
+    if (!ws.flags || (!write_out && !io.ht)) return cudaSuccess;
     return seq_fwd(pb, io, Flags{APC, GPC, gate}, std::is_same<TIn, float>::value, std::is_same<TG, float>::value,
                    ws.flags, nullptr, st);
 }
@@ -97,7 +97,7 @@ cudaError_t chunk_fwd_impl(const Problem& pb, const ChunkIO& io, const ChunkWs& 
                            cudaStream_t st) {
     return dispatch_chunk<TIn, TG>(pb, f, [&](auto apc, auto gpc, auto dk) {
         return chunk_fwd_t<TIn, TG, decltype(apc)::value, decltype(gpc)::value, decltype(dk)::value>(
-            pb, io, ws, f.gate, f.paired, true, st);
+            pb, io, ws, f.gate, f.paired, io.o != nullptr, st);
     });
 }
 

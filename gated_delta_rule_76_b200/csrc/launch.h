@@ -66,6 +66,12 @@ cudaError_t seq_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32,
 cudaError_t seq_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
                     float* dq, float* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st);
 
+// Sequence split along time (seqpar.cu): S = I for `pairs` states of d x d; S_out = op(M) S_in + N
+// per pair (op = transpose or not; S_in or N may be NULL: taken as zero).
+cudaError_t identity_states(float* S, long pairs, int d, cudaStream_t st);
+cudaError_t compose_states(const float* M, const float* N, const float* S_in, float* S_out, long pairs, int dk,
+                           int dv, bool transpose, cudaStream_t st);
+
 // Tensor-core chunk backward (tc_bwd.cu): same eligibility as the forward, without z.
 // The forward cache (what the backward needs from the forward): byte offsets from its start.
 struct TcCache {

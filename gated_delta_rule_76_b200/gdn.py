@@ -75,6 +75,7 @@ class LayerBwdArgs(ctypes.Structure):
 EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_cache_size", "gdn_layer_core_fwd_workspace_size",
             "gdn_layer_core_fwd", "gdn_layer_core_bwd_workspace_size", "gdn_layer_core_bwd",
+            "gdn_segment_map_workspace_size", "gdn_segment_map", "gdn_state_compose",
             "gdn_workspace_status", "gdn_last_error", "gdn_kernel_launches", "gdn_version"]
 
 _lib = None
@@ -116,6 +117,12 @@ def load(path: str = LIB_PATH):
     lib.gdn_layer_core_bwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_layer_core_bwd.argtypes = [ctypes.POINTER(LayerBwdArgs), P, ctypes.c_size_t, P]
     lib.gdn_layer_core_bwd.restype = ctypes.c_int
+    lib.gdn_segment_map_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
+    lib.gdn_segment_map_workspace_size.restype = ctypes.c_size_t
+    lib.gdn_segment_map.argtypes = [ctypes.POINTER(FwdArgs), P, P, ctypes.c_size_t, P]
+    lib.gdn_segment_map.restype = ctypes.c_int
+    lib.gdn_state_compose.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, P]
+    lib.gdn_state_compose.restype = ctypes.c_int
     lib.gdn_workspace_status.argtypes = [P, P]
     lib.gdn_workspace_status.restype = ctypes.c_int
     lib.gdn_last_error.argtypes = []
@@ -268,6 +275,37 @@ def gdn_chunk_fwd_noalloc(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=
     a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht)
     check(lib.gdn_chunk_fwd_noalloc(ctypes.byref(a), _stream(stream)), "gdn_chunk_fwd_noalloc")
     return o, ht
+
+
+def gdn_segment_map(q, k, v, alpha, b=None, w=None, beta=None, head_map=None, *, want_o: bool = False,
+                    workspace: Optional[torch.Tensor] = None, stream=None):
+    """The affine map of this segment of every sequence on the state: returns (M [B,Hv,dk,dk],
+    N [B,Hv,dk,dv]) with state_after = M state_before + N, plus the segment's output from a zero
+    entering state when ``want_o`` (then (M, N, o))."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    M = torch.empty((B, Hv, dk, dk), dtype=torch.float32, device=q.device)
+    N = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    o = torch.empty((B, T, Hv, dv), dtype=q.dtype, device=q.device) if want_o else None
+    lib = load()
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, None, None, head_map, 1.0, o, N)
+    need = lib.gdn_segment_map_workspace_size(ctypes.byref(a))
+    ws = _workspace(need, q.device, workspace)
+    check(lib.gdn_segment_map(ctypes.byref(a), _ptr(M), _ptr(ws), need, _stream(stream)), "gdn_segment_map")
+    return (M, N, o) if want_o else (M, N)
+
+
+def gdn_state_compose(M, N, S, *, transpose: bool = False, out: Optional[torch.Tensor] = None, stream=None):
+    """op(M) S + N per (sequence, head) on the device, op = transpose or identity.  M [..., dk, dk],
+    N and S [..., dk, dv] fp32 (S or N may be None: zero).  Returns the result (``out`` if given)."""
+    ref = S if S is not None else N
+    dk, dv = M.shape[-1], ref.shape[-1]
+    pairs = M.numel() // (dk * dk)
+    if out is None:
+        out = torch.empty(ref.shape, dtype=torch.float32, device=M.device)
+    check(load().gdn_state_compose(_ptr(M), _ptr(N), _ptr(S), _ptr(out), pairs, dk, dv, int(transpose),
+                                   _stream(stream)), "gdn_state_compose")
+    return out
 
 
 def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, scale=1.0,

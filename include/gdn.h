@@ -187,6 +187,34 @@ GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args* args, void* workspace, size
                          gdn_stream stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Sequence split along time (several GPUs, one segment of every sequence each).  The recurrent
+ * state has a fixed size whatever the context length (mkdocs chapter «Gated DeltaNet», «L'état,
+ * en mémoire»), and each token's update is affine in it (GDN-2 summary, «Méthodologie» §1):
+ * S_t = A_t S_{t-1} + k_t z_t^T with A_t = (I - k_t e_t^T) Diag(alpha_t).  A segment therefore
+ * maps the state entering it to M S + N, with M = A_T ... A_1 (dk x dk) and N the state after the
+ * segment entered with zeros (dk x dv).  The state entering segment r is the composition of the
+ * maps of segments 0 .. r-1 applied to h0; a state gradient crosses a segment backwards as
+ * M^T dS (+ the segment's own contribution, which a backward with zero dht gives as dh0).
+ *
+ * gdn_segment_map: for one segment of every (sequence, value head), M [B,Hv,dk,dk] fp32 and
+ * N = args->ht [B,Hv,dk,dv] fp32 (required).  args is read as by gdn_chunk_fwd, except that h0, z
+ * and bwd_cache must be NULL and o may be NULL (if given, it receives the segment's output from a
+ * zero entering state).  Needs dk == dv.  It runs the chunk forward twice: from a zero state (N),
+ * and from the identity with the writes zeroed (M), so the decay-range handling of
+ * gdn_chunk_fwd applies.  Workspace: gdn_segment_map_workspace_size(args) bytes, 256-byte aligned.
+ * ------------------------------------------------------------------------------------------ */
+GDN_API size_t gdn_segment_map_workspace_size(const gdn_fwd_args* args);
+GDN_API gdn_status gdn_segment_map(const gdn_fwd_args* args, float* M, void* workspace, size_t workspace_bytes,
+                                   gdn_stream stream);
+
+/* S_out = M S_in + N (transpose = 0) or M^T S_in + N (transpose = 1, needs dk == dv) for `pairs`
+ * independent (sequence, head) pairs, fp32: M [pairs,dk,dk], N and S_in and S_out [pairs,dk,dv].
+ * S_in or N may be NULL (taken as zero).  S_out must not overlap M, N or S_in.  dk, dv in
+ * {64, 128}.  The composition step of the sequence split above, on the device. */
+GDN_API gdn_status gdn_state_compose(const float* M, const float* N, const float* S_in, float* S_out, int64_t pairs,
+                                     int64_t dk, int64_t dv, int32_t transpose, gdn_stream stream);
+
+/* ------------------------------------------------------------------------------------------
  * Single-token decode step for N sequences: the recurrence applied once, with the fp32 state
  * read, updated and written back in place (constant memory per sequence; mkdocs chapter «Gated
  * DeltaNet», «L'état, en mémoire»).

@@ -228,3 +228,26 @@ def test_binding_checks_a_host_head_map():
     for bad in ([0, 2], [-1, 0]):
         with pytest.raises(gdn.GdnError):
             gdn._head_map(bad, "cpu", 2)
+
+
+def test_segment_map_and_compose_host_validation(lib):
+    """gdn_segment_map takes no h0 and needs ht (N) and M; gdn_state_compose checks its sizes and
+    overlaps.  Rejected on the host, before any launch (fake device addresses, never touched)."""
+    P = ctypes.c_void_p
+    M, N = P(1 << 24), P(1 << 25)
+    before = gdn.kernel_launches()
+    a = _fwd(o=None, ht=1 << 25, h0=1 << 26)
+    assert lib.gdn_segment_map(ctypes.byref(a), M, P(1 << 30), 1 << 30, None) == 1  # h0 given
+    a = _fwd(o=None, ht=None)
+    assert lib.gdn_segment_map(ctypes.byref(a), M, P(1 << 30), 1 << 30, None) == 1  # no ht
+    a = _fwd(o=None, ht=1 << 25)
+    assert lib.gdn_segment_map(ctypes.byref(a), None, P(1 << 30), 1 << 30, None) == 1  # no M
+    a = _fwd(o=None, ht=1 << 24)
+    assert lib.gdn_segment_map(ctypes.byref(a), M, P(1 << 30), 1 << 30, None) == 1  # M overlaps ht
+    a = _fwd(o=None, ht=1 << 25)
+    assert lib.gdn_segment_map(ctypes.byref(a), M, None, 0, None) == 4  # no workspace
+    assert lib.gdn_state_compose(M, None, None, N, 1, 32, 32, 0, None) == 2
+    assert lib.gdn_state_compose(None, None, None, N, 1, 128, 128, 0, None) == 1
+    assert lib.gdn_state_compose(M, None, None, M, 1, 128, 128, 0, None) == 1  # output overlaps M
+    assert lib.gdn_state_compose(M, None, None, N, 1, 64, 128, 1, None) == 1   # M^T needs dk == dv
+    assert gdn.kernel_launches() == before
