@@ -269,6 +269,19 @@ def l2norm(x, eps: float = L2_EPS):
     return x
 
 
+RMS_EPS = 1e-6
+
+
+def gated_rmsnorm(o, z, norm_w, eps: float = RMS_EPS):
+    """The layer's output norm and gate (explainer «Architecture et versions hybrides», Figure 1
+    caption: the output is normalised, then multiplied by a gate; mkdocs chapter «Gated DeltaNet»,
+    «Le décompte»: 128 norm weights shared by the heads): every (token, head) row of dv values is
+    divided by its root mean square, scaled by norm_w [dv], and multiplied by z sigmoid(z)."""
+    o, z, wn = f64(o), f64(z), f64(norm_w)
+    r = 1.0 / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    return o * r * wn * z * _sigmoid(z)
+
+
 def swish_gate(o, z):
     o = f64(o)
     z = f64(z)
@@ -278,7 +291,7 @@ def swish_gate(o, z):
 
 
 def layer_core_fwd(xq, xk, xv, conv_w, alpha, beta, z, head_map=None, scale=1.0, h0=None,
-                   pairs: Optional[Sequence[int]] = None):
+                   pairs: Optional[Sequence[int]] = None, norm_w=None):
     """GQA layer core: conv(k=4)+SiLU on the q, k, v projections (zero history), L2 norm on
     q and k, the recurrence, then the swish(z) output gate.  Conv channels are ordered
     q (Hk*dk), k (Hk*dk), v (Hv*dv).  Returns (y [B,T,Hv,dv], hT)."""
@@ -294,6 +307,8 @@ def layer_core_fwd(xq, xk, xv, conv_w, alpha, beta, z, head_map=None, scale=1.0,
     k = l2norm(k.reshape(B, T, Hk, dk))
     v = v.reshape(B, T, Hv, dv)
     o, hT = fwd(q, k, v, alpha, beta=beta, h0=h0, head_map=head_map, scale=scale, pairs=pairs)
+    if norm_w is not None:
+        return gated_rmsnorm(o, z, norm_w), hT
     return swish_gate(o, z), hT
 
 
@@ -338,9 +353,10 @@ def _sigmoid(x):
 
 
 def layer_core_bwd(xq, xk, xv, conv_w, alpha, z, dy, b=None, w=None, beta=None, head_map=None,
-                   scale=1.0, h0=None, dht=None) -> Dict[str, np.ndarray]:
+                   scale=1.0, h0=None, dht=None, norm_w=None) -> Dict[str, np.ndarray]:
     """Reverse mode of the GQA layer core for loss gradients dy (of y) and dht (of the final
-    state).  Returns dxq, dxk, dxv, dconv_w, dz, dalpha, db/dw or dbeta, dh0."""
+    state).  Returns dxq, dxk, dxv, dconv_w, dz, dalpha, db/dw or dbeta, dh0, and dnorm_w when the
+    output norm is on (norm_w given)."""
     xq, xk, xv, W = f64(xq), f64(xk), f64(xv), f64(conv_w)
     zz, g = f64(z), f64(dy)
     B, T, Hk, dk = xq.shape
@@ -363,10 +379,23 @@ def layer_core_bwd(xq, xk, xv, conv_w, alpha, z, dy, b=None, w=None, beta=None, 
     gk = dict(beta=beta) if beta is not None else dict(b=b, w=w)
     o, _ = fwd(q, k, v, alpha, head_map=head_map, scale=scale, h0=h0, **gk)
     sg = _sigmoid(zz)
-    do = g * zz * sg                                 # y = o * z * sigmoid(z)
-    dz = g * o * (sg + zz * sg * (1.0 - sg))
+    swz = zz * sg                                    # swish(z)
+    dswz = sg + zz * sg * (1.0 - sg)                 # its derivative
+    extra = {}
+    if norm_w is None:
+        do = g * swz                                 # y = o * swish(z)
+        dz = g * o * dswz
+    else:
+        # y = n * wn * swish(z),  n = o * r,  r = (mean_j o_j^2 + eps)^(-1/2) per (token, head) row
+        wn = f64(norm_w)
+        r = 1.0 / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + RMS_EPS)
+        n = o * r
+        dn = g * wn * swz
+        dz = g * n * wn * dswz
+        extra["dnorm_w"] = np.sum(g * n * swz, axis=(0, 1, 2))
+        do = r * (dn - n * np.mean(dn * n, axis=-1, keepdims=True))
     core = bwd(q, k, v, alpha, head_map=head_map, scale=scale, h0=h0, dout=do, dht=dht, **gk)
-    res = {"dz": dz, "dalpha": core["dalpha"], "dh0": core["dh0"]}
+    res = {"dz": dz, "dalpha": core["dalpha"], "dh0": core["dh0"], **extra}
     for key in ("dbeta", "db", "dw"):
         if key in core:
             res[key] = core[key]

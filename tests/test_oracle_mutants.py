@@ -111,8 +111,13 @@ def test_planted_mistake_is_caught(name, edits, workdir):
 PY = os.path.join(os.path.dirname(oracle.__file__), "oracle.py")
 LAYER_MUTANTS = [
     ("swish gate: dz without its z s (1 - s) term",
-     "dz = g * o * (sg + zz * sg * (1.0 - sg))", "dz = g * o * sg"),
-    ("swish gate: do without the factor z", "do = g * zz * sg", "do = g * sg"),
+     "dswz = sg + zz * sg * (1.0 - sg)", "dswz = sg"),
+    ("swish gate: do without the factor z", "swz = zz * sg ", "swz = sg "),
+    ("output norm backward without the mean term",
+     "do = r * (dn - n * np.mean(dn * n, axis=-1, keepdims=True))", "do = r * dn"),
+    ("output norm: weight gradient without the gate",
+     'extra["dnorm_w"] = np.sum(g * n * swz, axis=(0, 1, 2))', 'extra["dnorm_w"] = np.sum(g * n, axis=(0, 1, 2))'),
+    ("output norm: dz without the norm weight", "dz = g * n * wn * dswz", "dz = g * n * dswz"),
     ("L2 norm backward without the projection",
      "da = ((gout - out * dot) / n).reshape(a.shape)", "da = (gout / n).reshape(a.shape)"),
     ("SiLU backward: the sigmoid's derivative instead of SiLU's",
@@ -134,10 +139,17 @@ def _oracle_copy(src):
     return mod
 
 
+def _layer_pins():
+    """The finite-difference pins of the layer core's reverse mode, with and without the output norm."""
+    return [lambda: pins.test_layer_backward_finite_differences(False),
+            lambda: pins.test_layer_backward_finite_differences(True),
+            pins.test_layer_backward_with_output_norm_finite_differences]
+
+
 def test_unmutated_layer_oracle_copy_passes_its_pin(monkeypatch):
     monkeypatch.setattr(pins, "oracle", _oracle_copy(open(PY).read()))
-    for channel_gates in (False, True):
-        pins.test_layer_backward_finite_differences(channel_gates)
+    for pin in _layer_pins():
+        pin()
 
 
 @pytest.mark.parametrize("name,old,new", LAYER_MUTANTS, ids=[m[0] for m in LAYER_MUTANTS])
@@ -146,9 +158,9 @@ def test_planted_layer_backward_mistake_is_caught(name, old, new, monkeypatch):
     assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
     monkeypatch.setattr(pins, "oracle", _oracle_copy(src.replace(old, new)))
     caught = []
-    for channel_gates in (False, True):
+    for i, pin in enumerate(_layer_pins()):
         try:
-            pins.test_layer_backward_finite_differences(channel_gates)
+            pin()
         except AssertionError:
-            caught.append(channel_gates)
+            caught.append(i)
     assert caught, f"no pin caught the planted mistake: {name}"

@@ -538,3 +538,64 @@ def test_transposed_composition_carries_a_state_gradient_back():
         _, hm = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=x["h0"] - d, **_gates(x))
         fd = np.sum(G * (hp - hm)) / (2 * eps)
         assert abs(fd - grad[0, 0, i, j]) < 1e-7 * max(1.0, abs(fd))
+
+
+# ---- the layer's output norm ---------------------------------------------------------------------
+def test_gated_rmsnorm_matches_the_library_rms_norm():
+    """oracle.gated_rmsnorm against torch's own rms_norm (a library routine, float64) times
+    swish(z); and invariance of the normalised rows to a positive scale of o."""
+    import torch
+    rng = np.random.default_rng(75)
+    o = rng.standard_normal((2, 5, 3, 16))
+    z = rng.standard_normal((2, 5, 3, 16))
+    wn = rng.standard_normal(16)
+    y = oracle.gated_rmsnorm(o, z, wn)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(o), (16,), weight=torch.from_numpy(wn), eps=oracle.RMS_EPS)
+    ref = ref.numpy() * z / (1.0 + np.exp(-z))
+    assert relerr(y, ref) < 1e-13
+    assert relerr(oracle.gated_rmsnorm(7.5 * o, z, wn), y) < 1e-6
+
+
+def test_layer_backward_with_output_norm_finite_differences():
+    """The layer core with its output norm (y = RMSNorm(o) * norm_w * swish(z)): every gradient,
+    norm_w's included, against central differences of sum(y * dy) + sum(hT * dht)."""
+    rng = np.random.default_rng(76)
+    B, T, Hk, Hv, d = 1, 5, 1, 2, 4
+    cq = Hk * d
+    x = dict(xq=rng.standard_normal((B, T, Hk, d)), xk=rng.standard_normal((B, T, Hk, d)),
+             xv=rng.standard_normal((B, T, Hv, d)), conv_w=0.5 * rng.standard_normal((2 * cq + Hv * d, 4)),
+             alpha=np.exp(-0.1 * np.logaddexp(0.0, rng.standard_normal((B, T, Hv)))),
+             beta=1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, Hv)))),
+             z=rng.standard_normal((B, T, Hv, d)), h0=0.3 * rng.standard_normal((B, Hv, d, d)),
+             norm_w=rng.standard_normal(d))
+    dy = rng.standard_normal((B, T, Hv, d))
+    dht = rng.standard_normal((B, Hv, d, d))
+
+    def loss(vals):
+        W = vals["conv_w"]
+        q, _ = oracle.conv_silu(vals["xq"].reshape(B, T, cq), W[:cq])
+        k, _ = oracle.conv_silu(vals["xk"].reshape(B, T, cq), W[cq:2 * cq])
+        v, _ = oracle.conv_silu(vals["xv"].reshape(B, T, Hv * d), W[2 * cq:])
+        q = oracle.l2norm(q.reshape(B, T, Hk, d))
+        k = oracle.l2norm(k.reshape(B, T, Hk, d))
+        o, hT = oracle.fwd(q, k, v.reshape(B, T, Hv, d), vals["alpha"], beta=vals["beta"], h0=vals["h0"],
+                           nthreads=1)
+        return np.sum(oracle.gated_rmsnorm(o, vals["z"], vals["norm_w"]) * dy) + np.sum(hT * dht)
+
+    g = oracle.layer_core_bwd(x["xq"], x["xk"], x["xv"], x["conv_w"], x["alpha"], x["z"], dy, beta=x["beta"],
+                              h0=x["h0"], dht=dht, norm_w=x["norm_w"])
+    key = {"xq": "dxq", "xk": "dxk", "xv": "dxv", "conv_w": "dconv_w", "alpha": "dalpha", "z": "dz",
+           "h0": "dh0", "beta": "dbeta", "norm_w": "dnorm_w"}
+    h = 1e-6
+    for n in x:
+        fd = np.zeros_like(x[n])
+        it = np.nditer(x[n], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = {m: x[m].copy() for m in x}
+            minus = {m: x[m].copy() for m in x}
+            plus[n][idx] += h
+            minus[n][idx] -= h
+            fd[idx] = (loss(plus) - loss(minus)) / (2 * h)
+        err = np.max(np.abs(g[key[n]] - fd)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-6, (n, err)
