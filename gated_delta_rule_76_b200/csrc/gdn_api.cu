@@ -571,12 +571,21 @@ size_t gdn_layer_core_fwd_cache_size(const gdn_layer_args* a) {
     return plan_layer_cache(make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map)).bytes;
 }
 
+// The layer forward hands its conv results to the tensor-core forward as bf16 hi/lo pairs (bf16
+// tensors, scalar gates, d = 128); otherwise they stay fp32 for the CUDA-core forward.
+static bool layer_fwd_split(const gdn_layer_args* a, const Problem& pb) {
+    Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, true};
+    return a->dtype == GDN_BF16 && !f.apc && !f.gpc && tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
+}
+
 size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     // q, k, v after the convolution are kept in fp32 between the two kernels.
     const size_t conv = align256((size_t)(a->B * a->T) * (2 * a->Hk * a->dk + a->Hv * a->dv) * 4);
-    return 256 + conv + plan_chunk_ws(pb, false, false).bytes;
+    // the CUDA-core form with the output norm keeps o (fp32) for the norm + gate kernel
+    const size_t onorm = a->norm_w && !layer_fwd_split(a, pb) ? align256((size_t)(a->B * a->T * a->Hv * a->dv) * 4) : 0;
+    return 256 + conv + plan_chunk_ws(pb, false, false).bytes + onorm;
 }
 
 gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t workspace_bytes,
@@ -600,14 +609,17 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
         {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
         {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->z, BT * a->Hv * a->dv * es, "z"},
         {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        {a->norm_w, (size_t)a->dv * es, "norm_w"},
     };
     if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
+    if (a->norm_w && !(a->norm_eps >= 0.f && a->norm_eps < 1e30f))
+        return fail(GDN_ERR_INVALID_ARG, "norm_eps must be a finite number >= 0");
     const Buf out[] = {
         {a->y, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "y"}, {a->ht, st, "ht"},
         {a->conv_state_out, (size_t)a->B * cch * 3 * es, "conv_state_out"},
         {a->bwd_cache, a->bwd_cache ? a->bwd_cache_bytes : 0, "bwd_cache"},
     };
-    if ((s = check_buffers(in, 10, out, 4))) return s;
+    if ((s = check_buffers(in, 11, out, 4))) return s;
     if (a->bwd_cache) {
         if (!layer_tc_form(a->dtype, a->dk, a->dv, a->alpha_per_channel, a->gates_per_channel, a->h0))
             return fail(GDN_ERR_UNSUPPORTED, "bwd_cache: only the tensor-core form (bf16, d = 128, scalar gates, no h0) "
@@ -641,8 +653,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     // The conv outputs are fp32 values.  With scalar gates and bf16 tensors they go to the
     // tensor-core forward as bf16 hi/lo pairs (same bytes); otherwise they stay fp32 for the
     // CUDA-core forward.
-    const bool split = a->dtype == GDN_BF16 && !f.apc && !f.gpc &&
-                       tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
+    const bool split = layer_fwd_split(a, pb);
     if (a->bwd_cache && !split)
         return fail(GDN_ERR_UNSUPPORTED, "bwd_cache: the tensor-map encoder of the CUDA driver is unavailable");
     const size_t qn = BT * a->Hk * a->dk, vn = BT * a->Hv * a->dv;
@@ -669,6 +680,9 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     // y is written in dtype (bf16 -> o_type 2) unless out_f32.
     io.o_type = a->out_f32 || a->dtype == GDN_F32 ? 1 : 2;
     io.z_bf16 = a->dtype == GDN_BF16;
+    io.norm_w = a->norm_w;
+    io.norm_w_f32 = a->dtype == GDN_F32;
+    io.norm_eps = a->norm_eps;
     if (split) {
         io.q_lo = cp.q_lo; io.k_lo = cp.k_lo; io.v_lo = cp.v_lo;
         if (cache) {
@@ -680,6 +694,19 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
         } else {
             e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, nullptr, flags);
         }
+    } else if (a->norm_w) {
+        // the CUDA-core chunk kernels split a row's columns over blocks: o (fp32, no gate) first, then
+        // the norm and the gate row by row
+        float* onorm = reinterpret_cast<float*>(static_cast<char*>(workspace) + 256 + conv_bytes + chunk_plan.bytes);
+        io.o = onorm;
+        io.o_type = 1;
+        Flags fo = f;
+        fo.gate = false;
+        e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(chunk_plan, base + conv_bytes), fo, sm);
+        if (e == cudaSuccess)
+            e = layer_norm_gate_fwd(onorm, a->z, a->norm_w, a->dtype == GDN_F32, a->norm_eps, a->y,
+                                    a->out_f32 || a->dtype == GDN_F32, a->dtype == GDN_BF16, (long)BT * a->Hv,
+                                    (int)a->dv, sm);
     } else {
         e = run_fwd(a->gate_dtype == GDN_F32 ? 2 : 3, pb, io, carve_chunk_ws(chunk_plan, base + conv_bytes), f, sm);
     }
@@ -697,7 +724,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
 // (fp32), the q, k, v gradients, the conv-weight partials, then the CUDA-core chunk workspace.
 struct LayerBwdPlan {
     bool tc;
-    size_t q, k, v, o, dout, gq, gk, gv, wpart, cache, chunk, bytes;
+    size_t q, k, v, o, dout, npart, gq, gk, gv, wpart, cache, chunk, bytes;
     size_t gq2, gk2, gv2, ga2, gb2, gh2;  // tensor-core form: gradients from the lo half of do
 };
 static bool layer_bwd_tc_form(const gdn_layer_bwd_args* a) {
@@ -720,6 +747,7 @@ static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& p
         w.q = take(qn * 4); w.k = take(qn * 4); w.v = take(vn * 4); w.o = take(vn * 4);
     }
     w.dout = take(vn * 4);  // fp32, or bf16 hi then lo
+    w.npart = a->norm_w ? take(layer_norm_partials_floats((int)a->dv) * 4) : ~size_t(0);
     w.gq = take(qn * 4); w.gk = take(qn * 4); w.gv = take(vn * 4);
     w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk) * 4);
     if (w.tc) {
@@ -754,6 +782,10 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
                      !a->grad_xq || !a->grad_xk || !a->grad_xv || !a->grad_alpha || !a->grad_b || !a->grad_z))
         return fail(GDN_ERR_INVALID_ARG, "inputs, grad_y and the gradients of xq, xk, xv, alpha, b, z are required");
     if (!a->grad_conv_w) return fail(GDN_ERR_INVALID_ARG, "grad_conv_w is required");
+    if (a->norm_w && !a->grad_norm_w) return fail(GDN_ERR_INVALID_ARG, "grad_norm_w is required with norm_w");
+    if (!a->norm_w && a->grad_norm_w) return fail(GDN_ERR_INVALID_ARG, "grad_norm_w must be NULL without norm_w");
+    if (a->norm_w && !(a->norm_eps >= 0.f && a->norm_eps < 1e30f))
+        return fail(GDN_ERR_INVALID_ARG, "norm_eps must be a finite number >= 0");
     if (a->gates_per_channel ? (a->T > 0 && (!a->w || !a->grad_w)) : (a->w != nullptr || a->grad_w != nullptr))
         return fail(GDN_ERR_INVALID_ARG, "w and grad_w are required with channel gates and must be NULL otherwise");
     const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
@@ -769,14 +801,16 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
         {a->z, BT * a->Hv * a->dv * es, "z"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_y, BT * a->Hv * a->dv * es, "grad_y"}, {a->grad_ht, st, "grad_ht"},
         {a->fwd_cache, a->fwd_cache ? a->fwd_cache_bytes : 0, "fwd_cache"},
+        {a->norm_w, (size_t)a->dv * es, "norm_w"},
     };
     const Buf out[] = {
         {a->grad_xq, BT * a->Hk * a->dk * 4, "grad_xq"}, {a->grad_xk, BT * a->Hk * a->dk * 4, "grad_xk"},
         {a->grad_xv, BT * a->Hv * a->dv * 4, "grad_xv"}, {a->grad_conv_w, cch * 4 * 4, "grad_conv_w"},
         {a->grad_alpha, na * 4, "grad_alpha"}, {a->grad_b, nb * 4, "grad_b"}, {a->grad_w, nw * 4, "grad_w"},
         {a->grad_z, BT * a->Hv * a->dv * 4, "grad_z"}, {a->grad_h0, st, "grad_h0"},
+        {a->grad_norm_w, (size_t)a->dv * 4, "grad_norm_w"},
     };
-    if ((s = check_buffers(in, 13, out, 9))) return s;
+    if ((s = check_buffers(in, 14, out, 10))) return s;
     if (a->fwd_cache) {
         if (!layer_bwd_tc_form(a))
             return fail(GDN_ERR_UNSUPPORTED, "fwd_cache: only the tensor-core form (bf16, d = 128, scalar gates, no h0) "
@@ -819,6 +853,11 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     lio.dxq = a->grad_xq; lio.dxk = a->grad_xk; lio.dxv = a->grad_xv;
     lio.wpart = at(plan.wpart); lio.dconv_w = a->grad_conv_w;
     lio.B = (int)a->B; lio.T = (int)a->T; lio.Hk = (int)a->Hk; lio.Hv = (int)a->Hv; lio.d = (int)a->dk;
+    lio.norm_w = a->norm_w;
+    lio.norm_w_f32 = a->dtype == GDN_F32;
+    lio.norm_eps = a->norm_eps;
+    lio.npart = a->norm_w ? at(plan.npart) : nullptr;
+    lio.dnorm_w = a->grad_norm_w;
     ChunkIO io{};
     io.alpha = a->alpha; io.b = a->b; io.w = a->w; io.h0 = a->h0;
     if (plan.tc) {

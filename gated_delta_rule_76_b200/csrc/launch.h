@@ -101,8 +101,17 @@ struct LayerBwdIO {
     float *dxq, *dxk, *dxv;             // out: gradients of the conv inputs
     float *wpart, *dconv_w;             // per-tile partial sums of the conv-weight gradient; out
     int B, T, Hk, Hv, d;
+    // the output norm (y = RMSNorm(o) * norm_w * swish(z)), or norm_w NULL: y = o * swish(z)
+    const void* norm_w;
+    int norm_w_f32;
+    float norm_eps;
+    float *npart, *dnorm_w;             // per-warp partials of the norm weights' gradient; out [d]
 };
 size_t layer_bwd_wpart_floats(int B, int T, int Hk, int Hv, int d);
+size_t layer_norm_partials_floats(int d);
+// y = RMSNorm(o) * norm_w * swish(z) over rows of d values (o fp32; z, y in the layer dtype, or y fp32)
+cudaError_t layer_norm_gate_fwd(const float* o, const void* z, const void* norm_w, int norm_w_f32, float eps,
+                                void* y, int y_f32, bool bf16, long rows, int d, cudaStream_t st);
 cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
 cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
 // dst[i] += src[i], i < n (the two halves of a gradient computed from hi and lo cotangents).

@@ -1,8 +1,10 @@
-// Backward of the GQA layer core's elementwise parts: the swish(z) output gate, and the causal
-// depthwise convolution (kernel 4, zero history) + SiLU + L2 norm in front of the recurrence
-// (explainer «Architecture et versions hybrides», Figure 1 caption; mkdocs chapter «Gated
-// DeltaNet», «La convolution causale», «La porte de sortie»).  The recurrence's own backward is
-// the chunk backward; gdn_layer_core_bwd (gdn_api.cu) chains the pieces.
+// The GQA layer core's parts around the recurrence: the output norm and swish(z) gate (forward for
+// the CUDA-core form, whose chunk kernels split a row's columns over CTAs; the tensor-core forward
+// fuses them in its epilogue), and the backward of the gate, the norm, and the causal depthwise
+// convolution (kernel 4, zero history) + SiLU + L2 norm in front of the recurrence (explainer
+// «Architecture et versions hybrides», Figure 1 caption; mkdocs chapter «Gated DeltaNet», «La
+// convolution causale», «La porte de sortie», «Le décompte»).  The recurrence's own backward is the
+// chunk backward; gdn_layer_core_bwd (gdn_api.cu) chains the pieces.
 #include <cuda_runtime.h>
 
 #include <type_traits>
@@ -30,6 +32,108 @@ __global__ void __launch_bounds__(256) swish_gate_bwd_kernel(const float* __rest
         if (dout_lo) dout_lo[i] = from_f32<TO>(d - to_f32(hi));
         dz[i] = g * o[i] * (s + zz * s * (1.f - s));
     }
+}
+
+// ---- output norm + gate: one warp per (token, head) row of D values, lane l owns D/32 of them ------
+// forward   y = n * wn * swish(z),  n = o * r,  r = (mean_j o_j^2 + eps)^(-1/2)
+// backward  dn = dy * wn * swish(z),  dz = dy * n * wn * swish'(z),  dwn += dy * n * swish(z),
+//           do = r * (dn - n * mean_j(dn * n))
+constexpr int kNormBlocks = 148 * 8;  // 8 warps each: the backward's per-warp partials of dwn
+constexpr int kNormWarps = kNormBlocks * 8;
+
+__device__ __forceinline__ float warp_sum_all(float x) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+__device__ __forceinline__ float norm_weight(const void* w, int f32, int c) {
+    return f32 ? static_cast<const float*>(w)[c] : __bfloat162float(static_cast<const __nv_bfloat16*>(w)[c]);
+}
+
+template <class T, class TO, int D>
+__global__ void __launch_bounds__(256) rmsnorm_gate_fwd_kernel(const float* __restrict__ o, const T* __restrict__ z,
+                                                               const void* norm_w, int norm_w_f32, float eps,
+                                                               TO* __restrict__ y, long rows) {
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    float wn[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) wn[i] = norm_weight(norm_w, norm_w_f32, PER * lane + i);
+    for (long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5); row < rows; row += (long)gridDim.x * 8) {
+        const long base = row * D + PER * lane;
+        float ov[PER], ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            ov[i] = o[base + i];
+            ss += ov[i] * ov[i];
+        }
+        const float r = rsqrtf(warp_sum_all(ss) * (1.f / D) + eps);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const float zz = to_f32(z[base + i]);
+            y[base + i] = from_f32<TO>(ov[i] * r * wn[i] * zz * sigmoid_fast(zz));
+        }
+    }
+}
+
+// With dout_lo (bf16 outputs only), do is stored as hi = bf16(do) and lo = bf16(do - hi).  npart
+// receives each warp's partial sums of dwn ([kNormWarps][D]), reduced by sum_partials_kernel.
+template <class T, class TO, int D>
+__global__ void __launch_bounds__(256) rmsnorm_gate_bwd_kernel(const float* __restrict__ o, const T* __restrict__ z,
+                                                               const T* __restrict__ dy, const void* norm_w,
+                                                               int norm_w_f32, float eps, TO* __restrict__ dout,
+                                                               TO* __restrict__ dout_lo, float* __restrict__ dz,
+                                                               float* __restrict__ npart, long rows) {
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long gw = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    float wn[PER], dwn[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        wn[i] = norm_weight(norm_w, norm_w_f32, PER * lane + i);
+        dwn[i] = 0.f;
+    }
+    for (long row = gw; row < rows; row += (long)gridDim.x * 8) {
+        const long base = row * D + PER * lane;
+        float n[PER], dn[PER], ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            n[i] = o[base + i];
+            ss += n[i] * n[i];
+        }
+        const float r = rsqrtf(warp_sum_all(ss) * (1.f / D) + eps);
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            n[i] *= r;
+            const float zz = to_f32(z[base + i]), g = to_f32(dy[base + i]);
+            const float s = sigmoid_fast(zz), sw = zz * s;
+            dn[i] = g * wn[i] * sw;
+            dz[base + i] = g * n[i] * wn[i] * (s + zz * s * (1.f - s));
+            dwn[i] = fmaf(g * n[i], sw, dwn[i]);
+            m += dn[i] * n[i];
+        }
+        m = warp_sum_all(m) * (1.f / D);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const float d = r * (dn[i] - n[i] * m);
+            const TO hi = from_f32<TO>(d);
+            dout[base + i] = hi;
+            if (dout_lo) dout_lo[base + i] = from_f32<TO>(d - to_f32(hi));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) npart[gw * D + PER * lane + i] = dwn[i];
+}
+
+// out[j] = sum over partials p of part[p][j], one thread per j (a fixed order: deterministic).
+__global__ void __launch_bounds__(256) sum_partials_kernel(const float* __restrict__ part, float* __restrict__ out,
+                                                          long nj, int np) {
+    const long j = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= nj) return;
+    float s = 0.f;
+    for (int p = 0; p < np; ++p) s += part[(long)p * nj + j];
+    out[j] = s;
 }
 
 constexpr int kTile = 64;  // tokens per warp
@@ -213,8 +317,28 @@ cudaError_t conv_bwd_t(const LayerBwdIO& io, cudaStream_t st) {
                          io.dconv_w, nj, io.B * ntile);
 }
 
+template <class T, int D>
+cudaError_t norm_gate_bwd_t(const LayerBwdIO& io, cudaStream_t st) {
+    const long rows = (long)io.B * io.T * io.Hv;
+    const T* z = static_cast<const T*>(io.z);
+    const T* dy = static_cast<const T*>(io.dy);
+    cudaError_t e;
+    if (io.dout16)
+        e = launch_kernel(rmsnorm_gate_bwd_kernel<T, __nv_bfloat16, D>, dim3(kNormBlocks), dim3(256), 0, st,
+                          (const float*)io.o, z, dy, io.norm_w, io.norm_w_f32, io.norm_eps, io.dout16, io.dout16_lo,
+                          io.dz, io.npart, rows);
+    else
+        e = launch_kernel(rmsnorm_gate_bwd_kernel<T, float, D>, dim3(kNormBlocks), dim3(256), 0, st,
+                          (const float*)io.o, z, dy, io.norm_w, io.norm_w_f32, io.norm_eps, io.dout, (float*)nullptr,
+                          io.dz, io.npart, rows);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(sum_partials_kernel, dim3((unsigned)((D + 255) / 256)), dim3(256), 0, st,
+                         (const float*)io.npart, io.dnorm_w, (long)D, kNormWarps);
+}
+
 template <class T>
 cudaError_t gate_bwd_t(const LayerBwdIO& io, cudaStream_t st) {
+    if (io.norm_w) return io.d == 128 ? norm_gate_bwd_t<T, 128>(io, st) : norm_gate_bwd_t<T, 64>(io, st);
     const long n = (long)io.B * io.T * io.Hv * io.d;
     const long blocks = (n + 255) / 256 < 148L * 32 ? (n + 255) / 256 : 148L * 32;
     if (io.dout16)
@@ -226,6 +350,25 @@ cudaError_t gate_bwd_t(const LayerBwdIO& io, cudaStream_t st) {
 }
 
 }  // namespace
+
+size_t layer_norm_partials_floats(int d) { return (size_t)kNormWarps * d; }
+
+cudaError_t layer_norm_gate_fwd(const float* o, const void* z, const void* norm_w, int norm_w_f32, float eps,
+                                void* y, int y_f32, bool bf16, long rows, int d, cudaStream_t st) {
+    const long blocks = (rows + 7) / 8 < kNormBlocks ? (rows + 7) / 8 : kNormBlocks;
+    const dim3 grid((unsigned)(blocks > 0 ? blocks : 1));
+#define GDN_NG(T, TO, D)                                                                                   \
+    return launch_kernel(rmsnorm_gate_fwd_kernel<T, TO, D>, grid, dim3(256), 0, st, o, static_cast<const T*>(z), \
+                         norm_w, norm_w_f32, eps, static_cast<TO*>(y), rows)
+    if (bf16) {
+        if (d == 128) { if (y_f32) GDN_NG(__nv_bfloat16, float, 128); GDN_NG(__nv_bfloat16, __nv_bfloat16, 128); }
+        if (y_f32) GDN_NG(__nv_bfloat16, float, 64);
+        GDN_NG(__nv_bfloat16, __nv_bfloat16, 64);
+    }
+    if (d == 128) GDN_NG(float, float, 128);
+    GDN_NG(float, float, 64);
+#undef GDN_NG
+}
 
 size_t layer_bwd_wpart_floats(int B, int T, int Hk, int Hv, int d) {
     return (size_t)B * ((T + kTile - 1) / kTile) * (2 * (size_t)Hk * d + (size_t)Hv * d) * 4;

@@ -74,6 +74,9 @@ cudaError_t seq_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32,
     p.o = io.o;
     p.o_type = io.o_type;
     p.o_raw = f.gate ? o_raw : nullptr;
+    p.norm_w = f.gate ? io.norm_w : nullptr;
+    p.norm_w_f32 = io.norm_w_f32;
+    p.norm_eps = io.norm_eps;
     p.ht = io.ht;
     return dispatch(tin_f32, tg_f32, pb.dk, [&](auto tin, auto tg, auto d) {
         return launch_seq_fwd<typename decltype(tin)::type, typename decltype(tg)::type, decltype(d)::value>(p, st);

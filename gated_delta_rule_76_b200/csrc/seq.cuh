@@ -51,6 +51,9 @@ struct Params {
     void* o;                                 // [B,T,Hv,dv], or NULL
     int o_type;                              // 0: TIn, 1: fp32, 2: bf16
     float* o_raw;                            // with z: the output before the gate (fp32), or NULL
+    const void* norm_w;                      // with z: the output norm's weights [dv] (bf16 unless
+    int norm_w_f32;                          //   norm_w_f32), or NULL: no norm
+    float norm_eps;
     float* ht;                               // [B,Hv,dk,dv] or NULL
     // backward
     const void* dout;                        // [B,T,Hv,dv] TIn
@@ -174,7 +177,7 @@ __device__ __forceinline__ void store_out(const Params& p, long off, float x) {
 // ------------------------------------------------------------------------------------------
 template <int D>
 constexpr size_t seq_fwd_smem() {
-    return (size_t)2 * kTB * NVEC * D * sizeof(float) + 2 * kTB * 2 * sizeof(float);
+    return (size_t)2 * kTB * NVEC * D * sizeof(float) + 2 * kTB * 2 * sizeof(float) + 2 * 16 * sizeof(float);
 }
 
 template <class TIn, class TG, int D>
@@ -183,12 +186,17 @@ __global__ void __launch_bounds__(2 * D) seq_fwd_kernel(Params p) {
     extern __shared__ float4 smem_f4[];
     float* stage = reinterpret_cast<float*>(smem_f4);       // [2][kTB][NVEC][D]
     float* scal = stage + 2 * kTB * NVEC * D;               // [2][kTB][2]
+    float* nred = scal + 2 * kTB * 2;                       // [2 token parities][NTH / 32 warps]
     const Problem& pb = p.pb;
     const int pair = blockIdx.x;
     if (p.flags && !p.flags[pair]) return;
     const int b = pair / pb.Hv, hv = pair % pb.Hv, hk = pb.key_head(hv);
     const int tid = threadIdx.x;
     const int h = (tid >> 4) & 1, j = (tid & 15) + 16 * (tid >> 5);
+    const bool norm = p.z && p.norm_w;
+    const float wn = !norm ? 1.f
+                           : p.norm_w_f32 ? static_cast<const float*>(p.norm_w)[j]
+                                          : __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[j]);
     const int r0 = R * h;
     const long soff = pb.state_off(b, hv);
 
@@ -237,13 +245,28 @@ __global__ void __launch_bounds__(2 * D) seq_fwd_kernel(Params p) {
                 o = fmaf(qq.w, S[i + 3], o);
             }
             o += __shfl_xor_sync(0xffffffffu, o, 16);
+            float ov = pb.scale * o;
+            float rs = 1.f;
+            if (norm) {
+                // the row's sum of squares over the D columns: 16 columns per warp (each held by the
+                // two halves), then the warps' partials through shared memory (one barrier a token)
+                float sq = ov * ov;
+#pragma unroll
+                for (int m = 1; m < 16; m <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, m);
+                float* nr = nred + (t & 1) * 16;
+                if ((tid & 31) == 0) nr[tid >> 5] = sq;
+                __syncthreads();
+                float tot = 0.f;
+#pragma unroll
+                for (int w8 = 0; w8 < NTH / 32; ++w8) tot += nr[w8];
+                rs = rsqrtf(tot * (1.f / D) + p.norm_eps);
+            }
             if (h == 0 && p.o) {
-                float ov = pb.scale * o;
                 const long off = pb.v_row(b, t, hv) + j;
                 if (p.z) {
                     if (p.o_raw) p.o_raw[off] = ov;
                     const float zz = x[V_X * D + j];
-                    ov *= zz * sigmoidf_(zz);
+                    ov *= rs * wn * zz * sigmoidf_(zz);
                 }
                 store_out<TIn>(p, off, ov);
             }

@@ -58,6 +58,11 @@ struct ChunkIO {
     void* o;
     int o_type;  // 0: o in TIn, 1: fp32, 2: bf16
     int z_bf16;  // z stored as bf16 (else as TIn)
+    // The layer's output norm before the gate (tensor-core forward and sequential kernels only):
+    // weights [dv] (bf16 unless norm_w_f32), or NULL
+    const void* norm_w;
+    int norm_w_f32;
+    float norm_eps;
     float* ht;
     const void* dout;
     const float* dht;

@@ -98,7 +98,8 @@ constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, abort fl
 constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: alpha products per row group [8][128], then the
                                           // block-row products of the solve [16][LDR]
 constexpr uint32_t SM_SG = SM_RS + 4096;  // scalar gates of a chunk: [2 slots][alpha, beta][64] fp32
-constexpr uint32_t SM_END = SM_SG + 1024;
+constexpr uint32_t SM_NRM = SM_SG + 1024;  // output norm: [2 halves][4 warps][32 tokens] partial sums
+constexpr uint32_t SM_END = SM_NRM + 1024;
 constexpr int LDA = 68;  // fp32 row stride of the A/T scratch: float4 rows, rows 16 B apart in bank
 constexpr int LDR = 52;  // fp32 row stride of the block-row products
 constexpr size_t kSmemBytes = SM_END + 1024;
@@ -136,7 +137,31 @@ struct Params {
     __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
     float* o_raw;                // GATE only, may be NULL: the output before the gate, fp32 [B,T,Hv,dv]
     int* flags;                  // [B*Hv] or NULL: set for a pair with a chunk outside the decay range
+    // GATE only, may be NULL: the output norm before the gate (every (token, head) row of dv values
+    // divided by its root mean square, times norm_w[dv]); norm_w is bf16 unless norm_w_f32
+    const void* norm_w;
+    int norm_w_f32;
+    float norm_eps;
 };
+
+// Reduce-scatter of 32 values over the lanes of a warp: afterwards lane l holds the sum over the
+// warp of entry l.
+__device__ __forceinline__ float warp_reduce_scatter32(float (&x)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i < n / 2) {
+                const float send = upper ? x[i] : x[i + n / 2];
+                const float keep = upper ? x[i + n / 2] : x[i];
+                x[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+    }
+    return x[0];
+}
 
 __device__ __forceinline__ float bf(const uint8_t* tile, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
@@ -614,6 +639,24 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (i < nrow) rp[i * orow] = ov[i];
+                }
+                if (GATE && p.norm_w) {
+                    // token row 32h + i: sum of squares over the 128 columns = the 4 warps of this
+                    // half; lane l of each warp reduces token l over its 32 columns
+                    float sq[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) sq[i] = ov[i] * ov[i];
+                    float* nrm = reinterpret_cast<float*>(sm + SM_NRM);
+                    const int lane = tid & 31, w4 = (tid >> 5) & 3;
+                    nrm[(h * 4 + w4) * 32 + lane] = warp_reduce_scatter32(sq);
+                    named_bar(1, 256);
+                    const float tot = nrm[(h * 4) * 32 + lane] + nrm[(h * 4 + 1) * 32 + lane] +
+                                      nrm[(h * 4 + 2) * 32 + lane] + nrm[(h * 4 + 3) * 32 + lane];
+                    const float rs = rsqrtf(tot * (1.f / D) + p.norm_eps);
+                    const float wn = p.norm_w_f32 ? static_cast<const float*>(p.norm_w)[j]
+                                                  : __bfloat162float(static_cast<const __nv_bfloat16*>(p.norm_w)[j]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] *= __shfl_sync(0xffffffffu, rs, i) * wn;
                 }
                 if (GATE) {
                     // z column j, rows 32h .. 32h + 31, from the TMA tile (zero past the end)

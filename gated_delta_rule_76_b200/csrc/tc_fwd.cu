@@ -68,6 +68,9 @@ cudaError_t tc_chunk_fwd_kernel(const Problem& pb, const ChunkIO& io, Flags f, b
     p.ht = io.ht;
     p.err = err;
     p.flags = flags;
+    p.norm_w = f.gate ? io.norm_w : nullptr;
+    p.norm_w_f32 = io.norm_w_f32;
+    p.norm_eps = io.norm_eps;
     if (save) {
         p.s0_out = save->s0;
         p.vp_hi = save->vp_hi;

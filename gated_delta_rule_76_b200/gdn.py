@@ -59,7 +59,7 @@ class LayerArgs(ctypes.Structure):
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32), ("bwd_cache", P),
-                ("bwd_cache_bytes", ctypes.c_size_t)]
+                ("bwd_cache_bytes", ctypes.c_size_t), ("norm_w", P), ("norm_eps", F32)]
 
 
 class LayerBwdArgs(ctypes.Structure):
@@ -69,7 +69,8 @@ class LayerBwdArgs(ctypes.Structure):
                 ("grad_b", P), ("grad_w", P), ("grad_z", P), ("grad_h0", P),
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32), ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t)]
+                ("dtype", I32), ("gate_dtype", I32), ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t),
+                ("norm_w", P), ("norm_eps", F32), ("grad_norm_w", P)]
 
 
 EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
@@ -374,8 +375,11 @@ def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=N
     return o
 
 
+NORM_EPS = 1e-6  # the output norm's epsilon when the caller gives none
+
+
 def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y=None, ht=None, cs=None,
-                out_f32=0, bwd_cache=None):
+                out_f32=0, bwd_cache=None, norm_w=None, norm_eps=NORM_EPS):
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
@@ -385,25 +389,27 @@ def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y
                   conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
                   dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
                   gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha), out_f32=out_f32,
-                  bwd_cache=_ptr(bwd_cache), bwd_cache_bytes=bwd_cache.numel() if bwd_cache is not None else 0)
+                  bwd_cache=_ptr(bwd_cache), bwd_cache_bytes=bwd_cache.numel() if bwd_cache is not None else 0,
+                  norm_w=_ptr(norm_w), norm_eps=norm_eps)
     return a, hm
 
 
 def gdn_layer_core_fwd_cache_size(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, h0=None,
-                                  head_map=None, scale: float = 1.0) -> int:
+                                  head_map=None, scale: float = 1.0, norm_w=None) -> int:
     """Bytes of the layer forward's optional backward cache (0 where it cannot keep one)."""
-    a, _ = _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale)
+    a, _ = _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, norm_w=norm_w)
     return int(load().gdn_layer_core_fwd_cache_size(ctypes.byref(a)))
 
 
 def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, h0=None,
                        head_map=None, scale: float = 1.0, *, want_ht: bool = True,
                        want_conv_state: bool = False, y=None, out_f32: bool = False,
-                       bwd_cache: Optional[torch.Tensor] = None,
+                       bwd_cache: Optional[torch.Tensor] = None, norm_w=None, norm_eps: float = NORM_EPS,
                        workspace: Optional[torch.Tensor] = None, stream=None):
     """GQA layer core forward.  Returns (y, ht or None, conv_state or None).  ``bwd_cache``: a
     uint8 device tensor of gdn_layer_core_fwd_cache_size() bytes that a later
-    gdn_layer_core_bwd(..., fwd_cache=) over the same inputs reads."""
+    gdn_layer_core_bwd(..., fwd_cache=) over the same inputs reads.  ``norm_w`` [dv] (the layer's
+    dtype): the output norm before the gate, y = RMSNorm(o) * norm_w * swish(z)."""
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
     if y is None:
@@ -412,7 +418,8 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
     cs = (torch.empty((B, 2 * Hk * dk + Hv * dv, 3), dtype=xq.dtype, device=xq.device)
           if want_conv_state else None)
     a, hm = _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y=y, ht=ht, cs=cs,
-                        out_f32=int(y.dtype == torch.float32 and xq.dtype != torch.float32), bwd_cache=bwd_cache)
+                        out_f32=int(y.dtype == torch.float32 and xq.dtype != torch.float32), bwd_cache=bwd_cache,
+                        norm_w=norm_w, norm_eps=norm_eps)
     lib = load()
     need = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, xq.device, workspace)
@@ -423,10 +430,11 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
 
 def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, beta=None, h0=None,
                        grad_ht=None, head_map=None, scale: float = 1.0, *, want_h0_grad: bool = True,
-                       fwd_cache: Optional[torch.Tensor] = None,
+                       fwd_cache: Optional[torch.Tensor] = None, norm_w=None, norm_eps: float = NORM_EPS,
                        workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
     """GQA layer core backward (reverse mode of gdn_layer_core_fwd).  Returns a dict of fp32
-    gradients: dxq, dxk, dxv, dconv_w, dalpha, dz, dh0 (or None) and db/dw or dbeta.
+    gradients: dxq, dxk, dxv, dconv_w, dalpha, dz, dh0 (or None), db/dw or dbeta, and dnorm_w
+    with the output norm (``norm_w``).
     ``fwd_cache``: the cache a gdn_layer_core_fwd(..., bwd_cache=) call filled with these inputs."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = xq.shape
@@ -444,6 +452,8 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
     else:
         out["dbeta"] = torch.empty(tuple(bb.shape), **f32)
         gb, gw = out["dbeta"], None
+    if norm_w is not None:
+        out["dnorm_w"] = torch.empty((dv,), **f32)
     hm = _head_map(head_map, dev, Hk)
     a = LayerBwdArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
                      b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), head_map=_ptr(hm), grad_y=_ptr(grad_y),
@@ -453,7 +463,8 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
                      B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                      alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc, dtype=_dt(xq),
                      gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
-                     fwd_cache_bytes=fwd_cache.numel() if fwd_cache is not None else 0)
+                     fwd_cache_bytes=fwd_cache.numel() if fwd_cache is not None else 0,
+                     norm_w=_ptr(norm_w), norm_eps=norm_eps, grad_norm_w=_ptr(out.get("dnorm_w")))
     lib = load()
     need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, dev, workspace)

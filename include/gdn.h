@@ -293,6 +293,14 @@ typedef struct gdn_layer_args {
      * elsewhere the size is 0 and bwd_cache must be NULL. */
     void* bwd_cache;
     size_t bwd_cache_bytes;
+    /* Optional output norm before the gate (explainer «Architecture et versions hybrides», Figure 1
+     * caption: the output is normalised, then multiplied by a gate; mkdocs chapter «Gated
+     * DeltaNet», «Le décompte»: dv norm weights shared by the heads).  When norm_w [dv] (dtype) is
+     * not NULL: y = o / sqrt(mean_j o_j^2 + norm_eps) * norm_w * z * sigmoid(z) for every
+     * (token, value head) row o of dv values.  NULL: y = o * z * sigmoid(z).  The cache keeps o
+     * before the norm. */
+    const void* norm_w;
+    float norm_eps;
 } gdn_layer_args;
 
 /* Bytes of the optional layer forward cache (0 where the layer backward cannot use one). */
@@ -355,6 +363,11 @@ typedef struct gdn_layer_bwd_args {
      * gradients.  NULL: the forward parts are recomputed. */
     const void* fwd_cache;
     size_t fwd_cache_bytes;
+    /* The output norm of gdn_layer_args (NULL: none).  With it, grad_norm_w [dv] fp32 is required and
+     * receives the norm weights' gradient, summed over tokens and heads in a fixed order. */
+    const void* norm_w;
+    float norm_eps;
+    float* grad_norm_w;
 } gdn_layer_bwd_args;
 
 GDN_API size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* args);
