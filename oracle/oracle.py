@@ -198,6 +198,44 @@ def chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
     return o, hT
 
 
+# ---- gates from logits -----------------------------------------------------------------------
+# The gates as functions of the layer's projections (explainer «Architecture et versions hybrides»,
+# Figure 1 caption: alpha takes the Mamba-2 parametrisation; zubnet.ai news item: the erase and write
+# gates are two sigmoids): alpha = exp(-a_h softplus(x)) with a positive scale a_h per value head (the
+# Mamba-2 form exp(-A dt), dt = softplus(x), A = a_h), and b, w, beta = sigmoid(x).
+
+def _softplus(x):
+    return np.logaddexp(0.0, x)
+
+
+def gates_from_logits(x_alpha, a_scale, x_b=None, x_w=None, x_beta=None):
+    """(alpha, b, w, beta) from their logits; a_scale [Hv] (alpha's last axis is the channel axis when
+    it has one, the value head is axis 2)."""
+    xa = f64(x_alpha)
+    a = f64(a_scale)
+    ah = a.reshape((1, 1, -1) + (1,) * (xa.ndim - 3))
+    alpha = np.exp(-ah * _softplus(xa))
+    sig = lambda x: None if x is None else _sigmoid(f64(x))
+    return alpha, sig(x_b), sig(x_w), sig(x_beta)
+
+
+def logit_grads(x_alpha, a_scale, dalpha, x_b=None, db=None, x_w=None, dw=None, x_beta=None, dbeta=None):
+    """Chain rule from the gradients of the gates to those of their logits and of a_h:
+        d x_alpha = dalpha * alpha * (-a_h sigmoid(x)),   d a_h = sum dalpha * alpha * (-softplus(x)),
+        d x = dg * g (1 - g) for the sigmoid gates."""
+    xa, a = f64(x_alpha), f64(a_scale)
+    ah = a.reshape((1, 1, -1) + (1,) * (xa.ndim - 3))
+    alpha = np.exp(-ah * _softplus(xa))
+    out = {"dalpha": f64(dalpha) * alpha * (-ah * _sigmoid(xa))}
+    axes = (0, 1) + tuple(range(3, xa.ndim))
+    out["dalpha_scale"] = np.sum(f64(dalpha) * alpha * (-_softplus(xa)), axis=axes)
+    for name, x, d in (("db", x_b, db), ("dw", x_w, dw), ("dbeta", x_beta, dbeta)):
+        if x is not None:
+            g = _sigmoid(f64(x))
+            out[name] = f64(d) * g * (1.0 - g)
+    return out
+
+
 def segment_map(q, k, v, alpha, b=None, w=None, beta=None, head_map=None):
     """The affine map by which one segment of a sequence acts on the state.
 

@@ -599,3 +599,62 @@ def test_layer_backward_with_output_norm_finite_differences():
             fd[idx] = (loss(plus) - loss(minus)) / (2 * h)
         err = np.max(np.abs(g[key[n]] - fd)) / max(np.max(np.abs(fd)), 1e-12)
         assert err < 1e-6, (n, err)
+
+
+# ---- gates from logits -----------------------------------------------------------------------------
+def test_gates_from_logits_closed_forms():
+    """alpha = exp(-a softplus(x)): at x = 0 it is 2^-a; a = 0.1 is the input recipe's decay; the
+    sigmoid gates are 1/2 at 0 and symmetric."""
+    x = np.zeros((1, 2, 3, 4))
+    a, b, w, _ = oracle.gates_from_logits(x, np.array([0.1, 1.0, 2.0]), x_b=x, x_w=-x)
+    assert np.allclose(a[0, 0, :, 0], [2 ** -0.1, 0.5, 0.25], rtol=0, atol=1e-15)
+    assert np.all(b == 0.5) and np.all(w == 0.5)
+    rng = np.random.default_rng(77)
+    xr = rng.standard_normal((2, 3, 4))
+    _, _, _, beta = oracle.gates_from_logits(xr, np.ones(4), x_beta=xr)
+    _, _, _, beta_m = oracle.gates_from_logits(xr, np.ones(4), x_beta=-xr)
+    assert np.allclose(beta + beta_m, 1.0, atol=1e-15)
+
+
+@pytest.mark.parametrize("channel", [True, False])
+def test_logit_gradients_finite_differences(channel):
+    """The recurrence's gradients pushed through the gate functions, against central differences of
+    a loss of the outputs computed from the logits."""
+    rng = np.random.default_rng(78)
+    B, T, Hk, Hv, d = 1, 7, 1, 2, 4
+    x = rand_inputs(rng, B, T, Hk, Hv, d, d, channel_alpha=channel, channel_gates=channel, h0=True)
+    xa = rng.standard_normal(x["alpha"].shape)
+    a_scale = np.array([0.3, 1.7])
+    lg = {"x_b": rng.standard_normal(x["b"].shape), "x_w": rng.standard_normal(x["w"].shape)} if channel else \
+         {"x_beta": rng.standard_normal(x["beta"].shape)}
+    dout = rng.standard_normal((B, T, Hv, d))
+
+    def loss(xa_, a_, lg_):
+        al, b, w, beta = oracle.gates_from_logits(xa_, a_, **lg_)
+        gk = dict(b=b, w=w) if channel else dict(beta=beta)
+        o, _ = oracle.fwd(x["q"], x["k"], x["v"], al, h0=x["h0"], nthreads=1, **gk)
+        return np.sum(o * dout)
+
+    al, b, w, beta = oracle.gates_from_logits(xa, a_scale, **lg)
+    gk = dict(b=b, w=w) if channel else dict(beta=beta)
+    g = oracle.bwd(x["q"], x["k"], x["v"], al, h0=x["h0"], dout=dout, **gk)
+    if channel:
+        lgr = oracle.logit_grads(xa, a_scale, g["dalpha"], x_b=lg["x_b"], db=g["db"], x_w=lg["x_w"], dw=g["dw"])
+    else:
+        lgr = oracle.logit_grads(xa, a_scale, g["dalpha"], x_beta=lg["x_beta"], dbeta=g["dbeta"])
+    h = 1e-6
+    checks = [("dalpha", xa, lambda v: loss(v, a_scale, lg)),
+              ("dalpha_scale", a_scale, lambda v: loss(xa, v, lg))]
+    for name, key in (("db", "x_b"), ("dw", "x_w"), ("dbeta", "x_beta")):
+        if key in lg:
+            checks.append((name, lg[key], lambda v, key=key: loss(xa, a_scale, {**lg, key: v})))
+    for name, base, f in checks:
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            p, m = base.copy(), base.copy()
+            p[idx] += h
+            m[idx] -= h
+            fd[idx] = (f(p) - f(m)) / (2 * h)
+        assert relerr(lgr[name], fd) < 1e-6, name
