@@ -27,6 +27,21 @@ struct Problem {
     int NT;         // number of chunks, ceil(T / 64)
     float scale;
     const int32_t* head_map;  // may be null: hv / (Hv / Hk)
+    // Gates given as logits x (explainer «Architecture et versions hybrides», Figure 1 caption: alpha
+    // takes the Mamba-2 parametrisation; zubnet.ai news item: two sigmoid gates):
+    //   alpha = exp(-alpha_scale[hv] softplus(x)),  b, w, beta = sigmoid(x).
+    // Every kernel applies the transform where it reads a gate, in fp32.
+    int gate_logits;
+    const float* alpha_scale;  // [Hv] fp32 (gate_logits only)
+
+    __device__ __forceinline__ float alpha_of(int hv, float x) const {
+        if (!gate_logits) return x;
+        const float sp = fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));  // softplus(x)
+        return expf(-__ldg(alpha_scale + hv) * sp);
+    }
+    __device__ __forceinline__ float sig_of(float x) const {
+        return gate_logits ? 1.f / (1.f + expf(-x)) : x;
+    }
 
     // An explicit map entry outside [0, Hk) breaks the interface's precondition; it is clamped
     // into range so that no kernel reads outside q or k (the result is then unspecified).
@@ -54,10 +69,13 @@ struct Problem {
 // past the end of the sequence.  The load itself is unconditional, from the row clamped to the
 // last token: a load under a branch is waited for where the branch ends, which would serialise
 // the loads of an unrolled loop.
+// kind: 0 the value as stored, 1 a decay alpha, 2 a sigmoid gate (the transforms of gate logits).
 template <class TG>
 __device__ __forceinline__ float gate_or(const TG* g, const Problem& pb, int b, int t0, int r, int L, int hv,
-                                         float fill) {
-    const float x = to_f32(__ldg(g + pb.gate_row(b, t0 + (r < L ? r : L - 1), hv, 1)));
+                                         float fill, int kind = 0) {
+    float x = to_f32(__ldg(g + pb.gate_row(b, t0 + (r < L ? r : L - 1), hv, 1)));
+    if (kind == 1) x = pb.alpha_of(hv, x);
+    else if (kind == 2) x = pb.sig_of(x);
     return r < L ? x : fill;
 }
 

@@ -21,6 +21,8 @@ struct DecodeParams {
     const void* conv_state; const void* conv_w; const void* z;
     int N, Hk, Hv, dk, dv;
     float scale;
+    int gate_logits;           // gates as logits: alpha = exp(-alpha_scale[hv] softplus(x)), sigmoid b, w
+    const float* alpha_scale;  // [Hv] fp32 (gate_logits only)
 };
 
 template <class TIn, class TG, bool APC, bool GPC, int DK, int DV, bool CONV, bool GATE>
@@ -39,6 +41,11 @@ decode_step_kernel(DecodeParams p) {
     const int hv = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
     // a map entry outside [0, Hk) breaks the precondition: clamped, so no read leaves q or k
     const int hk = p.head_map ? min(max(__ldg(p.head_map + hv), 0), p.Hk - 1) : hv / (p.Hv / p.Hk);
+    auto alpha_of = [&](float x) {
+        if (!p.gate_logits) return x;
+        return expf(-__ldg(p.alpha_scale + hv) * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)))));
+    };
+    auto sig_of = [&](float x) { return p.gate_logits ? 1.f / (1.f + expf(-x)) : x; };
     const TIn* q = static_cast<const TIn*>(p.q) + ((long)n * p.Hk + hk) * DK;
     const TIn* k = static_cast<const TIn*>(p.k) + ((long)n * p.Hk + hk) * DK;
     const TIn* v = static_cast<const TIn*>(p.v) + ((long)n * p.Hv + hv) * DV;
@@ -82,10 +89,10 @@ decode_step_kernel(DecodeParams p) {
         __syncthreads();
     }
     for (int i = tid; i < DK; i += NTH) {
-        as_[i] = to_f32(al[APC ? i : 0]);
-        es[i] = to_f32(bg[GPC ? i : 0]) * ks[i];
+        as_[i] = alpha_of(to_f32(al[APC ? i : 0]));
+        es[i] = sig_of(to_f32(bg[GPC ? i : 0])) * ks[i];
     }
-    for (int j = tid; j < DV; j += NTH) zs[j] *= to_f32(wg[GPC ? j : 0]);
+    for (int j = tid; j < DV; j += NTH) zs[j] *= sig_of(to_f32(wg[GPC ? j : 0]));
     __syncthreads();
 
     // ---- state read, decay, erase read-out ---------------------------------------------

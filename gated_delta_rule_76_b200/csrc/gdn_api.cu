@@ -95,7 +95,7 @@ gdn_status check_common(int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk
 
 Problem make_problem(int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, int64_t dv,
                      float scale, const int32_t* head_map) {
-    Problem pb;
+    Problem pb{};
     pb.B = (int)B; pb.T = (int)T; pb.Hk = (int)Hk; pb.Hv = (int)Hv; pb.dk = (int)dk; pb.dv = (int)dv;
     pb.NT = (int)((T + kChunk - 1) / kChunk);
     pb.scale = scale;
@@ -104,6 +104,19 @@ Problem make_problem(int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, i
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Gates as logits: the flag and alpha's per-head scale (grad: the scale's gradient, optional).
+gdn_status check_logits(int32_t gate_logits, const float* alpha_scale, const float* grad_alpha_scale = nullptr) {
+    if (gate_logits != 0 && gate_logits != 1) return fail(GDN_ERR_INVALID_ARG, "gate_logits must be 0 or 1");
+    if (gate_logits && !alpha_scale) return fail(GDN_ERR_INVALID_ARG, "alpha_scale is required with gate_logits");
+    if (!gate_logits && (alpha_scale || grad_alpha_scale))
+        return fail(GDN_ERR_INVALID_ARG, "alpha_scale and grad_alpha_scale must be NULL without gate_logits");
+    return GDN_OK;
+}
+void apply_logits(Problem& pb, int32_t gate_logits, const float* alpha_scale) {
+    pb.gate_logits = gate_logits;
+    pb.alpha_scale = gate_logits ? alpha_scale : nullptr;
+}
 
 int variant(int32_t dtype, int32_t gate_dtype) {
     if (dtype == GDN_F32) return 2;
@@ -192,8 +205,10 @@ gdn_status check_fwd(const gdn_fwd_args* a, bool need_o = true) {
         {a->h0, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "h0"},
         {a->z, BT * a->Hv * a->dv * es, "z"},
         {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        {a->alpha_scale, (size_t)a->Hv * 4, "alpha_scale"},
     };
     if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
+    if ((s = check_logits(a->gate_logits, a->alpha_scale))) return s;
     const Buf out[] = {
         {a->o, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "o"},
         {a->ht, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "ht"},
@@ -201,7 +216,7 @@ gdn_status check_fwd(const gdn_fwd_args* a, bool need_o = true) {
     };
     if (a->bwd_cache && (reinterpret_cast<uintptr_t>(a->bwd_cache) & 255u))
         return fail(GDN_ERR_INVALID_ARG, "bwd_cache is not 256-byte aligned");
-    return check_buffers(in, 9, out, 3);
+    return check_buffers(in, 10, out, 3);
 }
 
 gdn_status check_bwd(const gdn_bwd_args* a) {
@@ -227,7 +242,9 @@ gdn_status check_bwd(const gdn_bwd_args* a) {
         {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_o, BT * a->Hv * a->dv * es, "grad_o"}, {a->grad_ht, st, "grad_ht"},
         {a->fwd_cache, a->fwd_cache ? a->fwd_cache_bytes : 0, "fwd_cache"},
+        {a->alpha_scale, (size_t)a->Hv * 4, "alpha_scale"},
     };
+    if ((s = check_logits(a->gate_logits, a->alpha_scale, a->grad_alpha_scale))) return s;
     if (a->fwd_cache && (reinterpret_cast<uintptr_t>(a->fwd_cache) & 255u))
         return fail(GDN_ERR_INVALID_ARG, "fwd_cache is not 256-byte aligned");
     const size_t na4 = na / gs * 4, nb4 = nb / gs * 4;
@@ -235,8 +252,9 @@ gdn_status check_bwd(const gdn_bwd_args* a) {
         {a->grad_q, BT * a->Hk * a->dk * 4, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * 4, "grad_k"},
         {a->grad_v, BT * a->Hv * a->dv * 4, "grad_v"}, {a->grad_alpha, na4, "grad_alpha"},
         {a->grad_b, nb4, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * 4, "grad_w"}, {a->grad_h0, st, "grad_h0"},
+        {a->grad_alpha_scale, (size_t)a->Hv * 4, "grad_alpha_scale"},
     };
-    return check_buffers(in, 11, out, 7);
+    return check_buffers(in, 12, out, 8);
 }
 
 gdn_status check_workspace(void* ws, size_t have, size_t need) {
@@ -323,6 +341,7 @@ static gdn_status chunk_fwd_core(const gdn_fwd_args* a, void* workspace, size_t 
     const size_t sbytes = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
     if (a->T == 0) return copy_state(a->ht, a->h0, sbytes, st, "gdn_chunk_fwd");
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    apply_logits(pb, a->gate_logits, a->alpha_scale);
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
     const bool tc = fwd_uses_tensor_cores(a, pb);
     if (a->bwd_cache) {
@@ -454,8 +473,15 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     if (s) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t sbytes = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
-    if (a->T == 0) return copy_state(a->grad_h0, a->grad_ht, sbytes, st, "gdn_chunk_bwd");
+    if (a->T == 0) {
+        if (a->grad_alpha_scale) {
+            cudaError_t e = cudaMemsetAsync(a->grad_alpha_scale, 0, (size_t)a->Hv * 4, st);
+            if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_bwd");
+        }
+        return copy_state(a->grad_h0, a->grad_ht, sbytes, st, "gdn_chunk_bwd");
+    }
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    apply_logits(pb, a->gate_logits, a->alpha_scale);
     const bool direct = identity_heads(pb);
     const bool tc = bwd_uses_tensor_cores(a, pb);
     WsPlan plan = plan_chunk_ws(pb, true, !direct);
@@ -480,14 +506,18 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     if (e != cudaSuccess) return cuda_fail(e, "gdn_chunk_bwd");
     if (tc) {
         e = tc_chunk_bwd(pb, io, f, a->gate_dtype == GDN_BF16, direct, tplan, workspace, a->fwd_cache, st);
-        return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_bwd");
+    } else {
+        ChunkWs ws = carve_chunk_ws(plan, workspace);
+        switch (variant(a->dtype, a->gate_dtype)) {
+            case 0: e = bf16_chunk_bwd(pb, io, ws, f, direct, st); break;
+            case 1: e = bf16_f32g_chunk_bwd(pb, io, ws, f, direct, st); break;
+            default: e = f32_chunk_bwd(pb, io, ws, f, direct, st); break;
+        }
     }
-    ChunkWs ws = carve_chunk_ws(plan, workspace);
-    switch (variant(a->dtype, a->gate_dtype)) {
-        case 0: e = bf16_chunk_bwd(pb, io, ws, f, direct, st); break;
-        case 1: e = bf16_f32g_chunk_bwd(pb, io, ws, f, direct, st); break;
-        default: e = f32_chunk_bwd(pb, io, ws, f, direct, st); break;
-    }
+    // gates as logits: the gradients of the gates become those of their logits
+    if (e == cudaSuccess && pb.gate_logits)
+        e = gate_logit_grads(pb, f, a->gate_dtype == GDN_F32, a->alpha, a->b, a->w, a->grad_alpha, a->grad_b,
+                             a->grad_w, a->grad_alpha_scale, st);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_bwd");
 }
 
@@ -525,6 +555,9 @@ gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
     p.conv_w = a->conv_w; p.z = a->z;
     p.N = (int)a->N; p.Hk = (int)a->Hk; p.Hv = (int)a->Hv; p.dk = (int)a->dk; p.dv = (int)a->dv;
     p.scale = a->scale;
+    if ((s = check_logits(a->gate_logits, a->alpha_scale))) return s;
+    p.gate_logits = a->gate_logits;
+    p.alpha_scale = a->gate_logits ? a->alpha_scale : nullptr;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, a->z != nullptr};
     cudaStream_t sm = static_cast<cudaStream_t>(stream);
     cudaError_t e;
@@ -614,6 +647,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
     if (a->norm_w && !(a->norm_eps >= 0.f && a->norm_eps < 1e30f))
         return fail(GDN_ERR_INVALID_ARG, "norm_eps must be a finite number >= 0");
+    if ((s = check_logits(a->gate_logits, a->alpha_scale))) return s;
     const Buf out[] = {
         {a->y, BT * a->Hv * a->dv * (a->out_f32 ? 4 : es), "y"}, {a->ht, st, "ht"},
         {a->conv_state_out, (size_t)a->B * cch * 3 * es, "conv_state_out"},
@@ -644,6 +678,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     const size_t conv_bytes = align256(BT * cch * 4);
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     // the chunk part of the workspace (after the conv results) holds the flag array in both forms
+    apply_logits(pb, a->gate_logits, a->alpha_scale);
     const WsPlan chunk_plan = plan_chunk_ws(pb, false, false);
     int* flags = carve_chunk_ws(chunk_plan, base + conv_bytes).flags;
     cudaError_t e0 = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), sm);
@@ -786,6 +821,7 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     if (!a->norm_w && a->grad_norm_w) return fail(GDN_ERR_INVALID_ARG, "grad_norm_w must be NULL without norm_w");
     if (a->norm_w && !(a->norm_eps >= 0.f && a->norm_eps < 1e30f))
         return fail(GDN_ERR_INVALID_ARG, "norm_eps must be a finite number >= 0");
+    if ((s = check_logits(a->gate_logits, a->alpha_scale, a->grad_alpha_scale))) return s;
     if (a->gates_per_channel ? (a->T > 0 && (!a->w || !a->grad_w)) : (a->w != nullptr || a->grad_w != nullptr))
         return fail(GDN_ERR_INVALID_ARG, "w and grad_w are required with channel gates and must be NULL otherwise");
     const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
@@ -829,6 +865,7 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
         return copy_state(a->grad_h0, a->grad_ht, st, sm, "gdn_layer_core_bwd");
     }
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
+    apply_logits(pb, a->gate_logits, a->alpha_scale);
     const LayerBwdPlan plan = plan_layer_bwd(a, pb);
     if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
     char* wsb = static_cast<char*>(workspace);
@@ -944,7 +981,12 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     }
     // 5. L2 norm, SiLU and conv backward, conv-weight gradient
     e = layer_conv_bwd(lio, bf16, sm);
-    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_bwd (conv)");
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
+    // 6. gates as logits: the gradients of the gates become those of their logits
+    if (pb.gate_logits)
+        e = gate_logit_grads(pb, f, a->gate_dtype == GDN_F32, a->alpha, a->b, a->w, a->grad_alpha, a->grad_b,
+                             a->grad_w, a->grad_alpha_scale, sm);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_bwd (gate logits)");
 }
 
 gdn_status gdn_workspace_status(const void* workspace, gdn_stream stream) {

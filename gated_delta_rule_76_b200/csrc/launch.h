@@ -66,6 +66,12 @@ cudaError_t seq_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32,
 cudaError_t seq_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
                     float* dq, float* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st);
 
+// Gates as logits (gates.cu): after a backward, the gates' gradients become those of their logits
+// (in place), and alpha's scale gets its gradient (dalpha_scale [Hv], may be NULL).
+cudaError_t gate_logit_grads(const Problem& pb, Flags f, bool tg_f32, const void* x_alpha, const void* x_b,
+                             const void* x_w, float* dalpha, float* db, float* dw, float* dalpha_scale,
+                             cudaStream_t st);
+
 // Sequence split along time (seqpar.cu): S = I for `pairs` states of d x d; S_out = op(M) S_in + N
 // per pair (op = transpose or not; S_in or N may be NULL: taken as zero).
 cudaError_t identity_states(float* S, long pairs, int d, cudaStream_t st);

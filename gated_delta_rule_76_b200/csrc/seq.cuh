@@ -97,9 +97,18 @@ struct Stager {
         long lo_off = 0;
         float4 x;
         switch (v) {
-            case V_A: return ld4(static_cast<const TG*>(p.alpha) + gc);
-            case V_B: return ld4(static_cast<const TG*>(p.b) + gc);
-            case V_W: return ld4(static_cast<const TG*>(p.w) + gc);
+            case V_A: {
+                float4 a = ld4(static_cast<const TG*>(p.alpha) + gc);
+                a.x = pb.alpha_of(hv, a.x); a.y = pb.alpha_of(hv, a.y);
+                a.z = pb.alpha_of(hv, a.z); a.w = pb.alpha_of(hv, a.w);
+                return a;
+            }
+            case V_B:
+            case V_W: {
+                float4 g = ld4(static_cast<const TG*>(v == V_B ? p.b : p.w) + gc);
+                g.x = pb.sig_of(g.x); g.y = pb.sig_of(g.y); g.z = pb.sig_of(g.z); g.w = pb.sig_of(g.w);
+                return g;
+            }
             case V_K: x = ld4(static_cast<const TIn*>(p.k) + qk); lo = static_cast<const __nv_bfloat16*>(p.k_lo); lo_off = qk; break;
             case V_Q: x = ld4(static_cast<const TIn*>(p.q) + qk); lo = static_cast<const __nv_bfloat16*>(p.q_lo); lo_off = qk; break;
             case V_V: x = ld4(static_cast<const TIn*>(p.v) + vv); lo = static_cast<const __nv_bfloat16*>(p.v_lo); lo_off = vv; break;
@@ -130,8 +139,8 @@ struct Stager {
         if (tid < kTB) {
             const bool in = t0 + tid < p.pb.T;
             const long g = p.pb.gate_row(b, in ? t0 + tid : 0, hv, 1);
-            scal[2 * tid] = in && !p.apc ? ld1(static_cast<const TG*>(p.alpha) + g) : 1.f;
-            scal[2 * tid + 1] = in && !p.gpc ? ld1(static_cast<const TG*>(p.b) + g) : 0.f;
+            scal[2 * tid] = in && !p.apc ? p.pb.alpha_of(hv, ld1(static_cast<const TG*>(p.alpha) + g)) : 1.f;
+            scal[2 * tid + 1] = in && !p.gpc ? p.pb.sig_of(ld1(static_cast<const TG*>(p.b) + g)) : 0.f;
         }
         __syncthreads();
 #pragma unroll

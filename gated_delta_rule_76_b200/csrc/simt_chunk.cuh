@@ -112,8 +112,8 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
                 const bool in = r < L;
                 kv[u] = in ? to_f32(k[pb.qk_row(b, t, hk) + c]) : 0.f;
                 qv[u] = in ? to_f32(q[pb.qk_row(b, t, hk) + c]) : 0.f;
-                av[u] = in ? to_f32(al[pb.gate_row(b, t, hv, APC ? DK : 1) + (APC ? c : 0)]) : 1.f;
-                bv[u] = in ? to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]) : 0.f;
+                av[u] = in ? pb.alpha_of(hv, to_f32(al[pb.gate_row(b, t, hv, APC ? DK : 1) + (APC ? c : 0)])) : 1.f;
+                bv[u] = in ? pb.sig_of(to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)])) : 0.f;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -231,7 +231,7 @@ chunk_scan_fwd_kernel(Problem pb, ChunkIO io, ChunkWs ws, int write_out, int sav
                 const int r = idx / W, j = idx % W, t = t0 + r;
                 if (r >= L) return 0.f;
                 return to_f32(vin[pb.v_row(b, t, hv) + j0 + j]) *
-                       to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
+                       pb.sig_of(to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]));
             },
             [&](int idx, float v) { Z[idx] = v; });
         if (save_states)
@@ -372,7 +372,7 @@ chunk_scan_bwd_kernel(Problem pb, ChunkIO io, ChunkWs ws) {
                 const int r = idx / W, j = idx % W, t = t0 + r;
                 if (r >= L) return 0.f;
                 return to_f32(vin[pb.v_row(b, t, hv) + j0 + j]) *
-                       to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
+                       pb.sig_of(to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]));
             },
             [&](int idx, float v) { Z[idx] = v; });
         cta_load<C * W>(
@@ -435,7 +435,7 @@ chunk_scan_bwd_kernel(Problem pb, ChunkIO io, ChunkWs ws) {
             if (r < L) {
                 const int t = t0 + r;
                 const long io_off = pb.v_row(b, t, hv) + j0 + j;
-                const float ww = to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]);
+                const float ww = pb.sig_of(to_f32(wg[pb.gate_row(b, t, hv, GPC ? dv : 1) + (GPC ? j0 + j : 0)]));
                 static_cast<float*>(io.dv)[io_off] = dY[idx] * ww;
                 if (GPC) static_cast<float*>(io.dw)[io_off] = dY[idx] * to_f32(vin[io_off]);
             }
@@ -620,7 +620,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
                     const int t = t0 + r;
                     const float de = v * Gm[r * DK + c];
                     const float kv = to_f32(kin[pb.qk_row(b, t, hk) + c]);
-                    const float bv = to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]);
+                    const float bv = pb.sig_of(to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]));
                     dk_acc[i][j] += de * bv;
                     if (GPC) static_cast<float*>(io.db)[pb.gate_row(b, t, hv, DK) + c] = de * kv;
                     else rsum[i] += de * kv;
@@ -716,7 +716,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
             const int r = idx / DK, c = idx % DK;
             if (r < L) {
                 const long off = pb.gate_row(b, t0 + r, hv, DK) + c;
-                static_cast<float*>(io.dalpha)[off] = dg[idx] / to_f32(al[off]);
+                static_cast<float*>(io.dalpha)[off] = dg[idx] / pb.alpha_of(hv, to_f32(al[off]));
             }
         }
     } else if (tid < C) {
@@ -725,7 +725,7 @@ chunk_grad_kernel(Problem pb, ChunkIO io, ChunkWs ws, int direct_qk) {
             float s = 0.f;
             for (int c = 0; c < DK; ++c) s += dg[r * DK + c];
             const long off = pb.gate_row(b, t0 + r, hv, 1);
-            static_cast<float*>(io.dalpha)[off] = s / to_f32(al[off]);
+            static_cast<float*>(io.dalpha)[off] = s / pb.alpha_of(hv, to_f32(al[off]));
         }
     }
     if (!GPC && tid < C) {

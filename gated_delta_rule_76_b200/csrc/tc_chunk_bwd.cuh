@@ -484,12 +484,16 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float a8[8];
                     if (APC) {
                         unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+                        if (pb.gate_logits) {  // alpha from its logit
+#pragma unroll
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                        }
                         if (r >= L) {
 #pragma unroll
                             for (int e = 0; e < 8; ++e) a8[e] = 1.f;
                         }
                     } else {
-                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a8[e] = av;
                     }
@@ -531,12 +535,16 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float a8[8], k8[8], q8[8], b8[8];
                     if (APC) {
                         unpack8(ld16(RA + o64), a8);
+                        if (pb.gate_logits) {  // alpha from its logit
+#pragma unroll
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                        }
                         if (r >= L) {
 #pragma unroll
                             for (int e = 0; e < 8; ++e) a8[e] = 1.f;
                         }
                     } else {
-                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a8[e] = av;
                     }
@@ -554,8 +562,12 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
+                        if (pb.gate_logits) {  // b from its logit
+#pragma unroll
+                            for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_of(b8[e_]);
+                        }
                     } else {
-                        const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f);
+                        const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f, 2);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) b8[e] = bv;
                     }
@@ -943,12 +955,16 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         float a8[8];
         if (APC) {
             unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+            if (pb.gate_logits) {  // alpha from its logit
+#pragma unroll
+                for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+            }
             if (r >= L) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a8[e] = 1.f;
             }
         } else {
-            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
 #pragma unroll
             for (int e = 0; e < 8; ++e) a8[e] = av;
         }
@@ -984,12 +1000,16 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         float a8[8], k8[8], q8[8], b8[8];
         if (APC) {
             unpack8(ld16(RA + o64), a8);
+            if (pb.gate_logits) {  // alpha from its logit
+#pragma unroll
+                for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+            }
             if (r >= L) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a8[e] = 1.f;
             }
         } else {
-            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f);
+            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
 #pragma unroll
             for (int e = 0; e < 8; ++e) a8[e] = av;
         }
@@ -1007,8 +1027,12 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         }
         if (GPC) {
             unpack8(ld16(RQB + oe), b8);
+            if (pb.gate_logits) {  // b from its logit
+#pragma unroll
+                for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_of(b8[e_]);
+            }
         } else {
-            const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f);
+            const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f, 2);
 #pragma unroll
             for (int e = 0; e < 8; ++e) b8[e] = bv;
         }
@@ -1054,7 +1078,7 @@ __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const
         vr[i] = __ldg(reinterpret_cast<const uint2*>(p.v + row + j));
         if (SPLIT) vl[i] = __ldg(reinterpret_cast<const uint2*>(p.v_lo + row + j));
         if (GPC) wr[i] = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.w) + row + j));
-        else bs[i] = gate_or(static_cast<const TG*>(p.b), pb, cp.b, cp.t0, r, cp.L, cp.hv, 0.f);
+        else bs[i] = gate_or(static_cast<const TG*>(p.b), pb, cp.b, cp.t0, r, cp.L, cp.hv, 0.f, 2);
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -1075,6 +1099,10 @@ __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const
         if (GPC) {
             w4[0] = __uint_as_float(wr[i].x << 16); w4[1] = __uint_as_float(wr[i].x & 0xFFFF0000u);
             w4[2] = __uint_as_float(wr[i].y << 16); w4[3] = __uint_as_float(wr[i].y & 0xFFFF0000u);
+            if (pb.gate_logits) {
+#pragma unroll
+                for (int e_ = 0; e_ < 4; ++e_) w4[e_] = pb.sig_of(w4[e_]);
+            }
         } else {
             w4[0] = w4[1] = w4[2] = w4[3] = bs[i];
         }
@@ -1172,8 +1200,9 @@ __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, c
             q0 += __bfloat162float(__ldg(p.q_lo + rp.qk + rr * rp.qk_s));
             k0 += __bfloat162float(__ldg(p.k_lo + rp.qk + rr * rp.qk_s));
         }
-        const float b0 = GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s));
-        const float a0 = APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s)) : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s));
+        const float b0 = p.pb.sig_of(GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s)));
+        const float a0 = p.pb.alpha_of(cp.hv, APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s))
+                                                  : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s)));
         const bool in = FULL || r < cp.L;
         x.q[i] = in ? q0 : 0.f;
         x.k[i] = in ? k0 : 0.f;
@@ -1255,7 +1284,7 @@ __device__ __forceinline__ void scalar_gate_finish(const Params& p, const ChunkP
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < 4; ++w) sum += scr[SX_RA / 4 + w * 64 + c];
-            p.dalpha[g1] = sum / to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1));
+            p.dalpha[g1] = sum / pb.alpha_of(cp.hv, to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1)));
         }
         if (!GPC) {
             float sum = scr[SX_DBV / 4 + c];

@@ -508,7 +508,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const uint32_t off = (uint32_t)ii * 128u + xo[ii & 7];
                         const float vv = SPLIT ? bf(vt, off) + bf(vt + 16384, off) : bf(vt, off);
                         float ww;
-                        if (GPC) ww = bf(vt + 16384, off);
+                        if (GPC) ww = pb.sig_of(bf(vt + 16384, off));
                         else ww = sgb[rr];
                         y2[e] = vv * ww - __uint_as_float(r[ii]);
                     }
@@ -750,15 +750,15 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float* sg = reinterpret_cast<float*>(sm + SM_SG) + pm * 128;
                 if (c < 64) {
                     if (m == 0) {
-                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t0, c, L, hv, 1.f);
-                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t0, c, L, hv, 0.f);
+                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t0, c, L, hv, 1.f, 1);
+                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t0, c, L, hv, 0.f, 2);
                     }
                     sg[c] = ga_next;
                     sg[64 + c] = gb_next;
                     if (m + 1 < NT) {
                         const int t1 = t0 + C, L1 = min(C, pb.T - t1);
-                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t1, c, L1, hv, 1.f);
-                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t1, c, L1, hv, 0.f);
+                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t1, c, L1, hv, 1.f, 1);
+                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t1, c, L1, hv, 0.f, 2);
                     }
                 }
             }
@@ -789,6 +789,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float a8[8];
                     if (APC) {
                         unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
+                        if (pb.gate_logits) {  // alpha from its logit
+#pragma unroll
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                        }
                         if (r >= L) {
 #pragma unroll
                             for (int i = 0; i < 8; ++i) a8[i] = 1.f;
@@ -836,6 +840,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float a8[8], k8[8], q8[8], b8[8];
                     if (APC) {
                         unpack8(ld16(RA + o64), a8);
+                        if (pb.gate_logits) {  // alpha from its logit
+#pragma unroll
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                        }
                         if (r >= L) {
 #pragma unroll
                             for (int i = 0; i < 8; ++i) a8[i] = 1.f;
@@ -859,6 +867,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
+                        if (pb.gate_logits) {  // b from its logit
+#pragma unroll
+                            for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_of(b8[e_]);
+                        }
                     } else {
                         const float bv = sga[pm * 128 + 64 + r];
 #pragma unroll

@@ -32,7 +32,8 @@ class FwdArgs(ctypes.Structure):
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32),
-                ("bwd_cache", P), ("bwd_cache_bytes", ctypes.c_size_t)]
+                ("bwd_cache", P), ("bwd_cache_bytes", ctypes.c_size_t), ("gate_logits", I32),
+                ("alpha_scale", P)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -42,7 +43,8 @@ class BwdArgs(ctypes.Structure):
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32),
-                ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t)]
+                ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t), ("gate_logits", I32),
+                ("alpha_scale", P), ("grad_alpha_scale", P)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -50,7 +52,8 @@ class DecodeArgs(ctypes.Structure):
                 ("o", P), ("head_map", P), ("conv_state", P), ("conv_w", P), ("z", P),
                 ("N", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
-                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32)]
+                ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32), ("gate_logits", I32),
+                ("alpha_scale", P)]
 
 
 class LayerArgs(ctypes.Structure):
@@ -59,7 +62,8 @@ class LayerArgs(ctypes.Structure):
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32), ("bwd_cache", P),
-                ("bwd_cache_bytes", ctypes.c_size_t), ("norm_w", P), ("norm_eps", F32)]
+                ("bwd_cache_bytes", ctypes.c_size_t), ("norm_w", P), ("norm_eps", F32), ("gate_logits", I32),
+                ("alpha_scale", P)]
 
 
 class LayerBwdArgs(ctypes.Structure):
@@ -70,7 +74,8 @@ class LayerBwdArgs(ctypes.Structure):
                 ("B", I64), ("T", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t),
-                ("norm_w", P), ("norm_eps", F32), ("grad_norm_w", P)]
+                ("norm_w", P), ("norm_eps", F32), ("grad_norm_w", P), ("gate_logits", I32),
+                ("alpha_scale", P), ("grad_alpha_scale", P)]
 
 
 EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
@@ -212,8 +217,10 @@ def _head_map(head_map, device, Hk: int):
 # public calls
 # ---------------------------------------------------------------------------------------------
 def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
-             scale: float = 1.0, o=None, ht=None, bwd_cache=None) -> Tuple[FwdArgs, list]:
-    """Build the gdn_fwd_args struct (the returned list keeps referenced tensors alive)."""
+             scale: float = 1.0, o=None, ht=None, bwd_cache=None, alpha_scale=None) -> Tuple[FwdArgs, list]:
+    """Build the gdn_fwd_args struct (the returned list keeps referenced tensors alive).
+    ``alpha_scale`` [Hv] fp32: the gates are logits (alpha = exp(-alpha_scale softplus(x)),
+    b, w, beta = sigmoid(x))."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
@@ -225,24 +232,25 @@ def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_ma
                 dtype=_dt(q), gate_dtype=_dt(alpha),
                 out_f32=int(o is not None and o.dtype == torch.float32 and q.dtype != torch.float32),
                 bwd_cache=_ptr(bwd_cache),
-                bwd_cache_bytes=0 if bwd_cache is None else bwd_cache.numel() * bwd_cache.element_size())
-    return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm, bwd_cache]
+                bwd_cache_bytes=0 if bwd_cache is None else bwd_cache.numel() * bwd_cache.element_size(),
+                gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale))
+    return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm, bwd_cache, alpha_scale]
 
 
 def gdn_chunk_fwd_cache_size(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
-                             scale: float = 1.0) -> int:
+                             scale: float = 1.0, alpha_scale=None) -> int:
     """Bytes of the forward cache gdn_chunk_fwd(..., bwd_cache=) can fill for a later backward
     (0: this problem runs on the CUDA-core path, which keeps none)."""
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
-    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, None, head_map, scale)
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, None, head_map, scale, alpha_scale=alpha_scale)
     return int(load().gdn_chunk_fwd_cache_size(ctypes.byref(a)))
 
 
 def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
                   scale: float = 1.0, *, o=None, ht=None, want_ht: bool = True, out_f32: bool = False,
-                  bwd_cache: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                  stream=None):
+                  bwd_cache: Optional[torch.Tensor] = None, alpha_scale: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
     """Chunkwise forward.  Returns (o [B,T,Hv,dv], ht [B,Hv,dk,dv] or None).
     ``out_f32`` writes o in fp32 (the unrounded accumulator) instead of the input dtype.
     ``bwd_cache``: a device byte tensor of gdn_chunk_fwd_cache_size() bytes that the forward fills
@@ -254,7 +262,7 @@ def gdn_chunk_fwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, he
     if ht is None and want_ht:
         ht = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
     lib = load()
-    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht, bwd_cache)
+    a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht, bwd_cache, alpha_scale)
     need = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, q.device, workspace)
     check(lib.gdn_chunk_fwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_fwd")
@@ -310,7 +318,7 @@ def gdn_state_compose(M, N, S, *, transpose: bool = False, out: Optional[torch.T
 
 
 def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, scale=1.0,
-             grad_o=None, grad_ht=None, grads=None, fwd_cache=None) -> Tuple[BwdArgs, list]:
+             grad_o=None, grad_ht=None, grads=None, fwd_cache=None, alpha_scale=None) -> Tuple[BwdArgs, list]:
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
@@ -324,17 +332,20 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
                 B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                 alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
                 dtype=_dt(q), gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
-                fwd_cache_bytes=0 if fwd_cache is None else fwd_cache.numel() * fwd_cache.element_size())
-    return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g, fwd_cache]
+                fwd_cache_bytes=0 if fwd_cache is None else fwd_cache.numel() * fwd_cache.element_size(),
+                gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale),
+                grad_alpha_scale=_ptr(g.get("dalpha_scale")))
+    return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g, fwd_cache, alpha_scale]
 
 
 def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
                   scale: float = 1.0, *, grad_o, grad_ht=None, want_dh0: bool = True,
-                  fwd_cache: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                  stream=None) -> Dict[str, torch.Tensor]:
+                  fwd_cache: Optional[torch.Tensor] = None, alpha_scale: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
     """Chunkwise backward.  Returns fp32 dq, dk, dv, dalpha and db/dw (or dbeta), dh0.
     ``fwd_cache``: the cache a gdn_chunk_fwd(..., bwd_cache=) call filled with these same inputs
-    (the forward is then not recomputed)."""
+    (the forward is then not recomputed).  With ``alpha_scale`` the gates are logits: dalpha, db,
+    dw, dbeta are the gradients of the logits, and dalpha_scale [Hv] that of alpha_scale."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=t.device)
     grads = {"dq": f32(q), "dk": f32(k), "dv": f32(v), "dalpha": f32(alpha)}
@@ -347,8 +358,11 @@ def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=N
         B, T, Hk, dk = q.shape
         Hv, dv = v.shape[2], v.shape[3]
         grads["dh0"] = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    if alpha_scale is not None:
+        grads["dalpha_scale"] = torch.empty(tuple(alpha_scale.shape), dtype=torch.float32, device=q.device)
     lib = load()
-    a, keep = bwd_args(q, k, v, alpha, b, w, beta, h0, head_map, scale, grad_o, grad_ht, grads, fwd_cache)
+    a, keep = bwd_args(q, k, v, alpha, b, w, beta, h0, head_map, scale, grad_o, grad_ht, grads, fwd_cache,
+                       alpha_scale)
     need = lib.gdn_chunk_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, q.device, workspace)
     check(lib.gdn_chunk_bwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_bwd")
@@ -357,7 +371,7 @@ def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=N
 
 def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=None,
                     scale: float = 1.0, *, conv_state=None, conv_w=None, z=None, o=None,
-                    out_f32: bool = False, stream=None):
+                    out_f32: bool = False, alpha_scale=None, stream=None):
     """One token for N sequences; ``state`` [N,Hv,dk,dv] fp32 is updated in place.  Returns o."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
     N, Hk, dk = q.shape
@@ -370,7 +384,8 @@ def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=N
                    conv_w=_ptr(conv_w), z=_ptr(z), N=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                    alpha_per_channel=int(alpha.dim() == 3), gates_per_channel=gpc,
                    dtype=_dt(q), gate_dtype=_dt(alpha),
-                   out_f32=int(o.dtype == torch.float32 and q.dtype != torch.float32))
+                   out_f32=int(o.dtype == torch.float32 and q.dtype != torch.float32),
+                   gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale))
     check(load().gdn_decode_step(ctypes.byref(a), _stream(stream)), "gdn_decode_step")
     return o
 
@@ -379,7 +394,7 @@ NORM_EPS = 1e-6  # the output norm's epsilon when the caller gives none
 
 
 def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y=None, ht=None, cs=None,
-                out_f32=0, bwd_cache=None, norm_w=None, norm_eps=NORM_EPS):
+                out_f32=0, bwd_cache=None, norm_w=None, norm_eps=NORM_EPS, alpha_scale=None):
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
@@ -390,7 +405,8 @@ def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y
                   dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
                   gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha), out_f32=out_f32,
                   bwd_cache=_ptr(bwd_cache), bwd_cache_bytes=bwd_cache.numel() if bwd_cache is not None else 0,
-                  norm_w=_ptr(norm_w), norm_eps=norm_eps)
+                  norm_w=_ptr(norm_w), norm_eps=norm_eps, gate_logits=int(alpha_scale is not None),
+                  alpha_scale=_ptr(alpha_scale))
     return a, hm
 
 
@@ -405,7 +421,7 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
                        head_map=None, scale: float = 1.0, *, want_ht: bool = True,
                        want_conv_state: bool = False, y=None, out_f32: bool = False,
                        bwd_cache: Optional[torch.Tensor] = None, norm_w=None, norm_eps: float = NORM_EPS,
-                       workspace: Optional[torch.Tensor] = None, stream=None):
+                       alpha_scale=None, workspace: Optional[torch.Tensor] = None, stream=None):
     """GQA layer core forward.  Returns (y, ht or None, conv_state or None).  ``bwd_cache``: a
     uint8 device tensor of gdn_layer_core_fwd_cache_size() bytes that a later
     gdn_layer_core_bwd(..., fwd_cache=) over the same inputs reads.  ``norm_w`` [dv] (the layer's
@@ -419,7 +435,7 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
           if want_conv_state else None)
     a, hm = _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y=y, ht=ht, cs=cs,
                         out_f32=int(y.dtype == torch.float32 and xq.dtype != torch.float32), bwd_cache=bwd_cache,
-                        norm_w=norm_w, norm_eps=norm_eps)
+                        norm_w=norm_w, norm_eps=norm_eps, alpha_scale=alpha_scale)
     lib = load()
     need = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, xq.device, workspace)
@@ -431,7 +447,8 @@ def gdn_layer_core_fwd(xq, xk, xv, conv_w, alpha, z, b=None, w=None, beta=None, 
 def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, beta=None, h0=None,
                        grad_ht=None, head_map=None, scale: float = 1.0, *, want_h0_grad: bool = True,
                        fwd_cache: Optional[torch.Tensor] = None, norm_w=None, norm_eps: float = NORM_EPS,
-                       workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
+                       alpha_scale=None, workspace: Optional[torch.Tensor] = None,
+                       stream=None) -> Dict[str, torch.Tensor]:
     """GQA layer core backward (reverse mode of gdn_layer_core_fwd).  Returns a dict of fp32
     gradients: dxq, dxk, dxv, dconv_w, dalpha, dz, dh0 (or None), db/dw or dbeta, and dnorm_w
     with the output norm (``norm_w``).
@@ -454,6 +471,8 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
         gb, gw = out["dbeta"], None
     if norm_w is not None:
         out["dnorm_w"] = torch.empty((dv,), **f32)
+    if alpha_scale is not None:
+        out["dalpha_scale"] = torch.empty(tuple(alpha_scale.shape), **f32)
     hm = _head_map(head_map, dev, Hk)
     a = LayerBwdArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
                      b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), head_map=_ptr(hm), grad_y=_ptr(grad_y),
@@ -464,7 +483,9 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
                      alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc, dtype=_dt(xq),
                      gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
                      fwd_cache_bytes=fwd_cache.numel() if fwd_cache is not None else 0,
-                     norm_w=_ptr(norm_w), norm_eps=norm_eps, grad_norm_w=_ptr(out.get("dnorm_w")))
+                     norm_w=_ptr(norm_w), norm_eps=norm_eps, grad_norm_w=_ptr(out.get("dnorm_w")),
+                     gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale),
+                     grad_alpha_scale=_ptr(out.get("dalpha_scale")))
     lib = load()
     need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, dev, workspace)

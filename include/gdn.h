@@ -46,6 +46,14 @@
  *    below it is recomputed by an exact sequential kernel in the same call (token by token, no
  *    ratio of decays), which overwrites that pair's results.  Such pairs cost several times more
  *    than the chunk form.  The single-token decode step has no ratio and no such bound.
+ *  - Gates as logits (optional, gate_logits = 1 in the args): alpha, b, w, beta are then given as
+ *    logits x (same layouts and gate_dtype) and every kernel applies, where it reads a gate,
+ *        alpha = exp(-alpha_scale[hv] * softplus(x)),   b, w, beta = sigmoid(x)
+ *    with alpha_scale [Hv] fp32 > 0 (explainer «Architecture et versions hybrides», Figure 1
+ *    caption: alpha takes the Mamba-2 parametrisation exp(-A dt), dt = softplus(x), A = alpha_scale;
+ *    the zubnet.ai news item: the erase and write gates are two sigmoids).  The backward then
+ *    returns the gradients of the logits in grad_alpha, grad_b, grad_w, and (if not NULL) that of
+ *    alpha_scale in grad_alpha_scale [Hv] (summed over batch, tokens and channels in a fixed order).
  *  - Errors: every call returns a gdn_status.  Invalid arguments are detected on the host before
  *    any launch and nothing is written.  gdn_last_error() returns a thread-local message about
  *    the last failure of the calling thread.  No C++ exception crosses this interface.
@@ -113,6 +121,8 @@ typedef struct gdn_fwd_args {
      * bwd_cache must be NULL.  The cache is independent of z. */
     void* bwd_cache;
     size_t bwd_cache_bytes;
+    int32_t gate_logits;       /* 1: alpha, b, w are logits (see the conventions above) */
+    const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
 } gdn_fwd_args;
 
 /* Bytes of the optional forward cache (0 where the problem cannot keep one). */
@@ -180,6 +190,9 @@ typedef struct gdn_bwd_args {
      * inputs: a stale cache gives wrong gradients.  NULL: the forward is recomputed. */
     const void* fwd_cache;
     size_t fwd_cache_bytes;
+    int32_t gate_logits;       /* 1: alpha, b, w are logits; the gradients returned are those of the logits */
+    const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
+    float* grad_alpha_scale;   /* out [Hv] fp32, may be NULL (must be NULL without gate_logits) */
 } gdn_bwd_args;
 
 GDN_API size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args);
@@ -247,6 +260,8 @@ typedef struct gdn_decode_args {
     int32_t dtype;
     int32_t gate_dtype;
     int32_t out_f32;      /* 1: o is written in fp32 instead of dtype */
+    int32_t gate_logits;       /* 1: alpha, b, w are logits */
+    const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
 } gdn_decode_args;
 
 GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, gdn_stream stream);
@@ -301,6 +316,8 @@ typedef struct gdn_layer_args {
      * before the norm. */
     const void* norm_w;
     float norm_eps;
+    int32_t gate_logits;       /* 1: alpha, b, w are logits */
+    const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
 } gdn_layer_args;
 
 /* Bytes of the optional layer forward cache (0 where the layer backward cannot use one). */
@@ -368,6 +385,9 @@ typedef struct gdn_layer_bwd_args {
     const void* norm_w;
     float norm_eps;
     float* grad_norm_w;
+    int32_t gate_logits;       /* 1: alpha, b, w are logits; the gradients returned are those of the logits */
+    const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
+    float* grad_alpha_scale;   /* out [Hv] fp32, may be NULL (must be NULL without gate_logits) */
 } gdn_layer_bwd_args;
 
 GDN_API size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* args);

@@ -251,3 +251,15 @@ def test_segment_map_and_compose_host_validation(lib):
     assert lib.gdn_state_compose(M, None, None, M, 1, 128, 128, 0, None) == 1  # output overlaps M
     assert lib.gdn_state_compose(M, None, None, N, 1, 64, 128, 1, None) == 1   # M^T needs dk == dv
     assert gdn.kernel_launches() == before
+
+
+def test_gate_logit_arguments_rejected_on_the_host(lib):
+    """gate_logits needs alpha_scale; alpha_scale without gate_logits, or a flag other than 0/1, is
+    an error; nothing is launched."""
+    before = gdn.kernel_launches()
+    ws = ctypes.c_void_p(1 << 30)
+    for kw in (dict(gate_logits=1), dict(alpha_scale=1 << 27), dict(gate_logits=2, alpha_scale=1 << 27)):
+        a = _fwd(**kw)
+        assert lib.gdn_chunk_fwd(ctypes.byref(a), ws, 1 << 30, None) == 1, kw
+        assert "gate_logits" in lib.gdn_last_error().decode() or "alpha_scale" in lib.gdn_last_error().decode()
+    assert gdn.kernel_launches() == before
