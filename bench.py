@@ -613,6 +613,26 @@ def _profile_train_b2_t2048():
     return 0
 
 
+def _profile_train_b8_t1024():
+    """GDN-2 training step on B=8 T=1024 H=16 d=128 bf16 (seed 21): the headline's 128 (sequence, head)
+    pairs, a quarter of its tokens; twice: the forward keeping the cache, then the backward from it."""
+    import torch
+    from gated_delta_rule_76_b200 import gdn
+    from gated_delta_rule_76_b200.inputs import draw
+    x = draw(8, 1024, 16, 16, 128, 128, alpha_per_channel=True, gates_per_channel=True, dtype="bf16",
+             gate_dtype="bf16", seed=21, has_h0=True, with_dout=True)
+    g = {k: v.cuda() for k, v in x.items()}
+    kw = dict(b=g["b"], w=g["w"], h0=g["h0"])
+    cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], **kw),
+                        dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
+        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache, **kw)
+    torch.cuda.synchronize()
+    print("ok", float(grads["dq"].abs().mean()))
+    return 0
+
+
 def _profile_fwd_b8_t1024():
     """GDN-2 forward on B=8 T=1024 H=16 d=128 bf16 (seed 21), twice, without a cache."""
     import torch
@@ -694,7 +714,8 @@ def _profile_decode_b256():
     return 0
 
 
-PROFILE_CASES = {"decode_b256": _profile_decode_b256, "train_b2_t2048": _profile_train_b2_t2048, "fwd_b8_t1024": _profile_fwd_b8_t1024,
+PROFILE_CASES = {"decode_b256": _profile_decode_b256, "train_b2_t2048": _profile_train_b2_t2048,
+                 "train_b8_t1024": _profile_train_b8_t1024, "fwd_b8_t1024": _profile_fwd_b8_t1024,
                  "layer_b2_t16384": _profile_layer_b2_t16384, "train_b8_t4096": _profile_train_b8_t4096,
                  "layer_train_b2_t16384": _profile_layer_train_b2_t16384}
 

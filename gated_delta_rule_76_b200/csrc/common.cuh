@@ -34,14 +34,29 @@ struct Problem {
     int gate_logits;
     const float* alpha_scale;  // [Hv] fp32 (gate_logits only)
 
+    // The transforms with the form chosen at compile time: kernels instantiated for logits (LG)
+    // apply them, the others read the gates as stored.  No branch then sits between a gate's load
+    // and its use (a branch on a loaded value waits for the load, which serialises the loads of an
+    // unrolled loop).
+    template <bool LG>
+    __device__ __forceinline__ float alpha_t(int hv, float x) const {
+        if constexpr (LG) {
+            const float sp = fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));  // softplus(x)
+            return expf(-__ldg(alpha_scale + hv) * sp);
+        } else {
+            return x;
+        }
+    }
+    template <bool LG>
+    __device__ __forceinline__ float sig_t(float x) const {
+        if constexpr (LG) return 1.f / (1.f + expf(-x));
+        else return x;
+    }
+    // Run-time forms, for the kernels not instantiated per form.
     __device__ __forceinline__ float alpha_of(int hv, float x) const {
-        if (!gate_logits) return x;
-        const float sp = fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));  // softplus(x)
-        return expf(-__ldg(alpha_scale + hv) * sp);
+        return gate_logits ? alpha_t<true>(hv, x) : x;
     }
-    __device__ __forceinline__ float sig_of(float x) const {
-        return gate_logits ? 1.f / (1.f + expf(-x)) : x;
-    }
+    __device__ __forceinline__ float sig_of(float x) const { return gate_logits ? sig_t<true>(x) : x; }
 
     // An explicit map entry outside [0, Hk) breaks the interface's precondition; it is clamped
     // into range so that no kernel reads outside q or k (the result is then unspecified).
@@ -69,13 +84,14 @@ struct Problem {
 // past the end of the sequence.  The load itself is unconditional, from the row clamped to the
 // last token: a load under a branch is waited for where the branch ends, which would serialise
 // the loads of an unrolled loop.
-// kind: 0 the value as stored, 1 a decay alpha, 2 a sigmoid gate (the transforms of gate logits).
-template <class TG>
+// KIND: 0 the value as stored, 1 a decay alpha, 2 a sigmoid gate; the transforms of gate logits
+// are applied when LG is set.
+template <int KIND = 0, bool LG = false, class TG>
 __device__ __forceinline__ float gate_or(const TG* g, const Problem& pb, int b, int t0, int r, int L, int hv,
-                                         float fill, int kind = 0) {
+                                         float fill) {
     float x = to_f32(__ldg(g + pb.gate_row(b, t0 + (r < L ? r : L - 1), hv, 1)));
-    if (kind == 1) x = pb.alpha_of(hv, x);
-    else if (kind == 2) x = pb.sig_of(x);
+    if constexpr (KIND == 1) x = pb.alpha_t<LG>(hv, x);
+    else if constexpr (KIND == 2) x = pb.sig_t<LG>(x);
     return r < L ? x : fill;
 }
 

@@ -112,8 +112,17 @@ chunk_prep_kernel(Problem pb, ChunkIO io, ChunkWs ws, int save_bwd) {
                 const bool in = r < L;
                 kv[u] = in ? to_f32(k[pb.qk_row(b, t, hk) + c]) : 0.f;
                 qv[u] = in ? to_f32(q[pb.qk_row(b, t, hk) + c]) : 0.f;
-                av[u] = in ? pb.alpha_of(hv, to_f32(al[pb.gate_row(b, t, hv, APC ? DK : 1) + (APC ? c : 0)])) : 1.f;
-                bv[u] = in ? pb.sig_of(to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)])) : 0.f;
+                av[u] = in ? to_f32(al[pb.gate_row(b, t, hv, APC ? DK : 1) + (APC ? c : 0)]) : 1.f;
+                bv[u] = in ? to_f32(bg[pb.gate_row(b, t, hv, GPC ? DK : 1) + (GPC ? c : 0)]) : 0.f;
+            }
+            if (pb.gate_logits) {  // one branch after the eight rows' loads, not one per load
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (r0 + u < L) {
+                        av[u] = pb.alpha_t<true>(hv, av[u]);
+                        bv[u] = pb.sig_t<true>(bv[u]);
+                    }
+                }
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {

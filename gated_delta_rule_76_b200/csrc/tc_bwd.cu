@@ -6,7 +6,7 @@
 #include <cuda.h>
 
 #include "launch.cuh"
-#include "tc_chunk_bwd.cuh"
+#include "tc_bwd_launch.cuh"
 #include "tma_host.h"
 
 namespace gdn {
@@ -14,42 +14,6 @@ namespace gdn {
 namespace {
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
-
-template <bool APC, bool GPC, class TG, bool SPLIT>
-cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cudaStream_t st) {
-    auto kernel = tcbwd::scan::chunk_bwd_scan_kernel<APC, GPC, TG, SPLIT>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tcbwd::scan::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    kernel<<<p.pb.B * p.pb.Hv, tcbwd::scan::kThreads, tcbwd::scan::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
-                                                                                    p);
-    count_launch();
-    return cudaGetLastError();
-}
-
-template <bool APC, bool GPC, class TG, bool SPLIT>
-cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cudaStream_t st) {
-    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG, SPLIT>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tcbwd::grad::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    const long nch = (long)p.pb.B * p.pb.Hv * p.pb.NT;
-    int dev = 0, nsm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    const long grid = nch < nsm ? nch : nsm;  // persistent: one CTA per SM walks the chunks
-    kernel<<<(unsigned)grid, tcbwd::grad::kThreads, tcbwd::grad::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
-                                                                                 m[5], m[6], m[7], m[8], p);
-    count_launch();
-    return cudaGetLastError();
-}
-
-template <bool APC, bool GPC, class TG, bool SPLIT = false>
-cudaError_t launch_both(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
-                        const tcbwd::grad::Params& gp, cudaStream_t st) {
-    cudaError_t e = launch_scan<APC, GPC, TG, SPLIT>(ms, sp, st);
-    if (e != cudaSuccess) return e;
-    return launch_grad<APC, GPC, TG, SPLIT>(mg, gp, st);
-}
 
 }  // namespace
 
@@ -175,13 +139,8 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     gp.direct = direct ? 1 : 0;
     gp.err = err;
 
-    if (split) e = bf16_gates ? launch_both<false, false, __nv_bfloat16, true>(ms, sp, m, gp, st)
-                              : launch_both<false, false, float, true>(ms, sp, m, gp, st);
-    else if (f.apc && f.gpc) e = launch_both<true, true, __nv_bfloat16>(ms, sp, m, gp, st);
-    else if (f.apc) e = launch_both<true, false, __nv_bfloat16>(ms, sp, m, gp, st);
-    else if (f.gpc) e = launch_both<false, true, __nv_bfloat16>(ms, sp, m, gp, st);
-    else if (bf16_gates) e = launch_both<false, false, __nv_bfloat16>(ms, sp, m, gp, st);
-    else e = launch_both<false, false, float>(ms, sp, m, gp, st);
+    e = pb.gate_logits ? tc_bwd_dispatch<true>(ms, sp, m, gp, f, split, bf16_gates, st)
+                       : tc_bwd_dispatch<false>(ms, sp, m, gp, f, split, bf16_gates, st);
     if (e != cudaSuccess) return e;
     // 3. pairs whose decay left the factors' range (marked by the scan): every gradient again,
     //    exactly; the pair's slice of the dS array holds its checkpoints
@@ -195,14 +154,3 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
 }
 
 }  // namespace gdn
-
-#ifdef GDN_BWD_TRACE
-// Profiling builds only: copy the phase timestamps of CTA 0 of the last gradient kernel to the host.
-extern "C" __attribute__((visibility("default"))) int gdn_bwd_trace_read(unsigned long long* host) {
-    return (int)cudaMemcpyFromSymbol(host, gdn::tcbwd::g_bwd_trace, sizeof(unsigned long long) * 16 * 16);
-}
-// ... and those of CTA 0 of the last reverse scan.
-extern "C" __attribute__((visibility("default"))) int gdn_scan_trace_read(unsigned long long* host) {
-    return (int)cudaMemcpyFromSymbol(host, gdn::tcbwd::g_scan_trace, sizeof(unsigned long long) * 64 * 32);
-}
-#endif

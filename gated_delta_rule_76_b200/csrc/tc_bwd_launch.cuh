@@ -1,0 +1,73 @@
+// Launches of the tensor-core chunk backward's two kernels (reverse state-gradient scan, chunk-parallel
+// gradients) for one gate form (LG: gates given as logits), with the dispatch over their
+// instantiations.  Each form is compiled in its own translation unit (tc_bwd_gates.cu,
+// tc_bwd_logits.cu); tc_bwd.cu plans the workspace and builds the tensor maps and parameters.
+#pragma once
+
+#include <cuda.h>
+
+#include "launch.h"
+#include "tc_chunk_bwd.cuh"
+
+namespace gdn {
+
+template <bool LG>
+cudaError_t tc_bwd_dispatch(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
+                            const tcbwd::grad::Params& gp, Flags f, bool split, bool bf16_gates, cudaStream_t st);
+
+#ifdef GDN_TC_BWD_INSTANTIATE
+namespace {
+
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
+cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cudaStream_t st) {
+    auto kernel = tcbwd::scan::chunk_bwd_scan_kernel<APC, GPC, TG, SPLIT, LG>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcbwd::scan::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kernel<<<p.pb.B * p.pb.Hv, tcbwd::scan::kThreads, tcbwd::scan::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                                    p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
+cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cudaStream_t st) {
+    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG, SPLIT, LG>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tcbwd::grad::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long nch = (long)p.pb.B * p.pb.Hv * p.pb.NT;
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const long grid = nch < nsm ? nch : nsm;  // persistent: one CTA per SM walks the chunks
+    kernel<<<(unsigned)grid, tcbwd::grad::kThreads, tcbwd::grad::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                                 m[5], m[6], m[7], m[8], p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
+cudaError_t launch_both(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
+                        const tcbwd::grad::Params& gp, cudaStream_t st) {
+    cudaError_t e = launch_scan<APC, GPC, TG, SPLIT, LG>(ms, sp, st);
+    if (e != cudaSuccess) return e;
+    return launch_grad<APC, GPC, TG, SPLIT, LG>(mg, gp, st);
+}
+
+}  // namespace
+
+template <bool LG>
+cudaError_t tc_bwd_dispatch(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* m,
+                            const tcbwd::grad::Params& gp, Flags f, bool split, bool bf16_gates, cudaStream_t st) {
+    if (split)
+        return bf16_gates ? launch_both<false, false, __nv_bfloat16, true, LG>(ms, sp, m, gp, st)
+                          : launch_both<false, false, float, true, LG>(ms, sp, m, gp, st);
+    if (f.apc && f.gpc) return launch_both<true, true, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
+    if (f.apc) return launch_both<true, false, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
+    if (f.gpc) return launch_both<false, true, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
+    if (bf16_gates) return launch_both<false, false, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
+    return launch_both<false, false, float, false, LG>(ms, sp, m, gp, st);
+}
+#endif  // GDN_TC_BWD_INSTANTIATE
+
+}  // namespace gdn

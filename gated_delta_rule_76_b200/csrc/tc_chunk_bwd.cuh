@@ -178,7 +178,7 @@ __device__ __forceinline__ void scan_load_do(const Ctx& cx, int n, int b, int hv
     tma4(dst + 8192, tdo, bar, 64, hv, n * C, b);
 }
 
-template <bool APC, bool GPC, class TG, bool SPLIT>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -484,16 +484,16 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float a8[8];
                     if (APC) {
                         unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
-                        if (pb.gate_logits) {  // alpha from its logit
+                        if constexpr (LG) {  // alpha from its logit
 #pragma unroll
-                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_t<LG>(hv, a8[e_]);
                         }
                         if (r >= L) {
 #pragma unroll
                             for (int e = 0; e < 8; ++e) a8[e] = 1.f;
                         }
                     } else {
-                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
+                        const float av = gate_or<1, LG>(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a8[e] = av;
                     }
@@ -535,16 +535,16 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float a8[8], k8[8], q8[8], b8[8];
                     if (APC) {
                         unpack8(ld16(RA + o64), a8);
-                        if (pb.gate_logits) {  // alpha from its logit
+                        if constexpr (LG) {  // alpha from its logit
 #pragma unroll
-                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_t<LG>(hv, a8[e_]);
                         }
                         if (r >= L) {
 #pragma unroll
                             for (int e = 0; e < 8; ++e) a8[e] = 1.f;
                         }
                     } else {
-                        const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
+                        const float av = gate_or<1, LG>(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) a8[e] = av;
                     }
@@ -562,12 +562,12 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
-                        if (pb.gate_logits) {  // b from its logit
+                        if constexpr (LG) {  // b from its logit
 #pragma unroll
-                            for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_of(b8[e_]);
+                            for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_t<LG>(b8[e_]);
                         }
                     } else {
-                        const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f, 2);
+                        const float bv = gate_or<2, LG>(beta_g, pb, b, t0, r, L, hv, 0.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) b8[e] = bv;
                     }
@@ -887,7 +887,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Staging group (128 threads, c = lane = channel): S0 and dS_end rows of the chunk into tensor
 // memory as split A operands and rowsum(dS_end .* S0) into xslot[c]; then, once the raw TMA tiles
 // have landed, the cumulative decay (gamma into gslot[c]) and the split [Ehat;Qhat], Ktil tiles.
-template <bool APC, bool GPC, class TG, bool SPLIT>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
 __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, const ChunkPos& cp, uint32_t tl, int c,
                                             float* xslot, float* gslot, uint32_t raw_parity, int it = 15) {
     const Problem& pb = p.pb;
@@ -955,16 +955,16 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         float a8[8];
         if (APC) {
             unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
-            if (pb.gate_logits) {  // alpha from its logit
+            if constexpr (LG) {  // alpha from its logit
 #pragma unroll
-                for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_t<LG>(hv, a8[e_]);
             }
             if (r >= L) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a8[e] = 1.f;
             }
         } else {
-            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
+            const float av = gate_or<1, LG>(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) a8[e] = av;
         }
@@ -1000,16 +1000,16 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         float a8[8], k8[8], q8[8], b8[8];
         if (APC) {
             unpack8(ld16(RA + o64), a8);
-            if (pb.gate_logits) {  // alpha from its logit
+            if constexpr (LG) {  // alpha from its logit
 #pragma unroll
-                for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_t<LG>(hv, a8[e_]);
             }
             if (r >= L) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a8[e] = 1.f;
             }
         } else {
-            const float av = gate_or(alpha_g, pb, b, t0, r, L, hv, 1.f, 1);
+            const float av = gate_or<1, LG>(alpha_g, pb, b, t0, r, L, hv, 1.f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) a8[e] = av;
         }
@@ -1027,12 +1027,12 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         }
         if (GPC) {
             unpack8(ld16(RQB + oe), b8);
-            if (pb.gate_logits) {  // b from its logit
+            if constexpr (LG) {  // b from its logit
 #pragma unroll
-                for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_of(b8[e_]);
+                for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_t<LG>(b8[e_]);
             }
         } else {
-            const float bv = gate_or(beta_g, pb, b, t0, r, L, hv, 0.f, 2);
+            const float bv = gate_or<2, LG>(beta_g, pb, b, t0, r, L, hv, 0.f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) b8[e] = bv;
         }
@@ -1062,7 +1062,7 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
 // dv = w .* dY, dw = v .* dY (a scalar beta: sum_j v dY per token into scr[SX_DBV]); run by the
 // staging group after its staging, warp w: tokens w, w + 4, ..., lane l: value channels 4l .. 4l + 3.
 
-template <bool GPC, class TG, bool SPLIT>
+template <bool GPC, class TG, bool SPLIT, bool LG>
 __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const ChunkPos& cp, int tt, float* scr) {
     const Problem& pb = p.pb;
     const int w = tt >> 5, l = tt & 31, j = 4 * l;
@@ -1078,7 +1078,7 @@ __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const
         vr[i] = __ldg(reinterpret_cast<const uint2*>(p.v + row + j));
         if (SPLIT) vl[i] = __ldg(reinterpret_cast<const uint2*>(p.v_lo + row + j));
         if (GPC) wr[i] = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.w) + row + j));
-        else bs[i] = gate_or(static_cast<const TG*>(p.b), pb, cp.b, cp.t0, r, cp.L, cp.hv, 0.f, 2);
+        else bs[i] = gate_or<2, LG>(static_cast<const TG*>(p.b), pb, cp.b, cp.t0, r, cp.L, cp.hv, 0.f);
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -1099,9 +1099,9 @@ __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const
         if (GPC) {
             w4[0] = __uint_as_float(wr[i].x << 16); w4[1] = __uint_as_float(wr[i].x & 0xFFFF0000u);
             w4[2] = __uint_as_float(wr[i].y << 16); w4[3] = __uint_as_float(wr[i].y & 0xFFFF0000u);
-            if (pb.gate_logits) {
+            if constexpr (LG) {
 #pragma unroll
-                for (int e_ = 0; e_ < 4; ++e_) w4[e_] = pb.sig_of(w4[e_]);
+                for (int e_ = 0; e_ < 4; ++e_) w4[e_] = pb.sig_t<LG>(w4[e_]);
             }
         } else {
             w4[0] = w4[1] = w4[2] = w4[3] = bs[i];
@@ -1187,7 +1187,7 @@ __device__ __forceinline__ RowPtrs row_ptrs(const Params& p, const ChunkPos& cp,
 // Inputs of tokens r0 .. r0 + RB - 1.  FULL: every row of the chunk is inside the sequence; else rows
 // past the sequence read its last token and are then replaced (a load under a branch would be waited
 // for where the branch ends).
-template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT>
+template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT, bool LG>
 __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, const RowPtrs& rp, int r0, RowIn& x) {
     const TG* ag = static_cast<const TG*>(p.alpha);
     const TG* bg = static_cast<const TG*>(p.b);
@@ -1200,8 +1200,8 @@ __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, c
             q0 += __bfloat162float(__ldg(p.q_lo + rp.qk + rr * rp.qk_s));
             k0 += __bfloat162float(__ldg(p.k_lo + rp.qk + rr * rp.qk_s));
         }
-        const float b0 = p.pb.sig_of(GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s)));
-        const float a0 = p.pb.alpha_of(cp.hv, APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s))
+        const float b0 = p.pb.sig_t<LG>(GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s)));
+        const float a0 = p.pb.alpha_t<LG>(cp.hv, APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s))
                                                   : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s)));
         const bool in = FULL || r < cp.L;
         x.q[i] = in ? q0 : 0.f;
@@ -1211,7 +1211,7 @@ __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, c
     }
 }
 
-template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT>
+template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT, bool LG>
 __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
                                                 float gam, float xtot, float* scr, int it) {
     const float scale = p.pb.scale;
@@ -1254,28 +1254,28 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
     };
     // two input buffers: a block's loads are in flight while the previous block is formed
     RowIn x0, x1;
-    load_rows<APC, GPC, FULL, TG, SPLIT>(p, cp, rp, 7 * RB, x0);
+    load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cp, rp, 7 * RB, x0);
 #pragma unroll 1
     for (int blk = C / RB - 1; blk > 0; blk -= 2) {
-        load_rows<APC, GPC, FULL, TG, SPLIT>(p, cp, rp, (blk - 1) * RB, x1);
+        load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cp, rp, (blk - 1) * RB, x1);
         do_block(blk, x0);
-        if (blk > 1) load_rows<APC, GPC, FULL, TG, SPLIT>(p, cp, rp, (blk - 2) * RB, x0);
+        if (blk > 1) load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cp, rp, (blk - 2) * RB, x0);
         do_block(blk - 1, x1);
         if (c == 0) GDN_BTRACE(it, 10 + (C / RB - 1 - blk) / 2);
     }
 }
 
 // Full chunks (every chunk but a ragged last one) take the variant without per-token guards.
-template <bool APC, bool GPC, class TG, bool SPLIT>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
 __device__ __forceinline__ void grad_epilogue(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
                                               float gam, float xtot, float* scr, int it = 15) {
-    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT>(p, cp, tl, c, warp, gam, xtot, scr, it);
-    else grad_epilogue_t<APC, GPC, false, TG, SPLIT>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT, LG>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    else grad_epilogue_t<APC, GPC, false, TG, SPLIT, LG>(p, cp, tl, c, warp, gam, xtot, scr, it);
 }
 
 // Scalar gates: per-token sums over the channels (the epilogue group's per-warp partials, the
 // dv/dw pass's sum_j v dY), then rows 0-63 of the G lo tile are zeroed again for the next P6.
-template <bool APC, bool GPC, class TG>
+template <bool APC, bool GPC, class TG, bool LG>
 __device__ __forceinline__ void scalar_gate_finish(const Params& p, const ChunkPos& cp, int c, float* scr) {
     const Problem& pb = p.pb;
     if (c < cp.L) {
@@ -1284,7 +1284,7 @@ __device__ __forceinline__ void scalar_gate_finish(const Params& p, const ChunkP
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < 4; ++w) sum += scr[SX_RA / 4 + w * 64 + c];
-            p.dalpha[g1] = sum / pb.alpha_of(cp.hv, to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1)));
+            p.dalpha[g1] = sum / pb.alpha_t<LG>(cp.hv, to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1)));
         }
         if (!GPC) {
             float sum = scr[SX_DBV / 4 + c];
@@ -1307,7 +1307,7 @@ __device__ __forceinline__ void bar_sync_all(uint32_t id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <bool APC, bool GPC, class TG, bool SPLIT>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -1369,7 +1369,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 st16(gl + (uint32_t)(idx >> 9) * 16384u + (uint32_t)(idx & 511) * 16u, make_uint4(0u, 0u, 0u, 0u));
             }
         } else {
-            stage_chunk<APC, GPC, TG, SPLIT>(p, cx, c0, tl, tid - 128, xslot, gslot, 0u);
+            stage_chunk<APC, GPC, TG, SPLIT, LG>(p, cx, c0, tl, tid - 128, xslot, gslot, 0u);
         }
     }
     for (int it = 0; ci < nch; ++it, ci += gridDim.x) {
@@ -1475,14 +1475,14 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             if (tid == 0) GDN_BTRACE(it, 9);
             if (!*cx.abort_flag)
-                grad_epilogue<APC, GPC, TG, SPLIT>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
+                grad_epilogue<APC, GPC, TG, SPLIT, LG>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
             if (tid == 0) GDN_BTRACE(it, 5);
             if (!APC || !GPC) bar_arrive_all(3);  // per-warp partials of the scalar gates written
         } else {
             if (nx < nch)
-                stage_chunk<APC, GPC, TG, SPLIT>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
+                stage_chunk<APC, GPC, TG, SPLIT, LG>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
             if (tid == 128) GDN_BTRACE(it, 8);
-            grad_dv_dw<GPC, TG, SPLIT>(p, cx, cp, tid - 128, scr);
+            grad_dv_dw<GPC, TG, SPLIT, LG>(p, cx, cp, tid - 128, scr);
             named_bar(2, 128);
             if (tid == 128) GDN_BTRACE(it, 4);
             // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land
@@ -1492,7 +1492,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             if (!APC || !GPC) {
                 bar_sync_all(3);
-                if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG>(p, cp, tid - 128, scr);
+                if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG, LG>(p, cp, tid - 128, scr);
             }
         }
         if (tid == 0) *stop_slot = *cx.abort_flag;

@@ -340,7 +340,7 @@ __device__ __forceinline__ void load_vw(const Ctx& cx, int n, int b, int hv, con
     }
 }
 
-template <bool APC, bool GPC, bool GATE, class TG, bool SPLIT>
+template <bool APC, bool GPC, bool GATE, class TG, bool SPLIT, bool LG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -508,7 +508,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const uint32_t off = (uint32_t)ii * 128u + xo[ii & 7];
                         const float vv = SPLIT ? bf(vt, off) + bf(vt + 16384, off) : bf(vt, off);
                         float ww;
-                        if (GPC) ww = pb.sig_of(bf(vt + 16384, off));
+                        if (GPC) ww = pb.sig_t<LG>(bf(vt + 16384, off));
                         else ww = sgb[rr];
                         y2[e] = vv * ww - __uint_as_float(r[ii]);
                     }
@@ -750,15 +750,15 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float* sg = reinterpret_cast<float*>(sm + SM_SG) + pm * 128;
                 if (c < 64) {
                     if (m == 0) {
-                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t0, c, L, hv, 1.f, 1);
-                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t0, c, L, hv, 0.f, 2);
+                        if (!APC) ga_next = gate_or<1, LG>(alpha_g, pb, b, t0, c, L, hv, 1.f);
+                        if (!GPC) gb_next = gate_or<2, LG>(beta_g, pb, b, t0, c, L, hv, 0.f);
                     }
                     sg[c] = ga_next;
                     sg[64 + c] = gb_next;
                     if (m + 1 < NT) {
                         const int t1 = t0 + C, L1 = min(C, pb.T - t1);
-                        if (!APC) ga_next = gate_or(alpha_g, pb, b, t1, c, L1, hv, 1.f, 1);
-                        if (!GPC) gb_next = gate_or(beta_g, pb, b, t1, c, L1, hv, 0.f, 2);
+                        if (!APC) ga_next = gate_or<1, LG>(alpha_g, pb, b, t1, c, L1, hv, 1.f);
+                        if (!GPC) gb_next = gate_or<2, LG>(beta_g, pb, b, t1, c, L1, hv, 0.f);
                     }
                 }
             }
@@ -789,9 +789,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float a8[8];
                     if (APC) {
                         unpack8(ld16(RA + a64 + u * 128u + ((ch ^ u) << 4)), a8);
-                        if (pb.gate_logits) {  // alpha from its logit
+                        if constexpr (LG) {  // alpha from its logit
 #pragma unroll
-                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_t<LG>(hv, a8[e_]);
                         }
                         if (r >= L) {
 #pragma unroll
@@ -840,9 +840,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float a8[8], k8[8], q8[8], b8[8];
                     if (APC) {
                         unpack8(ld16(RA + o64), a8);
-                        if (pb.gate_logits) {  // alpha from its logit
+                        if constexpr (LG) {  // alpha from its logit
 #pragma unroll
-                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_of(hv, a8[e_]);
+                            for (int e_ = 0; e_ < 8; ++e_) a8[e_] = pb.alpha_t<LG>(hv, a8[e_]);
                         }
                         if (r >= L) {
 #pragma unroll
@@ -867,9 +867,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     if (GPC) {
                         unpack8(ld16(RQB + oe), b8);
-                        if (pb.gate_logits) {  // b from its logit
+                        if constexpr (LG) {  // b from its logit
 #pragma unroll
-                            for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_of(b8[e_]);
+                            for (int e_ = 0; e_ < 8; ++e_) b8[e_] = pb.sig_t<LG>(b8[e_]);
                         }
                     } else {
                         const float bv = sga[pm * 128 + 64 + r];

@@ -1,34 +1,14 @@
-// Host side of the tensor-core chunk forward: TMA descriptors, dispatch, launch.
+// Host side of the tensor-core chunk forward: TMA descriptors and parameters; the launches of
+// each gate form are in tc_fwd_gates.cu and tc_fwd_logits.cu.
 #include <cuda.h>
 
 #include <type_traits>
 
 #include "launch.h"
-#include "tc_chunk_fwd.cuh"
+#include "tc_fwd_launch.cuh"
 #include "tma_host.h"
 
 namespace gdn {
-
-namespace {
-
-template <bool APC, bool GPC, bool GATE, class TG, bool SPLIT = false>
-cudaError_t launch_tc(const CUtensorMap* maps, const tcfwd::Params& p, cudaStream_t st) {
-    auto kernel = tcfwd::chunk_fwd_kernel<APC, GPC, GATE, TG, SPLIT>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tcfwd::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    kernel<<<p.pb.B * p.pb.Hv, tcfwd::kThreads, tcfwd::kSmemBytes, st>>>(maps[0], maps[1], maps[2], maps[3],
-                                                                        maps[4], maps[5], maps[6], p);
-    count_launch();
-    return cudaGetLastError();
-}
-
-template <bool APC, bool GPC, class TG>
-cudaError_t launch_tc_g(bool gate, const CUtensorMap* maps, const tcfwd::Params& p, cudaStream_t st) {
-    return gate ? launch_tc<APC, GPC, true, TG>(maps, p, st) : launch_tc<APC, GPC, false, TG>(maps, p, st);
-}
-
-}  // namespace
 
 bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags f) {
     if (!bf16_inputs || pb.dk != 128 || pb.dv != 128 || pb.T < 1) return false;
@@ -77,21 +57,8 @@ cudaError_t tc_chunk_fwd_kernel(const Problem& pb, const ChunkIO& io, Flags f, b
         p.vp_lo = save->vp_lo;
         p.o_raw = save->o_raw;
     }
-    const bool gate = f.gate;
-    if (split) {
-        // the layer core's form (scalar gates): with the swish output gate (its forward), or
-        // without it (the raw o and the chunk states for its backward)
-        if (gate)
-            return bf16_gates ? launch_tc<false, false, true, __nv_bfloat16, true>(maps, p, st)
-                              : launch_tc<false, false, true, float, true>(maps, p, st);
-        return bf16_gates ? launch_tc<false, false, false, __nv_bfloat16, true>(maps, p, st)
-                          : launch_tc<false, false, false, float, true>(maps, p, st);
-    }
-    if (f.apc && f.gpc) return launch_tc_g<true, true, __nv_bfloat16>(gate, maps, p, st);
-    if (f.apc) return launch_tc_g<true, false, __nv_bfloat16>(gate, maps, p, st);
-    if (f.gpc) return launch_tc_g<false, true, __nv_bfloat16>(gate, maps, p, st);
-    if (bf16_gates) return launch_tc_g<false, false, __nv_bfloat16>(gate, maps, p, st);
-    return launch_tc_g<false, false, float>(gate, maps, p, st);
+    return pb.gate_logits ? tc_fwd_dispatch<true>(maps, p, f, split, bf16_gates, st)
+                          : tc_fwd_dispatch<false>(maps, p, f, split, bf16_gates, st);
 }
 }  // namespace
 
@@ -107,10 +74,3 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
 }
 
 }  // namespace gdn
-
-#ifdef GDN_FWD_TRACE
-// Profiling builds only: copy the phase timestamps of CTA 0 of the last forward to the host.
-extern "C" __attribute__((visibility("default"))) int gdn_fwd_trace_read(unsigned long long* host) {
-    return (int)cudaMemcpyFromSymbol(host, gdn::tcfwd::g_fwd_trace, sizeof(unsigned long long) * 64 * 32);
-}
-#endif
