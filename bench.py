@@ -62,14 +62,12 @@ def fwd_bytes_per_token(wl, T=None, with_h0=None, gate=False):
     return b
 
 
-def bwd_bytes_per_token(wl, T=None, grad_bytes=None):
+def bwd_bytes_per_token(wl, T=None):
     """API-level bytes of one backward token: q, k, v, alpha, b, w and dO read; the gradients of
-    q, k, v, alpha, b, w written (+ h0 read, dh0 written).  The algorithmic count sizes every
-    gradient like its input (bf16 here); `grad_bytes=4` gives the bytes the library actually
-    writes (its gradients are fp32)."""
+    q, k, v, alpha, b, w written in their inputs' dtypes (+ h0 read, dh0 written in fp32)."""
     T = T or wl.T
     es, gs = _es(wl.dtype), _es(wl.gate_dtype)
-    ges, ggs = (grad_bytes or es), (grad_bytes or gs)
+    ges, ggs = es, gs
     n_qk = wl.Hk * 2 * wl.dk
     n_v = wl.Hv * wl.dv
     n_a = wl.Hv * (wl.dk if wl.alpha_per_channel else 1)
@@ -294,11 +292,12 @@ def bench_headline(args, dist, peaks, peak_kind, stream, device):
                         dtype=torch.uint8, device=device)
     fa, _ = gdn.fwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], o=o, ht=ht, bwd_cache=cache, **gates(g))
     ws_f = torch.empty(lib.gdn_chunk_fwd_workspace_size(ctypes.byref(fa)), dtype=torch.uint8, device=device)
-    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=device)
-    grads = {"dq": f32(g["q"]), "dk": f32(g["k"]), "dv": f32(g["v"]), "dalpha": f32(g["alpha"]),
-             "db": f32(g["b"]), "dw": f32(g["w"]), "dh0": f32(g["h0"])}
+    # gradients in the inputs' dtype (bf16; fp32 accumulation inside), dh0 in fp32
+    grads = {"dq": torch.empty_like(g["q"]), "dk": torch.empty_like(g["k"]), "dv": torch.empty_like(g["v"]),
+             "dalpha": torch.empty_like(g["alpha"]), "db": torch.empty_like(g["b"]), "dw": torch.empty_like(g["w"]),
+             "dh0": torch.empty_like(g["h0"])}
     ba, _ = gdn.bwd_args(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], grads=grads,
-                         fwd_cache=cache, **gates(g))
+                         fwd_cache=cache, grads_in_dtype=True, **gates(g))
     ws_b = torch.empty(lib.gdn_chunk_bwd_workspace_size(ctypes.byref(ba)), dtype=torch.uint8, device=device)
     sptr = ctypes.c_void_p(stream.cuda_stream)
 
@@ -343,9 +342,6 @@ def bench_headline(args, dist, peaks, peak_kind, stream, device):
     roof = roofline(dom[0], dom[1], dom[2] * 1e-3, peaks, peak_kind,
                     f"gdn_chunk_{dominant} call (dominant call of the step; its kernels back to back)",
                     traffic=BWD_CALL_TRAFFIC_BYTES if dominant == "bwd" else None)
-    if dominant == "bwd":
-        # the gradients leave as fp32: what the call writes, beside the algorithmic (bf16) count
-        roof["written_bytes_fp32_grads"] = int(bwd_bytes_per_token(wl, grad_bytes=4) * tokens)
     step_roof = roofline(bytes_f + bytes_b, flops_f + flops_b, ms * 1e-3, peaks, peak_kind,
                          "whole fwd+bwd step")
     return {"ms": ms, "tokens": tokens, "launches_per_step": launches_per_step, "fwd_ms": fwd_ms,
@@ -392,7 +388,7 @@ def bench_headline_e2e(args, dist, x, stream, device, slices=8):
             o, ht = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], b=d["b"], w=d["w"], h0=d["h0"],
                                       bwd_cache=caches[i], stream=stream)
             gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], b=d["b"], w=d["w"], h0=d["h0"],
-                                   grad_o=d["dout"], fwd_cache=caches[i], stream=stream)
+                                   grad_o=d["dout"], fwd_cache=caches[i], grads_in_dtype=True, stream=stream)
             res.append({"o": o, "ht": ht, **gr})
             ev_c.append(torch.cuda.Event())
             ev_c[-1].record(stream)
@@ -595,7 +591,7 @@ def run_reference(args):
 # --------------------------------------------------------------------------------------------
 def _profile_train_b2_t2048():
     """GDN-2 training step on B=2 T=2048 H=16 d=128 bf16 (seed 21), twice: the forward keeping the
-    backward cache, then the backward from it."""
+    backward cache, then the backward from it (gradients in bf16, as the benchmark takes them)."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     from gated_delta_rule_76_b200.inputs import draw
@@ -607,15 +603,17 @@ def _profile_train_b2_t2048():
                         dtype=torch.uint8, device="cuda")
     for _ in range(2):
         gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
-        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache, **kw)
+        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache,
+                                  grads_in_dtype=True, **kw)
     torch.cuda.synchronize()
-    print("ok", float(grads["dq"].abs().mean()))
+    print("ok", float(grads["dq"].float().abs().mean()))
     return 0
 
 
 def _profile_train_b8_t1024():
     """GDN-2 training step on B=8 T=1024 H=16 d=128 bf16 (seed 21): the headline's 128 (sequence, head)
-    pairs, a quarter of its tokens; twice: the forward keeping the cache, then the backward from it."""
+    pairs, a quarter of its tokens; twice: the forward keeping the cache, then the backward from it
+    (gradients in bf16, as the benchmark takes them)."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     from gated_delta_rule_76_b200.inputs import draw
@@ -627,9 +625,10 @@ def _profile_train_b8_t1024():
                         dtype=torch.uint8, device="cuda")
     for _ in range(2):
         gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
-        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache, **kw)
+        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache,
+                                  grads_in_dtype=True, **kw)
     torch.cuda.synchronize()
-    print("ok", float(grads["dq"].abs().mean()))
+    print("ok", float(grads["dq"].float().abs().mean()))
     return 0
 
 
@@ -664,8 +663,8 @@ def _profile_layer_b2_t16384():
 
 
 def _profile_train_b8_t4096():
-    """The headline training step (gdn_chunk_fwd keeping the cache, gdn_chunk_bwd from it) on its
-    full workload, three times."""
+    """The headline training step (gdn_chunk_fwd keeping the cache, gdn_chunk_bwd from it, gradients
+    in bf16) on its full workload, three times."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     x, g = chunk_inputs(HEADLINE, torch.device("cuda"), with_dout=True)
@@ -674,9 +673,10 @@ def _profile_train_b8_t4096():
                         dtype=torch.uint8, device="cuda")
     for _ in range(3):
         gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], bwd_cache=cache, **kw)
-        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache, **kw)
+        grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], grad_o=g["dout"], fwd_cache=cache,
+                                  grads_in_dtype=True, **kw)
     torch.cuda.synchronize()
-    print("ok", float(grads["dq"].abs().mean()))
+    print("ok", float(grads["dq"].float().abs().mean()))
     return 0
 
 

@@ -19,6 +19,22 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Gradient stores: fp32, or bf16 when the gradients are returned in the inputs' dtype (rounded
+// once, from the fp32 value).
+__device__ __forceinline__ void st_g(float* p, float v) { *p = v; }
+__device__ __forceinline__ void st_g(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+// Four consecutive elements (16-byte aligned for fp32, 8-byte aligned for bf16).
+__device__ __forceinline__ void st4_g(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void st4_g(__nv_bfloat16* p, float a, float b, float c, float d) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
 // ---- problem description passed to every kernel by value ---------------------------------

@@ -247,11 +247,15 @@ gdn_status check_bwd(const gdn_bwd_args* a) {
     if ((s = check_logits(a->gate_logits, a->alpha_scale, a->grad_alpha_scale))) return s;
     if (a->fwd_cache && (reinterpret_cast<uintptr_t>(a->fwd_cache) & 255u))
         return fail(GDN_ERR_INVALID_ARG, "fwd_cache is not 256-byte aligned");
-    const size_t na4 = na / gs * 4, nb4 = nb / gs * 4;
+    if (a->grads_in_dtype != 0 && a->grads_in_dtype != 1)
+        return fail(GDN_ERR_INVALID_ARG, "grads_in_dtype must be 0 or 1");
+    // element sizes of the gradients: fp32, or the inputs' dtypes
+    const size_t ge = a->grads_in_dtype ? es : 4, gg = a->grads_in_dtype ? gs : 4;
+    const size_t nag = na / gs * gg, nbg = nb / gs * gg;
     const Buf out[] = {
-        {a->grad_q, BT * a->Hk * a->dk * 4, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * 4, "grad_k"},
-        {a->grad_v, BT * a->Hv * a->dv * 4, "grad_v"}, {a->grad_alpha, na4, "grad_alpha"},
-        {a->grad_b, nb4, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * 4, "grad_w"}, {a->grad_h0, st, "grad_h0"},
+        {a->grad_q, BT * a->Hk * a->dk * ge, "grad_q"}, {a->grad_k, BT * a->Hk * a->dk * ge, "grad_k"},
+        {a->grad_v, BT * a->Hv * a->dv * ge, "grad_v"}, {a->grad_alpha, nag, "grad_alpha"},
+        {a->grad_b, nbg, "grad_b"}, {a->grad_w, BT * a->Hv * a->dv * gg, "grad_w"}, {a->grad_h0, st, "grad_h0"},
         {a->grad_alpha_scale, (size_t)a->Hv * 4, "grad_alpha_scale"},
     };
     return check_buffers(in, 12, out, 8);
@@ -491,6 +495,11 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
             return fail(GDN_ERR_INVALID_ARG, "fwd_cache has %zu bytes, %zu needed", a->fwd_cache_bytes,
                         plan_tc_cache(pb).bytes);
     }
+    // gradients in bf16: written by the tensor-core kernels (the CUDA-core backward writes fp32)
+    const bool grad_bf16 = a->grads_in_dtype && a->dtype == GDN_BF16;
+    if (grad_bf16 && !tc)
+        return fail(GDN_ERR_UNSUPPORTED, "grads_in_dtype with bf16 inputs: only the tensor-core backward (dk = dv = "
+                                         "128, bf16 channel gates) returns bf16 gradients");
     TcBwdWs tplan = tc ? plan_tc_bwd_ws(pb, !direct, a->fwd_cache != nullptr) : TcBwdWs{};
     if ((s = check_workspace(workspace, workspace_bytes, tc ? tplan.bytes : plan.bytes))) return s;
     ChunkIO io{};
@@ -498,6 +507,7 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     io.h0 = a->h0; io.dout = a->grad_o; io.dht = a->grad_ht; io.dq = a->grad_q; io.dk = a->grad_k;
     io.dv = a->grad_v; io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = a->grad_w;
     io.dh0 = a->grad_h0;
+    io.grad_type = grad_bf16 ? 1 : 0;
     Flags f{a->alpha_per_channel != 0, a->gates_per_channel != 0, false};
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
     if (e == cudaSuccess)
@@ -517,7 +527,7 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
     // gates as logits: the gradients of the gates become those of their logits
     if (e == cudaSuccess && pb.gate_logits)
         e = gate_logit_grads(pb, f, a->gate_dtype == GDN_F32, a->alpha, a->b, a->w, a->grad_alpha, a->grad_b,
-                             a->grad_w, a->grad_alpha_scale, st);
+                             a->grad_w, grad_bf16 && a->gate_dtype == GDN_BF16, a->grad_alpha_scale, st);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_chunk_bwd");
 }
 
@@ -985,7 +995,7 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     // 6. gates as logits: the gradients of the gates become those of their logits
     if (pb.gate_logits)
         e = gate_logit_grads(pb, f, a->gate_dtype == GDN_F32, a->alpha, a->b, a->w, a->grad_alpha, a->grad_b,
-                             a->grad_w, a->grad_alpha_scale, sm);
+                             a->grad_w, false, a->grad_alpha_scale, sm);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_layer_core_bwd (gate logits)");
 }
 

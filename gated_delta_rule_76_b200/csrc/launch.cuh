@@ -21,11 +21,16 @@ cudaError_t launch_kernel(K kernel, dim3 grid, dim3 block, size_t smem, cudaStre
 }
 
 // dq or dk of the key heads from the per-value-head partials [B,T,Hv,dk] (gqa_reduce_kernel).
-inline cudaError_t gqa_reduce(const Problem& pb, const float* part, float* out, cudaStream_t st) {
+// out_bf16: the sums are written in bf16 (else fp32).
+inline cudaError_t gqa_reduce(const Problem& pb, const float* part, void* out, bool out_bf16, cudaStream_t st) {
     const long rows = (long)pb.B * pb.T;
     const int blocks = (int)(rows < 148L * 8 ? rows : 148L * 8);
-    return launch_kernel(gqa_reduce_kernel, dim3(blocks), dim3(256), (size_t)(pb.Hv + pb.Hk + 1) * sizeof(int), st,
-                         pb, part, out);
+    const size_t smem = (size_t)(pb.Hv + pb.Hk + 1) * sizeof(int);
+    if (out_bf16)
+        return launch_kernel(gqa_reduce_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), smem, st, pb, part,
+                             static_cast<__nv_bfloat16*>(out));
+    return launch_kernel(gqa_reduce_kernel<float>, dim3(blocks), dim3(256), smem, st, pb, part,
+                         static_cast<float*>(out));
 }
 
 #define GDN_TRY(expr)                         \
@@ -72,8 +77,8 @@ cudaError_t chunk_bwd_t(const Problem& pb, const ChunkIO& io, const ChunkWs& ws,
                         direct_qk ? static_cast<float*>(io.dk) : ws.dk_v, direct_qk, ws.S0,
                         (long)pb.NT * DK * DK, ws.sbuf, st));
     if (!direct_qk) {
-        GDN_TRY(gqa_reduce(pb, (const float*)ws.dq_v, static_cast<float*>(io.dq), st));
-        GDN_TRY(gqa_reduce(pb, (const float*)ws.dk_v, static_cast<float*>(io.dk), st));
+        GDN_TRY(gqa_reduce(pb, (const float*)ws.dq_v, io.dq, false, st));
+        GDN_TRY(gqa_reduce(pb, (const float*)ws.dk_v, io.dk, false, st));
     }
     return cudaSuccess;
 }

@@ -58,18 +58,19 @@ cudaError_t tc_chunk_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
 
 // Exact sequential recurrence (seq.cu) for the pairs marked in flags: the forward (o, the output
 // before the gate, ht) and the backward (every gradient; ck: per pair ck_stride floats for the
-// states entering chunks 1..NT-1, sbuf: seq_sbuf_floats()).  dq, dk are per key head when direct,
-// else per value head.
+// states entering chunks 1..NT-1, sbuf: seq_sbuf_floats()).  dq, dk are per key head when direct
+// (in the gradients' type, io.grad_type), else per value head (fp32 partials).
 size_t seq_sbuf_floats(const Problem& pb);
 cudaError_t seq_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
                     float* o_raw, cudaStream_t st);
 cudaError_t seq_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
-                    float* dq, float* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st);
+                    void* dq, void* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st);
 
 // Gates as logits (gates.cu): after a backward, the gates' gradients become those of their logits
-// (in place), and alpha's scale gets its gradient (dalpha_scale [Hv], may be NULL).
+// (in place, fp32 or, with grad_bf16, bf16), and alpha's scale gets its gradient (dalpha_scale [Hv]
+// fp32, may be NULL).
 cudaError_t gate_logit_grads(const Problem& pb, Flags f, bool tg_f32, const void* x_alpha, const void* x_b,
-                             const void* x_w, float* dalpha, float* db, float* dw, float* dalpha_scale,
+                             const void* x_w, void* dalpha, void* db, void* dw, bool grad_bf16, float* dalpha_scale,
                              cudaStream_t st);
 
 // Sequence split along time (seqpar.cu): S = I for `pairs` states of d x d; S_out = op(M) S_in + N

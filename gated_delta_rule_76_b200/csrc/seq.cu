@@ -84,17 +84,19 @@ cudaError_t seq_fwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32,
 }
 
 cudaError_t seq_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32, bool tg_f32, const int* flags,
-                    float* dq, float* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st) {
+                    void* dq, void* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st) {
     seq::Params p = common_params(pb, io, f, flags);
     p.dout = io.dout;
     p.dht = io.dht;
     p.dq = dq;
     p.dk = dk;
     p.direct = direct ? 1 : 0;
-    p.dv = static_cast<float*>(io.dv);
-    p.dalpha = static_cast<float*>(io.dalpha);
-    p.db = static_cast<float*>(io.db);
-    p.dw = static_cast<float*>(io.dw);
+    p.dv = io.dv;
+    p.dalpha = io.dalpha;
+    p.db = io.db;
+    p.dw = io.dw;
+    p.grad_bf16 = io.grad_type == 1 ? 1 : 0;
+    p.gate_grad_bf16 = io.grad_type == 1 && !tg_f32 ? 1 : 0;
     p.dh0 = io.dh0;
     p.ck = ck;
     p.ck_stride = ck_stride;

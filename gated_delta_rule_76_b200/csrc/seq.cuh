@@ -58,13 +58,22 @@ struct Params {
     // backward
     const void* dout;                        // [B,T,Hv,dv] TIn
     const float* dht;                        // [B,Hv,dk,dv] or NULL
-    float *dq, *dk;                          // [B,T,Hk,dk] when direct, else [B,T,Hv,dk] per value head
+    void *dq, *dk;                           // [B,T,Hk,dk] when direct, else [B,T,Hv,dk] per value head
     int direct;
-    float *dv, *dalpha, *db, *dw, *dh0;      // shapes of v, alpha, b (or beta), w; dh0 may be NULL
+    void *dv, *dalpha, *db, *dw;             // shapes of v, alpha, b (or beta), w
+    int grad_bf16;                           // dv (and dq, dk when direct) in bf16
+    int gate_grad_bf16;                      // dalpha, db, dw in bf16
+    float* dh0;                              // may be NULL
     float* ck;                               // per pair ck_stride floats: states entering chunks 1..NT-1
     long ck_stride;
     float* sbuf;                             // per pair kTB states (floats kTB * dk * dv)
 };
+
+// One gradient element, fp32 or bf16.
+__device__ __forceinline__ void put_g(void* p, long i, float v, bool bf) {
+    if (bf) st_g(static_cast<__nv_bfloat16*>(p) + i, v);
+    else st_g(static_cast<float*>(p) + i, v);
+}
 
 // ---- staging of one block of kTB tokens ---------------------------------------------------
 // Vectors of a token, in the fp32 staging buffer [kTB][NVEC][D]: alpha, b, k, q, v, w, and the
@@ -526,13 +535,14 @@ __global__ void __launch_bounds__(D * D / 32) seq_bwd_kernel(Params p) {
                 for (int m = 0; m < NV_LANE; ++m) {
                     const int idx = NV_LANE * (lane % W) + m, qn = idx / 8, i = idx % 8, c = c0 + i;
                     const float val = red32[m];
-                    if (qn == 0) p.dq[tok_qk + c] = val;
-                    else if (qn == 1) p.dk[tok_qk + c] = val + bg[i] * de_l[m];
+                    const bool qbf = p.grad_bf16 && p.direct;  // per-value-head partials stay fp32
+                    if (qn == 0) put_g(p.dq, tok_qk + c, val, qbf);
+                    else if (qn == 1) put_g(p.dk, tok_qk + c, val + bg[i] * de_l[m], qbf);
                     else if (qn == 2) {
-                        if (p.gpc) p.db[pb.gate_row(b, t, hv, D) + c] = kk[i] * val;
+                        if (p.gpc) put_g(p.db, pb.gate_row(b, t, hv, D) + c, kk[i] * val, p.gate_grad_bf16);
                         else atomicAdd(acc + 1, kk[i] * val);
                     } else {
-                        if (p.apc) p.dalpha[pb.gate_row(b, t, hv, D) + c] = val;
+                        if (p.apc) put_g(p.dalpha, pb.gate_row(b, t, hv, D) + c, val, p.gate_grad_bf16);
                         else atomicAdd(acc + 0, val);
                     }
                 }
@@ -540,8 +550,8 @@ __global__ void __launch_bounds__(D * D / 32) seq_bwd_kernel(Params p) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const long off = pb.v_row(b, t, hv) + j0 + u;
-                        p.dv[off] = ww[u] * dvw[u];
-                        if (p.gpc) p.dw[off] = vv[u] * dvw[u];
+                        put_g(p.dv, off, ww[u] * dvw[u], p.grad_bf16);
+                        if (p.gpc) put_g(p.dw, off, vv[u] * dvw[u], p.gate_grad_bf16);
                         else atomicAdd(acc + 1, vv[u] * dvw[u]);
                     }
                 }
@@ -553,8 +563,8 @@ __global__ void __launch_bounds__(D * D / 32) seq_bwd_kernel(Params p) {
                 __syncthreads();
                 if (tid == 0 && (!p.apc || !p.gpc)) {
                     const long g1 = pb.gate_row(b, t, hv, 1);
-                    if (!p.apc) p.dalpha[g1] = acc[0];
-                    if (!p.gpc) p.db[g1] = acc[1];
+                    if (!p.apc) put_g(p.dalpha, g1, acc[0], p.gate_grad_bf16);
+                    if (!p.gpc) put_g(p.db, g1, acc[1], p.gate_grad_bf16);
                     acc[0] = 0.f;
                     acc[1] = 0.f;
                 }

@@ -67,6 +67,7 @@ struct ChunkIO {
     const void* dout;
     const float* dht;
     void *dq, *dk, *dv, *dalpha, *db, *dw;
+    int grad_type;  // 0: the gradients above in fp32; 1: in bf16 (tensor-core backward only)
     float* dh0;
 };
 
@@ -756,8 +757,10 @@ constexpr size_t chunk_grad_smem() {
 // Sum per-value-head dq/dk [B,T,Hv,dk] over the value heads of each key head, ascending hv
 // (fixed order: deterministic).  The block first lists the value heads of every key head in
 // shared memory (dynamic: Hv + Hk + 1 ints); then each thread sums float4 columns of one token
-// row at a time.  dk is a multiple of 4 and every row starts 16-byte aligned.
-static __global__ void __launch_bounds__(256) gqa_reduce_kernel(Problem pb, const float* part, float* out) {
+// row at a time.  dk is a multiple of 4 and every row starts 16-byte aligned.  The sums are written
+// in OT (fp32, or bf16 for gradients returned in the inputs' dtype).
+template <class OT>
+static __global__ void __launch_bounds__(256) gqa_reduce_kernel(Problem pb, const float* part, OT* out) {
     extern __shared__ int heads[];  // heads[0 .. Hv): value heads grouped by key head; then Hk + 1 starts
     int* beg = heads + pb.Hv;
     if (threadIdx.x == 0) {
@@ -773,7 +776,6 @@ static __global__ void __launch_bounds__(256) gqa_reduce_kernel(Problem pb, cons
     const int q4 = pb.dk / 4, per_row = pb.Hk * q4;
     const long rows = (long)pb.B * pb.T;
     const float4* src = reinterpret_cast<const float4*>(part);
-    float4* dst = reinterpret_cast<float4*>(out);
     for (long bt = blockIdx.x; bt < rows; bt += gridDim.x) {
         for (int i = threadIdx.x; i < per_row; i += blockDim.x) {
             const int hk = i / q4, c = i - hk * q4;
@@ -782,7 +784,7 @@ static __global__ void __launch_bounds__(256) gqa_reduce_kernel(Problem pb, cons
                 const float4 x = __ldg(src + (bt * pb.Hv + heads[j]) * q4 + c);
                 s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
             }
-            dst[bt * per_row + i] = s;
+            st4_g(out + (bt * per_row + i) * 4, s.x, s.y, s.z, s.w);
         }
     }
 }

@@ -70,8 +70,11 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     float* dsc = reinterpret_cast<float*>(base + plan.dsc);
     auto* nyh = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_hi);
     auto* nyl = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_lo);
-    float* dq_v = direct ? static_cast<float*>(io.dq) : reinterpret_cast<float*>(base + plan.dq_v);
-    float* dk_v = direct ? static_cast<float*>(io.dk) : reinterpret_cast<float*>(base + plan.dk_v);
+    // dq, dk: the outputs when value heads map one to one on key heads, else per-value-head fp32
+    // partials in the workspace, summed at the end
+    void* dq_v = direct ? io.dq : base + plan.dq_v;
+    void* dk_v = direct ? io.dk : base + plan.dk_v;
+    const bool gbf = io.grad_type == 1;  // gradients returned in bf16
     int* flags = reinterpret_cast<int*>(base + plan.flags);  // zeroed by the caller
 
     const bool split = io.q_lo != nullptr;
@@ -132,15 +135,26 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     gp.dsc = dsc;
     gp.dq = dq_v;
     gp.dk = dk_v;
-    gp.dv = static_cast<float*>(io.dv);
-    gp.dalpha = static_cast<float*>(io.dalpha);
-    gp.db = static_cast<float*>(io.db);
-    gp.dw = static_cast<float*>(io.dw);
+    gp.dv = io.dv;
+    gp.dalpha = io.dalpha;
+    gp.db = io.db;
+    gp.dw = io.dw;
     gp.direct = direct ? 1 : 0;
     gp.err = err;
 
-    e = pb.gate_logits ? tc_bwd_dispatch<true>(ms, sp, m, gp, f, split, bf16_gates, st)
-                       : tc_bwd_dispatch<false>(ms, sp, m, gp, f, split, bf16_gates, st);
+    if (split && gbf) return cudaErrorInvalidValue;  // the layer core's form returns fp32 gradients
+    e = pb.gate_logits ? tc_scan_dispatch<true>(ms, sp, f, split, bf16_gates, st)
+                       : tc_scan_dispatch<false>(ms, sp, f, split, bf16_gates, st);
+    if (e != cudaSuccess) return e;
+    if (!gbf)
+        e = pb.gate_logits ? tc_grad_dispatch<true, float, float>(m, gp, f, split, bf16_gates, st)
+                           : tc_grad_dispatch<false, float, float>(m, gp, f, split, bf16_gates, st);
+    else if (direct)
+        e = pb.gate_logits ? tc_grad_dispatch<true, __nv_bfloat16, __nv_bfloat16>(m, gp, f, split, bf16_gates, st)
+                           : tc_grad_dispatch<false, __nv_bfloat16, __nv_bfloat16>(m, gp, f, split, bf16_gates, st);
+    else
+        e = pb.gate_logits ? tc_grad_dispatch<true, __nv_bfloat16, float>(m, gp, f, split, bf16_gates, st)
+                           : tc_grad_dispatch<false, __nv_bfloat16, float>(m, gp, f, split, bf16_gates, st);
     if (e != cudaSuccess) return e;
     // 3. pairs whose decay left the factors' range (marked by the scan): every gradient again,
     //    exactly; the pair's slice of the dS array holds its checkpoints
@@ -149,8 +163,8 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     if (e != cudaSuccess || direct) return e;
 
     // 4. GQA: sum the per-value-head dq, dk over the value heads of each key head
-    GDN_TRY(gqa_reduce(pb, (const float*)dq_v, static_cast<float*>(io.dq), st));
-    return gqa_reduce(pb, (const float*)dk_v, static_cast<float*>(io.dk), st);
+    GDN_TRY(gqa_reduce(pb, static_cast<const float*>(dq_v), io.dq, gbf, st));
+    return gqa_reduce(pb, static_cast<const float*>(dk_v), io.dk, gbf, st);
 }
 
 }  // namespace gdn

@@ -1,10 +1,13 @@
-// Instantiations of the tensor-core chunk backward for gates given as values.
+// Instantiations of the tensor-core chunk backward: gates given as values, fp32 gradients.
 #define GDN_TC_BWD_INSTANTIATE
+#define GDN_TC_BWD_SCAN
 #include "tc_bwd_launch.cuh"
 
 namespace gdn {
-template cudaError_t tc_bwd_dispatch<false>(const CUtensorMap*, const tcbwd::scan::Params&, const CUtensorMap*,
-                                          const tcbwd::grad::Params&, Flags, bool, bool, cudaStream_t);
+template cudaError_t tc_scan_dispatch<false>(const CUtensorMap*, const tcbwd::scan::Params&, Flags,
+                                            bool, bool, cudaStream_t);
+template cudaError_t tc_grad_dispatch<false, float, float>(const CUtensorMap*, const tcbwd::grad::Params&,
+                                                     Flags, bool, bool, cudaStream_t);
 }  // namespace gdn
 
 #ifdef GDN_BWD_TRACE

@@ -1,7 +1,9 @@
 // Launches of the tensor-core chunk backward's two kernels (reverse state-gradient scan, chunk-parallel
-// gradients) for one gate form (LG: gates given as logits), with the dispatch over their
-// instantiations.  Each form is compiled in its own translation unit (tc_bwd_gates.cu,
-// tc_bwd_logits.cu); tc_bwd.cu plans the workspace and builds the tensor maps and parameters.
+// gradients), with the dispatch over their instantiations: LG, gates given as logits; GT, the
+// gradients' type (fp32, or bf16: the inputs' dtype); QT, that of dq and dk (fp32 when they are
+// per-value-head partials summed afterwards).  Each (LG, GT) is compiled in its own translation
+// unit (tc_bwd_{gates,logits}{,_bf16}.cu); tc_bwd.cu plans the workspace and builds the tensor maps
+// and parameters.
 #pragma once
 
 #include <cuda.h>
@@ -12,8 +14,11 @@
 namespace gdn {
 
 template <bool LG>
-cudaError_t tc_bwd_dispatch(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
-                            const tcbwd::grad::Params& gp, Flags f, bool split, bool bf16_gates, cudaStream_t st);
+cudaError_t tc_scan_dispatch(const CUtensorMap* ms, const tcbwd::scan::Params& sp, Flags f, bool split,
+                             bool bf16_gates, cudaStream_t st);
+template <bool LG, class GT, class QT>
+cudaError_t tc_grad_dispatch(const CUtensorMap* mg, const tcbwd::grad::Params& gp, Flags f, bool split,
+                             bool bf16_gates, cudaStream_t st);
 
 #ifdef GDN_TC_BWD_INSTANTIATE
 namespace {
@@ -30,9 +35,9 @@ cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cuda
     return cudaGetLastError();
 }
 
-template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG, class GT, class QT>
 cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cudaStream_t st) {
-    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG, SPLIT, LG>;
+    auto kernel = tcbwd::grad::chunk_bwd_grad_kernel<APC, GPC, TG, SPLIT, LG, GT, QT>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tcbwd::grad::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -46,27 +51,39 @@ cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cuda
     return cudaGetLastError();
 }
 
-template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
-cudaError_t launch_both(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* mg,
-                        const tcbwd::grad::Params& gp, cudaStream_t st) {
-    cudaError_t e = launch_scan<APC, GPC, TG, SPLIT, LG>(ms, sp, st);
-    if (e != cudaSuccess) return e;
-    return launch_grad<APC, GPC, TG, SPLIT, LG>(mg, gp, st);
-}
-
 }  // namespace
 
+#ifdef GDN_TC_BWD_SCAN
 template <bool LG>
-cudaError_t tc_bwd_dispatch(const CUtensorMap* ms, const tcbwd::scan::Params& sp, const CUtensorMap* m,
-                            const tcbwd::grad::Params& gp, Flags f, bool split, bool bf16_gates, cudaStream_t st) {
+cudaError_t tc_scan_dispatch(const CUtensorMap* ms, const tcbwd::scan::Params& sp, Flags f, bool split,
+                             bool bf16_gates, cudaStream_t st) {
     if (split)
-        return bf16_gates ? launch_both<false, false, __nv_bfloat16, true, LG>(ms, sp, m, gp, st)
-                          : launch_both<false, false, float, true, LG>(ms, sp, m, gp, st);
-    if (f.apc && f.gpc) return launch_both<true, true, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
-    if (f.apc) return launch_both<true, false, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
-    if (f.gpc) return launch_both<false, true, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
-    if (bf16_gates) return launch_both<false, false, __nv_bfloat16, false, LG>(ms, sp, m, gp, st);
-    return launch_both<false, false, float, false, LG>(ms, sp, m, gp, st);
+        return bf16_gates ? launch_scan<false, false, __nv_bfloat16, true, LG>(ms, sp, st)
+                          : launch_scan<false, false, float, true, LG>(ms, sp, st);
+    if (f.apc && f.gpc) return launch_scan<true, true, __nv_bfloat16, false, LG>(ms, sp, st);
+    if (f.apc) return launch_scan<true, false, __nv_bfloat16, false, LG>(ms, sp, st);
+    if (f.gpc) return launch_scan<false, true, __nv_bfloat16, false, LG>(ms, sp, st);
+    if (bf16_gates) return launch_scan<false, false, __nv_bfloat16, false, LG>(ms, sp, st);
+    return launch_scan<false, false, float, false, LG>(ms, sp, st);
+}
+#endif
+
+// The layer core's split form returns fp32 gradients only.
+template <bool LG, class GT, class QT>
+cudaError_t tc_grad_dispatch(const CUtensorMap* m, const tcbwd::grad::Params& gp, Flags f, bool split,
+                             bool bf16_gates, cudaStream_t st) {
+    if constexpr (std::is_same<GT, float>::value) {
+        if (split)
+            return bf16_gates ? launch_grad<false, false, __nv_bfloat16, true, LG, GT, QT>(m, gp, st)
+                              : launch_grad<false, false, float, true, LG, GT, QT>(m, gp, st);
+    } else {
+        if (split) return cudaErrorInvalidValue;
+    }
+    if (f.apc && f.gpc) return launch_grad<true, true, __nv_bfloat16, false, LG, GT, QT>(m, gp, st);
+    if (f.apc) return launch_grad<true, false, __nv_bfloat16, false, LG, GT, QT>(m, gp, st);
+    if (f.gpc) return launch_grad<false, true, __nv_bfloat16, false, LG, GT, QT>(m, gp, st);
+    if (bf16_gates) return launch_grad<false, false, __nv_bfloat16, false, LG, GT, QT>(m, gp, st);
+    return launch_grad<false, false, float, false, LG, GT, QT>(m, gp, st);
 }
 #endif  // GDN_TC_BWD_INSTANTIATE
 

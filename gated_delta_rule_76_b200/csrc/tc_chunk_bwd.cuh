@@ -30,6 +30,8 @@
 #pragma once
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "tc_chunk_fwd.cuh"
 #include "umma.cuh"
@@ -802,12 +804,12 @@ struct Params {
     const __nv_bfloat16* v_lo;
     const float* s0;     // [B*Hv][NT][dv/4][dk][4]: row c, columns 4q..4q+3 at float4 (q * dk + c)
     const float* dsc;    // same layout
-    float* dq;           // [B,T,Hk,dk] (direct) or [B,T,Hv,dk] per value head
-    float* dk;
-    float* dv;           // [B,T,Hv,dv]
-    float* dalpha;
-    float* db;
-    float* dw;
+    void* dq;            // [B,T,Hk,dk] (direct, the gradients' type) or [B,T,Hv,dk] per value head (fp32)
+    void* dk;
+    void* dv;            // [B,T,Hv,dv]; this and the gate gradients in the gradients' type (fp32 or bf16)
+    void* dalpha;
+    void* db;
+    void* dw;
     int direct;          // dq, dk written per key head (no head sharing)
     int* err;
     uint64_t wait_ns;    // limit of every bounded wait; 0 = kWaitNs
@@ -1062,7 +1064,7 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
 // dv = w .* dY, dw = v .* dY (a scalar beta: sum_j v dY per token into scr[SX_DBV]); run by the
 // staging group after its staging, warp w: tokens w, w + 4, ..., lane l: value channels 4l .. 4l + 3.
 
-template <bool GPC, class TG, bool SPLIT, bool LG>
+template <bool GPC, class TG, bool SPLIT, bool LG, class GT>
 __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const ChunkPos& cp, int tt, float* scr) {
     const Problem& pb = p.pb;
     const int w = tt >> 5, l = tt & 31, j = 4 * l;
@@ -1108,11 +1110,10 @@ __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const
         }
         const long row = pb.v_row(cp.b, cp.t0 + min(r, cp.L - 1), cp.hv);
         if (r < cp.L) {
-            *reinterpret_cast<float4*>(p.dv + row + j) =
-                make_float4(w4[0] * dy[0], w4[1] * dy[1], w4[2] * dy[2], w4[3] * dy[3]);
+            st4_g(static_cast<GT*>(p.dv) + row + j, w4[0] * dy[0], w4[1] * dy[1], w4[2] * dy[2], w4[3] * dy[3]);
             if (GPC)
-                *reinterpret_cast<float4*>(p.dw + row + j) =
-                    make_float4(v4[0] * dy[0], v4[1] * dy[1], v4[2] * dy[2], v4[3] * dy[3]);
+                st4_g(static_cast<GT*>(p.dw) + row + j, v4[0] * dy[0], v4[1] * dy[1], v4[2] * dy[2],
+                      v4[3] * dy[3]);
         }
         if (!GPC) {
             const float sum = warp_sum(fmaf(v4[0], dy[0], fmaf(v4[1], dy[1], fmaf(v4[2], dy[2], v4[3] * dy[3]))));
@@ -1211,7 +1212,7 @@ __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, c
     }
 }
 
-template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT, bool LG>
+template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT, bool LG, class GT, class QT>
 __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
                                                 float gam, float xtot, float* scr, int it) {
     const float scale = p.pb.scale;
@@ -1235,10 +1236,10 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
             run += fmaf(dQh, scale * qv * G, fmaf(dEh, bv * kv * G, -dkc * kv * rg));
             const float dla = run + xtot;
             if (FULL || r < cp.L) {
-                p.dq[rp.o + r * rp.o_s] = scale * G * dQh;
-                p.dk[rp.o + r * rp.o_s] = fmaf(de, bv, dkc * rg);
-                if (GPC) p.db[rp.g + r * rp.g_s] = de * kv;
-                if (APC) p.dalpha[rp.g + r * rp.g_s] = dla * ra;
+                st_g(static_cast<QT*>(p.dq) + rp.o + r * rp.o_s, scale * G * dQh);
+                st_g(static_cast<QT*>(p.dk) + rp.o + r * rp.o_s, fmaf(de, bv, dkc * rg));
+                if (GPC) st_g(static_cast<GT*>(p.db) + rp.g + r * rp.g_s, de * kv);
+                if (APC) st_g(static_cast<GT*>(p.dalpha) + rp.g + r * rp.g_s, dla * ra);
             }
             if (!GPC) {
                 const float sum = warp_sum(de * kv);
@@ -1266,31 +1267,34 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
 }
 
 // Full chunks (every chunk but a ragged last one) take the variant without per-token guards.
-template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG, class GT, class QT>
 __device__ __forceinline__ void grad_epilogue(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
                                               float gam, float xtot, float* scr, int it = 15) {
-    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT, LG>(p, cp, tl, c, warp, gam, xtot, scr, it);
-    else grad_epilogue_t<APC, GPC, false, TG, SPLIT, LG>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT, LG, GT, QT>(p, cp, tl, c, warp, gam, xtot, scr, it);
+    else grad_epilogue_t<APC, GPC, false, TG, SPLIT, LG, GT, QT>(p, cp, tl, c, warp, gam, xtot, scr, it);
 }
 
 // Scalar gates: per-token sums over the channels (the epilogue group's per-warp partials, the
 // dv/dw pass's sum_j v dY), then rows 0-63 of the G lo tile are zeroed again for the next P6.
-template <bool APC, bool GPC, class TG, bool LG>
+template <bool APC, bool GPC, class TG, bool LG, class GT>
 __device__ __forceinline__ void scalar_gate_finish(const Params& p, const ChunkPos& cp, int c, float* scr) {
     const Problem& pb = p.pb;
+    // gradients in the inputs' dtypes: the scalar gates' in the gates' own type
+    using SG = typename std::conditional<std::is_same<GT, float>::value, float, TG>::type;
     if (c < cp.L) {
         const long g1 = pb.gate_row(cp.b, cp.t0 + c, cp.hv, 1);
         if (!APC) {
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < 4; ++w) sum += scr[SX_RA / 4 + w * 64 + c];
-            p.dalpha[g1] = sum / pb.alpha_t<LG>(cp.hv, to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1)));
+            st_g(static_cast<SG*>(p.dalpha) + g1,
+                 sum / pb.alpha_t<LG>(cp.hv, to_f32(__ldg(static_cast<const TG*>(p.alpha) + g1))));
         }
         if (!GPC) {
             float sum = scr[SX_DBV / 4 + c];
 #pragma unroll
             for (int w = 0; w < 4; ++w) sum += scr[SX_RB / 4 + w * 64 + c];
-            p.db[g1] = sum;
+            st_g(static_cast<SG*>(p.db) + g1, sum);
         }
     }
     named_bar(2, 128);
@@ -1307,7 +1311,7 @@ __device__ __forceinline__ void bar_sync_all(uint32_t id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kThreads) : "memory");
 }
 
-template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
+template <bool APC, bool GPC, class TG, bool SPLIT, bool LG, class GT, class QT>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -1475,14 +1479,14 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             if (tid == 0) GDN_BTRACE(it, 9);
             if (!*cx.abort_flag)
-                grad_epilogue<APC, GPC, TG, SPLIT, LG>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
+                grad_epilogue<APC, GPC, TG, SPLIT, LG, GT, QT>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
             if (tid == 0) GDN_BTRACE(it, 5);
             if (!APC || !GPC) bar_arrive_all(3);  // per-warp partials of the scalar gates written
         } else {
             if (nx < nch)
                 stage_chunk<APC, GPC, TG, SPLIT, LG>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
             if (tid == 128) GDN_BTRACE(it, 8);
-            grad_dv_dw<GPC, TG, SPLIT, LG>(p, cx, cp, tid - 128, scr);
+            grad_dv_dw<GPC, TG, SPLIT, LG, GT>(p, cx, cp, tid - 128, scr);
             named_bar(2, 128);
             if (tid == 128) GDN_BTRACE(it, 4);
             // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land
@@ -1492,7 +1496,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             if (!APC || !GPC) {
                 bar_sync_all(3);
-                if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG, LG>(p, cp, tid - 128, scr);
+                if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG, LG, GT>(p, cp, tid - 128, scr);
             }
         }
         if (tid == 0) *stop_slot = *cx.abort_flag;

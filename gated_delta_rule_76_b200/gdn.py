@@ -44,7 +44,7 @@ class BwdArgs(ctypes.Structure):
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32),
                 ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t), ("gate_logits", I32),
-                ("alpha_scale", P), ("grad_alpha_scale", P)]
+                ("alpha_scale", P), ("grad_alpha_scale", P), ("grads_in_dtype", I32)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -318,7 +318,8 @@ def gdn_state_compose(M, N, S, *, transpose: bool = False, out: Optional[torch.T
 
 
 def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, scale=1.0,
-             grad_o=None, grad_ht=None, grads=None, fwd_cache=None, alpha_scale=None) -> Tuple[BwdArgs, list]:
+             grad_o=None, grad_ht=None, grads=None, fwd_cache=None, alpha_scale=None,
+             grads_in_dtype: bool = False) -> Tuple[BwdArgs, list]:
     bb, ww, gpc = _gates(alpha, b, w, beta)
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
@@ -334,26 +335,28 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
                 dtype=_dt(q), gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
                 fwd_cache_bytes=0 if fwd_cache is None else fwd_cache.numel() * fwd_cache.element_size(),
                 gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale),
-                grad_alpha_scale=_ptr(g.get("dalpha_scale")))
+                grad_alpha_scale=_ptr(g.get("dalpha_scale")), grads_in_dtype=int(grads_in_dtype))
     return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g, fwd_cache, alpha_scale]
 
 
 def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None,
                   scale: float = 1.0, *, grad_o, grad_ht=None, want_dh0: bool = True,
                   fwd_cache: Optional[torch.Tensor] = None, alpha_scale: Optional[torch.Tensor] = None,
-                  workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """Chunkwise backward.  Returns fp32 dq, dk, dv, dalpha and db/dw (or dbeta), dh0.
+                  grads_in_dtype: bool = False, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> Dict[str, torch.Tensor]:
+    """Chunkwise backward.  Returns dq, dk, dv, dalpha and db/dw (or dbeta) in fp32, or with
+    ``grads_in_dtype`` in the dtypes of q and of the gates; dh0 in fp32.
     ``fwd_cache``: the cache a gdn_chunk_fwd(..., bwd_cache=) call filled with these same inputs
     (the forward is then not recomputed).  With ``alpha_scale`` the gates are logits: dalpha, db,
     dw, dbeta are the gradients of the logits, and dalpha_scale [Hv] that of alpha_scale."""
     bb, ww, gpc = _gates(alpha, b, w, beta)
-    f32 = lambda t: torch.empty(t.shape, dtype=torch.float32, device=t.device)
-    grads = {"dq": f32(q), "dk": f32(k), "dv": f32(v), "dalpha": f32(alpha)}
+    like = lambda t: torch.empty(t.shape, dtype=t.dtype if grads_in_dtype else torch.float32, device=t.device)
+    grads = {"dq": like(q), "dk": like(k), "dv": like(v), "dalpha": like(alpha)}
     if gpc:
-        grads["db"] = f32(b)
-        grads["dw"] = f32(w)
+        grads["db"] = like(b)
+        grads["dw"] = like(w)
     else:
-        grads["dbeta"] = f32(beta)
+        grads["dbeta"] = like(beta)
     if want_dh0:
         B, T, Hk, dk = q.shape
         Hv, dv = v.shape[2], v.shape[3]
@@ -362,7 +365,7 @@ def gdn_chunk_bwd(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=N
         grads["dalpha_scale"] = torch.empty(tuple(alpha_scale.shape), dtype=torch.float32, device=q.device)
     lib = load()
     a, keep = bwd_args(q, k, v, alpha, b, w, beta, h0, head_map, scale, grad_o, grad_ht, grads, fwd_cache,
-                       alpha_scale)
+                       alpha_scale, grads_in_dtype)
     need = lib.gdn_chunk_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, q.device, workspace)
     check(lib.gdn_chunk_bwd(ctypes.byref(a), _ptr(ws), need, _stream(stream)), "gdn_chunk_bwd")

@@ -159,6 +159,12 @@ GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, gdn_stream st
  * (GDN-2 summary, «Passage Arrière Conscient des Portes»).
  * grad_alpha is the gradient with respect to alpha itself (not log alpha).  grad_q and grad_k are summed
  * over the value heads that share a key head, in a fixed order (deterministic).
+ * Gradient dtype: fp32 by default.  With grads_in_dtype = 1 they are returned in the inputs' dtypes:
+ * grad_q, grad_k, grad_v in `dtype`, grad_alpha, grad_b, grad_w in `gate_dtype`, each rounded once
+ * from its fp32 value (accumulation stays fp32; sums over value heads are taken in fp32 before the
+ * rounding).  grad_h0 and grad_alpha_scale are fp32 always.  grads_in_dtype = 1 with dtype BF16 is
+ * served by the tensor-core backward only (dk = dv = 128, bf16 gates with channel gates); other
+ * bf16 problems return GDN_ERR_UNSUPPORTED.  With dtype F32 the two settings are the same.
  * ------------------------------------------------------------------------------------------ */
 typedef struct gdn_bwd_args {
     const void* q;        /* forward inputs, same layouts and dtypes as gdn_fwd_args */
@@ -171,13 +177,14 @@ typedef struct gdn_bwd_args {
     const int32_t* head_map;
     const void* grad_o;   /* [B,T,Hv,dv] dtype, gradient of o */
     const float* grad_ht; /* [B,Hv,dk,dv] gradient of the final state, NULL = zeros */
-    float* grad_q;        /* out [B,T,Hk,dk] fp32 */
-    float* grad_k;        /* out [B,T,Hk,dk] fp32 */
-    float* grad_v;        /* out [B,T,Hv,dv] fp32 */
-    float* grad_alpha;    /* out, shape of alpha, fp32 */
-    float* grad_b;        /* out, shape of b (grad of beta [B,T,Hv] when gates are scalar), fp32 */
-    float* grad_w;        /* out, shape of w, fp32; must be NULL when gates are scalar */
-    float* grad_h0;       /* out [B,Hv,dk,dv], may be NULL */
+    void* grad_q;         /* out [B,T,Hk,dk] fp32 (dtype with grads_in_dtype) */
+    void* grad_k;         /* out [B,T,Hk,dk] fp32 (dtype with grads_in_dtype) */
+    void* grad_v;         /* out [B,T,Hv,dv] fp32 (dtype with grads_in_dtype) */
+    void* grad_alpha;     /* out, shape of alpha, fp32 (gate_dtype with grads_in_dtype) */
+    void* grad_b;         /* out, shape of b (grad of beta [B,T,Hv] when gates are scalar), fp32 (gate_dtype
+                           * with grads_in_dtype) */
+    void* grad_w;         /* out, shape of w, fp32 (gate_dtype with grads_in_dtype); NULL for scalar gates */
+    float* grad_h0;       /* out [B,Hv,dk,dv] fp32, may be NULL */
     int64_t B, T, Hk, Hv, dk, dv;
     float scale;
     int32_t alpha_per_channel;
@@ -193,6 +200,7 @@ typedef struct gdn_bwd_args {
     int32_t gate_logits;       /* 1: alpha, b, w are logits; the gradients returned are those of the logits */
     const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
     float* grad_alpha_scale;   /* out [Hv] fp32, may be NULL (must be NULL without gate_logits) */
+    int32_t grads_in_dtype;    /* 1: gradients in the inputs' dtypes (see above); 0: fp32 */
 } gdn_bwd_args;
 
 GDN_API size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args);

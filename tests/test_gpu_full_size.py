@@ -44,9 +44,10 @@ def gate_kw(x, sl=slice(None)):
 
 def test_gdn2_training_step_full_size():
     """The benchmark's step: gdn_chunk_fwd keeping the backward cache, then gdn_chunk_bwd reading
-    it; 2 heads of each of the 8 sequences (16 pairs) against the oracle's forward and reverse mode.
-    The output is also taken unrounded (fp32) from a forward without cache: the bf16 output of the
-    cached forward must be its rounding."""
+    it with the gradients in bf16; 2 heads of each of the 8 sequences (16 pairs) against the
+    oracle's forward and reverse mode.  The output is also taken unrounded (fp32) from a forward
+    without cache, and the gradients in fp32 from the same cache: the bf16 output and gradients must
+    be their roundings, and the fp32 values meet the parity bound."""
     name = "gdn2_fwd_bwd_bf16"
     wl = WORKLOADS[name]
     x = workload_inputs(name, with_dout=True)
@@ -54,10 +55,16 @@ def test_gdn2_training_step_full_size():
     cache = torch.empty(gdn.gdn_chunk_fwd_cache_size(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], **gate_kw(g)),
                         dtype=torch.uint8, device="cuda")
     o16, ht = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], bwd_cache=cache, **gate_kw(g))
+    g16 = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], fwd_cache=cache,
+                            grads_in_dtype=True, **gate_kw(g))
     grads = gdn.gdn_chunk_bwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], grad_o=g["dout"], fwd_cache=cache,
                               **gate_kw(g))
     torch.cuda.synchronize()
     del cache
+    for key in ("dq", "dk", "dv", "dalpha", "db", "dw"):
+        assert_bf16_is_rounding(g16[key], grads[key], key)
+    assert torch.equal(g16["dh0"], grads["dh0"])
+    del g16
     o, ht32 = gdn.gdn_chunk_fwd(g["q"], g["k"], g["v"], g["alpha"], h0=g["h0"], out_f32=True, **gate_kw(g))
     torch.cuda.synchronize()
     assert_bf16_is_rounding(o16, o, "o")

@@ -263,3 +263,34 @@ def test_gate_logit_arguments_rejected_on_the_host(lib):
         assert lib.gdn_chunk_fwd(ctypes.byref(a), ws, 1 << 30, None) == 1, kw
         assert "gate_logits" in lib.gdn_last_error().decode() or "alpha_scale" in lib.gdn_last_error().decode()
     assert gdn.kernel_launches() == before
+
+
+def _bwd(**kw):
+    base = dict(q=16, k=32, v=48, alpha=64, b=80, w=96, h0=None, head_map=None, grad_o=112, grad_ht=None,
+                grad_q=1 << 20, grad_k=2 << 20, grad_v=3 << 20, grad_alpha=4 << 20, grad_b=5 << 20,
+                grad_w=6 << 20, grad_h0=None, B=1, T=64, Hk=1, Hv=1, dk=64, dv=64, scale=1.0,
+                alpha_per_channel=1, gates_per_channel=1, dtype=0, gate_dtype=0)
+    base.update(kw)
+    return gdn.BwdArgs(**base)
+
+
+def test_gradient_dtype_option_on_the_host(lib):
+    """grads_in_dtype is 0 or 1; bf16 gradients of a bf16 problem the tensor-core backward does not
+    serve (here dk = 64) are refused as unsupported; nothing is launched (fake device addresses)."""
+    before = gdn.kernel_launches()
+    ws = ctypes.c_void_p(1 << 30)
+    a = _bwd(grads_in_dtype=2)
+    assert lib.gdn_chunk_bwd(ctypes.byref(a), ws, 1 << 30, None) == 1
+    assert "grads_in_dtype" in lib.gdn_last_error().decode()
+    a = _bwd(grads_in_dtype=1)
+    assert lib.gdn_chunk_bwd(ctypes.byref(a), ws, 1 << 30, None) == 2
+    assert "grads_in_dtype" in lib.gdn_last_error().decode()
+    # bf16 gradients take half the bytes: outputs that overlap as fp32 are disjoint as bf16 (the
+    # call then stops at the unsupported path, after the buffer checks)
+    close = dict(grad_k=(1 << 20) + 64 * 64 * 2)
+    a = _bwd(**close)
+    assert lib.gdn_chunk_bwd(ctypes.byref(a), ws, 1 << 30, None) == 1
+    assert "overlap" in lib.gdn_last_error().decode()
+    a = _bwd(grads_in_dtype=1, **close)
+    assert lib.gdn_chunk_bwd(ctypes.byref(a), ws, 1 << 30, None) == 2
+    assert gdn.kernel_launches() == before
