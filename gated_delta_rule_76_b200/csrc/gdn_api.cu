@@ -362,13 +362,7 @@ static gdn_status chunk_fwd_core(const gdn_fwd_args* a, void* workspace, size_t 
     if (e == cudaSuccess) e = clear_flags(flags, pb, st);
     if (e == cudaSuccess) {
         TcFwdSave save{};
-        if (a->bwd_cache) {
-            const TcCache cp = plan_tc_cache(pb);
-            char* cb = static_cast<char*>(a->bwd_cache);
-            save.s0 = reinterpret_cast<float*>(cb + cp.s0);
-            save.vp_hi = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_hi);
-            save.vp_lo = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_lo);
-        }
+        if (a->bwd_cache) save = tc_save_in(a->bwd_cache, pb, nullptr);
         if (tc)
             e = tc_chunk_fwd(pb, io_from(a), f, a->gate_dtype == GDN_BF16, ws_status(workspace), st,
                              a->bwd_cache ? &save : nullptr, flags);
@@ -731,10 +725,7 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     if (split) {
         io.q_lo = cp.q_lo; io.k_lo = cp.k_lo; io.v_lo = cp.v_lo;
         if (cache) {
-            const TcCache cc = plan_tc_cache(pb);
-            char* cb = cache + lc.tc;
-            const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
-                                 reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo), reinterpret_cast<float*>(cache + lc.o)};
+            const TcFwdSave save = tc_save_in(cache + lc.tc, pb, reinterpret_cast<float*>(cache + lc.o));
             e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, &save, flags);
         } else {
             e = tc_chunk_fwd(pb, io, f, a->gate_dtype == GDN_BF16, ws_status(workspace), sm, nullptr, flags);
@@ -928,9 +919,7 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
             e = bf16_conv(cp, sm);
             if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (conv)");
             io.o = o; io.o_type = 1;
-            const TcCache cc = plan_tc_cache(pb);
-            const TcFwdSave save{reinterpret_cast<float*>(cb + cc.s0), reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_hi),
-                                 reinterpret_cast<__nv_bfloat16*>(cb + cc.vp_lo), nullptr};
+            const TcFwdSave save = tc_save_in(cb, pb, nullptr);
             e = tc_chunk_fwd(pb, io, f, bf16g, ws_status(workspace), sm, &save, flags);
             if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (forward)");
         }

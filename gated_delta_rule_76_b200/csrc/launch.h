@@ -49,6 +49,7 @@ struct TcFwdSave {
     __nv_bfloat16* vp_hi;    // [B,T,Hv,dv]
     __nv_bfloat16* vp_lo;
     float* o_raw;            // with the swish gate, may be NULL: the output before the gate (fp32)
+    uint8_t* t;              // [B*Hv][NT] 8 KB images of each chunk's bf16 T tile (swizzled), or NULL
 };
 bool tc_fwd_eligible(const Problem& pb, bool bf16_inputs, bool bf16_gates, Flags f);
 // flags: [B*Hv] ints, zero on entry (or NULL): the kernel marks the pairs whose decay leaves the
@@ -84,8 +85,11 @@ cudaError_t compose_states(const float* M, const float* N, const float* S_in, fl
 struct TcCache {
     size_t bytes = 0;
     size_t s0, vp_hi, vp_lo;  // states [B*Hv][NT+1][dv/4][dk][4] fp32; V' hi, lo [B,T,Hv,dv] bf16
+    size_t t;                 // T tiles [B*Hv][NT][8 KB]: bf16, 64 rows of 128 swizzled bytes
 };
 TcCache plan_tc_cache(const Problem& pb);
+// The forward's save targets inside a cache laid out by plan_tc_cache.
+TcFwdSave tc_save_in(void* cache, const Problem& pb, float* o_raw);
 struct TcBwdWs {
     size_t bytes = 0;  // total, including the 256-byte status word at offset 0
     size_t cache;      // a forward cache inside the workspace (~0 when the caller passes one)

@@ -30,8 +30,21 @@ TcCache plan_tc_cache(const Problem& pb) {
     c.s0 = take(st1);  // entering state of every chunk, then the final state
     c.vp_hi = take(tok);
     c.vp_lo = take(tok);
+    c.t = take((size_t)pb.B * pb.Hv * pb.NT * 8192);
     c.bytes = off;
     return c;
+}
+
+TcFwdSave tc_save_in(void* cache, const Problem& pb, float* o_raw) {
+    const TcCache c = plan_tc_cache(pb);
+    char* cb = static_cast<char*>(cache);
+    TcFwdSave s{};
+    s.s0 = reinterpret_cast<float*>(cb + c.s0);
+    s.vp_hi = reinterpret_cast<__nv_bfloat16*>(cb + c.vp_hi);
+    s.vp_lo = reinterpret_cast<__nv_bfloat16*>(cb + c.vp_lo);
+    s.o_raw = o_raw;
+    s.t = reinterpret_cast<uint8_t*>(cb + c.t);
+    return s;
 }
 
 TcBwdWs plan_tc_bwd_ws(const Problem& pb, bool gqa_partials, bool caller_cache) {
@@ -62,11 +75,11 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
                          const TcBwdWs& plan, void* ws, const void* cache, cudaStream_t st) {
     char* base = static_cast<char*>(ws);
     int* err = static_cast<int*>(ws);
-    const TcCache cp = plan_tc_cache(pb);
     char* cb = cache ? static_cast<char*>(const_cast<void*>(cache)) : base + plan.cache;
-    float* s0 = reinterpret_cast<float*>(cb + cp.s0);
-    auto* vph = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_hi);
-    auto* vpl = reinterpret_cast<__nv_bfloat16*>(cb + cp.vp_lo);
+    const TcFwdSave save = tc_save_in(cb, pb, nullptr);
+    float* s0 = save.s0;
+    auto* vph = save.vp_hi;
+    auto* vpl = save.vp_lo;
     float* dsc = reinterpret_cast<float*>(base + plan.dsc);
     auto* nyh = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_hi);
     auto* nyl = reinterpret_cast<__nv_bfloat16*>(base + plan.ny_lo);
@@ -88,7 +101,6 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
         fio.z = nullptr;
         Flags ff = f;
         ff.gate = false;
-        const TcFwdSave save{s0, vph, vpl};
         e = tc_chunk_fwd(pb, fio, ff, bf16_gates, err, st, &save, flags);
         if (e != cudaSuccess) return e;
     }
@@ -119,6 +131,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     sp.ny_lo = nyl;
     sp.err = err;
     sp.flags = flags;
+    sp.t_in = save.t;
 
     tcbwd::grad::Params gp{};
     gp.pb = pb;

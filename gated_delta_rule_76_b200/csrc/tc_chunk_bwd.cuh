@@ -17,12 +17,13 @@
 //
 // Kernels of one backward call:
 //   1. the forward kernel (tc_chunk_fwd.cuh) in saving mode: the state entering every chunk
-//      (fp32) and V' of every token (bf16 hi/lo);
+//      (fp32), V' of every token (bf16 hi/lo) and the bf16 T tile of every chunk;
 //   2. chunk_bwd_scan_kernel (this file): one CTA per (batch, value head), chunks in reverse;
 //      the state gradient dS is carried in registers (thread j: column j), its chain per chunk
 //      is  XA = dO^T P + dS^T Kbar^T (= dV'^T)  ->  XC = dO^T Qhat - dV'^T W (= dS0^T without
 //      the decay term)  ->  dS = Diag(gamma) dS + XC^T;  off the chain it forms -dY^T = -dV'^T T.
-//      The prologue warps build the chunk's factors, X1, P and T; the chain warps form W^T from
+//      The prologue warps build the chunk's factors, X1 and P; T is the forward's own bf16 tile,
+//      copied in from the cache (the forward solved for it already); the chain warps form W^T from
 //      T and the split Ehat tiles and request the next chunk's raw tiles.  It saves dS_end of
 //      every chunk (fp32) and -dY of every token (bf16 hi/lo), and writes dh0;
 //   3. chunk_bwd_grad_kernel (this file): persistent, one CTA per SM walking the chunks; every
@@ -65,10 +66,8 @@ __device__ unsigned long long g_scan_trace[64][32];
 using namespace gdn::tc;
 using tcfwd::bf;
 using tcfwd::Ctx;
-using tcfwd::fma4;
 using tcfwd::ld16;
 using tcfwd::ldf4;
-using tcfwd::solve_block_row;
 using tcfwd::split8;
 using tcfwd::split_pack;
 using tcfwd::st16;
@@ -78,7 +77,6 @@ using tcfwd::wait1;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int LDA = tcfwd::LDA;
 constexpr uint64_t kWaitNs = tcfwd::kWaitNs;
 
 // =========================================== scan ===========================================
@@ -107,10 +105,10 @@ constexpr uint32_t SM_P = 131072;     // 16 KB: P hi [1][64], P lo [1][64] (row 
 constexpr uint32_t SM_T = 147456;     // 8 KB [1][64]: T (row r, columns s)
 constexpr uint32_t SM_WT = 155648;    // 32 KB: W^T hi [1][128], W^T lo [1][128] (row c, columns r)
 constexpr uint32_t SM_DO = 188416;    // 16 KB: dO, two boxes of 64 channels x 64 tokens
-constexpr uint32_t SM_ASCR = 204800;  // 17 KB: A, then T, fp32 [64][LDA]
+                                      // [204800, 222208): unused (T arrives from the forward's cache)
 constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats
 constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, flags
-constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: row-group products, then solve block rows
+constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: row-group products
 constexpr uint32_t SM_END = SM_RS + 4096;
 constexpr size_t kSmemBytes = SM_END + 1024;
 
@@ -120,7 +118,7 @@ enum Bar {
     B_X1,        // X1 complete
     B_WT,        // W^T complete
     B_PREADY,    // prologue -> scan: P, Kbar, [Ehat;Qhat] written
-    B_TREADY,    // prologue -> scan: T written
+    B_TREADY,    // T of the chain's chunk landed (bulk copy from the forward's cache)
     B_XA,        // XA complete
     B_XCPRE,     // dO^T Qhat complete: [Ehat;Qhat] and dO may be overwritten
     B_XC,        // XC complete
@@ -137,6 +135,7 @@ struct Params {
     float* dsc;            // [B*Hv][NT][dv/4][dk][4]: dS_end of every chunk
     __nv_bfloat16* ny_hi;  // [B,T,Hv,dv]: -dY of every token, hi / lo
     __nv_bfloat16* ny_lo;
+    const uint8_t* t_in;   // [B*Hv][NT][8 KB]: the forward's bf16 T tile of every chunk (swizzled image)
     int* err;
     uint64_t wait_ns;      // limit of every bounded wait; 0 = kWaitNs
     int* flags;            // [B*Hv] or NULL: set for a pair with a chunk outside the decay range
@@ -217,12 +216,20 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     // Chunks are processed in reverse: iteration i works on chunk NT - 1 - i.
-    int raw_issued = 0, do_issued = 0;  // meaningful in thread 0, which issues every load
+    int raw_issued = 0, do_issued = 0, t_issued = 0;  // meaningful in thread 0, which issues every load
+    // T of chunk n: the forward's tile, copied in once the scan's last reader of the previous T (its
+    // -dY product) has completed
+    auto load_t = [&](int n) {
+        mbar_arrive_expect_tx(cx.bars + B_TREADY, 8192u);
+        bulk_g2s(sbase + SM_T, p.t_in + ((long)blockIdx.x * NT + n) * 8192, 8192u, cx.bars + B_TREADY);
+        ++t_issued;
+    };
     if (tid == 0) {
         scan_load_raw<APC, GPC, SPLIT>(cx, NT - 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
         raw_issued = 1;
         scan_load_do(cx, NT - 1, b, hv, &tm_do);
         do_issued = 1;
+        load_t(NT - 1);
     }
 
     if (warp < 8) {
@@ -407,7 +414,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (tid == 0) {
                 GDN_STRACE(i, 6);
                 tc_fence_after();
-                wait1(cx, B_DY, pi);
+                if (wait1(cx, B_DY, pi) && i + 1 < NT && !*cx.abort_flag) load_t(n - 1);
                 GDN_STRACE(i, 7);
             }
             tc_fence_before();
@@ -449,7 +456,6 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
         const TG* alpha_g = static_cast<const TG*>(p.alpha);
         const TG* beta_g = static_cast<const TG*>(p.b);
-        float* ascr = reinterpret_cast<float*>(sm + SM_ASCR);
         float* rs = reinterpret_cast<float*>(sm + SM_RS);
         uint8_t* RQB = sm + SM_RQB;
         uint8_t* RK = sm + SM_RK;
@@ -613,25 +619,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             named_bar(2, 128);
             tc_fence_after();
-            if (c < 64) {
-                // A row c (lanes 0-63), strictly lower, into the fp32 scratch.
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tl + TM_X1 + 32 * half, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const int s0 = 32 * half + 4 * q4;
-                        float4 v4;
-                        v4.x = s0 + 0 < c ? __uint_as_float(r[4 * q4 + 0]) : 0.f;
-                        v4.y = s0 + 1 < c ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
-                        v4.z = s0 + 2 < c ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
-                        v4.w = s0 + 3 < c ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
-                        *reinterpret_cast<float4*>(ascr + c * LDA + s0) = v4;
-                    }
-                }
-            } else {
+            if (c >= 64) {
                 // P row s = c - 64 (lanes 64-127), lower with the diagonal, split: row s, columns r.
                 const int rr = c - 64;
                 uint8_t* Ph = sm + SM_P;
@@ -663,61 +651,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 GDN_STRACE(i, 19);
                 mbar_arrive(cx.bars + B_PREADY);
             }
-            // ---- T = (I + A)^-1 by 16 x 16 blocks, in place in the fp32 scratch ------------------
-            if (c < 64) {
-                const int base = 16 * (c >> 4), jc = c & 15;
-                float x[16];
-#pragma unroll
-                for (int s2 = 0; s2 < 16; ++s2) {
-                    const float* arow = ascr + (base + s2) * LDA + base;
-                    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                    for (int u4 = 0; u4 < (s2 + 3) / 4; ++u4) {
-                        const float4 a4 = ldf4(arow + 4 * u4);
-                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int u = 4 * u4 + e;
-                            if (u < s2) {
-                                if (u & 1) a1 = fmaf(av[e], x[u], a1);
-                                else a0 = fmaf(av[e], x[u], a0);
-                            }
-                        }
-                    }
-                    x[s2] = s2 == jc ? 1.f : (s2 > jc ? -(a0 + a1) : 0.f);
-                }
-                named_bar(3, 64);
-#pragma unroll
-                for (int s2 = 0; s2 < 16; ++s2) ascr[(base + s2) * LDA + base + jc] = x[s2];
-            }
-            named_bar(2, 128);
-            solve_block_row<1>(ascr, rs, c);
-            solve_block_row<2>(ascr, rs, c);
-            solve_block_row<3>(ascr, rs, c);
-            // ---- T (fp32) -> bf16 tile once the scan has finished with the previous T and W^T ------
-            if (c == 0) GDN_STRACE(i, 20);
-            if (c == 0 && i > 0) wait1(cx, B_DY, pi ^ 1u);
-            named_bar(2, 128);
-            {
-                const int row = c & 63, col0 = 32 * (c >> 6);
-                uint8_t* Tt = sm + SM_T;
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    const float4 f0 = ldf4(ascr + row * LDA + col0 + 8 * q8);
-                    const float4 f1 = ldf4(ascr + row * LDA + col0 + 8 * q8 + 4);
-                    st16(Tt + sw128_offset(row, col0 + 8 * q8, 64),
-                         make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
-                                    pack_bf16x2(f1.z, f1.w)));
-                }
-            }
-            fence_async_shared();
-            named_bar(2, 128);
-            if (c == 0) {
-                // T is in shared memory: the scan forms W^T and splits it.
-                mbar_arrive(cx.bars + B_TREADY);
-                GDN_STRACE(i, 22);
-                *stop_slot = *cx.abort_flag;
-            }
+            if (c == 0) *stop_slot = *cx.abort_flag;
             named_bar(2, 128);
             if (*stop_slot) break;
         }
@@ -733,6 +667,10 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         if (tid == 0 && raw_issued > 0)
             while (!mbar_try_wait(cx.bars + B_RAW, (uint32_t)((raw_issued - 1) & 1)) &&
+                   globaltimer_ns() - t0 < cx.wait_ns) {
+            }
+        if (tid == 0 && t_issued > 0)
+            while (!mbar_try_wait(cx.bars + B_TREADY, (uint32_t)((t_issued - 1) & 1)) &&
                    globaltimer_ns() - t0 < cx.wait_ns) {
             }
     }

@@ -136,6 +136,8 @@ struct Params {
     __nv_bfloat16* vp_hi;        // [B,T,Hv,dv]: V' = T (Z - Ehat S0) of every token, split
     __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
     float* o_raw;                // GATE only, may be NULL: the output before the gate, fp32 [B,T,Hv,dv]
+    uint8_t* t_out;              // [B*Hv][NT][8 KB] or NULL: the image of every chunk's bf16 T hi tile
+                                 //   (64 rows of 128 swizzled bytes), read back by the reverse scan
     int* flags;                  // [B*Hv] or NULL: set for a pair with a chunk outside the decay range
     // GATE only, may be NULL: the output norm before the gate (every (token, head) row of dv values
     // divided by its root mean square, times norm_w[dv]); norm_w is bf16 unless norm_w_f32
@@ -985,6 +987,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int row = c & 63, col0 = 32 * (c >> 6);
                 uint8_t* Tt = sm + SM_T;
                 uint8_t* Tl = sm + SM_TLO;
+                uint8_t* Tg = p.t_out ? p.t_out + ((long)blockIdx.x * NT + m) * 8192 : nullptr;
                 float tv[32];
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) {
@@ -1002,6 +1005,7 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const uint32_t off = sw128_offset(row, col0 + 8 * q8, 64);
                     st16(Tt + off, hi);
                     st16(Tl + off, lo);
+                    if (Tg) *reinterpret_cast<uint4*>(Tg + off) = hi;
                 }
             }
             fence_async_shared();

@@ -55,6 +55,7 @@ cudaError_t tc_chunk_fwd_kernel(const Problem& pb, const ChunkIO& io, Flags f, b
         p.s0_out = save->s0;
         p.vp_hi = save->vp_hi;
         p.vp_lo = save->vp_lo;
+        p.t_out = save->t;
         p.o_raw = save->o_raw;
     }
     return pb.gate_logits ? tc_fwd_dispatch<true>(maps, p, f, split, bf16_gates, st)
