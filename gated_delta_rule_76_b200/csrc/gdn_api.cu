@@ -754,14 +754,12 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
 // backward's own workspace
 // first (its status word is the call's, at offset 0), then the conv results as bf16 hi/lo pairs,
 // the recurrence's output o, the gradient of o (bf16 hi/lo), the q, k, v gradients from the
-// recurrence, the conv-weight partials, the forward cache (states, V'), and the second set of
-// recurrence gradients (those of the lo half of the gradient of o).
+// recurrence, the conv-weight partials and the forward cache (states, V', T tiles).
 // CUDA-core form (everything else): the status word, the fp32 conv results, o, the gradient of o
 // (fp32), the q, k, v gradients, the conv-weight partials, then the CUDA-core chunk workspace.
 struct LayerBwdPlan {
     bool tc;
     size_t q, k, v, o, dout, npart, gq, gk, gv, wpart, cache, chunk, bytes;
-    size_t gq2, gk2, gv2, ga2, gb2, gh2;  // tensor-core form: gradients from the lo half of do
 };
 static bool layer_bwd_tc_form(const gdn_layer_bwd_args* a) {
     return layer_tc_form(a->dtype, a->dk, a->dv, a->alpha_per_channel, a->gates_per_channel, a->h0);
@@ -788,10 +786,6 @@ static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& p
     w.wpart = take(layer_bwd_wpart_floats((int)a->B, (int)a->T, (int)a->Hk, (int)a->Hv, (int)a->dk) * 4);
     if (w.tc) {
         w.cache = cached ? ~size_t(0) : take(plan_tc_cache(pb).bytes);
-        const size_t ng = BT * a->Hv;  // scalar gates
-        w.gq2 = take(qn * 4); w.gk2 = take(qn * 4); w.gv2 = take(vn * 4);
-        w.ga2 = take(ng * 4); w.gb2 = take(ng * 4);
-        w.gh2 = take((size_t)a->B * a->Hv * a->dk * a->dv * 4);
     } else {
         w.cache = ~size_t(0);
         w.chunk = off;
@@ -928,30 +922,16 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
         lio.dout16_lo = lio.dout16 + vn;
         e = layer_gate_bwd(lio, bf16, sm);
         if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (gate)");
-        // 4. the tensor-core backward from the cache, once per half of do.  The backward is linear
-        //    in its cotangents (do, dht), so the gradients of (hi, dht) and of (lo, 0) add up to
-        //    those of (do, dht); a single bf16 do would move dq by ~5% of its RMS on this layer.
+        // 4. the tensor-core backward from the cache, with do as its bf16 hi/lo pair: the scan and
+        //    the gradient kernel take the lo tiles as a third operand of their dO products (a
+        //    single bf16 do would move dq by ~5% of its RMS on this layer).
         const TcBwdWs tplan = plan_tc_bwd_ws(pb, !direct, true);
         io.o = nullptr;
-        io.dout = lio.dout16; io.dht = a->grad_ht;
+        io.dout = lio.dout16; io.dout_lo = lio.dout16_lo; io.dht = a->grad_ht;
         io.dq = at(plan.gq); io.dk = at(plan.gk); io.dv = at(plan.gv);
         io.dalpha = a->grad_alpha; io.db = a->grad_b; io.dw = nullptr; io.dh0 = a->grad_h0;
         e = tc_chunk_bwd(pb, io, f, bf16g, direct, tplan, workspace, cb, sm);
         if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence)");
-        io.dout = lio.dout16_lo; io.dht = nullptr;
-        io.dq = at(plan.gq2); io.dk = at(plan.gk2); io.dv = at(plan.gv2);
-        io.dalpha = at(plan.ga2); io.db = at(plan.gb2); io.dh0 = a->grad_h0 ? at(plan.gh2) : nullptr;
-        e = tc_chunk_bwd(pb, io, f, bf16g, direct, tplan, workspace, cb, sm);
-        if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (recurrence, lo half)");
-        const long ng = (long)BT * a->Hv;
-        const struct { float* dst; const float* src; long n; } acc[] = {
-            {at(plan.gq), at(plan.gq2), (long)qn}, {at(plan.gk), at(plan.gk2), (long)qn},
-            {at(plan.gv), at(plan.gv2), (long)vn}, {a->grad_alpha, at(plan.ga2), ng}, {a->grad_b, at(plan.gb2), ng},
-            {a->grad_h0, at(plan.gh2), a->grad_h0 ? (long)(st / 4) : 0}};
-        for (const auto& x : acc) {
-            e = layer_accumulate(x.dst, x.src, x.n, sm);
-            if (e != cudaSuccess) return cuda_fail(e, "gdn_layer_core_bwd (accumulate)");
-        }
     } else {
         // 1. conv + SiLU + L2, fp32 results
         cp.q = at(plan.q); cp.k = at(plan.k); cp.v = at(plan.v);

@@ -125,8 +125,6 @@ cudaError_t layer_norm_gate_fwd(const float* o, const void* z, const void* norm_
                                 void* y, int y_f32, bool bf16, long rows, int d, cudaStream_t st);
 cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
 cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st);
-// dst[i] += src[i], i < n (the two halves of a gradient computed from hi and lo cotangents).
-cudaError_t layer_accumulate(float* dst, const float* src, long n, cudaStream_t st);
 
 GDN_DECLARE_LAUNCHERS(bf16)       // bf16 tensors, bf16 gates
 GDN_DECLARE_LAUNCHERS(bf16_f32g)  // bf16 tensors, fp32 gates

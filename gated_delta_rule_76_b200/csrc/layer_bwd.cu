@@ -270,20 +270,6 @@ __global__ void __launch_bounds__(128) conv_silu_l2_bwd_kernel(const TIn* __rest
     }
 }
 
-__global__ void __launch_bounds__(256) accumulate_kernel(float4* __restrict__ dst, const float4* __restrict__ src,
-                                                         float* __restrict__ dst1, const float* __restrict__ src1,
-                                                         long n4, long n) {
-    for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
-        float4 a = dst[i];
-        const float4 b = src[i];
-        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-        dst[i] = a;
-    }
-    // what the float4 body leaves (n % 4 elements, or all of them when the pointers are unaligned)
-    for (long t = 4 * n4 + (long)blockIdx.x * blockDim.x + threadIdx.x; t < n; t += (long)gridDim.x * blockDim.x)
-        dst1[t] += src1[t];
-}
-
 // dconv_w[j] = sum over partials p of wpart[p][j]  (j = channel * 4 + tap), one thread per j.
 __global__ void __launch_bounds__(256) dconv_reduce_kernel(const float* __restrict__ wpart, float* __restrict__ dw,
                                                            long nj, int np) {
@@ -380,17 +366,6 @@ cudaError_t layer_gate_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st) {
 
 cudaError_t layer_conv_bwd(const LayerBwdIO& io, bool bf16, cudaStream_t st) {
     return bf16 ? conv_bwd_t<__nv_bfloat16>(io, st) : conv_bwd_t<float>(io, st);
-}
-
-cudaError_t layer_accumulate(float* dst, const float* src, long n, cudaStream_t st) {
-    if (n <= 0) return cudaSuccess;
-    // float4 body only when both pointers are 16-byte aligned
-    const bool v4 = ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15u) == 0;
-    const long n4 = v4 ? n / 4 : 0;
-    const long work = n4 > n - 4 * n4 ? n4 : n - 4 * n4;
-    const long blocks = (work + 255) / 256 < 148L * 16 ? (work + 255) / 256 : 148L * 16;
-    return launch_kernel(accumulate_kernel, dim3((unsigned)(blocks > 0 ? blocks : 1)), dim3(256), 0, st,
-                         reinterpret_cast<float4*>(dst), reinterpret_cast<const float4*>(src), dst, src, n4, n);
 }
 
 }  // namespace gdn

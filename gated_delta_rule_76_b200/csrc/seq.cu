@@ -87,6 +87,7 @@ cudaError_t seq_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool tin_f32,
                     void* dq, void* dk, bool direct, float* ck, long ck_stride, float* sbuf, cudaStream_t st) {
     seq::Params p = common_params(pb, io, f, flags);
     p.dout = io.dout;
+    p.dout_lo = io.dout_lo;
     p.dht = io.dht;
     p.dq = dq;
     p.dk = dk;

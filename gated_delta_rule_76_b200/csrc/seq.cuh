@@ -57,6 +57,7 @@ struct Params {
     float* ht;                               // [B,Hv,dk,dv] or NULL
     // backward
     const void* dout;                        // [B,T,Hv,dv] TIn
+    const void* dout_lo;                     // bf16 lo half of dout (dout = dout + dout_lo), or NULL
     const float* dht;                        // [B,Hv,dk,dv] or NULL
     void *dq, *dk;                           // [B,T,Hk,dk] when direct, else [B,T,Hv,dk] per value head
     int direct;
@@ -122,7 +123,12 @@ struct Stager {
             case V_Q: x = ld4(static_cast<const TIn*>(p.q) + qk); lo = static_cast<const __nv_bfloat16*>(p.q_lo); lo_off = qk; break;
             case V_V: x = ld4(static_cast<const TIn*>(p.v) + vv); lo = static_cast<const __nv_bfloat16*>(p.v_lo); lo_off = vv; break;
             default:
-                if (bwd) return ld4(static_cast<const TIn*>(p.dout) + vv);
+                if (bwd) {
+                    x = ld4(static_cast<const TIn*>(p.dout) + vv);
+                    lo = static_cast<const __nv_bfloat16*>(p.dout_lo);
+                    lo_off = vv;
+                    break;
+                }
                 if (p.z_bf16) return ld4(static_cast<const __nv_bfloat16*>(p.z) + vv);
                 return ld4(static_cast<const TIn*>(p.z) + vv);
         }

@@ -65,6 +65,7 @@ struct ChunkIO {
     float norm_eps;
     float* ht;
     const void* dout;
+    const void* dout_lo;  // tensor-core backward only: dout as a bf16 hi/lo pair (dout = dout + dout_lo), or NULL
     const float* dht;
     void *dq, *dk, *dv, *dalpha, *db, *dw;
     int grad_type;  // 0: the gradients above in fp32; 1: in bf16 (tensor-core backward only)

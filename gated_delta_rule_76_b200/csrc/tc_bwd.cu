@@ -106,7 +106,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     }
 
     // 2. maps: q, k, alpha, b, dO, -dY hi/lo, V' hi/lo (unused gate maps copy a valid one)
-    CUtensorMap m[9];
+    CUtensorMap m[10];
     bool ok = make_map(&m[0], io.q, pb.B, pb.T, pb.Hk) && make_map(&m[1], io.k, pb.B, pb.T, pb.Hk) &&
               make_map(&m[4], io.dout, pb.B, pb.T, pb.Hv) && make_map(&m[5], nyh, pb.B, pb.T, pb.Hv) &&
               make_map(&m[6], nyl, pb.B, pb.T, pb.Hv) && make_map(&m[7], vph, pb.B, pb.T, pb.Hv) &&
@@ -118,7 +118,10 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     // split inputs: the lo halves of k and q take the alpha and b slots
     if (ok && split) ok = make_map(&m[2], io.k_lo, pb.B, pb.T, pb.Hk) && make_map(&m[3], io.q_lo, pb.B, pb.T, pb.Hk);
     if (!ok) return cudaErrorInvalidValue;
-    const CUtensorMap ms[5] = {m[0], m[1], m[2], m[3], m[4]};
+    // dO lo (the layer core's gradient of o as a bf16 hi/lo pair), else a copy of the dO map
+    m[9] = m[4];
+    if (io.dout_lo && !make_map(&m[9], io.dout_lo, pb.B, pb.T, pb.Hv)) return cudaErrorInvalidValue;
+    const CUtensorMap ms[6] = {m[0], m[1], m[2], m[3], m[4], m[9]};
 
     tcbwd::scan::Params sp{};
     sp.pb = pb;
@@ -132,6 +135,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     sp.err = err;
     sp.flags = flags;
     sp.t_in = save.t;
+    sp.do_lo = io.dout_lo ? 1 : 0;
 
     tcbwd::grad::Params gp{};
     gp.pb = pb;
@@ -153,6 +157,7 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     gp.db = io.db;
     gp.dw = io.dw;
     gp.direct = direct ? 1 : 0;
+    gp.do_lo = io.dout_lo ? 1 : 0;
     gp.err = err;
 
     if (split && gbf) return cudaErrorInvalidValue;  // the layer core's form returns fp32 gradients

@@ -30,7 +30,7 @@ cudaError_t launch_scan(const CUtensorMap* m, const tcbwd::scan::Params& p, cuda
                                          (int)tcbwd::scan::kSmemBytes);
     if (e != cudaSuccess) return e;
     kernel<<<p.pb.B * p.pb.Hv, tcbwd::scan::kThreads, tcbwd::scan::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
-                                                                                    p);
+                                                                                    m[5], p);
     count_launch();
     return cudaGetLastError();
 }
@@ -46,7 +46,7 @@ cudaError_t launch_grad(const CUtensorMap* m, const tcbwd::grad::Params& p, cuda
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const long grid = nch < nsm ? nch : nsm;  // persistent: one CTA per SM walks the chunks
     kernel<<<(unsigned)grid, tcbwd::grad::kThreads, tcbwd::grad::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], m[4],
-                                                                                 m[5], m[6], m[7], m[8], p);
+                                                                                 m[5], m[6], m[7], m[8], m[9], p);
     count_launch();
     return cudaGetLastError();
 }

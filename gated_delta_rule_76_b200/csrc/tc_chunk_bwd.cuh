@@ -105,7 +105,8 @@ constexpr uint32_t SM_P = 131072;     // 16 KB: P hi [1][64], P lo [1][64] (row 
 constexpr uint32_t SM_T = 147456;     // 8 KB [1][64]: T (row r, columns s)
 constexpr uint32_t SM_WT = 155648;    // 32 KB: W^T hi [1][128], W^T lo [1][128] (row c, columns r)
 constexpr uint32_t SM_DO = 188416;    // 16 KB: dO, two boxes of 64 channels x 64 tokens
-                                      // [204800, 222208): unused (T arrives from the forward's cache)
+constexpr uint32_t SM_DOL = 204800;   // 16 KB: dO lo (when dO is a hi/lo pair), as SM_DO
+                                      // [221184, 222208): unused
 constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats
 constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, flags
 constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: row-group products
@@ -136,6 +137,7 @@ struct Params {
     __nv_bfloat16* ny_hi;  // [B,T,Hv,dv]: -dY of every token, hi / lo
     __nv_bfloat16* ny_lo;
     const uint8_t* t_in;   // [B*Hv][NT][8 KB]: the forward's bf16 T tile of every chunk (swizzled image)
+    int do_lo;             // dO given as bf16 hi + lo (the lo tiles through the sixth tensor map)
     int* err;
     uint64_t wait_ns;      // limit of every bounded wait; 0 = kWaitNs
     int* flags;            // [B*Hv] or NULL: set for a pair with a chunk outside the decay range
@@ -171,19 +173,25 @@ __device__ __forceinline__ void scan_load_raw(const Ctx& cx, int n, int b, int h
     }
 }
 
-__device__ __forceinline__ void scan_load_do(const Ctx& cx, int n, int b, int hv, const CUtensorMap* tdo) {
-    const uint32_t dst = smem_u32(cx.sm) + SM_DO;
+__device__ __forceinline__ void scan_load_do(const Ctx& cx, int n, int b, int hv, const CUtensorMap* tdo,
+                                             const CUtensorMap* tdol, bool lo) {
+    const uint32_t dst = smem_u32(cx.sm) + SM_DO, dsl = smem_u32(cx.sm) + SM_DOL;
     uint64_t* bar = cx.bars + B_DO;
-    mbar_arrive_expect_tx(bar, 16384u);
+    mbar_arrive_expect_tx(bar, lo ? 32768u : 16384u);
     tma4(dst, tdo, bar, 0, hv, n * C, b);
     tma4(dst + 8192, tdo, bar, 64, hv, n * C, b);
+    if (lo) {
+        tma4(dsl, tdol, bar, 0, hv, n * C, b);
+        tma4(dsl + 8192, tdol, bar, 64, hv, n * C, b);
+    }
 }
 
 template <bool APC, bool GPC, class TG, bool SPLIT, bool LG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                      const __grid_constant__ CUtensorMap tm_do, Params p) {
+                      const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dol,
+                      Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
@@ -194,6 +202,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     cx.err = p.err;
     cx.wait_ns = p.wait_ns ? p.wait_ns : kWaitNs;
     float* gam = reinterpret_cast<float*>(sm + SM_GAM);
+    const bool dol = p.do_lo != 0;
 
     const Problem& pb = p.pb;
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -227,7 +236,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (tid == 0) {
         scan_load_raw<APC, GPC, SPLIT>(cx, NT - 1, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
         raw_issued = 1;
-        scan_load_do(cx, NT - 1, b, hv, &tm_do);
+        scan_load_do(cx, NT - 1, b, hv, &tm_do, &tm_dol, dol);
         do_issued = 1;
         load_t(NT - 1);
     }
@@ -277,6 +286,9 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         mma_ss(tbase + TM_XA, da, sdesc_mn_sw128(sbase + SM_P + (uint32_t)k * 128u, 8192u), id_dop, 1u);
                         mma_ss(tbase + TM_XA, da, sdesc_mn_sw128(sbase + SM_P + 8192u + (uint32_t)k * 128u, 8192u),
                                id_dop, 1u);
+                        if (dol)
+                            mma_ss(tbase + TM_XA, sdesc_mn_sw128(sbase + SM_DOL + (uint32_t)k * 128u, 8192u),
+                                   sdesc_mn_sw128(sbase + SM_P + (uint32_t)k * 128u, 8192u), id_dop, 1u);
                     }
                     mma_commit(cx.bars + B_XA);
 #pragma unroll
@@ -286,6 +298,9 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                id_doq, k > 0 ? 1u : 0u);
                         mma_ss(tbase + TM_XC, da, sdesc_mn_sw128(sbase + SM_RQB + 8192u + (uint32_t)k * 128u, 16384u),
                                id_doq, 1u);
+                        if (dol)
+                            mma_ss(tbase + TM_XC, sdesc_mn_sw128(sbase + SM_DOL + (uint32_t)k * 128u, 8192u),
+                                   sdesc_mn_sw128(sbase + SM_EQ + 8192u + (uint32_t)k * 128u, 16384u), id_doq, 1u);
                     }
                     mma_commit(cx.bars + B_XCPRE);
                     wait1(cx, B_XA, pi);
@@ -371,7 +386,7 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     mma_commit(cx.bars + B_DY);
                 }
                 if (do_issued < NT && wait1(cx, B_XCPRE, pi) && !*cx.abort_flag) {
-                    scan_load_do(cx, NT - 1 - do_issued, b, hv, &tm_do);
+                    scan_load_do(cx, NT - 1 - do_issued, b, hv, &tm_do, &tm_dol, dol);
                     ++do_issued;
                 }
                 wait1(cx, B_XC, pi);
@@ -749,6 +764,7 @@ struct Params {
     void* db;
     void* dw;
     int direct;          // dq, dk written per key head (no head sharing)
+    int do_lo;           // dO given as bf16 hi + lo: the lo tiles fill rows 0-63 of the G lo tile
     int* err;
     uint64_t wait_ns;    // limit of every bounded wait; 0 = kWaitNs
 };
@@ -772,7 +788,7 @@ __device__ __forceinline__ ChunkPos chunk_pos(const Problem& pb, long ci) {
 }
 
 struct Maps {
-    const CUtensorMap *q, *k, *a, *b, *dO, *yh, *yl, *vh, *vl;
+    const CUtensorMap *q, *k, *a, *b, *dO, *yh, *yl, *vh, *vl, *dOl;
 };
 
 // SPLIT: as in the scan, m.a maps k lo and m.b maps q lo.
@@ -801,10 +817,14 @@ __device__ __forceinline__ void load_raw_g(const Ctx& cx, const ChunkPos& cp, co
     }
 }
 
-__device__ __forceinline__ void load_gv(const Ctx& cx, const ChunkPos& cp, const Maps& m) {
+__device__ __forceinline__ void load_gv(const Ctx& cx, const ChunkPos& cp, const Maps& m, bool dol) {
     const uint32_t base = smem_u32(cx.sm);
     uint64_t* bar = cx.bars + B_GV;
-    mbar_arrive_expect_tx(bar, 5u * 16384u);
+    mbar_arrive_expect_tx(bar, (dol ? 6u : 5u) * 16384u);
+    if (dol) {  // rows 0-63 of the G lo tile: dO lo (else they hold zeros)
+        tma4(base + SM_GL, m.dOl, bar, 0, cp.hv, cp.t0, cp.b);
+        tma4(base + SM_GL + 16384, m.dOl, bar, 64, cp.hv, cp.t0, cp.b);
+    }
     tma4(base + SM_GH, m.dO, bar, 0, cp.hv, cp.t0, cp.b);
     tma4(base + SM_GH + 16384, m.dO, bar, 64, cp.hv, cp.t0, cp.b);
     tma4(base + SM_GH + 8192, m.yh, bar, 0, cp.hv, cp.t0, cp.b);
@@ -1236,8 +1256,10 @@ __device__ __forceinline__ void scalar_gate_finish(const Params& p, const ChunkP
         }
     }
     named_bar(2, 128);
-    uint4* z = reinterpret_cast<uint4*>(scr);
-    for (int i = c; i < (int)(SX_BYTES / 16); i += 128) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (!p.do_lo) {  // with dO lo the next chunk's tiles overwrite the scratch instead
+        uint4* z = reinterpret_cast<uint4*>(scr);
+        for (int i = c; i < (int)(SX_BYTES / 16); i += 128) z[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     fence_async_shared();
 }
 
@@ -1255,7 +1277,8 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                       const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_yh,
                       const __grid_constant__ CUtensorMap tm_yl, const __grid_constant__ CUtensorMap tm_vh,
-                      const __grid_constant__ CUtensorMap tm_vl, Params p) {
+                      const __grid_constant__ CUtensorMap tm_vl, const __grid_constant__ CUtensorMap tm_dol,
+                      Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
@@ -1274,7 +1297,8 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int tid = threadIdx.x, warp = tid >> 5;
     const long nch = (long)pb.B * pb.Hv * pb.NT;
     const uint32_t sbase = smem_u32(sm);
-    const Maps m{&tm_q, &tm_k, &tm_a, &tm_b, &tm_do, &tm_yh, &tm_yl, &tm_vh, &tm_vl};
+    const Maps m{&tm_q, &tm_k, &tm_a, &tm_b, &tm_do, &tm_yh, &tm_yl, &tm_vh, &tm_vl, &tm_dol};
+    const bool dol = p.do_lo != 0;
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) mbar_init(cx.bars + i, 1);
@@ -1300,13 +1324,13 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             raw_issued = 1;
         }
         if (tid == 128) {
-            load_gv(cx, c0, m);
+            load_gv(cx, c0, m, dol);
             gv_issued = 1;
         }
         if (warp < 4) {
-            uint8_t* gl = sm + SM_GL;  // rows 0-63 of the G lo tile: zeros (dO is exact in bf16)
+            uint8_t* gl = sm + SM_GL;  // rows 0-63 of the G lo tile: zeros when dO is exact in bf16
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 8 && !dol; ++u) {
                 const int idx = tid + 128 * u;
                 st16(gl + (uint32_t)(idx >> 9) * 16384u + (uint32_t)(idx & 511) * 16u, make_uint4(0u, 0u, 0u, 0u));
             }
@@ -1427,14 +1451,20 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             grad_dv_dw<GPC, TG, SPLIT, LG, GT>(p, cx, cp, tid - 128, scr);
             named_bar(2, 128);
             if (tid == 128) GDN_BTRACE(it, 4);
-            // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land
-            if (tid == 128 && nx < nch && !*cx.abort_flag) {
-                load_gv(cx, chunk_pos(pb, nx), m);
+            // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land; dO lo
+            // shares its rows with the scalar gates' scratch, so then only once that has been read
+            const bool late_gv = dol && (!APC || !GPC);
+            if (!late_gv && tid == 128 && nx < nch && !*cx.abort_flag) {
+                load_gv(cx, chunk_pos(pb, nx), m, dol);
                 ++gv_issued;
             }
             if (!APC || !GPC) {
                 bar_sync_all(3);
                 if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG, LG, GT>(p, cp, tid - 128, scr);
+                if (late_gv && tid == 128 && nx < nch && !*cx.abort_flag) {
+                    load_gv(cx, chunk_pos(pb, nx), m, dol);
+                    ++gv_issued;
+                }
             }
         }
         if (tid == 0) *stop_slot = *cx.abort_flag;
