@@ -41,17 +41,38 @@ decode_step_kernel(DecodeParams p) {
     const int hv = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
     // a map entry outside [0, Hk) breaks the precondition: clamped, so no read leaves q or k
     const int hk = p.head_map ? min(max(__ldg(p.head_map + hv), 0), p.Hk - 1) : hv / (p.Hv / p.Hk);
-    auto alpha_of = [&](float x) {
-        if (!p.gate_logits) return x;
-        return expf(-__ldg(p.alpha_scale + hv) * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)))));
-    };
-    auto sig_of = [&](float x) { return p.gate_logits ? 1.f / (1.f + expf(-x)) : x; };
     const TIn* q = static_cast<const TIn*>(p.q) + ((long)n * p.Hk + hk) * DK;
     const TIn* k = static_cast<const TIn*>(p.k) + ((long)n * p.Hk + hk) * DK;
     const TIn* v = static_cast<const TIn*>(p.v) + ((long)n * p.Hv + hv) * DV;
     const TG* al = static_cast<const TG*>(p.alpha) + ((long)n * p.Hv + hv) * (APC ? DK : 1);
     const TG* bg = static_cast<const TG*>(p.b) + ((long)n * p.Hv + hv) * (GPC ? DK : 1);
     const TG* wg = GPC ? static_cast<const TG*>(p.w) + ((long)n * p.Hv + hv) * DV : bg;
+
+    // ---- gates: every load issued first, then (gates as logits) the transforms under one branch,
+    // so that no load waits for another (a branch on a loaded value waits for the load) -----
+    constexpr int NI = (DK + NTH - 1) / NTH, NJ = (DV + NTH - 1) / NTH;
+    float ga[NI], gb[NI], gw[NJ];
+#pragma unroll
+    for (int u = 0; u < NI; ++u) {
+        const int i = tid + u * NTH;
+        ga[u] = i < DK ? to_f32(al[APC ? i : 0]) : 0.f;
+        gb[u] = i < DK ? to_f32(bg[GPC ? i : 0]) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < NJ; ++u) {
+        const int j = tid + u * NTH;
+        gw[u] = j < DV ? to_f32(wg[GPC ? j : 0]) : 0.f;
+    }
+    if (p.gate_logits) {  // alpha = exp(-alpha_scale[hv] softplus(x)); b, w = sigmoid(x)
+        const float a_h = __ldg(p.alpha_scale + hv);
+#pragma unroll
+        for (int u = 0; u < NI; ++u) {
+            ga[u] = expf(-a_h * (fmaxf(ga[u], 0.f) + log1pf(expf(-fabsf(ga[u])))));
+            gb[u] = 1.f / (1.f + expf(-gb[u]));
+        }
+#pragma unroll
+        for (int u = 0; u < NJ; ++u) gw[u] = 1.f / (1.f + expf(-gw[u]));
+    }
 
     // ---- per-token vectors -------------------------------------------------------------
     if (CONV) {
@@ -88,11 +109,19 @@ decode_step_kernel(DecodeParams p) {
         for (int j = tid; j < DV; j += NTH) zs[j] = to_f32(v[j]);
         __syncthreads();
     }
-    for (int i = tid; i < DK; i += NTH) {
-        as_[i] = alpha_of(to_f32(al[APC ? i : 0]));
-        es[i] = sig_of(to_f32(bg[GPC ? i : 0])) * ks[i];
+#pragma unroll
+    for (int u = 0; u < NI; ++u) {
+        const int i = tid + u * NTH;
+        if (i < DK) {
+            as_[i] = ga[u];
+            es[i] = gb[u] * ks[i];
+        }
     }
-    for (int j = tid; j < DV; j += NTH) zs[j] *= sig_of(to_f32(wg[GPC ? j : 0]));
+#pragma unroll
+    for (int u = 0; u < NJ; ++u) {
+        const int j = tid + u * NTH;
+        if (j < DV) zs[j] *= gw[u];
+    }
     __syncthreads();
 
     // ---- state read, decay, erase read-out ---------------------------------------------

@@ -71,7 +71,9 @@ using tcfwd::ldf4;
 using tcfwd::split8;
 using tcfwd::split_pack;
 using tcfwd::st16;
+using tcfwd::l2_evict_last_policy;
 using tcfwd::tma4;
+using tcfwd::tma4_pol;
 using tcfwd::unpack8;
 using tcfwd::wait1;
 
@@ -793,27 +795,30 @@ struct Maps {
 
 // SPLIT: as in the scan, m.a maps k lo and m.b maps q lo.
 template <bool APC, bool GPC, bool SPLIT>
+// The epilogue group reads the same q, k, alpha, b rows again with plain loads while the chunk is
+// walked: the tiles are loaded with L2 evict_last priority so that those reads hit L2.
 __device__ __forceinline__ void load_raw_g(const Ctx& cx, const ChunkPos& cp, const Maps& m) {
     const uint32_t base = smem_u32(cx.sm);
     uint64_t* bar = cx.bars + B_RAW;
+    const uint64_t pol = l2_evict_last_policy();
     mbar_arrive_expect_tx(bar, 32768u + (GPC || SPLIT ? 16384u : 0u) + (APC || SPLIT ? 16384u : 0u));
     if (SPLIT) {
-        tma4(base + SM_RQB, m.b, bar, 0, cp.hk, cp.t0, cp.b);  // q lo -> rows 0-63
-        tma4(base + SM_RQB + 16384, m.b, bar, 64, cp.hk, cp.t0, cp.b);
-        tma4(base + SM_RA, m.a, bar, 0, cp.hk, cp.t0, cp.b);    // k lo
-        tma4(base + SM_RA + 8192, m.a, bar, 64, cp.hk, cp.t0, cp.b);
+        tma4_pol(base + SM_RQB, m.b, bar, 0, cp.hk, cp.t0, cp.b, pol);  // q lo -> rows 0-63
+        tma4_pol(base + SM_RQB + 16384, m.b, bar, 64, cp.hk, cp.t0, cp.b, pol);
+        tma4_pol(base + SM_RA, m.a, bar, 0, cp.hk, cp.t0, cp.b, pol);    // k lo
+        tma4_pol(base + SM_RA + 8192, m.a, bar, 64, cp.hk, cp.t0, cp.b, pol);
     }
-    tma4(base + SM_RQB + 8192, m.q, bar, 0, cp.hk, cp.t0, cp.b);
-    tma4(base + SM_RQB + 16384 + 8192, m.q, bar, 64, cp.hk, cp.t0, cp.b);
-    tma4(base + SM_RK, m.k, bar, 0, cp.hk, cp.t0, cp.b);
-    tma4(base + SM_RK + 8192, m.k, bar, 64, cp.hk, cp.t0, cp.b);
+    tma4_pol(base + SM_RQB + 8192, m.q, bar, 0, cp.hk, cp.t0, cp.b, pol);
+    tma4_pol(base + SM_RQB + 16384 + 8192, m.q, bar, 64, cp.hk, cp.t0, cp.b, pol);
+    tma4_pol(base + SM_RK, m.k, bar, 0, cp.hk, cp.t0, cp.b, pol);
+    tma4_pol(base + SM_RK + 8192, m.k, bar, 64, cp.hk, cp.t0, cp.b, pol);
     if (GPC) {
-        tma4(base + SM_RQB, m.b, bar, 0, cp.hv, cp.t0, cp.b);
-        tma4(base + SM_RQB + 16384, m.b, bar, 64, cp.hv, cp.t0, cp.b);
+        tma4_pol(base + SM_RQB, m.b, bar, 0, cp.hv, cp.t0, cp.b, pol);
+        tma4_pol(base + SM_RQB + 16384, m.b, bar, 64, cp.hv, cp.t0, cp.b, pol);
     }
     if (APC) {
-        tma4(base + SM_RA, m.a, bar, 0, cp.hv, cp.t0, cp.b);
-        tma4(base + SM_RA + 8192, m.a, bar, 64, cp.hv, cp.t0, cp.b);
+        tma4_pol(base + SM_RA, m.a, bar, 0, cp.hv, cp.t0, cp.b, pol);
+        tma4_pol(base + SM_RA + 8192, m.a, bar, 64, cp.hv, cp.t0, cp.b, pol);
     }
 }
 

@@ -279,6 +279,22 @@ __device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint6
         : "memory");
 }
 
+// tma4 with an L2 cache policy (from createpolicy): tiles that plain loads read again soon stay
+// in L2 with evict_last priority.
+__device__ __forceinline__ void tma4_pol(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2,
+                                         int c3, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(pol)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // Raw tiles of chunk n.  With SPLIT (scalar gates only) q, k, v arrive as bf16 hi + lo pairs of
 // fp32 values; the lo halves take the tiles that scalar gates leave free: q lo the b rows of RQB,
 // k lo the alpha tile, v lo the w tile (the maps in the tb_, ta and tw slots point at them).
