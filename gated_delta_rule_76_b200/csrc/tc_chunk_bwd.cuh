@@ -707,10 +707,11 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 //   P9 = dS_end V'^T                                 -> dKbar^T
 // S0 and dS_end are A operands in tensor memory (lane c holds row c); every other operand is a
 // bf16 hi/lo pair of 128-byte-swizzled shared-memory tiles.  Once P7-P9 of chunk i are complete,
-// the epilogue group (warps 0-3, lane c = channel c) writes dv, dw and then every other gradient
-// of chunk i, walking the tokens from last to first so that the reverse cumulative sum of the
-// log-decay gradient is a running sum per thread, while the staging group (warps 4-7) loads
-// chunk i + 1: S0 and dS_end into tensor memory, the TMA tiles, the split factors.
+// the epilogue group (warps 0-3, lane c = channel c) writes dq, dk, db, dalpha of chunk i, walking
+// the tokens from last to first so that the reverse cumulative sum of the log-decay gradient is a
+// running sum per thread (its q, k, alpha, b rows from a TMA copy into tiles the products have
+// finished with), while the staging group (warps 4-7) loads chunk i + 1 (S0 and dS_end into
+// tensor memory, the TMA tiles, the split factors) and then writes dv, dw of chunk i.
 namespace grad {
 
 constexpr int kThreads = 256;
@@ -744,7 +745,21 @@ constexpr uint32_t SX_RA = 256;     // [4][64] per-warp sums over channels of d 
 constexpr uint32_t SX_RB = 1280;    // [4][64] per-warp sums over channels of de .* k
 constexpr uint32_t SX_BYTES = 2304;
 
-enum Bar { B_RAW = 0, B_GV, B_P6, B_P789, B_COUNT };
+enum Bar {
+    B_RAW = 0,  // q, k, alpha, b tiles of the staged chunk landed
+    B_GV,       // G and V' tiles landed
+    B_P6,
+    B_P789,
+    B_WK,       // the walk's q, k (and alpha, b, or q lo, k lo) tiles of the walked chunk landed
+    B_COUNT
+};
+// The epilogue walk reads its q, k, alpha, b rows from a second TMA copy of the chunk's tiles, taken
+// into tiles the products no longer need once P7-P9 are complete: q into the dO rows of the G hi
+// tile (its two 64-channel boxes 16 KB apart), k into the second half of the [dP; dA] tile (the
+// staging group's row-group products use the first), alpha and b (channel gates) or the lo halves
+// of q and k (split inputs) into the V' tile.
+constexpr uint32_t SW_Q = SM_GH, SW_K = SM_DPA + 16384, SW_A = SM_VP, SW_B = SM_VP + 16384;
+constexpr uint32_t SW_QBOX = 16384;  // byte distance of q's second box (8 KB for the others)
 
 struct Params {
     Problem pb;
@@ -842,6 +857,32 @@ __device__ __forceinline__ void load_gv(const Ctx& cx, const ChunkPos& cp, const
     tma4(base + SM_VP + 16384 + 8192, m.vl, bar, 64, cp.hv, cp.t0, cp.b);
 }
 
+// The walked chunk's q, k (and alpha, b with channel gates, or q lo, k lo with split inputs) tiles
+// once more, into the tiles P7-P9 have finished with, for the epilogue walk.
+template <bool APC, bool GPC, bool SPLIT>
+__device__ __forceinline__ void load_walk(const Ctx& cx, const ChunkPos& cp, const Maps& m) {
+    const uint32_t base = smem_u32(cx.sm);
+    uint64_t* bar = cx.bars + B_WK;
+    const bool ta = APC || SPLIT, tb = GPC || SPLIT;
+    mbar_arrive_expect_tx(bar, 32768u + (ta ? 16384u : 0u) + (tb ? 16384u : 0u));
+    tma4(base + SW_Q, m.q, bar, 0, cp.hk, cp.t0, cp.b);
+    tma4(base + SW_Q + SW_QBOX, m.q, bar, 64, cp.hk, cp.t0, cp.b);
+    tma4(base + SW_K, m.k, bar, 0, cp.hk, cp.t0, cp.b);
+    tma4(base + SW_K + 8192, m.k, bar, 64, cp.hk, cp.t0, cp.b);
+    if (ta) {  // alpha (value head), or q lo (key head; its map takes the b slot)
+        const CUtensorMap* t = SPLIT ? m.b : m.a;
+        const int h = SPLIT ? cp.hk : cp.hv;
+        tma4(base + SW_A, t, bar, 0, h, cp.t0, cp.b);
+        tma4(base + SW_A + 8192, t, bar, 64, h, cp.t0, cp.b);
+    }
+    if (tb) {  // b (value head), or k lo (key head; its map takes the alpha slot)
+        const CUtensorMap* t = SPLIT ? m.a : m.b;
+        const int h = SPLIT ? cp.hk : cp.hv;
+        tma4(base + SW_B, t, bar, 0, h, cp.t0, cp.b);
+        tma4(base + SW_B + 8192, t, bar, 64, h, cp.t0, cp.b);
+    }
+}
+
 // Sum of v over the 32 lanes of a warp.
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -904,7 +945,7 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
     uint8_t* RK = cx.sm + SM_RK;
     uint8_t* RA = cx.sm + SM_RA;
     uint8_t* EQ = cx.sm + SM_EQ;
-    float* part = reinterpret_cast<float*>(cx.sm + SM_DPA);  // [8][128], before [dP;dA] is written
+    float* part = reinterpret_cast<float*>(cx.sm + SM_DPA);  // [8][128]: before [dP;dA] is written, below the walk's k
     const float scale = pb.scale;
     const int b = cp.b, hv = cp.hv, t0 = cp.t0, L = cp.L;
     const int cg = c & 15, rg = c >> 4, r0 = 8 * rg;
@@ -1151,22 +1192,27 @@ __device__ __forceinline__ RowPtrs row_ptrs(const Params& p, const ChunkPos& cp,
 // Inputs of tokens r0 .. r0 + RB - 1.  FULL: every row of the chunk is inside the sequence; else rows
 // past the sequence read its last token and are then replaced (a load under a branch would be waited
 // for where the branch ends).
+// The walk tiles hold channel c of token r at box (c >> 6), row r, 16-byte chunk ((c & 63) >> 3) ^ (r & 7)
+// (128-byte swizzle), byte 2 (c & 7); boxes are 8 KB apart, q's SW_QBOX.
 template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT, bool LG>
-__device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, const RowPtrs& rp, int r0, RowIn& x) {
+__device__ __forceinline__ void load_rows(const Params& p, const Ctx& cx, const ChunkPos& cp, const RowPtrs& rp,
+                                          int c, int r0, RowIn& x) {
     const TG* ag = static_cast<const TG*>(p.alpha);
     const TG* bg = static_cast<const TG*>(p.b);
+    const uint32_t cb = (uint32_t)(c >> 6) * 8192u + (uint32_t)(c & 7) * 2u, cc = (uint32_t)((c & 63) >> 3);
+    const uint8_t* wq = cx.sm + SW_Q + (uint32_t)(c >> 6) * (SW_QBOX - 8192u);
 #pragma unroll
     for (int i = 0; i < RB; ++i) {
         const int r = r0 + i, rr = FULL ? r : min(r, cp.L - 1);
-        float q0 = __bfloat162float(__ldg(p.q + rp.qk + rr * rp.qk_s));
-        float k0 = __bfloat162float(__ldg(p.k + rp.qk + rr * rp.qk_s));
+        const uint32_t off = cb + (uint32_t)r * 128u + ((cc ^ (uint32_t)(r & 7)) << 4);
+        float q0 = bf(wq, off);
+        float k0 = bf(cx.sm + SW_K, off);
         if (SPLIT) {
-            q0 += __bfloat162float(__ldg(p.q_lo + rp.qk + rr * rp.qk_s));
-            k0 += __bfloat162float(__ldg(p.k_lo + rp.qk + rr * rp.qk_s));
+            q0 += bf(cx.sm + SW_A, off);
+            k0 += bf(cx.sm + SW_B, off);
         }
-        const float b0 = p.pb.sig_t<LG>(GPC ? to_f32(__ldg(bg + rp.g + rr * rp.g_s)) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s)));
-        const float a0 = p.pb.alpha_t<LG>(cp.hv, APC ? to_f32(__ldg(ag + rp.g + rr * rp.g_s))
-                                                  : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s)));
+        const float b0 = p.pb.sig_t<LG>(GPC ? bf(cx.sm + SW_B, off) : to_f32(__ldg(bg + rp.s1 + rr * rp.s1_s)));
+        const float a0 = p.pb.alpha_t<LG>(cp.hv, APC ? bf(cx.sm + SW_A, off) : to_f32(__ldg(ag + rp.s1 + rr * rp.s1_s)));
         const bool in = FULL || r < cp.L;
         x.q[i] = in ? q0 : 0.f;
         x.k[i] = in ? k0 : 0.f;
@@ -1176,8 +1222,8 @@ __device__ __forceinline__ void load_rows(const Params& p, const ChunkPos& cp, c
 }
 
 template <bool APC, bool GPC, bool FULL, class TG, bool SPLIT, bool LG, class GT, class QT>
-__device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
-                                                float gam, float xtot, float* scr, int it) {
+__device__ __forceinline__ void grad_epilogue_t(const Params& p, const Ctx& cx, const ChunkPos& cp, uint32_t tl, int c,
+                                                int warp, float gam, float xtot, float* scr, int it) {
     const float scale = p.pb.scale;
     const RowPtrs rp = row_ptrs(p, cp, c);
     float G = gam, rg = __fdividef(1.f, gam), run = 0.f;
@@ -1218,12 +1264,12 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
     };
     // two input buffers: a block's loads are in flight while the previous block is formed
     RowIn x0, x1;
-    load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cp, rp, 7 * RB, x0);
+    load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cx, cp, rp, c, 7 * RB, x0);
 #pragma unroll 1
     for (int blk = C / RB - 1; blk > 0; blk -= 2) {
-        load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cp, rp, (blk - 1) * RB, x1);
+        load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cx, cp, rp, c, (blk - 1) * RB, x1);
         do_block(blk, x0);
-        if (blk > 1) load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cp, rp, (blk - 2) * RB, x0);
+        if (blk > 1) load_rows<APC, GPC, FULL, TG, SPLIT, LG>(p, cx, cp, rp, c, (blk - 2) * RB, x0);
         do_block(blk - 1, x1);
         if (c == 0) GDN_BTRACE(it, 10 + (C / RB - 1 - blk) / 2);
     }
@@ -1231,10 +1277,10 @@ __device__ __forceinline__ void grad_epilogue_t(const Params& p, const ChunkPos&
 
 // Full chunks (every chunk but a ragged last one) take the variant without per-token guards.
 template <bool APC, bool GPC, class TG, bool SPLIT, bool LG, class GT, class QT>
-__device__ __forceinline__ void grad_epilogue(const Params& p, const ChunkPos& cp, uint32_t tl, int c, int warp,
-                                              float gam, float xtot, float* scr, int it = 15) {
-    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT, LG, GT, QT>(p, cp, tl, c, warp, gam, xtot, scr, it);
-    else grad_epilogue_t<APC, GPC, false, TG, SPLIT, LG, GT, QT>(p, cp, tl, c, warp, gam, xtot, scr, it);
+__device__ __forceinline__ void grad_epilogue(const Params& p, const Ctx& cx, const ChunkPos& cp, uint32_t tl, int c,
+                                              int warp, float gam, float xtot, float* scr, int it = 15) {
+    if (cp.L == C) grad_epilogue_t<APC, GPC, true, TG, SPLIT, LG, GT, QT>(p, cx, cp, tl, c, warp, gam, xtot, scr, it);
+    else grad_epilogue_t<APC, GPC, false, TG, SPLIT, LG, GT, QT>(p, cx, cp, tl, c, warp, gam, xtot, scr, it);
 }
 
 // Scalar gates: per-token sums over the channels (the epilogue group's per-warp partials, the
@@ -1320,7 +1366,8 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const uint32_t tl = tbase + ((uint32_t)((warp & 3) * 32) << 16);
-    int raw_issued = 0, gv_issued = 0;  // raw tiles: thread 0;  G and V' tiles: thread 128
+    // raw and walk tiles: thread 0;  G and V' tiles: thread 128
+    int raw_issued = 0, gv_issued = 0, wk_issued = 0;
     long ci = blockIdx.x;
     if (ci < nch) {
         const ChunkPos c0 = chunk_pos(pb, ci);
@@ -1431,7 +1478,11 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSL, sbase + SM_VP, id64, true);
             mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSH, sbase + SM_VP + 16384, id64, true);
             mma_commit(cx.bars + B_P789);
-            wait1(cx, B_P789, par);
+            if (wait1(cx, B_P789, par) && !*cx.abort_flag) {
+                // the [dP; dA] and V' tiles are free: the walk's rows of this chunk
+                load_walk<APC, GPC, SPLIT>(cx, cp, m);
+                ++wk_issued;
+            }
             GDN_BTRACE(it, 3);
         }
         __syncthreads();
@@ -1444,11 +1495,16 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 load_raw_g<APC, GPC, SPLIT>(cx, chunk_pos(pb, nx), m);
                 ++raw_issued;
             }
-            if (tid == 0) GDN_BTRACE(it, 9);
+            if (tid == 0) {
+                GDN_BTRACE(it, 9);
+                wait1(cx, B_WK, par);
+            }
+            named_bar(1, 128);
             if (!*cx.abort_flag)
-                grad_epilogue<APC, GPC, TG, SPLIT, LG, GT, QT>(p, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr, it);
+                grad_epilogue<APC, GPC, TG, SPLIT, LG, GT, QT>(p, cx, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr,
+                                                               it);
             if (tid == 0) GDN_BTRACE(it, 5);
-            if (!APC || !GPC) bar_arrive_all(3);  // per-warp partials of the scalar gates written
+            bar_arrive_all(3);  // the walk has read its tiles; per-warp partials of the scalar gates written
         } else {
             if (nx < nch)
                 stage_chunk<APC, GPC, TG, SPLIT, LG>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
@@ -1456,20 +1512,14 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             grad_dv_dw<GPC, TG, SPLIT, LG, GT>(p, cx, cp, tid - 128, scr);
             named_bar(2, 128);
             if (tid == 128) GDN_BTRACE(it, 4);
-            // the G tiles' last reader was dv/dw: the next chunk's G and V' tiles may land; dO lo
-            // shares its rows with the scalar gates' scratch, so then only once that has been read
-            const bool late_gv = dol && (!APC || !GPC);
-            if (!late_gv && tid == 128 && nx < nch && !*cx.abort_flag) {
+            // The next chunk's G and V' tiles may land once dv/dw (the G tiles' last reader) and the
+            // walk (its alpha, b or lo rows are in the V' tile) are done, and with scalar gates once
+            // their scratch (in rows of the G lo tile that dO lo overwrites) has been read.
+            bar_sync_all(3);
+            if ((!APC || !GPC) && !*cx.abort_flag) scalar_gate_finish<APC, GPC, TG, LG, GT>(p, cp, tid - 128, scr);
+            if (tid == 128 && nx < nch && !*cx.abort_flag) {
                 load_gv(cx, chunk_pos(pb, nx), m, dol);
                 ++gv_issued;
-            }
-            if (!APC || !GPC) {
-                bar_sync_all(3);
-                if (!*cx.abort_flag) scalar_gate_finish<APC, GPC, TG, LG, GT>(p, cp, tid - 128, scr);
-                if (late_gv && tid == 128 && nx < nch && !*cx.abort_flag) {
-                    load_gv(cx, chunk_pos(pb, nx), m, dol);
-                    ++gv_issued;
-                }
             }
         }
         if (tid == 0) *stop_slot = *cx.abort_flag;
@@ -1486,6 +1536,9 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         if (gv_issued > 0)
             while (!mbar_try_wait(cx.bars + B_GV, (uint32_t)((gv_issued - 1) & 1)) && globaltimer_ns() - tw < cx.wait_ns) {
+            }
+        if (wk_issued > 0)
+            while (!mbar_try_wait(cx.bars + B_WK, (uint32_t)((wk_issued - 1) & 1)) && globaltimer_ns() - tw < cx.wait_ns) {
             }
     }
     __syncthreads();
