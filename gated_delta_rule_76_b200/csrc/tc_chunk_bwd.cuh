@@ -710,8 +710,8 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // the epilogue group (warps 0-3, lane c = channel c) writes dq, dk, db, dalpha of chunk i, walking
 // the tokens from last to first so that the reverse cumulative sum of the log-decay gradient is a
 // running sum per thread (its q, k, alpha, b rows from a TMA copy into tiles the products have
-// finished with), while the staging group (warps 4-7) loads chunk i + 1 (S0 and dS_end into
-// tensor memory, the TMA tiles, the split factors) and then writes dv, dw of chunk i.
+// finished with), then dv, dw of chunk i, while the staging group (warps 4-7) loads chunk i + 1
+// (S0 and dS_end into tensor memory, the TMA tiles, the split factors).
 namespace grad {
 
 constexpr int kThreads = 256;
@@ -936,6 +936,7 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
         xslot[c] = dot;
         tmem_st_wait();
     }
+    if (c == 0) GDN_BTRACE(it, 6);
     if (c == 0) wait1(cx, B_RAW, raw_parity);
     if (c == 0) GDN_BTRACE(it, 7);
     named_bar(2, 128);
@@ -1066,7 +1067,7 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
 }
 
 // dv = w .* dY, dw = v .* dY (a scalar beta: sum_j v dY per token into scr[SX_DBV]); run by the
-// staging group after its staging, warp w: tokens w, w + 4, ..., lane l: value channels 4l .. 4l + 3.
+// epilogue group after its walk, warp w: tokens w, w + 4, ..., lane l: value channels 4l .. 4l + 3.
 
 template <bool GPC, class TG, bool SPLIT, bool LG, class GT>
 __device__ __forceinline__ void grad_dv_dw(const Params& p, const Ctx& cx, const ChunkPos& cp, int tt, float* scr) {
@@ -1504,14 +1505,16 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 grad_epilogue<APC, GPC, TG, SPLIT, LG, GT, QT>(p, cx, cp, tl, tid, warp, gam_c, gam_c * (xs + dot_c), scr,
                                                                it);
             if (tid == 0) GDN_BTRACE(it, 5);
-            bar_arrive_all(3);  // the walk has read its tiles; per-warp partials of the scalar gates written
+            // dv, dw of this chunk (the staging group's loads of the next chunk's states are the longer
+            // part of its work, so this group takes them after its walk)
+            grad_dv_dw<GPC, TG, SPLIT, LG, GT>(p, cx, cp, tid, scr);
+            if (tid == 0) GDN_BTRACE(it, 4);
+            // the walk and dv/dw have read their tiles; the scalar gates' partials are written
+            bar_arrive_all(3);
         } else {
             if (nx < nch)
                 stage_chunk<APC, GPC, TG, SPLIT, LG>(p, cx, chunk_pos(pb, nx), tl, tid - 128, xslot, gslot, par ^ 1u, it);
             if (tid == 128) GDN_BTRACE(it, 8);
-            grad_dv_dw<GPC, TG, SPLIT, LG, GT>(p, cx, cp, tid - 128, scr);
-            named_bar(2, 128);
-            if (tid == 128) GDN_BTRACE(it, 4);
             // The next chunk's G and V' tiles may land once dv/dw (the G tiles' last reader) and the
             // walk (its alpha, b or lo rows are in the V' tile) are done, and with scalar gates once
             // their scratch (in rows of the G lo tile that dO lo overwrites) has been read.
