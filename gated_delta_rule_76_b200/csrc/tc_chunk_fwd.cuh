@@ -6,20 +6,21 @@
 //   Gamma_r = prod_{i<=r} alpha_i,  gamma = Gamma_63;  Ehat = (b.*k).*Gamma,  Qhat = q.*Gamma,
 //   Ktil = k./Gamma,  Kbar = k.*gamma./Gamma;   A = strict_lower(Ehat Ktil^T),
 //   P = lower(Qhat Ktil^T),  T = (I + A)^-1,   V' = T (Z - Ehat S0),  Z = w.*v,
-//   O = scale (Qhat S0 + P V'),  S_end = Diag(gamma) S0 + Kbar^T V'.
+//   O = scale (Qhat S0 + P V'),  S_end = Diag(gamma) S0 + Kbar^T V' = Diag(gamma) (S0 + Ktil^T V').
 // Every product is issued with M = 128 by putting dv on the M side (D[j][..] = sum A[j][k] B[..][k]):
 //   X1 = [Ehat;Qhat] Ktil^T               (M = 128 rows of Ehat/Qhat, N = 64, K = 128)
 //   X2 = S0^T [Ehat;Qhat]^T               (M = dv, N = 2 x 64, K = dk; A = S0^T in tensor memory)
 //   X3 = Y^T T^T   with Y^T = Z^T - (Ehat S0)^T  (M = dv, N = 64, K = 64; A in tensor memory)
 //   X4 = V'^T P^T  accumulated onto (Qhat S0)^T  (M = dv, N = 64, K = 64)
-//   X5 = V'^T Kbar (B = Kbar^T, K-major)  (M = dv, N = dk, K = 64)
+//   X5 = V'^T Ktil (B = Ktil MN-major, the tile X1 read)  (M = dv, N = dk, K = 64); gamma is
+//        applied in the state update
 //
 // Precision.  A bf16 operand carries a relative rounding of up to 2^-9, and with seven rounded
 // operand families the output error reaches ~4% of its RMS at the largest entry.  Every derived
 // operand x is therefore carried as a pair hi = bf16(x), lo = bf16(x - hi) and the products take
 // the cross terms that matter (hi*hi + lo*hi + hi*lo), each in fp32 in tensor memory:
 //   X1: Ehat, Qhat and Ktil split (3 MMAs);  X2: S0 split, and Qhat split in Qhat S0 (2 + 3 MMAs);
-//   X3: Y and T split (3);  X4: V' and P split (3);  X5: V' and Kbar split (3).
+//   X3: Y and T split (3);  X4: V' and P split (3);  X5: V' and Ktil split (3).
 // T lo shares the fp32 scratch of the solve: the next chunk's A is written there only after X3 of
 // this chunk has completed.
 //
@@ -27,15 +28,16 @@
 // the fp32 state in registers, split between the warpgroups by halves of dk.
 // Roles (384 threads):
 //   warps 0-7  (scan)     : the sequential chain X2 -> Y -> X3 -> V' -> X4, X5 -> output, state;
-//                           while X2 runs they build Kbar^T (from the split Ktil and gamma), and
 //                           while the prologue solves for T they build P (from X1).  Thread 0
 //                           issues the scan's MMAs and all TMA loads (the z tile of a gated output
 //                           at the top of each chunk).
 //   warps 8-11 (prologue) : for the next chunk, the cumulative decay and the split operands, X1,
 //                           and the triangular solve T = (I + A)^-1; thread 256 issues X1.
-// Operand tiles are single-buffered.  [Ehat;Qhat] and T each have a "ready" barrier (prologue ->
-// scan) and a "free" barrier (the scan's MMA that read it has completed -> prologue); the raw TMA
-// stage is reloaded as soon as X1 and the Kbar^T pass (its last readers) are done.  Saving mode
+// The Ktil tiles (where the raw k and alpha tiles land) are double-buffered by chunk parity, so X5
+// of a chunk can read them while the next chunk's are formed; the other operand tiles are single-
+// buffered.  [Ehat;Qhat] and T each have a "ready" barrier (prologue -> scan) and a "free" barrier
+// (the scan's MMA that read it has completed -> prologue); the raw TMA stage is reloaded as soon as
+// X1 and X2 (the last readers of [Ehat;Qhat] lo) are done.  Saving mode
 // (the backward cache) stores the entering state and V' while the MMAs run.  Split inputs (fp32
 // q, k, v as bf16 hi/lo pairs, scalar gates only) take the lo tiles in the gate slots.  Every
 // mbarrier wait is bounded: on expiry the kernel sets an error word, stops issuing work and frees
@@ -74,7 +76,7 @@ constexpr uint64_t kWaitNs = 4000000000ull;
 // tensor memory columns
 constexpr uint32_t TM_X1 = 0;     // 64:  A (lanes 0-63), P (lanes 64-127), fp32
 constexpr uint32_t TM_X2 = 64;    // 128: (Ehat S0)^T | (Qhat S0 + P V')^T
-constexpr uint32_t TM_X5 = 192;   // 128: first V'^T = (Y^T T^T) in cols 0-63, then (Kbar^T V')^T
+constexpr uint32_t TM_X5 = 192;   // 128: first V'^T = (Y^T T^T) in cols 0-63, then V'^T Ktil
 constexpr uint32_t TM_S0H = 320;  // 64:  S0^T hi, bf16 pairs
 constexpr uint32_t TM_S0L = 384;  // 64:  S0^T lo
 constexpr uint32_t TM_YH = 448;   // 32:  Y^T (then V'^T) hi
@@ -83,13 +85,15 @@ constexpr uint32_t TM_COLS = 512;
 
 // shared memory offsets from the 1024-byte-aligned base (K-major 128-byte-swizzled bf16 tiles)
 constexpr uint32_t SM_RQB = 0;        // 32 KB [2 atoms][128 rows]: TMA b (rows 0-63), q (64-127) -> [Ehat;Qhat] lo
-constexpr uint32_t SM_RK = 32768;     // 16 KB [2][64]: TMA k -> Ktil hi
-constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo
+constexpr uint32_t SM_RK = 32768;     // 16 KB [2][64]: TMA k -> Ktil hi (even chunks)
+constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo (even chunks)
 constexpr uint32_t SM_EQ = 65536;     // 32 KB [2][128]: [Ehat;Qhat] hi
 constexpr uint32_t SM_Z = 98304;      // 16 KB [2][64]: TMA z tile of the scan's chunk (gated output)
 constexpr uint32_t SM_T = 114688;     // 8 KB [1][64]: T
 constexpr uint32_t SM_P = 122880;     // 16 KB: P hi [1][64], P lo [1][64]
-constexpr uint32_t SM_KB = 139264;    // 32 KB: Kbar^T hi [1][128], Kbar^T lo [1][128]
+constexpr uint32_t SM_KB = 139264;    // 32 KB: TMA k -> Ktil hi [2][64], TMA alpha -> Ktil lo [2][64]
+                                      // (odd chunks: the Ktil tiles are double-buffered, X5 of one
+                                      // chunk reads them while the next chunk's are formed)
 constexpr uint32_t SM_VW = 172032;    // 32 KB: v [2][64], w [2][64]
 constexpr uint32_t SM_ASCR = 204800;  // 17 KB: A, then T, fp32 [64][LDA] row-major; then T lo
 constexpr uint32_t SM_TLO = SM_ASCR;   // 8 KB [1][64]: T lo (bf16), from the solve until X3 has read it
@@ -103,6 +107,9 @@ constexpr uint32_t SM_END = SM_NRM + 1024;
 constexpr int LDA = 68;  // fp32 row stride of the A/T scratch: float4 rows, rows 16 B apart in bank
 constexpr int LDR = 52;  // fp32 row stride of the block-row products
 constexpr size_t kSmemBytes = SM_END + 1024;
+// Ktil hi / lo tiles of chunk n
+__device__ __forceinline__ uint32_t kt_hi(int n) { return (n & 1) ? SM_KB : SM_RK; }
+__device__ __forceinline__ uint32_t kt_lo(int n) { return (n & 1) ? SM_KB + 16384u : SM_RA; }
 
 enum Bar {
     B_RAW = 0,      // q, k, alpha, b tiles of the prologue's chunk landed
@@ -308,8 +315,8 @@ __device__ __forceinline__ void load_raw(const Ctx& cx, int n, int b, int hk, in
     mbar_arrive_expect_tx(bar, 32768u + (GPC || SPLIT ? 16384u : 0u) + (APC || SPLIT ? 16384u : 0u));
     tma4(base + SM_RQB + 8192, tq, bar, 0, hk, t0, b);           // q -> rows 64-127, channels 0-63
     tma4(base + SM_RQB + 16384 + 8192, tq, bar, 64, hk, t0, b);  // channels 64-127
-    tma4(base + SM_RK, tk, bar, 0, hk, t0, b);
-    tma4(base + SM_RK + 8192, tk, bar, 64, hk, t0, b);
+    tma4(base + kt_hi(n), tk, bar, 0, hk, t0, b);
+    tma4(base + kt_hi(n) + 8192, tk, bar, 64, hk, t0, b);
     if (GPC || SPLIT) {
         const int hb = SPLIT ? hk : hv;
         tma4(base + SM_RQB, tb_, bar, 0, hb, t0, b);              // b (or q lo) -> rows 0-63
@@ -317,8 +324,8 @@ __device__ __forceinline__ void load_raw(const Ctx& cx, int n, int b, int hk, in
     }
     if (APC || SPLIT) {
         const int ha = SPLIT ? hk : hv;
-        tma4(base + SM_RA, ta, bar, 0, ha, t0, b);                // alpha (or k lo)
-        tma4(base + SM_RA + 8192, ta, bar, 64, ha, t0, b);
+        tma4(base + kt_lo(n), ta, bar, 0, ha, t0, b);             // alpha (or k lo)
+        tma4(base + kt_lo(n) + 8192, ta, bar, 64, ha, t0, b);
     }
 }
 
@@ -456,32 +463,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_commit(cx.bars + B_EQ_FREE);
                 }
             }
-            // The prologue's Ktil and gamma of this chunk are in shared memory (EQ_READY).
-            named_bar(1, 256);
-            // ---- Kbar^T of this chunk (operand of X5), while X2 runs --------------------------------
-            {
-                // Kbar^T row j, tokens 32 h .. 32 h + 31: (Ktil hi + lo) * gamma, split.
-                uint8_t* KB = sm + SM_KB;
-                const uint8_t* RK = sm + SM_RK;
-                const uint8_t* RA = sm + SM_RA;
-                const float G = gam[(n % 3) * 128 + j];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int ch = 4 * h + cc;
-                    uint32_t wh[4], wl[4];
-                    const uint32_t ob = vbase + (uint32_t)ch * 1024u;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t o0 = ob + (2 * e) * 128u + xo[2 * e];
-                        const uint32_t o1 = ob + (2 * e + 1) * 128u + xo[2 * e + 1];
-                        const float k0 = (bf(RK, o0) + bf(RA, o0)) * G, k1 = (bf(RK, o1) + bf(RA, o1)) * G;
-                        split_pack(k0, k1, wh[e], wl[e]);
-                    }
-                    const uint32_t off = sw128_offset(j, 8 * ch, 128);
-                    st16(KB + off, make_uint4(wh[0], wh[1], wh[2], wh[3]));
-                    st16(KB + 16384 + off, make_uint4(wl[0], wl[1], wl[2], wl[3]));
-                }
-            }
             if (p.s0_out) {
                 // state entering chunk n (saving mode), stored while X2 runs: rows 64h .. 64h + 63
                 // of column j, in the layout [j / 4][row][j % 4] (a reader holding one row per
@@ -495,8 +476,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             named_bar(1, 256);
             if (tid == 0) {
                 tc_fence_after();
-                // X1 and the Kbar^T pass were the last readers of the raw stage: load the next chunk's.
+                // X1 and X2 of this chunk were the last readers of the [Ehat;Qhat] lo tile, and the
+                // next chunk's Ktil tiles were last read by X5 of the previous chunk: the next
+                // chunk's raw tiles may land.
                 wait1(cx, B_X1, pn);
+                wait1(cx, B_EQ_FREE, pn);
                 GDN_TRACE(n, 8);
                 if (raw_issued < NT && !*cx.abort_flag) {
                     load_raw<APC, GPC, SPLIT>(cx, raw_issued, b, hk, hv, &tm_q, &tm_k, &tm_a, &tm_b);
@@ -602,15 +586,24 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 GDN_TRACE(n, 7);
                 tc_fence_after();
                 if (!*cx.abort_flag) {
-                    const uint32_t P = sbase + SM_P, KB = sbase + SM_KB;
+                    const uint32_t P = sbase + SM_P, kh = sbase + kt_hi(n), kl = sbase + kt_lo(n);
                     if (p.o) {
                         mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P, id64, true);
                         mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YL, P, id64, true);
                         mma_ts_u<64, 64>(tbase + TM_X2 + 64, tbase + TM_YH, P + 8192, id64, true);
                     }
-                    mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB, id128, false);
-                    mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YL, KB, id128, true);
-                    mma_ts_u<64, 128>(tbase + TM_X5, tbase + TM_YH, KB + 16384, id128, true);
+                    // X5' = V'^T Ktil: the Ktil tiles are MN-major B operands (token rows, 64
+                    // channels per 128-byte row, the two channel halves 8 KB apart); gamma is
+                    // applied in the state update, S = Diag(gamma) (S0 + X5'^T)
+                    const uint32_t id_x5 = idesc_bf16_f32_mn(128, 128, false, true);
+#pragma unroll
+                    for (int k = 0; k < C; k += 16) {
+                        const uint64_t bh = sdesc_mn_sw128(kh + (uint32_t)k * 128u, 8192u);
+                        const uint64_t bl = sdesc_mn_sw128(kl + (uint32_t)k * 128u, 8192u);
+                        mma_ts(tbase + TM_X5, tbase + TM_YH + (uint32_t)(k >> 1), bh, id_x5, k > 0 ? 1u : 0u);
+                        mma_ts(tbase + TM_X5, tbase + TM_YL + (uint32_t)(k >> 1), bh, id_x5, 1u);
+                        mma_ts(tbase + TM_X5, tbase + TM_YH + (uint32_t)(k >> 1), bl, id_x5, 1u);
+                    }
                     mma_commit(cx.bars + B_X45);
                 }
             }
@@ -710,10 +703,10 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int i4 = 0; i4 < 8; ++i4) {
                         const float4 g = g4[8 * q2 + i4];
                         const int i = 4 * i4;
-                        S[32 * q2 + i + 0] = fmaf(g.x, S[32 * q2 + i + 0], __uint_as_float(r[i + 0]));
-                        S[32 * q2 + i + 1] = fmaf(g.y, S[32 * q2 + i + 1], __uint_as_float(r[i + 1]));
-                        S[32 * q2 + i + 2] = fmaf(g.z, S[32 * q2 + i + 2], __uint_as_float(r[i + 2]));
-                        S[32 * q2 + i + 3] = fmaf(g.w, S[32 * q2 + i + 3], __uint_as_float(r[i + 3]));
+                        S[32 * q2 + i + 0] = g.x * (S[32 * q2 + i + 0] + __uint_as_float(r[i + 0]));
+                        S[32 * q2 + i + 1] = g.y * (S[32 * q2 + i + 1] + __uint_as_float(r[i + 1]));
+                        S[32 * q2 + i + 2] = g.z * (S[32 * q2 + i + 2] + __uint_as_float(r[i + 2]));
+                        S[32 * q2 + i + 3] = g.w * (S[32 * q2 + i + 3] + __uint_as_float(r[i + 3]));
                     }
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
@@ -753,8 +746,6 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float* ascr = reinterpret_cast<float*>(sm + SM_ASCR);
         float* rs = reinterpret_cast<float*>(sm + SM_RS);
         uint8_t* RQB = sm + SM_RQB;
-        uint8_t* RK = sm + SM_RK;
-        uint8_t* RA = sm + SM_RA;
         uint8_t* EQ = sm + SM_EQ;
         const uint32_t id64 = idesc_bf16_f32(128, 64);
         float ga_next = 1.f, gb_next = 0.f;  // scalar gates of the next chunk (threads c < 64)
@@ -762,6 +753,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int m = 0; m < NT; ++m) {
             const uint32_t pm = m & 1, pprev = (m - 1) & 1;
             const int t0 = m * C, L = min(C, pb.T - t0);
+            uint8_t* RK = sm + kt_hi(m);  // raw k -> Ktil hi of this chunk
+            uint8_t* RA = sm + kt_lo(m);  // raw alpha (or k lo) -> Ktil lo
             if (!APC || !GPC) {
                 // Scalar gates of chunk m into slot m & 1 (the scan reads beta there); the next
                 // chunk's are loaded now and held in registers, so their latency is hidden.
@@ -921,9 +914,9 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (c == 0) {
                 tc_fence_after();
                 if (!*cx.abort_flag) {
-                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RK, id64, false);
-                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + SM_RA, id64, true);
-                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_RQB, sbase + SM_RK, id64, true);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + kt_hi(m), id64, false);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_EQ, sbase + kt_lo(m), id64, true);
+                    mma_ss_u<128, 128, 64>(tbase + TM_X1, sbase + SM_RQB, sbase + kt_hi(m), id64, true);
                     mma_commit(cx.bars + B_X1);
                 }
                 mbar_arrive(cx.bars + B_EQ_READY);
