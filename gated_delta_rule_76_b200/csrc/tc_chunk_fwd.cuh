@@ -100,12 +100,11 @@ constexpr uint32_t SM_TLO = SM_ASCR;   // 8 KB [1][64]: T lo (bf16), from the so
 constexpr uint32_t SM_GAM = 222208;   // gamma, 3 slots x 128 floats (chunk n uses slot n % 3)
 constexpr uint32_t SM_BAR = 223744;   // mbarriers, tensor memory base, abort flag
 constexpr uint32_t SM_RS = SM_BAR + 256;  // 4 KB: alpha products per row group [8][128], then the
-                                          // block-row products of the solve [16][LDR]
+                                          // solve's products: [2][16][16], then [32][32]
 constexpr uint32_t SM_SG = SM_RS + 4096;  // scalar gates of a chunk: [2 slots][alpha, beta][64] fp32
 constexpr uint32_t SM_NRM = SM_SG + 1024;  // output norm: [2 halves][4 warps][32 tokens] partial sums
 constexpr uint32_t SM_END = SM_NRM + 1024;
 constexpr int LDA = 68;  // fp32 row stride of the A/T scratch: float4 rows, rows 16 B apart in bank
-constexpr int LDR = 52;  // fp32 row stride of the block-row products
 constexpr size_t kSmemBytes = SM_END + 1024;
 // Ktil hi / lo tiles of chunk n
 __device__ __forceinline__ uint32_t kt_hi(int n) { return (n & 1) ? SM_KB : SM_RK; }
@@ -202,54 +201,6 @@ __device__ __forceinline__ void fma4(float (&acc)[4], float a, const float4 t) {
     acc[1] = fmaf(a, t.y, acc[1]);
     acc[2] = fmaf(a, t.z, acc[2]);
     acc[3] = fmaf(a, t.w, acc[3]);
-}
-
-// One block row IB (rows 16 IB .. 16 IB + 15) of T = (I + A)^-1, given the diagonal blocks
-// D_i = (I + A_ii)^-1 and the block rows above it, in place in the fp32 scratch t (row stride LDA):
-//   R = A_{IB, 0:IB} T_{0:IB, 0:IB},   T_{IB, 0:IB} = -D_IB R.
-// Thread c < 32 IB computes rows 2 rp, 2 rp + 1 of the block row and columns 4 cg .. 4 cg + 3.
-template <int IB>
-__device__ __forceinline__ void solve_block_row(float* t, float* rsb, int c) {
-    constexpr int NCG = 4 * IB;
-    const bool act = c < 8 * NCG;
-    const int cg = c % NCG, rp = c / NCG;
-    const int row = 16 * IB + 2 * rp, col = 4 * cg;
-    if (act) {
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-        const float* a0p = t + row * LDA;
-        // T_{0:IB, 0:IB} is lower triangular and the scratch holds zeros above it, so the sum runs
-        // over all 16 IB rows with compile-time bounds: fully unrolled, every load is issued early.
-#pragma unroll
-        for (int kk = 0; kk < 16 * IB; kk += 4) {
-            const float4 a0 = ldf4(a0p + kk), a1 = ldf4(a0p + LDA + kk);
-            const float4 t0 = ldf4(t + (kk + 0) * LDA + col), t1 = ldf4(t + (kk + 1) * LDA + col);
-            const float4 t2 = ldf4(t + (kk + 2) * LDA + col), t3 = ldf4(t + (kk + 3) * LDA + col);
-            fma4(acc0, a0.x, t0); fma4(acc1, a1.x, t0);
-            fma4(acc0, a0.y, t1); fma4(acc1, a1.y, t1);
-            fma4(acc0, a0.z, t2); fma4(acc1, a1.z, t2);
-            fma4(acc0, a0.w, t3); fma4(acc1, a1.w, t3);
-        }
-        *reinterpret_cast<float4*>(rsb + (2 * rp) * LDR + col) = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
-        *reinterpret_cast<float4*>(rsb + (2 * rp + 1) * LDR + col) = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
-    }
-    named_bar(2, 128);
-    if (act) {
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-        const float* d0p = t + row * LDA + 16 * IB;
-#pragma unroll
-        for (int sg = 0; sg < 16; sg += 4) {
-            const float4 d0 = ldf4(d0p + sg), d1 = ldf4(d0p + LDA + sg);
-            const float4 r0 = ldf4(rsb + (sg + 0) * LDR + col), r1 = ldf4(rsb + (sg + 1) * LDR + col);
-            const float4 r2 = ldf4(rsb + (sg + 2) * LDR + col), r3 = ldf4(rsb + (sg + 3) * LDR + col);
-            fma4(acc0, d0.x, r0); fma4(acc1, d1.x, r0);
-            fma4(acc0, d0.y, r1); fma4(acc1, d1.y, r1);
-            fma4(acc0, d0.z, r2); fma4(acc1, d1.z, r2);
-            fma4(acc0, d0.w, r3); fma4(acc1, d1.w, r3);
-        }
-        *reinterpret_cast<float4*>(t + row * LDA + col) = make_float4(-acc0[0], -acc0[1], -acc0[2], -acc0[3]);
-        *reinterpret_cast<float4*>(t + (row + 1) * LDA + col) = make_float4(-acc1[0], -acc1[1], -acc1[2], -acc1[3]);
-    }
-    named_bar(2, 128);
 }
 
 struct Ctx {
@@ -980,12 +931,74 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             named_bar(2, 128);
             if (c == 0) GDN_TRACE(m, 28);
-            // (2) block rows 1..3 below the diagonal.
-            solve_block_row<1>(ascr, rs, c);
+            // (2) the 32 x 32 diagonal halves: T_10 = -D_1 (A_10 D_0) and T_32 = -D_3 (A_32 D_2).
+            //     Thread c: block c >> 6, row i = (c >> 2) & 15 of it, columns 4 (c & 3) .. + 3.
+            {
+                const int bk = c >> 6, i = (c >> 2) & 15, j0 = 4 * (c & 3);
+                const int r0 = 16 + 32 * bk, c0 = 32 * bk;  // the block A_{r0.., c0..}; D above it at c0
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const float* arow = ascr + (r0 + i) * LDA + c0;
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    const float4 a4 = ldf4(arow + k);
+                    fma4(acc, a4.x, ldf4(ascr + (c0 + k + 0) * LDA + c0 + j0));
+                    fma4(acc, a4.y, ldf4(ascr + (c0 + k + 1) * LDA + c0 + j0));
+                    fma4(acc, a4.z, ldf4(ascr + (c0 + k + 2) * LDA + c0 + j0));
+                    fma4(acc, a4.w, ldf4(ascr + (c0 + k + 3) * LDA + c0 + j0));
+                }
+                *reinterpret_cast<float4*>(rs + bk * 256 + i * 16 + j0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                named_bar(2, 128);
+                float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                const float* drow = ascr + (r0 + i) * LDA + r0;  // D_{r0}: lower triangular, zeros above
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    const float4 d4 = ldf4(drow + k);
+                    fma4(t4, d4.x, ldf4(rs + bk * 256 + (k + 0) * 16 + j0));
+                    fma4(t4, d4.y, ldf4(rs + bk * 256 + (k + 1) * 16 + j0));
+                    fma4(t4, d4.z, ldf4(rs + bk * 256 + (k + 2) * 16 + j0));
+                    fma4(t4, d4.w, ldf4(rs + bk * 256 + (k + 3) * 16 + j0));
+                }
+                *reinterpret_cast<float4*>(ascr + (r0 + i) * LDA + c0 + j0) = make_float4(-t4[0], -t4[1], -t4[2], -t4[3]);
+            }
+            named_bar(2, 128);
             if (c == 0) GDN_TRACE(m, 29);
-            solve_block_row<2>(ascr, rs, c);
+            // (3) the lower-left quarter: X = A_LL T_00, then T_LL = -T_11 X (T_00, T_11 the 32 x 32
+            //     diagonal halves, lower triangular with zeros above, so the sums run over all 32).
+            //     Thread c: rows 2 (c >> 3), + 1 of the quarter, columns 4 (c & 7) .. + 3.
+            {
+                const int i = 2 * (c >> 3), j0 = 4 * (c & 7);
+                float x0[4] = {0.f, 0.f, 0.f, 0.f}, x1[4] = {0.f, 0.f, 0.f, 0.f};
+                const float* a0p = ascr + (32 + i) * LDA;
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                    const float4 a0 = ldf4(a0p + k), a1 = ldf4(a0p + LDA + k);
+                    const float4 t0 = ldf4(ascr + (k + 0) * LDA + j0), t1 = ldf4(ascr + (k + 1) * LDA + j0);
+                    const float4 t2 = ldf4(ascr + (k + 2) * LDA + j0), t3 = ldf4(ascr + (k + 3) * LDA + j0);
+                    fma4(x0, a0.x, t0); fma4(x1, a1.x, t0);
+                    fma4(x0, a0.y, t1); fma4(x1, a1.y, t1);
+                    fma4(x0, a0.z, t2); fma4(x1, a1.z, t2);
+                    fma4(x0, a0.w, t3); fma4(x1, a1.w, t3);
+                }
+                *reinterpret_cast<float4*>(rs + i * 32 + j0) = make_float4(x0[0], x0[1], x0[2], x0[3]);
+                *reinterpret_cast<float4*>(rs + (i + 1) * 32 + j0) = make_float4(x1[0], x1[1], x1[2], x1[3]);
+                named_bar(2, 128);
+                float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+                const float* t0p = ascr + (32 + i) * LDA + 32;
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                    const float4 d0 = ldf4(t0p + k), d1 = ldf4(t0p + LDA + k);
+                    const float4 r0 = ldf4(rs + (k + 0) * 32 + j0), r1 = ldf4(rs + (k + 1) * 32 + j0);
+                    const float4 r2 = ldf4(rs + (k + 2) * 32 + j0), r3 = ldf4(rs + (k + 3) * 32 + j0);
+                    fma4(y0, d0.x, r0); fma4(y1, d1.x, r0);
+                    fma4(y0, d0.y, r1); fma4(y1, d1.y, r1);
+                    fma4(y0, d0.z, r2); fma4(y1, d1.z, r2);
+                    fma4(y0, d0.w, r3); fma4(y1, d1.w, r3);
+                }
+                *reinterpret_cast<float4*>(ascr + (32 + i) * LDA + j0) = make_float4(-y0[0], -y0[1], -y0[2], -y0[3]);
+                *reinterpret_cast<float4*>(ascr + (33 + i) * LDA + j0) = make_float4(-y1[0], -y1[1], -y1[2], -y1[3]);
+            }
+            named_bar(2, 128);
             if (c == 0) GDN_TRACE(m, 30);
-            solve_block_row<3>(ascr, rs, c);
             // (3) T (fp32) -> K-major bf16 tiles T hi (SM_T) and T lo (the first 8 KB of the scratch,
             //     once every thread holds its values): thread c converts half c >> 6 of row c & 63.
             if (c == 0) GDN_TRACE(m, 21);
