@@ -110,11 +110,10 @@ def load_peaks():
 
 
 # DRAM bytes (read + write) of one gdn_chunk_bwd call on the headline workload, summed over its two
-# kernels (reverse scan, gradients) from ncu's dram__bytes_read.sum + dram__bytes_write.sum on
-# B=8 T=1024 (the same 128 (sequence, head) pairs, a quarter of the chunks; the traffic is per
-# chunk, so x4).  None until a capture of the kernels as they are now exists; to be reset to None
-# whenever those kernels change.
-BWD_CALL_TRAFFIC_BYTES = None
+# kernels (reverse scan 338,971,648 B, gradients 811,468,288 B) from ncu's dram__bytes_read.sum +
+# dram__bytes_write.sum on B=8 T=1024 (the same 128 (sequence, head) pairs, a quarter of the
+# chunks; the traffic is per chunk, so x4).  To be reset to None whenever those kernels change.
+BWD_CALL_TRAFFIC_BYTES = (338971648 + 811468288) * 4
 
 
 def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False,
