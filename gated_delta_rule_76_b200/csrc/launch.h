@@ -46,7 +46,7 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
 // entering every chunk and V' of every token are written for the backward (o and ht may be NULL).
 struct TcFwdSave {
     float* s0;               // [B*Hv][NT + 1][dv/4][dk][4]
-    __nv_bfloat16* vp_hi;    // [B,T,Hv,dv]
+    __nv_bfloat16* vp_hi;    // [B*Hv][NT][dv][64 tokens]: chunk-major, a column's tokens contiguous
     __nv_bfloat16* vp_lo;
     float* o_raw;            // with the swish gate, may be NULL: the output before the gate (fp32)
     uint8_t* t;              // [B*Hv][NT] 8 KB images of each chunk's bf16 T tile (swizzled), or NULL
@@ -84,7 +84,7 @@ cudaError_t compose_states(const float* M, const float* N, const float* S_in, fl
 // The forward cache (what the backward needs from the forward): byte offsets from its start.
 struct TcCache {
     size_t bytes = 0;
-    size_t s0, vp_hi, vp_lo;  // states [B*Hv][NT+1][dv/4][dk][4] fp32; V' hi, lo [B,T,Hv,dv] bf16
+    size_t s0, vp_hi, vp_lo;  // states [B*Hv][NT+1][dv/4][dk][4] fp32; V' hi, lo [B*Hv][NT][dv][64] bf16
     size_t t;                 // T tiles [B*Hv][NT][8 KB]: bf16, 64 rows of 128 swizzled bytes
 };
 TcCache plan_tc_cache(const Problem& pb);

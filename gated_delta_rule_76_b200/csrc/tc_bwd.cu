@@ -28,8 +28,9 @@ TcCache plan_tc_cache(const Problem& pb) {
         return o;
     };
     c.s0 = take(st1);  // entering state of every chunk, then the final state
-    c.vp_hi = take(tok);
-    c.vp_lo = take(tok);
+    const size_t vtile = (size_t)pb.B * pb.Hv * pb.NT * pb.dv * 64 * 2;  // chunk-major, padded to 64 tokens
+    c.vp_hi = take(vtile);
+    c.vp_lo = take(vtile);
     c.t = take((size_t)pb.B * pb.Hv * pb.NT * 8192);
     c.bytes = off;
     return c;
@@ -109,8 +110,9 @@ cudaError_t tc_chunk_bwd(const Problem& pb, const ChunkIO& io, Flags f, bool bf1
     CUtensorMap m[10];
     bool ok = make_map(&m[0], io.q, pb.B, pb.T, pb.Hk) && make_map(&m[1], io.k, pb.B, pb.T, pb.Hk) &&
               make_map(&m[4], io.dout, pb.B, pb.T, pb.Hv) && make_map(&m[5], nyh, pb.B, pb.T, pb.Hv) &&
-              make_map(&m[6], nyl, pb.B, pb.T, pb.Hv) && make_map(&m[7], vph, pb.B, pb.T, pb.Hv) &&
-              make_map(&m[8], vpl, pb.B, pb.T, pb.Hv);
+              make_map(&m[6], nyl, pb.B, pb.T, pb.Hv) &&
+              make_chunk_map(&m[7], vph, (long)pb.B * pb.Hv * pb.NT) &&
+              make_chunk_map(&m[8], vpl, (long)pb.B * pb.Hv * pb.NT);
     m[2] = m[4];
     m[3] = m[4];
     if (ok && f.apc) ok = make_map(&m[2], io.alpha, pb.B, pb.T, pb.Hv);

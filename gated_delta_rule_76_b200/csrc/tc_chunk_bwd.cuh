@@ -72,6 +72,7 @@ using tcfwd::split8;
 using tcfwd::split_pack;
 using tcfwd::st16;
 using tcfwd::l2_evict_last_policy;
+using tcfwd::tma3;
 using tcfwd::tma4;
 using tcfwd::tma4_pol;
 using tcfwd::unpack8;
@@ -731,7 +732,7 @@ constexpr uint32_t SM_RA = 49152;     // 16 KB [2][64]: TMA alpha -> Ktil lo
 constexpr uint32_t SM_EQ = 65536;     // 32 KB [2][128]: [Ehat;Qhat] hi
 constexpr uint32_t SM_GH = 98304;     // 32 KB [2][128]: dO (rows 0-63), -dY hi (rows 64-127)
 constexpr uint32_t SM_GL = 131072;    // 32 KB [2][128]: zeros (rows 0-63), -dY lo (rows 64-127)
-constexpr uint32_t SM_VP = 163840;    // 32 KB: V' hi [2][64], V' lo [2][64]
+constexpr uint32_t SM_VP = 163840;    // 32 KB: V' hi [128 channel rows][64 tokens], V' lo (MN-major operands)
 constexpr uint32_t SM_DPA = 196608;   // 32 KB: [dP;dA] hi [1][128], lo [1][128]
 constexpr uint32_t SM_BAR = 229376;   // mbarriers, tensor memory base, flags
 constexpr uint32_t SM_XSLOT = SM_BAR + 256;   // [128] rowsum(dS_end .* S0) of the staged chunk
@@ -851,10 +852,9 @@ __device__ __forceinline__ void load_gv(const Ctx& cx, const ChunkPos& cp, const
     tma4(base + SM_GH + 16384 + 8192, m.yh, bar, 64, cp.hv, cp.t0, cp.b);
     tma4(base + SM_GL + 8192, m.yl, bar, 0, cp.hv, cp.t0, cp.b);
     tma4(base + SM_GL + 16384 + 8192, m.yl, bar, 64, cp.hv, cp.t0, cp.b);
-    tma4(base + SM_VP, m.vh, bar, 0, cp.hv, cp.t0, cp.b);
-    tma4(base + SM_VP + 8192, m.vh, bar, 64, cp.hv, cp.t0, cp.b);
-    tma4(base + SM_VP + 16384, m.vl, bar, 0, cp.hv, cp.t0, cp.b);
-    tma4(base + SM_VP + 16384 + 8192, m.vl, bar, 64, cp.hv, cp.t0, cp.b);
+    // V' hi, lo: the chunk's column-major tiles (128 channel rows of its 64 tokens)
+    tma3(base + SM_VP, m.vh, bar, 0, 0, (int)cp.ci);
+    tma3(base + SM_VP + 16384, m.vl, bar, 0, 0, (int)cp.ci);
 }
 
 // The walked chunk's q, k (and alpha, b with channel gates, or q lo, k lo with split inputs) tiles
@@ -1406,10 +1406,19 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // ---- P6 = G V'^T --------------------------------------------------------------------------
         if (tid == 0) {
             if (wait1(cx, B_GV, par) && !*cx.abort_flag) {
-                const uint32_t id64 = idesc_bf16_f32(128, 64);
-                mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP, id64, false);
-                mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GL, sbase + SM_VP, id64, true);
-                mma_ss_u<128, 128, 64>(tbase + TM_P6, sbase + SM_GH, sbase + SM_VP + 16384, id64, true);
+                // G K-major (two 64-channel atoms of 128 rows); V' MN-major (its tile holds a
+                // channel per 128-byte row of 64 tokens, so K = channels steps 16 rows)
+                const uint32_t id_v = idesc_bf16_f32_mn(128, 64, false, true);
+                const uint64_t gh = sdesc_k_sw128(sbase + SM_GH), gl = sdesc_k_sw128(sbase + SM_GL);
+#pragma unroll
+                for (int k = 0; k < 128; k += 16) {
+                    const uint32_t ao = ((uint32_t)(k >> 6) * 128u * 128u + (uint32_t)(k & 63) * 2u) >> 4;
+                    const uint64_t vh = sdesc_mn_sw128(sbase + SM_VP + (uint32_t)k * 128u, 8192u);
+                    const uint64_t vl = sdesc_mn_sw128(sbase + SM_VP + 16384u + (uint32_t)k * 128u, 8192u);
+                    mma_ss(tbase + TM_P6, gh + ao, vh, id_v, k > 0 ? 1u : 0u);
+                    mma_ss(tbase + TM_P6, gl + ao, vh, id_v, 1u);
+                    mma_ss(tbase + TM_P6, gh + ao, vl, id_v, 1u);
+                }
                 mma_commit(cx.bars + B_P6);
                 wait1(cx, B_P6, par);
             }
@@ -1447,7 +1456,7 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // ---- P7 = S0 G^T + Ktil^T [dP;dA]^T,  P8 = [Qhat^T|Ehat^T] [dP;dA],  P9 = dS V'^T ----------
         if (tid == 0) GDN_BTRACE(it, 2);
         if (tid == 0 && !*cx.abort_flag) {
-            const uint32_t id64 = idesc_bf16_f32(128, 64), id128 = idesc_bf16_f32(128, 128);
+            const uint32_t id128 = idesc_bf16_f32(128, 128);
             mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0H, sbase + SM_GH, id128, false);
             mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0L, sbase + SM_GH, id128, true);
             mma_ts_u<128, 128>(tbase + TM_P7, tbase + TM_S0H, sbase + SM_GL, id128, true);
@@ -1475,9 +1484,17 @@ chunk_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 mma_ss(tbase + TM_P6, al, bh_, id_k8, 1u);
                 mma_ss(tbase + TM_P6, ah, bl_, id_k8, 1u);
             }
-            mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSH, sbase + SM_VP, id64, false);
-            mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSL, sbase + SM_VP, id64, true);
-            mma_ts_u<128, 64>(tbase + TM_P9, tbase + TM_DSH, sbase + SM_VP + 16384, id64, true);
+            {
+                const uint32_t id_v = idesc_bf16_f32_mn(128, 64, false, true);
+#pragma unroll
+                for (int k = 0; k < 128; k += 16) {
+                    const uint64_t vh = sdesc_mn_sw128(sbase + SM_VP + (uint32_t)k * 128u, 8192u);
+                    const uint64_t vl = sdesc_mn_sw128(sbase + SM_VP + 16384u + (uint32_t)k * 128u, 8192u);
+                    mma_ts(tbase + TM_P9, tbase + TM_DSH + (uint32_t)(k >> 1), vh, id_v, k > 0 ? 1u : 0u);
+                    mma_ts(tbase + TM_P9, tbase + TM_DSL + (uint32_t)(k >> 1), vh, id_v, 1u);
+                    mma_ts(tbase + TM_P9, tbase + TM_DSH + (uint32_t)(k >> 1), vl, id_v, 1u);
+                }
+            }
             mma_commit(cx.bars + B_P789);
             if (wait1(cx, B_P789, par) && !*cx.abort_flag) {
                 // the [dP; dA] and V' tiles are free: the walk's rows of this chunk

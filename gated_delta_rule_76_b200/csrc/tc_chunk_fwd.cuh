@@ -139,8 +139,8 @@ struct Params {
     // Backward support (all NULL in a plain forward).  o may be NULL then: no output is formed.
     float* s0_out;               // [B*Hv][NT + 1][dv/4][dk][4] fp32: the state entering every chunk, then
                                  //   the final state
-    __nv_bfloat16* vp_hi;        // [B,T,Hv,dv]: V' = T (Z - Ehat S0) of every token, split
-    __nv_bfloat16* vp_lo;        //   into hi = bf16(V') and lo = bf16(V' - hi)
+    __nv_bfloat16* vp_hi;        // [B*Hv][NT][dv][64]: V' = T (Z - Ehat S0) of every chunk, column-major
+    __nv_bfloat16* vp_lo;        //   (a column's 64 tokens contiguous), as hi = bf16(V'), lo = bf16(V' - hi)
     float* o_raw;                // GATE only, may be NULL: the output before the gate, fp32 [B,T,Hv,dv]
     uint8_t* t_out;              // [B*Hv][NT][8 KB] or NULL: the image of every chunk's bf16 T hi tile
                                  //   (64 rows of 128 swizzled bytes), read back by the reverse scan
@@ -234,6 +234,15 @@ __device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint6
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// A 3-D tile (the backward cache's chunk-major tiles).
+__device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 
@@ -559,22 +568,23 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             if (p.vp_hi) {
-                // V' (saving mode), stored while X4 / X5 run: rows 32h .. 32h + 31 of column j,
-                // token-major (coalesced over j)
-                const long vrow = (long)pb.Hv * D;
-                const long vb = pb.v_row(b, t0 + 32 * h, hv) + j;
-                const int nrow = min(32, L - 32 * h);
+                // V' (saving mode), stored while X4 / X5 run: rows 32h .. 32h + 31 of column j are
+                // 64 contiguous bytes of the chunk-major tile (rows past the sequence as zeros)
+                const long vo = (((long)blockIdx.x * NT + n) * D + j) * 64 + 32 * h;
+                uint32_t vh[16], vl[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int r0 = 2 * i;
-                    if (r0 < nrow) {
-                        p.vp_hi[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(vhi[i] & 0xFFFFu));
-                        p.vp_lo[vb + r0 * vrow] = __ushort_as_bfloat16((unsigned short)(vlo[i] & 0xFFFFu));
-                    }
-                    if (r0 + 1 < nrow) {
-                        p.vp_hi[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(vhi[i] >> 16));
-                        p.vp_lo[vb + (r0 + 1) * vrow] = __ushort_as_bfloat16((unsigned short)(vlo[i] >> 16));
-                    }
+                    const int r0 = 32 * h + 2 * i;
+                    const uint32_t keep = (r0 < L ? 0x0000FFFFu : 0u) | (r0 + 1 < L ? 0xFFFF0000u : 0u);
+                    vh[i] = vhi[i] & keep;
+                    vl[i] = vlo[i] & keep;
+                }
+                uint4* dh = reinterpret_cast<uint4*>(p.vp_hi + vo);
+                uint4* dl = reinterpret_cast<uint4*>(p.vp_lo + vo);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    dh[q4] = make_uint4(vh[4 * q4], vh[4 * q4 + 1], vh[4 * q4 + 2], vh[4 * q4 + 3]);
+                    dl[q4] = make_uint4(vl[4 * q4], vl[4 * q4 + 1], vl[4 * q4 + 2], vl[4 * q4 + 3]);
                 }
             }
             if (tid == 0) {

@@ -36,4 +36,18 @@ inline bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The backward cache's chunk-major tiles, [chunks][128 channels][64 tokens] bf16: one box is a
+// whole chunk's tile (128 rows of 64 tokens), 128-byte swizzle.
+inline bool make_chunk_map(CUtensorMap* m, const void* base, long chunks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || !base || chunks < 1) return false;
+    const cuuint64_t dims[3] = {64, 128, (cuuint64_t)chunks};
+    const cuuint64_t strides[2] = {128, 128 * 128};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace gdn
