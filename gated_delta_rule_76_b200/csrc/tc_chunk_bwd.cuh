@@ -70,6 +70,7 @@ using tcfwd::ld16;
 using tcfwd::ldf4;
 using tcfwd::split8;
 using tcfwd::split_pack;
+using tcfwd::store_state_block;
 using tcfwd::st16;
 using tcfwd::l2_evict_last_policy;
 using tcfwd::tma3;
@@ -395,12 +396,8 @@ chunk_bwd_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 wait1(cx, B_XC, pi);
                 GDN_STRACE(i, 5);
             }
-            if (p.dsc) {
-                // dS_end of chunk n, rows 64h .. 64h + 63 of column j, layout [j / 4][row][j % 4]
-                float* dst = p.dsc + ((long)blockIdx.x * NT + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
-#pragma unroll
-                for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
-            }
+            if (p.dsc)  // dS_end of chunk n, in the layout of the forward's chunk states
+                store_state_block(p.dsc + ((long)blockIdx.x * NT + n) * (D * D), S, j, h);
             named_bar(1, 256);
             tc_fence_after();
             // ---- dS <- Diag(gamma) dS + XC^T; split for the next chunk ----------------------------

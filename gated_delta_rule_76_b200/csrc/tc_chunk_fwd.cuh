@@ -237,6 +237,30 @@ __device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint6
         : "memory");
 }
 
+// Rows 64h .. 64h + 63 of state column j (thread j holds them in S) into one dk x dv block in the
+// layout [j / 4][row][j % 4] (float4 (j / 4) * D + row holds columns 4 (j / 4) .. + 3 of a row, so
+// a reader holding one row per thread loads it as float4s).  The four lanes of a column quad
+// transpose each 4 x 4 block in two butterfly steps, so that every lane stores whole float4s (16
+// 16-byte stores instead of 64 4-byte ones).  All 32 lanes of the warp take part.
+__device__ __forceinline__ void store_state_block(float* blk, const float (&S)[64], int j, int h) {
+    const int e = j & 3;
+    const bool b0 = (e & 1) != 0, b1 = (e & 2) != 0;
+    float4* dst = reinterpret_cast<float4*>(blk) + (j >> 2) * D + 64 * h + e;
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 4) {
+        float v0 = S[c0], v1 = S[c0 + 1], v2 = S[c0 + 2], v3 = S[c0 + 3];
+        float s0 = b0 ? v0 : v1, s1 = b0 ? v2 : v3;
+        float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+        if (b0) { v0 = r0; v2 = r1; } else { v1 = r0; v3 = r1; }
+        s0 = b1 ? v0 : v2;
+        s1 = b1 ? v1 : v3;
+        r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
+        r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+        if (b1) { v0 = r0; v1 = r1; } else { v2 = r0; v3 = r1; }
+        dst[c0] = make_float4(v0, v1, v2, v3);  // row 64h + c0 + e, columns 4 (j / 4) .. + 3
+    }
+}
+
 // A 3-D tile (the backward cache's chunk-major tiles).
 __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
     asm volatile(
@@ -426,7 +450,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (p.s0_out) {
                 // state entering chunk n (saving mode), stored while X2 runs: rows 64h .. 64h + 63
                 // of column j, in the layout [j / 4][row][j % 4] (a reader holding one row per
-                // thread loads it as float4s)
+                // thread loads it as float4s).  Plain 4-byte stores: the quad transpose of
+                // store_state_block, which the reverse scan uses, made this chain slower.
                 float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
 #pragma unroll
                 for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
@@ -691,12 +716,8 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int c = 0; c < 64; ++c) p.ht[soff + (long)(64 * h + c) * D + j] = S[c];
         }
-        if (p.s0_out && !*cx.abort_flag) {
-            // the final state follows the last chunk's entering state
-            float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + NT) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
-#pragma unroll
-            for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
-        }
+        if (p.s0_out && !*cx.abort_flag)  // the final state follows the last chunk's entering state
+            store_state_block(p.s0_out + ((long)blockIdx.x * (NT + 1) + NT) * (D * D), S, j, h);
     } else {
         // =================================== chunk prologue ===================================
         const int c = tid - 256;  // key channel; also TMEM lane of X1
