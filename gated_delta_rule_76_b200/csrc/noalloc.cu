@@ -53,3 +53,10 @@ extern "C" GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* a, gdn_s
     if ((s = scratch_of_current_device(&ws))) return s;
     return gdn_chunk_fwd(a, ws, kScratchBytes, stream);
 }
+
+extern "C" GDN_API gdn_status gdn_chunk_fwd_noalloc_status(gdn_stream stream) {
+    void* ws = nullptr;
+    gdn_status s = scratch_of_current_device(&ws);
+    if (s) return s;
+    return gdn_workspace_status(ws, stream);
+}

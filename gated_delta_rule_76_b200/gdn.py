@@ -78,7 +78,8 @@ class LayerBwdArgs(ctypes.Structure):
                 ("alpha_scale", P), ("grad_alpha_scale", P)]
 
 
-EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc", "gdn_chunk_bwd_workspace_size",
+EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc",
+            "gdn_chunk_fwd_noalloc_status", "gdn_chunk_bwd_workspace_size",
             "gdn_chunk_bwd", "gdn_decode_step", "gdn_layer_core_fwd_cache_size", "gdn_layer_core_fwd_workspace_size",
             "gdn_layer_core_fwd", "gdn_layer_core_bwd_workspace_size", "gdn_layer_core_bwd",
             "gdn_segment_map_workspace_size", "gdn_segment_map", "gdn_state_compose",
@@ -107,6 +108,8 @@ def load(path: str = LIB_PATH):
     lib.gdn_chunk_fwd.restype = ctypes.c_int
     lib.gdn_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(FwdArgs), P]
     lib.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.gdn_chunk_fwd_noalloc_status.argtypes = [P]
+    lib.gdn_chunk_fwd_noalloc_status.restype = ctypes.c_int
     lib.gdn_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
     lib.gdn_chunk_bwd_workspace_size.restype = ctypes.c_size_t
     lib.gdn_chunk_bwd.argtypes = [ctypes.POINTER(BwdArgs), P, ctypes.c_size_t, P]
@@ -284,6 +287,12 @@ def gdn_chunk_fwd_noalloc(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=
     a, keep = fwd_args(q, k, v, alpha, b, w, beta, h0, z, head_map, scale, o, ht)
     check(lib.gdn_chunk_fwd_noalloc(ctypes.byref(a), _stream(stream)), "gdn_chunk_fwd_noalloc")
     return o, ht
+
+
+def gdn_chunk_fwd_noalloc_status(stream=None) -> int:
+    """The status word of the built-in scratch after gdn_chunk_fwd_noalloc calls (synchronises
+    ``stream``): 0, or GDN_ERR_TIMEOUT (5) if a bounded wait inside a kernel expired."""
+    return int(load().gdn_chunk_fwd_noalloc_status(_stream(stream)))
 
 
 def gdn_segment_map(q, k, v, alpha, b=None, w=None, beta=None, head_map=None, *, want_o: bool = False,

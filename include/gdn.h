@@ -145,12 +145,17 @@ GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size
  *    lookups are host-side; each call then launches work on `stream` only.
  *  - Nothing is allocated (no cudaMalloc, no host or device allocation by any library).  The
  *    status word at the start of the scratch is cleared on `stream` at the start of every call;
- *    nothing else in the scratch needs to start at zero.  The status word is not readable by the
- *    caller: an expired bounded wait inside a kernel is not reported by this call.
+ *    nothing else in the scratch needs to start at zero.  An expired bounded wait inside a kernel
+ *    is not reported by this call (it returns before the kernels run); gdn_chunk_fwd_noalloc_status
+ *    reads the status word afterwards.
  *  - Concurrency: every call on a device uses the same scratch array.  Calls whose execution can
  *    overlap (different streams, or different host threads without ordering) race on it; the
  *    caller must order them, e.g. by issuing them all on one stream. */
 GDN_API gdn_status gdn_chunk_fwd_noalloc(const gdn_fwd_args* args, gdn_stream stream);
+/* The status word of the current device's scratch, as gdn_workspace_status reads a workspace's:
+ * synchronises `stream`, then GDN_OK, or GDN_ERR_TIMEOUT if a bounded wait of the last
+ * gdn_chunk_fwd_noalloc call on this device expired. */
+GDN_API gdn_status gdn_chunk_fwd_noalloc_status(gdn_stream stream);
 
 /* ------------------------------------------------------------------------------------------
  * Chunkwise backward.  Reverse mode of gdn_chunk_fwd (without z): the chunk-boundary states are

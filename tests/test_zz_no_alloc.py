@@ -49,6 +49,8 @@ def test_noalloc_matches_workspace_call_twice(case):
         assert rel_error(ht, ht_ref, case["prec"]) <= tol, f"ht, call {call + 1}"
         # The same kernels on the same inputs, only the scratch differs: the bits agree too.
         assert torch.equal(o, o_ref) and torch.equal(ht, ht_ref), f"bits differ, call {call + 1}"
+        # no bounded wait expired: the scratch's status word reads OK
+        assert gdn.gdn_chunk_fwd_noalloc_status() == 0, f"status, call {call + 1}"
 
 
 def test_noalloc_rejects_a_problem_larger_than_its_scratch():
