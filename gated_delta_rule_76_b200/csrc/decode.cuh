@@ -19,6 +19,8 @@ struct DecodeParams {
     int o_f32;  // o written in fp32 instead of TIn
     const int32_t* head_map;
     const void* conv_state; const void* conv_w; const void* z;
+    // elements from one sequence's token to the next (Hk*dk, Hv*dv, ... when dense)
+    long sq, sk, sv, sa, sb, sw, sz;
     int N, Hk, Hv, dk, dv;
     float scale;
     int gate_logits;           // gates as logits: alpha = exp(-alpha_scale[hv] softplus(x)), sigmoid b, w
@@ -41,12 +43,12 @@ decode_step_kernel(DecodeParams p) {
     const int hv = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
     // a map entry outside [0, Hk) breaks the precondition: clamped, so no read leaves q or k
     const int hk = p.head_map ? min(max(__ldg(p.head_map + hv), 0), p.Hk - 1) : hv / (p.Hv / p.Hk);
-    const TIn* q = static_cast<const TIn*>(p.q) + ((long)n * p.Hk + hk) * DK;
-    const TIn* k = static_cast<const TIn*>(p.k) + ((long)n * p.Hk + hk) * DK;
-    const TIn* v = static_cast<const TIn*>(p.v) + ((long)n * p.Hv + hv) * DV;
-    const TG* al = static_cast<const TG*>(p.alpha) + ((long)n * p.Hv + hv) * (APC ? DK : 1);
-    const TG* bg = static_cast<const TG*>(p.b) + ((long)n * p.Hv + hv) * (GPC ? DK : 1);
-    const TG* wg = GPC ? static_cast<const TG*>(p.w) + ((long)n * p.Hv + hv) * DV : bg;
+    const TIn* q = static_cast<const TIn*>(p.q) + n * p.sq + hk * DK;
+    const TIn* k = static_cast<const TIn*>(p.k) + n * p.sk + hk * DK;
+    const TIn* v = static_cast<const TIn*>(p.v) + n * p.sv + hv * DV;
+    const TG* al = static_cast<const TG*>(p.alpha) + n * p.sa + hv * (APC ? DK : 1);
+    const TG* bg = static_cast<const TG*>(p.b) + n * p.sb + hv * (GPC ? DK : 1);
+    const TG* wg = GPC ? static_cast<const TG*>(p.w) + n * p.sw + hv * DV : bg;
 
     // ---- gates: every load issued first, then (gates as logits) the transforms under one branch,
     // so that no load waits for another (a branch on a loaded value waits for the load) -----
@@ -172,7 +174,7 @@ decode_step_kernel(DecodeParams p) {
         float ov[4] = {acc.x * p.scale, acc.y * p.scale, acc.z * p.scale, acc.w * p.scale};
         TIn* o = static_cast<TIn*>(p.o) + ((long)n * p.Hv + hv) * DV + 4 * cq;
         if (GATE) {
-            const TIn* zg = static_cast<const TIn*>(p.z) + ((long)n * p.Hv + hv) * DV + 4 * cq;
+            const TIn* zg = static_cast<const TIn*>(p.z) + n * p.sz + hv * DV + 4 * cq;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const float zz = to_f32(zg[c]);
@@ -192,16 +194,17 @@ decode_step_kernel(DecodeParams p) {
 // After the decode kernel: shift every channel's stored inputs and append the new raw input.
 template <class TIn>
 __global__ void conv_state_shift_kernel(void* conv_state, const void* q, const void* k,
-                                        const void* v, int N, int Hk, int Hv, int dk, int dv) {
+                                        const void* v, long sq, long sk, long sv, int N, int Hk, int Hv, int dk,
+                                        int dv) {
     const long cch = 2L * Hk * dk + (long)Hv * dv;
     const long total = (long)N * cch;
     for (long idx = blockIdx.x * (long)blockDim.x + threadIdx.x; idx < total;
          idx += (long)gridDim.x * blockDim.x) {
         const long n = idx / cch, ch = idx % cch;
         TIn x;
-        if (ch < (long)Hk * dk) x = static_cast<const TIn*>(q)[n * Hk * dk + ch];
-        else if (ch < 2L * Hk * dk) x = static_cast<const TIn*>(k)[n * Hk * dk + ch - (long)Hk * dk];
-        else x = static_cast<const TIn*>(v)[n * Hv * dv + ch - 2L * Hk * dk];
+        if (ch < (long)Hk * dk) x = static_cast<const TIn*>(q)[n * sq + ch];
+        else if (ch < 2L * Hk * dk) x = static_cast<const TIn*>(k)[n * sk + ch - (long)Hk * dk];
+        else x = static_cast<const TIn*>(v)[n * sv + ch - 2L * Hk * dk];
         TIn* cs = static_cast<TIn*>(conv_state) + idx * 3;
         cs[0] = cs[1];
         cs[1] = cs[2];

@@ -43,6 +43,7 @@ struct Buf {
     const void* p;
     size_t bytes;
     const char* name;
+    size_t align = 16;  // required alignment of p (a strided input: its element size)
 };
 
 bool overlaps(const Buf& a, const Buf& b) {
@@ -54,8 +55,8 @@ bool overlaps(const Buf& a, const Buf& b) {
 // Every output against every input and every other output.
 gdn_status check_buffers(const Buf* in, int nin, const Buf* out, int nout) {
     for (int i = 0; i < nin; ++i)
-        if (in[i].p && !aligned16(in[i].p))
-            return fail(GDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", in[i].name);
+        if (in[i].p && (reinterpret_cast<uintptr_t>(in[i].p) & (in[i].align - 1)))
+            return fail(GDN_ERR_INVALID_ARG, "%s is not %zu-byte aligned", in[i].name, in[i].align);
     for (int i = 0; i < nout; ++i) {
         if (out[i].p && !aligned16(out[i].p))
             return fail(GDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", out[i].name);
@@ -104,6 +105,54 @@ Problem make_problem(int64_t B, int64_t T, int64_t Hk, int64_t Hv, int64_t dk, i
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---- token strides (gdn_strides) ---------------------------------------------------------
+// A token-major input of `rows` tokens of `row` elements whose tokens are `stride` elements apart
+// (0: dense).  One that is not dense is copied into the workspace before the call's kernels run.
+bool strided(int64_t stride, int64_t row) { return stride != 0 && stride != row; }
+
+// The input as a buffer: from its first to its last element; a strided one needs only the
+// alignment of its element type.
+Buf tok(const void* p, size_t rows, int64_t row, int64_t stride, size_t es, const char* name) {
+    const size_t step = (size_t)(stride ? stride : row);
+    return Buf{p, p && rows ? ((rows - 1) * step + (size_t)row) * es : 0, name, strided(stride, row) ? es : 16};
+}
+
+gdn_status check_stride(int64_t stride, int64_t row, const char* name) {
+    if (stride != 0 && (stride < row || stride > (int64_t(1) << 31)))
+        return fail(GDN_ERR_INVALID_ARG, "token stride of %s is %lld: it must be 0 or in [%lld, 2^31]", name,
+                    (long long)stride, (long long)row);
+    return GDN_OK;
+}
+
+// One input of a call, for the copies: where the call reads its pointer, its row and stride.
+struct StridedIn {
+    const void** slot;
+    int64_t row, stride;
+    size_t es;
+};
+
+// Bytes of the dense copies of the strided inputs (each 256-byte aligned).
+size_t pack_bytes(const StridedIn* in, int n, size_t rows) {
+    size_t bytes = 0;
+    for (int i = 0; i < n; ++i)
+        if (*in[i].slot && strided(in[i].stride, in[i].row)) bytes += align256(rows * (size_t)in[i].row * in[i].es);
+    return bytes;
+}
+
+// Copies every strided input into `dst` (the workspace past the call's own part) and points its
+// slot at the copy.
+cudaError_t pack_inputs(const StridedIn* in, int n, size_t rows, char* dst, cudaStream_t st) {
+    for (int i = 0; i < n; ++i) {
+        if (!*in[i].slot || !strided(in[i].stride, in[i].row)) continue;
+        const long row_bytes = (long)(in[i].row * (int64_t)in[i].es);
+        cudaError_t e = pack_rows(*in[i].slot, dst, (long)rows, row_bytes, (long)(in[i].stride * (int64_t)in[i].es), st);
+        if (e != cudaSuccess) return e;
+        *in[i].slot = dst;
+        dst += align256(rows * (size_t)row_bytes);
+    }
+    return cudaSuccess;
+}
 
 // Gates as logits: the flag and alpha's per-head scale (grad: the scale's gradient, optional).
 gdn_status check_logits(int32_t gate_logits, const float* alpha_scale, const float* grad_alpha_scale = nullptr) {
@@ -195,15 +244,22 @@ gdn_status check_fwd(const gdn_fwd_args* a, bool need_o = true) {
         return fail(GDN_ERR_INVALID_ARG, "w must be NULL for scalar gates (b holds beta)");
     const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype);
     const size_t BT = (size_t)(a->B * a->T);
+    const gdn_strides& sd = a->strides;
+    const int64_t ra = a->Hv * (a->alpha_per_channel ? a->dk : 1), rb = a->Hv * (a->gates_per_channel ? a->dk : 1);
+    if ((s = check_stride(sd.q, a->Hk * a->dk, "q")) || (s = check_stride(sd.k, a->Hk * a->dk, "k")) ||
+        (s = check_stride(sd.v, a->Hv * a->dv, "v")) || (s = check_stride(sd.alpha, ra, "alpha")) ||
+        (s = check_stride(sd.b, rb, "b")) || (s = check_stride(sd.w, a->Hv * a->dv, "w")) ||
+        (s = check_stride(sd.z, a->Hv * a->dv, "z")))
+        return s;
     const Buf in[] = {
-        {a->q, BT * a->Hk * a->dk * es, "q"},
-        {a->k, BT * a->Hk * a->dk * es, "k"},
-        {a->v, BT * a->Hv * a->dv * es, "v"},
-        {a->alpha, BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
-        {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
-        {a->w, BT * a->Hv * a->dv * gs, "w"},
+        tok(a->q, BT, a->Hk * a->dk, sd.q, es, "q"),
+        tok(a->k, BT, a->Hk * a->dk, sd.k, es, "k"),
+        tok(a->v, BT, a->Hv * a->dv, sd.v, es, "v"),
+        tok(a->alpha, BT, ra, sd.alpha, gs, "alpha"),
+        tok(a->b, BT, rb, sd.b, gs, "b"),
+        tok(a->w, BT, a->Hv * a->dv, sd.w, gs, "w"),
         {a->h0, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "h0"},
-        {a->z, BT * a->Hv * a->dv * es, "z"},
+        tok(a->z, BT, a->Hv * a->dv, sd.z, es, "z"),
         {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->alpha_scale, (size_t)a->Hv * 4, "alpha_scale"},
     };
@@ -236,10 +292,18 @@ gdn_status check_bwd(const gdn_bwd_args* a) {
     const size_t st = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
     const size_t na = BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs;
     const size_t nb = BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs;
+    const gdn_strides& sd = a->strides;
+    const int64_t ra = a->Hv * (a->alpha_per_channel ? a->dk : 1), rb = a->Hv * (a->gates_per_channel ? a->dk : 1);
+    if ((s = check_stride(sd.q, a->Hk * a->dk, "q")) || (s = check_stride(sd.k, a->Hk * a->dk, "k")) ||
+        (s = check_stride(sd.v, a->Hv * a->dv, "v")) || (s = check_stride(sd.alpha, ra, "alpha")) ||
+        (s = check_stride(sd.b, rb, "b")) || (s = check_stride(sd.w, a->Hv * a->dv, "w")))
+        return s;
+    if (sd.z != 0) return fail(GDN_ERR_INVALID_ARG, "strides.z must be 0: the backward takes no z");
     const Buf in[] = {
-        {a->q, BT * a->Hk * a->dk * es, "q"}, {a->k, BT * a->Hk * a->dk * es, "k"},
-        {a->v, BT * a->Hv * a->dv * es, "v"}, {a->alpha, na, "alpha"}, {a->b, nb, "b"},
-        {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        tok(a->q, BT, a->Hk * a->dk, sd.q, es, "q"), tok(a->k, BT, a->Hk * a->dk, sd.k, es, "k"),
+        tok(a->v, BT, a->Hv * a->dv, sd.v, es, "v"), tok(a->alpha, BT, ra, sd.alpha, gs, "alpha"),
+        tok(a->b, BT, rb, sd.b, gs, "b"), tok(a->w, BT, a->Hv * a->dv, sd.w, gs, "w"), {a->h0, st, "h0"},
+        {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_o, BT * a->Hv * a->dv * es, "grad_o"}, {a->grad_ht, st, "grad_ht"},
         {a->fwd_cache, a->fwd_cache ? a->fwd_cache_bytes : 0, "fwd_cache"},
         {a->alpha_scale, (size_t)a->Hv * 4, "alpha_scale"},
@@ -275,6 +339,70 @@ ChunkIO io_from(const gdn_fwd_args* a) {
     io.z = a->z; io.h0 = a->h0; io.o = a->o; io.ht = a->ht; io.o_type = a->out_f32 ? 1 : 0;
     io.z_bf16 = 0;
     return io;
+}
+
+// The token-major inputs of a forward, a backward and a layer call, for the copies of the strided
+// ones; `p` is the call's own copy of its arguments, whose pointers the copies replace.
+int fwd_inputs(gdn_fwd_args* p, StridedIn* in) {
+    const size_t es = elem_size(p->dtype), gs = elem_size(p->gate_dtype);
+    const int64_t ra = p->Hv * (p->alpha_per_channel ? p->dk : 1), rb = p->Hv * (p->gates_per_channel ? p->dk : 1);
+    in[0] = {&p->q, p->Hk * p->dk, p->strides.q, es};
+    in[1] = {&p->k, p->Hk * p->dk, p->strides.k, es};
+    in[2] = {&p->v, p->Hv * p->dv, p->strides.v, es};
+    in[3] = {&p->alpha, ra, p->strides.alpha, gs};
+    in[4] = {&p->b, rb, p->strides.b, gs};
+    in[5] = {&p->w, p->Hv * p->dv, p->strides.w, gs};
+    in[6] = {&p->z, p->Hv * p->dv, p->strides.z, es};
+    return 7;
+}
+int bwd_inputs(gdn_bwd_args* p, StridedIn* in) {
+    const size_t es = elem_size(p->dtype), gs = elem_size(p->gate_dtype);
+    const int64_t ra = p->Hv * (p->alpha_per_channel ? p->dk : 1), rb = p->Hv * (p->gates_per_channel ? p->dk : 1);
+    in[0] = {&p->q, p->Hk * p->dk, p->strides.q, es};
+    in[1] = {&p->k, p->Hk * p->dk, p->strides.k, es};
+    in[2] = {&p->v, p->Hv * p->dv, p->strides.v, es};
+    in[3] = {&p->alpha, ra, p->strides.alpha, gs};
+    in[4] = {&p->b, rb, p->strides.b, gs};
+    in[5] = {&p->w, p->Hv * p->dv, p->strides.w, gs};
+    return 6;
+}
+template <class LA>
+int layer_inputs(LA* p, StridedIn* in) {
+    const size_t es = elem_size(p->dtype), gs = elem_size(p->gate_dtype);
+    const int64_t ra = p->Hv * (p->alpha_per_channel ? p->dk : 1), rb = p->Hv * (p->gates_per_channel ? p->dk : 1);
+    in[0] = {&p->xq, p->Hk * p->dk, p->strides.q, es};
+    in[1] = {&p->xk, p->Hk * p->dk, p->strides.k, es};
+    in[2] = {&p->xv, p->Hv * p->dv, p->strides.v, es};
+    in[3] = {&p->alpha, ra, p->strides.alpha, gs};
+    in[4] = {&p->b, rb, p->strides.b, gs};
+    in[5] = {&p->w, p->Hv * p->dv, p->strides.w, gs};
+    in[6] = {&p->z, p->Hv * p->dv, p->strides.z, es};
+    return 7;
+}
+template <class A, int (*LIST)(A*, StridedIn*)>
+size_t args_pack_bytes(const A* a) {
+    A p = *a;
+    StridedIn in[7];
+    const int n = LIST(&p, in);
+    return pack_bytes(in, n, (size_t)(a->B * a->T));
+}
+// Workspace of a call's own part plus the copies of its strided inputs after it.
+size_t with_copies(size_t own, size_t copies) { return copies ? align256(own) + copies : own; }
+
+// Validates the workspace for a call's own part and its copies, then copies the strided inputs
+// of *a past its own part and points *a (the call's copy of its arguments) at them.
+template <class A>
+gdn_status copy_strided(A* p, int (*list)(A*, StridedIn*), void* ws, size_t ws_bytes, size_t own, cudaStream_t st,
+                        const char* who) {
+    StridedIn in[7];
+    const int n = list(p, in);
+    const size_t rows = (size_t)(p->B * p->T), copies = pack_bytes(in, n, rows);
+    gdn_status s = check_workspace(ws, ws_bytes, with_copies(own, copies));
+    if (s || !copies) return s;
+    cudaError_t e = pack_inputs(in, n, rows, static_cast<char*>(ws) + align256(own), st);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+    p->strides = gdn_strides{};
+    return GDN_OK;
 }
 
 // Status word at the start of every workspace, cleared at the start of each call.
@@ -328,11 +456,16 @@ size_t gdn_chunk_fwd_cache_size(const gdn_fwd_args* a) {
     return fwd_uses_tensor_cores(a, pb) ? plan_tc_cache(pb).bytes : 0;
 }
 
-size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
-    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+// The forward's own workspace (without the copies of strided inputs).
+static size_t fwd_own_ws(const gdn_fwd_args* a) {
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     if (fwd_uses_tensor_cores(a, pb)) return tc_fwd_ws_bytes(pb);
     return plan_chunk_ws(pb, false, false).bytes;
+}
+
+size_t gdn_chunk_fwd_workspace_size(const gdn_fwd_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    return with_copies(fwd_own_ws(a), args_pack_bytes<gdn_fwd_args, fwd_inputs>(a));
 }
 
 }  // extern "C"
@@ -356,7 +489,12 @@ static gdn_status chunk_fwd_core(const gdn_fwd_args* a, void* workspace, size_t 
                         plan_tc_cache(pb).bytes);
     }
     WsPlan plan = plan_chunk_ws(pb, false, false);
-    if ((s = check_workspace(workspace, workspace_bytes, tc ? tc_fwd_ws_bytes(pb) : plan.bytes))) return s;
+    // the workspace, then the dense copies of strided inputs, which the rest reads instead
+    gdn_fwd_args pa = *a;
+    if ((s = copy_strided(&pa, fwd_inputs, workspace, workspace_bytes, tc ? tc_fwd_ws_bytes(pb) : plan.bytes, st,
+                          "gdn_chunk_fwd (strided inputs)")))
+        return s;
+    a = &pa;
     int* flags = tc ? tc_fwd_flags(workspace) : carve_chunk_ws(plan, workspace).flags;
     cudaError_t e = cudaMemsetAsync(ws_status(workspace), 0, sizeof(int), st);
     if (e == cudaSuccess) e = clear_flags(flags, pb, st);
@@ -382,11 +520,16 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args* a, void* workspace, size_t workspac
 
 // Segment map: the forward from a zero state (N = ht, o optional), then the forward from the
 // identity with the writes zeroed (v = 0), whose final state is M.
+// Its own part: the forward's workspace, the identity states, the zero v; then the copies.
+static size_t segment_map_own_ws(const gdn_fwd_args* a) {
+    const size_t es = elem_size(a->dtype);
+    return align256(fwd_own_ws(a)) + align256((size_t)(a->B * a->Hv * a->dk * a->dk) * 4) +
+           align256((size_t)(a->B * a->T * a->Hv * a->dv) * es);
+}
+
 size_t gdn_segment_map_workspace_size(const gdn_fwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
-    const size_t es = elem_size(a->dtype);
-    return align256(gdn_chunk_fwd_workspace_size(a)) + align256((size_t)(a->B * a->Hv * a->dk * a->dk) * 4) +
-           align256((size_t)(a->B * a->T * a->Hv * a->dv) * es);
+    return with_copies(segment_map_own_ws(a), args_pack_bytes<gdn_fwd_args, fwd_inputs>(a));
 }
 
 gdn_status gdn_segment_map(const gdn_fwd_args* a, float* M, void* workspace, size_t workspace_bytes,
@@ -398,27 +541,29 @@ gdn_status gdn_segment_map(const gdn_fwd_args* a, float* M, void* workspace, siz
     // validated as a forward whose o is optional; M must not overlap any input or output
     gdn_status s = check_fwd(a, false);
     if (s) return s;
-    const gdn_fwd_args x = *a;
+    gdn_fwd_args x = *a;
     const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype), BT = (size_t)(a->B * a->T);
     const size_t mbytes = (size_t)(a->B * a->Hv * a->dk * a->dk) * 4;
-    const Buf in[] = {{a->q, BT * a->Hk * a->dk * es, "q"}, {a->k, BT * a->Hk * a->dk * es, "k"},
-                      {a->v, BT * a->Hv * a->dv * es, "v"},
-                      {a->alpha, BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
-                      {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
-                      {a->w, a->w ? BT * a->Hv * a->dv * gs : 0, "w"}, {a->head_map, (size_t)a->Hv * 4, "head_map"}};
+    const gdn_strides& sd = a->strides;
+    const Buf in[] = {tok(a->q, BT, a->Hk * a->dk, sd.q, es, "q"), tok(a->k, BT, a->Hk * a->dk, sd.k, es, "k"),
+                      tok(a->v, BT, a->Hv * a->dv, sd.v, es, "v"),
+                      tok(a->alpha, BT, a->Hv * (a->alpha_per_channel ? a->dk : 1), sd.alpha, gs, "alpha"),
+                      tok(a->b, BT, a->Hv * (a->gates_per_channel ? a->dk : 1), sd.b, gs, "b"),
+                      tok(a->w, BT, a->Hv * a->dv, sd.w, gs, "w"), {a->head_map, (size_t)a->Hv * 4, "head_map"}};
     const Buf out[] = {{M, mbytes, "M"}, {a->ht, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, "ht"},
                        {a->o, a->o ? BT * a->Hv * a->dv * (a->out_f32 ? 4 : es) : 0, "o"}};
     if ((s = check_buffers(in, 7, out, 3))) return s;
-    const size_t need = gdn_segment_map_workspace_size(a);
-    if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (a->T > 0 && (s = copy_strided(&x, fwd_inputs, workspace, workspace_bytes, segment_map_own_ws(a), st,
+                                      "gdn_segment_map (strided inputs)")))
+        return s;
     if (a->T == 0) {
         cudaError_t e = cudaMemsetAsync(a->ht, 0, (size_t)(a->B * a->Hv * a->dk * a->dv) * 4, st);
         if (e == cudaSuccess) e = identity_states(M, a->B * a->Hv, (int)a->dk, st);
         return e == cudaSuccess ? GDN_OK : cuda_fail(e, "gdn_segment_map");
     }
     char* base = static_cast<char*>(workspace);
-    const size_t fw = align256(gdn_chunk_fwd_workspace_size(a));
+    const size_t fw = align256(fwd_own_ws(a));
     float* ident = reinterpret_cast<float*>(base + fw);
     void* zero_v = base + fw + align256(mbytes);
     // N: the segment from a zero state
@@ -461,8 +606,9 @@ static bool bwd_uses_tensor_cores(const gdn_bwd_args* a, const Problem& pb) {
 size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    if (bwd_uses_tensor_cores(a, pb)) return plan_tc_bwd_ws(pb, !identity_heads(pb), a->fwd_cache != nullptr).bytes;
-    return plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
+    const size_t own = bwd_uses_tensor_cores(a, pb) ? plan_tc_bwd_ws(pb, !identity_heads(pb), a->fwd_cache != nullptr).bytes
+                                                    : plan_chunk_ws(pb, true, !identity_heads(pb)).bytes;
+    return with_copies(own, args_pack_bytes<gdn_bwd_args, bwd_inputs>(a));
 }
 
 gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspace_bytes,
@@ -495,7 +641,12 @@ gdn_status gdn_chunk_bwd(const gdn_bwd_args* a, void* workspace, size_t workspac
         return fail(GDN_ERR_UNSUPPORTED, "grads_in_dtype with bf16 inputs: only the tensor-core backward (dk = dv = "
                                          "128, bf16 channel gates) returns bf16 gradients");
     TcBwdWs tplan = tc ? plan_tc_bwd_ws(pb, !direct, a->fwd_cache != nullptr) : TcBwdWs{};
-    if ((s = check_workspace(workspace, workspace_bytes, tc ? tplan.bytes : plan.bytes))) return s;
+    // the workspace, then the dense copies of strided inputs, which the rest reads instead
+    gdn_bwd_args pa = *a;
+    if ((s = copy_strided(&pa, bwd_inputs, workspace, workspace_bytes, tc ? tplan.bytes : plan.bytes, st,
+                          "gdn_chunk_bwd (strided inputs)")))
+        return s;
+    a = &pa;
     ChunkIO io{};
     io.q = a->q; io.k = a->k; io.v = a->v; io.alpha = a->alpha; io.b = a->b; io.w = a->w;
     io.h0 = a->h0; io.dout = a->grad_o; io.dht = a->grad_ht; io.dq = a->grad_q; io.dk = a->grad_k;
@@ -539,13 +690,19 @@ gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
     const size_t es = elem_size(a->dtype), gs = elem_size(a->gate_dtype), N = (size_t)a->N;
     const size_t cch = (size_t)(2 * a->Hk * a->dk + a->Hv * a->dv);
     const size_t st = N * a->Hv * a->dk * a->dv * 4;
+    // per-sequence strides (read in place; the kernels load one element at a time)
+    const gdn_strides& sd = a->strides;
+    const int64_t rq = a->Hk * a->dk, rv = a->Hv * a->dv;
+    const int64_t ra = a->Hv * (a->alpha_per_channel ? a->dk : 1), rb = a->Hv * (a->gates_per_channel ? a->dk : 1);
+    if ((s = check_stride(sd.q, rq, "q")) || (s = check_stride(sd.k, rq, "k")) || (s = check_stride(sd.v, rv, "v")) ||
+        (s = check_stride(sd.alpha, ra, "alpha")) || (s = check_stride(sd.b, rb, "b")) ||
+        (s = check_stride(sd.w, rv, "w")) || (s = check_stride(sd.z, rv, "z")))
+        return s;
     const Buf in[] = {
-        {a->q, N * a->Hk * a->dk * es, "q"}, {a->k, N * a->Hk * a->dk * es, "k"},
-        {a->v, N * a->Hv * a->dv * es, "v"},
-        {a->alpha, N * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
-        {a->b, N * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
-        {a->w, N * a->Hv * a->dv * gs, "w"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
-        {a->conv_w, cch * 4 * es, "conv_w"}, {a->z, N * a->Hv * a->dv * es, "z"},
+        tok(a->q, N, rq, sd.q, es, "q"), tok(a->k, N, rq, sd.k, es, "k"), tok(a->v, N, rv, sd.v, es, "v"),
+        tok(a->alpha, N, ra, sd.alpha, gs, "alpha"), tok(a->b, N, rb, sd.b, gs, "b"),
+        tok(a->w, N, rv, sd.w, gs, "w"), {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        {a->conv_w, cch * 4 * es, "conv_w"}, tok(a->z, N, rv, sd.z, es, "z"),
     };
     if (a->out_f32 != 0 && a->out_f32 != 1) return fail(GDN_ERR_INVALID_ARG, "out_f32 must be 0 or 1");
     const Buf out[] = {
@@ -557,6 +714,8 @@ gdn_status gdn_decode_step(const gdn_decode_args* a, gdn_stream stream) {
     p.q = a->q; p.k = a->k; p.v = a->v; p.alpha = a->alpha; p.b = a->b; p.w = a->w;
     p.state = a->state; p.o = a->o; p.o_f32 = a->out_f32; p.head_map = a->head_map; p.conv_state = a->conv_state;
     p.conv_w = a->conv_w; p.z = a->z;
+    p.sq = sd.q ? sd.q : rq; p.sk = sd.k ? sd.k : rq; p.sv = sd.v ? sd.v : rv;
+    p.sa = sd.alpha ? sd.alpha : ra; p.sb = sd.b ? sd.b : rb; p.sw = sd.w ? sd.w : rv; p.sz = sd.z ? sd.z : rv;
     p.N = (int)a->N; p.Hk = (int)a->Hk; p.Hv = (int)a->Hv; p.dk = (int)a->dk; p.dv = (int)a->dv;
     p.scale = a->scale;
     if ((s = check_logits(a->gate_logits, a->alpha_scale))) return s;
@@ -615,14 +774,18 @@ static bool layer_fwd_split(const gdn_layer_args* a, const Problem& pb) {
     return a->dtype == GDN_BF16 && !f.apc && !f.gpc && tc_fwd_eligible(pb, true, a->gate_dtype == GDN_BF16, f);
 }
 
-size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
-    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+static size_t layer_fwd_own_ws(const gdn_layer_args* a) {
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     // q, k, v after the convolution are kept in fp32 between the two kernels.
     const size_t conv = align256((size_t)(a->B * a->T) * (2 * a->Hk * a->dk + a->Hv * a->dv) * 4);
     // the CUDA-core form with the output norm keeps o (fp32) for the norm + gate kernel
     const size_t onorm = a->norm_w && !layer_fwd_split(a, pb) ? align256((size_t)(a->B * a->T * a->Hv * a->dv) * 4) : 0;
     return 256 + conv + plan_chunk_ws(pb, false, false).bytes + onorm;
+}
+
+size_t gdn_layer_core_fwd_workspace_size(const gdn_layer_args* a) {
+    if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
+    return with_copies(layer_fwd_own_ws(a), args_pack_bytes<gdn_layer_args, layer_inputs<gdn_layer_args>>(a));
 }
 
 gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t workspace_bytes,
@@ -639,12 +802,18 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
     const size_t BT = (size_t)(a->B * a->T);
     const size_t cch = (size_t)(2 * a->Hk * a->dk + a->Hv * a->dv);
     const size_t st = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
+    const gdn_strides& sd = a->strides;
+    const int64_t ra = a->Hv * (a->alpha_per_channel ? a->dk : 1), rb = a->Hv * (a->gates_per_channel ? a->dk : 1);
+    if ((s = check_stride(sd.q, a->Hk * a->dk, "xq")) || (s = check_stride(sd.k, a->Hk * a->dk, "xk")) ||
+        (s = check_stride(sd.v, a->Hv * a->dv, "xv")) || (s = check_stride(sd.alpha, ra, "alpha")) ||
+        (s = check_stride(sd.b, rb, "b")) || (s = check_stride(sd.w, a->Hv * a->dv, "w")) ||
+        (s = check_stride(sd.z, a->Hv * a->dv, "z")))
+        return s;
     const Buf in[] = {
-        {a->xq, BT * a->Hk * a->dk * es, "xq"}, {a->xk, BT * a->Hk * a->dk * es, "xk"},
-        {a->xv, BT * a->Hv * a->dv * es, "xv"}, {a->conv_w, cch * 4 * es, "conv_w"},
-        {a->alpha, BT * a->Hv * (a->alpha_per_channel ? a->dk : 1) * gs, "alpha"},
-        {a->b, BT * a->Hv * (a->gates_per_channel ? a->dk : 1) * gs, "b"},
-        {a->w, BT * a->Hv * a->dv * gs, "w"}, {a->z, BT * a->Hv * a->dv * es, "z"},
+        tok(a->xq, BT, a->Hk * a->dk, sd.q, es, "xq"), tok(a->xk, BT, a->Hk * a->dk, sd.k, es, "xk"),
+        tok(a->xv, BT, a->Hv * a->dv, sd.v, es, "xv"), {a->conv_w, cch * 4 * es, "conv_w"},
+        tok(a->alpha, BT, ra, sd.alpha, gs, "alpha"), tok(a->b, BT, rb, sd.b, gs, "b"),
+        tok(a->w, BT, a->Hv * a->dv, sd.w, gs, "w"), tok(a->z, BT, a->Hv * a->dv, sd.z, es, "z"),
         {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->norm_w, (size_t)a->dv * es, "norm_w"},
     };
@@ -676,8 +845,12 @@ gdn_status gdn_layer_core_fwd(const gdn_layer_args* a, void* workspace, size_t w
         }
         return copy_state(a->ht, a->h0, st, sm, "gdn_layer_core_fwd");
     }
-    const size_t need = gdn_layer_core_fwd_workspace_size(a);
-    if ((s = check_workspace(workspace, workspace_bytes, need))) return s;
+    // the workspace, then the dense copies of strided inputs, which the rest reads instead
+    gdn_layer_args pa = *a;
+    if ((s = copy_strided(&pa, layer_inputs<gdn_layer_args>, workspace, workspace_bytes, layer_fwd_own_ws(a), sm,
+                          "gdn_layer_core_fwd (strided inputs)")))
+        return s;
+    a = &pa;
     char* base = static_cast<char*>(workspace) + 256;
     const size_t conv_bytes = align256(BT * cch * 4);
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
@@ -798,7 +971,8 @@ static LayerBwdPlan plan_layer_bwd(const gdn_layer_bwd_args* a, const Problem& p
 size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* a) {
     if (!a || a->B < 1 || a->T < 1 || a->Hv < 1 || a->dk < 1 || a->dv < 1) return 0;
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
-    return plan_layer_bwd(a, pb).bytes;
+    return with_copies(plan_layer_bwd(a, pb).bytes,
+                       args_pack_bytes<gdn_layer_bwd_args, layer_inputs<gdn_layer_bwd_args>>(a));
 }
 
 gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size_t workspace_bytes,
@@ -825,11 +999,19 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     const size_t st = (size_t)(a->B * a->Hv * a->dk * a->dv) * 4;
     const size_t na = BT * a->Hv * (a->alpha_per_channel ? a->dk : 1), nb = BT * a->Hv * (a->gates_per_channel ? a->dk : 1);
     const size_t nw = a->gates_per_channel ? BT * a->Hv * a->dv : 0;
+    const gdn_strides& sd = a->strides;
+    const int64_t ra = a->Hv * (a->alpha_per_channel ? a->dk : 1), rb = a->Hv * (a->gates_per_channel ? a->dk : 1);
+    if ((s = check_stride(sd.q, a->Hk * a->dk, "xq")) || (s = check_stride(sd.k, a->Hk * a->dk, "xk")) ||
+        (s = check_stride(sd.v, a->Hv * a->dv, "xv")) || (s = check_stride(sd.alpha, ra, "alpha")) ||
+        (s = check_stride(sd.b, rb, "b")) || (s = check_stride(sd.w, a->Hv * a->dv, "w")) ||
+        (s = check_stride(sd.z, a->Hv * a->dv, "z")))
+        return s;
     const Buf in[] = {
-        {a->xq, BT * a->Hk * a->dk * es, "xq"}, {a->xk, BT * a->Hk * a->dk * es, "xk"},
-        {a->xv, BT * a->Hv * a->dv * es, "xv"}, {a->conv_w, cch * 4 * es, "conv_w"},
-        {a->alpha, na * gs, "alpha"}, {a->b, nb * gs, "b"}, {a->w, nw * gs, "w"},
-        {a->z, BT * a->Hv * a->dv * es, "z"}, {a->h0, st, "h0"}, {a->head_map, (size_t)a->Hv * 4, "head_map"},
+        tok(a->xq, BT, a->Hk * a->dk, sd.q, es, "xq"), tok(a->xk, BT, a->Hk * a->dk, sd.k, es, "xk"),
+        tok(a->xv, BT, a->Hv * a->dv, sd.v, es, "xv"), {a->conv_w, cch * 4 * es, "conv_w"},
+        tok(a->alpha, BT, ra, sd.alpha, gs, "alpha"), tok(a->b, BT, rb, sd.b, gs, "b"),
+        tok(a->w, BT, a->Hv * a->dv, sd.w, gs, "w"), tok(a->z, BT, a->Hv * a->dv, sd.z, es, "z"), {a->h0, st, "h0"},
+        {a->head_map, (size_t)a->Hv * 4, "head_map"},
         {a->grad_y, BT * a->Hv * a->dv * es, "grad_y"}, {a->grad_ht, st, "grad_ht"},
         {a->fwd_cache, a->fwd_cache ? a->fwd_cache_bytes : 0, "fwd_cache"},
         {a->norm_w, (size_t)a->dv * es, "norm_w"},
@@ -862,7 +1044,12 @@ gdn_status gdn_layer_core_bwd(const gdn_layer_bwd_args* a, void* workspace, size
     Problem pb = make_problem(a->B, a->T, a->Hk, a->Hv, a->dk, a->dv, a->scale, a->head_map);
     apply_logits(pb, a->gate_logits, a->alpha_scale);
     const LayerBwdPlan plan = plan_layer_bwd(a, pb);
-    if ((s = check_workspace(workspace, workspace_bytes, plan.bytes))) return s;
+    // the workspace, then the dense copies of strided inputs, which the rest reads instead
+    gdn_layer_bwd_args pa = *a;
+    if ((s = copy_strided(&pa, layer_inputs<gdn_layer_bwd_args>, workspace, workspace_bytes, plan.bytes, sm,
+                          "gdn_layer_core_bwd (strided inputs)")))
+        return s;
+    a = &pa;
     char* wsb = static_cast<char*>(workspace);
     auto at = [&](size_t o) { return reinterpret_cast<float*>(wsb + o); };
     const bool bf16 = a->dtype == GDN_BF16, bf16g = a->gate_dtype == GDN_BF16;

@@ -138,8 +138,8 @@ cudaError_t decode_conv_shift(const DecodeParams& p, cudaStream_t st) {
     const long total = (long)p.N * (2L * p.Hk * p.dk + (long)p.Hv * p.dv);
     const long blocks = (total + 255) / 256;
     return launch_kernel(conv_state_shift_kernel<TIn>, dim3(static_cast<unsigned>(blocks < 65535 ? blocks : 65535)),
-                         dim3(256), 0, st, const_cast<void*>(p.conv_state), p.q, p.k, p.v, p.N,
-                         p.Hk, p.Hv, p.dk, p.dv);
+                         dim3(256), 0, st, const_cast<void*>(p.conv_state), p.q, p.k, p.v, p.sq, p.sk,
+                         p.sv, p.N, p.Hk, p.Hv, p.dk, p.dv);
 }
 
 template <class TIn>

@@ -80,6 +80,10 @@ cudaError_t identity_states(float* S, long pairs, int d, cudaStream_t st);
 cudaError_t compose_states(const float* M, const float* N, const float* S_in, float* S_out, long pairs, int dk,
                            int dv, bool transpose, cudaStream_t st);
 
+// Strided inputs (strides.cu): `rows` rows of row_bytes bytes, stride_bytes apart in src, copied
+// back to back into dst (256-byte aligned).  cudaErrorMisalignedAddress if src is odd.
+cudaError_t pack_rows(const void* src, void* dst, long rows, long row_bytes, long stride_bytes, cudaStream_t st);
+
 // Tensor-core chunk backward (tc_bwd.cu): same eligibility as the forward, without z.
 // The forward cache (what the backward needs from the forward): byte offsets from its start.
 struct TcCache {

@@ -26,6 +26,11 @@ I32 = ctypes.c_int32
 F32 = ctypes.c_float
 
 
+class Strides(ctypes.Structure):
+    """gdn_strides: token strides in elements (0 = dense)."""
+    _fields_ = [("q", I64), ("k", I64), ("v", I64), ("alpha", I64), ("b", I64), ("w", I64), ("z", I64)]
+
+
 class FwdArgs(ctypes.Structure):
     _fields_ = [("q", P), ("k", P), ("v", P), ("alpha", P), ("b", P), ("w", P), ("h0", P),
                 ("z", P), ("o", P), ("ht", P), ("head_map", P),
@@ -33,7 +38,7 @@ class FwdArgs(ctypes.Structure):
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32),
                 ("bwd_cache", P), ("bwd_cache_bytes", ctypes.c_size_t), ("gate_logits", I32),
-                ("alpha_scale", P)]
+                ("alpha_scale", P), ("strides", Strides)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -44,7 +49,7 @@ class BwdArgs(ctypes.Structure):
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32),
                 ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t), ("gate_logits", I32),
-                ("alpha_scale", P), ("grad_alpha_scale", P), ("grads_in_dtype", I32)]
+                ("alpha_scale", P), ("grad_alpha_scale", P), ("grads_in_dtype", I32), ("strides", Strides)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -53,7 +58,7 @@ class DecodeArgs(ctypes.Structure):
                 ("N", I64), ("Hk", I64), ("Hv", I64), ("dk", I64), ("dv", I64),
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32), ("gate_logits", I32),
-                ("alpha_scale", P)]
+                ("alpha_scale", P), ("strides", Strides)]
 
 
 class LayerArgs(ctypes.Structure):
@@ -63,7 +68,7 @@ class LayerArgs(ctypes.Structure):
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("out_f32", I32), ("bwd_cache", P),
                 ("bwd_cache_bytes", ctypes.c_size_t), ("norm_w", P), ("norm_eps", F32), ("gate_logits", I32),
-                ("alpha_scale", P)]
+                ("alpha_scale", P), ("strides", Strides)]
 
 
 class LayerBwdArgs(ctypes.Structure):
@@ -75,7 +80,7 @@ class LayerBwdArgs(ctypes.Structure):
                 ("scale", F32), ("alpha_per_channel", I32), ("gates_per_channel", I32),
                 ("dtype", I32), ("gate_dtype", I32), ("fwd_cache", P), ("fwd_cache_bytes", ctypes.c_size_t),
                 ("norm_w", P), ("norm_eps", F32), ("grad_norm_w", P), ("gate_logits", I32),
-                ("alpha_scale", P), ("grad_alpha_scale", P)]
+                ("alpha_scale", P), ("grad_alpha_scale", P), ("strides", Strides)]
 
 
 EXPORTED = ["gdn_chunk_fwd_cache_size", "gdn_chunk_fwd_workspace_size", "gdn_chunk_fwd", "gdn_chunk_fwd_noalloc",
@@ -169,6 +174,45 @@ def _ptr(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _tok(t: Optional[torch.Tensor], lead: int = 2):
+    """A token-major input as (pointer, token stride in elements, 0 when dense).  Besides a
+    contiguous tensor it takes a view whose heads and channels are dense and whose tokens are
+    evenly spaced, such as a slice of a fused projection [B, T, C] viewed as [B, T, H, d].
+    ``lead`` is the number of token dimensions (2: [B, T, ...]; 1: the decode step's [N, ...])."""
+    if t is None:
+        return None, 0
+    if t.is_contiguous():
+        return _ptr(t), 0
+    if not t.is_cuda:
+        raise GdnError("libgdn takes CUDA tensors only (there is no CPU path)")
+    return ctypes.c_void_p(t.data_ptr()), _token_stride(tuple(t.shape), tuple(t.stride()), lead)
+
+
+def _token_stride(shape, strides, lead: int) -> int:
+    """The token stride, in elements, of a tensor of this shape and these strides (0 when its
+    tokens are dense); its first ``lead`` dimensions index tokens."""
+    row = 1
+    for dim in range(len(shape) - 1, lead - 1, -1):
+        if shape[dim] != 1 and strides[dim] != row:
+            raise GdnError("libgdn takes token-major tensors whose heads and channels are dense")
+        row *= shape[dim]
+    dims = [d for d in range(lead) if shape[d] != 1]
+    s = strides[dims[-1]] if dims else row
+    if len(dims) == 2 and strides[dims[0]] != shape[dims[1]] * s:
+        raise GdnError("libgdn takes token-major tensors whose tokens are evenly spaced")
+    if s < row:
+        raise GdnError(f"token stride {s} is below the {row} elements of a token")
+    return 0 if s == row else s
+
+
+def _inputs(lead: int, q, k, v, alpha, b, w, z=None):
+    """Pointers and gdn_strides of a call's token-major inputs."""
+    ptrs, strides = {}, {}
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("b", b), ("w", w), ("z", z)):
+        ptrs[name], strides[name] = _tok(t, lead)
+    return ptrs, Strides(**strides)
+
+
 def _dt(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return GDN_BF16
@@ -228,15 +272,16 @@ def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_ma
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     hm = _head_map(head_map, q.device, q.shape[-2])
-    a = FwdArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
-                h0=_ptr(h0), z=_ptr(z), o=_ptr(o), ht=_ptr(ht), head_map=_ptr(hm),
+    tp, ts = _inputs(2, q, k, v, alpha, bb, ww, z)
+    a = FwdArgs(q=tp["q"], k=tp["k"], v=tp["v"], alpha=tp["alpha"], b=tp["b"], w=tp["w"],
+                h0=_ptr(h0), z=tp["z"], o=_ptr(o), ht=_ptr(ht), head_map=_ptr(hm),
                 B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                 alpha_per_channel=int(alpha.dim() == 4), gates_per_channel=gpc,
                 dtype=_dt(q), gate_dtype=_dt(alpha),
                 out_f32=int(o is not None and o.dtype == torch.float32 and q.dtype != torch.float32),
                 bwd_cache=_ptr(bwd_cache),
                 bwd_cache_bytes=0 if bwd_cache is None else bwd_cache.numel() * bwd_cache.element_size(),
-                gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale))
+                gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale), strides=ts)
     return a, [q, k, v, alpha, bb, ww, h0, z, o, ht, hm, bwd_cache, alpha_scale]
 
 
@@ -334,7 +379,8 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
     Hv, dv = v.shape[2], v.shape[3]
     hm = _head_map(head_map, q.device, q.shape[-2])
     g = grads
-    a = BwdArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
+    tp, ts = _inputs(2, q, k, v, alpha, bb, ww)
+    a = BwdArgs(q=tp["q"], k=tp["k"], v=tp["v"], alpha=tp["alpha"], b=tp["b"], w=tp["w"],
                 h0=_ptr(h0), head_map=_ptr(hm), grad_o=_ptr(grad_o), grad_ht=_ptr(grad_ht),
                 grad_q=_ptr(g["dq"]), grad_k=_ptr(g["dk"]), grad_v=_ptr(g["dv"]),
                 grad_alpha=_ptr(g["dalpha"]), grad_b=_ptr(g["db"] if gpc else g["dbeta"]),
@@ -344,7 +390,7 @@ def bwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, head_map=None, 
                 dtype=_dt(q), gate_dtype=_dt(alpha), fwd_cache=_ptr(fwd_cache),
                 fwd_cache_bytes=0 if fwd_cache is None else fwd_cache.numel() * fwd_cache.element_size(),
                 gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale),
-                grad_alpha_scale=_ptr(g.get("dalpha_scale")), grads_in_dtype=int(grads_in_dtype))
+                grad_alpha_scale=_ptr(g.get("dalpha_scale")), grads_in_dtype=int(grads_in_dtype), strides=ts)
     return a, [q, k, v, alpha, bb, ww, h0, hm, grad_o, grad_ht, g, fwd_cache, alpha_scale]
 
 
@@ -391,13 +437,14 @@ def gdn_decode_step(state, q, k, v, alpha, b=None, w=None, beta=None, head_map=N
     if o is None:
         o = torch.empty((N, Hv, dv), dtype=torch.float32 if out_f32 else q.dtype, device=q.device)
     hm = _head_map(head_map, q.device, q.shape[-2])
-    a = DecodeArgs(q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), b=_ptr(bb), w=_ptr(ww),
+    tp, ts = _inputs(1, q, k, v, alpha, bb, ww, z)
+    a = DecodeArgs(q=tp["q"], k=tp["k"], v=tp["v"], alpha=tp["alpha"], b=tp["b"], w=tp["w"],
                    state=_ptr(state), o=_ptr(o), head_map=_ptr(hm), conv_state=_ptr(conv_state),
-                   conv_w=_ptr(conv_w), z=_ptr(z), N=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
+                   conv_w=_ptr(conv_w), z=tp["z"], N=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, scale=scale,
                    alpha_per_channel=int(alpha.dim() == 3), gates_per_channel=gpc,
                    dtype=_dt(q), gate_dtype=_dt(alpha),
                    out_f32=int(o.dtype == torch.float32 and q.dtype != torch.float32),
-                   gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale))
+                   gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale), strides=ts)
     check(load().gdn_decode_step(ctypes.byref(a), _stream(stream)), "gdn_decode_step")
     return o
 
@@ -411,14 +458,15 @@ def _layer_args(xq, xk, xv, conv_w, alpha, z, b, w, beta, h0, head_map, scale, y
     B, T, Hk, dk = xq.shape
     Hv, dv = xv.shape[2], xv.shape[3]
     hm = _head_map(head_map, xq.device, xq.shape[-2])
-    a = LayerArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
-                  b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
+    tp, ts = _inputs(2, xq, xk, xv, alpha, bb, ww, z)
+    a = LayerArgs(xq=tp["q"], xk=tp["k"], xv=tp["v"], conv_w=_ptr(conv_w), alpha=tp["alpha"],
+                  b=tp["b"], w=tp["w"], z=tp["z"], h0=_ptr(h0), y=_ptr(y), ht=_ptr(ht),
                   conv_state_out=_ptr(cs), head_map=_ptr(hm), B=B, T=T, Hk=Hk, Hv=Hv, dk=dk,
                   dv=dv, scale=scale, alpha_per_channel=int(alpha.dim() == 4),
                   gates_per_channel=gpc, dtype=_dt(xq), gate_dtype=_dt(alpha), out_f32=out_f32,
                   bwd_cache=_ptr(bwd_cache), bwd_cache_bytes=bwd_cache.numel() if bwd_cache is not None else 0,
                   norm_w=_ptr(norm_w), norm_eps=norm_eps, gate_logits=int(alpha_scale is not None),
-                  alpha_scale=_ptr(alpha_scale))
+                  alpha_scale=_ptr(alpha_scale), strides=ts)
     return a, hm
 
 
@@ -486,8 +534,9 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
     if alpha_scale is not None:
         out["dalpha_scale"] = torch.empty(tuple(alpha_scale.shape), **f32)
     hm = _head_map(head_map, dev, Hk)
-    a = LayerBwdArgs(xq=_ptr(xq), xk=_ptr(xk), xv=_ptr(xv), conv_w=_ptr(conv_w), alpha=_ptr(alpha),
-                     b=_ptr(bb), w=_ptr(ww), z=_ptr(z), h0=_ptr(h0), head_map=_ptr(hm), grad_y=_ptr(grad_y),
+    tp, ts = _inputs(2, xq, xk, xv, alpha, bb, ww, z)
+    a = LayerBwdArgs(xq=tp["q"], xk=tp["k"], xv=tp["v"], conv_w=_ptr(conv_w), alpha=tp["alpha"],
+                     b=tp["b"], w=tp["w"], z=tp["z"], h0=_ptr(h0), head_map=_ptr(hm), grad_y=_ptr(grad_y),
                      grad_ht=_ptr(grad_ht), grad_xq=_ptr(out["dxq"]), grad_xk=_ptr(out["dxk"]),
                      grad_xv=_ptr(out["dxv"]), grad_conv_w=_ptr(out["dconv_w"]), grad_alpha=_ptr(out["dalpha"]),
                      grad_b=_ptr(gb), grad_w=_ptr(gw), grad_z=_ptr(out["dz"]), grad_h0=_ptr(out["dh0"]),
@@ -497,7 +546,7 @@ def gdn_layer_core_bwd(xq, xk, xv, conv_w, alpha, z, grad_y, b=None, w=None, bet
                      fwd_cache_bytes=fwd_cache.numel() if fwd_cache is not None else 0,
                      norm_w=_ptr(norm_w), norm_eps=norm_eps, grad_norm_w=_ptr(out.get("dnorm_w")),
                      gate_logits=int(alpha_scale is not None), alpha_scale=_ptr(alpha_scale),
-                     grad_alpha_scale=_ptr(out.get("dalpha_scale")))
+                     grad_alpha_scale=_ptr(out.get("dalpha_scale")), strides=ts)
     lib = load()
     need = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(a))
     ws = _workspace(need, dev, workspace)

@@ -21,8 +21,10 @@
  *    memory is a caller workspace whose size the *_workspace_size() calls return (the workspace
  *    may be reused across calls on the same stream; its contents on entry do not matter).
  *  - Pointers: every tensor pointer is a device pointer (cudaMalloc'd or equivalent) to a dense,
- *    contiguous array in the layout stated; all must be 16-byte aligned.  Outputs must not
- *    overlap inputs or each other (in-place arguments say so explicitly).
+ *    contiguous array in the layout stated; all must be 16-byte aligned.  Token-major inputs
+ *    may instead be given with a token stride (gdn_strides below).  Outputs must not overlap
+ *    inputs (a strided input spans its first to its last element) or each other (in-place
+ *    arguments say so explicitly).
  *  - Execution: every call is asynchronous on the given stream and never synchronises.
  *    Outputs are valid once the stream reaches the end of the call.
  *  - Layouts: token-major.  q, k: [B,T,Hk,dk]; v, o, z: [B,T,Hv,dv]; channel gates alpha, b:
@@ -36,9 +38,10 @@
  *    DeltaNet», «Les projections d'entrée».
  *  - Sizes: dk, dv in {64, 128}; B, T, Hk, Hv >= 1 (T = 0 is accepted and does nothing but copy
  *    h0 to ht).  T need not be a multiple of the chunk length 64.
- *  - Dtypes: q, k, v, o, z in `dtype`; alpha, b, w, beta in `gate_dtype`; states and every
- *    gradient are fp32 (gradients leave the fp32 accumulators unrounded: several of them are
- *    heavy-tailed, and a bf16 store alone would cost up to half an ulp of their largest entry).
+ *  - Dtypes: q, k, v, o, z in `dtype`; alpha, b, w, beta in `gate_dtype`; states are fp32;
+ *    gradients are fp32 by default (they leave the fp32 accumulators unrounded: several of them
+ *    are heavy-tailed, and a bf16 store alone would cost up to half an ulp of their largest
+ *    entry), or in the inputs' dtypes with gdn_chunk_bwd's grads_in_dtype.
  *  - Range: every alpha in [0, 1] is supported.  The chunked kernels carry the decay inside a
  *    chunk of 64 tokens as a ratio Gamma_r / Gamma_s of running products of alpha, which fp32
  *    holds while the product over a chunk stays at or above 2^-100 (~7.9e-31) on every channel.
@@ -87,6 +90,23 @@ typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
 /* Opaque stream handle: a cudaStream_t (NULL = the legacy default stream). */
 typedef void* gdn_stream;
 
+/* Token strides of the token-major inputs of a call, in elements (every field optional).
+ *  - 0: the tensor is dense in the layout stated for it.
+ *  - s > 0: token t of sequence b starts at element (b * T + t) * s (the decode step: sequence n
+ *    at n * s), and that token's heads and channels follow it densely.  This lets a caller pass
+ *    the slices of one fused projection buffer ([B, T, C] with the q, k, v, gate columns side by
+ *    side) without copying them first.  s must be at least the token's own element count (H * d,
+ *    or H for a scalar gate) and at most 2^31; a tensor given with s > that count needs only the
+ *    alignment of its element type.
+ *  - Chunk forward, backward, segment map and layer calls copy every tensor whose stride is not
+ *    its dense one into a dense part of the workspace first (one copy kernel per tensor; the
+ *    bytes are part of *_workspace_size()).  The decode step reads strided tensors in place.
+ *  - The layer calls read q, k, v as the strides of xq, xk, xv.  A field whose tensor the call
+ *    does not take (z of gdn_chunk_bwd) must be 0. */
+typedef struct gdn_strides {
+    int64_t q, k, v, alpha, b, w, z;
+} gdn_strides;
+
 /* ------------------------------------------------------------------------------------------
  * Chunkwise forward.  Chunkwise-parallel form with chunk length 64: inside a chunk the decay is
  * absorbed into the erase and write factors and the lower-triangular system (I + A)^-1 is solved
@@ -123,6 +143,7 @@ typedef struct gdn_fwd_args {
     size_t bwd_cache_bytes;
     int32_t gate_logits;       /* 1: alpha, b, w are logits (see the conventions above) */
     const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
+    gdn_strides strides;       /* token strides of q, k, v, alpha, b, w, z (all 0: dense) */
 } gdn_fwd_args;
 
 /* Bytes of the optional forward cache (0 where the problem cannot keep one). */
@@ -206,6 +227,7 @@ typedef struct gdn_bwd_args {
     const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
     float* grad_alpha_scale;   /* out [Hv] fp32, may be NULL (must be NULL without gate_logits) */
     int32_t grads_in_dtype;    /* 1: gradients in the inputs' dtypes (see above); 0: fp32 */
+    gdn_strides strides;       /* token strides of q, k, v, alpha, b, w (z: 0); gradients are dense */
 } gdn_bwd_args;
 
 GDN_API size_t gdn_chunk_bwd_workspace_size(const gdn_bwd_args* args);
@@ -275,6 +297,7 @@ typedef struct gdn_decode_args {
     int32_t out_f32;      /* 1: o is written in fp32 instead of dtype */
     int32_t gate_logits;       /* 1: alpha, b, w are logits */
     const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
+    gdn_strides strides;       /* per-sequence strides of q, k, v, alpha, b, w, z, read in place */
 } gdn_decode_args;
 
 GDN_API gdn_status gdn_decode_step(const gdn_decode_args* args, gdn_stream stream);
@@ -331,6 +354,7 @@ typedef struct gdn_layer_args {
     float norm_eps;
     int32_t gate_logits;       /* 1: alpha, b, w are logits */
     const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
+    gdn_strides strides;       /* token strides of xq, xk, xv (fields q, k, v), alpha, b, w, z */
 } gdn_layer_args;
 
 /* Bytes of the optional layer forward cache (0 where the layer backward cannot use one). */
@@ -401,6 +425,7 @@ typedef struct gdn_layer_bwd_args {
     int32_t gate_logits;       /* 1: alpha, b, w are logits; the gradients returned are those of the logits */
     const float* alpha_scale;  /* [Hv] fp32, with gate_logits */
     float* grad_alpha_scale;   /* out [Hv] fp32, may be NULL (must be NULL without gate_logits) */
+    gdn_strides strides;       /* token strides of xq, xk, xv (fields q, k, v), alpha, b, w, z */
 } gdn_layer_bwd_args;
 
 GDN_API size_t gdn_layer_core_bwd_workspace_size(const gdn_layer_bwd_args* args);

@@ -8,6 +8,7 @@ import subprocess
 import tempfile
 
 import pytest
+import torch
 
 from gated_delta_rule_76_b200 import build as gbuild
 from gated_delta_rule_76_b200 import gdn
@@ -54,7 +55,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 STRUCTS = {"gdn_fwd_args": gdn.FwdArgs, "gdn_bwd_args": gdn.BwdArgs,
            "gdn_decode_args": gdn.DecodeArgs, "gdn_layer_args": gdn.LayerArgs,
-           "gdn_layer_bwd_args": gdn.LayerBwdArgs}
+           "gdn_layer_bwd_args": gdn.LayerBwdArgs, "gdn_strides": gdn.Strides}
 
 
 def test_ctypes_structs_match_c_layout():
@@ -294,3 +295,71 @@ def test_gradient_dtype_option_on_the_host(lib):
     a = _bwd(grads_in_dtype=1, **close)
     assert lib.gdn_chunk_bwd(ctypes.byref(a), ws, 1 << 30, None) == 2
     assert gdn.kernel_launches() == before
+
+
+def test_token_strides_on_the_host(lib):
+    """gdn_strides: a stride below a token's element count (or above 2^31) is refused; a strided
+    input needs only its element alignment and adds its dense copy to the workspace; an output
+    inside a strided input's span overlaps it; the backward refuses a z stride.  Fake device
+    addresses: every call here stops before a launch."""
+    before = gdn.kernel_launches()
+    ws = ctypes.c_void_p(1 << 30)
+    row = 64  # Hk * dk of _fwd()
+    a = _fwd()
+    a.strides.q = row - 1
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ws, 1 << 30, None) == 1
+    assert "token stride of q" in lib.gdn_last_error().decode()
+    a.strides.q = (1 << 31) + 1
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ws, 1 << 30, None) == 1
+    # dense stride given explicitly: same workspace as 0
+    dense = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(_fwd()))
+    a = _fwd()
+    a.strides.q = row
+    assert lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a)) == dense
+    # a strided q (2-byte aligned, 3 * row apart) and a strided alpha: their dense copies
+    a = _fwd(q=18, o=1 << 22)
+    a.strides.q = 3 * row
+    a.strides.alpha = 2 * row
+    need = lib.gdn_chunk_fwd_workspace_size(ctypes.byref(a))
+    copy = 64 * row * 2  # 64 tokens of 64 bf16 values, a multiple of 256 bytes
+    assert need == (dense + 255) // 256 * 256 + 2 * copy
+    # accepted by the buffer checks (a dense q at 18 is not), then stopped by a short workspace
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ws, need - 1, None) == 4
+    assert lib.gdn_chunk_fwd(ctypes.byref(_fwd(q=18)), ws, 1 << 30, None) == 1
+    # o placed inside q's span (3 * row * 63 + row elements from 18) overlaps it
+    a = _fwd(q=1 << 20, o=(1 << 20) + 2 * 64 * row * 2)
+    a.strides.q = 3 * row
+    assert lib.gdn_chunk_fwd(ctypes.byref(a), ws, 1 << 30, None) == 1
+    assert "overlap" in lib.gdn_last_error().decode()
+    # the backward takes no z
+    b = _bwd()
+    b.strides.z = 64
+    assert lib.gdn_chunk_bwd(ctypes.byref(b), ws, 1 << 30, None) == 1
+    assert "strides.z" in lib.gdn_last_error().decode()
+    b = _bwd()
+    b.strides.v = 63
+    assert lib.gdn_chunk_bwd(ctypes.byref(b), ws, 1 << 30, None) == 1
+    assert gdn.kernel_launches() == before
+
+
+def test_binding_token_strides():
+    """The binding's token stride of a view (CPU tensors: the rule only, nothing is called)."""
+    buf = torch.zeros((2 * 5, 200))
+    v = buf[:, 64:128].view(2, 5, 1, 64)  # a slice of a fused projection buffer
+    assert gdn._token_stride(v.shape, v.stride(), 2) == 200
+    d = torch.zeros((2, 5, 2, 64))
+    assert gdn._token_stride(d.shape, d.stride(), 2) == 0
+    one = buf[:5, 0:64].view(1, 5, 1, 64)  # B = 1: the T stride alone
+    assert gdn._token_stride(one.shape, one.stride(), 2) == 200
+    tok = buf[:1, 0:128].view(1, 1, 2, 64)  # a single token: dense
+    assert gdn._token_stride(tok.shape, tok.stride(), 2) == 0
+    dec = buf[:, 64:128].view(10, 1, 64)  # decode: [N, H, d]
+    assert gdn._token_stride(dec.shape, dec.stride(), 1) == 200
+    with pytest.raises(gdn.GdnError, match="heads and channels are dense"):
+        x = d[:, :, :, :32]
+        gdn._token_stride(x.shape, x.stride(), 2)
+    with pytest.raises(gdn.GdnError, match="evenly spaced"):
+        x = torch.zeros((2, 7, 64))[:, :5]
+        gdn._token_stride(x.shape, x.stride(), 2)
+    with pytest.raises(gdn.GdnError, match="CUDA tensors only"):
+        gdn._tok(v)
