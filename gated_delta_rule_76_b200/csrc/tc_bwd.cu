@@ -20,7 +20,6 @@ size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 TcCache plan_tc_cache(const Problem& pb) {
     TcCache c;
     const size_t st1 = (size_t)pb.B * pb.Hv * (pb.NT + 1) * pb.dk * pb.dv * sizeof(float);
-    const size_t tok = (size_t)pb.B * pb.T * pb.Hv * pb.dv * 2;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;

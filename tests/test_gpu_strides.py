@@ -16,7 +16,7 @@ import torch
 from gated_delta_rule_76_b200 import gdn
 from gated_delta_rule_76_b200.inputs import draw
 from oracle import oracle
-from parity import assert_parity, to_cuda
+from parity import assert_bf16_is_rounding, assert_parity, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -86,10 +86,13 @@ def test_forward_and_backward_on_strided_inputs(c):
     assert torch.equal(o, os_) and torch.equal(ht, hts)
     for key, val in gd.items():
         assert torch.equal(val, gs[key]), key
-    if c["offset"] == 1:  # this case also against the oracle (forward with the swish gate)
+    if c["offset"] == 1:
+        # this case also against the oracle: the gated output unrounded (out_f32), whose bf16
+        # rounding the strided call returned, and the final state
+        y32, _ = gdn.gdn_chunk_fwd(s["q"], s["k"], s["v"], s["alpha"], h0=g["h0"], z=zs, out_f32=True, **gates(s))
         o_ref, ht_ref = oracle.fwd(x["q"], x["k"], x["v"], x["alpha"], h0=x["h0"], **gates(x))
-        y_ref = oracle.swish_gate(o_ref, x["z"])
-        assert_parity(os_, y_ref, "bf16", "o")
+        assert_parity(y32, oracle.swish_gate(o_ref, x["z"]), "bf16", "o")
+        assert_bf16_is_rounding(os_, y32, "o")
         assert_parity(hts, ht_ref, "bf16", "ht")
 
 
