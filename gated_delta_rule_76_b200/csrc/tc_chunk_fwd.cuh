@@ -593,9 +593,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             if (p.vp_hi) {
-                // V' (saving mode), stored while X4 / X5 run: rows 32h .. 32h + 31 of column j are
-                // 64 contiguous bytes of the chunk-major tile (rows past the sequence as zeros)
-                const long vo = (((long)blockIdx.x * NT + n) * D + j) * 64 + 32 * h;
+                // V' (saving mode), stored while X4 / X5 run.  Column j's rows 32h .. 32h + 31 are 64
+                // contiguous bytes of the chunk-major tile (rows past the sequence as zeros), four
+                // 16-byte chunks.  A 4 x 4 transpose of those chunks within the lane quad gives lane e
+                // chunk e of the quad's four columns, so that each store writes whole 64-byte column
+                // pieces (8 per warp instruction instead of 32 scattered 16-byte pieces: the stores
+                // of the saving mode are what throttles this chain's global-memory queue).
                 uint32_t vh[16], vl[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -604,12 +607,48 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     vh[i] = vhi[i] & keep;
                     vl[i] = vlo[i] & keep;
                 }
-                uint4* dh = reinterpret_cast<uint4*>(p.vp_hi + vo);
-                uint4* dl = reinterpret_cast<uint4*>(p.vp_lo + vo);
+                const int e = j & 3;
+                const bool b0 = (e & 1) != 0, b1 = (e & 2) != 0;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    dh[q4] = make_uint4(vh[4 * q4], vh[4 * q4 + 1], vh[4 * q4 + 2], vh[4 * q4 + 3]);
-                    dl[q4] = make_uint4(vl[4 * q4], vl[4 * q4 + 1], vl[4 * q4 + 2], vl[4 * q4 + 3]);
+                for (int w = 0; w < 4; ++w) {
+                    // chunks (0,1) and (2,3) swap across lane pairs, then chunk pairs across lane pairs of pairs
+#pragma unroll
+                    for (int k = 0; k < 4; k += 2) {
+                        const uint32_t sh = b0 ? vh[4 * k + w] : vh[4 * (k + 1) + w];
+                        const uint32_t sl = b0 ? vl[4 * k + w] : vl[4 * (k + 1) + w];
+                        const uint32_t rh = __shfl_xor_sync(0xffffffffu, sh, 1);
+                        const uint32_t rl = __shfl_xor_sync(0xffffffffu, sl, 1);
+                        if (b0) {
+                            vh[4 * k + w] = rh;
+                            vl[4 * k + w] = rl;
+                        } else {
+                            vh[4 * (k + 1) + w] = rh;
+                            vl[4 * (k + 1) + w] = rl;
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const uint32_t sh = b1 ? vh[4 * k + w] : vh[4 * (k + 2) + w];
+                        const uint32_t sl = b1 ? vl[4 * k + w] : vl[4 * (k + 2) + w];
+                        const uint32_t rh = __shfl_xor_sync(0xffffffffu, sh, 2);
+                        const uint32_t rl = __shfl_xor_sync(0xffffffffu, sl, 2);
+                        if (b1) {
+                            vh[4 * k + w] = rh;
+                            vl[4 * k + w] = rl;
+                        } else {
+                            vh[4 * (k + 2) + w] = rh;
+                            vl[4 * (k + 2) + w] = rl;
+                        }
+                    }
+                }
+                // lane e: chunk e (tokens 32h + 8e .. + 7) of columns 4 (j / 4) + i, i = 0 .. 3
+                const long vo = (((long)blockIdx.x * NT + n) * D + (j & ~3)) * 64 + 32 * h + 8 * e;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    *reinterpret_cast<uint4*>(p.vp_hi + vo + 64 * i) =
+                        make_uint4(vh[4 * i], vh[4 * i + 1], vh[4 * i + 2], vh[4 * i + 3]);
+                    *reinterpret_cast<uint4*>(p.vp_lo + vo + 64 * i) =
+                        make_uint4(vl[4 * i], vl[4 * i + 1], vl[4 * i + 2], vl[4 * i + 3]);
                 }
             }
             if (tid == 0) {
