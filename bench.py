@@ -110,10 +110,10 @@ def load_peaks():
 
 
 # DRAM bytes (read + write) of one gdn_chunk_bwd call on the headline workload, summed over its two
-# kernels (reverse scan 340,207,616 B, gradients 811,751,168 B) from ncu's dram__bytes_read.sum +
+# kernels (reverse scan 341,024,768 B, gradients 811,200,512 B) from ncu's dram__bytes_read.sum +
 # dram__bytes_write.sum on B=8 T=1024 (the same 128 (sequence, head) pairs, a quarter of the
 # chunks; the traffic is per chunk, so x4).  To be reset to None whenever those kernels change.
-BWD_CALL_TRAFFIC_BYTES = (340207616 + 811751168) * 4
+BWD_CALL_TRAFFIC_BYTES = (341024768 + 811200512) * 4
 
 
 def roofline(bytes_per_launch, flops_per_launch, seconds, peaks, peak_kind, scope, sustained=False,

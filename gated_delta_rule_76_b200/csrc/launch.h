@@ -45,7 +45,7 @@ ChunkWs carve_chunk_ws(const WsPlan& plan, void* base);
 // Tensor-core chunk forward (tc_fwd.cu): bf16 q/k/v with dk = dv = 128.  With `save`, the state
 // entering every chunk and V' of every token are written for the backward (o and ht may be NULL).
 struct TcFwdSave {
-    float* s0;               // [B*Hv][NT + 1][dv/4][dk][4]
+    float* s0;               // [B*Hv][NT + 1][dv/8][dk][8]
     __nv_bfloat16* vp_hi;    // [B*Hv][NT][dv][64 tokens]: chunk-major, a column's tokens contiguous
     __nv_bfloat16* vp_lo;
     float* o_raw;            // with the swish gate, may be NULL: the output before the gate (fp32)
@@ -88,7 +88,7 @@ cudaError_t pack_rows(const void* src, void* dst, long rows, long row_bytes, lon
 // The forward cache (what the backward needs from the forward): byte offsets from its start.
 struct TcCache {
     size_t bytes = 0;
-    size_t s0, vp_hi, vp_lo;  // states [B*Hv][NT+1][dv/4][dk][4] fp32; V' hi, lo [B*Hv][NT][dv][64] bf16
+    size_t s0, vp_hi, vp_lo;  // states [B*Hv][NT+1][dv/8][dk][8] fp32; V' hi, lo [B*Hv][NT][dv][64] bf16
     size_t t;                 // T tiles [B*Hv][NT][8 KB]: bf16, 64 rows of 128 swizzled bytes
 };
 TcCache plan_tc_cache(const Problem& pb);

@@ -770,8 +770,8 @@ struct Params {
     const __nv_bfloat16* q_lo;  // SPLIT: lo halves of q, k, v (hi in q, k, v)
     const __nv_bfloat16* k_lo;
     const __nv_bfloat16* v_lo;
-    const float* s0;     // [B*Hv][NT][dv/4][dk][4]: row c, columns 4q..4q+3 at float4 (q * dk + c)
-    const float* dsc;    // same layout
+    const float* s0;     // [B*Hv][NT + 1][dv/8][dk][8]: row c, columns 8q..8q+7 at float (q * dk + c) * 8
+    const float* dsc;    // [B*Hv][NT][dv/4][dk][4]: row c, columns 4u..4u+3 at float4 (u * dk + c)
     void* dq;            // [B,T,Hk,dk] (direct, the gradients' type) or [B,T,Hv,dk] per value head (fp32)
     void* dk;
     void* dv;            // [B,T,Hv,dv]; this and the gate gradients in the gradients' type (fp32 or bf16)
@@ -887,6 +887,14 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// 32 bytes (8 floats) from global memory written by an earlier kernel, in one 256-bit load through
+// the non-coherent path; p must be 32-byte aligned.
+__device__ __forceinline__ void ldg_v8(const float* p, float4& x, float4& y) {
+    asm("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w), "=f"(y.x), "=f"(y.y), "=f"(y.z), "=f"(y.w)
+        : "l"(p));
+}
+
 // Staging group (128 threads, c = lane = channel): S0 and dS_end rows of the chunk into tensor
 // memory as split A operands and rowsum(dS_end .* S0) into xslot[c]; then, once the raw TMA tiles
 // have landed, the cumulative decay (gamma into gslot[c]) and the split [Ehat;Qhat], Ktil tiles.
@@ -895,19 +903,19 @@ __device__ __forceinline__ void stage_chunk(const Params& p, const Ctx& cx, cons
                                             float* xslot, float* gslot, uint32_t raw_parity, int it = 15) {
     const Problem& pb = p.pb;
     {
-        // row c: columns 4u .. 4u + 3 are the float4 u * D (coalesced over the group's rows)
+        // row c: S0 columns 8v .. 8v + 7 are 32 contiguous bytes at float (v * D + c) * 8 (one
+        // 256-bit load; a warp reads 1 KB contiguous), dS columns 4u .. 4u + 3 the float4 u * D + c
         const long bh = cp.ci / pb.NT;
-        const float4* s0r = reinterpret_cast<const float4*>(p.s0 + (bh * (pb.NT + 1) + cp.n) * D * D) + c;
+        const float* s0r = p.s0 + (bh * (pb.NT + 1) + cp.n) * D * D + 8 * c;
         const float4* dsr = reinterpret_cast<const float4*>(p.dsc + cp.ci * D * D) + c;
         float dot = 0.f;
 #pragma unroll 1
         for (int q8 = 0; q8 < 2; ++q8) {
             float4 a[16], d[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                a[u] = __ldg(s0r + (16 * q8 + u) * D);
-                d[u] = __ldg(dsr + (16 * q8 + u) * D);
-            }
+            for (int u = 0; u < 16; u += 2) ldg_v8(s0r + ((16 * q8 + u) >> 1) * (8 * D), a[u], a[u + 1]);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) d[u] = __ldg(dsr + (16 * q8 + u) * D);
 #pragma unroll
             for (int hq = 0; hq < 2; ++hq) {
                 uint32_t ah[16], al[16], dh[16], dl[16];

@@ -137,7 +137,7 @@ struct Params {
     int* err;    // device error word (bit 0: a bounded wait expired)
     uint64_t wait_ns;  // limit of every bounded wait; 0 = kWaitNs
     // Backward support (all NULL in a plain forward).  o may be NULL then: no output is formed.
-    float* s0_out;               // [B*Hv][NT + 1][dv/4][dk][4] fp32: the state entering every chunk, then
+    float* s0_out;               // [B*Hv][NT + 1][dv/8][dk][8] fp32: the state entering every chunk, then
                                  //   the final state
     __nv_bfloat16* vp_hi;        // [B*Hv][NT][dv][64]: V' = T (Z - Ehat S0) of every chunk, column-major
     __nv_bfloat16* vp_lo;        //   (a column's 64 tokens contiguous), as hi = bf16(V'), lo = bf16(V' - hi)
@@ -449,12 +449,14 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             if (p.s0_out) {
                 // state entering chunk n (saving mode), stored while X2 runs: rows 64h .. 64h + 63
-                // of column j, in the layout [j / 4][row][j % 4] (a reader holding one row per
-                // thread loads it as float4s).  Plain 4-byte stores: the quad transpose of
-                // store_state_block, which the reverse scan uses, made this chain slower.
-                float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 2) * (4 * D) + (64 * h) * 4 + (j & 3);
+                // of column j, in the layout [j / 8][row][j % 8]: each group of 8 lanes fills one
+                // 32-byte sector per store (a reader holding one row per thread loads a row's 8
+                // columns of a block as one 32-byte vector).  Plain 4-byte stores: transposing
+                // the state across lanes first (store_state_block, as the reverse scan does) made
+                // this chain slower.
+                float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 3) * (8 * D) + (64 * h) * 8 + (j & 7);
 #pragma unroll
-                for (int c = 0; c < 64; ++c) dst[4 * c] = S[c];
+                for (int c = 0; c < 64; ++c) dst[8 * c] = S[c];
             }
             tc_fence_before();
             fence_async_shared();
@@ -755,8 +757,11 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int c = 0; c < 64; ++c) p.ht[soff + (long)(64 * h + c) * D + j] = S[c];
         }
-        if (p.s0_out && !*cx.abort_flag)  // the final state follows the last chunk's entering state
-            store_state_block(p.s0_out + ((long)blockIdx.x * (NT + 1) + NT) * (D * D), S, j, h);
+        if (p.s0_out && !*cx.abort_flag) {  // the final state follows the last chunk's entering state
+            float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + NT) * (D * D) + (j >> 3) * (8 * D) + (64 * h) * 8 + (j & 7);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) dst[8 * c] = S[c];
+        }
     } else {
         // =================================== chunk prologue ===================================
         const int c = tid - 256;  // key channel; also TMEM lane of X1
