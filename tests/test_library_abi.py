@@ -363,3 +363,50 @@ def test_binding_token_strides():
         gdn._token_stride(x.shape, x.stride(), 2)
     with pytest.raises(gdn.GdnError, match="CUDA tensors only"):
         gdn._tok(v)
+
+
+def test_token_strides_on_every_call(lib):
+    """Stride validation and the dense copies' workspace on the segment map, the decode step and
+    both layer calls (fake device addresses; every call stops on the host)."""
+    before = gdn.kernel_launches()
+    P = ctypes.c_void_p
+    ws = P(1 << 34)
+    # segment map: a k stride below the token's 64 elements
+    a = _fwd(o=None, ht=1 << 25)
+    a.strides.k = 63
+    assert lib.gdn_segment_map(ctypes.byref(a), P(1 << 24), ws, 1 << 34, None) == 1
+    assert "token stride of k" in lib.gdn_last_error().decode()
+    a = _fwd(o=None, ht=1 << 25)
+    dense = lib.gdn_segment_map_workspace_size(ctypes.byref(a))
+    a.strides.q = 128
+    assert lib.gdn_segment_map_workspace_size(ctypes.byref(a)) == (dense + 255) // 256 * 256 + 64 * 64 * 2
+    # decode: strides are read in place, so only the bounds are checked
+    d = gdn.DecodeArgs(q=16, k=32, v=48, alpha=64, b=80, w=96, state=1 << 20, o=1 << 21, N=2, Hk=1, Hv=1, dk=64,
+                       dv=64, scale=1.0, alpha_per_channel=1, gates_per_channel=1, dtype=0, gate_dtype=0)
+    d.strides.v = 10
+    assert lib.gdn_decode_step(ctypes.byref(d), None) == 1
+    assert "token stride of v" in lib.gdn_last_error().decode()
+    d.strides.v = 0
+    d.strides.z = (1 << 31) + 1
+    assert lib.gdn_decode_step(ctypes.byref(d), None) == 1
+    # layer forward: z below its 128 elements; a strided xq adds its copy and needs its element alignment only
+    f = _layer_fwd()
+    f.strides.z = 127
+    assert lib.gdn_layer_core_fwd(ctypes.byref(f), ws, 1 << 34, None) == 1
+    assert "token stride of z" in lib.gdn_last_error().decode()
+    dense = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(_layer_fwd()))
+    f = _layer_fwd(xq=18)
+    assert lib.gdn_layer_core_fwd(ctypes.byref(f), ws, 1 << 34, None) == 1  # dense xq at 18: misaligned
+    f.strides.q = 256
+    need = lib.gdn_layer_core_fwd_workspace_size(ctypes.byref(f))
+    assert need == (dense + 255) // 256 * 256 + 64 * 128 * 2
+    assert lib.gdn_layer_core_fwd(ctypes.byref(f), ws, need - 1, None) == 4
+    # layer backward: a negative stride, then a strided alpha's copy in the workspace
+    g = _layer_bwd()
+    g.strides.b = -1
+    assert lib.gdn_layer_core_bwd(ctypes.byref(g), ws, 1 << 34, None) == 1
+    dense = lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(_layer_bwd()))
+    g = _layer_bwd()
+    g.strides.alpha = 4  # scalar alpha: 1 element a token
+    assert lib.gdn_layer_core_bwd_workspace_size(ctypes.byref(g)) == (dense + 255) // 256 * 256 + 256
+    assert gdn.kernel_launches() == before
