@@ -164,3 +164,32 @@ def test_planted_layer_backward_mistake_is_caught(name, old, new, monkeypatch):
         except AssertionError:
             caught.append(i)
     assert caught, f"no pin caught the planted mistake: {name}"
+
+
+# The layer core's forward composition (numpy in oracle.py around the compiled pieces): planted
+# mistakes that the closed forms of test_layer_core_forward_closed_forms must catch.
+LAYER_FWD_MUTANTS = [
+    ("layer forward: q and k convolution weight blocks swapped",
+     [("q, _ = conv_silu(xq.reshape(B, T, cq), w[:cq])", "q, _ = conv_silu(xq.reshape(B, T, cq), w[cq:2 * cq])"),
+      ("k, _ = conv_silu(xk.reshape(B, T, cq), w[cq:2 * cq])", "k, _ = conv_silu(xk.reshape(B, T, cq), w[:cq])")]),
+    ("layer forward: k left without its L2 norm",
+     [("k = l2norm(k.reshape(B, T, Hk, dk))", "k = k.reshape(B, T, Hk, dk)")]),
+    ("layer forward: v taken before its convolution",
+     [("v = v.reshape(B, T, Hv, dv)", "v = xv")]),
+]
+
+
+def test_unmutated_layer_forward_copy_passes_its_pin(monkeypatch):
+    monkeypatch.setattr(pins, "oracle", _oracle_copy(open(PY).read()))
+    pins.test_layer_core_forward_closed_forms()
+
+
+@pytest.mark.parametrize("name,edits", LAYER_FWD_MUTANTS, ids=[m[0] for m in LAYER_FWD_MUTANTS])
+def test_planted_layer_forward_mistake_is_caught(name, edits, monkeypatch):
+    src = open(PY).read()
+    for old, new in edits:
+        assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+        src = src.replace(old, new)
+    monkeypatch.setattr(pins, "oracle", _oracle_copy(src))
+    with pytest.raises(AssertionError):
+        pins.test_layer_core_forward_closed_forms()

@@ -658,3 +658,59 @@ def test_logit_gradients_finite_differences(channel):
             m[idx] -= h
             fd[idx] = (f(p) - f(m)) / (2 * h)
         assert relerr(lgr[name], fd) < 1e-6, name
+
+
+def test_layer_core_forward_closed_forms():
+    """The oracle's layer composition (conv k=4 + SiLU, L2 norm of q and k, the recurrence, the
+    swish(z) gate; explainer «Architecture et versions hybrides», Figure 1 caption; mkdocs chapter
+    «Gated DeltaNet») against closed forms that fix the conv tap orientation, the channel order of
+    the convolution weights (q, k, v) and the order of the steps:
+    - only the current-token tap, alpha = 1, beta = 0: the state stays h0, so
+      y_t = swish(z_t) * h0^T l2(silu(xq_t));
+    - only the oldest tap: token t sees xq_{t-3}; the first three tokens see zeros (SiLU(0) = 0,
+      and the L2 norm of 0 is 0), so their y is 0;
+    - one token, alpha = 1, beta = 1, h0 = 0: S = k v^T, so y = swish(z) * v (k . q) with
+      q = l2(silu(xq)), k = l2(silu(2 xk)), v = silu(3 xv) when the current-token tap weighs the
+      q, k, v channel blocks 1, 2, 3 (a misplaced block would differ)."""
+    rng = np.random.default_rng(41)
+    B, T, Hk, Hv, d = 1, 6, 1, 2, 4
+    cch = 2 * Hk * d + Hv * d
+    xq = rng.standard_normal((B, T, Hk, d))
+    xk = rng.standard_normal((B, T, Hk, d))
+    xv = rng.standard_normal((B, T, Hv, d))
+    z = rng.standard_normal((B, T, Hv, d))
+    h0 = rng.standard_normal((B, Hv, d, d))
+    silu = lambda x: x / (1.0 + np.exp(-x))
+    swish = lambda x: x / (1.0 + np.exp(-x))
+    l2 = lambda x: x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + 1e-6)
+    ones = np.ones((B, T, Hv))
+    zeros = np.zeros((B, T, Hv))
+    # current-token tap only
+    w = np.zeros((cch, 4))
+    w[:, 3] = 1.0
+    y, hT = oracle.layer_core_fwd(xq, xk, xv, w, ones, zeros, z, h0=h0)
+    q = l2(silu(xq))
+    for hv in range(Hv):
+        want = swish(z[:, :, hv]) * np.einsum("bij,bti->btj", h0[:, hv], q[:, :, 0])
+        np.testing.assert_allclose(y[:, :, hv], want, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(hT, h0, rtol=0, atol=1e-14)
+    # oldest tap only: token t reads xq_{t-3}
+    w = np.zeros((cch, 4))
+    w[:, 0] = 1.0
+    y, _ = oracle.layer_core_fwd(xq, xk, xv, w, ones, zeros, z, h0=h0)
+    np.testing.assert_allclose(y[:, :3], 0.0, atol=1e-14)
+    q3 = l2(silu(xq[:, :T - 3]))
+    for hv in range(Hv):
+        want = swish(z[:, 3:, hv]) * np.einsum("bij,bti->btj", h0[:, hv], q3[:, :, 0])
+        np.testing.assert_allclose(y[:, 3:, hv], want, rtol=1e-12, atol=1e-14)
+    # one token, a full write from a zero state; the current tap weighs the q, k and v channel
+    # blocks 1, 2 and 3, so a misplaced block changes the result
+    cq = Hk * d
+    w = np.zeros((cch, 4))
+    w[:cq, 3], w[cq:2 * cq, 3], w[2 * cq:, 3] = 1.0, 2.0, 3.0
+    y, hT = oracle.layer_core_fwd(xq[:, :1], xk[:, :1], xv[:, :1], w, ones[:, :1], ones[:, :1], z[:, :1])
+    qn, kn, vs = l2(silu(xq[:, 0, 0])), l2(silu(2.0 * xk[:, 0, 0])), silu(3.0 * xv[:, 0])
+    for hv in range(Hv):
+        want = swish(z[:, 0, hv]) * vs[:, hv] * np.sum(kn * qn, axis=-1, keepdims=True)
+        np.testing.assert_allclose(y[:, 0, hv], want, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(hT[:, hv], np.einsum("bi,bj->bij", kn, vs[:, hv]), rtol=1e-12, atol=1e-14)
