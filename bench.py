@@ -354,12 +354,18 @@ def bench_headline_e2e(args, dist, x, stream, device, slices=8):
     memory, forward + backward, D2H of every result, all inside the timed region.  The batch's
     sequences are independent, so the step runs as `slices` slices of the batch on three streams
     (copy in, compute, copy out): the copies of one slice overlap the compute and the
-    other-direction copies of the others, and the PCIe link carries both directions at once."""
+    other-direction copies of the others, and the PCIe link carries both directions at once.
+    The device inputs are double-buffered across steps, so that a step's copies in overlap the
+    previous step's copies out; a set is overwritten only after the compute that read it two
+    steps before."""
     import torch
     from gated_delta_rule_76_b200 import gdn
     names_in = ["q", "k", "v", "alpha", "b", "w", "h0", "dout"]
     host = {n: x[n].pin_memory() for n in names_in}
     dev = {n: torch.empty_like(host[n], device=device) for n in names_in}
+    dev_sets = [dev, {n: torch.empty_like(host[n], device=device) for n in names_in}]
+    set_free = [None, None]  # per set: an event on `stream` after the last compute that read it
+    n_steps = [0]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     B = host["q"].shape[0]
     ns = slices if B % slices == 0 else 1
@@ -373,18 +379,22 @@ def bench_headline_e2e(args, dist, x, stream, device, slices=8):
     out_host = {}
 
     def step():
-        s_in.wait_stream(stream)
+        cur = n_steps[0] & 1
+        n_steps[0] += 1
+        dset = dev_sets[cur]
+        if set_free[cur] is not None:
+            s_in.wait_event(set_free[cur])
         ev_in = []
         with torch.cuda.stream(s_in):
             for i in range(ns):
                 for n in names_in:
-                    cut(dev[n], i).copy_(cut(host[n], i), non_blocking=True)
+                    cut(dset[n], i).copy_(cut(host[n], i), non_blocking=True)
                 ev_in.append(torch.cuda.Event())
                 ev_in[-1].record(s_in)
         res, ev_c = [], []
         for i in range(ns):
             stream.wait_event(ev_in[i])
-            d = {n: cut(dev[n], i) for n in names_in}
+            d = {n: cut(dset[n], i) for n in names_in}
             o, ht = gdn.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], b=d["b"], w=d["w"], h0=d["h0"],
                                       bwd_cache=caches[i], stream=stream)
             gr = gdn.gdn_chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], b=d["b"], w=d["w"], h0=d["h0"],
@@ -392,6 +402,7 @@ def bench_headline_e2e(args, dist, x, stream, device, slices=8):
             res.append({"o": o, "ht": ht, **gr})
             ev_c.append(torch.cuda.Event())
             ev_c[-1].record(stream)
+        set_free[cur] = ev_c[-1]
         with torch.cuda.stream(s_out):
             for i in range(ns):
                 s_out.wait_event(ev_c[i])
