@@ -159,7 +159,7 @@ GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args* args, void* workspace, size
  *  - Limit: a problem whose gdn_chunk_fwd_workspace_size() exceeds 16 MiB is rejected with
  *    GDN_ERR_WORKSPACE before anything is launched (the tensor-core path needs 256 bytes plus
  *    4 bytes per (sequence, value head), so bf16 problems with dk = dv = 128 fit up to ~4 million
- *    pairs; the CUDA-core path needs per-chunk factors).
+ *    pairs; the CUDA-core path needs per-chunk factors; strided inputs add their dense copies).
  *  - Set-up: every call looks up the array's address on the current device with
  *    cudaGetSymbolAddress (so a device reset between calls is harmless).  The first call on a
  *    device may load the library's device code there; make it before any stream capture.  Later
