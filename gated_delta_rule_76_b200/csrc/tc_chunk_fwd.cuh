@@ -448,15 +448,17 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             if (p.s0_out) {
-                // state entering chunk n (saving mode), stored while X2 runs: rows 64h .. 64h + 63
-                // of column j, in the layout [j / 8][row][j % 8]: each group of 8 lanes fills one
-                // 32-byte sector per store (a reader holding one row per thread loads a row's 8
-                // columns of a block as one 32-byte vector).  Plain 4-byte stores: transposing
-                // the state across lanes first (store_state_block, as the reverse scan does) made
-                // this chain slower.
+                // state entering chunk n (saving mode): rows 64h .. 64h + 63 of column j, in the
+                // layout [j / 8][row][j % 8]: each group of 8 lanes fills one 32-byte sector per
+                // store (a reader holding one row per thread loads a row's 8 columns of a block as
+                // one 32-byte vector).  Plain 4-byte stores: transposing the state across lanes
+                // first (store_state_block, as the reverse scan does) made this chain slower.  The
+                // first 32 rows are stored while X2 runs, the other 32 while X4 / X5 run (S changes
+                // only in the state update): split so, the stores queue behind the chain's waits
+                // instead of in one burst (all 64 in either place was slower).
                 float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 3) * (8 * D) + (64 * h) * 8 + (j & 7);
 #pragma unroll
-                for (int c = 0; c < 64; ++c) dst[8 * c] = S[c];
+                for (int c = 0; c < 32; ++c) dst[8 * c] = S[c];
             }
             tc_fence_before();
             fence_async_shared();
@@ -652,6 +654,12 @@ chunk_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     *reinterpret_cast<uint4*>(p.vp_lo + vo + 64 * i) =
                         make_uint4(vl[4 * i], vl[4 * i + 1], vl[4 * i + 2], vl[4 * i + 3]);
                 }
+            }
+            if (p.s0_out) {
+                // the other 32 rows of the state entering chunk n (see the X2 phase)
+                float* dst = p.s0_out + ((long)blockIdx.x * (NT + 1) + n) * (D * D) + (j >> 3) * (8 * D) + (64 * h) * 8 + (j & 7);
+#pragma unroll
+                for (int c = 32; c < 64; ++c) dst[8 * c] = S[c];
             }
             if (tid == 0) {
                 if (!*cx.abort_flag) {
