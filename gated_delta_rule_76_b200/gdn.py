@@ -262,6 +262,11 @@ def _head_map(head_map, device, Hk: int):
 
 # ---------------------------------------------------------------------------------------------
 # public calls
+#
+# Token-major inputs (q, k, v, the gates, z; xq, xk, xv for the layer calls) may be views whose
+# tokens are evenly spaced and whose heads and channels are dense, such as column slices of one
+# fused projection buffer viewed as [B, T, H, d]: they are passed with their token stride
+# (gdn_strides), without a copy here.  Every other tensor must be contiguous.
 # ---------------------------------------------------------------------------------------------
 def fwd_args(q, k, v, alpha, b=None, w=None, beta=None, h0=None, z=None, head_map=None,
              scale: float = 1.0, o=None, ht=None, bwd_cache=None, alpha_scale=None) -> Tuple[FwdArgs, list]:
