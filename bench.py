@@ -190,8 +190,9 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
         loaded = [s for s in sm if s > 0.5 * smax] or sm
+        power = [float(r[4]) for r in rows if r[4] not in ("[N/A]", "")]
         return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[4]) for r in rows if r[4] not in ("[N/A]", ""))}
+                "samples": len(rows), "power_w_max": max(power) if power else None}
 
 
 # --------------------------------------------------------------------------------------------
